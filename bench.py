@@ -1,0 +1,448 @@
+"""Benchmark of one EntmaxKV sparse alpha-entmax decode step on B200.
+
+A step is the whole hot path for one batch: refresh the metadata of the page
+the newest token went to (entmaxkv_build_meta, one page per sequence), score
+every page (entmaxkv_score_pages), select (entmaxkv_select, top-k or Gaussian
+tau_hat - Delta) and decode over the selected pages (entmaxkv_decode_sparse).
+Default workload: B=1, Hq=32, Hkv=8, d=128, 1,048,576-token context, 64-token
+pages, alpha=1.5, Gaussian selection with Delta=0.5 (the long-context setting of
+the EntmaxKV efficiency study), synthetic clustered keys with 64 needles per
+head.  Inputs live in HBM before timing; L2 is flushed (256 MiB write) before
+every step, outside the per-step CUDA events.
+
+Reported value: effective KV bandwidth = bytes the step must touch (metadata
+scanned by scoring + K tiles of the selected pages + value rows with non-zero
+weight) / device time per step, summed over all ranks (one independent
+problem per GPU, weak scaling, no data-path collective).
+
+  python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME] [--impl reference]
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import os
+import statistics
+import subprocess
+import sys
+import time
+
+import numpy as np
+import torch
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+METRIC = "sparse α-entmax decode µs/step & KV GB/s vs HBM roofline at 1M ctx"
+PAPER_CONTEXT = {"speedup_vs_full_softmax_flashdecoding": 3.36, "speedup_vs_full_entmax": 5.43,
+                 "context_tokens": 1048576, "hardware": "not stated on the pages",
+                 "source": "EntmaxKV summary, section 4 (Efficiency)"}
+
+# DRAM bytes per launch from ncu captures (dram__bytes_read.sum + dram__bytes_write.sum),
+# keyed by kernel and workload, valid only while the kernel source is unchanged.
+NCU_TRAFFIC = {}
+
+
+def _src_hash(fname):
+    p = os.path.join(ROOT, "sparse_entmax_kv_b200", "csrc", fname)
+    return hashlib.sha1(open(p, "rb").read()).hexdigest()[:12]
+
+
+def measured_peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        d = json.load(open(p))
+        return d.get("hbm_gbs", 6650.0), "measured"
+    return 6650.0, "fallback"
+
+
+class ClockSampler:
+    """nvidia-smi clock / throttle sampling while the timed region runs."""
+
+    def __init__(self, index):
+        self.proc = None
+        self.path = os.path.join(ROOT, "gpurun_out", f"clocks_rank{index}.csv")
+        self.index = index
+
+    def __enter__(self):
+        try:
+            os.makedirs(os.path.dirname(self.path), exist_ok=True)
+            self.f = open(self.path, "w")
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", "-i", str(self.index),
+                 "--query-gpu=index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+                 "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+                 "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap",
+                 "--format=csv,noheader,nounits", "-lms", "200"], stdout=self.f, stderr=subprocess.DEVNULL)
+        except (OSError, FileNotFoundError):
+            self.proc = None
+        return self
+
+    def __exit__(self, *exc):
+        if self.proc is not None:
+            self.proc.terminate()
+            try:
+                self.proc.wait(timeout=5)
+            except subprocess.TimeoutExpired:
+                self.proc.kill()
+            self.f.close()
+
+    def summary(self):
+        if self.proc is None or not os.path.exists(self.path):
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
+        sm, mx, reasons = [], [], set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for line in open(self.path):
+            f = [x.strip() for x in line.split(",")]
+            if len(f) < 9:
+                continue
+            try:
+                sm.append(float(f[1]))
+                mx.append(float(f[2]))
+            except ValueError:
+                continue
+            for n, v in zip(names, f[5:9]):
+                if v.lower() == "active":
+                    reasons.add(n)
+        return {"sm_mhz": statistics.median(sm) if sm else None, "sm_max_mhz": max(mx) if mx else None,
+                "reasons": sorted(reasons), "samples": len(sm)}
+
+
+# ------------------------------------------------------------ byte model
+
+def step_bytes(wl, dec, support_rows):
+    """Algorithmic bytes of one step.  meta: records scanned by scoring;
+    gather_k: K tiles of each GQA group's union of selected pages; gather_v:
+    value rows with non-zero weight for some head of the group."""
+    seq = dec.seq_lens.cpu().numpy()
+    npb = -(-seq // wl.P)
+    rec_bytes = (12 if wl.policy == "gauss" else 4) * wl.d
+    meta = int(npb.sum()) * wl.Hkv * rec_bytes
+    sel, cnt = dec.sel.cpu().numpy(), dec.cnt.cpu().numpy()
+    union = 0
+    for b in range(wl.B):
+        for kvh in range(wl.Hkv):
+            s = set()
+            for g in range(wl.G):
+                h = kvh * wl.G + g
+                s.update(sel[b, h, :cnt[b, h]].tolist())
+            union += len(s)
+    gather_k = union * wl.P * wl.d * 2
+    gather_v = support_rows * wl.d * 2
+    scores = wl.B * wl.Hq * int(npb.max()) * (12 if wl.policy == "gauss" else 4)
+    qo = wl.B * wl.Hq * wl.d * (2 + 4)
+    return dict(meta=meta, gather_k=gather_k, gather_v=gather_v, scores=scores, qo=qo,
+                kv_touched=meta + gather_k + gather_v, union_pages=union, support_rows=support_rows)
+
+
+def support_rows_of(wl, p_out):
+    """Distinct (sequence, kv head, token) rows with p > 0 for some head of the group."""
+    pz = (p_out > 0).view(wl.B, wl.Hkv, wl.G, -1).any(dim=2)
+    return int(pz.sum().item())
+
+
+# ------------------------------------------------------------- GPU arm
+
+def run_gpu(args, rank, world):
+    from sparse_entmax_kv_b200 import native as nv
+    from sparse_entmax_kv_b200.decoder import EntmaxKVDecoder, kernels_per_step
+    from sparse_entmax_kv_b200.workloads import CONFIGS, make_inputs
+
+    wl = CONFIGS[args.workload]
+    policy = wl.policy if wl.policy != "dense" else "topk"
+    k = wl.k or 64
+    delta = wl.delta or 0.5
+    dev = torch.device("cuda", torch.cuda.current_device())
+    inp = make_inputs(wl, 1000 * 4 + rank, device=dev)
+    dec = EntmaxKVDecoder(inp["k_cache"], inp["v_cache"], inp["page_table"], inp["seq_lens"], wl.Hq,
+                          alpha=wl.alpha, policy=policy, k=k, delta=delta)
+    dec.build_meta()
+    # the newest token of sequence 0 sits in its last page; appends rewrite it
+    L0 = int(inp["seq_lens"][0])
+    append_page = (L0 - 1) // wl.P
+    flush = torch.empty(256 << 20, dtype=torch.uint8, device=dev)
+    q = inp["q"]
+    st = torch.cuda.current_stream()
+
+    # byte model from one untimed step with p written out
+    p_out = torch.zeros((wl.B, wl.Hq, wl.max_pages * wl.P), device=dev)
+    dec.step(q, append_page, p_out=p_out)
+    torch.cuda.synchronize()
+    nbytes = step_bytes(wl, dec, support_rows_of(wl, p_out))
+    del p_out
+    torch.cuda.empty_cache()
+
+    for _ in range(args.warmup):
+        flush.fill_(1)
+        dec.step(q, append_page)
+    torch.cuda.synchronize()
+    assert nv.get_status(clear=True) & ~nv.STATUS_OVERFLOW == 0
+
+    nst = 4
+    ev = [[torch.cuda.Event(enable_timing=True) for _ in range(nst + 1)] for _ in range(args.steps)]
+    if world > 1:
+        torch.distributed.barrier()
+    torch.cuda.synchronize()
+    with ClockSampler(dev.index) as clk:
+        t_wall = time.perf_counter()
+        for i in range(args.steps):
+            flush.fill_(1)
+            e = ev[i]
+            e[0].record(st)
+            nv.entmaxkv_build_meta(dec.shape, dec.k_cache, dec.page_table, dec.seq_lens, append_page, 1, dec.meta)
+            e[1].record(st)
+            nv.entmaxkv_score_pages(dec.shape, q, dec.meta, dec.page_table, dec.seq_lens, dec.bbox, dec.mu,
+                                    dec.sigma)
+            e[2].record(st)
+            nv.entmaxkv_select(dec.shape, dec.seq_lens, dec.bbox, dec.mu, dec.sigma, dec.policy, dec.k, dec.alpha,
+                               dec.delta, dec.sel, dec.cnt, dec.tau_hat)
+            e[3].record(st)
+            nv.entmaxkv_decode_sparse(dec.shape, q, dec.k_cache, dec.v_cache, dec.page_table, dec.seq_lens,
+                                      dec.sel, dec.cnt, dec.alpha, dec.out, dec.tau, None, dec.ws)
+            e[4].record(st)
+        torch.cuda.synchronize()
+        if world > 1:
+            torch.distributed.barrier()
+        t_wall = time.perf_counter() - t_wall
+    clocks = clk.summary()
+    stage_ms = np.array([[ev[i][j].elapsed_time(ev[i][j + 1]) for j in range(nst)] for i in range(args.steps)])
+    step_ms = float(stage_ms.sum(axis=1).mean())
+    if world > 1:
+        t = torch.tensor([step_ms], device=dev)
+        torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
+        step_ms = float(t.item())
+    stage_us = dict(zip(["build_meta_append", "score_pages", "select", "decode_sparse"],
+                        (stage_ms.mean(axis=0) * 1e3).round(2).tolist()))
+
+    # comparison paths at the same context: full-cache entmax and softmax
+    dense = {}
+    if not args.skip_dense:
+        out = torch.empty((wl.B, wl.Hq, wl.d), device=dev)
+        ws = nv.alloc_workspace(dec.shape, nv.CALL_DECODE_DENSE, dev)
+        for alpha, name in ((wl.alpha, "dense_entmax"), (1.0, "dense_softmax")):
+            ts = []
+            for i in range(3 + args.dense_steps):
+                flush.fill_(1)
+                a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+                a.record(st)
+                nv.entmaxkv_decode_dense(dec.shape, q, dec.k_cache, dec.v_cache, dec.page_table, dec.seq_lens,
+                                         alpha, out, None, None, ws)
+                b.record(st)
+                torch.cuda.synchronize()
+                if i >= 3:
+                    ts.append(a.elapsed_time(b))
+            dense[name] = statistics.median(ts) * 1e3
+        del ws
+
+    # end to end through the C ABI with host buffers: q and the appended token's
+    # k/v come from pinned host memory each step, the output goes back to host
+    G = wl.G
+    tok = (L0 - 1) % wl.P
+    blk = int(inp["page_table"][0, append_page])
+    k_new = inp["k_cache"][blk, :, tok].clone().cpu().pin_memory()
+    v_new = inp["v_cache"][blk, :, tok].clone().cpu().pin_memory()
+    q_host = q.cpu().pin_memory()
+    out_host = torch.empty((wl.B, wl.Hq, wl.d), dtype=torch.float32).pin_memory()
+    k_dev = torch.empty_like(inp["k_cache"][blk, :, tok])
+    v_dev = torch.empty_like(k_dev)
+    q_dev = torch.empty_like(q)
+    e2e_ms = []
+    for i in range(args.warmup + args.steps):
+        flush.fill_(1)
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a.record(st)
+        q_dev.copy_(q_host, non_blocking=True)
+        k_dev.copy_(k_new, non_blocking=True)
+        v_dev.copy_(v_new, non_blocking=True)
+        inp["k_cache"][blk, :, tok] = k_dev
+        inp["v_cache"][blk, :, tok] = v_dev
+        dec.step(q_dev, append_page)
+        out_host.copy_(dec.out, non_blocking=True)
+        b.record(st)
+        torch.cuda.synchronize()
+        if i >= args.warmup:
+            e2e_ms.append(a.elapsed_time(b))
+    e2e_step_ms = float(np.mean(e2e_ms))
+    if world > 1:
+        t = torch.tensor([e2e_step_ms], device=dev)
+        torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
+        e2e_step_ms = float(t.item())
+    assert nv.get_status(clear=True) & ~nv.STATUS_OVERFLOW == 0
+
+    peak, peak_kind = measured_peaks()
+    # dominant kernel of the step
+    dom = max(("score_pages", "decode_sparse"), key=lambda s: stage_us[s])
+    if dom == "score_pages":
+        alg = nbytes["meta"] + nbytes["scores"] + wl.B * wl.Hq * wl.d * 2
+        src = "score.cu"
+    else:
+        alg = nbytes["gather_k"] + nbytes["gather_v"] + nbytes["qo"]
+        src = "decode.cu"
+    achieved = alg / (stage_us[dom] * 1e-6) / 1e9
+    tr = NCU_TRAFFIC.get(f"{dom}/{args.workload}")
+    traffic = tr["bytes"] if tr and tr.get("src") == _src_hash(src) else None
+    roofline = {"bound": "hbm", "kernel": dom, "achieved": round(achieved, 1), "peak": peak, "unit": "GB/s",
+                "frac": round(achieved / peak, 4), "traffic": traffic, "algorithmic_bytes": alg,
+                "peak_kind": f"{peak_kind} copy bandwidth (burst)"}
+    res = dict(wl=wl, step_ms=step_ms, stage_us=stage_us, dense=dense, nbytes=nbytes, clocks=clocks,
+               roofline=roofline, e2e_ms=e2e_step_ms, e2e_bytes=(q_host.numel() * 2 + k_new.numel() * 4,
+                                                               out_host.numel() * 4),
+               launches=kernels_per_step(policy == "gauss", True) * args.steps, t_wall=t_wall,
+               host=dict(inp=inp, dec=dec) if (rank == 0 and not args.no_cpu_baseline) else None)
+    return res
+
+
+# --------------------------------------------------------- CPU oracle arm
+
+def oracle_step_sample(wl, inp_host, seconds_target=10.0, max_reps=3):
+    """Time the fp64 oracle on one step of the workload (score + select +
+    sparse decode, metadata prepared beforehand), repeated up to max_reps or
+    until seconds_target is reached.  Returns (seconds per step, bytes per
+    step by the same byte model, threads)."""
+    import oracle as orc
+
+    policy = wl.policy if wl.policy != "dense" else "topk"
+    h = inp_host
+    meta = orc.build_meta(h["K"], h["page_table"], h["seq_lens"], wl.Hkv, wl.d, wl.P, wl.num_blocks)
+    times = []
+    t_end = time.perf_counter() + seconds_target
+    for _ in range(max_reps):
+        t0 = time.perf_counter()
+        bbox, mu, sig = orc.score_pages(h["q"], meta, h["page_table"], h["seq_lens"], wl.Hkv, wl.P)
+        sel, cnt, _ = orc.select(h["seq_lens"], bbox, mu, sig, wl.P, policy, wl.k or 64, wl.alpha,
+                                 wl.delta or 0.5)
+        o, tau, pw, _ = orc.decode(h["q"], h["K"], h["V"], h["page_table"], h["seq_lens"], wl.Hkv, wl.P,
+                                   wl.alpha, sel=sel, cnt=cnt, want_p=True)
+        times.append(time.perf_counter() - t0)
+        if time.perf_counter() > t_end:
+            break
+    npb = -(-h["seq_lens"] // wl.P)
+    meta_b = int(npb.sum()) * wl.Hkv * (12 if policy == "gauss" else 4) * wl.d
+    union = 0
+    supp = 0
+    for b in range(wl.B):
+        for kvh in range(wl.Hkv):
+            s = set()
+            rows = None
+            for g in range(wl.G):
+                hh = kvh * wl.G + g
+                s.update(sel[b, hh, :cnt[b, hh]].tolist())
+                r = pw[b, hh] > 0
+                rows = r if rows is None else (rows | r)
+            union += len(s)
+            supp += int(rows.sum())
+    nbytes = meta_b + union * wl.P * wl.d * 2 + supp * wl.d * 2
+    return statistics.median(times), nbytes, orc.num_threads(), len(times)
+
+
+def host_copy(inp, b0=0, nb=None):
+    from sparse_entmax_kv_b200.workloads import to_host_u16
+    return dict(q=to_host_u16(inp["q"]), K=to_host_u16(inp["k_cache"]), V=to_host_u16(inp["v_cache"]),
+                page_table=inp["page_table"].cpu().numpy(), seq_lens=inp["seq_lens"].cpu().numpy())
+
+
+def sample_workload(wl):
+    """The bounded oracle sample of a workload: the first sequence, all its
+    heads, at the full context (one sequence of the batch)."""
+    return wl.shrink(B=1)
+
+
+def run_reference(args, rank, world):
+    """Reference arm: the fp64 CPU oracle, timed on the host cores, on a
+    bounded sample of the same workload (rank 0 only)."""
+    from sparse_entmax_kv_b200.workloads import CONFIGS, make_inputs
+    if rank != 0:
+        return
+    wl = CONFIGS[args.workload]
+    swl = sample_workload(wl)
+    inp = make_inputs(swl, 1000 * 4, device="cpu")
+    host = host_copy(inp)
+    per = []
+    for i in range(args.warmup + args.steps):
+        sec, nbytes, thr, reps = oracle_step_sample(swl, host, seconds_target=0.0, max_reps=1)
+        if i >= args.warmup:
+            per.append(sec)
+    sec = statistics.median(per)
+    gbs = nbytes / sec / 1e9
+    sample = f"{swl.B} of {wl.B} sequence(s), all {wl.Hq} heads, full {wl.L}-token context, one step per timed step"
+    line = {"impl": "reference", "metric": METRIC, "value": round(gbs, 4), "unit": "GB/s", "n_gpus": world,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(sec * 1e3, 3),
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+            "data": "synthetic", "config": config_of(wl),
+            "cpu_baseline": {"value": round(gbs, 4), "unit": "GB/s", "cores": thr, "kind": "oracle",
+                             "sample": sample},
+            "e2e": {"value": round(gbs, 4), "unit": "GB/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+
+
+def config_of(wl):
+    return {"workload": wl.name, "B": wl.B, "Hq": wl.Hq, "Hkv": wl.Hkv, "d": wl.d, "L": wl.L,
+            "page_size": wl.P, "alpha": wl.alpha, "policy": wl.policy, "k": wl.k, "delta": wl.delta,
+            "keys": wl.keys, "needles_per_head": wl.needles,
+            "l2": "flushed before every step (256 MiB write), outside the per-step events"}
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--workload", default="gauss_gqa_L1m")
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--dense-steps", type=int, default=5)
+    ap.add_argument("--skip-dense", action="store_true")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args()
+    args.warmup = max(args.warmup, 3)
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if args.impl == "reference":
+        run_reference(args, rank, world)
+        return
+
+    torch.cuda.set_device(local)
+    if world > 1:
+        import datetime
+        torch.distributed.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                             device_id=torch.device("cuda", local))
+    from sparse_entmax_kv_b200 import native as nv  # noqa: F401  (fails loudly if not built)
+
+    res = run_gpu(args, rank, world)
+    wl = res["wl"]
+    nb = res["nbytes"]
+    value = world * nb["kv_touched"] / (res["step_ms"] * 1e-3) / 1e9
+    e2e_val = world * nb["kv_touched"] / (res["e2e_ms"] * 1e-3) / 1e9
+    line = {"metric": METRIC, "value": round(value, 2), "unit": "GB/s", "n_gpus": world, "steps": args.steps,
+            "warmup": args.warmup, "ms_per_step": round(res["step_ms"], 5),
+            "us_per_step": round(res["step_ms"] * 1e3, 2), "higher_is_better": True, "scaling": "weak",
+            "vs_baseline": None, "dtype": "bf16", "data": "synthetic", "config": config_of(wl),
+            "frac_of_hbm_peak": round(value / world / res["roofline"]["peak"], 4),
+            "roofline": res["roofline"], "stages_us": res["stage_us"], "bytes_per_step": nb,
+            "e2e": {"value": round(e2e_val, 2), "unit": "GB/s", "us_per_step": round(res["e2e_ms"] * 1e3, 2),
+                    "h2d_bytes_per_step": res["e2e_bytes"][0], "d2h_bytes_per_step": res["e2e_bytes"][1]},
+            "gpu_launches": res["launches"], "clocks": res["clocks"], "paper_context": PAPER_CONTEXT}
+    if res["dense"]:
+        de, ds = res["dense"]["dense_entmax"], res["dense"]["dense_softmax"]
+        sp = res["step_ms"] * 1e3
+        line["dense_us"] = {"entmax_full_cache": round(de, 1), "softmax_full_cache_splitk": round(ds, 1)}
+        line["speedup"] = {"vs_dense_entmax": round(de / sp, 2), "vs_dense_softmax": round(ds / sp, 2)}
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        swl = sample_workload(wl)
+        inp = res["host"]["inp"]
+        host = host_copy({k: (v[:1] if k in ("q", "page_table", "seq_lens") else v) for k, v in inp.items()})
+        sec, nbytes, thr, reps = oracle_step_sample(swl, host)
+        line["cpu_baseline"] = {"value": round(nbytes / sec / 1e9, 4), "unit": "GB/s", "cores": thr,
+                                "kind": "oracle",
+                                "sample": f"sequence 0 of {wl.B}, all {wl.Hq} heads, full context; "
+                                          f"median of {reps} oracle step(s), {sec:.2f} s each"}
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+    if world > 1:
+        torch.distributed.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

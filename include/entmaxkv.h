@@ -1,0 +1,238 @@
+/*
+ * entmaxkv.h -- C ABI of libentmaxkv.so: paged, support-aware alpha-entmax
+ * decode attention for NVIDIA B200 (sm_100a).
+ *
+ * The operations follow "EntmaxKV - Support-aware decoding for entmax
+ * attention" (technical summary, gist.science paper 2605.21649; the same text
+ * exists in Spanish, Japanese, Korean and Arabic).  One decode step, for
+ * every (sequence b, query head h), against a paged bf16 K/V cache:
+ *
+ *   entmaxkv_build_meta     per-page metadata (section 2.A)
+ *   entmaxkv_score_pages    query-aware page scores (section 2.A)
+ *   entmaxkv_select         candidate pages: top-k or Gaussian tau_hat - Delta
+ *                           (section 2.B)
+ *   entmaxkv_decode_sparse  exact alpha-entmax attention over the selected
+ *                           pages only (section 2.C)
+ *   entmaxkv_decode_dense   full-cache entmax, or full-cache softmax split-K,
+ *                           the comparison points of section 4 "Efficiency"
+ *
+ * Conventions shared by every entry point
+ * ---------------------------------------
+ * - Pointers named *_cache, q, meta, page_table, seq_lens, scores, sel, cnt,
+ *   out, workspace are DEVICE pointers owned by the caller; the library never
+ *   allocates, frees or keeps them.  `stream` is a cudaStream_t passed as
+ *   void* (NULL = legacy default stream).  Every call only enqueues work on
+ *   that stream and returns; it never synchronises the host (except
+ *   entmaxkv_get_status, which is a query).
+ * - Return value: ENTMAXKV_OK (0) or a negative ENTMAXKV_ERR_* code.  All
+ *   argument checks run on the host before anything is launched, so an error
+ *   return means nothing was enqueued.  ENTMAXKV_ERR_CUDA reports a failed
+ *   launch (cudaGetLastError).
+ * - Errors the host cannot see (a page-table entry outside [0, num_blocks), a
+ *   selected page index outside the sequence, a wait that ran out) are
+ *   recorded in a per-device status word (ENTMAXKV_STATUS_* bits, OR-ed) read
+ *   with entmaxkv_get_status.  Kernels never trap; the offending page is
+ *   skipped.
+ * - Layouts (row-major, all contiguous):
+ *     k_cache, v_cache  bf16  [num_blocks][Hkv][P][d]   16-byte aligned
+ *     q                 bf16  [B][Hq][d]                 16-byte aligned
+ *     page_table        int32 [B][max_pages]  logical page -> physical block
+ *     seq_lens          int32 [B]             tokens per sequence (<= max_pages*P)
+ *   Query head h reads kv head h / G, G = Hq / Hkv.  Sequence b has
+ *   N_b = ceil(seq_lens[b] / P) pages; page p holds min(P, seq_lens[b] - p*P)
+ *   valid tokens.  Scores are s = q.k / sqrt(d); entmax uses z = (alpha-1) s
+ *   and p = [z - tau]_+^(1/(alpha-1)) with tau such that sum p = 1.
+ * - Supported: d in {64, 128}; P in {16, 32, 64}; G in {1, 2, 4, 8};
+ *   max_pages * P < 2^31; max_pages <= 196608 for entmaxkv_select and
+ *   entmaxkv_decode_sparse.
+ */
+#ifndef ENTMAXKV_H
+#define ENTMAXKV_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#if defined(__GNUC__)
+#define ENTMAXKV_API __attribute__((visibility("default")))
+#else
+#define ENTMAXKV_API
+#endif
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef struct entmaxkv_shape {
+    int32_t B;          /* sequences in the batch */
+    int32_t Hq;         /* query heads per sequence */
+    int32_t Hkv;        /* key/value heads; Hq % Hkv == 0 */
+    int32_t d;          /* head dimension */
+    int32_t page_size;  /* P, tokens per page */
+    int32_t max_pages;  /* row length of page_table (pages per sequence at most) */
+    int32_t num_blocks; /* physical blocks held by k_cache / v_cache */
+} entmaxkv_shape;
+
+enum {
+    ENTMAXKV_OK = 0,
+    ENTMAXKV_ERR_NULL = -1,        /* a required pointer is NULL */
+    ENTMAXKV_ERR_SHAPE = -2,       /* shape field out of range or inconsistent */
+    ENTMAXKV_ERR_ALPHA = -3,       /* alpha out of range for the call */
+    ENTMAXKV_ERR_POLICY = -4,      /* unknown policy, k < 1, or Delta not finite */
+    ENTMAXKV_ERR_WORKSPACE = -5,   /* workspace missing or smaller than required */
+    ENTMAXKV_ERR_CUDA = -6,        /* CUDA runtime/driver error */
+    ENTMAXKV_ERR_UNSUPPORTED = -7, /* valid but not implemented (e.g. non-integer r) */
+    ENTMAXKV_ERR_ALIGN = -8        /* pointer not 16-byte aligned */
+};
+
+enum { ENTMAXKV_TOPK = 0, ENTMAXKV_GAUSS = 1 };
+
+/* `call` argument of entmaxkv_workspace_size */
+enum {
+    ENTMAXKV_CALL_SELECT = 2,
+    ENTMAXKV_CALL_DECODE_SPARSE = 3,
+    ENTMAXKV_CALL_DECODE_DENSE = 4
+};
+
+/* bits of the device status word */
+enum {
+    ENTMAXKV_STATUS_BAD_PAGE = 1,      /* page_table entry outside [0, num_blocks) */
+    ENTMAXKV_STATUS_BAD_SELECTION = 2, /* sel entry outside [0, N_b) or cnt > N_b */
+    ENTMAXKV_STATUS_TIMEOUT = 4,       /* an on-device wait hit its limit */
+    ENTMAXKV_STATUS_OVERFLOW = 8       /* a candidate list overflowed on-chip storage
+                                          (handled by a slower exact path) */
+};
+
+/* Text for an ENTMAXKV_* return code. Static storage; never NULL. */
+ENTMAXKV_API const char *entmaxkv_strerror(int code);
+
+/* Library version as 10000*major + 100*minor + patch. */
+ENTMAXKV_API int entmaxkv_version(void);
+
+/*
+ * Bytes of the metadata buffer written by entmaxkv_build_meta and read by
+ * entmaxkv_score_pages: num_blocks * Hkv * 12 * d.  Layout (record r =
+ * block * Hkv + kv_head):
+ *   bytes [0, R*4d):          bound region, record r at r*4d:
+ *                             kmin bf16[d] then kmax bf16[d]
+ *   bytes [R*4d, R*12d):      moment region, record r at R*4d + r*8d:
+ *                             mean f32[d] then var f32[d]
+ * with R = num_blocks * Hkv.  Returns 0 for an invalid shape.
+ */
+ENTMAXKV_API size_t entmaxkv_meta_bytes(const entmaxkv_shape *shape);
+
+/*
+ * Workspace bytes needed by `call` (ENTMAXKV_CALL_*) for this shape on the
+ * current device; 0 means the call needs none.  Returns (size_t)-1 for an
+ * invalid shape or call.  The caller allocates it (any device memory, 256-byte
+ * aligned) and passes it with its size; contents need not be initialised and
+ * are scratch after the call.  Calls that may overlap on the GPU need separate
+ * workspaces.
+ */
+ENTMAXKV_API size_t entmaxkv_workspace_size(const entmaxkv_shape *shape, int call);
+
+/*
+ * Read the device status word of the current device into *status_out
+ * (ENTMAXKV_STATUS_* bits) after synchronising `stream`; clear it when
+ * `clear` != 0.  The word is shared by all calls on the device.
+ */
+ENTMAXKV_API int entmaxkv_get_status(int32_t *status_out, int clear, void *stream);
+
+/*
+ * Section 2.A (bounding box and Gaussian statistics, "maintained on append"):
+ * for each sequence b, each logical page p in [first_page, first_page+n_pages)
+ * with p < N_b (n_pages = -1: to the end), and each kv head, recompute the
+ * metadata record of block page_table[b][p] from its n = min(P, seq_len - pP)
+ * valid tokens, per coordinate j:
+ *   kmin_j, kmax_j : the bf16 extreme (first token wins exact ties)
+ *   mean_j = fp32(S1/n),  var_j = fp32(max(0, S2/n - (S1/n)^2))
+ * with S1 = sum k_tj, S2 = sum k_tj^2 accumulated in fp64 in token order (the
+ * result is defined to the bit).  Calling it on the page a new token was
+ * appended to keeps the metadata current.  Records of blocks no listed page
+ * maps to are not touched.
+ */
+ENTMAXKV_API int entmaxkv_build_meta(const entmaxkv_shape *shape, const void *k_cache,
+                        const int32_t *page_table, const int32_t *seq_lens,
+                        int32_t first_page, int32_t n_pages, void *meta,
+                        void *stream);
+
+/*
+ * Section 2.A (query-aware page scoring): for every (b, h) and page p < N_b,
+ *   bbox[b][h][p]  = fp32( (sum_j max(q_j kmin_j, q_j kmax_j)) / sqrt(d) )
+ *   mu[b][h][p]    = fp32( (sum_j q_j mean_j) / sqrt(d) )
+ *   sigma[b][h][p] = fp32( sqrt( (sum_j q_j^2 var_j) / d ) )
+ * bbox bounds every token score s of the page from above.  Each sum runs in
+ * fp64 over j in index order (products are exact), so results are defined to
+ * the bit.  Outputs are fp32 [B][Hq][max_pages]; entries for p >= N_b are not
+ * written.  mu and sigma may both be NULL (bound only, reads 4d bytes per
+ * record instead of 12d); if one is non-NULL both must be.
+ */
+ENTMAXKV_API int entmaxkv_score_pages(const entmaxkv_shape *shape, const void *q,
+                         const void *meta, const int32_t *page_table,
+                         const int32_t *seq_lens, float *bbox, float *mu,
+                         float *sigma, void *stream);
+
+/*
+ * Section 2.B (candidate selection), per (b, h), written to
+ * sel[b][h][0..cnt[b][h]) in ascending page order:
+ *  ENTMAXKV_TOPK:  the k pages of largest bbox (k clipped to N_b; ties go to
+ *                  the lower page index).  mu, sigma, delta, tau_hat unused.
+ *  ENTMAXKV_GAUSS: tau_hat solves the approximate normalisation equation
+ *                    sum_p n_p E[(X_p - tau)_+^r] = 1,
+ *                    X_p ~ N((alpha-1) mu_p, (alpha-1)^2 sigma_p^2),
+ *                    r = 1/(alpha-1) (must be an integer 1..8, else
+ *                    ENTMAXKV_ERR_UNSUPPORTED),
+ *                  and the pages kept are those with (alpha-1) bbox_p >
+ *                  tau_hat - delta (the bound is the estimated max score).
+ *                  tau_hat (nullable, fp32 [B][Hq]) receives the solution.
+ * sel is int32 [B][Hq][max_pages], cnt int32 [B][Hq].  Needs alpha > 1 for
+ * the Gaussian policy.  workspace may be NULL when entmaxkv_workspace_size
+ * reports 0.
+ */
+ENTMAXKV_API int entmaxkv_select(const entmaxkv_shape *shape, const int32_t *seq_lens,
+                    const float *bbox, const float *mu, const float *sigma,
+                    int32_t policy, int32_t k, float alpha, float delta,
+                    int32_t *sel, int32_t *cnt, float *tau_hat,
+                    void *workspace, size_t ws_bytes, void *stream);
+
+/*
+ * Section 2.C (sparse entmax attention): for each (b, h), over the tokens T of
+ * the pages sel[b][h][0..cnt[b][h]) (ascending, as written by
+ * entmaxkv_select), compute s_t, z_t = (alpha-1) s_t, the exact threshold
+ * tau with sum_{t in T} [z_t - tau]_+^(1/(alpha-1)) = 1, p_t and
+ *   out[b][h] = sum_t p_t v_t      (fp32 [B][Hq][d]).
+ * If T contains the full-cache support, out equals the full-cache result.
+ * Each page selected by any head of a GQA group is read once for the whole
+ * group; value rows whose weight is zero for every head of the group are not
+ * read.  alpha > 1.  tau_out (nullable) fp32 [B][Hq].  p_out (nullable, for
+ * checking) fp32 [B][Hq][max_pages*P] in logical token order: for every
+ * selected page, p of its valid tokens is written (0 off the support); other
+ * entries are left untouched.  A head with no selected page gets out = 0 and
+ * tau = NaN.
+ */
+ENTMAXKV_API int entmaxkv_decode_sparse(const entmaxkv_shape *shape, const void *q,
+                           const void *k_cache, const void *v_cache,
+                           const int32_t *page_table, const int32_t *seq_lens,
+                           const int32_t *sel, const int32_t *cnt, float alpha,
+                           float *out, float *tau_out, float *p_out,
+                           void *workspace, size_t ws_bytes, void *stream);
+
+/*
+ * Section 4 comparison paths, over every token of every sequence:
+ *  alpha > 1:  full-cache alpha-entmax (all of K and all of V are read):
+ *              out = sum_t p_t v_t; tau_out (nullable) gets tau.
+ *  alpha == 1: full-cache softmax, split over pages with a combine step:
+ *              out = sum_t softmax(s)_t v_t; tau_out (nullable) gets max_t s_t.
+ * out fp32 [B][Hq][d].  p_out as in entmaxkv_decode_sparse (alpha > 1 only;
+ * must be NULL for alpha == 1).
+ */
+ENTMAXKV_API int entmaxkv_decode_dense(const entmaxkv_shape *shape, const void *q,
+                          const void *k_cache, const void *v_cache,
+                          const int32_t *page_table, const int32_t *seq_lens,
+                          float alpha, float *out, float *tau_out, float *p_out,
+                          void *workspace, size_t ws_bytes, void *stream);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* ENTMAXKV_H */

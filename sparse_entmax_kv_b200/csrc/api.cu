@@ -1,0 +1,319 @@
+// api.cu -- the C ABI declared in include/entmaxkv.h: argument checks (all on
+// the host, before any CUDA call), workspace carving, TMA descriptor set-up,
+// and the per-device status word.
+#include <cudaTypedefs.h>
+
+#include <cmath>
+#include <cstring>
+#include <mutex>
+
+#include "common.cuh"
+#include "internal.h"
+
+using namespace ekv;
+
+namespace {
+
+__device__ int g_status;  // ENTMAXKV_STATUS_* bits, one word per device
+
+constexpr int MAX_DEV = 64;
+std::mutex g_mu;
+DevInfo g_dev[MAX_DEV];
+bool g_dev_ok[MAX_DEV];
+
+int device_info(DevInfo *out) {
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= MAX_DEV) return ENTMAXKV_ERR_CUDA;
+    std::lock_guard<std::mutex> lk(g_mu);
+    if (!g_dev_ok[dev]) {
+        DevInfo d{};
+        if (cudaDeviceGetAttribute(&d.sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess)
+            return ENTMAXKV_ERR_CUDA;
+        if (cudaGetSymbolAddress(reinterpret_cast<void **>(&d.status), g_status) != cudaSuccess)
+            return ENTMAXKV_ERR_CUDA;
+        g_dev[dev] = d;
+        g_dev_ok[dev] = true;
+    }
+    *out = g_dev[dev];
+    return ENTMAXKV_OK;
+}
+
+PFN_cuTensorMapEncodeTiled_v12000 g_encode = nullptr;
+
+int get_encoder() {
+    std::lock_guard<std::mutex> lk(g_mu);
+    if (g_encode) return ENTMAXKV_OK;
+    void *fn = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &fn, cudaEnableDefault, &q) != cudaSuccess ||
+        q != cudaDriverEntryPointSuccess || fn == nullptr)
+        return ENTMAXKV_ERR_CUDA;
+    g_encode = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(fn);
+    return ENTMAXKV_OK;
+}
+
+// 2-D view of a paged cache: rows = num_blocks*Hkv*P tokens, d bf16 columns;
+// box = 64 columns x P rows, 128-byte swizzle (conflict-free ldmatrix reads).
+int make_kv_map(CUtensorMap *m, const void *base, const entmaxkv_shape *s) {
+    int rc = get_encoder();
+    if (rc) return rc;
+    cuuint64_t dims[2] = {(cuuint64_t)s->d, (cuuint64_t)s->num_blocks * s->Hkv * s->page_size};
+    cuuint64_t strides[1] = {(cuuint64_t)s->d * 2};
+    cuuint32_t box[2] = {64, (cuuint32_t)s->page_size};
+    cuuint32_t estr[2] = {1, 1};
+    CUresult r = g_encode(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void *>(base), dims, strides, box, estr,
+                          CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                          CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    return r == CUDA_SUCCESS ? ENTMAXKV_OK : ENTMAXKV_ERR_CUDA;
+}
+
+bool aligned16(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+constexpr int MAX_SEL_PAGES = 196608;
+
+int check_shape(const entmaxkv_shape *s) {
+    if (!s) return ENTMAXKV_ERR_NULL;
+    if (s->B < 1 || s->Hq < 1 || s->Hkv < 1 || s->max_pages < 1 || s->num_blocks < 1) return ENTMAXKV_ERR_SHAPE;
+    if (s->Hq % s->Hkv) return ENTMAXKV_ERR_SHAPE;
+    const int G = s->Hq / s->Hkv;
+    if (G != 1 && G != 2 && G != 4 && G != 8) return ENTMAXKV_ERR_SHAPE;
+    if (s->d != 64 && s->d != 128) return ENTMAXKV_ERR_SHAPE;
+    if (s->page_size != 16 && s->page_size != 32 && s->page_size != 64) return ENTMAXKV_ERR_SHAPE;
+    if ((long long)s->max_pages * s->page_size >= (1ll << 31)) return ENTMAXKV_ERR_SHAPE;
+    if ((long long)s->num_blocks * s->Hkv * s->page_size >= (1ll << 31)) return ENTMAXKV_ERR_SHAPE;
+    if (s->B > 65535 || s->Hq > 65535 || (long long)s->B * s->Hq >= (1ll << 31)) return ENTMAXKV_ERR_SHAPE;
+    return ENTMAXKV_OK;
+}
+
+// 1/(alpha-1) when it is an integer in 1..8, else 0.
+int integer_r(float alpha) {
+    const double r = 1.0 / ((double)alpha - 1.0);
+    const double ri = std::floor(r + 0.5);
+    if (ri >= 1.0 && ri <= 8.0 && std::fabs(r - ri) <= 1e-5 * ri) return (int)ri;
+    return 0;
+}
+
+int cuda_rc(cudaError_t e) { return e == cudaSuccess ? ENTMAXKV_OK : ENTMAXKV_ERR_CUDA; }
+
+}  // namespace
+
+extern "C" {
+
+const char *entmaxkv_strerror(int code) {
+    switch (code) {
+        case ENTMAXKV_OK: return "ok";
+        case ENTMAXKV_ERR_NULL: return "a required pointer is NULL";
+        case ENTMAXKV_ERR_SHAPE: return "shape out of range or inconsistent";
+        case ENTMAXKV_ERR_ALPHA: return "alpha out of range for this call";
+        case ENTMAXKV_ERR_POLICY: return "unknown selection policy, k < 1, or delta not finite";
+        case ENTMAXKV_ERR_WORKSPACE: return "workspace missing or too small";
+        case ENTMAXKV_ERR_CUDA: return "CUDA runtime or driver error";
+        case ENTMAXKV_ERR_UNSUPPORTED: return "valid arguments that this build does not support";
+        case ENTMAXKV_ERR_ALIGN: return "pointer not 16-byte aligned";
+        default: return "unknown error code";
+    }
+}
+
+int entmaxkv_version(void) { return 100; }
+
+size_t entmaxkv_meta_bytes(const entmaxkv_shape *s) {
+    if (check_shape(s)) return 0;
+    return (size_t)s->num_blocks * s->Hkv * 12 * s->d;
+}
+
+size_t entmaxkv_workspace_size(const entmaxkv_shape *s, int call) {
+    if (check_shape(s)) return (size_t)-1;
+    switch (call) {
+        case ENTMAXKV_CALL_SELECT: return 0;
+        case ENTMAXKV_CALL_DECODE_SPARSE:
+        case ENTMAXKV_CALL_DECODE_DENSE:
+            return decode_ws_bytes(s->B, s->Hq, s->Hkv, s->d, s->page_size, s->max_pages, nullptr, nullptr);
+        default: return (size_t)-1;
+    }
+}
+
+int entmaxkv_get_status(int32_t *status_out, int clear, void *stream) {
+    if (!status_out) return ENTMAXKV_ERR_NULL;
+    DevInfo di;
+    int rc = device_info(&di);
+    if (rc) return rc;
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    int v = 0;
+    if (cudaMemcpyAsync(&v, di.status, sizeof(int), cudaMemcpyDeviceToHost, st) != cudaSuccess)
+        return ENTMAXKV_ERR_CUDA;
+    if (cudaStreamSynchronize(st) != cudaSuccess) return ENTMAXKV_ERR_CUDA;
+    if (clear && cudaMemsetAsync(di.status, 0, sizeof(int), st) != cudaSuccess) return ENTMAXKV_ERR_CUDA;
+    *status_out = v;
+    return ENTMAXKV_OK;
+}
+
+int entmaxkv_build_meta(const entmaxkv_shape *s, const void *k_cache, const int32_t *page_table,
+                        const int32_t *seq_lens, int32_t first_page, int32_t n_pages, void *meta, void *stream) {
+    int rc = check_shape(s);
+    if (rc) return rc;
+    if (!k_cache || !page_table || !seq_lens || !meta) return ENTMAXKV_ERR_NULL;
+    if (!aligned16(k_cache) || !aligned16(meta)) return ENTMAXKV_ERR_ALIGN;
+    if (first_page < 0 || first_page > s->max_pages || n_pages < -1) return ENTMAXKV_ERR_SHAPE;
+    int n = n_pages < 0 ? s->max_pages - first_page : n_pages;
+    if (first_page + n > s->max_pages) n = s->max_pages - first_page;
+    DevInfo di;
+    if ((rc = device_info(&di))) return rc;
+    MetaArgs a{};
+    a.k = static_cast<const uint16_t *>(k_cache);
+    a.page_table = page_table;
+    a.seq_lens = seq_lens;
+    a.meta = static_cast<uint8_t *>(meta);
+    a.R = (long long)s->num_blocks * s->Hkv;
+    a.B = s->B;
+    a.Hkv = s->Hkv;
+    a.d = s->d;
+    a.P = s->page_size;
+    a.max_pages = s->max_pages;
+    a.num_blocks = s->num_blocks;
+    a.first_page = first_page;
+    a.n_pages = n;
+    a.status = di.status;
+    return cuda_rc(launch_build_meta(a, static_cast<cudaStream_t>(stream)));
+}
+
+int entmaxkv_score_pages(const entmaxkv_shape *s, const void *q, const void *meta, const int32_t *page_table,
+                         const int32_t *seq_lens, float *bbox, float *mu, float *sigma, void *stream) {
+    int rc = check_shape(s);
+    if (rc) return rc;
+    if (!q || !meta || !page_table || !seq_lens || !bbox) return ENTMAXKV_ERR_NULL;
+    if ((mu == nullptr) != (sigma == nullptr)) return ENTMAXKV_ERR_NULL;
+    if (!aligned16(q) || !aligned16(meta)) return ENTMAXKV_ERR_ALIGN;
+    DevInfo di;
+    if ((rc = device_info(&di))) return rc;
+    ScoreArgs a{};
+    a.q = static_cast<const uint16_t *>(q);
+    a.meta = static_cast<const uint8_t *>(meta);
+    a.page_table = page_table;
+    a.seq_lens = seq_lens;
+    a.bbox = bbox;
+    a.mu = mu;
+    a.sigma = sigma;
+    a.R = (long long)s->num_blocks * s->Hkv;
+    a.B = s->B;
+    a.Hq = s->Hq;
+    a.Hkv = s->Hkv;
+    a.d = s->d;
+    a.P = s->page_size;
+    a.max_pages = s->max_pages;
+    a.num_blocks = s->num_blocks;
+    a.status = di.status;
+    return cuda_rc(launch_score_pages(a, static_cast<cudaStream_t>(stream)));
+}
+
+int entmaxkv_select(const entmaxkv_shape *s, const int32_t *seq_lens, const float *bbox, const float *mu,
+                    const float *sigma, int32_t policy, int32_t k, float alpha, float delta, int32_t *sel,
+                    int32_t *cnt, float *tau_hat, void *workspace, size_t ws_bytes, void *stream) {
+    (void)workspace;
+    (void)ws_bytes;
+    int rc = check_shape(s);
+    if (rc) return rc;
+    if (s->max_pages > MAX_SEL_PAGES) return ENTMAXKV_ERR_SHAPE;
+    if (!seq_lens || !bbox || !sel || !cnt) return ENTMAXKV_ERR_NULL;
+    SelectArgs a{};
+    if (policy == ENTMAXKV_TOPK) {
+        if (k < 1) return ENTMAXKV_ERR_POLICY;
+    } else if (policy == ENTMAXKV_GAUSS) {
+        if (!mu || !sigma) return ENTMAXKV_ERR_NULL;
+        if (!std::isfinite(delta)) return ENTMAXKV_ERR_POLICY;
+        if (!std::isfinite(alpha) || !(alpha > 1.f)) return ENTMAXKV_ERR_ALPHA;
+        a.r_int = integer_r(alpha);
+        if (a.r_int == 0) return ENTMAXKV_ERR_UNSUPPORTED;
+    } else {
+        return ENTMAXKV_ERR_POLICY;
+    }
+    DevInfo di;
+    if ((rc = device_info(&di))) return rc;
+    a.seq_lens = seq_lens;
+    a.bbox = bbox;
+    a.mu = mu;
+    a.sigma = sigma;
+    a.sel = sel;
+    a.cnt = cnt;
+    a.tau_hat = tau_hat;
+    a.B = s->B;
+    a.Hq = s->Hq;
+    a.P = s->page_size;
+    a.max_pages = s->max_pages;
+    a.policy = policy;
+    a.k = k;
+    a.alpha = alpha;
+    a.delta = delta;
+    a.status = di.status;
+    return cuda_rc(launch_select(a, static_cast<cudaStream_t>(stream)));
+}
+
+static int fill_decode(const entmaxkv_shape *s, const void *q, const void *k_cache, const void *v_cache,
+                       const int32_t *page_table, const int32_t *seq_lens, float alpha, float *out, float *tau_out,
+                       float *p_out, void *workspace, size_t ws_bytes, DecodeArgs *a) {
+    int rc = check_shape(s);
+    if (rc) return rc;
+    if (!q || !k_cache || !v_cache || !page_table || !seq_lens || !out) return ENTMAXKV_ERR_NULL;
+    if (!aligned16(q) || !aligned16(k_cache) || !aligned16(v_cache)) return ENTMAXKV_ERR_ALIGN;
+    if (!std::isfinite(alpha)) return ENTMAXKV_ERR_ALPHA;
+    const size_t need = decode_ws_bytes(s->B, s->Hq, s->Hkv, s->d, s->page_size, s->max_pages, nullptr, nullptr);
+    if (!workspace || ws_bytes < need) return ENTMAXKV_ERR_WORKSPACE;
+    if ((reinterpret_cast<uintptr_t>(workspace) & 255u) != 0) return ENTMAXKV_ERR_ALIGN;
+    DevInfo di;
+    if ((rc = device_info(&di))) return rc;
+    std::memset(a, 0, sizeof(*a));
+    a->q = static_cast<const uint16_t *>(q);
+    a->k = static_cast<const uint16_t *>(k_cache);
+    a->v = static_cast<const uint16_t *>(v_cache);
+    a->page_table = page_table;
+    a->seq_lens = seq_lens;
+    a->out = out;
+    a->tau_out = tau_out;
+    a->p_out = p_out;
+    decode_ws_bytes(s->B, s->Hq, s->Hkv, s->d, s->page_size, s->max_pages, &a->ws, workspace);
+    a->B = s->B;
+    a->Hq = s->Hq;
+    a->Hkv = s->Hkv;
+    a->d = s->d;
+    a->P = s->page_size;
+    a->max_pages = s->max_pages;
+    a->num_blocks = s->num_blocks;
+    a->alpha = alpha;
+    a->r_int = alpha > 1.f ? integer_r(alpha) : 0;
+    a->sms = di.sms;
+    a->status = di.status;
+    return ENTMAXKV_OK;
+}
+
+int entmaxkv_decode_sparse(const entmaxkv_shape *s, const void *q, const void *k_cache, const void *v_cache,
+                           const int32_t *page_table, const int32_t *seq_lens, const int32_t *sel,
+                           const int32_t *cnt, float alpha, float *out, float *tau_out, float *p_out,
+                           void *workspace, size_t ws_bytes, void *stream) {
+    if (!sel || !cnt) return ENTMAXKV_ERR_NULL;
+    if (!(alpha > 1.f)) return ENTMAXKV_ERR_ALPHA;
+    if (s && s->max_pages > MAX_SEL_PAGES) return ENTMAXKV_ERR_SHAPE;
+    DecodeArgs a;
+    int rc = fill_decode(s, q, k_cache, v_cache, page_table, seq_lens, alpha, out, tau_out, p_out, workspace,
+                         ws_bytes, &a);
+    if (rc) return rc;
+    a.sel = sel;
+    a.cnt = cnt;
+    if ((rc = make_kv_map(&a.kmap, k_cache, s))) return rc;
+    return cuda_rc(launch_decode_sparse(a, static_cast<cudaStream_t>(stream)));
+}
+
+int entmaxkv_decode_dense(const entmaxkv_shape *s, const void *q, const void *k_cache, const void *v_cache,
+                          const int32_t *page_table, const int32_t *seq_lens, float alpha, float *out,
+                          float *tau_out, float *p_out, void *workspace, size_t ws_bytes, void *stream) {
+    if (!(alpha >= 1.f)) return ENTMAXKV_ERR_ALPHA;
+    if (alpha == 1.f && p_out) return ENTMAXKV_ERR_NULL;
+    DecodeArgs a;
+    int rc = fill_decode(s, q, k_cache, v_cache, page_table, seq_lens, alpha, out, tau_out, p_out, workspace,
+                         ws_bytes, &a);
+    if (rc) return rc;
+    if ((rc = make_kv_map(&a.kmap, k_cache, s))) return rc;
+    if ((rc = make_kv_map(&a.vmap, v_cache, s))) return rc;
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    return cuda_rc(alpha == 1.f ? launch_decode_dense_softmax(a, st) : launch_decode_dense_entmax(a, st));
+}
+
+}  // extern "C"

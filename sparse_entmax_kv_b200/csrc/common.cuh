@@ -1,0 +1,205 @@
+// common.cuh -- device helpers shared by the EntmaxKV kernels (sm_100a).
+//
+// PTX wrappers for mbarriers, 1-D bulk copies and 2-D tiled TMA loads (no
+// cluster multicast anywhere), warp-level mma.sync for the bf16 q.K^T tiles,
+// bf16 unpacking and the order-preserving float <-> int32 map used for
+// atomic max.
+#pragma once
+
+#include <cuda.h>
+#include <cuda_bf16.h>
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+#include "../../include/entmaxkv.h"
+
+namespace ekv {
+
+constexpr unsigned FULL = 0xffffffffu;
+// Longest an mbarrier wait may spin before it reports ENTMAXKV_STATUS_TIMEOUT
+// and gives up (nanoseconds of %globaltimer).
+constexpr unsigned long long WAIT_LIMIT_NS = 2000000000ull;
+
+__device__ __forceinline__ unsigned smem_u32(const void *p) {
+    return static_cast<unsigned>(__cvta_generic_to_shared(p));
+}
+
+__device__ __forceinline__ unsigned long long globaltimer() {
+    unsigned long long t;
+    asm volatile("mov.u64 %0, %globaltimer;" : "=l"(t));
+    return t;
+}
+
+// ------------------------------------------------------------- mbarrier
+
+__device__ __forceinline__ void mbar_init(uint64_t *bar, unsigned count) {
+    asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(smem_u32(bar)), "r"(count)
+                 : "memory");
+}
+
+__device__ __forceinline__ void mbar_fence_init() {
+    asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+}
+
+__device__ __forceinline__ void mbar_arrive_expect_tx(uint64_t *bar, unsigned bytes) {
+    asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(smem_u32(bar)),
+                 "r"(bytes)
+                 : "memory");
+}
+
+__device__ __forceinline__ void mbar_arrive(uint64_t *bar) {
+    asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(smem_u32(bar)) : "memory");
+}
+
+__device__ __forceinline__ bool mbar_test(uint64_t *bar, unsigned parity) {
+    unsigned ok;
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "mbarrier.test_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+        "selp.u32 %0, 1, 0, p;\n\t}"
+        : "=r"(ok)
+        : "r"(smem_u32(bar)), "r"(parity)
+        : "memory");
+    return ok != 0;
+}
+
+// Bounded wait for the phase with the given parity.  Returns false (and sets
+// the TIMEOUT status bit) if it did not complete within WAIT_LIMIT_NS.
+__device__ __forceinline__ bool mbar_wait(uint64_t *bar, unsigned parity, int *status) {
+    if (mbar_test(bar, parity)) return true;
+    unsigned long long t0 = globaltimer();
+    for (unsigned it = 0; it < (1u << 30); ++it) {
+        if (mbar_test(bar, parity)) return true;
+        if ((it & 63u) == 63u) {
+            __nanosleep(64);
+            if (globaltimer() - t0 > WAIT_LIMIT_NS) break;
+        }
+    }
+    if (status) atomicOr(status, ENTMAXKV_STATUS_TIMEOUT);
+    return false;
+}
+
+// -------------------------------------------------------- bulk / TMA copies
+
+// 1-D bulk copy global -> shared, completion counted on `bar` (bytes).
+// dst, src 16-byte aligned; bytes a multiple of 16.
+__device__ __forceinline__ void bulk_g2s(void *dst, const void *src, unsigned bytes, uint64_t *bar) {
+    asm volatile(
+        "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(
+            smem_u32(dst)),
+        "l"(src), "r"(bytes), "r"(smem_u32(bar))
+        : "memory");
+}
+
+// 2-D tiled TMA load of one box at element coordinates (x, y) (x = innermost).
+// x * sizeof(element) must be a multiple of 16 bytes.
+__device__ __forceinline__ void tma_load_2d(void *dst, const CUtensorMap *map, int x, int y, uint64_t *bar) {
+    asm volatile(
+        "cp.async.bulk.tensor.2d.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1, {%2, %3}], [%4];" ::"r"(
+            smem_u32(dst)),
+        "l"(reinterpret_cast<uint64_t>(map)), "r"(x), "r"(y), "r"(smem_u32(bar))
+        : "memory");
+}
+
+__device__ __forceinline__ void prefetch_tmap(const CUtensorMap *map) {
+    asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(map)) : "memory");
+}
+
+// Ampere-style 16-byte async copy (bypasses L1), grouped with commit/wait.
+__device__ __forceinline__ void cp_async16(void *dst, const void *src) {
+    asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(smem_u32(dst)), "l"(src) : "memory");
+}
+__device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
+template <int N>
+__device__ __forceinline__ void cp_async_wait() {
+    asm volatile("cp.async.wait_group %0;" ::"n"(N) : "memory");
+}
+
+// ------------------------------------------------------------ tensor cores
+
+// ldmatrix x4 (four 8x8 b16 matrices), one row address per lane.
+__device__ __forceinline__ void ldsm_x4(unsigned addr, unsigned &r0, unsigned &r1, unsigned &r2, unsigned &r3) {
+    asm volatile("ldmatrix.sync.aligned.m8n8.x4.shared.b16 {%0, %1, %2, %3}, [%4];"
+                 : "=r"(r0), "=r"(r1), "=r"(r2), "=r"(r3)
+                 : "r"(addr));
+}
+
+// D = A(16x16 bf16, row) * B(16x8 bf16, col) + C, fp32 accumulate.
+__device__ __forceinline__ void mma_bf16_16816(float (&c)[4], unsigned a0, unsigned a1, unsigned a2, unsigned a3,
+                                               unsigned b0, unsigned b1) {
+    asm volatile(
+        "mma.sync.aligned.m16n8k16.row.col.f32.bf16.bf16.f32 {%0, %1, %2, %3}, {%4, %5, %6, %7}, {%8, %9}, "
+        "{%0, %1, %2, %3};"
+        : "+f"(c[0]), "+f"(c[1]), "+f"(c[2]), "+f"(c[3])
+        : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
+}
+
+// --------------------------------------------------------------- numbers
+
+__device__ __forceinline__ float bf16lo(unsigned w) { return __uint_as_float(w << 16); }
+__device__ __forceinline__ float bf16hi(unsigned w) { return __uint_as_float(w & 0xffff0000u); }
+__device__ __forceinline__ float bf16f(uint16_t h) { return __uint_as_float(((unsigned)h) << 16); }
+
+// Order-preserving map float -> int32 (for atomicMax) and back.
+__device__ __forceinline__ int f2ord(float f) {
+    int i = __float_as_int(f);
+    return i >= 0 ? i : i ^ 0x7fffffff;
+}
+__device__ __forceinline__ float ord2f(int i) { return __int_as_float(i >= 0 ? i : i ^ 0x7fffffff); }
+constexpr int ORD_NEG_INF = (int)(0xff800000u ^ 0x7fffffffu);  // f2ord(-inf)
+
+__host__ __device__ __forceinline__ int ceil_div(int a, int b) { return (a + b - 1) / b; }
+
+__device__ __forceinline__ int n_pages_of(int seq_len, int P) { return seq_len > 0 ? (seq_len + P - 1) / P : 0; }
+__device__ __forceinline__ int tokens_in_page(int seq_len, int P, int p) {
+    int n = seq_len - p * P;
+    return n > P ? P : (n < 0 ? 0 : n);
+}
+
+// [x]_+^r.  ri = r when r is an integer in 1..8 (repeated products), ri = 0
+// for any other exponent (powf).
+__device__ __forceinline__ float pos_pow(float x, float r, int ri) {
+    if (!(x > 0.f)) return 0.f;
+    switch (ri) {
+        case 1: return x;
+        case 2: return x * x;
+        case 3: return x * x * x;
+        case 4: { float y = x * x; return y * y; }
+        case 5: { float y = x * x; return y * y * x; }
+        case 6: { float y = x * x * x; return y * y; }
+        case 7: { float y = x * x * x; return y * y * x; }
+        case 8: { float y = x * x; y = y * y; return y * y; }
+        default: return powf(x, r);
+    }
+}
+
+// Block-wide exclusive scan of one int per thread, in thread order.  `sh`
+// needs 65 ints of shared memory; *total receives the block total.
+__device__ __forceinline__ int block_excl_scan(int v, int *sh, int *total) {
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5, nw = blockDim.x >> 5;
+    int x = v;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+        int y = __shfl_up_sync(FULL, x, o);
+        if (lane >= o) x += y;
+    }
+    __syncthreads();
+    if (lane == 31) sh[warp] = x;
+    __syncthreads();
+    if (warp == 0) {
+        int w = lane < nw ? sh[lane] : 0;
+        int ws = w;
+#pragma unroll
+        for (int o = 1; o < 32; o <<= 1) {
+            int y = __shfl_up_sync(FULL, ws, o);
+            if (lane >= o) ws += y;
+        }
+        if (lane < nw) sh[32 + lane] = ws - w;
+        if (lane == nw - 1) sh[64] = ws;
+    }
+    __syncthreads();
+    *total = sh[64];
+    return sh[32 + warp] + x - v;
+}
+
+}  // namespace ekv

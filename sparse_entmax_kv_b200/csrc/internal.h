@@ -1,0 +1,88 @@
+// internal.h -- host-side launch interface between the C ABI (api.cu) and the
+// kernel translation units.  Not part of the public header.
+#pragma once
+
+#include <cuda.h>
+#include <cuda_runtime.h>
+#include <stddef.h>
+#include <stdint.h>
+
+namespace ekv {
+
+// Most split-K slots a decode call may use per (sequence, head).
+constexpr int MAX_SPLITS = 64;
+
+struct DevInfo {
+    int sms;
+    int *status;  // device address of the status word
+};
+
+struct MetaArgs {
+    const uint16_t *k;
+    const int *page_table;
+    const int *seq_lens;
+    uint8_t *meta;
+    long long R;  // records = num_blocks * Hkv
+    int B, Hkv, d, P, max_pages, num_blocks;
+    int first_page, n_pages;  // n_pages >= 0 here (resolved by the caller)
+    int *status;
+};
+cudaError_t launch_build_meta(const MetaArgs &a, cudaStream_t st);
+
+struct ScoreArgs {
+    const uint16_t *q;
+    const uint8_t *meta;
+    const int *page_table;
+    const int *seq_lens;
+    float *bbox, *mu, *sigma;
+    long long R;
+    int B, Hq, Hkv, d, P, max_pages, num_blocks;
+    int *status;
+};
+cudaError_t launch_score_pages(const ScoreArgs &a, cudaStream_t st);
+
+struct SelectArgs {
+    const int *seq_lens;
+    const float *bbox, *mu, *sigma;
+    int *sel, *cnt;
+    float *tau_hat;
+    int B, Hq, P, max_pages;
+    int policy, k;
+    float alpha, delta;
+    int r_int;  // 1/(alpha-1) for the Gaussian policy
+    int *status;
+};
+cudaError_t launch_select(const SelectArgs &a, cudaStream_t st);
+
+// Workspace carve-up shared by the decode paths.
+struct DecodeWs {
+    int *union_e;    // [B*Hkv][max_pages]   (page << 8) | head mask
+    int *union_cnt;  // [B*Hkv]
+    int *zmax;       // [B*Hq] order-mapped max z
+    float *tau;      // [B*Hq]
+    int *counters;   // [B*Hkv]
+    float *partial;  // [MAX_SPLITS][B*Hq][d+2]
+    float *zbuf;     // [B*Hq][max_pages*P]
+};
+
+struct DecodeArgs {
+    const uint16_t *q;
+    const uint16_t *k, *v;
+    const int *page_table, *seq_lens;
+    const int *sel, *cnt;  // sparse only
+    float *out, *tau_out, *p_out;
+    CUtensorMap kmap, vmap;  // 2-D maps over [num_blocks*Hkv*P rows][d] bf16
+    DecodeWs ws;
+    int B, Hq, Hkv, d, P, max_pages, num_blocks;
+    float alpha;
+    int r_int;  // 1/(alpha-1) if an integer 1..8, else 0
+    int sms;
+    int *status;
+};
+cudaError_t launch_decode_sparse(const DecodeArgs &a, cudaStream_t st);
+cudaError_t launch_decode_dense_entmax(const DecodeArgs &a, cudaStream_t st);
+cudaError_t launch_decode_dense_softmax(const DecodeArgs &a, cudaStream_t st);
+
+size_t decode_ws_bytes(int B, int Hq, int Hkv, int d, int P, int max_pages, DecodeWs *carve, void *base);
+
+}  // namespace ekv

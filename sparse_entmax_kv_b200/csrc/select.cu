@@ -1,0 +1,353 @@
+// select.cu -- candidate page selection (EntmaxKV summary, section 2.B).
+//
+// One CTA per (sequence, query head).
+//
+// Top-k: radix select on the order-preserving 32-bit image of the fp32 bound
+// (four 8-bit digits, most significant first; warp-aggregated shared-memory
+// histograms), which pins the k-th largest key T and how many keys equal to T
+// are still needed; a single ordered pass then keeps keys > T plus the first
+// such keys == T in page order (ties to the lower page index) and writes them
+// in ascending page order.  No sort.
+//
+// Gaussian: tau_hat solves F(tau) = sum_p n_p E[(X_p - tau)_+^r] = 1 with
+// X_p ~ N(m_p, s_p^2), m_p = (alpha-1) mu_p, s_p = (alpha-1) sigma_p, using the
+// closed-form Gaussian partial moments.  F >= 1 at tau0 = max_p m_p - 1
+// (Jensen), and g(tau) = F(tau)^(1/r) is convex and decreasing (an L^r norm of
+// (X - tau)_+), so Newton on g started at tau0 climbs monotonically to the
+// root without overshoot.  Pages with m_p + 10 s_p < tau0 contribute below
+// n_p s_p^r J_r(10) ~ 1e-25 n_p s_p^r at any tau >= tau0 and are pruned before
+// the iterations.  Pages are then kept when (alpha-1) bbox_p > tau_hat - Delta.
+#include "common.cuh"
+#include "internal.h"
+
+namespace ekv {
+
+namespace {
+
+constexpr int SEL_THREADS = 1024;
+constexpr int ITEMS = 16;  // keys per thread per tile
+constexpr int TILE = SEL_THREADS * ITEMS;
+
+__device__ __forceinline__ unsigned key_of(float f) {
+    unsigned x = __float_as_uint(f);
+    return (x & 0x80000000u) ? ~x : (x | 0x80000000u);
+}
+
+__device__ float block_max(float v, float *sh) {
+#pragma unroll
+    for (int o = 16; o; o >>= 1) v = fmaxf(v, __shfl_xor_sync(FULL, v, o));
+    __syncthreads();
+    if ((threadIdx.x & 31) == 0) sh[threadIdx.x >> 5] = v;
+    __syncthreads();
+    float m = -INFINITY;
+    for (int w = 0; w < (int)(blockDim.x >> 5); ++w) m = fmaxf(m, sh[w]);
+    return m;
+}
+
+__device__ void block_sum2(float &a, float &b, float *sh) {
+#pragma unroll
+    for (int o = 16; o; o >>= 1) {
+        a += __shfl_xor_sync(FULL, a, o);
+        b += __shfl_xor_sync(FULL, b, o);
+    }
+    __syncthreads();
+    if ((threadIdx.x & 31) == 0) {
+        sh[2 * (threadIdx.x >> 5)] = a;
+        sh[2 * (threadIdx.x >> 5) + 1] = b;
+    }
+    __syncthreads();
+    float sa = 0.f, sb = 0.f;
+    for (int w = 0; w < (int)(blockDim.x >> 5); ++w) {
+        sa += sh[2 * w];
+        sb += sh[2 * w + 1];
+    }
+    a = sa;
+    b = sb;
+}
+
+// Write sel[] for the pages p < n for which keep(p) holds, ascending.
+template <class Keep>
+__device__ int compact_ascending(int n, int *sel, int *sh, Keep keep) {
+    int base = 0;
+    for (int t0 = 0; t0 < n; t0 += TILE) {
+        const int p0 = t0 + threadIdx.x * ITEMS;
+        unsigned bits = 0;
+#pragma unroll
+        for (int i = 0; i < ITEMS; ++i) {
+            const int p = p0 + i;
+            if (p < n && keep(p)) bits |= 1u << i;
+        }
+        int tot;
+        int off = block_excl_scan(__popc(bits), sh, &tot);
+        int w = base + off;
+#pragma unroll
+        for (int i = 0; i < ITEMS; ++i)
+            if (bits & (1u << i)) sel[w++] = p0 + i;
+        base += tot;
+    }
+    return base;
+}
+
+__global__ void __launch_bounds__(SEL_THREADS) topk_kernel(SelectArgs a) {
+    __shared__ int hist[256];
+    __shared__ int sh[72];
+    __shared__ int pick[2];
+    const int bh = blockIdx.x;
+    const int b = bh / a.Hq;
+    const int n = n_pages_of(a.seq_lens[b], a.P);
+    const float *sc = a.bbox + (size_t)bh * a.max_pages;
+    int *sel = a.sel + (size_t)bh * a.max_pages;
+    const int k = min(a.k, n);
+    if (k >= n) {
+        for (int p = threadIdx.x; p < n; p += blockDim.x) sel[p] = p;
+        if (threadIdx.x == 0) a.cnt[bh] = n;
+        return;
+    }
+    const int lane = threadIdx.x & 31;
+    unsigned prefix = 0, mask = 0;
+    int remaining = k;
+    for (int shift = 24; shift >= 0; shift -= 8) {
+        for (int i = threadIdx.x; i < 256; i += blockDim.x) hist[i] = 0;
+        __syncthreads();
+        const int nround = ceil_div(n, blockDim.x) * blockDim.x;
+        for (int p = threadIdx.x; p < nround; p += blockDim.x) {
+            int bucket = 256 + lane;  // unique dummy for lanes with nothing to count
+            if (p < n) {
+                const unsigned key = key_of(__ldg(sc + p));
+                if ((key & mask) == prefix) bucket = (key >> shift) & 255;
+            }
+            const unsigned peers = __match_any_sync(FULL, bucket);
+            if (bucket < 256 && lane == __ffs(peers) - 1) atomicAdd(&hist[bucket], __popc(peers));
+        }
+        __syncthreads();
+        if (threadIdx.x < 32) {
+            // lane l owns buckets [8l, 8l+8); suffix sums from the top bucket down
+            int c[8], s = 0;
+#pragma unroll
+            for (int i = 0; i < 8; ++i) {
+                c[i] = hist[8 * lane + i];
+                s += c[i];
+            }
+            int suf = s;  // inclusive suffix over lanes >= lane
+#pragma unroll
+            for (int o = 1; o < 32; o <<= 1) {
+                int y = __shfl_down_sync(FULL, suf, o);
+                if (lane + o < 32) suf += y;
+            }
+            const int above = suf - s;  // keys in higher lanes' buckets
+            const bool here = above < remaining && remaining <= suf;
+            const unsigned who = __ballot_sync(FULL, here);
+            if (lane == __ffs(who) - 1) {
+                int acc = above, bsel = 8 * lane;
+                for (int i = 7; i >= 0; --i) {
+                    if (acc + c[i] >= remaining) {
+                        bsel = 8 * lane + i;
+                        break;
+                    }
+                    acc += c[i];
+                }
+                pick[0] = bsel;
+                pick[1] = remaining - acc;
+            }
+        }
+        __syncthreads();
+        prefix |= (unsigned)pick[0] << shift;
+        mask |= 255u << shift;
+        remaining = pick[1];
+        __syncthreads();
+    }
+    const unsigned T = prefix;
+    // keys == T are taken in page order up to `remaining` of them
+    int eq_base = 0, base = 0;
+    for (int t0 = 0; t0 < n; t0 += TILE) {
+        const int p0 = t0 + threadIdx.x * ITEMS;
+        unsigned gt = 0, eq = 0;
+#pragma unroll
+        for (int i = 0; i < ITEMS; ++i) {
+            const int p = p0 + i;
+            if (p < n) {
+                const unsigned key = key_of(__ldg(sc + p));
+                if (key > T) gt |= 1u << i;
+                if (key == T) eq |= 1u << i;
+            }
+        }
+        int eq_tot;
+        int eq_off = eq_base + block_excl_scan(__popc(eq), sh, &eq_tot);
+        unsigned take = gt;
+#pragma unroll
+        for (int i = 0; i < ITEMS; ++i)
+            if (eq & (1u << i)) {
+                if (eq_off < remaining) take |= 1u << i;
+                ++eq_off;
+            }
+        int tot;
+        int w = base + block_excl_scan(__popc(take), sh, &tot);
+#pragma unroll
+        for (int i = 0; i < ITEMS; ++i)
+            if (take & (1u << i)) sel[w++] = p0 + i;
+        base += tot;
+        eq_base += eq_tot;
+    }
+    if (threadIdx.x == 0) a.cnt[bh] = base;
+}
+
+// Gaussian partial moments of a standard normal: J_R(c) = E[(Z-c)_+^R] and
+// J_{R-1}(c), from M_i(c) = E[Z^i 1{Z>c}] (M_0 = erfc(c/sqrt2)/2, M_1 = phi(c),
+// M_i = c^{i-1} phi(c) + (i-1) M_{i-2}) and the binomial expansion of (Z-c)^R.
+__host__ __device__ constexpr float binomf(int n, int k) {
+    float r = 1.f;
+    for (int t = 0; t < k; ++t) r = r * (float)(n - t) / (float)(t + 1);
+    return r;
+}
+
+template <int R>
+__device__ __forceinline__ void gauss_JJ(float c, float &jr, float &jr1) {
+    float M[R + 1], pw[R + 1];
+    const float phi = 0.3989422804014327f * expf(-0.5f * c * c);
+    M[0] = 0.5f * erfcf(c * 0.7071067811865476f);
+    if (R >= 1) M[1] = phi;
+    float cp = 1.f;  // c^{i-1}
+#pragma unroll
+    for (int i = 2; i <= R; ++i) {
+        cp *= c;
+        M[i] = cp * phi + (float)(i - 1) * M[i - 2];
+    }
+    pw[0] = 1.f;
+#pragma unroll
+    for (int i = 1; i <= R; ++i) pw[i] = pw[i - 1] * (-c);
+    float s = 0.f, s1 = 0.f;
+#pragma unroll
+    for (int i = 0; i <= R; ++i) s += binomf(R, i) * pw[R - i] * M[i];
+#pragma unroll
+    for (int i = 0; i <= R - 1; ++i) s1 += binomf(R - 1, i) * pw[R - 1 - i] * M[i];
+    jr = fmaxf(s, 0.f);
+    jr1 = fmaxf(s1, 0.f);
+}
+
+constexpr int GCAP = 3072;  // pruned candidate pages held on chip
+
+template <int R>
+__global__ void __launch_bounds__(SEL_THREADS) gauss_kernel(SelectArgs a) {
+    __shared__ float cm[GCAP], cs[GCAP], cn[GCAP];
+    __shared__ float shf[2 * 32 + 2];
+    __shared__ int shi[72];
+    __shared__ int ncand;
+    const int bh = blockIdx.x;
+    const int b = bh / a.Hq;
+    const int seq = a.seq_lens[b];
+    const int n = n_pages_of(seq, a.P);
+    const size_t row = (size_t)bh * a.max_pages;
+    const float a1 = a.alpha - 1.f;
+    if (n == 0) {
+        if (threadIdx.x == 0) {
+            a.cnt[bh] = 0;
+            if (a.tau_hat) a.tau_hat[bh] = __int_as_float(0x7fc00000);
+        }
+        return;
+    }
+    float mloc = -INFINITY;
+    for (int p = threadIdx.x; p < n; p += blockDim.x) mloc = fmaxf(mloc, a1 * a.mu[row + p]);
+    const float mmax = block_max(mloc, shf);
+    const float tau0 = mmax - 1.f;
+
+    if (threadIdx.x == 0) ncand = 0;
+    __syncthreads();
+    const int nround = ceil_div(n, blockDim.x) * blockDim.x;
+    for (int p = threadIdx.x; p < nround; p += blockDim.x) {
+        float m = 0.f, s = 0.f;
+        bool keep = false;
+        if (p < n) {
+            m = a1 * a.mu[row + p];
+            s = a1 * a.sigma[row + p];
+            keep = m + 10.f * s >= tau0;
+        }
+        const unsigned bal = __ballot_sync(FULL, keep);
+        int base = 0;
+        if ((threadIdx.x & 31) == 0 && bal) base = atomicAdd(&ncand, __popc(bal));
+        base = __shfl_sync(FULL, base, 0);
+        if (keep) {
+            const int slot = base + __popc(bal & ((1u << (threadIdx.x & 31)) - 1u));
+            if (slot < GCAP) {
+                cm[slot] = m;
+                cs[slot] = s;
+                cn[slot] = (float)tokens_in_page(seq, a.P, p);
+            }
+        }
+    }
+    __syncthreads();
+    const int nc = ncand;
+    const bool overflow = nc > GCAP;
+    if (overflow && threadIdx.x == 0) atomicOr(a.status, ENTMAXKV_STATUS_OVERFLOW);
+
+    auto contrib = [&](float m, float s, float w, float tau, float &F, float &Fp) {
+        if (s > 1e-30f) {
+            const float c = (tau - m) / s;
+            if (c > 38.f) return;
+            float jr, jr1;
+            gauss_JJ<R>(c, jr, jr1);
+            float sp = 1.f;
+#pragma unroll
+            for (int i = 1; i < R; ++i) sp *= s;  // s^(R-1)
+            F += w * sp * s * jr;
+            Fp -= (float)R * w * sp * jr1;
+        } else {
+            const float x = m - tau;
+            if (x > 0.f) {
+                float xp = 1.f;
+#pragma unroll
+                for (int i = 1; i < R; ++i) xp *= x;
+                F += w * xp * x;
+                Fp -= (float)R * w * xp;
+            }
+        }
+    };
+
+    float tau = tau0;
+    for (int it = 0; it < 64; ++it) {
+        float F = 0.f, Fp = 0.f;
+        if (!overflow) {
+            for (int i = threadIdx.x; i < nc; i += blockDim.x) contrib(cm[i], cs[i], cn[i], tau, F, Fp);
+        } else {
+            for (int p = threadIdx.x; p < n; p += blockDim.x)
+                contrib(a1 * a.mu[row + p], a1 * a.sigma[row + p], (float)tokens_in_page(seq, a.P, p), tau, F,
+                        Fp);
+        }
+        block_sum2(F, Fp, shf);
+        if (!(F > 1.f + 2e-6f) || !(Fp < 0.f)) break;
+        // Newton on g = F^(1/R): step = R (F - F^(1-1/R)) / (-F')
+        const float step = (float)R * (F - powf(F, 1.f - 1.f / (float)R)) / (-Fp);
+        tau += step;
+        if (!(step > 1e-7f * fmaxf(1.f, fabsf(tau)))) break;
+    }
+    if (threadIdx.x == 0 && a.tau_hat) a.tau_hat[bh] = tau;
+
+    const float thr = tau - a.delta;
+    const float *bb = a.bbox + row;
+    int *sel = a.sel + row;
+    const int cnt = compact_ascending(n, sel, shi, [&](int p) { return a1 * __ldg(bb + p) > thr; });
+    if (threadIdx.x == 0) a.cnt[bh] = cnt;
+}
+
+}  // namespace
+
+cudaError_t launch_select(const SelectArgs &a, cudaStream_t st) {
+    const int grid = a.B * a.Hq;
+    if (a.policy == ENTMAXKV_TOPK) {
+        topk_kernel<<<grid, SEL_THREADS, 0, st>>>(a);
+    } else {
+        switch (a.r_int) {
+            case 1: gauss_kernel<1><<<grid, SEL_THREADS, 0, st>>>(a); break;
+            case 2: gauss_kernel<2><<<grid, SEL_THREADS, 0, st>>>(a); break;
+            case 3: gauss_kernel<3><<<grid, SEL_THREADS, 0, st>>>(a); break;
+            case 4: gauss_kernel<4><<<grid, SEL_THREADS, 0, st>>>(a); break;
+            case 5: gauss_kernel<5><<<grid, SEL_THREADS, 0, st>>>(a); break;
+            case 6: gauss_kernel<6><<<grid, SEL_THREADS, 0, st>>>(a); break;
+            case 7: gauss_kernel<7><<<grid, SEL_THREADS, 0, st>>>(a); break;
+            case 8: gauss_kernel<8><<<grid, SEL_THREADS, 0, st>>>(a); break;
+            default: return cudaErrorInvalidValue;
+        }
+    }
+    return cudaGetLastError();
+}
+
+}  // namespace ekv

@@ -1,0 +1,70 @@
+"""One EntmaxKV decode step over a paged cache, as a sequence of C-ABI calls.
+
+``EntmaxKVDecoder`` owns the device buffers the calls need (metadata, page
+scores, selections, workspace, output) and issues, on the current stream:
+
+  entmaxkv_build_meta    (the page each sequence's newest token landed in)
+  entmaxkv_score_pages
+  entmaxkv_select        (top-k or Gaussian tau_hat - Delta)
+  entmaxkv_decode_sparse
+
+It does no arithmetic itself; see include/entmaxkv.h for what each call
+computes.
+"""
+from __future__ import annotations
+
+import torch
+
+from . import native as nv
+
+
+class EntmaxKVDecoder:
+    def __init__(self, k_cache, v_cache, page_table, seq_lens, Hq, *, alpha=1.5, policy="topk",
+                 k=64, delta=0.5):
+        dev = k_cache.device
+        nb, Hkv, P, d = k_cache.shape
+        B, max_pages = page_table.shape
+        self.shape = nv.Shape(B, Hq, Hkv, d, P, max_pages, nb)
+        self.k_cache, self.v_cache = k_cache, v_cache
+        self.page_table, self.seq_lens = page_table, seq_lens
+        self.alpha, self.k, self.delta = float(alpha), int(k), float(delta)
+        self.policy = {"topk": nv.TOPK, "gauss": nv.GAUSS}[policy]
+        gauss = self.policy == nv.GAUSS
+        self.meta = nv.alloc_meta(self.shape, dev)
+        f32 = dict(dtype=torch.float32, device=dev)
+        self.bbox = torch.empty((B, Hq, max_pages), **f32)
+        self.mu = torch.empty((B, Hq, max_pages), **f32) if gauss else None
+        self.sigma = torch.empty((B, Hq, max_pages), **f32) if gauss else None
+        self.sel = torch.empty((B, Hq, max_pages), dtype=torch.int32, device=dev)
+        self.cnt = torch.empty((B, Hq), dtype=torch.int32, device=dev)
+        self.tau_hat = torch.empty((B, Hq), **f32)
+        self.tau = torch.empty((B, Hq), **f32)
+        self.out = torch.empty((B, Hq, d), **f32)
+        self.ws = nv.alloc_workspace(self.shape, nv.CALL_DECODE_SPARSE, dev)
+        self.launches_per_step = 0
+
+    def build_meta(self, first_page=0, n_pages=-1):
+        nv.entmaxkv_build_meta(self.shape, self.k_cache, self.page_table, self.seq_lens,
+                               first_page, n_pages, self.meta)
+
+    def step(self, q, append_page=None, p_out=None):
+        """One decode step for query q (bf16 [B, Hq, d]).  ``append_page``:
+        logical page whose metadata is refreshed first (the page the newest
+        token was written to), or None."""
+        if append_page is not None:
+            nv.entmaxkv_build_meta(self.shape, self.k_cache, self.page_table, self.seq_lens,
+                                   append_page, 1, self.meta)
+        nv.entmaxkv_score_pages(self.shape, q, self.meta, self.page_table, self.seq_lens,
+                                self.bbox, self.mu, self.sigma)
+        nv.entmaxkv_select(self.shape, self.seq_lens, self.bbox, self.mu, self.sigma, self.policy,
+                           self.k, self.alpha, self.delta, self.sel, self.cnt, self.tau_hat)
+        nv.entmaxkv_decode_sparse(self.shape, q, self.k_cache, self.v_cache, self.page_table,
+                                  self.seq_lens, self.sel, self.cnt, self.alpha, self.out,
+                                  self.tau, p_out, self.ws)
+        return self.out
+
+
+def kernels_per_step(policy_gauss: bool, append: bool) -> int:
+    """Kernel launches one ``step`` issues: build_meta (1, if appending),
+    score (1), select (1), decode_sparse (union, q.K, tau, p.V = 4)."""
+    return (1 if append else 0) + 1 + 1 + 4

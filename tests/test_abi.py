@@ -1,0 +1,117 @@
+"""The C-ABI library on the host: it loads, exports every declared symbol, and
+rejects bad arguments with the documented codes before touching the GPU
+(every call below returns from its host-side checks; none reaches CUDA)."""
+import ctypes as C
+import os
+import re
+
+import pytest
+
+from sparse_entmax_kv_b200 import native as nv
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HDR = os.path.join(ROOT, "include", "entmaxkv.h")
+
+FAKE = C.c_void_p(0x10000)       # aligned, never dereferenced
+FAKE_ODD = C.c_void_p(0x10008)   # 8-byte aligned only
+
+
+def _declared():
+    txt = open(HDR).read()
+    return sorted(set(re.findall(r"ENTMAXKV_API\s+[\w\s\*]+?\b(entmaxkv_\w+)\s*\(", txt)))
+
+
+def test_library_exports_every_declared_symbol():
+    L = nv.lib()
+    names = _declared()
+    assert len(names) == 10
+    assert set(names) == set(nv.EXPORTED)
+    for n in names:
+        assert hasattr(L, n)
+
+
+def test_strerror_and_version():
+    L = nv.lib()
+    assert L.entmaxkv_version() == 100
+    for code in list(nv.ERR) + [-99]:
+        assert L.entmaxkv_strerror(code)
+
+
+def shp(**kw):
+    d = dict(B=2, Hq=8, Hkv=2, d=128, page_size=32, max_pages=64, num_blocks=128)
+    d.update(kw)
+    return nv.Shape(*[d[f] for f, _ in nv.Shape._fields_])
+
+
+def test_sizes():
+    s = shp()
+    assert nv.meta_bytes(s) == 128 * 2 * 12 * 128
+    assert nv.workspace_size(s, nv.CALL_SELECT) == 0
+    ws = nv.workspace_size(s, nv.CALL_DECODE_SPARSE)
+    assert ws >= 2 * 8 * 64 * 32 * 4            # the z scratch alone
+    assert ws == nv.workspace_size(s, nv.CALL_DECODE_DENSE)
+    assert nv.workspace_size(s, 99) == (1 << 64) - 1
+    assert nv.meta_bytes(shp(d=96)) == 0
+
+
+@pytest.mark.parametrize("bad", [dict(d=96), dict(page_size=8), dict(Hq=6, Hkv=4), dict(Hq=24, Hkv=2),
+                                 dict(B=0), dict(max_pages=0), dict(num_blocks=0),
+                                 dict(max_pages=1 << 26, page_size=64)])
+def test_bad_shapes_rejected_everywhere(bad):
+    L = nv.lib()
+    s = C.byref(shp(**bad))
+    E = -2
+    assert L.entmaxkv_build_meta(s, FAKE, FAKE, FAKE, 0, -1, FAKE, None) == E
+    assert L.entmaxkv_score_pages(s, FAKE, FAKE, FAKE, FAKE, FAKE, None, None, None) == E
+    assert L.entmaxkv_select(s, FAKE, FAKE, None, None, 0, 4, 1.5, 0.0, FAKE, FAKE, None, None, 0, None) == E
+    assert L.entmaxkv_decode_sparse(s, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, 1.5, FAKE, None, None,
+                                    FAKE, 1 << 40, None) == E
+    assert L.entmaxkv_decode_dense(s, FAKE, FAKE, FAKE, FAKE, FAKE, 1.5, FAKE, None, None, FAKE, 1 << 40,
+                                   None) == E
+
+
+def test_null_alignment_and_argument_codes():
+    L = nv.lib()
+    s = C.byref(shp())
+    assert L.entmaxkv_build_meta(None, FAKE, FAKE, FAKE, 0, -1, FAKE, None) == -1
+    assert L.entmaxkv_build_meta(s, None, FAKE, FAKE, 0, -1, FAKE, None) == -1
+    assert L.entmaxkv_build_meta(s, FAKE_ODD, FAKE, FAKE, 0, -1, FAKE, None) == -8
+    assert L.entmaxkv_build_meta(s, FAKE, FAKE, FAKE, -1, -1, FAKE, None) == -2
+    assert L.entmaxkv_build_meta(s, FAKE, FAKE, FAKE, 0, -2, FAKE, None) == -2
+    assert L.entmaxkv_score_pages(s, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, None, None) == -1  # mu w/o sigma
+    assert L.entmaxkv_score_pages(s, FAKE_ODD, FAKE, FAKE, FAKE, FAKE, None, None, None) == -8
+    # select
+    sel = lambda pol, k, a, dl, mu=FAKE: L.entmaxkv_select(s, FAKE, FAKE, mu, mu, pol, k, a, dl, FAKE, FAKE,
+                                                           None, None, 0, None)
+    assert sel(0, 0, 1.5, 0.0) == -4
+    assert sel(7, 4, 1.5, 0.0) == -4
+    assert sel(1, 0, 1.5, float("inf")) == -4
+    assert sel(1, 0, 1.0, 0.5) == -3
+    assert sel(1, 0, float("nan"), 0.5) == -3
+    assert sel(1, 0, 1.3, 0.5) == -7            # r = 1/0.3 not an integer
+    assert sel(1, 0, 1.5, 0.5, mu=None) == -1
+    assert L.entmaxkv_select(shp(max_pages=200000), FAKE, FAKE, None, None, 0, 4, 1.5, 0.0, FAKE, FAKE,
+                             None, None, 0, None) == -2
+    # decode
+    need = nv.workspace_size(shp(), nv.CALL_DECODE_SPARSE)
+    dec = lambda a, ws, wsb, q=FAKE, sl=FAKE: L.entmaxkv_decode_sparse(
+        s, q, FAKE, FAKE, FAKE, FAKE, sl, FAKE, a, FAKE, None, None, ws, wsb, None)
+    assert dec(1.0, FAKE, need) == -3
+    assert dec(0.5, FAKE, need) == -3
+    assert dec(1.5, FAKE, need, sl=None) == -1
+    assert dec(1.5, FAKE, need - 1) == -5
+    assert dec(1.5, None, need) == -5
+    assert dec(1.5, C.c_void_p(0x10010), need) == -8   # workspace must be 256-byte aligned
+    assert dec(1.5, FAKE, need, q=FAKE_ODD) == -8
+    dd = lambda a, p=None: L.entmaxkv_decode_dense(s, FAKE, FAKE, FAKE, FAKE, FAKE, a, FAKE, None, p,
+                                                   FAKE, need, None)
+    assert dd(0.9) == -3
+    assert dd(float("inf")) == -3
+    assert dd(1.0, FAKE) == -1                   # no p_out for softmax
+
+
+def test_binding_refuses_cpu_tensors():
+    import torch
+    q = torch.zeros(1, 1, 64, dtype=torch.bfloat16)
+    with pytest.raises(ValueError, match="CUDA"):
+        nv._ptr(q, torch.bfloat16, "q")

@@ -1,0 +1,442 @@
+"""CUDA path vs the fp64 CPU oracle on identical seeded inputs.
+
+Tolerances (EntmaxKV hot-path contract):
+  * page metadata, bbox / mu / sigma scores, top-k indices: bit-exact;
+  * Gaussian selection: exact except pages whose bound lies within 1e-5
+    (relative) of the cutoff tau_hat - Delta; tau_hat within 1e-5 max(1,|tau_hat|);
+  * outputs: max abs error <= 2e-3 and relative L2 <= 1e-3 (fp32 accumulation);
+  * support sets: exact except tokens with |z - tau| < 1e-5.
+Small cases run every stage on the whole batch; full-size workloads are
+checked on sampled (sequence, kv head) sub-problems the oracle can finish.
+"""
+import math
+
+import numpy as np
+import pytest
+import torch
+
+import oracle as orc
+from sparse_entmax_kv_b200 import native as nv
+from sparse_entmax_kv_b200.decoder import EntmaxKVDecoder
+from sparse_entmax_kv_b200.workloads import CONFIGS, Workload, make_inputs, to_host_u16
+
+pytestmark = pytest.mark.gpu
+
+OUT_ABS, OUT_REL = 2e-3, 1e-3
+BAND = 1e-5
+
+# ------------------------------------------------------------- workloads
+
+SMALL = {
+    "tiny_full": CONFIGS["tiny_h1_L4k"],
+    "tiny_ragged": CONFIGS["tiny_h1_L4k"].shrink(name="tiny_ragged", B=3, L=3000, ragged=True),
+    "dense_small": CONFIGS["dense_gqa_L32k"].shrink(name="dense_small", B=2, Hq=8, Hkv=2, L=4096 + 32,
+                                                    ragged=True, needles=8),
+    "topk_small": CONFIGS["topk_gqa_L128k"].shrink(name="topk_small", B=2, Hq=8, Hkv=2, L=8192,
+                                                   ragged=True, needles=8),
+    "gauss_small": CONFIGS["gauss_gqa_L1m"].shrink(name="gauss_small", B=2, Hq=8, Hkv=2, L=32768,
+                                                   ragged=True, needles=16),
+    "mha_small": CONFIGS["sweep_mha_L64k"].shrink(name="mha_small", B=3, Hq=4, Hkv=4, L=2048,
+                                                  ragged=True, needles=4),
+    "gqa2_d64": Workload("gqa2_d64", B=2, Hq=4, Hkv=2, d=64, L=1500, P=16, alpha=1.25, policy="topk",
+                         k=20, keys="offset", needles=3, ragged=True),
+    "gqa8_d128": Workload("gqa8_d128", B=1, Hq=8, Hkv=1, d=128, L=2000, P=64, alpha=2.0, policy="gauss",
+                          delta=0.25, keys="cluster", needles=2, ragged=True),
+}
+
+
+def gpu_inputs(wl, seed):
+    inp = make_inputs(wl, seed, device="cuda")
+    host = dict(q=to_host_u16(inp["q"]), K=to_host_u16(inp["k_cache"]), V=to_host_u16(inp["v_cache"]),
+                page_table=inp["page_table"].cpu().numpy(), seq_lens=inp["seq_lens"].cpu().numpy())
+    return inp, host
+
+
+def shape_of(wl):
+    return nv.Shape(wl.B, wl.Hq, wl.Hkv, wl.d, wl.P, wl.max_pages, wl.num_blocks)
+
+
+def unpack_meta(meta: torch.Tensor, R: int, d: int):
+    m = meta.cpu().numpy()
+    bb = m[:R * 4 * d].view(np.uint16).reshape(R, 2, d)
+    mo = m[R * 4 * d:R * 12 * d].view(np.float32).reshape(R, 2, d)
+    return bb[:, 0], bb[:, 1], mo[:, 0], mo[:, 1]
+
+
+def referenced_records(host, wl):
+    recs = []
+    for b in range(wl.B):
+        np_b = -(-int(host["seq_lens"][b]) // wl.P)
+        for p in range(np_b):
+            blk = int(host["page_table"][b, p])
+            recs.extend(blk * wl.Hkv + h for h in range(wl.Hkv))
+    return np.array(sorted(recs))
+
+
+def n_pages(host, wl, b):
+    return -(-int(host["seq_lens"][b]) // wl.P)
+
+
+def assert_outputs_close(got, want, what=""):
+    got = np.asarray(got, np.float64)
+    want = np.asarray(want, np.float64)
+    err = np.abs(got - want).max()
+    rel = np.linalg.norm(got - want) / max(np.linalg.norm(want), 1e-30)
+    assert err <= OUT_ABS, f"{what}: max abs err {err:.3e}"
+    assert rel <= OUT_REL, f"{what}: rel L2 err {rel:.3e}"
+
+
+def check_support(p_gpu, z_orc, tau_orc, what=""):
+    """Support of the GPU weights vs the oracle's {z > tau}, exempting |z-tau| < BAND."""
+    sup_g = p_gpu > 0
+    sup_o = z_orc > tau_orc
+    diff = sup_g != sup_o
+    if diff.any():
+        near = np.abs(z_orc - tau_orc) < BAND
+        assert np.all(near[diff]), f"{what}: {int((diff & ~near).sum())} support tokens differ"
+
+
+def check_selection(sel_g, sel_o, cutoff_scores, cutoff, what=""):
+    a, b = set(sel_g.tolist()), set(sel_o.tolist())
+    if a == b:
+        return
+    for p in a ^ b:
+        s = float(cutoff_scores[p])
+        assert abs(s - cutoff) <= BAND * max(1.0, abs(cutoff)), f"{what}: page {p} differs (score {s}, cutoff {cutoff})"
+
+
+@pytest.fixture(autouse=True)
+def _clear_status():
+    nv.get_status(clear=True)
+    yield
+    st = nv.get_status(clear=True)
+    assert st & ~nv.STATUS_OVERFLOW == 0, f"device status {st}"
+
+
+# ------------------------------------------------------------ per stage
+
+@pytest.mark.parametrize("name", list(SMALL))
+def test_meta_and_scores_bit_exact(name):
+    wl = SMALL[name]
+    inp, host = gpu_inputs(wl, 1)
+    s = shape_of(wl)
+    meta = nv.alloc_meta(s, "cuda")
+    nv.entmaxkv_build_meta(s, inp["k_cache"], inp["page_table"], inp["seq_lens"], 0, -1, meta)
+    R = wl.num_blocks * wl.Hkv
+    g = unpack_meta(meta, R, wl.d)
+    o = orc.build_meta(host["K"], host["page_table"], host["seq_lens"], wl.Hkv, wl.d, wl.P, wl.num_blocks)
+    recs = referenced_records(host, wl)
+    for gi, oi, nm in zip(g, o, ("kmin", "kmax", "mean", "var")):
+        np.testing.assert_array_equal(gi[recs].view(np.uint32 if gi.dtype == np.float32 else np.uint16),
+                                      oi[recs].view(np.uint32 if oi.dtype == np.float32 else np.uint16),
+                                      err_msg=nm)
+    B, Hq, mp = wl.B, wl.Hq, wl.max_pages
+    out = [torch.full((B, Hq, mp), float("nan"), device="cuda") for _ in range(3)]
+    nv.entmaxkv_score_pages(s, inp["q"], meta, inp["page_table"], inp["seq_lens"], *out)
+    ob = orc.score_pages(host["q"], o, host["page_table"], host["seq_lens"], wl.Hkv, wl.P)
+    for gt, ot, nm in zip(out, ob, ("bbox", "mu", "sigma")):
+        gt = gt.cpu().numpy()
+        for b in range(B):
+            npb = n_pages(host, wl, b)
+            np.testing.assert_array_equal(gt[b, :, :npb].view(np.uint32), ot[b, :, :npb].view(np.uint32),
+                                          err_msg=nm)
+    # bound-only scoring gives the same bound
+    bb2 = torch.full((B, Hq, mp), float("nan"), device="cuda")
+    nv.entmaxkv_score_pages(s, inp["q"], meta, inp["page_table"], inp["seq_lens"], bb2)
+    for b in range(B):
+        npb = n_pages(host, wl, b)
+        assert torch.equal(bb2[b, :, :npb], out[0][b, :, :npb])
+
+
+def _oracle_scores(host, wl):
+    meta = orc.build_meta(host["K"], host["page_table"], host["seq_lens"], wl.Hkv, wl.d, wl.P, wl.num_blocks)
+    return orc.score_pages(host["q"], meta, host["page_table"], host["seq_lens"], wl.Hkv, wl.P)
+
+
+@pytest.mark.parametrize("name", list(SMALL))
+@pytest.mark.parametrize("policy", ["topk", "gauss"])
+def test_select_parity(name, policy):
+    wl = SMALL[name]
+    if policy == "gauss" and abs(1.0 / (wl.alpha - 1) - round(1.0 / (wl.alpha - 1))) > 1e-9:
+        pytest.skip("Gaussian policy needs integer 1/(alpha-1)")
+    inp, host = gpu_inputs(wl, 2)
+    bbox, mu, sig = _oracle_scores(host, wl)   # oracle scores as the shared input
+    s = shape_of(wl)
+    B, Hq, mp = wl.B, wl.Hq, wl.max_pages
+    tb, tm, ts = (torch.from_numpy(np.nan_to_num(x, nan=0.0)).cuda() for x in (bbox, mu, sig))
+    sel = torch.full((B, Hq, mp), -1, dtype=torch.int32, device="cuda")
+    cnt = torch.zeros((B, Hq), dtype=torch.int32, device="cuda")
+    th = torch.zeros((B, Hq), device="cuda")
+    k = wl.k if wl.k else 16
+    delta = wl.delta if wl.delta else 0.5
+    pol = nv.TOPK if policy == "topk" else nv.GAUSS
+    nv.entmaxkv_select(s, inp["seq_lens"], tb, tm, ts, pol, k, wl.alpha, delta, sel, cnt, th)
+    osel, ocnt, oth = orc.select(host["seq_lens"], np.nan_to_num(bbox, nan=0.0), np.nan_to_num(mu, nan=0.0),
+                                 np.nan_to_num(sig, nan=0.0), wl.P, policy, k, wl.alpha, delta)
+    sel, cnt, th = sel.cpu().numpy(), cnt.cpu().numpy(), th.cpu().numpy()
+    for b in range(B):
+        for h in range(Hq):
+            gs = sel[b, h, :cnt[b, h]]
+            assert np.all(np.diff(gs) > 0), "ascending, no repeats"
+            os_ = osel[b, h, :ocnt[b, h]]
+            if policy == "topk":
+                np.testing.assert_array_equal(gs, os_)
+            else:
+                assert th[b, h] == pytest.approx(oth[b, h], abs=1e-5 * max(1.0, abs(oth[b, h])))
+                check_selection(gs, os_, (wl.alpha - 1) * bbox[b, h].astype(np.float64),
+                                oth[b, h] - delta, f"b{b}h{h}")
+
+
+def _oracle_selection(host, wl, policy, k, delta):
+    bbox, mu, sig = _oracle_scores(host, wl)
+    return orc.select(host["seq_lens"], np.nan_to_num(bbox, nan=0.0), np.nan_to_num(mu, nan=0.0),
+                      np.nan_to_num(sig, nan=0.0), wl.P, policy, k, wl.alpha, delta)
+
+
+@pytest.mark.parametrize("name", list(SMALL))
+def test_decode_sparse_parity(name):
+    wl = SMALL[name]
+    inp, host = gpu_inputs(wl, 3)
+    policy = wl.policy if wl.policy != "dense" else "topk"
+    k = wl.k if wl.k else 32
+    osel, ocnt, _ = _oracle_selection(host, wl, policy, k, wl.delta or 0.5)
+    s = shape_of(wl)
+    B, Hq, d = wl.B, wl.Hq, wl.d
+    sel = torch.from_numpy(osel).cuda()
+    cnt = torch.from_numpy(ocnt).cuda()
+    out = torch.empty((B, Hq, d), device="cuda")
+    tau = torch.empty((B, Hq), device="cuda")
+    pw = torch.zeros((B, Hq, wl.max_pages * wl.P), device="cuda")
+    ws = nv.alloc_workspace(s, nv.CALL_DECODE_SPARSE, "cuda")
+    nv.entmaxkv_decode_sparse(s, inp["q"], inp["k_cache"], inp["v_cache"], inp["page_table"], inp["seq_lens"],
+                              sel, cnt, wl.alpha, out, tau, pw, ws)
+    o, otau, op, oz = orc.decode(host["q"], host["K"], host["V"], host["page_table"], host["seq_lens"], wl.Hkv,
+                                 wl.P, wl.alpha, sel=osel, cnt=ocnt, want_p=True, want_z=True)
+    assert_outputs_close(out.cpu().numpy(), o, name)
+    np.testing.assert_allclose(tau.cpu().numpy(), otau, atol=2e-5 * max(1.0, np.abs(otau).max()))
+    pw = pw.cpu().numpy()
+    for b in range(B):
+        for h in range(Hq):
+            kept = np.isfinite(oz[b, h])
+            check_support(pw[b, h][kept], oz[b, h][kept], otau[b, h], f"b{b}h{h}")
+            np.testing.assert_allclose(pw[b, h][kept], op[b, h][kept], atol=2e-4)
+    # a second call on the same workspace gives identical bits
+    out2 = torch.empty_like(out)
+    nv.entmaxkv_decode_sparse(s, inp["q"], inp["k_cache"], inp["v_cache"], inp["page_table"], inp["seq_lens"],
+                              sel, cnt, wl.alpha, out2, None, None, ws)
+    assert torch.equal(out, out2)
+
+
+@pytest.mark.parametrize("name", ["tiny_ragged", "dense_small", "mha_small", "gqa2_d64", "gqa8_d128"])
+@pytest.mark.parametrize("alpha", [1.0, 1.5, 2.0, 1.25])
+def test_decode_dense_parity(name, alpha):
+    wl = SMALL[name]
+    inp, host = gpu_inputs(wl, 4)
+    s = shape_of(wl)
+    B, Hq, d = wl.B, wl.Hq, wl.d
+    out = torch.empty((B, Hq, d), device="cuda")
+    tau = torch.empty((B, Hq), device="cuda")
+    pw = torch.zeros((B, Hq, wl.max_pages * wl.P), device="cuda") if alpha > 1 else None
+    ws = nv.alloc_workspace(s, nv.CALL_DECODE_DENSE, "cuda")
+    nv.entmaxkv_decode_dense(s, inp["q"], inp["k_cache"], inp["v_cache"], inp["page_table"], inp["seq_lens"],
+                             alpha, out, tau, pw, ws)
+    o, otau, op, oz = orc.decode(host["q"], host["K"], host["V"], host["page_table"], host["seq_lens"], wl.Hkv,
+                                 wl.P, alpha, want_p=alpha > 1, want_z=True)
+    assert_outputs_close(out.cpu().numpy(), o, f"{name} alpha={alpha}")
+    np.testing.assert_allclose(tau.cpu().numpy(), otau, atol=2e-5 * max(1.0, np.abs(otau).max()))
+    if alpha > 1:
+        pw = pw.cpu().numpy()
+        for b in range(B):
+            for h in range(Hq):
+                kept = np.isfinite(oz[b, h])
+                check_support(pw[b, h][kept], oz[b, h][kept], otau[b, h], f"b{b}h{h}")
+
+
+# ------------------------------------------------------- edge cases
+
+def test_empty_selection_and_single_token_sequences():
+    wl = Workload("edge", B=3, Hq=4, Hkv=2, d=128, L=64, P=32, alpha=1.5, policy="topk", k=4)
+    inp, host = gpu_inputs(wl, 5)
+    inp["seq_lens"] = torch.tensor([1, 33, 64], dtype=torch.int32, device="cuda")
+    host["seq_lens"] = inp["seq_lens"].cpu().numpy()
+    s = shape_of(wl)
+    osel, ocnt, _ = orc.select(host["seq_lens"], np.zeros((3, 4, 2), np.float32), None, None, wl.P, "topk", 4,
+                               1.5, 0.0)
+    ocnt[2, 1] = 0  # one head selects nothing
+    sel, cnt = torch.from_numpy(osel).cuda(), torch.from_numpy(ocnt).cuda()
+    out = torch.full((3, 4, 128), 7.0, device="cuda")
+    tau = torch.empty((3, 4), device="cuda")
+    ws = nv.alloc_workspace(s, nv.CALL_DECODE_SPARSE, "cuda")
+    nv.entmaxkv_decode_sparse(s, inp["q"], inp["k_cache"], inp["v_cache"], inp["page_table"], inp["seq_lens"],
+                              sel, cnt, 1.5, out, tau, None, ws)
+    o, otau, _, _ = orc.decode(host["q"], host["K"], host["V"], host["page_table"], host["seq_lens"], 2, 32, 1.5,
+                               sel=osel, cnt=ocnt)
+    out, tau = out.cpu().numpy(), tau.cpu().numpy()
+    assert np.all(out[2, 1] == 0.0) and math.isnan(tau[2, 1])
+    mask = np.ones((3, 4), bool)
+    mask[2, 1] = False
+    assert_outputs_close(out[mask], o[mask], "edge")
+    # single-token sequence: p = 1 on that token, so out = its value row
+    np.testing.assert_allclose(out[0], o[0], atol=1e-6)
+
+
+def test_bad_page_table_entry_sets_status_and_skips():
+    wl = SMALL["topk_small"]
+    inp, _ = gpu_inputs(wl, 6)
+    s = shape_of(wl)
+    pt = inp["page_table"].clone()
+    pt[0, 3] = wl.num_blocks + 5          # out of range: must be skipped, not read
+    meta = nv.alloc_meta(s, "cuda")
+    nv.get_status(clear=True)
+    nv.entmaxkv_build_meta(s, inp["k_cache"], pt, inp["seq_lens"], 0, -1, meta)
+    torch.cuda.synchronize()
+    assert nv.get_status(clear=True) & nv.STATUS_BAD_PAGE
+
+
+def test_append_rebuild_matches_full_build():
+    """Section 2.A 'maintained on append': rewriting the newest token and
+    rebuilding only its page gives the same metadata as a full rebuild."""
+    wl = SMALL["gauss_small"]
+    inp, _ = gpu_inputs(wl, 7)
+    s = shape_of(wl)
+    meta = nv.alloc_meta(s, "cuda")
+    nv.entmaxkv_build_meta(s, inp["k_cache"], inp["page_table"], inp["seq_lens"], 0, -1, meta)
+    b = 1
+    L = int(inp["seq_lens"][b])
+    p_last = (L - 1) // wl.P
+    blk = int(inp["page_table"][b, p_last])
+    inp["k_cache"][blk, :, (L - 1) % wl.P] = torch.randn(wl.Hkv, wl.d, device="cuda").to(torch.bfloat16) * 3
+    nv.entmaxkv_build_meta(s, inp["k_cache"], inp["page_table"], inp["seq_lens"], p_last, 1, meta)
+    full = nv.alloc_meta(s, "cuda")
+    nv.entmaxkv_build_meta(s, inp["k_cache"], inp["page_table"], inp["seq_lens"], 0, -1, full)
+    R = wl.num_blocks * wl.Hkv
+    a, c = unpack_meta(meta, R, wl.d), unpack_meta(full, R, wl.d)
+    for b2 in range(wl.B):
+        for p in range(-(-int(inp["seq_lens"][b2]) // wl.P)):
+            bl = int(inp["page_table"][b2, p])
+            for x, y in zip(a, c):
+                assert np.array_equal(x[bl * wl.Hkv:(bl + 1) * wl.Hkv].view(np.uint8),
+                                      y[bl * wl.Hkv:(bl + 1) * wl.Hkv].view(np.uint8))
+
+
+# ---------------------------------------------------- full-size workloads
+
+def _sub_problem(inp, wl, b, kvh):
+    """(sequence b, kv head kvh) as a self-contained host problem (identity page table)."""
+    L = int(inp["seq_lens"][b])
+    npb = -(-L // wl.P)
+    blocks = inp["page_table"][b, :npb].long()
+    G = wl.G
+    K = inp["k_cache"][blocks, kvh:kvh + 1].contiguous()
+    V = inp["v_cache"][blocks, kvh:kvh + 1].contiguous()
+    q = inp["q"][b:b + 1, kvh * G:(kvh + 1) * G].contiguous()
+    return dict(q=to_host_u16(q), K=to_host_u16(K), V=to_host_u16(V),
+                page_table=np.arange(npb, dtype=np.int32)[None], seq_lens=np.array([L], np.int32), npb=npb,
+                blocks=blocks.cpu().numpy())
+
+
+FULL = ["tiny_h1_L4k", "dense_gqa_L32k", "topk_gqa_L128k", "gauss_gqa_L1m", "sweep_mha_L64k"]
+
+
+@pytest.mark.parametrize("name", FULL)
+def test_full_size_step_sampled(name):
+    """The decode step exactly as the benchmark launches it (EntmaxKVDecoder
+    over the whole batch), checked on sampled (sequence, kv head) groups."""
+    wl = CONFIGS[name]
+    policy = wl.policy if wl.policy != "dense" else "topk"
+    k = wl.k if wl.k else 64
+    delta = wl.delta if wl.delta else 0.5
+    inp = make_inputs(wl, 11, device="cuda")
+    dec = EntmaxKVDecoder(inp["k_cache"], inp["v_cache"], inp["page_table"], inp["seq_lens"], wl.Hq,
+                          alpha=wl.alpha, policy=policy, k=k, delta=delta)
+    dec.build_meta()
+    dec.step(inp["q"])
+    torch.cuda.synchronize()
+    R = wl.num_blocks * wl.Hkv
+    gmeta = unpack_meta(dec.meta, R, wl.d)
+    rng = np.random.default_rng(0)
+    groups = [(0, 0), (wl.B - 1, wl.Hkv - 1), (int(rng.integers(wl.B)), int(rng.integers(wl.Hkv)))]
+    G = wl.G
+    for b, kvh in groups:
+        sp = _sub_problem(inp, wl, b, kvh)
+        om = orc.build_meta(sp["K"], sp["page_table"], sp["seq_lens"], 1, wl.d, wl.P, sp["npb"])
+        recs = sp["blocks"] * wl.Hkv + kvh
+        for gi, oi in zip(gmeta, om):
+            assert np.array_equal(gi[recs].view(np.uint8), oi.view(np.uint8))
+        ob, omu, osg = orc.score_pages(sp["q"], om, sp["page_table"], sp["seq_lens"], 1, wl.P)
+        hs = slice(kvh * G, (kvh + 1) * G)
+        gb = dec.bbox[b, hs, :sp["npb"]].cpu().numpy()
+        assert np.array_equal(gb.view(np.uint32), ob[0].view(np.uint32))
+        if policy == "gauss":
+            assert np.array_equal(dec.mu[b, hs, :sp["npb"]].cpu().numpy().view(np.uint32), omu[0].view(np.uint32))
+            assert np.array_equal(dec.sigma[b, hs, :sp["npb"]].cpu().numpy().view(np.uint32),
+                                  osg[0].view(np.uint32))
+        osel, ocnt, oth = orc.select(sp["seq_lens"], ob, omu, osg, wl.P, policy, k, wl.alpha, delta)
+        o, otau, _, _ = orc.decode(sp["q"], sp["K"], sp["V"], sp["page_table"], sp["seq_lens"], 1, wl.P,
+                                   wl.alpha, sel=osel, cnt=ocnt)
+        gsel = dec.sel[b, hs].cpu().numpy()
+        gcnt = dec.cnt[b, hs].cpu().numpy()
+        gout = dec.out[b, hs].cpu().numpy()
+        for g in range(G):
+            gs, os_ = gsel[g, :gcnt[g]], osel[0, g, :ocnt[0, g]]
+            if policy == "topk":
+                np.testing.assert_array_equal(gs, os_)
+            else:
+                gth = float(dec.tau_hat[b, kvh * G + g])
+                assert gth == pytest.approx(oth[0, g], abs=1e-5 * max(1.0, abs(oth[0, g])))
+                check_selection(gs, os_, (wl.alpha - 1) * ob[0, g].astype(np.float64), oth[0, g] - delta)
+            if np.array_equal(gs, os_):
+                assert_outputs_close(gout[g], o[0, g], f"{name} b{b} h{kvh * G + g}")
+                assert float(dec.tau[b, kvh * G + g]) == pytest.approx(otau[0, g], abs=2e-5 * max(1, abs(otau[0, g])))
+
+
+@pytest.mark.parametrize("name,alpha", [("dense_gqa_L32k", 1.5), ("dense_gqa_L32k", 1.0),
+                                        ("gauss_gqa_L1m", 1.5), ("gauss_gqa_L1m", 1.0)])
+def test_full_size_dense_sampled(name, alpha):
+    wl = CONFIGS[name]
+    inp = make_inputs(wl, 12, device="cuda")
+    s = shape_of(wl)
+    out = torch.empty((wl.B, wl.Hq, wl.d), device="cuda")
+    tau = torch.empty((wl.B, wl.Hq), device="cuda")
+    ws = nv.alloc_workspace(s, nv.CALL_DECODE_DENSE, "cuda")
+    nv.entmaxkv_decode_dense(s, inp["q"], inp["k_cache"], inp["v_cache"], inp["page_table"], inp["seq_lens"],
+                             alpha, out, tau, None, ws)
+    torch.cuda.synchronize()
+    G = wl.G
+    for b, kvh in [(0, 0), (wl.B - 1, wl.Hkv - 1)]:
+        sp = _sub_problem(inp, wl, b, kvh)
+        o, otau, _, _ = orc.decode(sp["q"], sp["K"], sp["V"], sp["page_table"], sp["seq_lens"], 1, wl.P, alpha)
+        assert_outputs_close(out[b, kvh * G:(kvh + 1) * G].cpu().numpy(), o[0], f"{name} b{b} kvh{kvh}")
+        np.testing.assert_allclose(tau[b, kvh * G:(kvh + 1) * G].cpu().numpy(), otau[0],
+                                   atol=2e-5 * max(1.0, np.abs(otau).max()))
+
+
+@pytest.mark.parametrize("pt", [dict(alpha=1.25, P=16, policy="topk", k=128, delta=0.0, needles=256),
+                                dict(alpha=2.0, P=64, policy="gauss", k=0, delta=1.0, needles=1),
+                                dict(alpha=1.5, P=32, policy="gauss", k=0, delta=0.25, needles=16)])
+def test_sweep_points_reduced_batch(pt):
+    wl = CONFIGS["sweep_mha_L64k"].shrink(B=2, Hq=4, Hkv=4, **pt)
+    inp = make_inputs(wl, 13, device="cuda")
+    dec = EntmaxKVDecoder(inp["k_cache"], inp["v_cache"], inp["page_table"], inp["seq_lens"], wl.Hq,
+                          alpha=wl.alpha, policy=wl.policy, k=wl.k or 32, delta=wl.delta or 0.5)
+    dec.build_meta()
+    dec.step(inp["q"])
+    torch.cuda.synchronize()
+    host = dict(q=to_host_u16(inp["q"]), K=to_host_u16(inp["k_cache"]), V=to_host_u16(inp["v_cache"]),
+                page_table=inp["page_table"].cpu().numpy(), seq_lens=inp["seq_lens"].cpu().numpy())
+    ob, omu, osg = _oracle_scores(host, wl)
+    assert np.array_equal(dec.bbox.cpu().numpy().view(np.uint32), ob.view(np.uint32))
+    osel, ocnt, oth = orc.select(host["seq_lens"], ob, omu, osg, wl.P, wl.policy, wl.k or 32, wl.alpha,
+                                 wl.delta or 0.5)
+    o, _, _, _ = orc.decode(host["q"], host["K"], host["V"], host["page_table"], host["seq_lens"], wl.Hkv, wl.P,
+                            wl.alpha, sel=osel, cnt=ocnt)
+    gsel, gcnt, gout = dec.sel.cpu().numpy(), dec.cnt.cpu().numpy(), dec.out.cpu().numpy()
+    for b in range(wl.B):
+        for h in range(wl.Hq):
+            gs, os_ = gsel[b, h, :gcnt[b, h]], osel[b, h, :ocnt[b, h]]
+            if wl.policy == "gauss":
+                check_selection(gs, os_, (wl.alpha - 1) * ob[b, h].astype(np.float64), oth[b, h] - wl.delta)
+            else:
+                np.testing.assert_array_equal(gs, os_)
+            if np.array_equal(gs, os_):
+                assert_outputs_close(gout[b, h], o[b, h], f"b{b}h{h}")
