@@ -74,7 +74,7 @@ class ClockSampler:
                  "--query-gpu=index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
                  "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
                  "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap",
-                 "--format=csv,noheader,nounits", "-lms", "200"], stdout=self.f, stderr=subprocess.DEVNULL)
+                 "--format=csv,noheader,nounits", "-lms", "100"], stdout=self.f, stderr=subprocess.DEVNULL)
         except (OSError, FileNotFoundError):
             self.proc = None
         return self
@@ -106,7 +106,8 @@ class ClockSampler:
                 if v.lower() == "active":
                     reasons.add(n)
         return {"sm_mhz": statistics.median(sm) if sm else None, "sm_max_mhz": max(mx) if mx else None,
-                "reasons": sorted(reasons), "samples": len(sm)}
+                "reasons": sorted(reasons), "samples": len(sm),
+                "window": "loaded steps bracketing the timed region (>= 1 s before, >= 0.5 s after)"}
 
 
 # ------------------------------------------------------------ byte model
@@ -173,18 +174,25 @@ def run_gpu(args, rank, world):
     del p_out
     torch.cuda.empty_cache()
 
-    for _ in range(args.warmup):
-        flush.fill_(1)
-        dec.step(q, append_page)
-    torch.cuda.synchronize()
-    assert nv.get_status(clear=True) & ~nv.STATUS_OVERFLOW == 0
-
     nst = 4
     ev = [[torch.cuda.Event(enable_timing=True) for _ in range(nst + 1)] for _ in range(args.steps)]
-    if world > 1:
-        torch.distributed.barrier()
-    torch.cuda.synchronize()
+    # The timed region lasts milliseconds, far below nvidia-smi's sampling
+    # period, so clocks are sampled over a loaded window that brackets it:
+    # warm-up steps for >= 1 s before, untimed steps for >= 0.5 s after.
     with ClockSampler(dev.index) as clk:
+        t0 = time.perf_counter()
+        i = 0
+        while i < args.warmup or time.perf_counter() - t0 < 1.0:
+            flush.fill_(1)
+            dec.step(q, append_page)
+            if i % 16 == 15:
+                torch.cuda.synchronize()
+            i += 1
+        torch.cuda.synchronize()
+        assert nv.get_status(clear=True) & ~nv.STATUS_OVERFLOW == 0
+        if world > 1:
+            torch.distributed.barrier()
+        torch.cuda.synchronize()
         t_wall = time.perf_counter()
         for i in range(args.steps):
             flush.fill_(1)
@@ -205,6 +213,12 @@ def run_gpu(args, rank, world):
         if world > 1:
             torch.distributed.barrier()
         t_wall = time.perf_counter() - t_wall
+        t1 = time.perf_counter()
+        while time.perf_counter() - t1 < 0.5:
+            for _ in range(16):
+                flush.fill_(1)
+                dec.step(q, append_page)
+            torch.cuda.synchronize()
     clocks = clk.summary()
     stage_ms = np.array([[ev[i][j].elapsed_time(ev[i][j + 1]) for j in range(nst)] for i in range(args.steps)])
     step_ms = float(stage_ms.sum(axis=1).mean())
