@@ -127,7 +127,8 @@ size_t entmaxkv_workspace_size(const entmaxkv_shape *s, int call) {
         case ENTMAXKV_CALL_SELECT: return 0;
         case ENTMAXKV_CALL_DECODE_SPARSE:
         case ENTMAXKV_CALL_DECODE_DENSE:
-            return decode_ws_bytes(s->B, s->Hq, s->Hkv, s->d, s->page_size, s->max_pages, nullptr, nullptr);
+            return decode_ws_bytes(call == ENTMAXKV_CALL_DECODE_DENSE, s->B, s->Hq, s->Hkv, s->d, s->page_size,
+                                   s->max_pages, nullptr, nullptr);
         default: return (size_t)-1;
     }
 }
@@ -247,7 +248,7 @@ int entmaxkv_select(const entmaxkv_shape *s, const int32_t *seq_lens, const floa
     return cuda_rc(launch_select(a, static_cast<cudaStream_t>(stream)));
 }
 
-static int fill_decode(const entmaxkv_shape *s, const void *q, const void *k_cache, const void *v_cache,
+static int fill_decode(bool dense, const entmaxkv_shape *s, const void *q, const void *k_cache, const void *v_cache,
                        const int32_t *page_table, const int32_t *seq_lens, float alpha, float *out, float *tau_out,
                        float *p_out, void *workspace, size_t ws_bytes, DecodeArgs *a) {
     int rc = check_shape(s);
@@ -255,7 +256,8 @@ static int fill_decode(const entmaxkv_shape *s, const void *q, const void *k_cac
     if (!q || !k_cache || !v_cache || !page_table || !seq_lens || !out) return ENTMAXKV_ERR_NULL;
     if (!aligned16(q) || !aligned16(k_cache) || !aligned16(v_cache)) return ENTMAXKV_ERR_ALIGN;
     if (!std::isfinite(alpha)) return ENTMAXKV_ERR_ALPHA;
-    const size_t need = decode_ws_bytes(s->B, s->Hq, s->Hkv, s->d, s->page_size, s->max_pages, nullptr, nullptr);
+    const size_t need =
+        decode_ws_bytes(dense, s->B, s->Hq, s->Hkv, s->d, s->page_size, s->max_pages, nullptr, nullptr);
     if (!workspace || ws_bytes < need) return ENTMAXKV_ERR_WORKSPACE;
     if ((reinterpret_cast<uintptr_t>(workspace) & 255u) != 0) return ENTMAXKV_ERR_ALIGN;
     DevInfo di;
@@ -269,7 +271,7 @@ static int fill_decode(const entmaxkv_shape *s, const void *q, const void *k_cac
     a->out = out;
     a->tau_out = tau_out;
     a->p_out = p_out;
-    decode_ws_bytes(s->B, s->Hq, s->Hkv, s->d, s->page_size, s->max_pages, &a->ws, workspace);
+    decode_ws_bytes(dense, s->B, s->Hq, s->Hkv, s->d, s->page_size, s->max_pages, &a->ws, workspace);
     a->B = s->B;
     a->Hq = s->Hq;
     a->Hkv = s->Hkv;
@@ -292,7 +294,7 @@ int entmaxkv_decode_sparse(const entmaxkv_shape *s, const void *q, const void *k
     if (!(alpha > 1.f)) return ENTMAXKV_ERR_ALPHA;
     if (s && s->max_pages > MAX_SEL_PAGES) return ENTMAXKV_ERR_SHAPE;
     DecodeArgs a;
-    int rc = fill_decode(s, q, k_cache, v_cache, page_table, seq_lens, alpha, out, tau_out, p_out, workspace,
+    int rc = fill_decode(false, s, q, k_cache, v_cache, page_table, seq_lens, alpha, out, tau_out, p_out, workspace,
                          ws_bytes, &a);
     if (rc) return rc;
     a.sel = sel;
@@ -307,7 +309,7 @@ int entmaxkv_decode_dense(const entmaxkv_shape *s, const void *q, const void *k_
     if (!(alpha >= 1.f)) return ENTMAXKV_ERR_ALPHA;
     if (alpha == 1.f && p_out) return ENTMAXKV_ERR_NULL;
     DecodeArgs a;
-    int rc = fill_decode(s, q, k_cache, v_cache, page_table, seq_lens, alpha, out, tau_out, p_out, workspace,
+    int rc = fill_decode(true, s, q, k_cache, v_cache, page_table, seq_lens, alpha, out, tau_out, p_out, workspace,
                          ws_bytes, &a);
     if (rc) return rc;
     if ((rc = make_kv_map(&a.kmap, k_cache, s))) return rc;

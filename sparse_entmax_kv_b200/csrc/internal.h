@@ -54,15 +54,20 @@ struct SelectArgs {
 };
 cudaError_t launch_select(const SelectArgs &a, cudaStream_t st);
 
-// Workspace carve-up shared by the decode paths.
+// Workspace carve-up shared by the decode paths.  A candidate is a token
+// whose z exceeded (running max of z seen so far) - 1 when it was scored: a
+// superset of the tokens that can carry weight, since tau >= max z - 1.
 struct DecodeWs {
-    int *union_e;    // [B*Hkv][max_pages]   (page << 8) | head mask
+    int *union_e;    // [B*Hkv][max_pages]   (page << 8) | head mask (sparse)
     int *union_cnt;  // [B*Hkv]
     int *zmax;       // [B*Hq] order-mapped max z
     float *tau;      // [B*Hq]
-    int *counters;   // [B*Hkv]
-    float *partial;  // [MAX_SPLITS][B*Hq][d+2]
-    float *zbuf;     // [B*Hq][max_pages*P]
+    int *counters;   // [B*Hkv] last-CTA combine counters
+    int *cand_cnt;   // [B*Hq]
+    int2 *cand;      // [B*Hq][max_pages*P]  (z bits, value row index)
+    int *cand_lpos;  // [B*Hq][max_pages*P]  logical token position (only with p_out)
+    float *partial;  // [MAX_SPLITS][B*Hq][d+2]  (dense paths)
+    float *zbuf;     // [B*Hq][max_pages*P]      (dense entmax path)
 };
 
 struct DecodeArgs {
@@ -83,6 +88,7 @@ cudaError_t launch_decode_sparse(const DecodeArgs &a, cudaStream_t st);
 cudaError_t launch_decode_dense_entmax(const DecodeArgs &a, cudaStream_t st);
 cudaError_t launch_decode_dense_softmax(const DecodeArgs &a, cudaStream_t st);
 
-size_t decode_ws_bytes(int B, int Hq, int Hkv, int d, int P, int max_pages, DecodeWs *carve, void *base);
+size_t decode_ws_bytes(bool dense, int B, int Hq, int Hkv, int d, int P, int max_pages, DecodeWs *carve,
+                      void *base);
 
 }  // namespace ekv

@@ -11,49 +11,41 @@
 
 namespace ekv {
 
-template <int D>
+template <int D, int P>
 __global__ void __launch_bounds__(D) build_meta_kernel(MetaArgs a) {
     const int b = blockIdx.y;
     const int kvh = blockIdx.z;
     const int p = a.first_page + blockIdx.x;
     const int seq = a.seq_lens[b];
-    if (p >= n_pages_of(seq, a.P)) return;
+    if (p >= n_pages_of(seq, P)) return;
     const int blk = a.page_table[(size_t)b * a.max_pages + p];
     if (blk < 0 || blk >= a.num_blocks) {
         if (threadIdx.x == 0) atomicOr(a.status, ENTMAXKV_STATUS_BAD_PAGE);
         return;
     }
-    const int n = tokens_in_page(seq, a.P, p);
+    const int n = tokens_in_page(seq, P, p);
     const long long rec = (long long)blk * a.Hkv + kvh;
     const int j = threadIdx.x;
-    const uint16_t *col = a.k + (size_t)rec * a.P * D + j;
+    const uint16_t *col = a.k + (size_t)rec * P * D + j;
 
-    uint16_t bmin = col[0], bmax = col[0];
+    // every load of the page is issued before the first use
+    uint16_t h[P];
+#pragma unroll
+    for (int t = 0; t < P; ++t) h[t] = t < n ? __ldg(col + (size_t)t * D) : (uint16_t)0;
+
+    uint16_t bmin = h[0], bmax = h[0];
     float vmin = bf16f(bmin), vmax = vmin;
     double s1 = 0.0, s2 = 0.0;
-    int t = 0;
-    for (; t + 8 <= n; t += 8) {
-        uint16_t h[8];
 #pragma unroll
-        for (int i = 0; i < 8; ++i) h[i] = __ldg(col + (size_t)(t + i) * D);
-#pragma unroll
-        for (int i = 0; i < 8; ++i) {
-            float x = bf16f(h[i]);
-            if (x < vmin) { vmin = x; bmin = h[i]; }
-            if (x > vmax) { vmax = x; bmax = h[i]; }
-            double xd = (double)x;
+    for (int t = 0; t < P; ++t) {
+        if (t < n) {
+            const float x = bf16f(h[t]);
+            if (x < vmin) { vmin = x; bmin = h[t]; }
+            if (x > vmax) { vmax = x; bmax = h[t]; }
+            const double xd = (double)x;
             s1 = __dadd_rn(s1, xd);
-            s2 = __fma_rn(xd, xd, s2);  // xd*xd is exact, so this equals s2 + xd*xd rounded once
+            s2 = __fma_rn(xd, xd, s2);  // xd*xd is exact, so this is s2 + xd*xd rounded once
         }
-    }
-    for (; t < n; ++t) {
-        uint16_t h = __ldg(col + (size_t)t * D);
-        float x = bf16f(h);
-        if (x < vmin) { vmin = x; bmin = h; }
-        if (x > vmax) { vmax = x; bmax = h; }
-        double xd = (double)x;
-        s1 = __dadd_rn(s1, xd);
-        s2 = __fma_rn(xd, xd, s2);
     }
     const double dn = (double)n;
     const double m = __ddiv_rn(s1, dn);
@@ -68,14 +60,21 @@ __global__ void __launch_bounds__(D) build_meta_kernel(MetaArgs a) {
     mm[D + j] = (float)v;
 }
 
+template <int D>
+cudaError_t launch_d(const MetaArgs &a, cudaStream_t st) {
+    dim3 grid(a.n_pages, a.B, a.Hkv);
+    switch (a.P) {
+        case 16: build_meta_kernel<D, 16><<<grid, D, 0, st>>>(a); break;
+        case 32: build_meta_kernel<D, 32><<<grid, D, 0, st>>>(a); break;
+        case 64: build_meta_kernel<D, 64><<<grid, D, 0, st>>>(a); break;
+        default: return cudaErrorInvalidValue;
+    }
+    return cudaGetLastError();
+}
+
 cudaError_t launch_build_meta(const MetaArgs &a, cudaStream_t st) {
     if (a.n_pages <= 0) return cudaSuccess;
-    dim3 grid(a.n_pages, a.B, a.Hkv);
-    if (a.d == 64)
-        build_meta_kernel<64><<<grid, 64, 0, st>>>(a);
-    else
-        build_meta_kernel<128><<<grid, 128, 0, st>>>(a);
-    return cudaGetLastError();
+    return a.d == 64 ? launch_d<64>(a, st) : launch_d<128>(a, st);
 }
 
 }  // namespace ekv

@@ -33,61 +33,12 @@ __device__ __forceinline__ unsigned key_of(float f) {
     return (x & 0x80000000u) ? ~x : (x | 0x80000000u);
 }
 
-__device__ float block_max(float v, float *sh) {
-#pragma unroll
-    for (int o = 16; o; o >>= 1) v = fmaxf(v, __shfl_xor_sync(FULL, v, o));
-    __syncthreads();
-    if ((threadIdx.x & 31) == 0) sh[threadIdx.x >> 5] = v;
-    __syncthreads();
-    float m = -INFINITY;
-    for (int w = 0; w < (int)(blockDim.x >> 5); ++w) m = fmaxf(m, sh[w]);
-    return m;
-}
 
-__device__ void block_sum2(float &a, float &b, float *sh) {
-#pragma unroll
-    for (int o = 16; o; o >>= 1) {
-        a += __shfl_xor_sync(FULL, a, o);
-        b += __shfl_xor_sync(FULL, b, o);
-    }
-    __syncthreads();
-    if ((threadIdx.x & 31) == 0) {
-        sh[2 * (threadIdx.x >> 5)] = a;
-        sh[2 * (threadIdx.x >> 5) + 1] = b;
-    }
-    __syncthreads();
-    float sa = 0.f, sb = 0.f;
-    for (int w = 0; w < (int)(blockDim.x >> 5); ++w) {
-        sa += sh[2 * w];
-        sb += sh[2 * w + 1];
-    }
-    a = sa;
-    b = sb;
-}
 
-// Write sel[] for the pages p < n for which keep(p) holds, ascending.
-template <class Keep>
-__device__ int compact_ascending(int n, int *sel, int *sh, Keep keep) {
-    int base = 0;
-    for (int t0 = 0; t0 < n; t0 += TILE) {
-        const int p0 = t0 + threadIdx.x * ITEMS;
-        unsigned bits = 0;
-#pragma unroll
-        for (int i = 0; i < ITEMS; ++i) {
-            const int p = p0 + i;
-            if (p < n && keep(p)) bits |= 1u << i;
-        }
-        int tot;
-        int off = block_excl_scan(__popc(bits), sh, &tot);
-        int w = base + off;
-#pragma unroll
-        for (int i = 0; i < ITEMS; ++i)
-            if (bits & (1u << i)) sel[w++] = p0 + i;
-        base += tot;
-    }
-    return base;
-}
 
+// Top-k: the keys of one tile (TILE pages) stay in registers, ITEMS
+// consecutive pages per thread, through the four radix passes and the final
+// ordered compaction; longer sequences take several tiles per pass.
 __global__ void __launch_bounds__(SEL_THREADS) topk_kernel(SelectArgs a) {
     __shared__ int hist[256];
     __shared__ int sh[72];
@@ -104,20 +55,29 @@ __global__ void __launch_bounds__(SEL_THREADS) topk_kernel(SelectArgs a) {
         return;
     }
     const int lane = threadIdx.x & 31;
+    const bool one_tile = n <= TILE;
+    unsigned key[ITEMS];
+    auto load_tile = [&](int t0) {
+        const int p0 = t0 + threadIdx.x * ITEMS;
+#pragma unroll
+        for (int i = 0; i < ITEMS; ++i) key[i] = (p0 + i < n) ? key_of(__ldg(sc + p0 + i)) : 0u;
+    };
+    if (one_tile) load_tile(0);
     unsigned prefix = 0, mask = 0;
     int remaining = k;
     for (int shift = 24; shift >= 0; shift -= 8) {
         for (int i = threadIdx.x; i < 256; i += blockDim.x) hist[i] = 0;
         __syncthreads();
-        const int nround = ceil_div(n, blockDim.x) * blockDim.x;
-        for (int p = threadIdx.x; p < nround; p += blockDim.x) {
-            int bucket = 256 + lane;  // unique dummy for lanes with nothing to count
-            if (p < n) {
-                const unsigned key = key_of(__ldg(sc + p));
-                if ((key & mask) == prefix) bucket = (key >> shift) & 255;
+        for (int t0 = 0; t0 < n; t0 += TILE) {
+            if (!one_tile) load_tile(t0);
+            const int p0 = t0 + threadIdx.x * ITEMS;
+#pragma unroll
+            for (int i = 0; i < ITEMS; ++i) {
+                int bucket = 256 + lane;  // unique dummy for lanes with nothing to count
+                if (p0 + i < n && (key[i] & mask) == prefix) bucket = (key[i] >> shift) & 255;
+                const unsigned peers = __match_any_sync(FULL, bucket);
+                if (bucket < 256 && lane == __ffs(peers) - 1) atomicAdd(&hist[bucket], __popc(peers));
             }
-            const unsigned peers = __match_any_sync(FULL, bucket);
-            if (bucket < 256 && lane == __ffs(peers) - 1) atomicAdd(&hist[bucket], __popc(peers));
         }
         __syncthreads();
         if (threadIdx.x < 32) {
@@ -160,15 +120,14 @@ __global__ void __launch_bounds__(SEL_THREADS) topk_kernel(SelectArgs a) {
     // keys == T are taken in page order up to `remaining` of them
     int eq_base = 0, base = 0;
     for (int t0 = 0; t0 < n; t0 += TILE) {
+        if (!one_tile) load_tile(t0);
         const int p0 = t0 + threadIdx.x * ITEMS;
         unsigned gt = 0, eq = 0;
 #pragma unroll
         for (int i = 0; i < ITEMS; ++i) {
-            const int p = p0 + i;
-            if (p < n) {
-                const unsigned key = key_of(__ldg(sc + p));
-                if (key > T) gt |= 1u << i;
-                if (key == T) eq |= 1u << i;
+            if (p0 + i < n) {
+                if (key[i] > T) gt |= 1u << i;
+                if (key[i] == T) eq |= 1u << i;
             }
         }
         int eq_tot;
@@ -226,10 +185,16 @@ __device__ __forceinline__ void gauss_JJ(float c, float &jr, float &jr1) {
 
 constexpr int GCAP = 3072;  // pruned candidate pages held on chip
 
+// Gaussian selection.  One tile (TILE pages, ITEMS per thread) of mu, sigma
+// and the bound is loaded up front; pages are interleaved across threads for
+// the max / pruning pass and contiguous per thread for the ordered
+// compaction.  Newton iterations reduce F and F' with one barrier each
+// (double-buffered partials).
 template <int R>
 __global__ void __launch_bounds__(SEL_THREADS) gauss_kernel(SelectArgs a) {
     __shared__ float cm[GCAP], cs[GCAP], cn[GCAP];
-    __shared__ float shf[2 * 32 + 2];
+    __shared__ float shf[2][2 * 32];
+    __shared__ float shm[32];
     __shared__ int shi[72];
     __shared__ int ncand;
     const int bh = blockIdx.x;
@@ -238,6 +203,7 @@ __global__ void __launch_bounds__(SEL_THREADS) gauss_kernel(SelectArgs a) {
     const int n = n_pages_of(seq, a.P);
     const size_t row = (size_t)bh * a.max_pages;
     const float a1 = a.alpha - 1.f;
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
     if (n == 0) {
         if (threadIdx.x == 0) {
             a.cnt[bh] = 0;
@@ -245,32 +211,57 @@ __global__ void __launch_bounds__(SEL_THREADS) gauss_kernel(SelectArgs a) {
         }
         return;
     }
+    const bool one_tile = n <= TILE;
+    // bound of this thread's contiguous pages (for the final compaction)
+    float ub[ITEMS];
+    if (one_tile) {
+        const int p0 = threadIdx.x * ITEMS;
+#pragma unroll
+        for (int i = 0; i < ITEMS; ++i) ub[i] = (p0 + i < n) ? __ldg(a.bbox + row + p0 + i) : 0.f;
+    }
+    // interleaved pages p = t0 + tid + SEL_THREADS*i
+    float mm[ITEMS], ss[ITEMS];
+    auto load_ms = [&](int t0) {
+#pragma unroll
+        for (int i = 0; i < ITEMS; ++i) {
+            const int p = t0 + threadIdx.x + SEL_THREADS * i;
+            mm[i] = p < n ? a1 * __ldg(a.mu + row + p) : -INFINITY;
+            ss[i] = p < n ? a1 * __ldg(a.sigma + row + p) : 0.f;
+        }
+    };
     float mloc = -INFINITY;
-    for (int p = threadIdx.x; p < n; p += blockDim.x) mloc = fmaxf(mloc, a1 * a.mu[row + p]);
-    const float mmax = block_max(mloc, shf);
-    const float tau0 = mmax - 1.f;
-
+    for (int t0 = 0; t0 < n; t0 += TILE) {
+        load_ms(t0);
+#pragma unroll
+        for (int i = 0; i < ITEMS; ++i) mloc = fmaxf(mloc, mm[i]);
+    }
+#pragma unroll
+    for (int o = 16; o; o >>= 1) mloc = fmaxf(mloc, __shfl_xor_sync(FULL, mloc, o));
+    if (lane == 0) shm[warp] = mloc;
     if (threadIdx.x == 0) ncand = 0;
     __syncthreads();
-    const int nround = ceil_div(n, blockDim.x) * blockDim.x;
-    for (int p = threadIdx.x; p < nround; p += blockDim.x) {
-        float m = 0.f, s = 0.f;
-        bool keep = false;
-        if (p < n) {
-            m = a1 * a.mu[row + p];
-            s = a1 * a.sigma[row + p];
-            keep = m + 10.f * s >= tau0;
-        }
-        const unsigned bal = __ballot_sync(FULL, keep);
-        int base = 0;
-        if ((threadIdx.x & 31) == 0 && bal) base = atomicAdd(&ncand, __popc(bal));
-        base = __shfl_sync(FULL, base, 0);
-        if (keep) {
-            const int slot = base + __popc(bal & ((1u << (threadIdx.x & 31)) - 1u));
-            if (slot < GCAP) {
-                cm[slot] = m;
-                cs[slot] = s;
-                cn[slot] = (float)tokens_in_page(seq, a.P, p);
+    float mmax = -INFINITY;
+    for (int w = 0; w < SEL_THREADS / 32; ++w) mmax = fmaxf(mmax, shm[w]);
+    const float tau0 = mmax - 1.f;
+
+    for (int t0 = 0; t0 < n; t0 += TILE) {
+        if (!one_tile) load_ms(t0);
+#pragma unroll
+        for (int i = 0; i < ITEMS; ++i) {
+            const int p = t0 + threadIdx.x + SEL_THREADS * i;
+            const bool keep = p < n && mm[i] + 10.f * ss[i] >= tau0;
+            const unsigned bal = __ballot_sync(FULL, keep);
+            if (!bal) continue;
+            int base = 0;
+            if (lane == __ffs(bal) - 1) base = atomicAdd(&ncand, __popc(bal));
+            base = __shfl_sync(FULL, base, __ffs(bal) - 1);
+            if (keep) {
+                const int slot = base + __popc(bal & ((1u << lane) - 1u));
+                if (slot < GCAP) {
+                    cm[slot] = mm[i];
+                    cs[slot] = ss[i];
+                    cn[slot] = (float)tokens_in_page(seq, a.P, p);
+                }
             }
         }
     }
@@ -306,13 +297,29 @@ __global__ void __launch_bounds__(SEL_THREADS) gauss_kernel(SelectArgs a) {
     for (int it = 0; it < 64; ++it) {
         float F = 0.f, Fp = 0.f;
         if (!overflow) {
-            for (int i = threadIdx.x; i < nc; i += blockDim.x) contrib(cm[i], cs[i], cn[i], tau, F, Fp);
+            for (int i = threadIdx.x; i < nc; i += SEL_THREADS) contrib(cm[i], cs[i], cn[i], tau, F, Fp);
         } else {
-            for (int p = threadIdx.x; p < n; p += blockDim.x)
+            for (int p = threadIdx.x; p < n; p += SEL_THREADS)
                 contrib(a1 * a.mu[row + p], a1 * a.sigma[row + p], (float)tokens_in_page(seq, a.P, p), tau, F,
                         Fp);
         }
-        block_sum2(F, Fp, shf);
+#pragma unroll
+        for (int o = 16; o; o >>= 1) {
+            F += __shfl_xor_sync(FULL, F, o);
+            Fp += __shfl_xor_sync(FULL, Fp, o);
+        }
+        float *buf = shf[it & 1];
+        if (lane == 0) {
+            buf[2 * warp] = F;
+            buf[2 * warp + 1] = Fp;
+        }
+        __syncthreads();
+        F = 0.f;
+        Fp = 0.f;
+        for (int w = 0; w < SEL_THREADS / 32; ++w) {
+            F += buf[2 * w];
+            Fp += buf[2 * w + 1];
+        }
         if (!(F > 1.f + 2e-6f) || !(Fp < 0.f)) break;
         // Newton on g = F^(1/R): step = R (F - F^(1-1/R)) / (-F')
         const float step = (float)R * (F - powf(F, 1.f - 1.f / (float)R)) / (-Fp);
@@ -322,10 +329,26 @@ __global__ void __launch_bounds__(SEL_THREADS) gauss_kernel(SelectArgs a) {
     if (threadIdx.x == 0 && a.tau_hat) a.tau_hat[bh] = tau;
 
     const float thr = tau - a.delta;
-    const float *bb = a.bbox + row;
     int *sel = a.sel + row;
-    const int cnt = compact_ascending(n, sel, shi, [&](int p) { return a1 * __ldg(bb + p) > thr; });
-    if (threadIdx.x == 0) a.cnt[bh] = cnt;
+    int base = 0;
+    for (int t0 = 0; t0 < n; t0 += TILE) {
+        const int p0 = t0 + threadIdx.x * ITEMS;
+        if (!one_tile) {
+#pragma unroll
+            for (int i = 0; i < ITEMS; ++i) ub[i] = (p0 + i < n) ? __ldg(a.bbox + row + p0 + i) : 0.f;
+        }
+        unsigned bits = 0;
+#pragma unroll
+        for (int i = 0; i < ITEMS; ++i)
+            if (p0 + i < n && a1 * ub[i] > thr) bits |= 1u << i;
+        int tot;
+        int w = base + block_excl_scan(__popc(bits), shi, &tot);
+#pragma unroll
+        for (int i = 0; i < ITEMS; ++i)
+            if (bits & (1u << i)) sel[w++] = p0 + i;
+        base += tot;
+    }
+    if (threadIdx.x == 0) a.cnt[bh] = base;
 }
 
 }  // namespace

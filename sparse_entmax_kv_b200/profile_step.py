@@ -21,8 +21,11 @@ def main():
     ap.add_argument("--workload", default="gauss_gqa_L1m")
     ap.add_argument("--steps", type=int, default=2)
     ap.add_argument("--dense", action="store_true")
+    ap.add_argument("--L", type=int, default=0, help="override the context length")
     args = ap.parse_args()
     wl = CONFIGS[args.workload]
+    if args.L:
+        wl = wl.shrink(L=args.L)
     policy = wl.policy if wl.policy != "dense" else "topk"
     inp = make_inputs(wl, 4000, device="cuda")
     dec = EntmaxKVDecoder(inp["k_cache"], inp["v_cache"], inp["page_table"], inp["seq_lens"], wl.Hq,
