@@ -468,8 +468,10 @@ __global__ void __launch_bounds__(TAU_THREADS) tau_pv_kernel(const __grid_consta
     const float thr = zmax - 1.f;
     if (threadIdx.x == 0) ncand = 0;
     __syncthreads();
-    // keep the candidates above the final max - 1; eight loads in flight
-    for (int i0 = threadIdx.x; i0 < n_all; i0 += 8 * TAU_THREADS) {
+    // keep the candidates above the final max - 1; eight loads in flight.
+    // The loop bound is block-uniform so every lane reaches the ballots.
+    for (int base0 = 0; base0 < n_all; base0 += 8 * TAU_THREADS) {
+        const int i0 = base0 + threadIdx.x;
         float zz[8];
 #pragma unroll
         for (int u = 0; u < 8; ++u) {
