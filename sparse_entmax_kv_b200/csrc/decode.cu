@@ -443,10 +443,15 @@ constexpr int ZCAP = 4096;  // filtered candidates held on chip per head
 template <int D, bool GATHER>
 __global__ void __launch_bounds__(TAU_THREADS) tau_pv_kernel(const __grid_constant__ DecodeArgs a) {
     constexpr int CPL = D / 32;
-    __shared__ float cz[ZCAP];
-    __shared__ int ci[ZCAP];  // index into the head's global candidate list
-    __shared__ float red[TAU_WARPS][33];
-    __shared__ float accs[TAU_WARPS][D];
+    // candidates (z and their index in the head's global list); once the
+    // gather has read them, the same bytes hold the per-warp output partials
+    __shared__ __align__(16) unsigned char cbuf[ZCAP * 8];
+    float *cz = reinterpret_cast<float *>(cbuf);
+    int *ci = reinterpret_cast<int *>(cbuf + ZCAP * 4);
+    double(*accs)[D] = reinterpret_cast<double(*)[D]>(cbuf);
+    static_assert(TAU_WARPS * D * 8 <= ZCAP * 8, "partials must fit the candidate buffer");
+    __shared__ double red[TAU_WARPS][33];
+    __shared__ unsigned balw[2][TAU_WARPS];
     __shared__ int ncand;
     __shared__ float br[2];
     const int bh = blockIdx.x;
@@ -512,14 +517,13 @@ __global__ void __launch_bounds__(TAU_THREADS) tau_pv_kernel(const __grid_consta
             for (int pass = 0; pass < 4 && hi - lo > tol; ++pass) {
                 const float w = (hi - lo) / (float)(TAU_THREADS + 1);
                 const float t = lo + w * (float)(threadIdx.x + 1);
-                float f = 0.f;
-                for (int c = 0; c < nc; ++c) f += pos_pow(cz[c] - t, r, ri);
-                const unsigned bal = __ballot_sync(FULL, f >= 1.f);  // still left of the root
-                if (lane == 0) reinterpret_cast<unsigned *>(&red[pass & 1][0])[warp] = bal;
+                double f = 0.0;  // fp64: the candidates' order on chip varies between calls
+                for (int c = 0; c < nc; ++c) f += (double)pos_pow(cz[c] - t, r, ri);
+                const unsigned bal = __ballot_sync(FULL, f >= 1.0);  // still left of the root
+                if (lane == 0) balw[pass & 1][warp] = bal;
                 __syncthreads();
                 int cntge = 0;  // points increase with thread index and f decreases: a prefix
-                for (int ww = 0; ww < TAU_WARPS; ++ww)
-                    cntge += __popc(reinterpret_cast<unsigned *>(&red[pass & 1][0])[ww]);
+                for (int ww = 0; ww < TAU_WARPS; ++ww) cntge += __popc(balw[pass & 1][ww]);
                 const float nlo = cntge > 0 ? lo + w * (float)cntge : lo;
                 const float nhi = cntge < TAU_THREADS ? lo + w * (float)(cntge + 1) : hi;
                 lo = nlo;
@@ -529,14 +533,14 @@ __global__ void __launch_bounds__(TAU_THREADS) tau_pv_kernel(const __grid_consta
             // 32 points per pass, candidates spread over the block
             for (int pass = 0; pass < 12 && hi - lo > tol; ++pass) {
                 const float w = (hi - lo) / 33.f;
-                float f[32];
+                double f[32];
 #pragma unroll
-                for (int j = 0; j < 32; ++j) f[j] = 0.f;
+                for (int j = 0; j < 32; ++j) f[j] = 0.0;
                 for (int c = threadIdx.x; c < nloop; c += TAU_THREADS) {
                     const float z = cz_at(c);
                     if (!(z > thr)) continue;
 #pragma unroll
-                    for (int j = 0; j < 32; ++j) f[j] += pos_pow(z - (lo + w * (float)(j + 1)), r, ri);
+                    for (int j = 0; j < 32; ++j) f[j] += (double)pos_pow(z - (lo + w * (float)(j + 1)), r, ri);
                 }
                 // transpose-reduce: lane l ends with the warp sum of point l
 #pragma unroll
@@ -544,17 +548,17 @@ __global__ void __launch_bounds__(TAU_THREADS) tau_pv_kernel(const __grid_consta
 #pragma unroll
                     for (int i = 0; i < s; ++i) {
                         const bool up = lane & s;
-                        const float send = up ? f[i] : f[i + s];
-                        const float keep = up ? f[i + s] : f[i];
+                        const double send = up ? f[i] : f[i + s];
+                        const double keep = up ? f[i + s] : f[i];
                         f[i] = keep + __shfl_xor_sync(FULL, send, s);
                     }
                 }
                 red[warp][lane] = f[0];
                 __syncthreads();
                 if (warp == 0) {
-                    float tot = 0.f;
+                    double tot = 0.0;
                     for (int ww = 0; ww < TAU_WARPS; ++ww) tot += red[ww][lane];
-                    const unsigned bal = __ballot_sync(FULL, tot >= 1.f);
+                    const unsigned bal = __ballot_sync(FULL, tot >= 1.0);
                     if (lane == 0) {
                         const int cntge = __popc(bal);
                         br[0] = cntge > 0 ? lo + w * (float)cntge : lo;
@@ -578,10 +582,12 @@ __global__ void __launch_bounds__(TAU_THREADS) tau_pv_kernel(const __grid_consta
     if (!GATHER) return;
 
     // p v over the support: each warp takes its share of the candidates with
-    // z > tau, up to eight value rows in flight at a time
-    float acc[CPL];
+    // z > tau, up to eight value rows in flight at a time.  Sums run in fp64
+    // (p v is exact there), so the varying order of the candidates on chip
+    // does not show in the fp32 result.
+    double acc[CPL];
 #pragma unroll
-    for (int c = 0; c < CPL; ++c) acc[c] = 0.f;
+    for (int c = 0; c < CPL; ++c) acc[c] = 0.0;
     const size_t lstride = (size_t)a.max_pages * a.P;
     for (int c0 = warp * 32; c0 < nloop; c0 += TAU_WARPS * 32) {
         const int c = c0 + lane;
@@ -632,17 +638,18 @@ __global__ void __launch_bounds__(TAU_THREADS) tau_pv_kernel(const __grid_consta
 #pragma unroll
             for (int i = 0; i < 8; ++i)
 #pragma unroll
-                for (int cc = 0; cc < CPL; ++cc) acc[cc] = fmaf(pp[i], vv[i][cc], acc[cc]);
+                for (int cc = 0; cc < CPL; ++cc) acc[cc] = fma((double)pp[i], (double)vv[i][cc], acc[cc]);
         }
     }
+    __syncthreads();  // every warp is done with the candidates
 #pragma unroll
     for (int cc = 0; cc < CPL; ++cc) accs[warp][lane * CPL + cc] = acc[cc];
     __syncthreads();
     for (int j = threadIdx.x; j < D; j += TAU_THREADS) {
-        float s = 0.f;
+        double s = 0.0;
 #pragma unroll
         for (int w = 0; w < TAU_WARPS; ++w) s += accs[w][j];
-        a.out[(size_t)bh * D + j] = s;
+        a.out[(size_t)bh * D + j] = (float)s;
     }
 }
 
