@@ -12,17 +12,17 @@
 //                  rows 32 steps at a time); z = (alpha-1) q.k/sqrt(d) for all
 //                  G heads of the group from one copy of each tile (tensor-core
 //                  m16n8k16, tokens as M and the heads as N, when G >= 2; CUDA
-//                  cores when G == 1).  Every z above (running max - 1) is
-//                  appended to the head's candidate list with its value-row
-//                  index; since tau >= max z - 1 (no weight exceeds 1), no
-//                  token outside the list can carry weight.
-//   tau_pv_kernel  per (sequence, query head): filters the candidates against
-//                  the final max, solves sum (z - tau)_+^r = 1 exactly by
-//                  multisection on [z_max - 1, z_max - n^(1-alpha)], and sums
-//                  p v over the support, reading only those value rows.
-// Full-cache entmax runs qk_kernel over every page (also writing z for every
-// token), tau_pv_kernel for tau, and pv_stream_kernel, which streams every V
-// tile through the TMA ring.  Full-cache softmax runs softmax_kernel (K and V
+//                  cores when G == 1), stored in list order, and the per-head
+//                  max of z.
+//   tau_pv_kernel  per (sequence, query head): every token that can carry
+//                  weight has z > max z - 1 (no weight exceeds 1), so those
+//                  candidates are compacted on chip in list order; the exact
+//                  root of sum (z - tau)_+^r = 1 is bracketed in
+//                  [z_max - 1, z_max - n^(1-alpha)] and narrowed by
+//                  multisection, and p v is summed over the support, reading
+//                  only those value rows.
+// Full-cache entmax runs qk_kernel over every page, tau_pv_kernel for tau, and
+// pv_stream_kernel, which streams every V tile through the TMA ring.  Full-cache softmax runs softmax_kernel (K and V
 // tiles per stage, online max / sum per split); both dense paths combine
 // their splits in a fixed order in the last CTA of each group.
 #include "common.cuh"
@@ -74,7 +74,6 @@ __global__ void __launch_bounds__(512) union_kernel(DecodeArgs a) {
         }
         cnts[threadIdx.x] = c;
         a.ws.zmax[bh] = ORD_NEG_INF;
-        a.ws.cand_cnt[bh] = 0;
     }
     __syncthreads();
     if (threadIdx.x == 0) {
@@ -136,10 +135,7 @@ __global__ void __launch_bounds__(512) union_kernel(DecodeArgs a) {
 
 __global__ void dense_init_kernel(DecodeArgs a) {
     const int i = blockIdx.x * blockDim.x + threadIdx.x;
-    if (i < a.B * a.Hq) {
-        a.ws.zmax[i] = ORD_NEG_INF;
-        a.ws.cand_cnt[i] = 0;
-    }
+    if (i < a.B * a.Hq) a.ws.zmax[i] = ORD_NEG_INF;
     if (i < a.B * a.Hkv) a.ws.counters[i] = 0;
 }
 
@@ -203,6 +199,7 @@ __device__ void produce(const DecodeArgs &a, const CUtensorMap *m0, const CUtens
                 } else {
                     atomicOr(a.status, ENTMAXKV_STATUS_BAD_PAGE);
                 }
+                if (!dense) a.ws.union_blk[(size_t)bk * a.max_pages + e] = r.blk;
             }
             stash[k] = r;
         }
@@ -247,22 +244,6 @@ __device__ void produce(const DecodeArgs &a, const CUtensorMap *m0, const CUtens
 __device__ __forceinline__ const unsigned char *tile_chunk(const unsigned char *page_base, int P, int r, int c16) {
     const int box = c16 >> 3, cc = c16 & 7;
     return page_base + box * P * 128 + r * 128 + ((cc ^ (r & 7)) << 4);
-}
-
-// Append the lanes' candidates (pred) of one head to its list.
-__device__ __forceinline__ void emit_candidates(const DecodeArgs &a, int bh, bool pred, float z, int row, int lpos) {
-    const unsigned bal = __ballot_sync(FULL, pred);
-    if (!bal) return;
-    const int lane = threadIdx.x & 31;
-    const int leader = __ffs(bal) - 1;
-    int base = 0;
-    if (lane == leader) base = atomicAdd(&a.ws.cand_cnt[bh], __popc(bal));
-    base = __shfl_sync(FULL, base, leader);
-    if (pred) {
-        const size_t pos = (size_t)bh * a.max_pages * a.P + base + __popc(bal & ((1u << lane) - 1u));
-        a.ws.cand[pos] = make_int2(__float_as_int(z), row);
-        if (a.p_out) a.ws.cand_lpos[pos] = lpos;
-    }
 }
 
 // ----------------------------------------------------------------- q . K^T
@@ -323,9 +304,7 @@ __global__ void __launch_bounds__(DEC_THREADS) qk_kernel(const __grid_constant__
         const int h0 = 2 * (lane & 3);  // this lane's two heads: h0, h0+1
         const int bh0 = b * a.Hq + kvh * G + (h0 < G ? h0 : 0);
         const int bh1 = b * a.Hq + kvh * G + (h0 + 1 < G ? h0 + 1 : 0);
-        // running max of z per head (warp-wide), seeded from the global max
-        float run0 = h0 < G ? ord2f(a.ws.zmax[bh0]) : -INFINITY;
-        float run1 = h0 + 1 < G ? ord2f(a.ws.zmax[bh1]) : -INFINITY;
+        float run0 = -INFINITY, run1 = -INFINITY;  // this lane's max of z for heads h0, h0+1
         for (int it = 0; it < my_n; ++it) {
             const int st = it % NS, ph = (it / NS) & 1;
             if (!mbar_wait(&R.full[st], ph, a.status)) return;
@@ -355,33 +334,19 @@ __global__ void __launch_bounds__(DEC_THREADS) qk_kernel(const __grid_constant__
                     const int t = r0 + (lane >> 2) + 8 * (v >> 1);
                     const bool use = hh < G && t < pi.nval && ((pi.mask >> hh) & 1);
                     z[v] = use ? acc[v] * zs : -INFINITY;
-                    if (DENSE && hh < G) a.ws.zbuf[tok_row(a, b, kvh * G + hh) + (size_t)pi.upos * P + t] = z[v];
+                    if (hh < G) a.ws.zbuf[tok_row(a, b, kvh * G + hh) + (size_t)pi.upos * P + t] = z[v];
                     if (a.p_out && use) a.p_out[tok_row(a, b, kvh * G + hh) + (size_t)pi.page * P + t] = 0.f;
                 }
-                float m0 = fmaxf(z[0], z[2]), m1 = fmaxf(z[1], z[3]);
-#pragma unroll
-                for (int o = 4; o < 32; o <<= 1) {
-                    m0 = fmaxf(m0, __shfl_xor_sync(FULL, m0, o));
-                    m1 = fmaxf(m1, __shfl_xor_sync(FULL, m1, o));
-                }
-                run0 = fmaxf(run0, m0);
-                run1 = fmaxf(run1, m1);
-#pragma unroll
-                for (int hh = 0; hh < G; ++hh) {
-#pragma unroll
-                    for (int tt = 0; tt < 2; ++tt) {
-                        const int v = (hh & 1) + 2 * tt;
-                        const bool mine = (lane & 3) == (hh >> 1);
-                        const float thr = ((hh & 1) ? run1 : run0) - 1.f;
-                        const bool pred = mine && z[v] > thr;
-                        const int t = r0 + (lane >> 2) + 8 * tt;
-                        emit_candidates(a, b * a.Hq + kvh * G + hh, pred, z[v], (pi.blk * a.Hkv + kvh) * P + t,
-                                        pi.page * P + t);
-                    }
-                }
+                run0 = fmaxf(run0, fmaxf(z[0], z[2]));
+                run1 = fmaxf(run1, fmaxf(z[1], z[3]));
             }
             __syncwarp();
             if (lane == 0) mbar_arrive(&R.empty[st]);
+        }
+#pragma unroll
+        for (int o = 4; o < 32; o <<= 1) {
+            run0 = fmaxf(run0, __shfl_xor_sync(FULL, run0, o));
+            run1 = fmaxf(run1, __shfl_xor_sync(FULL, run1, o));
         }
         if (lane < 4) {
             if (h0 < G && run0 > -INFINITY) atomicMax(&a.ws.zmax[bh0], f2ord(run0));
@@ -390,7 +355,7 @@ __global__ void __launch_bounds__(DEC_THREADS) qk_kernel(const __grid_constant__
     } else {
         // G == 1: thread per token, q broadcast from shared memory
         const int bh = b * a.Hq + kvh;
-        float run = ord2f(a.ws.zmax[bh]);
+        float run = -INFINITY;
         const int ti = threadIdx.x;  // token within the stage
         for (int it = 0; it < my_n; ++it) {
             const int st = it % NS, ph = (it / NS) & 1;
@@ -420,15 +385,13 @@ __global__ void __launch_bounds__(DEC_THREADS) qk_kernel(const __grid_constant__
                 z = acc * zs;
                 if (a.p_out) a.p_out[tok_row(a, b, kvh) + (size_t)pi.page * P + r] = 0.f;
             }
-            if (DENSE && pi.page >= 0) a.ws.zbuf[tok_row(a, b, kvh) + (size_t)pi.upos * P + r] = z;
-            float m = z;
-#pragma unroll
-            for (int o = 16; o; o >>= 1) m = fmaxf(m, __shfl_xor_sync(FULL, m, o));
-            run = fmaxf(run, m);
-            emit_candidates(a, bh, use && z > run - 1.f, z, (pi.blk * a.Hkv + kvh) * P + r, pi.page * P + r);
+            if (pi.page >= 0) a.ws.zbuf[tok_row(a, b, kvh) + (size_t)pi.upos * P + r] = z;
+            run = fmaxf(run, z);
             __syncwarp();
             if (lane == 0) mbar_arrive(&R.empty[st]);
         }
+#pragma unroll
+        for (int o = 16; o; o >>= 1) run = fmaxf(run, __shfl_xor_sync(FULL, run, o));
         if (lane == 0 && run > -INFINITY) atomicMax(&a.ws.zmax[bh], f2ord(run));
     }
 }
@@ -437,31 +400,37 @@ __global__ void __launch_bounds__(DEC_THREADS) qk_kernel(const __grid_constant__
 
 constexpr int TAU_THREADS = 512;
 constexpr int TAU_WARPS = TAU_THREADS / 32;
-constexpr int ZCAP = 4096;  // filtered candidates held on chip per head
+constexpr int ZCAP = 4096;  // candidates held on chip per head
+constexpr int TAU_C = 32;   // list positions per thread per scan tile
 
 // Exact threshold and (GATHER) the weighted sum of the support's value rows.
 template <int D, bool GATHER>
-__global__ void __launch_bounds__(TAU_THREADS) tau_pv_kernel(const __grid_constant__ DecodeArgs a) {
+__global__ void __launch_bounds__(TAU_THREADS) tau_pv_kernel(const __grid_constant__ DecodeArgs a, int dense) {
     constexpr int CPL = D / 32;
-    // candidates (z and their index in the head's global list); once the
-    // gather has read them, the same bytes hold the per-warp output partials
+    // candidates (z and list position) in list order; once the gather has
+    // read them, the same bytes hold the per-warp output partials
     __shared__ __align__(16) unsigned char cbuf[ZCAP * 8];
     float *cz = reinterpret_cast<float *>(cbuf);
-    int *ci = reinterpret_cast<int *>(cbuf + ZCAP * 4);
+    int *cpos = reinterpret_cast<int *>(cbuf + ZCAP * 4);
     double(*accs)[D] = reinterpret_cast<double(*)[D]>(cbuf);
     static_assert(TAU_WARPS * D * 8 <= ZCAP * 8, "partials must fit the candidate buffer");
     __shared__ double red[TAU_WARPS][33];
     __shared__ unsigned balw[2][TAU_WARPS];
-    __shared__ int ncand;
+    __shared__ int sh[72];
     __shared__ float br[2];
     const int bh = blockIdx.x;
+    const int b = bh / a.Hq, h = bh % a.Hq;
+    const int G = a.Hq / a.Hkv, kvh = h / G;
+    const int bk = b * a.Hkv + kvh;
+    const int P = a.P;
     const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+    const int np = n_pages_of(a.seq_lens[b], P);
+    const int U = dense ? np : a.ws.union_cnt[bk];
+    const int n_tok = U * P;  // a multiple of 16
     const float zmax = ord2f(a.ws.zmax[bh]);
-    const int n_all = a.ws.cand_cnt[bh];
-    const int2 *cl = a.ws.cand + (size_t)bh * a.max_pages * a.P;
     const float r = 1.f / (a.alpha - 1.f);
     const int ri = a.r_int;
-    if (!(zmax > -INFINITY) || n_all <= 0) {  // no token at all
+    if (!(zmax > -INFINITY)) {  // no token at all
         if (GATHER)
             for (int j = threadIdx.x; j < D; j += TAU_THREADS) a.out[(size_t)bh * D + j] = 0.f;
         if (threadIdx.x == 0) {
@@ -471,42 +440,51 @@ __global__ void __launch_bounds__(TAU_THREADS) tau_pv_kernel(const __grid_consta
         return;
     }
     const float thr = zmax - 1.f;
-    if (threadIdx.x == 0) ncand = 0;
-    __syncthreads();
-    // keep the candidates above the final max - 1; eight loads in flight.
-    // The loop bound is block-uniform so every lane reaches the ballots.
-    for (int base0 = 0; base0 < n_all; base0 += 8 * TAU_THREADS) {
-        const int i0 = base0 + threadIdx.x;
-        float zz[8];
+    const float *zr = a.ws.zbuf + tok_row(a, b, h);
+
+    // ordered compaction of the positions with z > thr: each thread scans
+    // TAU_C consecutive positions per tile (all loads issued first), and one
+    // block scan places them
+    int nc = 0;
+    for (int t0 = 0; t0 < n_tok; t0 += TAU_THREADS * TAU_C) {
+        const int p0 = t0 + threadIdx.x * TAU_C;
+        float4 v[TAU_C / 4];
 #pragma unroll
-        for (int u = 0; u < 8; ++u) {
-            const int i = i0 + u * TAU_THREADS;
-            zz[u] = i < n_all ? __int_as_float(__ldcg(&cl[i].x)) : -INFINITY;
+        for (int i = 0; i < TAU_C / 4; ++i)
+            v[i] = p0 + 4 * i < n_tok ? __ldcg(reinterpret_cast<const float4 *>(zr + p0 + 4 * i))
+                                      : make_float4(-INFINITY, -INFINITY, -INFINITY, -INFINITY);
+        unsigned bits = 0;
+#pragma unroll
+        for (int i = 0; i < TAU_C / 4; ++i) {
+            if (v[i].x > thr) bits |= 1u << (4 * i);
+            if (v[i].y > thr) bits |= 1u << (4 * i + 1);
+            if (v[i].z > thr) bits |= 1u << (4 * i + 2);
+            if (v[i].w > thr) bits |= 1u << (4 * i + 3);
         }
+        int tot;
+        int w = nc + block_excl_scan(__popc(bits), sh, &tot);
 #pragma unroll
-        for (int u = 0; u < 8; ++u) {
-            const bool c = zz[u] > thr;
-            const unsigned bal = __ballot_sync(FULL, c);
-            if (!bal) continue;
-            int base = 0;
-            if (lane == __ffs(bal) - 1) base = atomicAdd(&ncand, __popc(bal));
-            base = __shfl_sync(FULL, base, __ffs(bal) - 1);
-            if (c) {
-                const int slot = base + __popc(bal & ((1u << lane) - 1u));
-                if (slot < ZCAP) {
-                    cz[slot] = zz[u];
-                    ci[slot] = i0 + u * TAU_THREADS;
+        for (int i = 0; i < TAU_C / 4; ++i) {
+            const float vv[4] = {v[i].x, v[i].y, v[i].z, v[i].w};
+#pragma unroll
+            for (int j = 0; j < 4; ++j) {
+                if (bits & (1u << (4 * i + j))) {
+                    if (w < ZCAP) {
+                        cz[w] = vv[j];
+                        cpos[w] = p0 + 4 * i + j;
+                    }
+                    ++w;
                 }
             }
         }
+        nc += tot;
     }
     __syncthreads();
-    const int nc = ncand;
     const bool onchip = nc <= ZCAP;
     if (!onchip && threadIdx.x == 0) atomicOr(a.status, ENTMAXKV_STATUS_OVERFLOW);
-    // off chip: scan the head's whole list, filtering on thr
-    const int nloop = onchip ? nc : n_all;
-    auto cz_at = [&](int i) -> float { return onchip ? cz[i] : __int_as_float(__ldcg(&cl[i].x)); };
+    // off chip: scan the head's whole z row, filtering on thr
+    const int nloop = onchip ? nc : n_tok;
+    auto cz_at = [&](int i) -> float { return onchip ? cz[i] : __ldcg(zr + i); };
 
     float lo = thr;
     float hi = zmax - powf((float)nc, 1.f - a.alpha);
@@ -517,7 +495,7 @@ __global__ void __launch_bounds__(TAU_THREADS) tau_pv_kernel(const __grid_consta
             for (int pass = 0; pass < 4 && hi - lo > tol; ++pass) {
                 const float w = (hi - lo) / (float)(TAU_THREADS + 1);
                 const float t = lo + w * (float)(threadIdx.x + 1);
-                double f = 0.0;  // fp64: the candidates' order on chip varies between calls
+                double f = 0.0;
                 for (int c = 0; c < nc; ++c) f += (double)pos_pow(cz[c] - t, r, ri);
                 const unsigned bal = __ballot_sync(FULL, f >= 1.0);  // still left of the root
                 if (lane == 0) balw[pass & 1][warp] = bal;
@@ -583,22 +561,27 @@ __global__ void __launch_bounds__(TAU_THREADS) tau_pv_kernel(const __grid_consta
 
     // p v over the support: each warp takes its share of the candidates with
     // z > tau, up to eight value rows in flight at a time.  Sums run in fp64
-    // (p v is exact there), so the varying order of the candidates on chip
-    // does not show in the fp32 result.
+    // (p v is exact there).
     double acc[CPL];
 #pragma unroll
     for (int c = 0; c < CPL; ++c) acc[c] = 0.0;
-    const size_t lstride = (size_t)a.max_pages * a.P;
+    const size_t lstride = (size_t)a.max_pages * P;
     for (int c0 = warp * 32; c0 < nloop; c0 += TAU_WARPS * 32) {
         const int c = c0 + lane;
         const float z = c < nloop ? cz_at(c) : -INFINITY;
-        const int gi = c < nloop ? (onchip ? ci[c] : c) : 0;
+        const int pos = c < nloop ? (onchip ? cpos[c] : c) : 0;
         const float p = pos_pow(z - tau, r, ri);
         unsigned bal = __ballot_sync(FULL, p > 0.f);
         int row = 0;
         if (p > 0.f) {
-            row = __ldcg(&cl[gi].y);
-            if (a.p_out) a.p_out[(size_t)bh * lstride + __ldcg(&a.ws.cand_lpos[(size_t)bh * lstride + gi])] = p;
+            const int up = pos / P, t = pos - up * P;
+            const int blk = dense ? __ldg(a.page_table + (size_t)b * a.max_pages + up)
+                                  : __ldcg(a.ws.union_blk + (size_t)bk * a.max_pages + up);
+            row = (blk * a.Hkv + kvh) * P + t;
+            if (a.p_out) {
+                const int page = dense ? up : (__ldcg(a.ws.union_e + (size_t)bk * a.max_pages + up) >> 8);
+                a.p_out[(size_t)bh * lstride + (size_t)page * P + t] = p;
+            }
         }
         while (bal) {
             int src[8];
@@ -1014,8 +997,10 @@ __global__ void __launch_bounds__(DEC_THREADS) softmax_kernel(const __grid_const
 
 // ---------------------------------------------------------------- launch
 
+// Splits per (sequence, kv head) so that the whole grid fits one wave of
+// per_sm resident CTAs on every SM.
 int pick_splits(int sms, int per_sm, int groups, int max_steps, int cap) {
-    int s = ceil_div(sms * per_sm, groups > 0 ? groups : 1);
+    int s = (sms * per_sm) / (groups > 0 ? groups : 1);
     if (s > max_steps) s = max_steps;
     if (s > cap) s = cap;
     return s < 1 ? 1 : s;
@@ -1047,7 +1032,7 @@ cudaError_t sparse_t(const DecodeArgs &a, cudaStream_t st) {
     union_kernel<<<groups, 512, ub, st>>>(a);
     if ((e = cudaGetLastError()) != cudaSuccess) return e;
     if ((e = launch_qk<D, G, false>(a, st)) != cudaSuccess) return e;
-    tau_pv_kernel<D, true><<<a.B * a.Hq, TAU_THREADS, 0, st>>>(a);
+    tau_pv_kernel<D, true><<<a.B * a.Hq, TAU_THREADS, 0, st>>>(a, 0);
     return cudaGetLastError();
 }
 
@@ -1059,7 +1044,7 @@ cudaError_t dense_entmax_t(const DecodeArgs &a, cudaStream_t st) {
     dense_init_kernel<<<ceil_div(n, 256), 256, 0, st>>>(a);
     if ((e = cudaGetLastError()) != cudaSuccess) return e;
     if ((e = launch_qk<D, G, true>(a, st)) != cudaSuccess) return e;
-    tau_pv_kernel<D, false><<<a.B * a.Hq, TAU_THREADS, 0, st>>>(a);
+    tau_pv_kernel<D, false><<<a.B * a.Hq, TAU_THREADS, 0, st>>>(a, 1);
     if ((e = cudaGetLastError()) != cudaSuccess) return e;
     using RG = Ring<D, G, 4, 1>;
     auto k = pv_stream_kernel<D, G>;
@@ -1123,25 +1108,21 @@ size_t decode_ws_bytes(bool dense, int B, int Hq, int Hkv, int d, int P, int max
     };
     const size_t tokens = (size_t)B * Hq * max_pages * P;
     const size_t o_union = take(dense ? 0 : (size_t)B * Hkv * max_pages * 4);
+    const size_t o_ublk = take(dense ? 0 : (size_t)B * Hkv * max_pages * 4);
     const size_t o_ucnt = take((size_t)B * Hkv * 4);
     const size_t o_zmax = take((size_t)B * Hq * 4);
     const size_t o_tau = take((size_t)B * Hq * 4);
     const size_t o_cnt = take((size_t)B * Hkv * 4);
-    const size_t o_ccnt = take((size_t)B * Hq * 4);
-    const size_t o_cand = take(tokens * 8);
-    const size_t o_lpos = take(tokens * 4);
     const size_t o_part = take(dense ? (size_t)MAX_SPLITS * B * Hq * (d + 2) * 4 : 0);
-    const size_t o_z = take(dense ? tokens * 4 : 0);
+    const size_t o_z = take(tokens * 4);
     if (carve && base) {
         char *p = static_cast<char *>(base);
         carve->union_e = reinterpret_cast<int *>(p + o_union);
+        carve->union_blk = reinterpret_cast<int *>(p + o_ublk);
         carve->union_cnt = reinterpret_cast<int *>(p + o_ucnt);
         carve->zmax = reinterpret_cast<int *>(p + o_zmax);
         carve->tau = reinterpret_cast<float *>(p + o_tau);
         carve->counters = reinterpret_cast<int *>(p + o_cnt);
-        carve->cand_cnt = reinterpret_cast<int *>(p + o_ccnt);
-        carve->cand = reinterpret_cast<int2 *>(p + o_cand);
-        carve->cand_lpos = reinterpret_cast<int *>(p + o_lpos);
         carve->partial = reinterpret_cast<float *>(p + o_part);
         carve->zbuf = reinterpret_cast<float *>(p + o_z);
     }

@@ -54,20 +54,16 @@ struct SelectArgs {
 };
 cudaError_t launch_select(const SelectArgs &a, cudaStream_t st);
 
-// Workspace carve-up shared by the decode paths.  A candidate is a token
-// whose z exceeded (running max of z seen so far) - 1 when it was scored: a
-// superset of the tokens that can carry weight, since tau >= max z - 1.
+// Workspace carve-up shared by the decode paths.
 struct DecodeWs {
     int *union_e;    // [B*Hkv][max_pages]   (page << 8) | head mask (sparse)
+    int *union_blk;  // [B*Hkv][max_pages]   physical block of each union entry (sparse)
     int *union_cnt;  // [B*Hkv]
     int *zmax;       // [B*Hq] order-mapped max z
     float *tau;      // [B*Hq]
     int *counters;   // [B*Hkv] last-CTA combine counters
-    int *cand_cnt;   // [B*Hq]
-    int2 *cand;      // [B*Hq][max_pages*P]  (z bits, value row index)
-    int *cand_lpos;  // [B*Hq][max_pages*P]  logical token position (only with p_out)
     float *partial;  // [MAX_SPLITS][B*Hq][d+2]  (dense paths)
-    float *zbuf;     // [B*Hq][max_pages*P]      (dense entmax path)
+    float *zbuf;     // [B*Hq][max_pages*P]  z of every token of the page list, in list order
 };
 
 struct DecodeArgs {

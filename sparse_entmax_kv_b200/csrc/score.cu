@@ -4,10 +4,12 @@
 //   bbox  = (sum_j max(q_j kmin_j, q_j kmax_j)) / sqrt(d)   upper bound on s
 //   mu    = (sum_j q_j mean_j) / sqrt(d)                    Gaussian mean
 //   sigma = sqrt((sum_j q_j^2 var_j) / d)                   Gaussian std
-// Each sum is one fp64 chain over j in index order; every product is exact in
-// fp64, so the chain is reproducible to the bit.  max(q a, q b) with a <= b is
-// q*b for q >= 0 and q*a otherwise, which turns the bound into one fused
-// multiply-add per coordinate.
+// The bound is one fp64 chain over j in index order with exact products, so
+// it is reproducible to the bit.  With q+ = max(q, 0) and q- = min(q, 0),
+// max(q a, q b) (a <= b) equals q+ b + q- a with one of the two terms an exact
+// zero, so two fused multiply-adds per coordinate give the same chain with no
+// selects.  mu and sigma feed only the approximate tau_hat; they are fp32
+// chains over j in index order.
 //
 // Layout of the work: a CTA owns 256 consecutive logical pages of one
 // (b, kv head); thread = page, and the thread scores that page for all G query
@@ -17,7 +19,9 @@
 // (consecutive lanes take consecutive 16-byte pieces of a record, so whole
 // 32-byte sectors move per instruction) into padded per-thread slots, and each
 // thread then reads its own slot.  The slot pitch keeps the 16-byte reads of
-// any 8 consecutive lanes on distinct banks.
+// any 8 consecutive lanes on distinct banks.  q is kept in shared memory
+// coordinate-major ([j][head]) so one vector load serves all heads of a
+// coordinate.
 #include "common.cuh"
 #include "internal.h"
 
@@ -37,14 +41,24 @@ struct ScoreCfg {
     static constexpr int WARP_STAGE = 32 * SLOT;
 };
 
+template <int D, int G>
+struct QLayout {
+    // qpn: [D][G][2] fp64 (q+, q-); qf, qqf: [D][G] fp32 (q, q^2)
+    static constexpr int PN_BYTES = D * G * 2 * 8;
+    static constexpr int F_BYTES = D * G * 4;
+    static constexpr int BYTES = PN_BYTES + 2 * F_BYTES;
+};
+
 template <int D, int G, bool GAUSS>
 __global__ void __launch_bounds__(SC_THREADS, 2) score_kernel(ScoreArgs a) {
     using Cfg = ScoreCfg<GAUSS>;
+    using QL = QLayout<D, G>;
     constexpr int NCH = D / CH;
     extern __shared__ __align__(16) unsigned char smem[];
-    double *qd = reinterpret_cast<double *>(smem);   // [G][D]
-    double *qq = qd + G * D;                          // [G][D] (GAUSS)
-    unsigned char *ring = smem + (GAUSS ? 2 : 1) * G * D * sizeof(double);
+    double *qpn = reinterpret_cast<double *>(smem);
+    float *qf = reinterpret_cast<float *>(smem + QL::PN_BYTES);
+    float *qqf = qf + D * G;
+    unsigned char *ring = smem + QL::BYTES;
 
     const int bk = blockIdx.y;
     const int b = bk / a.Hkv, kvh = bk % a.Hkv;
@@ -52,9 +66,11 @@ __global__ void __launch_bounds__(SC_THREADS, 2) score_kernel(ScoreArgs a) {
 
     for (int i = threadIdx.x; i < G * D; i += SC_THREADS) {
         const int g = i / D, j = i % D;
-        double v = (double)bf16f(a.q[((size_t)b * a.Hq + kvh * G + g) * D + j]);
-        qd[i] = v;
-        if (GAUSS) qq[i] = v * v;
+        const float v = bf16f(a.q[((size_t)b * a.Hq + kvh * G + g) * D + j]);
+        qpn[(j * G + g) * 2] = v > 0.f ? (double)v : 0.0;
+        qpn[(j * G + g) * 2 + 1] = v < 0.f ? (double)v : 0.0;
+        qf[j * G + g] = v;
+        qqf[j * G + g] = v * v;  // exact: bf16 squared fits in fp32
     }
     __syncthreads();
 
@@ -112,9 +128,13 @@ __global__ void __launch_bounds__(SC_THREADS, 2) score_kernel(ScoreArgs a) {
         cp_async_commit();
     }
 
-    double ab[G], am[G], av[G];
+    double ab[G];
+    float am[G], av[G];
 #pragma unroll
-    for (int g = 0; g < G; ++g) ab[g] = am[g] = av[g] = 0.0;
+    for (int g = 0; g < G; ++g) {
+        ab[g] = 0.0;
+        am[g] = av[g] = 0.f;
+    }
 
     const unsigned char *myslot0 = wring + lane * Cfg::SLOT;
     for (int c = 0; c < NCH; ++c) {
@@ -140,22 +160,22 @@ __global__ void __launch_bounds__(SC_THREADS, 2) score_kernel(ScoreArgs a) {
                 vv[4 * i] = v4.x; vv[4 * i + 1] = v4.y; vv[4 * i + 2] = v4.z; vv[4 * i + 3] = v4.w;
             }
         }
-        const double *qc = qd + c * CH;
-        const double *qqc = qq + c * CH;
+        const double *qpc = qpn + (size_t)c * CH * G * 2;
+        const float *qfc = qf + c * CH * G;
+        const float *qqc = qqf + c * CH * G;
 #pragma unroll
         for (int jj = 0; jj < CH; ++jj) {
             const unsigned w_n = wn[jj >> 1], w_x = wx[jj >> 1];
             const double lo = (double)((jj & 1) ? bf16hi(w_n) : bf16lo(w_n));
             const double hi = (double)((jj & 1) ? bf16hi(w_x) : bf16lo(w_x));
-            double md = 0.0, vd = 0.0;
-            if (GAUSS) { md = (double)mv[jj]; vd = (double)vv[jj]; }
 #pragma unroll
             for (int g = 0; g < G; ++g) {
-                const double qv = qc[g * D + jj];
-                ab[g] = __fma_rn(qv, (__double2hiint(qv) < 0) ? lo : hi, ab[g]);
+                const double2 pn = *reinterpret_cast<const double2 *>(qpc + (jj * G + g) * 2);
+                ab[g] = __fma_rn(pn.x, hi, ab[g]);  // q+ * kmax (zero when q < 0)
+                ab[g] = __fma_rn(pn.y, lo, ab[g]);  // q- * kmin (zero when q >= 0)
                 if (GAUSS) {
-                    am[g] = __fma_rn(qv, md, am[g]);
-                    av[g] = __fma_rn(qqc[g * D + jj], vd, av[g]);
+                    am[g] = __fmaf_rn(qfc[jj * G + g], mv[jj], am[g]);
+                    av[g] = __fmaf_rn(qqc[jj * G + g], vv[jj], av[g]);
                 }
             }
         }
@@ -165,13 +185,14 @@ __global__ void __launch_bounds__(SC_THREADS, 2) score_kernel(ScoreArgs a) {
 
     if (rec < 0) return;
     const double inv_sqrt_d = __ddiv_rn(1.0, __dsqrt_rn((double)D));
+    const float inv_sqrt_df = D == 64 ? 0.125f : 0.08838834764831845f;
 #pragma unroll
     for (int g = 0; g < G; ++g) {
         const size_t o = ((size_t)b * a.Hq + kvh * G + g) * a.max_pages + page;
         a.bbox[o] = (float)__dmul_rn(ab[g], inv_sqrt_d);
         if (GAUSS) {
-            a.mu[o] = (float)__dmul_rn(am[g], inv_sqrt_d);
-            a.sigma[o] = (float)__dsqrt_rn(__ddiv_rn(av[g], (double)D));
+            a.mu[o] = am[g] * inv_sqrt_df;
+            a.sigma[o] = sqrtf(av[g] * (1.f / (float)D));
         }
     }
 }
@@ -179,7 +200,7 @@ __global__ void __launch_bounds__(SC_THREADS, 2) score_kernel(ScoreArgs a) {
 template <int D, int G, bool GAUSS>
 cudaError_t launch_t(const ScoreArgs &a, cudaStream_t st) {
     using Cfg = ScoreCfg<GAUSS>;
-    const size_t smem = (GAUSS ? 2 : 1) * G * D * sizeof(double) + (size_t)SC_WARPS * Cfg::NST * Cfg::WARP_STAGE;
+    const size_t smem = QLayout<D, G>::BYTES + (size_t)SC_WARPS * Cfg::NST * Cfg::WARP_STAGE;
     auto kern = score_kernel<D, G, GAUSS>;
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e != cudaSuccess) return e;

@@ -48,7 +48,7 @@ def test_sizes():
     assert nv.meta_bytes(s) == 128 * 2 * 12 * 128
     assert nv.workspace_size(s, nv.CALL_SELECT) == 0
     ws = nv.workspace_size(s, nv.CALL_DECODE_SPARSE)
-    assert ws >= 2 * 8 * 64 * 32 * 8            # the candidate lists alone
+    assert ws >= 2 * 8 * 64 * 32 * 4            # z of every token of the page list
     assert nv.workspace_size(s, nv.CALL_DECODE_DENSE) > ws
     assert nv.workspace_size(s, 99) == (1 << 64) - 1
     assert nv.meta_bytes(shp(d=96)) == 0
