@@ -559,69 +559,118 @@ __global__ void __launch_bounds__(TAU_THREADS) tau_pv_kernel(const __grid_consta
     }
     if (!GATHER) return;
 
-    // p v over the support: each warp takes its share of the candidates with
-    // z > tau, up to eight value rows in flight at a time.  Sums run in fp64
-    // (p v is exact there).
+    // p v over the support.  On chip: the support (z > tau) is first compacted
+    // in list order, then dealt round-robin to the warps, eight rows at a time
+    // per warp with all their loads in flight.  Off chip: each warp scans its
+    // share of the z row.  Sums run in fp64 (p v is exact there).
     double acc[CPL];
 #pragma unroll
     for (int c = 0; c < CPL; ++c) acc[c] = 0.0;
     const size_t lstride = (size_t)a.max_pages * P;
-    for (int c0 = warp * 32; c0 < nloop; c0 += TAU_WARPS * 32) {
-        const int c = c0 + lane;
-        const float z = c < nloop ? cz_at(c) : -INFINITY;
-        const int pos = c < nloop ? (onchip ? cpos[c] : c) : 0;
-        const float p = pos_pow(z - tau, r, ri);
-        unsigned bal = __ballot_sync(FULL, p > 0.f);
-        int row = 0;
-        if (p > 0.f) {
-            const int up = pos / P, t = pos - up * P;
-            const int blk = dense ? __ldg(a.page_table + (size_t)b * a.max_pages + up)
-                                  : __ldcg(a.ws.union_blk + (size_t)bk * a.max_pages + up);
-            row = (blk * a.Hkv + kvh) * P + t;
-            if (a.p_out) {
-                const int page = dense ? up : (__ldcg(a.ws.union_e + (size_t)bk * a.max_pages + up) >> 8);
-                a.p_out[(size_t)bh * lstride + (size_t)page * P + t] = p;
+    auto row_of = [&](int pos, float p) -> int {
+        const int up = pos / P, t = pos - up * P;
+        const int blk = dense ? __ldg(a.page_table + (size_t)b * a.max_pages + up)
+                              : __ldcg(a.ws.union_blk + (size_t)bk * a.max_pages + up);
+        if (a.p_out) {
+            const int page = dense ? up : (__ldcg(a.ws.union_e + (size_t)bk * a.max_pages + up) >> 8);
+            a.p_out[(size_t)bh * lstride + (size_t)page * P + t] = p;
+        }
+        return (blk * a.Hkv + kvh) * P + t;
+    };
+    auto gather8 = [&](int nr, int row, float p) {
+        // lanes 0..nr-1 hold (row, p) of up to eight support tokens
+        float vv[8][CPL], pp[8];
+#pragma unroll
+        for (int i = 0; i < 8; ++i) {
+            const int rw = __shfl_sync(FULL, row, i);
+            pp[i] = i < nr ? __shfl_sync(FULL, p, i) : 0.f;
+            if (i < nr) {
+                const uint16_t *vr = a.v + (size_t)rw * D + lane * CPL;
+                if (CPL == 4) {
+                    const uint2 w = __ldg(reinterpret_cast<const uint2 *>(vr));
+                    vv[i][0] = bf16lo(w.x);
+                    vv[i][1] = bf16hi(w.x);
+                    vv[i][2] = bf16lo(w.y);
+                    vv[i][3] = bf16hi(w.y);
+                } else {
+                    const unsigned w = __ldg(reinterpret_cast<const unsigned *>(vr));
+                    vv[i][0] = bf16lo(w);
+                    vv[i][1] = bf16hi(w);
+                }
+            } else {
+#pragma unroll
+                for (int cc = 0; cc < CPL; ++cc) vv[i][cc] = 0.f;
             }
         }
-        while (bal) {
-            int src[8];
-            int nr = 0;
 #pragma unroll
-            for (int i = 0; i < 8; ++i) {
-                src[i] = 0;
-                if (bal) {
-                    src[i] = __ffs(bal) - 1;
-                    bal &= bal - 1;
-                    nr = i + 1;
-                }
+        for (int i = 0; i < 8; ++i)
+#pragma unroll
+            for (int cc = 0; cc < CPL; ++cc) acc[cc] = fma((double)pp[i], (double)vv[i][cc], acc[cc]);
+    };
+    if (onchip) {
+        // in-place ordered compaction of the support: p overwrites z, position kept
+        constexpr int PER = ZCAP / TAU_THREADS;
+        const int per = ceil_div(nc, TAU_THREADS);
+        const int c0 = threadIdx.x * per;
+        float pz[PER];
+        int pp_[PER];
+        unsigned bits = 0;
+#pragma unroll
+        for (int k = 0; k < PER; ++k) {
+            pz[k] = 0.f;
+            pp_[k] = 0;
+            if (k < per && c0 + k < nc) {
+                pz[k] = pos_pow(cz[c0 + k] - tau, r, ri);
+                pp_[k] = cpos[c0 + k];
+                if (pz[k] > 0.f) bits |= 1u << k;
             }
-            float vv[8][CPL], pp[8];
+        }
+        int ns;
+        int w = block_excl_scan(__popc(bits), sh, &ns);
+        __syncthreads();
 #pragma unroll
-            for (int i = 0; i < 8; ++i) {
-                const int rw = __shfl_sync(FULL, row, src[i]);
-                pp[i] = i < nr ? __shfl_sync(FULL, p, src[i]) : 0.f;
-                if (i < nr) {
-                    const uint16_t *vr = a.v + (size_t)rw * D + lane * CPL;
-                    if (CPL == 4) {
-                        const uint2 w = __ldg(reinterpret_cast<const uint2 *>(vr));
-                        vv[i][0] = bf16lo(w.x);
-                        vv[i][1] = bf16hi(w.x);
-                        vv[i][2] = bf16lo(w.y);
-                        vv[i][3] = bf16hi(w.y);
-                    } else {
-                        const unsigned w = __ldg(reinterpret_cast<const unsigned *>(vr));
-                        vv[i][0] = bf16lo(w);
-                        vv[i][1] = bf16hi(w);
+        for (int k = 0; k < PER; ++k)
+            if (bits & (1u << k)) {
+                cz[w] = pz[k];
+                cpos[w] = pp_[k];
+                ++w;
+            }
+        __syncthreads();
+        const int mine = ns > warp ? ceil_div(ns - warp, TAU_WARPS) : 0;  // tokens warp, warp+16, ...
+        for (int base = 0; base < mine; base += 8) {
+            const int nr = min(8, mine - base);
+            int row = 0;
+            float p = 0.f;
+            if (lane < nr) {
+                const int i = warp + TAU_WARPS * (base + lane);
+                p = cz[i];
+                row = row_of(cpos[i], p);
+            }
+            gather8(nr, row, p);
+        }
+    } else {
+        for (int c0 = warp * 32; c0 < nloop; c0 += TAU_WARPS * 32) {
+            const int c = c0 + lane;
+            const float z = c < nloop ? cz_at(c) : -INFINITY;
+            const float p = pos_pow(z - tau, r, ri);
+            unsigned bal = __ballot_sync(FULL, p > 0.f);
+            while (bal) {
+                // the next (up to) eight lanes with weight move to lanes 0..7
+                int src = 0, nr = 0;
+#pragma unroll
+                for (int i = 0; i < 8; ++i)
+                    if (bal) {
+                        const int l = __ffs(bal) - 1;
+                        bal &= bal - 1;
+                        if (lane == i) src = l;
+                        nr = i + 1;
                     }
-                } else {
-#pragma unroll
-                    for (int cc = 0; cc < CPL; ++cc) vv[i][cc] = 0.f;
-                }
+                const int cc = c0 + __shfl_sync(FULL, lane, src);
+                const float pl = __shfl_sync(FULL, p, src);
+                int row = 0;
+                if (lane < nr) row = row_of(cc, pl);
+                gather8(nr, row, lane < nr ? pl : 0.f);
             }
-#pragma unroll
-            for (int i = 0; i < 8; ++i)
-#pragma unroll
-                for (int cc = 0; cc < CPL; ++cc) acc[cc] = fma((double)pp[i], (double)vv[i][cc], acc[cc]);
         }
     }
     __syncthreads();  // every warp is done with the candidates

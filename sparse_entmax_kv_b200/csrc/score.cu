@@ -14,7 +14,7 @@
 // Layout of the work: a CTA owns 256 consecutive logical pages of one
 // (b, kv head); thread = page, and the thread scores that page for all G query
 // heads of the group, so each metadata record crosses HBM once per group.
-// Records are streamed through a per-warp ring of 16-coordinate chunks with
+// Records are streamed through a per-warp ring of 8-coordinate chunks with
 // 16-byte cp.async copies: the 32 records of a warp are fetched cooperatively
 // (consecutive lanes take consecutive 16-byte pieces of a record, so whole
 // 32-byte sectors move per instruction) into padded per-thread slots, and each
@@ -31,13 +31,13 @@ namespace {
 
 constexpr int SC_THREADS = 256;
 constexpr int SC_WARPS = SC_THREADS / 32;
-constexpr int CH = 16;  // coordinates per chunk
+constexpr int CH = 8;  // coordinates per chunk
 
 template <bool GAUSS>
 struct ScoreCfg {
-    static constexpr int PIECES = GAUSS ? 12 : 4;  // 16-byte pieces per record chunk
+    static constexpr int PIECES = GAUSS ? 6 : 2;   // 16-byte pieces per record chunk
     static constexpr int SLOT = PIECES * 16 + 16;  // padded slot pitch (bytes)
-    static constexpr int NST = GAUSS ? 2 : 4;      // ring depth (chunks in flight per warp)
+    static constexpr int NST = GAUSS ? 3 : 6;      // ring depth (chunks in flight per warp)
     static constexpr int WARP_STAGE = 32 * SLOT;
 };
 
@@ -88,10 +88,10 @@ __global__ void __launch_bounds__(SC_THREADS, 2) score_kernel(ScoreArgs a) {
             atomicOr(a.status, ENTMAXKV_STATUS_BAD_PAGE);
     }
 
-    // Piece i*32+lane of a chunk belongs to record (i*32+lane)/PIECES.  Pieces
-    // 0-1 are kmin, 2-3 kmax (bound region: kmin at [0,2D) bytes of the record,
-    // kmax at [2D,4D), chunk c adds 32c); pieces 4-7 are mean, 8-11 var
-    // (moment region: mean at [0,4D), var at [4D,8D), chunk c adds 64c).
+    // Piece i*32+lane of a chunk belongs to record (i*32+lane)/PIECES.  Piece
+    // 0 is kmin, 1 kmax (bound region: kmin at [0,2D) bytes of the record,
+    // kmax at [2D,4D), chunk c adds 16c); pieces 2-3 are mean, 4-5 var
+    // (moment region: mean at [0,4D), var at [4D,8D), chunk c adds 32c).
     const unsigned char *src[Cfg::PIECES];
     int dst_off[Cfg::PIECES];
 #pragma unroll
@@ -102,11 +102,11 @@ __global__ void __launch_bounds__(SC_THREADS, 2) score_kernel(ScoreArgs a) {
         dst_off[i] = rl * Cfg::SLOT + pc * 16;
         if (r < 0) {
             src[i] = nullptr;
-        } else if (pc < 4) {
-            src[i] = a.meta + (size_t)r * 4 * D + (pc < 2 ? pc * 16 : 2 * D + (pc - 2) * 16);
+        } else if (pc < 2) {
+            src[i] = a.meta + (size_t)r * 4 * D + pc * 2 * D;
         } else {
             src[i] = a.meta + (size_t)a.R * 4 * D + (size_t)r * 8 * D +
-                     (pc < 8 ? (pc - 4) * 16 : 4 * D + (pc - 8) * 16);
+                     (pc < 4 ? (pc - 2) * 16 : 4 * D + (pc - 4) * 16);
         }
     }
 
@@ -116,8 +116,8 @@ __global__ void __launch_bounds__(SC_THREADS, 2) score_kernel(ScoreArgs a) {
 #pragma unroll
         for (int i = 0; i < Cfg::PIECES; ++i) {
             if (src[i] == nullptr) continue;
-            // bound pieces sit in the first 64 bytes of the slot
-            const int cstride = dst_off[i] % Cfg::SLOT < 64 ? 32 : 64;
+            // bound pieces sit in the first 32 bytes of the slot
+            const int cstride = dst_off[i] % Cfg::SLOT < 32 ? 16 : 32;
             cp_async16(st + dst_off[i], src[i] + c * cstride);
         }
     };
@@ -143,19 +143,16 @@ __global__ void __launch_bounds__(SC_THREADS, 2) score_kernel(ScoreArgs a) {
         cp_async_wait<Cfg::NST - 1>();
         __syncwarp();
         const unsigned char *slot = myslot0 + (c % Cfg::NST) * Cfg::WARP_STAGE;
-        uint4 kn[2], kx[2];
-        kn[0] = *reinterpret_cast<const uint4 *>(slot + 0);
-        kn[1] = *reinterpret_cast<const uint4 *>(slot + 16);
-        kx[0] = *reinterpret_cast<const uint4 *>(slot + 32);
-        kx[1] = *reinterpret_cast<const uint4 *>(slot + 48);
-        const unsigned *wn = reinterpret_cast<const unsigned *>(kn);
-        const unsigned *wx = reinterpret_cast<const unsigned *>(kx);
+        const uint4 kn = *reinterpret_cast<const uint4 *>(slot + 0);
+        const uint4 kx = *reinterpret_cast<const uint4 *>(slot + 16);
+        const unsigned wn[4] = {kn.x, kn.y, kn.z, kn.w};
+        const unsigned wx[4] = {kx.x, kx.y, kx.z, kx.w};
         float mv[CH], vv[CH];
         if (GAUSS) {
 #pragma unroll
-            for (int i = 0; i < 4; ++i) {
-                float4 m4 = *reinterpret_cast<const float4 *>(slot + 64 + 16 * i);
-                float4 v4 = *reinterpret_cast<const float4 *>(slot + 128 + 16 * i);
+            for (int i = 0; i < 2; ++i) {
+                float4 m4 = *reinterpret_cast<const float4 *>(slot + 32 + 16 * i);
+                float4 v4 = *reinterpret_cast<const float4 *>(slot + 64 + 16 * i);
                 mv[4 * i] = m4.x; mv[4 * i + 1] = m4.y; mv[4 * i + 2] = m4.z; mv[4 * i + 3] = m4.w;
                 vv[4 * i] = v4.x; vv[4 * i + 1] = v4.y; vv[4 * i + 2] = v4.z; vv[4 * i + 3] = v4.w;
             }
