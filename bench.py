@@ -41,7 +41,11 @@ PAPER_CONTEXT = {"speedup_vs_full_softmax_flashdecoding": 3.36, "speedup_vs_full
 
 # DRAM bytes per launch from ncu captures (dram__bytes_read.sum + dram__bytes_write.sum),
 # keyed by kernel and workload, valid only while the kernel source is unchanged.
-NCU_TRAFFIC = {}
+NCU_TRAFFIC = {
+    # captured at L=524,288 (100.73 MB read + 5.94 MB written per launch), scaled by 2 for the
+    # 1,048,576-token context: the scan is linear in the page count (profiles/step_kernels_*)
+    "score_pages/gauss_gqa_L1m": {"bytes": 2 * (100726016 + 5942016), "src": "761bf1cf5895"},
+}
 
 
 def _src_hash(fname):
@@ -295,7 +299,7 @@ def run_gpu(args, rank, world):
         src = "decode.cu"
     achieved = alg / (stage_us[dom] * 1e-6) / 1e9
     tr = NCU_TRAFFIC.get(f"{dom}/{args.workload}")
-    traffic = tr["bytes"] if tr and tr.get("src") == _src_hash(src) else None
+    traffic = tr["bytes"] if tr and tr.get("src") == _src_hash(src) else None  # null once the kernel changed
     roofline = {"bound": "hbm", "kernel": dom, "achieved": round(achieved, 1), "peak": peak, "unit": "GB/s",
                 "frac": round(achieved / peak, 4), "traffic": traffic, "algorithmic_bytes": alg,
                 "peak_kind": f"{peak_kind} copy bandwidth (burst)"}
