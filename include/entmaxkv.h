@@ -81,8 +81,13 @@ enum {
     ENTMAXKV_ERR_WORKSPACE = -5,   /* workspace missing or smaller than required */
     ENTMAXKV_ERR_CUDA = -6,        /* CUDA runtime/driver error */
     ENTMAXKV_ERR_UNSUPPORTED = -7, /* valid but not implemented (e.g. non-integer r) */
-    ENTMAXKV_ERR_ALIGN = -8        /* pointer not 16-byte aligned */
+    ENTMAXKV_ERR_ALIGN = -8,       /* pointer not 16-byte aligned */
+    ENTMAXKV_ERR_TOO_LARGE = -9    /* problem needs more than the fixed scratch of
+                                      entmaxkv_decode_sparse_static */
 };
+
+/* Size of the fixed on-device scratch used by entmaxkv_decode_sparse_static. */
+#define ENTMAXKV_STATIC_SCRATCH_BYTES ((size_t)16 << 20)
 
 enum { ENTMAXKV_TOPK = 0, ENTMAXKV_GAUSS = 1 };
 
@@ -215,6 +220,35 @@ ENTMAXKV_API int entmaxkv_decode_sparse(const entmaxkv_shape *shape, const void 
                            const int32_t *sel, const int32_t *cnt, float alpha,
                            float *out, float *tau_out, float *p_out,
                            void *workspace, size_t ws_bytes, void *stream);
+
+/*
+ * Allocation-free form of entmaxkv_decode_sparse (the EntmaxKV summary has no
+ * counterpart; this is a library convenience).  Same arguments, results and
+ * errors, minus the workspace: the scratch lives in a fixed array of
+ * ENTMAXKV_STATIC_SCRATCH_BYTES (16 MiB) of device memory that the library
+ * declares at file scope, so every GPU that loads the library holds it until
+ * the process exits.  Meant for callers that cannot call cudaMalloc at decode
+ * time -- for instance code that runs inside a memory pool or graph-building
+ * framework that forbids allocation, or an embedding host whose allocator
+ * owns all device memory.  The call itself allocates nothing.
+ * - Problems whose entmaxkv_workspace_size(.., ENTMAXKV_CALL_DECODE_SPARSE)
+ *   exceeds ENTMAXKV_STATIC_SCRATCH_BYTES return ENTMAXKV_ERR_TOO_LARGE (about
+ *   four million (query head, context token) pairs fit).
+ * - The first call on each device looks up the array's device address
+ *   (cudaGetSymbolAddress) with that device current; make that first call
+ *   before any stream capture.
+ * - All calls on a device share the one array, which keeps the last call's
+ *   contents (every kernel initialises what it reads, so nothing needs to be
+ *   cleared between calls).  Calls that may overlap on the GPU -- different
+ *   streams without ordering, or two host threads -- race on it; serialise
+ *   them.
+ */
+ENTMAXKV_API int entmaxkv_decode_sparse_static(const entmaxkv_shape *shape, const void *q,
+                                  const void *k_cache, const void *v_cache,
+                                  const int32_t *page_table, const int32_t *seq_lens,
+                                  const int32_t *sel, const int32_t *cnt, float alpha,
+                                  float *out, float *tau_out, float *p_out,
+                                  void *stream);
 
 /*
  * Section 4 comparison paths, over every token of every sequence:

@@ -110,6 +110,8 @@ const char *entmaxkv_strerror(int code) {
         case ENTMAXKV_ERR_CUDA: return "CUDA runtime or driver error";
         case ENTMAXKV_ERR_UNSUPPORTED: return "valid arguments that this build does not support";
         case ENTMAXKV_ERR_ALIGN: return "pointer not 16-byte aligned";
+        case ENTMAXKV_ERR_TOO_LARGE:
+            return "problem needs more scratch than the fixed array of entmaxkv_decode_sparse_static";
         default: return "unknown error code";
     }
 }
@@ -319,3 +321,49 @@ int entmaxkv_decode_dense(const entmaxkv_shape *s, const void *q, const void *k_
 }
 
 }  // extern "C"
+
+// ------------------------------------------------ allocation-free decode
+//
+// entmaxkv_decode_sparse_static: the sparse decode with its scratch in a
+// fixed file-scope device array instead of a caller-provided workspace, for
+// callers that cannot allocate device memory at decode time.  In host code
+// g_static_scratch names a host-side stand-in, not device memory, so the
+// device address is looked up once per device (with that device current) and
+// that pointer is what the kernels receive.
+namespace {
+
+__device__ __align__(256) unsigned char g_static_scratch[ENTMAXKV_STATIC_SCRATCH_BYTES];
+
+void *g_static_ptr[MAX_DEV];
+bool g_static_ok[MAX_DEV];
+
+int static_scratch(void **out) {
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= MAX_DEV) return ENTMAXKV_ERR_CUDA;
+    std::lock_guard<std::mutex> lk(g_mu);
+    if (!g_static_ok[dev]) {
+        void *p = nullptr;
+        if (cudaGetSymbolAddress(&p, g_static_scratch) != cudaSuccess || p == nullptr) return ENTMAXKV_ERR_CUDA;
+        g_static_ptr[dev] = p;
+        g_static_ok[dev] = true;
+    }
+    *out = g_static_ptr[dev];
+    return ENTMAXKV_OK;
+}
+
+}  // namespace
+
+extern "C" int entmaxkv_decode_sparse_static(const entmaxkv_shape *s, const void *q, const void *k_cache,
+                                             const void *v_cache, const int32_t *page_table,
+                                             const int32_t *seq_lens, const int32_t *sel, const int32_t *cnt,
+                                             float alpha, float *out, float *tau_out, float *p_out, void *stream) {
+    int rc = check_shape(s);
+    if (rc) return rc;
+    const size_t need =
+        decode_ws_bytes(false, s->B, s->Hq, s->Hkv, s->d, s->page_size, s->max_pages, nullptr, nullptr);
+    if (need > ENTMAXKV_STATIC_SCRATCH_BYTES) return ENTMAXKV_ERR_TOO_LARGE;
+    void *ws = nullptr;
+    if ((rc = static_scratch(&ws))) return rc;
+    return entmaxkv_decode_sparse(s, q, k_cache, v_cache, page_table, seq_lens, sel, cnt, alpha, out, tau_out,
+                                  p_out, ws, ENTMAXKV_STATIC_SCRATCH_BYTES, stream);
+}

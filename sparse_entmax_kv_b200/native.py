@@ -19,7 +19,8 @@ LIB_PATH = os.path.join(_HERE, "libentmaxkv.so")
 
 OK = 0
 ERR = {0: "OK", -1: "ERR_NULL", -2: "ERR_SHAPE", -3: "ERR_ALPHA", -4: "ERR_POLICY",
-       -5: "ERR_WORKSPACE", -6: "ERR_CUDA", -7: "ERR_UNSUPPORTED", -8: "ERR_ALIGN"}
+       -5: "ERR_WORKSPACE", -6: "ERR_CUDA", -7: "ERR_UNSUPPORTED", -8: "ERR_ALIGN", -9: "ERR_TOO_LARGE"}
+STATIC_SCRATCH_BYTES = 16 << 20
 TOPK, GAUSS = 0, 1
 CALL_SELECT, CALL_DECODE_SPARSE, CALL_DECODE_DENSE = 2, 3, 4
 STATUS_BAD_PAGE, STATUS_BAD_SELECTION, STATUS_TIMEOUT, STATUS_OVERFLOW = 1, 2, 4, 8
@@ -27,7 +28,7 @@ STATUS_BAD_PAGE, STATUS_BAD_SELECTION, STATUS_TIMEOUT, STATUS_OVERFLOW = 1, 2, 4
 EXPORTED = ("entmaxkv_strerror", "entmaxkv_version", "entmaxkv_meta_bytes",
             "entmaxkv_workspace_size", "entmaxkv_get_status", "entmaxkv_build_meta",
             "entmaxkv_score_pages", "entmaxkv_select", "entmaxkv_decode_sparse",
-            "entmaxkv_decode_dense")
+            "entmaxkv_decode_sparse_static", "entmaxkv_decode_dense")
 
 
 class EntmaxKVError(RuntimeError):
@@ -77,6 +78,7 @@ def lib():
         L.entmaxkv_select.argtypes = [sp, vp, vp, vp, vp, i32, i32, f32, f32, vp, vp, vp, vp, sz, vp]
         L.entmaxkv_decode_sparse.argtypes = [sp, vp, vp, vp, vp, vp, vp, vp, f32, vp, vp, vp, vp, sz, vp]
         L.entmaxkv_decode_dense.argtypes = [sp, vp, vp, vp, vp, vp, f32, vp, vp, vp, vp, sz, vp]
+        L.entmaxkv_decode_sparse_static.argtypes = [sp, vp, vp, vp, vp, vp, vp, vp, f32, vp, vp, vp, vp]
         for fn in EXPORTED:
             if fn not in ("entmaxkv_strerror", "entmaxkv_version", "entmaxkv_meta_bytes",
                           "entmaxkv_workspace_size"):
@@ -180,3 +182,14 @@ def entmaxkv_decode_dense(shape, q, k_cache, v_cache, page_table, seq_lens, alph
         _ptr(seq_lens, torch.int32, "seq_lens"), float(alpha), _ptr(out, torch.float32, "out"),
         _ptr(tau_out, torch.float32, "tau_out"), _ptr(p_out, torch.float32, "p_out"),
         _ptr(workspace, None, "workspace"), 0 if workspace is None else workspace.numel(), _stream(stream)))
+
+
+def entmaxkv_decode_sparse_static(shape, q, k_cache, v_cache, page_table, seq_lens, sel, cnt, alpha, out,
+                                  tau_out=None, p_out=None, stream=None):
+    """entmaxkv_decode_sparse with the library's fixed on-device scratch instead of a workspace."""
+    _check("entmaxkv_decode_sparse_static", lib().entmaxkv_decode_sparse_static(
+        C.byref(shape), _ptr(q, torch.bfloat16, "q"), _ptr(k_cache, torch.bfloat16, "k_cache"),
+        _ptr(v_cache, torch.bfloat16, "v_cache"), _ptr(page_table, torch.int32, "page_table"),
+        _ptr(seq_lens, torch.int32, "seq_lens"), _ptr(sel, torch.int32, "sel"), _ptr(cnt, torch.int32, "cnt"),
+        float(alpha), _ptr(out, torch.float32, "out"), _ptr(tau_out, torch.float32, "tau_out"),
+        _ptr(p_out, torch.float32, "p_out"), _stream(stream)))

@@ -24,7 +24,7 @@ def _declared():
 def test_library_exports_every_declared_symbol():
     L = nv.lib()
     names = _declared()
-    assert len(names) == 10
+    assert len(names) == 11
     assert set(names) == set(nv.EXPORTED)
     for n in names:
         assert hasattr(L, n)
@@ -115,3 +115,16 @@ def test_binding_refuses_cpu_tensors():
     q = torch.zeros(1, 1, 64, dtype=torch.bfloat16)
     with pytest.raises(ValueError, match="CUDA"):
         nv._ptr(q, torch.bfloat16, "q")
+
+
+def test_static_decode_rejects_problems_beyond_its_scratch():
+    """The allocation-free decode checks its fixed scratch size on the host."""
+    L = nv.lib()
+    big = shp(B=4, Hq=32, Hkv=8, max_pages=16384, page_size=64, num_blocks=65536)
+    assert nv.workspace_size(big, nv.CALL_DECODE_SPARSE) > nv.STATIC_SCRATCH_BYTES
+    rc = L.entmaxkv_decode_sparse_static(C.byref(big), FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, 1.5, FAKE,
+                                         None, None, None)
+    assert rc == -9
+    assert b"fixed" in L.entmaxkv_strerror(-9)
+    assert L.entmaxkv_decode_sparse_static(C.byref(shp(d=96)), FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, 1.5,
+                                           FAKE, None, None, None) == -2
