@@ -180,6 +180,22 @@ def run_gpu(args, rank, world):
 
     nst = 4
     ev = [[torch.cuda.Event(enable_timing=True) for _ in range(nst + 1)] for _ in range(args.steps)]
+
+    # One step (the four C-ABI calls) captured as a CUDA graph: the timed
+    # region replays it, so host launch latency does not enter the device time.
+    dec.step(q, append_page)  # eager first call: per-device set-up happens outside capture
+    torch.cuda.synchronize()
+    graph = torch.cuda.CUDAGraph()
+    side = torch.cuda.Stream()
+    side.wait_stream(torch.cuda.current_stream())
+    with torch.cuda.stream(side):
+        dec.step(q, append_page)
+    torch.cuda.current_stream().wait_stream(side)
+    with torch.cuda.graph(graph):
+        dec.step(q, append_page)
+    torch.cuda.synchronize()
+    gev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(args.steps)]
+
     # The timed region lasts milliseconds, far below nvidia-smi's sampling
     # period, so clocks are sampled over a loaded window that brackets it:
     # warm-up steps for >= 1 s before, untimed steps for >= 0.5 s after.
@@ -188,7 +204,7 @@ def run_gpu(args, rank, world):
         i = 0
         while i < args.warmup or time.perf_counter() - t0 < 1.0:
             flush.fill_(1)
-            dec.step(q, append_page)
+            graph.replay()
             if i % 16 == 15:
                 torch.cuda.synchronize()
             i += 1
@@ -198,6 +214,19 @@ def run_gpu(args, rank, world):
             torch.distributed.barrier()
         torch.cuda.synchronize()
         t_wall = time.perf_counter()
+        for i in range(args.steps):
+            flush.fill_(1)  # L2 flush, outside the step's events
+            gev[i][0].record(st)
+            graph.replay()
+            gev[i][1].record(st)
+        torch.cuda.synchronize()
+        if world > 1:
+            torch.distributed.barrier()
+        t_wall = time.perf_counter() - t_wall
+
+        # per-stage device times: the same step issued call by call, each call
+        # bracketed by events (the 256 MiB flush before each step keeps the
+        # host ahead of the GPU, so the events see kernel time, not host gaps)
         for i in range(args.steps):
             flush.fill_(1)
             e = ev[i]
@@ -214,18 +243,16 @@ def run_gpu(args, rank, world):
                                       dec.sel, dec.cnt, dec.alpha, dec.out, dec.tau, None, dec.ws)
             e[4].record(st)
         torch.cuda.synchronize()
-        if world > 1:
-            torch.distributed.barrier()
-        t_wall = time.perf_counter() - t_wall
         t1 = time.perf_counter()
         while time.perf_counter() - t1 < 0.5:
             for _ in range(16):
                 flush.fill_(1)
-                dec.step(q, append_page)
+                graph.replay()
             torch.cuda.synchronize()
     clocks = clk.summary()
+    step_ms = float(np.mean([a.elapsed_time(b) for a, b in gev]))
     stage_ms = np.array([[ev[i][j].elapsed_time(ev[i][j + 1]) for j in range(nst)] for i in range(args.steps)])
-    step_ms = float(stage_ms.sum(axis=1).mean())
+    eager_step_ms = float(stage_ms.sum(axis=1).mean())
     if world > 1:
         t = torch.tensor([step_ms], device=dev)
         torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
@@ -265,11 +292,7 @@ def run_gpu(args, rank, world):
     k_dev = torch.empty_like(inp["k_cache"][blk, :, tok])
     v_dev = torch.empty_like(k_dev)
     q_dev = torch.empty_like(q)
-    e2e_ms = []
-    for i in range(args.warmup + args.steps):
-        flush.fill_(1)
-        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-        a.record(st)
+    def e2e_once():
         q_dev.copy_(q_host, non_blocking=True)
         k_dev.copy_(k_new, non_blocking=True)
         v_dev.copy_(v_new, non_blocking=True)
@@ -277,15 +300,36 @@ def run_gpu(args, rank, world):
         inp["v_cache"][blk, :, tok] = v_dev
         dec.step(q_dev, append_page)
         out_host.copy_(dec.out, non_blocking=True)
-        b.record(st)
-        torch.cuda.synchronize()
-        if i >= args.warmup:
-            e2e_ms.append(a.elapsed_time(b))
-    e2e_step_ms = float(np.mean(e2e_ms))
+
+    def time_e2e(fn):
+        ts = []
+        for i in range(args.warmup + args.steps):
+            flush.fill_(1)
+            a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            a.record(st)
+            fn()
+            b.record(st)
+            torch.cuda.synchronize()
+            if i >= args.warmup:
+                ts.append(a.elapsed_time(b))
+        return float(np.mean(ts))
+
+    e2e_once()
+    torch.cuda.synchronize()
+    g2 = torch.cuda.CUDAGraph()
+    side.wait_stream(torch.cuda.current_stream())
+    with torch.cuda.stream(side):
+        e2e_once()
+    torch.cuda.current_stream().wait_stream(side)
+    with torch.cuda.graph(g2):
+        e2e_once()
+    torch.cuda.synchronize()
+    e2e_step_ms = time_e2e(g2.replay)
+    e2e_eager_ms = time_e2e(e2e_once)
     if world > 1:
-        t = torch.tensor([e2e_step_ms], device=dev)
+        t = torch.tensor([e2e_step_ms, e2e_eager_ms], device=dev)
         torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
-        e2e_step_ms = float(t.item())
+        e2e_step_ms, e2e_eager_ms = (float(x) for x in t.tolist())
     assert nv.get_status(clear=True) & ~nv.STATUS_OVERFLOW == 0
 
     peak, peak_kind = measured_peaks()
@@ -303,7 +347,8 @@ def run_gpu(args, rank, world):
     roofline = {"bound": "hbm", "kernel": dom, "achieved": round(achieved, 1), "peak": peak, "unit": "GB/s",
                 "frac": round(achieved / peak, 4), "traffic": traffic, "algorithmic_bytes": alg,
                 "peak_kind": f"{peak_kind} copy bandwidth (burst)"}
-    res = dict(wl=wl, step_ms=step_ms, stage_us=stage_us, dense=dense, nbytes=nbytes, clocks=clocks,
+    res = dict(wl=wl, step_ms=step_ms, eager_step_ms=eager_step_ms, e2e_eager_ms=e2e_eager_ms,
+               stage_us=stage_us, dense=dense, nbytes=nbytes, clocks=clocks,
                roofline=roofline, e2e_ms=e2e_step_ms, e2e_bytes=(q_host.numel() * 2 + k_new.numel() * 4,
                                                                out_host.numel() * 4),
                launches=kernels_per_step(policy == "gauss", True) * args.steps, t_wall=t_wall,
@@ -440,7 +485,12 @@ def main():
             "frac_of_hbm_peak": round(value / world / res["roofline"]["peak"], 4),
             "roofline": res["roofline"], "stages_us": res["stage_us"], "bytes_per_step": nb,
             "e2e": {"value": round(e2e_val, 2), "unit": "GB/s", "us_per_step": round(res["e2e_ms"] * 1e3, 2),
-                    "h2d_bytes_per_step": res["e2e_bytes"][0], "d2h_bytes_per_step": res["e2e_bytes"][1]},
+                    "h2d_bytes_per_step": res["e2e_bytes"][0], "d2h_bytes_per_step": res["e2e_bytes"][1],
+                    "how": "H2D of q and the appended token's k/v from pinned memory, append, step, D2H of the "
+                           "output, captured as one CUDA graph",
+                    "eager_us_per_step": round(res["e2e_eager_ms"] * 1e3, 2)},
+            "timing": "step = CUDA-graph replay of the four C-ABI calls; stages_us from the same calls issued "
+                      "eagerly with events around each (eager step sum %.2f us)" % (res["eager_step_ms"] * 1e3),
             "gpu_launches": res["launches"], "clocks": res["clocks"], "paper_context": PAPER_CONTEXT}
     if res["dense"]:
         de, ds = res["dense"]["dense_entmax"], res["dense"]["dense_softmax"]

@@ -54,7 +54,44 @@ int get_encoder() {
 
 // 2-D view of a paged cache: rows = num_blocks*Hkv*P tokens, d bf16 columns;
 // box = 64 columns x P rows, 128-byte swizzle (conflict-free ldmatrix reads).
+// The last few descriptors are kept, keyed by (address, geometry): a cache
+// passed again gets its descriptor without a driver call.
+struct MapEntry {
+    const void *base;
+    int d, rows, P;
+    CUtensorMap map;
+};
+MapEntry g_maps[16];
+int g_nmaps = 0, g_next_map = 0;
+
+int make_kv_map_uncached(CUtensorMap *m, const void *base, const entmaxkv_shape *s);
+
 int make_kv_map(CUtensorMap *m, const void *base, const entmaxkv_shape *s) {
+    const int rows = s->num_blocks * s->Hkv * s->page_size;
+    {
+        std::lock_guard<std::mutex> lk(g_mu);
+        for (int i = 0; i < g_nmaps; ++i)
+            if (g_maps[i].base == base && g_maps[i].d == s->d && g_maps[i].rows == rows &&
+                g_maps[i].P == s->page_size) {
+                *m = g_maps[i].map;
+                return ENTMAXKV_OK;
+            }
+    }
+    int rc = make_kv_map_uncached(m, base, s);
+    if (rc) return rc;
+    std::lock_guard<std::mutex> lk(g_mu);
+    MapEntry &e = g_maps[g_next_map];
+    e.base = base;
+    e.d = s->d;
+    e.rows = rows;
+    e.P = s->page_size;
+    e.map = *m;
+    g_next_map = (g_next_map + 1) % 16;
+    if (g_nmaps < 16) ++g_nmaps;
+    return ENTMAXKV_OK;
+}
+
+int make_kv_map_uncached(CUtensorMap *m, const void *base, const entmaxkv_shape *s) {
     int rc = get_encoder();
     if (rc) return rc;
     cuuint64_t dims[2] = {(cuuint64_t)s->d, (cuuint64_t)s->num_blocks * s->Hkv * s->page_size};

@@ -11,6 +11,8 @@
 #include <cuda_runtime.h>
 #include <stdint.h>
 
+#include <mutex>
+
 #include "../../include/entmaxkv.h"
 
 namespace ekv {
@@ -200,6 +202,30 @@ __device__ __forceinline__ int block_excl_scan(int v, int *sh, int *total) {
     __syncthreads();
     *total = sh[64];
     return sh[32 + warp] + x - v;
+}
+
+
+// cudaFuncSetAttribute(MaxDynamicSharedMemorySize) once per (kernel, device,
+// size): the setting persists, and repeating the driver call on every launch
+// costs host time on the decode path.
+inline cudaError_t ensure_smem(const void *func, size_t bytes) {
+    struct Entry {
+        const void *f;
+        int dev;
+        size_t bytes;
+    };
+    static std::mutex mu;
+    static Entry cache[256];
+    static int n = 0;
+    int dev = 0;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e != cudaSuccess) return e;
+    std::lock_guard<std::mutex> lk(mu);
+    for (int i = 0; i < n; ++i)
+        if (cache[i].f == func && cache[i].dev == dev && cache[i].bytes >= bytes) return cudaSuccess;
+    e = cudaFuncSetAttribute(func, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)bytes);
+    if (e == cudaSuccess && n < 256) cache[n++] = Entry{func, dev, bytes};
+    return e;
 }
 
 }  // namespace ekv

@@ -414,8 +414,7 @@ __global__ void __launch_bounds__(TAU_THREADS) tau_pv_kernel(const __grid_consta
     int *cpos = reinterpret_cast<int *>(cbuf + ZCAP * 4);
     double(*accs)[D] = reinterpret_cast<double(*)[D]>(cbuf);
     static_assert(TAU_WARPS * D * 8 <= ZCAP * 8, "partials must fit the candidate buffer");
-    __shared__ double red[TAU_WARPS][33];
-    __shared__ unsigned balw[2][TAU_WARPS];
+    __shared__ float red[TAU_WARPS][33];
     __shared__ int sh[72];
     __shared__ float br[2];
     const int bh = blockIdx.x;
@@ -486,68 +485,44 @@ __global__ void __launch_bounds__(TAU_THREADS) tau_pv_kernel(const __grid_consta
     const int nloop = onchip ? nc : n_tok;
     auto cz_at = [&](int i) -> float { return onchip ? cz[i] : __ldcg(zr + i); };
 
+    // Multisection on [z_max - 1, z_max - n^(1-alpha)]: 32 points per pass,
+    // lane l of every warp evaluates point l over the warp's slice of the
+    // candidates (slices and order are fixed, so the sums are reproducible),
+    // and the warps' partial sums are added in warp order.
     float lo = thr;
     float hi = zmax - powf((float)nc, 1.f - a.alpha);
     if (nc > 1 && hi > lo) {
         const float tol = 1e-7f * fmaxf(1.f, fabsf(zmax));
-        if (onchip && nc <= 256) {
-            // every thread evaluates one point over all candidates
-            for (int pass = 0; pass < 4 && hi - lo > tol; ++pass) {
-                const float w = (hi - lo) / (float)(TAU_THREADS + 1);
-                const float t = lo + w * (float)(threadIdx.x + 1);
-                double f = 0.0;
-                for (int c = 0; c < nc; ++c) f += (double)pos_pow(cz[c] - t, r, ri);
-                const unsigned bal = __ballot_sync(FULL, f >= 1.0);  // still left of the root
-                if (lane == 0) balw[pass & 1][warp] = bal;
-                __syncthreads();
-                int cntge = 0;  // points increase with thread index and f decreases: a prefix
-                for (int ww = 0; ww < TAU_WARPS; ++ww) cntge += __popc(balw[pass & 1][ww]);
-                const float nlo = cntge > 0 ? lo + w * (float)cntge : lo;
-                const float nhi = cntge < TAU_THREADS ? lo + w * (float)(cntge + 1) : hi;
-                lo = nlo;
-                hi = nhi;
+        for (int pass = 0; pass < 12 && hi - lo > tol; ++pass) {
+            const float w = (hi - lo) / 33.f;
+            const float t = lo + w * (float)(lane + 1);
+            float f = 0.f;
+            if (onchip) {
+                const int per = ceil_div(nc, TAU_WARPS);
+                const int c1 = min(nc, (warp + 1) * per);
+                for (int c = warp * per; c < c1; ++c) f += pos_pow(cz[c] - t, r, ri);
+            } else {
+                for (int c = warp; c < n_tok; c += TAU_WARPS) {
+                    const float z = __ldcg(zr + c);
+                    if (z > thr) f += pos_pow(z - t, r, ri);
+                }
             }
-        } else {
-            // 32 points per pass, candidates spread over the block
-            for (int pass = 0; pass < 12 && hi - lo > tol; ++pass) {
-                const float w = (hi - lo) / 33.f;
-                double f[32];
-#pragma unroll
-                for (int j = 0; j < 32; ++j) f[j] = 0.0;
-                for (int c = threadIdx.x; c < nloop; c += TAU_THREADS) {
-                    const float z = cz_at(c);
-                    if (!(z > thr)) continue;
-#pragma unroll
-                    for (int j = 0; j < 32; ++j) f[j] += (double)pos_pow(z - (lo + w * (float)(j + 1)), r, ri);
+            red[warp][lane] = f;
+            __syncthreads();
+            if (warp == 0) {
+                float tot = 0.f;
+                for (int ww = 0; ww < TAU_WARPS; ++ww) tot += red[ww][lane];
+                // points increase with the lane and F decreases: the ones at or
+                // left of the root form a prefix
+                const int cntge = __popc(__ballot_sync(FULL, tot >= 1.f));
+                if (lane == 0) {
+                    br[0] = cntge > 0 ? lo + w * (float)cntge : lo;
+                    br[1] = cntge < 32 ? lo + w * (float)(cntge + 1) : hi;
                 }
-                // transpose-reduce: lane l ends with the warp sum of point l
-#pragma unroll
-                for (int s = 16; s >= 1; s >>= 1) {
-#pragma unroll
-                    for (int i = 0; i < s; ++i) {
-                        const bool up = lane & s;
-                        const double send = up ? f[i] : f[i + s];
-                        const double keep = up ? f[i + s] : f[i];
-                        f[i] = keep + __shfl_xor_sync(FULL, send, s);
-                    }
-                }
-                red[warp][lane] = f[0];
-                __syncthreads();
-                if (warp == 0) {
-                    double tot = 0.0;
-                    for (int ww = 0; ww < TAU_WARPS; ++ww) tot += red[ww][lane];
-                    const unsigned bal = __ballot_sync(FULL, tot >= 1.0);
-                    if (lane == 0) {
-                        const int cntge = __popc(bal);
-                        br[0] = cntge > 0 ? lo + w * (float)cntge : lo;
-                        br[1] = cntge < 32 ? lo + w * (float)(cntge + 1) : hi;
-                    }
-                }
-                __syncthreads();
-                lo = br[0];
-                hi = br[1];
-                __syncthreads();
             }
+            __syncthreads();
+            lo = br[0];
+            hi = br[1];
         }
     } else {
         hi = lo;
@@ -1057,7 +1032,7 @@ int pick_splits(int sms, int per_sm, int groups, int max_steps, int cap) {
 
 template <class K>
 cudaError_t set_smem(K kern, size_t bytes) {
-    return cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)bytes);
+    return ensure_smem(reinterpret_cast<const void *>(kern), bytes);
 }
 
 template <int D, int G, bool DENSE>

@@ -199,7 +199,7 @@ cudaError_t launch_t(const ScoreArgs &a, cudaStream_t st) {
     using Cfg = ScoreCfg<GAUSS>;
     const size_t smem = QLayout<D, G>::BYTES + (size_t)SC_WARPS * Cfg::NST * Cfg::WARP_STAGE;
     auto kern = score_kernel<D, G, GAUSS>;
-    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    cudaError_t e = ensure_smem(reinterpret_cast<const void *>(kern), smem);
     if (e != cudaSuccess) return e;
     dim3 grid(ceil_div(a.max_pages, SC_THREADS), a.B * a.Hkv);
     kern<<<grid, SC_THREADS, smem, st>>>(a);

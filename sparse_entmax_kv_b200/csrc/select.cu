@@ -11,12 +11,14 @@
 //
 // Gaussian: tau_hat solves F(tau) = sum_p n_p E[(X_p - tau)_+^r] = 1 with
 // X_p ~ N(m_p, s_p^2), m_p = (alpha-1) mu_p, s_p = (alpha-1) sigma_p, using the
-// closed-form Gaussian partial moments.  F >= 1 at tau0 = max_p m_p - 1
-// (Jensen), and g(tau) = F(tau)^(1/r) is convex and decreasing (an L^r norm of
-// (X - tau)_+), so Newton on g started at tau0 climbs monotonically to the
-// root without overshoot.  Pages with m_p + 10 s_p < tau0 contribute below
-// n_p s_p^r J_r(10) ~ 1e-25 n_p s_p^r at any tau >= tau0 and are pruned before
-// the iterations.  Pages are then kept when (alpha-1) bbox_p > tau_hat - Delta.
+// closed-form Gaussian partial moments.  F is decreasing, F >= 1 at
+// tau0 = max_p m_p - 1 (Jensen) and F < 1 at max_p (m_p + 10 s_p) (every page
+// is then 10 standard deviations into its tail).  Pages with
+// m_p + 10 s_p < tau0 contribute below n_p s_p^r J_r(10) ~ 1e-25 n_p s_p^r
+// anywhere in that bracket and are pruned.  The bracket is narrowed by
+// multisection: each pass evaluates F at 32 points, one warp per point with
+// the lanes splitting the pages.  Pages are then kept when
+// (alpha-1) bbox_p > tau_hat - Delta.
 #include "common.cuh"
 #include "internal.h"
 
@@ -193,8 +195,7 @@ constexpr int GCAP = 3072;  // pruned candidate pages held on chip
 template <int R>
 __global__ void __launch_bounds__(SEL_THREADS) gauss_kernel(SelectArgs a) {
     __shared__ float cm[GCAP], cs[GCAP], cn[GCAP];
-    __shared__ float shf[2][2 * 32];
-    __shared__ float shm[32];
+    __shared__ float shm[32], shm2[32];
     __shared__ int shi[72];
     __shared__ int ncand;
     const int bh = blockIdx.x;
@@ -244,11 +245,13 @@ __global__ void __launch_bounds__(SEL_THREADS) gauss_kernel(SelectArgs a) {
     for (int w = 0; w < SEL_THREADS / 32; ++w) mmax = fmaxf(mmax, shm[w]);
     const float tau0 = mmax - 1.f;
 
+    float hloc = -INFINITY;  // max over pages of m + 10 s: F < 1 there
     for (int t0 = 0; t0 < n; t0 += TILE) {
         if (!one_tile) load_ms(t0);
 #pragma unroll
         for (int i = 0; i < ITEMS; ++i) {
             const int p = t0 + threadIdx.x + SEL_THREADS * i;
+            if (p < n) hloc = fmaxf(hloc, mm[i] + 10.f * ss[i]);
             const bool keep = p < n && mm[i] + 10.f * ss[i] >= tau0;
             const unsigned bal = __ballot_sync(FULL, keep);
             if (!bal) continue;
@@ -265,9 +268,15 @@ __global__ void __launch_bounds__(SEL_THREADS) gauss_kernel(SelectArgs a) {
             }
         }
     }
+#pragma unroll
+    for (int o = 16; o; o >>= 1) hloc = fmaxf(hloc, __shfl_xor_sync(FULL, hloc, o));
+    if (lane == 0) shm2[warp] = hloc;
     __syncthreads();
     const int nc = ncand;
     const bool overflow = nc > GCAP;
+    float hmax = -INFINITY;
+    for (int w = 0; w < SEL_THREADS / 32; ++w) hmax = fmaxf(hmax, shm2[w]);
+    hmax = fmaxf(hmax, tau0 + 1.f);
     if (overflow && threadIdx.x == 0) atomicOr(a.status, ENTMAXKV_STATUS_OVERFLOW);
 
     auto contrib = [&](float m, float s, float w, float tau, float &F, float &Fp) {
@@ -293,39 +302,37 @@ __global__ void __launch_bounds__(SEL_THREADS) gauss_kernel(SelectArgs a) {
         }
     };
 
-    float tau = tau0;
-    for (int it = 0; it < 64; ++it) {
+    // multisection on [tau0, hi]: warp w evaluates F at point w
+    __shared__ float fpt[32];
+    __shared__ float brk[2];
+    float lo = tau0, hi = hmax;
+    for (int pass = 0; pass < 8 && hi - lo > 1e-7f * fmaxf(1.f, fabsf(lo)); ++pass) {
+        const float w = (hi - lo) / 33.f;
+        const float t = lo + w * (float)(warp + 1);
         float F = 0.f, Fp = 0.f;
         if (!overflow) {
-            for (int i = threadIdx.x; i < nc; i += SEL_THREADS) contrib(cm[i], cs[i], cn[i], tau, F, Fp);
+            for (int i = lane; i < nc; i += 32) contrib(cm[i], cs[i], cn[i], t, F, Fp);
         } else {
-            for (int p = threadIdx.x; p < n; p += SEL_THREADS)
-                contrib(a1 * a.mu[row + p], a1 * a.sigma[row + p], (float)tokens_in_page(seq, a.P, p), tau, F,
-                        Fp);
+            for (int p = lane; p < n; p += 32)
+                contrib(a1 * a.mu[row + p], a1 * a.sigma[row + p], (float)tokens_in_page(seq, a.P, p), t, F, Fp);
         }
 #pragma unroll
-        for (int o = 16; o; o >>= 1) {
-            F += __shfl_xor_sync(FULL, F, o);
-            Fp += __shfl_xor_sync(FULL, Fp, o);
-        }
-        float *buf = shf[it & 1];
-        if (lane == 0) {
-            buf[2 * warp] = F;
-            buf[2 * warp + 1] = Fp;
+        for (int o = 16; o; o >>= 1) F += __shfl_xor_sync(FULL, F, o);
+        if (lane == 0) fpt[warp] = F;
+        __syncthreads();
+        if (warp == 0) {
+            // points increase with the warp index and F decreases: a prefix
+            const int cntge = __popc(__ballot_sync(FULL, fpt[lane] >= 1.f));
+            if (lane == 0) {
+                brk[0] = cntge > 0 ? lo + w * (float)cntge : lo;
+                brk[1] = cntge < 32 ? lo + w * (float)(cntge + 1) : hi;
+            }
         }
         __syncthreads();
-        F = 0.f;
-        Fp = 0.f;
-        for (int w = 0; w < SEL_THREADS / 32; ++w) {
-            F += buf[2 * w];
-            Fp += buf[2 * w + 1];
-        }
-        if (!(F > 1.f + 2e-6f) || !(Fp < 0.f)) break;
-        // Newton on g = F^(1/R): step = R (F - F^(1-1/R)) / (-F')
-        const float step = (float)R * (F - powf(F, 1.f - 1.f / (float)R)) / (-Fp);
-        tau += step;
-        if (!(step > 1e-7f * fmaxf(1.f, fabsf(tau)))) break;
+        lo = brk[0];
+        hi = brk[1];
     }
+    const float tau = 0.5f * (lo + hi);
     if (threadIdx.x == 0 && a.tau_hat) a.tau_hat[bh] = tau;
 
     const float thr = tau - a.delta;
