@@ -52,6 +52,9 @@ struct PageInfo {
 __device__ __forceinline__ size_t tok_row(const DecodeArgs &a, int b, int h) {
     return ((size_t)b * a.Hq + h) * (size_t)a.max_pages * a.P;
 }
+__device__ __forceinline__ size_t tile_row(const DecodeArgs &a, int b, int h) {
+    return ((size_t)b * a.Hq + h) * (size_t)a.max_pages * a.P / 16;
+}
 
 // ------------------------------------------------------------------ union
 
@@ -337,16 +340,24 @@ __global__ void __launch_bounds__(DEC_THREADS) qk_kernel(const __grid_constant__
                     if (hh < G) a.ws.zbuf[tok_row(a, b, kvh * G + hh) + (size_t)pi.upos * P + t] = z[v];
                     if (a.p_out && use) a.p_out[tok_row(a, b, kvh * G + hh) + (size_t)pi.page * P + t] = 0.f;
                 }
-                run0 = fmaxf(run0, fmaxf(z[0], z[2]));
-                run1 = fmaxf(run1, fmaxf(z[1], z[3]));
+                // max over the m-tile's 16 tokens, per head (lanes with equal lane%4
+                // hold the same two heads)
+                float m0 = fmaxf(z[0], z[2]), m1 = fmaxf(z[1], z[3]);
+#pragma unroll
+                for (int o = 4; o < 32; o <<= 1) {
+                    m0 = fmaxf(m0, __shfl_xor_sync(FULL, m0, o));
+                    m1 = fmaxf(m1, __shfl_xor_sync(FULL, m1, o));
+                }
+                run0 = fmaxf(run0, m0);
+                run1 = fmaxf(run1, m1);
+                if (lane < 4) {
+                    const size_t ti = ((size_t)pi.upos * P + r0) / 16;
+                    if (h0 < G) a.ws.tmax[tile_row(a, b, kvh * G + h0) + ti] = m0;
+                    if (h0 + 1 < G) a.ws.tmax[tile_row(a, b, kvh * G + h0 + 1) + ti] = m1;
+                }
             }
             __syncwarp();
             if (lane == 0) mbar_arrive(&R.empty[st]);
-        }
-#pragma unroll
-        for (int o = 4; o < 32; o <<= 1) {
-            run0 = fmaxf(run0, __shfl_xor_sync(FULL, run0, o));
-            run1 = fmaxf(run1, __shfl_xor_sync(FULL, run1, o));
         }
         if (lane < 4) {
             if (h0 < G && run0 > -INFINITY) atomicMax(&a.ws.zmax[bh0], f2ord(run0));
@@ -386,6 +397,12 @@ __global__ void __launch_bounds__(DEC_THREADS) qk_kernel(const __grid_constant__
                 if (a.p_out) a.p_out[tok_row(a, b, kvh) + (size_t)pi.page * P + r] = 0.f;
             }
             if (pi.page >= 0) a.ws.zbuf[tok_row(a, b, kvh) + (size_t)pi.upos * P + r] = z;
+            // max of each 16-token tile (a half warp; tiles never straddle pages)
+            float tm = z;
+#pragma unroll
+            for (int o = 1; o < 16; o <<= 1) tm = fmaxf(tm, __shfl_xor_sync(FULL, tm, o));
+            if ((lane & 15) == 0 && pi.page >= 0)
+                a.ws.tmax[tile_row(a, b, kvh) + ((size_t)pi.upos * P + r) / 16] = tm;
             run = fmaxf(run, z);
             __syncwarp();
             if (lane == 0) mbar_arrive(&R.empty[st]);
@@ -402,6 +419,7 @@ constexpr int TAU_THREADS = 512;
 constexpr int TAU_WARPS = TAU_THREADS / 32;
 constexpr int ZCAP = 4096;  // candidates held on chip per head
 constexpr int TAU_C = 32;   // list positions per thread per scan tile
+constexpr int TCAP = 2048;  // candidate 16-token tiles held on chip per head
 
 // Exact threshold and (GATHER) the weighted sum of the support's value rows.
 template <int D, bool GATHER>
@@ -415,6 +433,7 @@ __global__ void __launch_bounds__(TAU_THREADS) tau_pv_kernel(const __grid_consta
     double(*accs)[D] = reinterpret_cast<double(*)[D]>(cbuf);
     static_assert(TAU_WARPS * D * 8 <= ZCAP * 8, "partials must fit the candidate buffer");
     __shared__ float red[TAU_WARPS][33];
+    __shared__ int ctile[TCAP];  // candidate 16-token tiles, in list order
     __shared__ int sh[72];
     __shared__ float br[2];
     const int bh = blockIdx.x;
@@ -441,43 +460,58 @@ __global__ void __launch_bounds__(TAU_THREADS) tau_pv_kernel(const __grid_consta
     const float thr = zmax - 1.f;
     const float *zr = a.ws.zbuf + tok_row(a, b, h);
 
-    // ordered compaction of the positions with z > thr: each thread scans
-    // TAU_C consecutive positions per tile (all loads issued first), and one
-    // block scan places them
-    int nc = 0;
-    for (int t0 = 0; t0 < n_tok; t0 += TAU_THREADS * TAU_C) {
+    // Candidates in list order, in two ordered compactions: first the 16-token
+    // tiles whose max exceeds thr, then the tokens of those tiles.  Each uses
+    // one block scan per pass over TAU_THREADS * TAU_C entries.
+    const int n_tiles = n_tok / 16;
+    const float *tr = a.ws.tmax + tile_row(a, b, h);
+    int ntc = 0;
+    for (int t0 = 0; t0 < n_tiles; t0 += TAU_THREADS * TAU_C) {
         const int p0 = t0 + threadIdx.x * TAU_C;
-        float4 v[TAU_C / 4];
+        float v[TAU_C];
 #pragma unroll
-        for (int i = 0; i < TAU_C / 4; ++i)
-            v[i] = p0 + 4 * i < n_tok ? __ldcg(reinterpret_cast<const float4 *>(zr + p0 + 4 * i))
-                                      : make_float4(-INFINITY, -INFINITY, -INFINITY, -INFINITY);
+        for (int i = 0; i < TAU_C; ++i) v[i] = p0 + i < n_tiles ? __ldcg(tr + p0 + i) : -INFINITY;
         unsigned bits = 0;
 #pragma unroll
-        for (int i = 0; i < TAU_C / 4; ++i) {
-            if (v[i].x > thr) bits |= 1u << (4 * i);
-            if (v[i].y > thr) bits |= 1u << (4 * i + 1);
-            if (v[i].z > thr) bits |= 1u << (4 * i + 2);
-            if (v[i].w > thr) bits |= 1u << (4 * i + 3);
-        }
+        for (int i = 0; i < TAU_C; ++i)
+            if (v[i] > thr) bits |= 1u << i;
         int tot;
-        int w = nc + block_excl_scan(__popc(bits), sh, &tot);
-#pragma unroll
-        for (int i = 0; i < TAU_C / 4; ++i) {
-            const float vv[4] = {v[i].x, v[i].y, v[i].z, v[i].w};
-#pragma unroll
-            for (int j = 0; j < 4; ++j) {
-                if (bits & (1u << (4 * i + j))) {
-                    if (w < ZCAP) {
-                        cz[w] = vv[j];
-                        cpos[w] = p0 + 4 * i + j;
-                    }
-                    ++w;
-                }
-            }
+        int w = ntc + block_excl_scan(__popc(bits), sh, &tot);
+        while (bits) {
+            const int k = __ffs(bits) - 1;
+            bits &= bits - 1;
+            if (w < TCAP) ctile[w] = p0 + k;
+            ++w;
         }
-        nc += tot;
+        ntc += tot;
     }
+    __syncthreads();
+    int nc = 0;
+    if (ntc <= TCAP) {
+        // the tokens of the candidate tiles
+        for (int e0 = 0; e0 < ntc * 16; e0 += TAU_THREADS) {
+            const int e = e0 + threadIdx.x;
+            float z = -INFINITY;
+            int pos = 0;
+            if (e < ntc * 16) {
+                pos = ctile[e >> 4] * 16 + (e & 15);
+                z = __ldcg(zr + pos);
+            }
+            const bool c = z > thr;
+            int tot;
+            const int w = nc + block_excl_scan(c ? 1 : 0, sh, &tot);
+            __syncthreads();  // every thread has read its tile entry
+            if (c && w < ZCAP) {
+                cz[w] = z;
+                cpos[w] = pos;
+            }
+            nc += tot;
+            __syncthreads();
+        }
+    } else {
+        nc = ZCAP + 1;  // too many tiles to list: take the whole-row path below
+    }
+    __syncthreads();
     __syncthreads();
     const bool onchip = nc <= ZCAP;
     if (!onchip && threadIdx.x == 0) atomicOr(a.status, ENTMAXKV_STATUS_OVERFLOW);
@@ -1139,6 +1173,7 @@ size_t decode_ws_bytes(bool dense, int B, int Hq, int Hkv, int d, int P, int max
     const size_t o_cnt = take((size_t)B * Hkv * 4);
     const size_t o_part = take(dense ? (size_t)MAX_SPLITS * B * Hq * (d + 2) * 4 : 0);
     const size_t o_z = take(tokens * 4);
+    const size_t o_t = take(tokens / 16 * 4);
     if (carve && base) {
         char *p = static_cast<char *>(base);
         carve->union_e = reinterpret_cast<int *>(p + o_union);
@@ -1149,6 +1184,7 @@ size_t decode_ws_bytes(bool dense, int B, int Hq, int Hkv, int d, int P, int max
         carve->counters = reinterpret_cast<int *>(p + o_cnt);
         carve->partial = reinterpret_cast<float *>(p + o_part);
         carve->zbuf = reinterpret_cast<float *>(p + o_z);
+        carve->tmax = reinterpret_cast<float *>(p + o_t);
     }
     return off;
 }

@@ -64,6 +64,7 @@ struct DecodeWs {
     int *counters;   // [B*Hkv] last-CTA combine counters
     float *partial;  // [MAX_SPLITS][B*Hq][d+2]  (dense paths)
     float *zbuf;     // [B*Hq][max_pages*P]  z of every token of the page list, in list order
+    float *tmax;     // [B*Hq][max_pages*P/16]  max z of each 16-token tile of zbuf
 };
 
 struct DecodeArgs {

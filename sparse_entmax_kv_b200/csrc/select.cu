@@ -302,11 +302,15 @@ __global__ void __launch_bounds__(SEL_THREADS) gauss_kernel(SelectArgs a) {
         }
     };
 
-    // multisection on [tau0, hi]: warp w evaluates F at point w
+    // One multisection pass on [tau0, hmax] (warp w evaluates F at point w),
+    // then Newton on g = F^(1/R) from the bracket's left end: g is convex and
+    // decreasing, so the iterates climb monotonically to the root.  Each
+    // Newton evaluation is spread over the whole block (one barrier each).
     __shared__ float fpt[32];
     __shared__ float brk[2];
+    __shared__ float nred[2][64];
     float lo = tau0, hi = hmax;
-    for (int pass = 0; pass < 8 && hi - lo > 1e-7f * fmaxf(1.f, fabsf(lo)); ++pass) {
+    {
         const float w = (hi - lo) / 33.f;
         const float t = lo + w * (float)(warp + 1);
         float F = 0.f, Fp = 0.f;
@@ -332,7 +336,42 @@ __global__ void __launch_bounds__(SEL_THREADS) gauss_kernel(SelectArgs a) {
         lo = brk[0];
         hi = brk[1];
     }
-    const float tau = 0.5f * (lo + hi);
+    float tau = lo;
+    for (int it = 0; it < 32; ++it) {
+        float F = 0.f, Fp = 0.f;
+        if (!overflow) {
+            for (int i = threadIdx.x; i < nc; i += SEL_THREADS) contrib(cm[i], cs[i], cn[i], tau, F, Fp);
+        } else {
+            for (int p = threadIdx.x; p < n; p += SEL_THREADS)
+                contrib(a1 * a.mu[row + p], a1 * a.sigma[row + p], (float)tokens_in_page(seq, a.P, p), tau, F,
+                        Fp);
+        }
+#pragma unroll
+        for (int o = 16; o; o >>= 1) {
+            F += __shfl_xor_sync(FULL, F, o);
+            Fp += __shfl_xor_sync(FULL, Fp, o);
+        }
+        float *buf = nred[it & 1];
+        if (lane == 0) {
+            buf[2 * warp] = F;
+            buf[2 * warp + 1] = Fp;
+        }
+        __syncthreads();
+        F = 0.f;
+        Fp = 0.f;
+        for (int w = 0; w < SEL_THREADS / 32; ++w) {
+            F += buf[2 * w];
+            Fp += buf[2 * w + 1];
+        }
+        if (!(F > 1.f + 2e-6f) || !(Fp < 0.f)) break;
+        // Newton on g = F^(1/R): step = R (F - F^(1-1/R)) / (-F')
+        const float step = (float)R * (F - powf(F, 1.f - 1.f / (float)R)) / (-Fp);
+        float nt = tau + step;
+        if (!(nt < hi)) nt = 0.5f * (tau + hi);  // stay inside the bracket
+        const bool done = !(nt - tau > 1e-7f * fmaxf(1.f, fabsf(tau)));
+        tau = nt;
+        if (done) break;
+    }
     if (threadIdx.x == 0 && a.tau_hat) a.tau_hat[bh] = tau;
 
     const float thr = tau - a.delta;
