@@ -5,11 +5,9 @@
 //   mu    = (sum_j q_j mean_j) / sqrt(d)                    Gaussian mean
 //   sigma = sqrt((sum_j q_j^2 var_j) / d)                   Gaussian std
 // The bound is one fp64 chain over j in index order with exact products, so
-// it is reproducible to the bit.  With q+ = max(q, 0) and q- = min(q, 0),
-// max(q a, q b) (a <= b) equals q+ b + q- a with one of the two terms an exact
-// zero, so two fused multiply-adds per coordinate give the same chain with no
-// selects.  mu and sigma feed only the approximate tau_hat; they are fp32
-// chains over j in index order.
+// it is reproducible to the bit; max(q a, q b) with a <= b is q b for q >= 0
+// and q a otherwise, one fused multiply-add per coordinate.  mu and sigma feed
+// only the approximate tau_hat; they are fp32 chains over j in index order.
 //
 // Layout of the work: a CTA owns 256 consecutive logical pages of one
 // (b, kv head); thread = page, and the thread scores that page for all G query
@@ -43,10 +41,10 @@ struct ScoreCfg {
 
 template <int D, int G>
 struct QLayout {
-    // qpn: [D][G][2] fp64 (q+, q-); qf, qqf: [D][G] fp32 (q, q^2)
-    static constexpr int PN_BYTES = D * G * 2 * 8;
+    // qd: [D][G] fp64; qf: [D][G] fp32 (the same bf16 values)
+    static constexpr int D_BYTES = D * G * 8;
     static constexpr int F_BYTES = D * G * 4;
-    static constexpr int BYTES = PN_BYTES + 2 * F_BYTES;
+    static constexpr int BYTES = D_BYTES + F_BYTES;
 };
 
 template <int D, int G, bool GAUSS>
@@ -55,9 +53,8 @@ __global__ void __launch_bounds__(SC_THREADS, 2) score_kernel(ScoreArgs a) {
     using QL = QLayout<D, G>;
     constexpr int NCH = D / CH;
     extern __shared__ __align__(16) unsigned char smem[];
-    double *qpn = reinterpret_cast<double *>(smem);
-    float *qf = reinterpret_cast<float *>(smem + QL::PN_BYTES);
-    float *qqf = qf + D * G;
+    double *qd = reinterpret_cast<double *>(smem);
+    float *qf = reinterpret_cast<float *>(smem + QL::D_BYTES);
     unsigned char *ring = smem + QL::BYTES;
 
     const int bk = blockIdx.y;
@@ -67,10 +64,8 @@ __global__ void __launch_bounds__(SC_THREADS, 2) score_kernel(ScoreArgs a) {
     for (int i = threadIdx.x; i < G * D; i += SC_THREADS) {
         const int g = i / D, j = i % D;
         const float v = bf16f(a.q[((size_t)b * a.Hq + kvh * G + g) * D + j]);
-        qpn[(j * G + g) * 2] = v > 0.f ? (double)v : 0.0;
-        qpn[(j * G + g) * 2 + 1] = v < 0.f ? (double)v : 0.0;
+        qd[j * G + g] = (double)v;
         qf[j * G + g] = v;
-        qqf[j * G + g] = v * v;  // exact: bf16 squared fits in fp32
     }
     __syncthreads();
 
@@ -157,9 +152,8 @@ __global__ void __launch_bounds__(SC_THREADS, 2) score_kernel(ScoreArgs a) {
                 vv[4 * i] = v4.x; vv[4 * i + 1] = v4.y; vv[4 * i + 2] = v4.z; vv[4 * i + 3] = v4.w;
             }
         }
-        const double *qpc = qpn + (size_t)c * CH * G * 2;
+        const double *qdc = qd + (size_t)c * CH * G;
         const float *qfc = qf + c * CH * G;
-        const float *qqc = qqf + c * CH * G;
 #pragma unroll
         for (int jj = 0; jj < CH; ++jj) {
             const unsigned w_n = wn[jj >> 1], w_x = wx[jj >> 1];
@@ -167,12 +161,12 @@ __global__ void __launch_bounds__(SC_THREADS, 2) score_kernel(ScoreArgs a) {
             const double hi = (double)((jj & 1) ? bf16hi(w_x) : bf16lo(w_x));
 #pragma unroll
             for (int g = 0; g < G; ++g) {
-                const double2 pn = *reinterpret_cast<const double2 *>(qpc + (jj * G + g) * 2);
-                ab[g] = __fma_rn(pn.x, hi, ab[g]);  // q+ * kmax (zero when q < 0)
-                ab[g] = __fma_rn(pn.y, lo, ab[g]);  // q- * kmin (zero when q >= 0)
+                const double qv = qdc[jj * G + g];
+                ab[g] = __fma_rn(qv, (__double2hiint(qv) < 0) ? lo : hi, ab[g]);
                 if (GAUSS) {
-                    am[g] = __fmaf_rn(qfc[jj * G + g], mv[jj], am[g]);
-                    av[g] = __fmaf_rn(qqc[jj * G + g], vv[jj], av[g]);
+                    const float qs = qfc[jj * G + g];
+                    am[g] = __fmaf_rn(qs, mv[jj], am[g]);
+                    av[g] = __fmaf_rn(__fmul_rn(qs, qs), vv[jj], av[g]);  // q^2 exact in fp32
                 }
             }
         }
