@@ -115,13 +115,25 @@ ENTMAXKV_API int entmaxkv_version(void);
 
 /*
  * Bytes of the metadata buffer written by entmaxkv_build_meta and read by
- * entmaxkv_score_pages: num_blocks * Hkv * 12 * d.  Layout (record r =
- * block * Hkv + kv_head):
- *   bytes [0, R*4d):          bound region, record r at r*4d:
- *                             kmin bf16[d] then kmax bf16[d]
- *   bytes [R*4d, R*12d):      moment region, record r at R*4d + r*8d:
- *                             mean f32[d] then var f32[d]
- * with R = num_blocks * Hkv.  Returns 0 for an invalid shape.
+ * entmaxkv_score_pages: B * Hkv * n_tiles * 384 * d, n_tiles =
+ * ceil(max_pages / 32).  Records are kept in logical page order, so a score
+ * pass streams contiguous memory however the page table scatters the blocks.
+ * Pages are grouped in tiles of 32 consecutive logical pages of one
+ * (sequence b, kv head): tile T = (b * Hkv + kv_head) * n_tiles + p / 32,
+ * page slot s = p % 32.  Coordinates are grouped in chunks of 16: chunk
+ * c = j / 16, e = j % 16.
+ *   bound region, bytes [0, NT*128d) with NT = B*Hkv*n_tiles:
+ *     tile T at T*128d, chunk c at +2048c, kmin block at +0, kmax block at
+ *     +1024; in a block, slot s holds its 16 bf16 values in two 16-byte
+ *     halves h = e/8 stored at 32s + 16*(h ^ ((s>>2)&1)), element at +2(e%8).
+ *   moment region, bytes [NT*128d, NT*384d):
+ *     tile T at NT*128d + T*256d, chunk c at +4096c, mean block at +0, var
+ *     block at +2048; in a block, slot s holds its 16 fp32 values in four
+ *     16-byte quarters h = e/4 stored at 64s + 16*(h ^ ((s>>1)&3)),
+ *     element at +4(e%4).
+ * (The XOR places the pieces eight neighbouring pages read at one time on
+ * distinct shared-memory banks once a chunk block is copied on chip.)
+ * d must be a multiple of 16.  Returns 0 for an invalid shape.
  */
 ENTMAXKV_API size_t entmaxkv_meta_bytes(const entmaxkv_shape *shape);
 
@@ -146,14 +158,14 @@ ENTMAXKV_API int entmaxkv_get_status(int32_t *status_out, int clear, void *strea
  * Section 2.A (bounding box and Gaussian statistics, "maintained on append"):
  * for each sequence b, each logical page p in [first_page, first_page+n_pages)
  * with p < N_b (n_pages = -1: to the end), and each kv head, recompute the
- * metadata record of block page_table[b][p] from its n = min(P, seq_len - pP)
- * valid tokens, per coordinate j:
+ * metadata record of logical page p (its keys are in block page_table[b][p])
+ * from its n = min(P, seq_len - pP) valid tokens, per coordinate j:
  *   kmin_j, kmax_j : the bf16 extreme (first token wins exact ties)
  *   mean_j = fp32(S1/n),  var_j = fp32(max(0, S2/n - (S1/n)^2))
  * with S1 = sum k_tj, S2 = sum k_tj^2 accumulated in fp64 in token order (the
  * result is defined to the bit).  Calling it on the page a new token was
- * appended to keeps the metadata current.  Records of blocks no listed page
- * maps to are not touched.
+ * appended to keeps the metadata current.  Records of pages outside the
+ * range are not touched.
  */
 ENTMAXKV_API int entmaxkv_build_meta(const entmaxkv_shape *shape, const void *k_cache,
                         const int32_t *page_table, const int32_t *seq_lens,
@@ -169,12 +181,13 @@ ENTMAXKV_API int entmaxkv_build_meta(const entmaxkv_shape *shape, const void *k_
  * fp64 over j in index order (products are exact), so results are defined to
  * the bit.  Outputs are fp32 [B][Hq][max_pages]; entries for p >= N_b are not
  * written.  mu and sigma may both be NULL (bound only, reads 4d bytes per
- * record instead of 12d); if one is non-NULL both must be.
+ * page and kv head instead of 12d); if one is non-NULL both must be.  The
+ * metadata is addressed by logical page, so no page table is needed; pages
+ * whose keys are not all finite have unspecified scores.
  */
 ENTMAXKV_API int entmaxkv_score_pages(const entmaxkv_shape *shape, const void *q,
-                         const void *meta, const int32_t *page_table,
-                         const int32_t *seq_lens, float *bbox, float *mu,
-                         float *sigma, void *stream);
+                         const void *meta, const int32_t *seq_lens, float *bbox,
+                         float *mu, float *sigma, void *stream);
 
 /*
  * Section 2.B (candidate selection), per (b, h), written to

@@ -157,7 +157,7 @@ int entmaxkv_version(void) { return 100; }
 
 size_t entmaxkv_meta_bytes(const entmaxkv_shape *s) {
     if (check_shape(s)) return 0;
-    return (size_t)s->num_blocks * s->Hkv * 12 * s->d;
+    return (size_t)s->B * s->Hkv * meta_tiles(s->max_pages) * META_TILE * 12 * s->d;
 }
 
 size_t entmaxkv_workspace_size(const entmaxkv_shape *s, int call) {
@@ -203,7 +203,8 @@ int entmaxkv_build_meta(const entmaxkv_shape *s, const void *k_cache, const int3
     a.page_table = page_table;
     a.seq_lens = seq_lens;
     a.meta = static_cast<uint8_t *>(meta);
-    a.R = (long long)s->num_blocks * s->Hkv;
+    a.n_tiles = meta_tiles(s->max_pages);
+    a.n_tiles_total = (long long)s->B * s->Hkv * a.n_tiles;
     a.B = s->B;
     a.Hkv = s->Hkv;
     a.d = s->d;
@@ -216,11 +217,11 @@ int entmaxkv_build_meta(const entmaxkv_shape *s, const void *k_cache, const int3
     return cuda_rc(launch_build_meta(a, static_cast<cudaStream_t>(stream)));
 }
 
-int entmaxkv_score_pages(const entmaxkv_shape *s, const void *q, const void *meta, const int32_t *page_table,
-                         const int32_t *seq_lens, float *bbox, float *mu, float *sigma, void *stream) {
+int entmaxkv_score_pages(const entmaxkv_shape *s, const void *q, const void *meta, const int32_t *seq_lens,
+                         float *bbox, float *mu, float *sigma, void *stream) {
     int rc = check_shape(s);
     if (rc) return rc;
-    if (!q || !meta || !page_table || !seq_lens || !bbox) return ENTMAXKV_ERR_NULL;
+    if (!q || !meta || !seq_lens || !bbox) return ENTMAXKV_ERR_NULL;
     if ((mu == nullptr) != (sigma == nullptr)) return ENTMAXKV_ERR_NULL;
     if (!aligned16(q) || !aligned16(meta)) return ENTMAXKV_ERR_ALIGN;
     DevInfo di;
@@ -228,19 +229,18 @@ int entmaxkv_score_pages(const entmaxkv_shape *s, const void *q, const void *met
     ScoreArgs a{};
     a.q = static_cast<const uint16_t *>(q);
     a.meta = static_cast<const uint8_t *>(meta);
-    a.page_table = page_table;
     a.seq_lens = seq_lens;
     a.bbox = bbox;
     a.mu = mu;
     a.sigma = sigma;
-    a.R = (long long)s->num_blocks * s->Hkv;
+    a.n_tiles = meta_tiles(s->max_pages);
+    a.n_tiles_total = (long long)s->B * s->Hkv * a.n_tiles;
     a.B = s->B;
     a.Hq = s->Hq;
     a.Hkv = s->Hkv;
     a.d = s->d;
     a.P = s->page_size;
     a.max_pages = s->max_pages;
-    a.num_blocks = s->num_blocks;
     a.status = di.status;
     return cuda_rc(launch_score_pages(a, static_cast<cudaStream_t>(stream)));
 }

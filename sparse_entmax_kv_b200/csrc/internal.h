@@ -17,12 +17,17 @@ struct DevInfo {
     int *status;  // device address of the status word
 };
 
+// Pages per metadata tile and the tile count of one (sequence, kv head).
+constexpr int META_TILE = 32;
+inline int meta_tiles(int max_pages) { return (max_pages + META_TILE - 1) / META_TILE; }
+
 struct MetaArgs {
     const uint16_t *k;
     const int *page_table;
     const int *seq_lens;
     uint8_t *meta;
-    long long R;  // records = num_blocks * Hkv
+    int n_tiles;              // tiles per (sequence, kv head)
+    long long n_tiles_total;  // B * Hkv * n_tiles
     int B, Hkv, d, P, max_pages, num_blocks;
     int first_page, n_pages;  // n_pages >= 0 here (resolved by the caller)
     int *status;
@@ -32,11 +37,11 @@ cudaError_t launch_build_meta(const MetaArgs &a, cudaStream_t st);
 struct ScoreArgs {
     const uint16_t *q;
     const uint8_t *meta;
-    const int *page_table;
     const int *seq_lens;
     float *bbox, *mu, *sigma;
-    long long R;
-    int B, Hq, Hkv, d, P, max_pages, num_blocks;
+    int n_tiles;
+    long long n_tiles_total;
+    int B, Hq, Hkv, d, P, max_pages;
     int *status;
 };
 cudaError_t launch_score_pages(const ScoreArgs &a, cudaStream_t st);

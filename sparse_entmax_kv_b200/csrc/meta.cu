@@ -6,6 +6,8 @@
 // the page's valid tokens in order.  Sums run in fp64 (every bf16 value and
 // square is exact there) and are rounded once to fp32, so the record is
 // defined to the bit:  mean = fp32(S1/n), var = fp32(max(0, S2/n - (S1/n)^2)).
+// The record is stored at its logical page in the tiled, swizzled layout the
+// scoring pass streams (include/entmaxkv.h, entmaxkv_meta_bytes).
 #include "common.cuh"
 #include "internal.h"
 
@@ -24,7 +26,7 @@ __global__ void __launch_bounds__(D) build_meta_kernel(MetaArgs a) {
         return;
     }
     const int n = tokens_in_page(seq, P, p);
-    const long long rec = (long long)blk * a.Hkv + kvh;
+    const long long rec = (long long)blk * a.Hkv + kvh;  // the page's keys: k_cache[blk][kvh]
     const int j = threadIdx.x;
     const uint16_t *col = a.k + (size_t)rec * P * D + j;
 
@@ -52,12 +54,17 @@ __global__ void __launch_bounds__(D) build_meta_kernel(MetaArgs a) {
     double v = __dsub_rn(__ddiv_rn(s2, dn), __dmul_rn(m, m));
     if (v < 0.0) v = 0.0;
 
-    uint16_t *bb = reinterpret_cast<uint16_t *>(a.meta + (size_t)rec * 4 * D);
-    bb[j] = bmin;
-    bb[D + j] = bmax;
-    float *mm = reinterpret_cast<float *>(a.meta + (size_t)a.R * 4 * D + (size_t)rec * 8 * D);
-    mm[j] = (float)m;
-    mm[D + j] = (float)v;
+    const int tile = p / META_TILE, sl = p % META_TILE;
+    const long long T = ((long long)b * a.Hkv + kvh) * a.n_tiles + tile;
+    const int c = j / 16, e = j % 16;
+    uint8_t *bb = a.meta + T * 128 * D + c * 2048;
+    const int ob = sl * 32 + 16 * ((e >> 3) ^ ((sl >> 2) & 1)) + 2 * (e & 7);
+    *reinterpret_cast<uint16_t *>(bb + ob) = bmin;
+    *reinterpret_cast<uint16_t *>(bb + 1024 + ob) = bmax;
+    uint8_t *mm = a.meta + a.n_tiles_total * 128 * D + T * 256 * D + c * 4096;
+    const int om = sl * 64 + 16 * ((e >> 2) ^ ((sl >> 1) & 3)) + 4 * (e & 3);
+    *reinterpret_cast<float *>(mm + om) = (float)m;
+    *reinterpret_cast<float *>(mm + 2048 + om) = (float)v;
 }
 
 template <int D>

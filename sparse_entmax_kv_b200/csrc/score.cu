@@ -4,22 +4,24 @@
 //   bbox  = (sum_j max(q_j kmin_j, q_j kmax_j)) / sqrt(d)   upper bound on s
 //   mu    = (sum_j q_j mean_j) / sqrt(d)                    Gaussian mean
 //   sigma = sqrt((sum_j q_j^2 var_j) / d)                   Gaussian std
-// The bound is one fp64 chain over j in index order with exact products, so
-// it is reproducible to the bit; max(q a, q b) with a <= b is q b for q >= 0
-// and q a otherwise, one fused multiply-add per coordinate.  mu and sigma feed
-// only the approximate tau_hat; they are fp32 chains over j in index order.
 //
-// Layout of the work: a CTA owns 256 consecutive logical pages of one
-// (b, kv head); thread = page, and the thread scores that page for all G query
-// heads of the group, so each metadata record crosses HBM once per group.
-// Records are streamed through a per-warp ring of 8-coordinate chunks with
-// 16-byte cp.async copies: the 32 records of a warp are fetched cooperatively
-// (consecutive lanes take consecutive 16-byte pieces of a record, so whole
-// 32-byte sectors move per instruction) into padded per-thread slots, and each
-// thread then reads its own slot.  The slot pitch keeps the 16-byte reads of
-// any 8 consecutive lanes on distinct banks.  q is kept in shared memory
-// coordinate-major ([j][head]) so one vector load serves all heads of a
-// coordinate.
+// The bound is one fp64 chain over j in index order, so it is reproducible to
+// the bit.  max(q a, q b) with a <= b equals q- a + q+ b, q+ = max(q, 0) and
+// q- = min(q, 0): one of the two products is an exact zero, so two fused
+// multiply-adds per coordinate add exactly the oracle's term with no select.
+// mu and sigma feed only the approximate tau_hat; they are fp32 sums kept as
+// two interleaved chains (even and odd j) so that packed f32x2 FMAs do two
+// coordinates per instruction.
+//
+// Layout of the work: the metadata sits in logical page order, in tiles of 32
+// pages whose 16-coordinate chunk blocks are contiguous (see include/
+// entmaxkv.h).  A warp owns one tile: lane = page.  It streams the tile chunk
+// by chunk through a two-stage ring in shared memory, each stage filled by
+// two 1-D bulk copies (2 KB of bounds, 4 KB of moments) completing on an
+// mbarrier, so HBM sees long contiguous reads and the SM issues no per-lane
+// copy instructions.  Each lane scores its page for all G query heads of the
+// group, so every byte crosses HBM once per group.  q sits in shared memory
+// as q+ and q- (fp64, [j][head]) and fp32 ([head][j]).
 #include "common.cuh"
 #include "internal.h"
 
@@ -27,154 +29,137 @@ namespace ekv {
 
 namespace {
 
-constexpr int SC_THREADS = 256;
-constexpr int SC_WARPS = SC_THREADS / 32;
-constexpr int CH = 8;  // coordinates per chunk
+constexpr int TP = 32;       // pages per tile (= lanes)
+constexpr int CHK = 16;      // coordinates per chunk
+constexpr int WARPS = 8;
+constexpr int THREADS = WARPS * 32;
+constexpr int BOUND_CHUNK = 128 * CHK;  // kmin + kmax block of one chunk: 2048 B
+constexpr int MOM_CHUNK = 256 * CHK;    // mean + var block of one chunk:  4096 B
 
 template <bool GAUSS>
-struct ScoreCfg {
-    static constexpr int PIECES = GAUSS ? 6 : 2;   // 16-byte pieces per record chunk
-    static constexpr int SLOT = PIECES * 16 + 16;  // padded slot pitch (bytes)
-    static constexpr int NST = GAUSS ? 3 : 6;      // ring depth (chunks in flight per warp)
-    static constexpr int WARP_STAGE = 32 * SLOT;
+struct Ring {
+    static constexpr int STAGE = GAUSS ? BOUND_CHUNK + MOM_CHUNK : BOUND_CHUNK;
+    static constexpr int NST = GAUSS ? 2 : 4;
 };
 
 template <int D, int G>
-struct QLayout {
-    // qd: [D][G] fp64; qf: [D][G] fp32 (the same bf16 values)
-    static constexpr int D_BYTES = D * G * 8;
-    static constexpr int F_BYTES = D * G * 4;
-    static constexpr int BYTES = D_BYTES + F_BYTES;
+struct QBytes {
+    static constexpr int VALUE = D * G * 8 * 2 + D * G * 4;
 };
 
 template <int D, int G, bool GAUSS>
-__global__ void __launch_bounds__(SC_THREADS, 2) score_kernel(ScoreArgs a) {
-    using Cfg = ScoreCfg<GAUSS>;
-    using QL = QLayout<D, G>;
-    constexpr int NCH = D / CH;
-    extern __shared__ __align__(16) unsigned char smem[];
-    double *qd = reinterpret_cast<double *>(smem);
-    float *qf = reinterpret_cast<float *>(smem + QL::D_BYTES);
-    unsigned char *ring = smem + QL::BYTES;
+constexpr size_t smem_bytes() {
+    return ((QBytes<D, G>::VALUE + WARPS * Ring<GAUSS>::NST * 8 + 127) & ~size_t(127)) +
+           (size_t)WARPS * Ring<GAUSS>::NST * Ring<GAUSS>::STAGE;
+}
+
+template <int D, int G, bool GAUSS>
+__global__ void __launch_bounds__(THREADS, G <= 4 ? 2 : 1) score_kernel(ScoreArgs a) {
+    using RG = Ring<GAUSS>;
+    constexpr int NCH = D / CHK;
+    constexpr int NST = RG::NST;
+    extern __shared__ __align__(128) unsigned char smem[];
+    double *qp = reinterpret_cast<double *>(smem);  // [D][G] max(q, 0)
+    double *qn = qp + D * G;                         // [D][G] min(q, 0)
+    float *qh = reinterpret_cast<float *>(qn + D * G);  // [G][D] q
+    uint64_t *bars = reinterpret_cast<uint64_t *>(smem + QBytes<D, G>::VALUE);
+    unsigned char *ring = smem + ((QBytes<D, G>::VALUE + WARPS * NST * 8 + 127) & ~127);
 
     const int bk = blockIdx.y;
     const int b = bk / a.Hkv, kvh = bk % a.Hkv;
     const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
 
-    for (int i = threadIdx.x; i < G * D; i += SC_THREADS) {
+    for (int i = threadIdx.x; i < G * D; i += THREADS) {
         const int g = i / D, j = i % D;
         const float v = bf16f(a.q[((size_t)b * a.Hq + kvh * G + g) * D + j]);
-        qd[j * G + g] = (double)v;
-        qf[j * G + g] = v;
+        qp[j * G + g] = v > 0.f ? (double)v : 0.0;
+        qn[j * G + g] = v < 0.f ? (double)v : 0.0;
+        qh[g * D + j] = v;
     }
+    if (threadIdx.x < WARPS * NST) mbar_init(&bars[threadIdx.x], 1);
+    mbar_fence_init();
     __syncthreads();
 
-    const int seq = a.seq_lens[b];
-    const int np = n_pages_of(seq, a.P);
-    const int page0 = blockIdx.x * SC_THREADS + warp * 32;
+    const int np = n_pages_of(a.seq_lens[b], a.P);
+    const int tile = blockIdx.x * WARPS + warp;
+    const int page0 = tile * TP;
     if (page0 >= np) return;  // whole warp past the end
-    const int page = page0 + lane;
-    long long rec = -1;
-    if (page < np) {
-        int blk = a.page_table[(size_t)b * a.max_pages + page];
-        if (blk >= 0 && blk < a.num_blocks)
-            rec = (long long)blk * a.Hkv + kvh;
-        else
-            atomicOr(a.status, ENTMAXKV_STATUS_BAD_PAGE);
-    }
 
-    // Piece i*32+lane of a chunk belongs to record (i*32+lane)/PIECES.  Piece
-    // 0 is kmin, 1 kmax (bound region: kmin at [0,2D) bytes of the record,
-    // kmax at [2D,4D), chunk c adds 16c); pieces 2-3 are mean, 4-5 var
-    // (moment region: mean at [0,4D), var at [4D,8D), chunk c adds 32c).
-    const unsigned char *src[Cfg::PIECES];
-    int dst_off[Cfg::PIECES];
-#pragma unroll
-    for (int i = 0; i < Cfg::PIECES; ++i) {
-        const int idx = i * 32 + lane;
-        const int rl = idx / Cfg::PIECES, pc = idx % Cfg::PIECES;
-        const long long r = __shfl_sync(FULL, rec, rl);
-        dst_off[i] = rl * Cfg::SLOT + pc * 16;
-        if (r < 0) {
-            src[i] = nullptr;
-        } else if (pc < 2) {
-            src[i] = a.meta + (size_t)r * 4 * D + pc * 2 * D;
-        } else {
-            src[i] = a.meta + (size_t)a.R * 4 * D + (size_t)r * 8 * D +
-                     (pc < 4 ? (pc - 2) * 16 : 4 * D + (pc - 4) * 16);
-        }
-    }
+    const long long T = ((long long)b * a.Hkv + kvh) * a.n_tiles + tile;
+    const unsigned char *gb = a.meta + T * 128 * D;
+    const unsigned char *gm = a.meta + (size_t)a.n_tiles_total * 128 * D + T * 256 * D;
+    unsigned char *wring = ring + warp * NST * RG::STAGE;
+    uint64_t *wbar = bars + warp * NST;
 
-    unsigned char *wring = ring + warp * Cfg::NST * Cfg::WARP_STAGE;
     auto issue = [&](int c) {
-        unsigned char *st = wring + (c % Cfg::NST) * Cfg::WARP_STAGE;
-#pragma unroll
-        for (int i = 0; i < Cfg::PIECES; ++i) {
-            if (src[i] == nullptr) continue;
-            // bound pieces sit in the first 32 bytes of the slot
-            const int cstride = dst_off[i] % Cfg::SLOT < 32 ? 16 : 32;
-            cp_async16(st + dst_off[i], src[i] + c * cstride);
+        if (lane == 0) {
+            unsigned char *st = wring + (c % NST) * RG::STAGE;
+            uint64_t *bar = &wbar[c % NST];
+            mbar_arrive_expect_tx(bar, RG::STAGE);
+            bulk_g2s(st, gb + c * BOUND_CHUNK, BOUND_CHUNK, bar);
+            if (GAUSS) bulk_g2s(st + BOUND_CHUNK, gm + c * MOM_CHUNK, MOM_CHUNK, bar);
         }
     };
-
 #pragma unroll
-    for (int c = 0; c < Cfg::NST - 1; ++c) {
+    for (int c = 0; c < NST - 1; ++c)
         if (c < NCH) issue(c);
-        cp_async_commit();
-    }
 
     double ab[G];
-    float am[G], av[G];
+    float2 am[G], av[G];
 #pragma unroll
     for (int g = 0; g < G; ++g) {
         ab[g] = 0.0;
-        am[g] = av[g] = 0.f;
+        am[g] = av[g] = make_float2(0.f, 0.f);
     }
-
-    const unsigned char *myslot0 = wring + lane * Cfg::SLOT;
+    const int s = lane;
+    const int xb = (s >> 2) & 1, xm = (s >> 1) & 3;  // the layout's swizzles
+    bool ok = true;
     for (int c = 0; c < NCH; ++c) {
-        if (c + Cfg::NST - 1 < NCH) issue(c + Cfg::NST - 1);
-        cp_async_commit();
-        cp_async_wait<Cfg::NST - 1>();
-        __syncwarp();
-        const unsigned char *slot = myslot0 + (c % Cfg::NST) * Cfg::WARP_STAGE;
-        const uint4 kn = *reinterpret_cast<const uint4 *>(slot + 0);
-        const uint4 kx = *reinterpret_cast<const uint4 *>(slot + 16);
-        const unsigned wn[4] = {kn.x, kn.y, kn.z, kn.w};
-        const unsigned wx[4] = {kx.x, kx.y, kx.z, kx.w};
-        float mv[CH], vv[CH];
-        if (GAUSS) {
+        if (c + NST - 1 < NCH) issue(c + NST - 1);
+        ok &= mbar_wait(&wbar[c % NST], (c / NST) & 1, a.status);
+        const unsigned char *st = wring + (c % NST) * RG::STAGE;
 #pragma unroll
-            for (int i = 0; i < 2; ++i) {
-                float4 m4 = *reinterpret_cast<const float4 *>(slot + 32 + 16 * i);
-                float4 v4 = *reinterpret_cast<const float4 *>(slot + 64 + 16 * i);
-                mv[4 * i] = m4.x; mv[4 * i + 1] = m4.y; mv[4 * i + 2] = m4.z; mv[4 * i + 3] = m4.w;
-                vv[4 * i] = v4.x; vv[4 * i + 1] = v4.y; vv[4 * i + 2] = v4.z; vv[4 * i + 3] = v4.w;
+        for (int hf = 0; hf < 2; ++hf) {  // two halves of 8 coordinates
+            const uint4 kn = *reinterpret_cast<const uint4 *>(st + s * 32 + 16 * (hf ^ xb));
+            const uint4 kx = *reinterpret_cast<const uint4 *>(st + 1024 + s * 32 + 16 * (hf ^ xb));
+            const unsigned wn[4] = {kn.x, kn.y, kn.z, kn.w};
+            const unsigned wx[4] = {kx.x, kx.y, kx.z, kx.w};
+            const int j0 = c * CHK + 8 * hf;
+            if (GAUSS) {
+#pragma unroll
+                for (int qt = 0; qt < 2; ++qt) {  // quarters of 4 coordinates
+                    const int pc = (2 * hf + qt) ^ xm;
+                    const float4 m4 = *reinterpret_cast<const float4 *>(st + BOUND_CHUNK + s * 64 + 16 * pc);
+                    const float4 v4 = *reinterpret_cast<const float4 *>(st + BOUND_CHUNK + 2048 + s * 64 + 16 * pc);
+#pragma unroll
+                    for (int g = 0; g < G; ++g) {
+                        const float4 q4 = *reinterpret_cast<const float4 *>(qh + g * D + j0 + 4 * qt);
+                        const float2 q01 = make_float2(q4.x, q4.y), q23 = make_float2(q4.z, q4.w);
+                        am[g] = __ffma2_rn(q01, make_float2(m4.x, m4.y), am[g]);
+                        am[g] = __ffma2_rn(q23, make_float2(m4.z, m4.w), am[g]);
+                        av[g] = __ffma2_rn(__fmul2_rn(q01, q01), make_float2(v4.x, v4.y), av[g]);  // q^2 exact
+                        av[g] = __ffma2_rn(__fmul2_rn(q23, q23), make_float2(v4.z, v4.w), av[g]);
+                    }
+                }
             }
-        }
-        const double *qdc = qd + (size_t)c * CH * G;
-        const float *qfc = qf + c * CH * G;
 #pragma unroll
-        for (int jj = 0; jj < CH; ++jj) {
-            const unsigned w_n = wn[jj >> 1], w_x = wx[jj >> 1];
-            const double lo = (double)((jj & 1) ? bf16hi(w_n) : bf16lo(w_n));
-            const double hi = (double)((jj & 1) ? bf16hi(w_x) : bf16lo(w_x));
+            for (int jj = 0; jj < 8; ++jj) {
+                const unsigned w_n = wn[jj >> 1], w_x = wx[jj >> 1];
+                const double lo = (double)((jj & 1) ? bf16hi(w_n) : bf16lo(w_n));
+                const double hi = (double)((jj & 1) ? bf16hi(w_x) : bf16lo(w_x));
+                const int j = j0 + jj;
 #pragma unroll
-            for (int g = 0; g < G; ++g) {
-                const double qv = qdc[jj * G + g];
-                ab[g] = __fma_rn(qv, (__double2hiint(qv) < 0) ? lo : hi, ab[g]);
-                if (GAUSS) {
-                    const float qs = qfc[jj * G + g];
-                    am[g] = __fmaf_rn(qs, mv[jj], am[g]);
-                    av[g] = __fmaf_rn(__fmul_rn(qs, qs), vv[jj], av[g]);  // q^2 exact in fp32
+                for (int g = 0; g < G; ++g) {
+                    ab[g] = __fma_rn(qn[j * G + g], lo, ab[g]);
+                    ab[g] = __fma_rn(qp[j * G + g], hi, ab[g]);
                 }
             }
         }
-        __syncwarp();
+        __syncwarp();  // every lane is done with this stage before it is refilled
     }
-    cp_async_wait<0>();
 
-    if (rec < 0) return;
+    const int page = page0 + lane;
+    if (!ok || page >= np) return;
     const double inv_sqrt_d = __ddiv_rn(1.0, __dsqrt_rn((double)D));
     const float inv_sqrt_df = D == 64 ? 0.125f : 0.08838834764831845f;
 #pragma unroll
@@ -182,21 +167,20 @@ __global__ void __launch_bounds__(SC_THREADS, 2) score_kernel(ScoreArgs a) {
         const size_t o = ((size_t)b * a.Hq + kvh * G + g) * a.max_pages + page;
         a.bbox[o] = (float)__dmul_rn(ab[g], inv_sqrt_d);
         if (GAUSS) {
-            a.mu[o] = am[g] * inv_sqrt_df;
-            a.sigma[o] = sqrtf(av[g] * (1.f / (float)D));
+            a.mu[o] = (am[g].x + am[g].y) * inv_sqrt_df;
+            a.sigma[o] = sqrtf((av[g].x + av[g].y) * (1.f / (float)D));
         }
     }
 }
 
 template <int D, int G, bool GAUSS>
 cudaError_t launch_t(const ScoreArgs &a, cudaStream_t st) {
-    using Cfg = ScoreCfg<GAUSS>;
-    const size_t smem = QLayout<D, G>::BYTES + (size_t)SC_WARPS * Cfg::NST * Cfg::WARP_STAGE;
+    constexpr size_t smem = smem_bytes<D, G, GAUSS>();
     auto kern = score_kernel<D, G, GAUSS>;
     cudaError_t e = ensure_smem(reinterpret_cast<const void *>(kern), smem);
     if (e != cudaSuccess) return e;
-    dim3 grid(ceil_div(a.max_pages, SC_THREADS), a.B * a.Hkv);
-    kern<<<grid, SC_THREADS, smem, st>>>(a);
+    dim3 grid(ceil_div(a.n_tiles, WARPS), a.B * a.Hkv);
+    kern<<<grid, THREADS, smem, st>>>(a);
     return cudaGetLastError();
 }
 

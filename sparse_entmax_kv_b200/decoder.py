@@ -54,7 +54,7 @@ class EntmaxKVDecoder:
         if append_page is not None:
             nv.entmaxkv_build_meta(self.shape, self.k_cache, self.page_table, self.seq_lens,
                                    append_page, 1, self.meta)
-        nv.entmaxkv_score_pages(self.shape, q, self.meta, self.page_table, self.seq_lens,
+        nv.entmaxkv_score_pages(self.shape, q, self.meta, self.seq_lens,
                                 self.bbox, self.mu, self.sigma)
         nv.entmaxkv_select(self.shape, self.seq_lens, self.bbox, self.mu, self.sigma, self.policy,
                            self.k, self.alpha, self.delta, self.sel, self.cnt, self.tau_hat)

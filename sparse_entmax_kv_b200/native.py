@@ -74,7 +74,7 @@ def lib():
         L.entmaxkv_workspace_size.argtypes = [sp, C.c_int]
         L.entmaxkv_get_status.argtypes = [C.POINTER(i32), C.c_int, vp]
         L.entmaxkv_build_meta.argtypes = [sp, vp, vp, vp, i32, i32, vp, vp]
-        L.entmaxkv_score_pages.argtypes = [sp, vp, vp, vp, vp, vp, vp, vp, vp]
+        L.entmaxkv_score_pages.argtypes = [sp, vp, vp, vp, vp, vp, vp, vp]
         L.entmaxkv_select.argtypes = [sp, vp, vp, vp, vp, i32, i32, f32, f32, vp, vp, vp, vp, sz, vp]
         L.entmaxkv_decode_sparse.argtypes = [sp, vp, vp, vp, vp, vp, vp, vp, f32, vp, vp, vp, vp, sz, vp]
         L.entmaxkv_decode_dense.argtypes = [sp, vp, vp, vp, vp, vp, f32, vp, vp, vp, vp, sz, vp]
@@ -144,10 +144,10 @@ def entmaxkv_build_meta(shape, k_cache, page_table, seq_lens, first_page, n_page
         _stream(stream)))
 
 
-def entmaxkv_score_pages(shape, q, meta, page_table, seq_lens, bbox, mu=None, sigma=None, stream=None):
+def entmaxkv_score_pages(shape, q, meta, seq_lens, bbox, mu=None, sigma=None, stream=None):
     _check("entmaxkv_score_pages", lib().entmaxkv_score_pages(
         C.byref(shape), _ptr(q, torch.bfloat16, "q"), _ptr(meta, None, "meta"),
-        _ptr(page_table, torch.int32, "page_table"), _ptr(seq_lens, torch.int32, "seq_lens"),
+        _ptr(seq_lens, torch.int32, "seq_lens"),
         _ptr(bbox, torch.float32, "bbox"), _ptr(mu, torch.float32, "mu"), _ptr(sigma, torch.float32, "sigma"),
         _stream(stream)))
 

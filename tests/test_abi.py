@@ -45,7 +45,8 @@ def shp(**kw):
 
 def test_sizes():
     s = shp()
-    assert nv.meta_bytes(s) == 128 * 2 * 12 * 128
+    assert nv.meta_bytes(s) == 2 * 2 * 2 * 32 * 12 * 128    # B * Hkv * ceil(64/32) tiles * 32 pages * 12d
+    assert nv.meta_bytes(shp(max_pages=65)) == 2 * 2 * 3 * 32 * 12 * 128
     assert nv.workspace_size(s, nv.CALL_SELECT) == 0
     ws = nv.workspace_size(s, nv.CALL_DECODE_SPARSE)
     assert ws >= 2 * 8 * 64 * 32 * 4            # z of every token of the page list
@@ -62,7 +63,7 @@ def test_bad_shapes_rejected_everywhere(bad):
     s = C.byref(shp(**bad))
     E = -2
     assert L.entmaxkv_build_meta(s, FAKE, FAKE, FAKE, 0, -1, FAKE, None) == E
-    assert L.entmaxkv_score_pages(s, FAKE, FAKE, FAKE, FAKE, FAKE, None, None, None) == E
+    assert L.entmaxkv_score_pages(s, FAKE, FAKE, FAKE, FAKE, None, None, None) == E
     assert L.entmaxkv_select(s, FAKE, FAKE, None, None, 0, 4, 1.5, 0.0, FAKE, FAKE, None, None, 0, None) == E
     assert L.entmaxkv_decode_sparse(s, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, 1.5, FAKE, None, None,
                                     FAKE, 1 << 40, None) == E
@@ -78,8 +79,9 @@ def test_null_alignment_and_argument_codes():
     assert L.entmaxkv_build_meta(s, FAKE_ODD, FAKE, FAKE, 0, -1, FAKE, None) == -8
     assert L.entmaxkv_build_meta(s, FAKE, FAKE, FAKE, -1, -1, FAKE, None) == -2
     assert L.entmaxkv_build_meta(s, FAKE, FAKE, FAKE, 0, -2, FAKE, None) == -2
-    assert L.entmaxkv_score_pages(s, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, None, None) == -1  # mu w/o sigma
-    assert L.entmaxkv_score_pages(s, FAKE_ODD, FAKE, FAKE, FAKE, FAKE, None, None, None) == -8
+    assert L.entmaxkv_score_pages(s, FAKE, FAKE, FAKE, FAKE, FAKE, None, None) == -1  # mu w/o sigma
+    assert L.entmaxkv_score_pages(s, FAKE, FAKE, None, FAKE, None, None, None) == -1  # no seq_lens
+    assert L.entmaxkv_score_pages(s, FAKE_ODD, FAKE, FAKE, FAKE, None, None, None) == -8
     # select
     sel = lambda pol, k, a, dl, mu=FAKE: L.entmaxkv_select(s, FAKE, FAKE, mu, mu, pol, k, a, dl, FAKE, FAKE,
                                                            None, None, 0, None)

@@ -59,11 +59,32 @@ def shape_of(wl):
     return nv.Shape(wl.B, wl.Hq, wl.Hkv, wl.d, wl.P, wl.max_pages, wl.num_blocks)
 
 
-def unpack_meta(meta: torch.Tensor, R: int, d: int):
+def unpack_meta(meta: torch.Tensor, wl, page_table, seq_lens):
+    """Decode the library's metadata (32-page tiles in logical page order,
+    16-coordinate chunks, swizzled 16-byte pieces: include/entmaxkv.h) into
+    kmin, kmax, mean, var arrays indexed like the oracle's, [block*Hkv + kv
+    head][d].  Rows of blocks no valid page maps to stay zero."""
+    d, Hkv, B = wl.d, wl.Hkv, wl.B
+    nt = -(-wl.max_pages // 32)
+    NT, nch = B * Hkv * nt, d // 16
     m = meta.cpu().numpy()
-    bb = m[:R * 4 * d].view(np.uint16).reshape(R, 2, d)
-    mo = m[R * 4 * d:R * 12 * d].view(np.float32).reshape(R, 2, d)
-    return bb[:, 0], bb[:, 1], mo[:, 0], mo[:, 1]
+    assert m.size == NT * 384 * d
+    slot = np.arange(32)[:, None]
+    bnd = m[:NT * 128 * d].view(np.uint16).reshape(NT, nch, 2, 32, 2, 8)
+    bnd = bnd[:, :, :, slot, np.arange(2)[None, :] ^ ((slot >> 2) & 1), :]
+    mom = m[NT * 128 * d:].view(np.float32).reshape(NT, nch, 2, 32, 4, 4)
+    mom = mom[:, :, :, slot, np.arange(4)[None, :] ^ ((slot >> 1) & 3), :]
+    logical = [x[:, :, part].transpose(0, 2, 1, 3, 4).reshape(B, Hkv, nt * 32, d)
+               for x in (bnd, mom) for part in (0, 1)]
+    pt = np.asarray(page_table)
+    seq = np.asarray(seq_lens)
+    out = [np.zeros((wl.num_blocks * Hkv, d), x.dtype) for x in logical]
+    for b in range(B):
+        npb = -(-int(seq[b]) // wl.P)
+        rows = (pt[b, :npb].astype(np.int64)[None, :] * Hkv + np.arange(Hkv)[:, None])  # [Hkv][npb]
+        for o, x in zip(out, logical):
+            o[rows.reshape(-1)] = x[b, :, :npb].reshape(-1, d)
+    return tuple(out)
 
 
 def referenced_records(host, wl):
@@ -141,8 +162,7 @@ def test_meta_and_scores_bit_exact(name):
     s = shape_of(wl)
     meta = nv.alloc_meta(s, "cuda")
     nv.entmaxkv_build_meta(s, inp["k_cache"], inp["page_table"], inp["seq_lens"], 0, -1, meta)
-    R = wl.num_blocks * wl.Hkv
-    g = unpack_meta(meta, R, wl.d)
+    g = unpack_meta(meta, wl, host["page_table"], host["seq_lens"])
     o = orc.build_meta(host["K"], host["page_table"], host["seq_lens"], wl.Hkv, wl.d, wl.P, wl.num_blocks)
     recs = referenced_records(host, wl)
     for gi, oi, nm in zip(g, o, ("kmin", "kmax", "mean", "var")):
@@ -151,7 +171,7 @@ def test_meta_and_scores_bit_exact(name):
                                       err_msg=nm)
     B, Hq, mp = wl.B, wl.Hq, wl.max_pages
     out = [torch.full((B, Hq, mp), float("nan"), device="cuda") for _ in range(3)]
-    nv.entmaxkv_score_pages(s, inp["q"], meta, inp["page_table"], inp["seq_lens"], *out)
+    nv.entmaxkv_score_pages(s, inp["q"], meta, inp["seq_lens"], *out)
     ob = orc.score_pages(host["q"], o, host["page_table"], host["seq_lens"], wl.Hkv, wl.P)
     gb, gm, gs = (t.cpu().numpy() for t in out)
     for b in range(B):
@@ -163,7 +183,7 @@ def test_meta_and_scores_bit_exact(name):
                        o[2], o[3], recs, f"b{b}")
     # bound-only scoring gives the same bound
     bb2 = torch.full((B, Hq, mp), float("nan"), device="cuda")
-    nv.entmaxkv_score_pages(s, inp["q"], meta, inp["page_table"], inp["seq_lens"], bb2)
+    nv.entmaxkv_score_pages(s, inp["q"], meta, inp["seq_lens"], bb2)
     for b in range(B):
         npb = n_pages(host, wl, b)
         assert torch.equal(bb2[b, :, :npb], out[0][b, :, :npb])
@@ -330,8 +350,8 @@ def test_append_rebuild_matches_full_build():
     nv.entmaxkv_build_meta(s, inp["k_cache"], inp["page_table"], inp["seq_lens"], p_last, 1, meta)
     full = nv.alloc_meta(s, "cuda")
     nv.entmaxkv_build_meta(s, inp["k_cache"], inp["page_table"], inp["seq_lens"], 0, -1, full)
-    R = wl.num_blocks * wl.Hkv
-    a, c = unpack_meta(meta, R, wl.d), unpack_meta(full, R, wl.d)
+    pt, sl = inp["page_table"].cpu().numpy(), inp["seq_lens"].cpu().numpy()
+    a, c = unpack_meta(meta, wl, pt, sl), unpack_meta(full, wl, pt, sl)
     for b2 in range(wl.B):
         for p in range(-(-int(inp["seq_lens"][b2]) // wl.P)):
             bl = int(inp["page_table"][b2, p])
@@ -373,8 +393,7 @@ def test_full_size_step_sampled(name):
     dec.build_meta()
     dec.step(inp["q"])
     torch.cuda.synchronize()
-    R = wl.num_blocks * wl.Hkv
-    gmeta = unpack_meta(dec.meta, R, wl.d)
+    gmeta = unpack_meta(dec.meta, wl, inp["page_table"].cpu().numpy(), inp["seq_lens"].cpu().numpy())
     rng = np.random.default_rng(0)
     groups = [(0, 0), (wl.B - 1, wl.Hkv - 1), (int(rng.integers(wl.B)), int(rng.integers(wl.Hkv)))]
     G = wl.G
