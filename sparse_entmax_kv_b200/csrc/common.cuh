@@ -117,6 +117,38 @@ __device__ __forceinline__ void cp_async_wait() {
     asm volatile("cp.async.wait_group %0;" ::"n"(N) : "memory");
 }
 
+// ------------------------------------------------------- thread-block clusters
+
+__device__ __forceinline__ unsigned cl_rank() {
+    unsigned r;
+    asm volatile("mov.u32 %0, %%cluster_ctarank;" : "=r"(r));
+    return r;
+}
+// Barrier over every thread of every CTA of the cluster; shared-memory
+// writes (local or pushed into a peer) before it are visible after it.
+__device__ __forceinline__ void cl_sync() {
+    __syncwarp();
+    asm volatile(
+        "barrier.cluster.arrive.release.aligned;\n\t"
+        "barrier.cluster.wait.acquire.aligned;" ::
+            : "memory");
+}
+// Address of `p` (a shared variable of this CTA) in the CTA of rank `rank`.
+__device__ __forceinline__ unsigned cl_map(const void *p, unsigned rank) {
+    unsigned r;
+    asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(r) : "r"(smem_u32(p)), "r"(rank));
+    return r;
+}
+// Stores into a peer CTA's shared memory (visible there after the next
+// cluster barrier).  Exchanges push data to the CTAs that read it, so every
+// read after a barrier is local.
+__device__ __forceinline__ void cl_stf(unsigned addr, float v) {
+    asm volatile("st.shared::cluster.f32 [%0], %1;" ::"r"(addr), "f"(v) : "memory");
+}
+__device__ __forceinline__ void cl_sti(unsigned addr, int v) {
+    asm volatile("st.shared::cluster.s32 [%0], %1;" ::"r"(addr), "r"(v) : "memory");
+}
+
 // ------------------------------------------------------------ tensor cores
 
 // ldmatrix x4 (four 8x8 b16 matrices), one row address per lane.

@@ -25,36 +25,11 @@
 // pv_stream_kernel, which streams every V tile through the TMA ring.  Full-cache softmax runs softmax_kernel (K and V
 // tiles per stage, online max / sum per split); both dense paths combine
 // their splits in a fixed order in the last CTA of each group.
-#include "common.cuh"
-#include "internal.h"
+#include "pipeline.cuh"
 
 namespace ekv {
 
 namespace {
-
-constexpr int NWC = 4;                       // consumer warps
-constexpr int DEC_THREADS = (NWC + 1) * 32;  // + one producer warp
-constexpr int PPS_MAX = 8;
-
-template <int G>
-struct Tile {
-    static constexpr int TPS = G == 1 ? 128 : 64;  // tokens per pipeline stage
-};
-
-struct PageInfo {
-    int page;  // logical page (-1: none)
-    int mask;  // heads of the group that use it
-    int nval;  // valid tokens (0 if the page could not be loaded)
-    int upos;  // position in the union (page index on the dense paths)
-    int blk;   // physical block (-1: none)
-};
-
-__device__ __forceinline__ size_t tok_row(const DecodeArgs &a, int b, int h) {
-    return ((size_t)b * a.Hq + h) * (size_t)a.max_pages * a.P;
-}
-__device__ __forceinline__ size_t tile_row(const DecodeArgs &a, int b, int h) {
-    return ((size_t)b * a.Hq + h) * (size_t)a.max_pages * a.P / 16;
-}
 
 // ------------------------------------------------------------------ union
 
@@ -142,31 +117,7 @@ __global__ void dense_init_kernel(DecodeArgs a) {
     if (i < a.B * a.Hkv) a.ws.counters[i] = 0;
 }
 
-// ------------------------------------------------------ shared TMA pipeline
-
-template <int D, int G, int NS, int NMAP>
-struct Ring {
-    static constexpr int TPS = Tile<G>::TPS;
-    static constexpr int STAGE = TPS * D * 2 * NMAP;  // bytes per stage (K and/or V)
-    static constexpr size_t BYTES = 1024 + (size_t)NS * STAGE + 2 * NS * 8 + NS * PPS_MAX * sizeof(PageInfo) +
-                                    32 * PPS_MAX * sizeof(PageInfo);
-};
-
-template <int D, int G, int NS, int NMAP>
-struct RingView {
-    unsigned char *stages;
-    uint64_t *full, *empty;
-    PageInfo *pinfo;  // [NS][PPS_MAX]
-    PageInfo *stash;  // [32 * PPS_MAX], producer scratch
-    __device__ RingView(unsigned char *raw) {
-        using RG = Ring<D, G, NS, NMAP>;
-        stages = reinterpret_cast<unsigned char *>(((uintptr_t)raw + 1023) & ~(uintptr_t)1023);
-        full = reinterpret_cast<uint64_t *>(stages + (size_t)NS * RG::STAGE);
-        empty = full + NS;
-        pinfo = reinterpret_cast<PageInfo *>(empty + NS);
-        stash = pinfo + NS * PPS_MAX;
-    }
-};
+// ------------------------------------------------------ page producer
 
 // Producer warp: for the CTA's local steps 0..my_n-1 (global step
 // blockIdx.x + it*gridDim.x, covering entries [step*PPS, step*PPS+PPS) of the
@@ -241,12 +192,6 @@ __device__ void produce(const DecodeArgs &a, const CUtensorMap *m0, const CUtens
         if (!ok) return;
         __syncwarp();
     }
-}
-
-// Address of the 16-byte chunk `c16` (8 bf16) of row r in a swizzled page tile.
-__device__ __forceinline__ const unsigned char *tile_chunk(const unsigned char *page_base, int P, int r, int c16) {
-    const int box = c16 >> 3, cc = c16 & 7;
-    return page_base + box * P * 128 + r * 128 + ((cc ^ (r & 7)) << 4);
 }
 
 // ----------------------------------------------------------------- q . K^T
@@ -555,8 +500,10 @@ __global__ void __launch_bounds__(TAU_THREADS) tau_pv_kernel(const __grid_consta
                 }
             }
             __syncthreads();
+            const float wold = hi - lo;
             lo = br[0];
             hi = br[1];
+            if (!(hi - lo < wold)) break;  // at the float resolution of the bracket
         }
     } else {
         hi = lo;

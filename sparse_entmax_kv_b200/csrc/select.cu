@@ -12,13 +12,12 @@
 // Gaussian: tau_hat solves F(tau) = sum_p n_p E[(X_p - tau)_+^r] = 1 with
 // X_p ~ N(m_p, s_p^2), m_p = (alpha-1) mu_p, s_p = (alpha-1) sigma_p, using the
 // closed-form Gaussian partial moments.  F is decreasing, F >= 1 at
-// tau0 = max_p m_p - 1 (Jensen) and F < 1 at max_p (m_p + 10 s_p) (every page
-// is then 10 standard deviations into its tail).  Pages with
+// tau0 = max_p (m_p - n_p^(-1/r)) (Jensen) and F < 1 at max_p (m_p + 10 s_p)
+// (every page is then 10 standard deviations into its tail).  Pages with
 // m_p + 10 s_p < tau0 contribute below n_p s_p^r J_r(10) ~ 1e-25 n_p s_p^r
-// anywhere in that bracket and are pruned.  The bracket is narrowed by
-// multisection: each pass evaluates F at 32 points, one warp per point with
-// the lanes splitting the pages.  Pages are then kept when
-// (alpha-1) bbox_p > tau_hat - Delta.
+// anywhere in that bracket and are pruned.  Newton's method on F^(1/r),
+// which is convex, climbs from tau0 to the root without overshooting.  Pages
+// are then kept when (alpha-1) bbox_p > tau_hat - Delta.
 #include "common.cuh"
 #include "internal.h"
 
@@ -185,6 +184,46 @@ __device__ __forceinline__ void gauss_JJ(float c, float &jr, float &jr1) {
     jr1 = fmaxf(s1, 0.f);
 }
 
+// Adds page (m, s, weight w)'s term of F(tau) = sum_p n_p E[(X_p - tau)_+^R]
+// and of its derivative F'(tau) = -R sum_p n_p E[(X_p - tau)_+^(R-1)].
+template <int R>
+__device__ __forceinline__ void gauss_contrib(float m, float s, float w, float tau, float &F, float &Fp) {
+    if (s > 1e-30f) {
+        const float c = (tau - m) / s;
+        if (c > 38.f) return;
+        float jr, jr1;
+        gauss_JJ<R>(c, jr, jr1);
+        float sp = 1.f;
+#pragma unroll
+        for (int i = 1; i < R; ++i) sp *= s;  // s^(R-1)
+        F += w * sp * s * jr;
+        Fp -= (float)R * w * sp * jr1;
+    } else {
+        const float x = m - tau;
+        if (x > 0.f) {
+            float xp = 1.f;
+#pragma unroll
+            for (int i = 1; i < R; ++i) xp *= x;
+            F += w * xp * x;
+            Fp -= (float)R * w * xp;
+        }
+    }
+}
+
+// One Newton step on g = F^(1/R) from tau towards the root, kept below hi.
+// Returns false when tau has converged (F <= 1 within 2e-6, or a step below
+// 1e-7 max(1, |tau|)).
+template <int R>
+__device__ __forceinline__ bool newton_step(float F, float Fp, float hi, float &tau) {
+    if (!(F > 1.f + 2e-6f) || !(Fp < 0.f)) return false;
+    const float step = (float)R * (F - powf(F, 1.f - 1.f / (float)R)) / (-Fp);
+    float nt = tau + step;
+    if (!(nt < hi)) nt = 0.5f * (tau + hi);  // stay inside the bracket
+    const bool done = !(nt - tau > 1e-7f * fmaxf(1.f, fabsf(tau)));
+    tau = nt;
+    return !done;
+}
+
 constexpr int GCAP = 3072;  // pruned candidate pages held on chip
 
 // Gaussian selection.  One tile (TILE pages, ITEMS per thread) of mu, sigma
@@ -230,21 +269,33 @@ __global__ void __launch_bounds__(SEL_THREADS) gauss_kernel(SelectArgs a) {
             ss[i] = p < n ? a1 * __ldg(a.sigma + row + p) : 0.f;
         }
     };
+    // Lower end of the bracket.  Jensen: E[(X-tau)_+^R] >= (E[X]-tau)_+^R, so
+    // F(tau) >= 1 wherever some page has n_p (m_p - tau)^R >= 1, i.e.
+    // tau_hat >= max_p (m_p - n_p^(-1/R)).  Every page but the sequence's last
+    // is full, so the root n_p^(-1/R) takes two values.
+    const float inv_r = 1.f / (float)R;
+    const float drop_full = powf((float)a.P, -inv_r);
+    const int n_last = tokens_in_page(seq, a.P, n - 1);
+    const float drop_last = powf((float)n_last, -inv_r);
     float mloc = -INFINITY;
     for (int t0 = 0; t0 < n; t0 += TILE) {
         load_ms(t0);
 #pragma unroll
-        for (int i = 0; i < ITEMS; ++i) mloc = fmaxf(mloc, mm[i]);
+        for (int i = 0; i < ITEMS; ++i) {
+            const int p = t0 + threadIdx.x + SEL_THREADS * i;
+            mloc = fmaxf(mloc, mm[i] - (p == n - 1 ? drop_last : drop_full));
+        }
     }
 #pragma unroll
     for (int o = 16; o; o >>= 1) mloc = fmaxf(mloc, __shfl_xor_sync(FULL, mloc, o));
     if (lane == 0) shm[warp] = mloc;
     if (threadIdx.x == 0) ncand = 0;
     __syncthreads();
-    float mmax = -INFINITY;
-    for (int w = 0; w < SEL_THREADS / 32; ++w) mmax = fmaxf(mmax, shm[w]);
-    const float tau0 = mmax - 1.f;
+    float tau0 = -INFINITY;
+    for (int w = 0; w < SEL_THREADS / 32; ++w) tau0 = fmaxf(tau0, shm[w]);
 
+    // Pages with m + 10 s below tau0 add less than n_p s^R J_R(10) to F at any
+    // tau >= tau0 (a relative 1e-23 of one page's worth): they are dropped.
     float hloc = -INFINITY;  // max over pages of m + 10 s: F < 1 there
     for (int t0 = 0; t0 < n; t0 += TILE) {
         if (!one_tile) load_ms(t0);
@@ -280,64 +331,18 @@ __global__ void __launch_bounds__(SEL_THREADS) gauss_kernel(SelectArgs a) {
     if (overflow && threadIdx.x == 0) atomicOr(a.status, ENTMAXKV_STATUS_OVERFLOW);
 
     auto contrib = [&](float m, float s, float w, float tau, float &F, float &Fp) {
-        if (s > 1e-30f) {
-            const float c = (tau - m) / s;
-            if (c > 38.f) return;
-            float jr, jr1;
-            gauss_JJ<R>(c, jr, jr1);
-            float sp = 1.f;
-#pragma unroll
-            for (int i = 1; i < R; ++i) sp *= s;  // s^(R-1)
-            F += w * sp * s * jr;
-            Fp -= (float)R * w * sp * jr1;
-        } else {
-            const float x = m - tau;
-            if (x > 0.f) {
-                float xp = 1.f;
-#pragma unroll
-                for (int i = 1; i < R; ++i) xp *= x;
-                F += w * xp * x;
-                Fp -= (float)R * w * xp;
-            }
-        }
+        gauss_contrib<R>(m, s, w, tau, F, Fp);
     };
 
-    // One multisection pass on [tau0, hmax] (warp w evaluates F at point w),
-    // then Newton on g = F^(1/R) from the bracket's left end: g is convex and
-    // decreasing, so the iterates climb monotonically to the root.  Each
-    // Newton evaluation is spread over the whole block (one barrier each).
-    __shared__ float fpt[32];
-    __shared__ float brk[2];
+    // Newton on g = F^(1/R) from the bracket's left end.  F^(1/R) is R-norm of
+    // (X - tau)_+ under the pages' mixture (times a constant), hence convex and
+    // decreasing in tau: every tangent meets zero left of the root, so the
+    // iterates climb monotonically to it.  Each evaluation is spread over the
+    // whole block (one barrier each, double-buffered partials).
     __shared__ float nred[2][64];
-    float lo = tau0, hi = hmax;
-    {
-        const float w = (hi - lo) / 33.f;
-        const float t = lo + w * (float)(warp + 1);
-        float F = 0.f, Fp = 0.f;
-        if (!overflow) {
-            for (int i = lane; i < nc; i += 32) contrib(cm[i], cs[i], cn[i], t, F, Fp);
-        } else {
-            for (int p = lane; p < n; p += 32)
-                contrib(a1 * a.mu[row + p], a1 * a.sigma[row + p], (float)tokens_in_page(seq, a.P, p), t, F, Fp);
-        }
-#pragma unroll
-        for (int o = 16; o; o >>= 1) F += __shfl_xor_sync(FULL, F, o);
-        if (lane == 0) fpt[warp] = F;
-        __syncthreads();
-        if (warp == 0) {
-            // points increase with the warp index and F decreases: a prefix
-            const int cntge = __popc(__ballot_sync(FULL, fpt[lane] >= 1.f));
-            if (lane == 0) {
-                brk[0] = cntge > 0 ? lo + w * (float)cntge : lo;
-                brk[1] = cntge < 32 ? lo + w * (float)(cntge + 1) : hi;
-            }
-        }
-        __syncthreads();
-        lo = brk[0];
-        hi = brk[1];
-    }
-    float tau = lo;
-    for (int it = 0; it < 32; ++it) {
+    const float hi = hmax;
+    float tau = tau0;
+    for (int it = 0; it < 48; ++it) {
         float F = 0.f, Fp = 0.f;
         if (!overflow) {
             for (int i = threadIdx.x; i < nc; i += SEL_THREADS) contrib(cm[i], cs[i], cn[i], tau, F, Fp);
@@ -363,14 +368,7 @@ __global__ void __launch_bounds__(SEL_THREADS) gauss_kernel(SelectArgs a) {
             F += buf[2 * w];
             Fp += buf[2 * w + 1];
         }
-        if (!(F > 1.f + 2e-6f) || !(Fp < 0.f)) break;
-        // Newton on g = F^(1/R): step = R (F - F^(1-1/R)) / (-F')
-        const float step = (float)R * (F - powf(F, 1.f - 1.f / (float)R)) / (-Fp);
-        float nt = tau + step;
-        if (!(nt < hi)) nt = 0.5f * (tau + hi);  // stay inside the bracket
-        const bool done = !(nt - tau > 1e-7f * fmaxf(1.f, fabsf(tau)));
-        tau = nt;
-        if (done) break;
+        if (!newton_step<R>(F, Fp, hi, tau)) break;
     }
     if (threadIdx.x == 0 && a.tau_hat) a.tau_hat[bh] = tau;
 
@@ -397,12 +395,247 @@ __global__ void __launch_bounds__(SEL_THREADS) gauss_kernel(SelectArgs a) {
     if (threadIdx.x == 0) a.cnt[bh] = base;
 }
 
+// ------------------------------------------- Gaussian selection, cluster form
+//
+// A cluster of GCL CTAs per (sequence, head) for sequences of up to
+// GCL * GTH * GIT pages.  CTA r keeps pages [r Q, (r+1) Q), Q = ceil(n/GCL),
+// GIT consecutive pages per thread, in registers from first load to last use.
+// Exchanges are pushes into the peers' shared memory followed by one cluster
+// barrier each: (1) the CTAs' maxima give the bracket, (2) each CTA pushes its
+// pruned candidates to rank 0, (3) rank 0 solves for tau_hat (its whole block
+// evaluates each Newton step) and pushes it back, (4) the CTAs' selected-page
+// counts give each CTA its offset in the ascending list.  If a CTA has more
+// candidates than rank 0 holds for it, every Newton step is instead reduced
+// over the cluster (one barrier per step); the iterates are the same in every
+// CTA.
+constexpr int GCL = 4;
+constexpr int GTH = 256;
+constexpr int GIT = 16;
+constexpr int GCAPR = 256;  // candidates per CTA that rank 0 holds
+
+template <int R>
+__global__ void __cluster_dims__(GCL, 1, 1) __launch_bounds__(GTH) gauss_cluster_kernel(SelectArgs a) {
+    __shared__ float rmax[GCL], rhmax[GCL];             // pushed by every CTA
+    __shared__ int rcnt[GCL], rsel[GCL];                // pushed by every CTA
+    __shared__ float cm[GCL * GCAPR], cs[GCL * GCAPR], cn[GCL * GCAPR];  // candidates (rank 0)
+    __shared__ float s_tau;                             // pushed by rank 0
+    __shared__ float rF[2][GCL], rFp[2][GCL];           // pushed Newton partials (fallback)
+    __shared__ float rNw[2][2 * (GTH / 32)];            // per-warp Newton partials (rank 0)
+    __shared__ float wa[GTH / 32], wb[GTH / 32];
+    __shared__ int sh[72];
+    const unsigned rank = cl_rank();
+    const int bh = blockIdx.x / GCL;
+    const int b = bh / a.Hq;
+    const int seq = a.seq_lens[b];
+    const int n = n_pages_of(seq, a.P);
+    const size_t row = (size_t)bh * a.max_pages;
+    const float a1 = a.alpha - 1.f;
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+    if (n == 0) {  // the same in every CTA of the cluster: no barrier is skipped by half of it
+        if (rank == 0 && threadIdx.x == 0) {
+            a.cnt[bh] = 0;
+            if (a.tau_hat) a.tau_hat[bh] = __int_as_float(0x7fc00000);
+        }
+        return;
+    }
+    const int Q = ceil_div(n, GCL);
+    const int lo_p = min(n, (int)rank * Q), hi_p = min(n, (int)(rank + 1) * Q);
+    const int p0 = lo_p + threadIdx.x * GIT;
+    float ub[GIT], mm[GIT], ss[GIT];
+#pragma unroll
+    for (int i = 0; i < GIT; ++i) {
+        const bool v = p0 + i < hi_p;
+        ub[i] = v ? __ldg(a.bbox + row + p0 + i) : 0.f;
+        mm[i] = v ? a1 * __ldg(a.mu + row + p0 + i) : -INFINITY;
+        ss[i] = v ? a1 * __ldg(a.sigma + row + p0 + i) : 0.f;
+    }
+    // (1) bracket: tau_hat >= max_p (m_p - n_p^(-1/R)) (Jensen); F < 1 at
+    // max_p (m_p + 10 s_p)
+    const float inv_r = 1.f / (float)R;
+    const float drop_full = powf((float)a.P, -inv_r);
+    const float drop_last = powf((float)tokens_in_page(seq, a.P, n - 1), -inv_r);
+    float lmx = -INFINITY, lhx = -INFINITY;
+#pragma unroll
+    for (int i = 0; i < GIT; ++i) {
+        if (p0 + i < hi_p) {
+            lmx = fmaxf(lmx, mm[i] - (p0 + i == n - 1 ? drop_last : drop_full));
+            lhx = fmaxf(lhx, mm[i] + 10.f * ss[i]);
+        }
+    }
+#pragma unroll
+    for (int o = 16; o; o >>= 1) {
+        lmx = fmaxf(lmx, __shfl_xor_sync(FULL, lmx, o));
+        lhx = fmaxf(lhx, __shfl_xor_sync(FULL, lhx, o));
+    }
+    if (lane == 0) {
+        wa[warp] = lmx;
+        wb[warp] = lhx;
+    }
+    __syncthreads();
+    if (threadIdx.x < GCL) {
+        float x = -INFINITY, y = -INFINITY;
+        for (int w = 0; w < GTH / 32; ++w) {
+            x = fmaxf(x, wa[w]);
+            y = fmaxf(y, wb[w]);
+        }
+        cl_stf(cl_map(&rmax[rank], threadIdx.x), x);
+        cl_stf(cl_map(&rhmax[rank], threadIdx.x), y);
+    }
+    cl_sync();
+    float tau0 = -INFINITY, hmax = -INFINITY;
+#pragma unroll
+    for (int r = 0; r < GCL; ++r) {
+        tau0 = fmaxf(tau0, rmax[r]);
+        hmax = fmaxf(hmax, rhmax[r]);
+    }
+    hmax = fmaxf(hmax, tau0 + 1.f);
+
+    // (2) candidates: pages with m + 10 s >= tau0 (the rest add less than
+    // n_p s^R J_R(10) to F anywhere right of tau0), pushed to rank 0
+    unsigned keep = 0;
+#pragma unroll
+    for (int i = 0; i < GIT; ++i)
+        if (p0 + i < hi_p && mm[i] + 10.f * ss[i] >= tau0) keep |= 1u << i;
+    int lc;
+    int w = block_excl_scan(__popc(keep), sh, &lc);
+#pragma unroll
+    for (int i = 0; i < GIT; ++i)
+        if (keep & (1u << i)) {
+            if (w < GCAPR) {
+                const int slot = (int)rank * GCAPR + w;
+                cl_stf(cl_map(&cm[slot], 0), mm[i]);
+                cl_stf(cl_map(&cs[slot], 0), ss[i]);
+                cl_stf(cl_map(&cn[slot], 0), (float)tokens_in_page(seq, a.P, p0 + i));
+            }
+            ++w;
+        }
+    if (threadIdx.x < GCL) cl_sti(cl_map(&rcnt[rank], threadIdx.x), lc);
+    cl_sync();
+    bool spill = false;
+#pragma unroll
+    for (int r = 0; r < GCL; ++r) spill |= rcnt[r] > GCAPR;
+    if (spill && rank == 0 && threadIdx.x == 0) atomicOr(a.status, ENTMAXKV_STATUS_OVERFLOW);
+
+    // (3) tau_hat: Newton on g = F^(1/R) from tau0 (g is convex and
+    // decreasing, so the iterates climb to the root without overshooting)
+    float tau = tau0;
+    if (!spill) {
+        if (rank == 0) {
+            // rank 0 alone: candidate c of CTA r is item (r, c); thread t
+            // takes items t, t + GTH, ... of the concatenated lists
+            const int n0 = rcnt[0], n1 = n0 + rcnt[1], n2 = n1 + rcnt[2], n3 = n2 + rcnt[3];
+            for (int it = 0; it < 48; ++it) {
+                float F = 0.f, Fp = 0.f;
+                for (int k = threadIdx.x; k < n3; k += GTH) {
+                    const int r = k < n0 ? 0 : k < n1 ? 1 : k < n2 ? 2 : 3;
+                    const int c = r * GCAPR + k - (r == 0 ? 0 : r == 1 ? n0 : r == 2 ? n1 : n2);
+                    gauss_contrib<R>(cm[c], cs[c], cn[c], tau, F, Fp);
+                }
+#pragma unroll
+                for (int o = 16; o; o >>= 1) {
+                    F += __shfl_xor_sync(FULL, F, o);
+                    Fp += __shfl_xor_sync(FULL, Fp, o);
+                }
+                float *buf = rNw[it & 1];  // double-buffered: one barrier per step
+                if (lane == 0) {
+                    buf[2 * warp] = F;
+                    buf[2 * warp + 1] = Fp;
+                }
+                __syncthreads();
+                F = 0.f;
+                Fp = 0.f;
+#pragma unroll
+                for (int ww = 0; ww < GTH / 32; ++ww) {
+                    F += buf[2 * ww];
+                    Fp += buf[2 * ww + 1];
+                }
+                if (!newton_step<R>(F, Fp, hmax, tau)) break;  // the same in every thread
+            }
+            if (threadIdx.x < GCL) cl_stf(cl_map(&s_tau, threadIdx.x), tau);
+        }
+        cl_sync();
+        tau = s_tau;
+    } else {
+        for (int it = 0; it < 48; ++it) {
+            float F = 0.f, Fp = 0.f;
+#pragma unroll
+            for (int i = 0; i < GIT; ++i)
+                if (keep & (1u << i)) gauss_contrib<R>(mm[i], ss[i], (float)tokens_in_page(seq, a.P, p0 + i), tau, F, Fp);
+#pragma unroll
+            for (int o = 16; o; o >>= 1) {
+                F += __shfl_xor_sync(FULL, F, o);
+                Fp += __shfl_xor_sync(FULL, Fp, o);
+            }
+            __syncthreads();  // the previous step's wa/wb are read
+            if (lane == 0) {
+                wa[warp] = F;
+                wb[warp] = Fp;
+            }
+            __syncthreads();
+            if (threadIdx.x < GCL) {
+                float x = 0.f, y = 0.f;
+                for (int ww = 0; ww < GTH / 32; ++ww) {
+                    x += wa[ww];
+                    y += wb[ww];
+                }
+                cl_stf(cl_map(&rF[it & 1][rank], threadIdx.x), x);
+                cl_stf(cl_map(&rFp[it & 1][rank], threadIdx.x), y);
+            }
+            cl_sync();
+            F = 0.f;
+            Fp = 0.f;
+#pragma unroll
+            for (int r = 0; r < GCL; ++r) {
+                F += rF[it & 1][r];
+                Fp += rFp[it & 1][r];
+            }
+            if (!newton_step<R>(F, Fp, hmax, tau)) break;  // the same decision in every CTA
+        }
+    }
+    if (rank == 0 && threadIdx.x == 0 && a.tau_hat) a.tau_hat[bh] = tau;
+
+    // (4) pages with (alpha-1) bbox > tau_hat - Delta, ascending
+    const float thr = tau - a.delta;
+    unsigned bits = 0;
+#pragma unroll
+    for (int i = 0; i < GIT; ++i)
+        if (p0 + i < hi_p && a1 * ub[i] > thr) bits |= 1u << i;
+    int ls;
+    int o = block_excl_scan(__popc(bits), sh, &ls);
+    if (threadIdx.x < GCL) cl_sti(cl_map(&rsel[rank], threadIdx.x), ls);
+    cl_sync();
+    int off = 0, total = 0;
+#pragma unroll
+    for (int r = 0; r < GCL; ++r) {
+        off += r < (int)rank ? rsel[r] : 0;
+        total += rsel[r];
+    }
+    int *sel = a.sel + row;
+    o += off;
+#pragma unroll
+    for (int i = 0; i < GIT; ++i)
+        if (bits & (1u << i)) sel[o++] = p0 + i;
+    if (rank == 0 && threadIdx.x == 0) a.cnt[bh] = total;
+}
+
 }  // namespace
 
 cudaError_t launch_select(const SelectArgs &a, cudaStream_t st) {
     const int grid = a.B * a.Hq;
     if (a.policy == ENTMAXKV_TOPK) {
         topk_kernel<<<grid, SEL_THREADS, 0, st>>>(a);
+    } else if (a.max_pages <= GCL * GTH * GIT) {
+        switch (a.r_int) {
+            case 1: gauss_cluster_kernel<1><<<grid * GCL, GTH, 0, st>>>(a); break;
+            case 2: gauss_cluster_kernel<2><<<grid * GCL, GTH, 0, st>>>(a); break;
+            case 3: gauss_cluster_kernel<3><<<grid * GCL, GTH, 0, st>>>(a); break;
+            case 4: gauss_cluster_kernel<4><<<grid * GCL, GTH, 0, st>>>(a); break;
+            case 5: gauss_cluster_kernel<5><<<grid * GCL, GTH, 0, st>>>(a); break;
+            case 6: gauss_cluster_kernel<6><<<grid * GCL, GTH, 0, st>>>(a); break;
+            case 7: gauss_cluster_kernel<7><<<grid * GCL, GTH, 0, st>>>(a); break;
+            case 8: gauss_cluster_kernel<8><<<grid * GCL, GTH, 0, st>>>(a); break;
+            default: return cudaErrorInvalidValue;
+        }
     } else {
         switch (a.r_int) {
             case 1: gauss_kernel<1><<<grid, SEL_THREADS, 0, st>>>(a); break;

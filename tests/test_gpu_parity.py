@@ -321,6 +321,46 @@ def test_empty_selection_and_single_token_sequences():
     np.testing.assert_allclose(out[0], o[0], atol=1e-6)
 
 
+def _sparse_vs_oracle(wl, inp, host, policy, k, label):
+    """Oracle selection, then the library's sparse decode against the oracle's."""
+    osel, ocnt, _ = _oracle_selection(host, wl, policy, k, wl.delta or 0.5)
+    s = shape_of(wl)
+    sel, cnt = torch.from_numpy(osel).cuda(), torch.from_numpy(ocnt).cuda()
+    out = torch.empty((wl.B, wl.Hq, wl.d), device="cuda")
+    tau = torch.empty((wl.B, wl.Hq), device="cuda")
+    ws = nv.alloc_workspace(s, nv.CALL_DECODE_SPARSE, "cuda")
+    nv.entmaxkv_decode_sparse(s, inp["q"], inp["k_cache"], inp["v_cache"], inp["page_table"], inp["seq_lens"],
+                              sel, cnt, wl.alpha, out, tau, None, ws)
+    o, otau, _, _ = orc.decode(host["q"], host["K"], host["V"], host["page_table"], host["seq_lens"], wl.Hkv,
+                               wl.P, wl.alpha, sel=osel, cnt=ocnt)
+    assert_outputs_close(out.cpu().numpy(), o, label)
+    np.testing.assert_allclose(tau.cpu().numpy(), otau, atol=2e-5 * max(1.0, np.abs(otau).max()))
+
+
+def test_decode_sparse_long_sequence_small_pages():
+    """32771 pages of 16 tokens in one sequence (half a million tokens): page
+    lists and z rows far longer than any on-chip buffer."""
+    wl = Workload("long_p16", B=1, Hq=2, Hkv=1, d=64, L=32768 * 16 + 40, P=16, alpha=1.5, policy="topk",
+                  k=48, keys="offset", needles=6, needle_scale=4.0)
+    assert wl.max_pages > 32768
+    inp, host = gpu_inputs(wl, 12)
+    _sparse_vs_oracle(wl, inp, host, "topk", wl.k, "long_p16")
+
+
+def test_decode_sparse_all_tokens_candidates():
+    """Equal keys put every selected token within 1 of the max z, more
+    candidates than a head holds on chip: the exact path that rescans the z
+    row (status OVERFLOW, nothing else) gives the oracle's result."""
+    wl = Workload("flat", B=1, Hq=2, Hkv=1, d=64, L=64 * 600, P=64, alpha=2.0, policy="topk", k=512,
+                  keys="offset", needles=0)
+    inp, host = gpu_inputs(wl, 13)
+    inp["k_cache"][:] = inp["k_cache"][0, 0, 0]
+    host["K"] = to_host_u16(inp["k_cache"])
+    nv.get_status(clear=True)
+    _sparse_vs_oracle(wl, inp, host, "topk", wl.k, "flat")
+    assert nv.get_status(clear=True) & nv.STATUS_OVERFLOW
+
+
 def test_bad_page_table_entry_sets_status_and_skips():
     wl = SMALL["topk_small"]
     inp, _ = gpu_inputs(wl, 6)
