@@ -117,6 +117,34 @@ __device__ __forceinline__ void cp_async_wait() {
     asm volatile("cp.async.wait_group %0;" ::"n"(N) : "memory");
 }
 
+// ------------------------------------------------ programmatic dependent launch
+//
+// Every kernel of the library is launched with programmatic stream
+// serialisation and starts with pdl_wait(), which blocks until the previous
+// kernel of the stream has completed and its writes are visible.  The launch
+// of a kernel is thereby processed while its predecessor still runs.  No
+// kernel triggers its dependants early: CTAs of the next kernel parked on
+// the SMs slowed the running one down.  Because every CTA waits before doing
+// anything else, a kernel completes only after its predecessor, so completion
+// stays ordered along the stream.
+__device__ __forceinline__ void pdl_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+
+template <typename... KArgs, typename... Args>
+inline cudaError_t launch_pdl(void (*kern)(KArgs...), dim3 grid, dim3 block, size_t smem, cudaStream_t st,
+                              Args &&...args) {
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = grid;
+    cfg.blockDim = block;
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = st;
+    cudaLaunchAttribute at[1];
+    at[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    at[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = at;
+    cfg.numAttrs = 1;
+    return cudaLaunchKernelEx(&cfg, kern, static_cast<Args &&>(args)...);
+}
+
 // ------------------------------------------------------- thread-block clusters
 
 __device__ __forceinline__ unsigned cl_rank() {

@@ -34,6 +34,7 @@ namespace {
 // ------------------------------------------------------------------ union
 
 __global__ void __launch_bounds__(512) union_kernel(DecodeArgs a) {
+    pdl_wait();
     extern __shared__ unsigned words[];
     __shared__ int sh[72];
     __shared__ int cnts[8], offs[9];
@@ -112,6 +113,7 @@ __global__ void __launch_bounds__(512) union_kernel(DecodeArgs a) {
 }
 
 __global__ void dense_init_kernel(DecodeArgs a) {
+    pdl_wait();
     const int i = blockIdx.x * blockDim.x + threadIdx.x;
     if (i < a.B * a.Hq) a.ws.zmax[i] = ORD_NEG_INF;
     if (i < a.B * a.Hkv) a.ws.counters[i] = 0;
@@ -198,6 +200,7 @@ __device__ void produce(const DecodeArgs &a, const CUtensorMap *m0, const CUtens
 
 template <int D, int G, bool DENSE>
 __global__ void __launch_bounds__(DEC_THREADS) qk_kernel(const __grid_constant__ DecodeArgs a) {
+    pdl_wait();
     constexpr int NS = 4;
     using RG = Ring<D, G, NS, 1>;
     constexpr int TPS = RG::TPS;
@@ -369,6 +372,7 @@ constexpr int TCAP = 2048;  // candidate 16-token tiles held on chip per head
 // Exact threshold and (GATHER) the weighted sum of the support's value rows.
 template <int D, bool GATHER>
 __global__ void __launch_bounds__(TAU_THREADS) tau_pv_kernel(const __grid_constant__ DecodeArgs a, int dense) {
+    pdl_wait();
     constexpr int CPL = D / 32;
     // candidates (z and list position) in list order; once the gather has
     // read them, the same bytes hold the per-warp output partials
@@ -686,6 +690,7 @@ __device__ __forceinline__ void combine_last(const DecodeArgs &a, int bk, int b,
 
 template <int D, int G>
 __global__ void __launch_bounds__(DEC_THREADS) pv_stream_kernel(const __grid_constant__ DecodeArgs a) {
+    pdl_wait();
     constexpr int NS = 4;
     using RG = Ring<D, G, NS, 1>;
     constexpr int TPS = RG::TPS;
@@ -802,6 +807,7 @@ __global__ void __launch_bounds__(DEC_THREADS) pv_stream_kernel(const __grid_con
 
 template <int D, int G>
 __global__ void __launch_bounds__(DEC_THREADS) softmax_kernel(const __grid_constant__ DecodeArgs a) {
+    pdl_wait();
     constexpr int NS = 3;
     using RG = Ring<D, G, NS, 2>;
     constexpr int TPS = RG::TPS;
@@ -1024,8 +1030,7 @@ cudaError_t launch_qk(const DecodeArgs &a, cudaStream_t st) {
     if (e != cudaSuccess) return e;
     const int groups = a.B * a.Hkv;
     const int S = pick_splits(a.sms, 3, groups, ceil_div(a.max_pages, RG::TPS / a.P), 1 << 16);
-    k<<<dim3(S, groups), DEC_THREADS, RG::BYTES, st>>>(a);
-    return cudaGetLastError();
+    return launch_pdl(k, dim3(S, groups), dim3(DEC_THREADS), RG::BYTES, st, a);
 }
 
 template <int D, int G>
@@ -1034,11 +1039,9 @@ cudaError_t sparse_t(const DecodeArgs &a, cudaStream_t st) {
     const int groups = a.B * a.Hkv;
     const size_t ub = (size_t)ceil_div(a.max_pages, 4) * 4;
     if ((e = set_smem(union_kernel, ub)) != cudaSuccess) return e;
-    union_kernel<<<groups, 512, ub, st>>>(a);
-    if ((e = cudaGetLastError()) != cudaSuccess) return e;
+    if ((e = launch_pdl(union_kernel, dim3(groups), dim3(512), ub, st, a)) != cudaSuccess) return e;
     if ((e = launch_qk<D, G, false>(a, st)) != cudaSuccess) return e;
-    tau_pv_kernel<D, true><<<a.B * a.Hq, TAU_THREADS, 0, st>>>(a, 0);
-    return cudaGetLastError();
+    return launch_pdl(tau_pv_kernel<D, true>, dim3(a.B * a.Hq), dim3(TAU_THREADS), 0, st, a, 0);
 }
 
 template <int D, int G>
@@ -1046,17 +1049,14 @@ cudaError_t dense_entmax_t(const DecodeArgs &a, cudaStream_t st) {
     cudaError_t e;
     const int groups = a.B * a.Hkv;
     const int n = a.B * a.Hq > groups ? a.B * a.Hq : groups;
-    dense_init_kernel<<<ceil_div(n, 256), 256, 0, st>>>(a);
-    if ((e = cudaGetLastError()) != cudaSuccess) return e;
+    if ((e = launch_pdl(dense_init_kernel, dim3(ceil_div(n, 256)), dim3(256), 0, st, a)) != cudaSuccess) return e;
     if ((e = launch_qk<D, G, true>(a, st)) != cudaSuccess) return e;
-    tau_pv_kernel<D, false><<<a.B * a.Hq, TAU_THREADS, 0, st>>>(a, 1);
-    if ((e = cudaGetLastError()) != cudaSuccess) return e;
+    if ((e = launch_pdl(tau_pv_kernel<D, false>, dim3(a.B * a.Hq), dim3(TAU_THREADS), 0, st, a, 1)) != cudaSuccess) return e;
     using RG = Ring<D, G, 4, 1>;
     auto k = pv_stream_kernel<D, G>;
     if ((e = set_smem(k, RG::BYTES)) != cudaSuccess) return e;
     const int S = pick_splits(a.sms, 3, groups, ceil_div(a.max_pages, RG::TPS / a.P), MAX_SPLITS);
-    k<<<dim3(S, groups), DEC_THREADS, RG::BYTES, st>>>(a);
-    return cudaGetLastError();
+    return launch_pdl(k, dim3(S, groups), dim3(DEC_THREADS), RG::BYTES, st, a);
 }
 
 template <int D, int G>
@@ -1064,14 +1064,12 @@ cudaError_t dense_softmax_t(const DecodeArgs &a, cudaStream_t st) {
     cudaError_t e;
     const int groups = a.B * a.Hkv;
     const int n = a.B * a.Hq > groups ? a.B * a.Hq : groups;
-    dense_init_kernel<<<ceil_div(n, 256), 256, 0, st>>>(a);
-    if ((e = cudaGetLastError()) != cudaSuccess) return e;
+    if ((e = launch_pdl(dense_init_kernel, dim3(ceil_div(n, 256)), dim3(256), 0, st, a)) != cudaSuccess) return e;
     using RG = Ring<D, G, 3, 2>;
     auto k = softmax_kernel<D, G>;
     if ((e = set_smem(k, RG::BYTES)) != cudaSuccess) return e;
     const int S = pick_splits(a.sms, 2, groups, ceil_div(a.max_pages, RG::TPS / a.P), MAX_SPLITS);
-    k<<<dim3(S, groups), DEC_THREADS, RG::BYTES, st>>>(a);
-    return cudaGetLastError();
+    return launch_pdl(k, dim3(S, groups), dim3(DEC_THREADS), RG::BYTES, st, a);
 }
 
 }  // namespace

@@ -15,6 +15,7 @@ namespace ekv {
 
 template <int D, int P>
 __global__ void __launch_bounds__(D) build_meta_kernel(MetaArgs a) {
+    pdl_wait();
     const int b = blockIdx.y;
     const int kvh = blockIdx.z;
     const int p = a.first_page + blockIdx.x;
@@ -70,13 +71,14 @@ __global__ void __launch_bounds__(D) build_meta_kernel(MetaArgs a) {
 template <int D>
 cudaError_t launch_d(const MetaArgs &a, cudaStream_t st) {
     dim3 grid(a.n_pages, a.B, a.Hkv);
+    cudaError_t e = cudaSuccess;
     switch (a.P) {
-        case 16: build_meta_kernel<D, 16><<<grid, D, 0, st>>>(a); break;
-        case 32: build_meta_kernel<D, 32><<<grid, D, 0, st>>>(a); break;
-        case 64: build_meta_kernel<D, 64><<<grid, D, 0, st>>>(a); break;
+        case 16: e = launch_pdl(build_meta_kernel<D, 16>, dim3(grid), dim3(D), 0, st, a); break;
+        case 32: e = launch_pdl(build_meta_kernel<D, 32>, dim3(grid), dim3(D), 0, st, a); break;
+        case 64: e = launch_pdl(build_meta_kernel<D, 64>, dim3(grid), dim3(D), 0, st, a); break;
         default: return cudaErrorInvalidValue;
     }
-    return cudaGetLastError();
+    return e;
 }
 
 cudaError_t launch_build_meta(const MetaArgs &a, cudaStream_t st) {

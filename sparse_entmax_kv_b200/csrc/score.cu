@@ -55,6 +55,7 @@ constexpr size_t smem_bytes() {
 
 template <int D, int G, bool GAUSS>
 __global__ void __launch_bounds__(THREADS, G <= 4 ? 2 : 1) score_kernel(ScoreArgs a) {
+    pdl_wait();
     using RG = Ring<GAUSS>;
     constexpr int NCH = D / CHK;
     constexpr int NST = RG::NST;
@@ -180,8 +181,7 @@ cudaError_t launch_t(const ScoreArgs &a, cudaStream_t st) {
     cudaError_t e = ensure_smem(reinterpret_cast<const void *>(kern), smem);
     if (e != cudaSuccess) return e;
     dim3 grid(ceil_div(a.n_tiles, WARPS), a.B * a.Hkv);
-    kern<<<grid, THREADS, smem, st>>>(a);
-    return cudaGetLastError();
+    return launch_pdl(kern, dim3(grid), dim3(THREADS), smem, st, a);
 }
 
 template <int D, bool GAUSS>

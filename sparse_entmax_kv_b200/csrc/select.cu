@@ -41,6 +41,7 @@ __device__ __forceinline__ unsigned key_of(float f) {
 // consecutive pages per thread, through the four radix passes and the final
 // ordered compaction; longer sequences take several tiles per pass.
 __global__ void __launch_bounds__(SEL_THREADS) topk_kernel(SelectArgs a) {
+    pdl_wait();
     __shared__ int hist[256];
     __shared__ int sh[72];
     __shared__ int pick[2];
@@ -233,6 +234,7 @@ constexpr int GCAP = 3072;  // pruned candidate pages held on chip
 // (double-buffered partials).
 template <int R>
 __global__ void __launch_bounds__(SEL_THREADS) gauss_kernel(SelectArgs a) {
+    pdl_wait();
     __shared__ float cm[GCAP], cs[GCAP], cn[GCAP];
     __shared__ float shm[32], shm2[32];
     __shared__ int shi[72];
@@ -415,6 +417,7 @@ constexpr int GCAPR = 256;  // candidates per CTA that rank 0 holds
 
 template <int R>
 __global__ void __cluster_dims__(GCL, 1, 1) __launch_bounds__(GTH) gauss_cluster_kernel(SelectArgs a) {
+    pdl_wait();
     __shared__ float rmax[GCL], rhmax[GCL];             // pushed by every CTA
     __shared__ int rcnt[GCL], rsel[GCL];                // pushed by every CTA
     __shared__ float cm[GCL * GCAPR], cs[GCL * GCAPR], cn[GCL * GCAPR];  // candidates (rank 0)
@@ -622,34 +625,35 @@ __global__ void __cluster_dims__(GCL, 1, 1) __launch_bounds__(GTH) gauss_cluster
 
 cudaError_t launch_select(const SelectArgs &a, cudaStream_t st) {
     const int grid = a.B * a.Hq;
+    cudaError_t e = cudaSuccess;
     if (a.policy == ENTMAXKV_TOPK) {
-        topk_kernel<<<grid, SEL_THREADS, 0, st>>>(a);
+        e = launch_pdl(topk_kernel, dim3(grid), dim3(SEL_THREADS), 0, st, a);
     } else if (a.max_pages <= GCL * GTH * GIT) {
         switch (a.r_int) {
-            case 1: gauss_cluster_kernel<1><<<grid * GCL, GTH, 0, st>>>(a); break;
-            case 2: gauss_cluster_kernel<2><<<grid * GCL, GTH, 0, st>>>(a); break;
-            case 3: gauss_cluster_kernel<3><<<grid * GCL, GTH, 0, st>>>(a); break;
-            case 4: gauss_cluster_kernel<4><<<grid * GCL, GTH, 0, st>>>(a); break;
-            case 5: gauss_cluster_kernel<5><<<grid * GCL, GTH, 0, st>>>(a); break;
-            case 6: gauss_cluster_kernel<6><<<grid * GCL, GTH, 0, st>>>(a); break;
-            case 7: gauss_cluster_kernel<7><<<grid * GCL, GTH, 0, st>>>(a); break;
-            case 8: gauss_cluster_kernel<8><<<grid * GCL, GTH, 0, st>>>(a); break;
+            case 1: e = launch_pdl(gauss_cluster_kernel<1>, dim3(grid * GCL), dim3(GTH), 0, st, a); break;
+            case 2: e = launch_pdl(gauss_cluster_kernel<2>, dim3(grid * GCL), dim3(GTH), 0, st, a); break;
+            case 3: e = launch_pdl(gauss_cluster_kernel<3>, dim3(grid * GCL), dim3(GTH), 0, st, a); break;
+            case 4: e = launch_pdl(gauss_cluster_kernel<4>, dim3(grid * GCL), dim3(GTH), 0, st, a); break;
+            case 5: e = launch_pdl(gauss_cluster_kernel<5>, dim3(grid * GCL), dim3(GTH), 0, st, a); break;
+            case 6: e = launch_pdl(gauss_cluster_kernel<6>, dim3(grid * GCL), dim3(GTH), 0, st, a); break;
+            case 7: e = launch_pdl(gauss_cluster_kernel<7>, dim3(grid * GCL), dim3(GTH), 0, st, a); break;
+            case 8: e = launch_pdl(gauss_cluster_kernel<8>, dim3(grid * GCL), dim3(GTH), 0, st, a); break;
             default: return cudaErrorInvalidValue;
         }
     } else {
         switch (a.r_int) {
-            case 1: gauss_kernel<1><<<grid, SEL_THREADS, 0, st>>>(a); break;
-            case 2: gauss_kernel<2><<<grid, SEL_THREADS, 0, st>>>(a); break;
-            case 3: gauss_kernel<3><<<grid, SEL_THREADS, 0, st>>>(a); break;
-            case 4: gauss_kernel<4><<<grid, SEL_THREADS, 0, st>>>(a); break;
-            case 5: gauss_kernel<5><<<grid, SEL_THREADS, 0, st>>>(a); break;
-            case 6: gauss_kernel<6><<<grid, SEL_THREADS, 0, st>>>(a); break;
-            case 7: gauss_kernel<7><<<grid, SEL_THREADS, 0, st>>>(a); break;
-            case 8: gauss_kernel<8><<<grid, SEL_THREADS, 0, st>>>(a); break;
+            case 1: e = launch_pdl(gauss_kernel<1>, dim3(grid), dim3(SEL_THREADS), 0, st, a); break;
+            case 2: e = launch_pdl(gauss_kernel<2>, dim3(grid), dim3(SEL_THREADS), 0, st, a); break;
+            case 3: e = launch_pdl(gauss_kernel<3>, dim3(grid), dim3(SEL_THREADS), 0, st, a); break;
+            case 4: e = launch_pdl(gauss_kernel<4>, dim3(grid), dim3(SEL_THREADS), 0, st, a); break;
+            case 5: e = launch_pdl(gauss_kernel<5>, dim3(grid), dim3(SEL_THREADS), 0, st, a); break;
+            case 6: e = launch_pdl(gauss_kernel<6>, dim3(grid), dim3(SEL_THREADS), 0, st, a); break;
+            case 7: e = launch_pdl(gauss_kernel<7>, dim3(grid), dim3(SEL_THREADS), 0, st, a); break;
+            case 8: e = launch_pdl(gauss_kernel<8>, dim3(grid), dim3(SEL_THREADS), 0, st, a); break;
             default: return cudaErrorInvalidValue;
         }
     }
-    return cudaGetLastError();
+    return e;
 }
 
 }  // namespace ekv
