@@ -3,9 +3,9 @@
 // full-cache entmax and full-cache softmax as comparison points).
 //
 // Sparse path, three launches on one stream, no host round trip:
-//   union_kernel   per (sequence, kv head): union of the G query heads'
-//                  selected pages, ascending, each with a G-bit head mask;
-//                  also resets the per-head maxima and candidate counters.
+//   union_kernel   per (sequence, kv head), a cluster of 8 CTAs: union of
+//                  the G query heads' selected pages, ascending, each with a
+//                  G-bit head mask; also resets the per-head maxima.
 //   qk_kernel      split over the union: TMA 2-D loads (128-byte swizzle) of
 //                  the K tiles through a 4-stage mbarrier ring fed by one
 //                  producer warp (which resolves union entries and page-table
@@ -33,26 +33,39 @@ namespace {
 
 // ------------------------------------------------------------------ union
 
-__global__ void __launch_bounds__(512) union_kernel(DecodeArgs a) {
+// Union of the G heads' selections of a group, ascending, each entry with its
+// head mask.  A cluster of UCL CTAs per (sequence, kv head): CTA r owns pages
+// [r Q, (r+1) Q) (Q a multiple of 4), reads every head's list and marks the
+// pages in its range in a shared-memory bitmap (one byte of head bits per
+// page), compacts them in page order, and learns where its entries start
+// from the counts the lower-ranked CTAs push into its shared memory.
+constexpr int UCL = 8;
+constexpr int UTH = 256;
+
+__global__ void __cluster_dims__(UCL, 1, 1) __launch_bounds__(UTH) union_kernel(DecodeArgs a) {
     pdl_wait();
     extern __shared__ unsigned words[];
     __shared__ int sh[72];
     __shared__ int cnts[8], offs[9];
-    const int bk = blockIdx.x;
+    __shared__ int rcount[UCL];  // pushed by every CTA of the cluster
+    const unsigned rank = cl_rank();
+    const int bk = blockIdx.x / UCL;
     const int b = bk / a.Hkv, kvh = bk % a.Hkv;
     const int G = a.Hq / a.Hkv;
     const int np = n_pages_of(a.seq_lens[b], a.P);
-    const int nw = ceil_div(np, 4);
-    for (int i = threadIdx.x; i < nw; i += blockDim.x) words[i] = 0u;
+    const int Q = ceil_div(ceil_div(np, UCL), 4) * 4;
+    const int lo = min(np, (int)rank * Q), hi = min(np, (int)(rank + 1) * Q);
+    const int nw = ceil_div(hi - lo, 4);
+    for (int i = threadIdx.x; i < nw; i += UTH) words[i] = 0u;
     if (threadIdx.x < G) {
         const int bh = b * a.Hq + kvh * G + threadIdx.x;
         int c = a.cnt[bh];
         if (c < 0 || c > np) {
-            atomicOr(a.status, ENTMAXKV_STATUS_BAD_SELECTION);
+            if (rank == 0) atomicOr(a.status, ENTMAXKV_STATUS_BAD_SELECTION);
             c = c < 0 ? 0 : np;
         }
         cnts[threadIdx.x] = c;
-        a.ws.zmax[bh] = ORD_NEG_INF;
+        if (rank == 0) a.ws.zmax[bh] = ORD_NEG_INF;
     }
     __syncthreads();
     if (threadIdx.x == 0) {
@@ -60,56 +73,63 @@ __global__ void __launch_bounds__(512) union_kernel(DecodeArgs a) {
         for (int g = 0; g < G; ++g) offs[g + 1] = offs[g] + cnts[g];
     }
     __syncthreads();
-    // all heads' entries as one flat range, four loads in flight per thread
+    // every head's entries as one flat range, four loads in flight per thread
     const int total = offs[G];
-    for (int k0 = threadIdx.x; k0 < total; k0 += 4 * blockDim.x) {
+    for (int k0 = threadIdx.x; k0 < total; k0 += 4 * UTH) {
         int p[4], g[4];
 #pragma unroll
         for (int u = 0; u < 4; ++u) {
-            const int k = k0 + u * blockDim.x;
+            const int k = k0 + u * UTH;
             p[u] = -1;
             g[u] = 0;
             if (k < total) {
                 int gg = 0;
                 while (k >= offs[gg + 1]) ++gg;
                 g[u] = gg;
-                p[u] = a.sel[(size_t)(b * a.Hq + kvh * G + gg) * a.max_pages + (k - offs[gg])];
+                p[u] = __ldg(a.sel + (size_t)(b * a.Hq + kvh * G + gg) * a.max_pages + (k - offs[gg]));
             }
         }
 #pragma unroll
         for (int u = 0; u < 4; ++u) {
-            if (k0 + u * (int)blockDim.x >= total) continue;
-            if (p[u] >= 0 && p[u] < np)
-                atomicOr(&words[p[u] >> 2], 1u << ((p[u] & 3) * 8 + g[u]));
-            else
+            if (k0 + u * UTH >= total) continue;
+            if (p[u] >= lo && p[u] < hi)
+                atomicOr(&words[(p[u] - lo) >> 2], 1u << ((p[u] & 3) * 8 + g[u]));
+            else if ((p[u] < 0 || p[u] >= np) && rank == 0)
                 atomicOr(a.status, ENTMAXKV_STATUS_BAD_SELECTION);
         }
     }
     __syncthreads();
-    constexpr int IT = 16;
-    int *ue = a.ws.union_e + (size_t)bk * a.max_pages;
-    int base = 0;
-    for (int t0 = 0; t0 < np; t0 += 512 * IT) {
-        const int p0 = t0 + threadIdx.x * IT;
-        unsigned bytes[IT];
+    // this CTA's entries in page order: thread t owns words [t*wpt, (t+1)*wpt)
+    const int wpt = ceil_div(nw, UTH);
+    const int w0 = threadIdx.x * wpt;
+    int mine = 0;
+    for (int i = 0; i < wpt; ++i)
+        if (w0 + i < nw) {
+            const unsigned w = words[w0 + i];
 #pragma unroll
-        for (int i = 0; i < IT; i += 4) {
-            const unsigned w = (p0 + i < np) ? words[(p0 + i) >> 2] : 0u;
-#pragma unroll
-            for (int j = 0; j < 4; ++j) bytes[i + j] = (p0 + i + j < np) ? (w >> (8 * j)) & 0xffu : 0u;
+            for (int j = 0; j < 4; ++j) mine += ((w >> (8 * j)) & 0xffu) ? 1 : 0;
         }
-        unsigned bits = 0;
+    int local;
+    int pos = block_excl_scan(mine, sh, &local);
+    if (threadIdx.x < UCL) cl_sti(cl_map(&rcount[rank], threadIdx.x), local);
+    cl_sync();
+    int before = 0, all = 0;
 #pragma unroll
-        for (int i = 0; i < IT; ++i)
-            if (bytes[i]) bits |= 1u << i;
-        int tot;
-        int w = base + block_excl_scan(__popc(bits), sh, &tot);
-#pragma unroll
-        for (int i = 0; i < IT; ++i)
-            if (bits & (1u << i)) ue[w++] = ((p0 + i) << 8) | (int)bytes[i];
-        base += tot;
+    for (int r = 0; r < UCL; ++r) {
+        before += r < (int)rank ? rcount[r] : 0;
+        all += rcount[r];
     }
-    if (threadIdx.x == 0) a.ws.union_cnt[bk] = base;
+    int *ue = a.ws.union_e + (size_t)bk * a.max_pages + before;
+    for (int i = 0; i < wpt; ++i) {
+        if (w0 + i >= nw) break;
+        const unsigned w = words[w0 + i];
+#pragma unroll
+        for (int j = 0; j < 4; ++j) {
+            const unsigned m = (w >> (8 * j)) & 0xffu;
+            if (m) ue[pos++] = ((lo + 4 * (w0 + i) + j) << 8) | (int)m;
+        }
+    }
+    if (rank == 0 && threadIdx.x == 0) a.ws.union_cnt[bk] = all;
 }
 
 __global__ void dense_init_kernel(DecodeArgs a) {
@@ -366,24 +386,25 @@ __global__ void __launch_bounds__(DEC_THREADS) qk_kernel(const __grid_constant__
 constexpr int TAU_THREADS = 512;
 constexpr int TAU_WARPS = TAU_THREADS / 32;
 constexpr int ZCAP = 4096;  // candidates held on chip per head
-constexpr int TAU_C = 32;   // list positions per thread per scan tile
-constexpr int TCAP = 2048;  // candidate 16-token tiles held on chip per head
+constexpr int TAU_TB = 8;   // tile maxima in flight per lane
+constexpr size_t TAU_SMEM = (size_t)ZCAP * 16;
 
 // Exact threshold and (GATHER) the weighted sum of the support's value rows.
 template <int D, bool GATHER>
 __global__ void __launch_bounds__(TAU_THREADS) tau_pv_kernel(const __grid_constant__ DecodeArgs a, int dense) {
     pdl_wait();
     constexpr int CPL = D / 32;
-    // candidates (z and list position) in list order; once the gather has
-    // read them, the same bytes hold the per-warp output partials
-    __shared__ __align__(16) unsigned char cbuf[ZCAP * 8];
-    float *cz = reinterpret_cast<float *>(cbuf);
-    int *cpos = reinterpret_cast<int *>(cbuf + ZCAP * 4);
-    double(*accs)[D] = reinterpret_cast<double(*)[D]>(cbuf);
-    static_assert(TAU_WARPS * D * 8 <= ZCAP * 8, "partials must fit the candidate buffer");
+    // candidates in list order: z, value row and list position; once the
+    // gather has read them, the same bytes hold the per-warp output partials
+    extern __shared__ __align__(16) unsigned char tsm[];
+    float *cz = reinterpret_cast<float *>(tsm);
+    int *crow = reinterpret_cast<int *>(tsm + ZCAP * 4);
+    int *cpos = reinterpret_cast<int *>(tsm + ZCAP * 8);
+    int *ctile = reinterpret_cast<int *>(tsm + ZCAP * 12);  // candidate 16-token tiles
+    double(*accs)[D] = reinterpret_cast<double(*)[D]>(tsm);
+    static_assert(TAU_WARPS * D * 8 <= TAU_SMEM, "partials must fit the candidate buffer");
+    __shared__ int wcnt[72];  // block scan scratch
     __shared__ float red[TAU_WARPS][33];
-    __shared__ int ctile[TCAP];  // candidate 16-token tiles, in list order
-    __shared__ int sh[72];
     __shared__ float br[2];
     const int bh = blockIdx.x;
     const int b = bh / a.Hq, h = bh % a.Hq;
@@ -408,63 +429,80 @@ __global__ void __launch_bounds__(TAU_THREADS) tau_pv_kernel(const __grid_consta
     }
     const float thr = zmax - 1.f;
     const float *zr = a.ws.zbuf + tok_row(a, b, h);
-
-    // Candidates in list order, in two ordered compactions: first the 16-token
-    // tiles whose max exceeds thr, then the tokens of those tiles.  Each uses
-    // one block scan per pass over TAU_THREADS * TAU_C entries.
-    const int n_tiles = n_tok / 16;
     const float *tr = a.ws.tmax + tile_row(a, b, h);
+    auto row_of_pos = [&](int pos) -> int {
+        const int up = pos / P, t = pos - up * P;
+        const int blk = dense ? __ldg(a.page_table + (size_t)b * a.max_pages + up)
+                              : __ldcg(a.ws.union_blk + (size_t)bk * a.max_pages + up);
+        return (blk * a.Hkv + kvh) * P + t;
+    };
+
+    // Candidates (z > z_max - 1) in list order, in two ordered block-wide
+    // compactions: the 16-token tiles whose max clears the bar, then their
+    // tokens (z and, for the gather, the value row are loaded together).
+    const int n_tiles = n_tok / 16;
     int ntc = 0;
-    for (int t0 = 0; t0 < n_tiles; t0 += TAU_THREADS * TAU_C) {
-        const int p0 = t0 + threadIdx.x * TAU_C;
-        float v[TAU_C];
+    for (int t0 = 0; t0 < n_tiles; t0 += TAU_THREADS * TAU_TB) {
+        const int p0 = t0 + threadIdx.x * TAU_TB;
+        float v[TAU_TB];
 #pragma unroll
-        for (int i = 0; i < TAU_C; ++i) v[i] = p0 + i < n_tiles ? __ldcg(tr + p0 + i) : -INFINITY;
+        for (int i = 0; i < TAU_TB; ++i) v[i] = p0 + i < n_tiles ? __ldcg(tr + p0 + i) : -INFINITY;
         unsigned bits = 0;
 #pragma unroll
-        for (int i = 0; i < TAU_C; ++i)
+        for (int i = 0; i < TAU_TB; ++i)
             if (v[i] > thr) bits |= 1u << i;
         int tot;
-        int w = ntc + block_excl_scan(__popc(bits), sh, &tot);
+        int w = ntc + block_excl_scan(__popc(bits), wcnt, &tot);
         while (bits) {
             const int k = __ffs(bits) - 1;
             bits &= bits - 1;
-            if (w < TCAP) ctile[w] = p0 + k;
+            if (w < ZCAP) ctile[w] = p0 + k;
             ++w;
         }
         ntc += tot;
     }
     __syncthreads();
     int nc = 0;
-    if (ntc <= TCAP) {
-        // the tokens of the candidate tiles
-        for (int e0 = 0; e0 < ntc * 16; e0 += TAU_THREADS) {
-            const int e = e0 + threadIdx.x;
-            float z = -INFINITY;
-            int pos = 0;
-            if (e < ntc * 16) {
-                pos = ctile[e >> 4] * 16 + (e & 15);
-                z = __ldcg(zr + pos);
+    if (ntc <= ZCAP) {
+        // the tiles' tokens, ZCAP at a time, TPT consecutive ones per thread
+        constexpr int TPT = ZCAP / TAU_THREADS;
+        for (int e0 = 0; e0 < ntc * 16 && nc <= ZCAP; e0 += ZCAP) {
+            float zz[TPT];
+            int pp[TPT], rr[TPT];
+            unsigned bits = 0;
+#pragma unroll
+            for (int i = 0; i < TPT; ++i) {
+                const int e = e0 + threadIdx.x * TPT + i;
+                zz[i] = -INFINITY;
+                pp[i] = 0;
+                rr[i] = 0;
+                if (e < ntc * 16) {
+                    pp[i] = ctile[e >> 4] * 16 + (e & 15);
+                    zz[i] = __ldcg(zr + pp[i]);
+                    if (GATHER) rr[i] = row_of_pos(pp[i]);
+                    if (zz[i] > thr) bits |= 1u << i;
+                }
             }
-            const bool c = z > thr;
             int tot;
-            const int w = nc + block_excl_scan(c ? 1 : 0, sh, &tot);
-            __syncthreads();  // every thread has read its tile entry
-            if (c && w < ZCAP) {
-                cz[w] = z;
-                cpos[w] = pos;
-            }
+            int w = nc + block_excl_scan(__popc(bits), wcnt, &tot);
+#pragma unroll
+            for (int i = 0; i < TPT; ++i)
+                if (bits & (1u << i)) {
+                    if (w < ZCAP) {
+                        cz[w] = zz[i];
+                        cpos[w] = pp[i];
+                        if (GATHER) crow[w] = rr[i];
+                    }
+                    ++w;
+                }
             nc += tot;
-            __syncthreads();
         }
     } else {
-        nc = ZCAP + 1;  // too many tiles to list: take the whole-row path below
+        nc = ZCAP + 1;  // too many candidate tiles to list: the whole-row path below
     }
-    __syncthreads();
     __syncthreads();
     const bool onchip = nc <= ZCAP;
     if (!onchip && threadIdx.x == 0) atomicOr(a.status, ENTMAXKV_STATUS_OVERFLOW);
-    // off chip: scan the head's whole z row, filtering on thr
     const int nloop = onchip ? nc : n_tok;
     auto cz_at = [&](int i) -> float { return onchip ? cz[i] : __ldcg(zr + i); };
 
@@ -472,8 +510,10 @@ __global__ void __launch_bounds__(TAU_THREADS) tau_pv_kernel(const __grid_consta
     // lane l of every warp evaluates point l over the warp's slice of the
     // candidates (slices and order are fixed, so the sums are reproducible),
     // and the warps' partial sums are added in warp order.
+    // (on chip nc is the exact candidate count; off chip only a lower bound on
+    // it, so the bracket uses every token of the list)
     float lo = thr;
-    float hi = zmax - powf((float)nc, 1.f - a.alpha);
+    float hi = zmax - powf((float)(onchip ? nc : n_tok), 1.f - a.alpha);
     if (nc > 1 && hi > lo) {
         const float tol = 1e-7f * fmaxf(1.f, fabsf(zmax));
         for (int pass = 0; pass < 12 && hi - lo > tol; ++pass) {
@@ -519,23 +559,18 @@ __global__ void __launch_bounds__(TAU_THREADS) tau_pv_kernel(const __grid_consta
     }
     if (!GATHER) return;
 
-    // p v over the support.  On chip: the support (z > tau) is first compacted
-    // in list order, then dealt round-robin to the warps, eight rows at a time
-    // per warp with all their loads in flight.  Off chip: each warp scans its
-    // share of the z row.  Sums run in fp64 (p v is exact there).
+    // p v over the support: every warp takes a strided share of the
+    // candidates, moves the lanes with weight to the front eight at a time and
+    // sums p v of their value rows in fp64 (exact products).
     double acc[CPL];
 #pragma unroll
     for (int c = 0; c < CPL; ++c) acc[c] = 0.0;
     const size_t lstride = (size_t)a.max_pages * P;
-    auto row_of = [&](int pos, float p) -> int {
+    auto put_p = [&](int pos, float p) {
+        if (!a.p_out) return;
         const int up = pos / P, t = pos - up * P;
-        const int blk = dense ? __ldg(a.page_table + (size_t)b * a.max_pages + up)
-                              : __ldcg(a.ws.union_blk + (size_t)bk * a.max_pages + up);
-        if (a.p_out) {
-            const int page = dense ? up : (__ldcg(a.ws.union_e + (size_t)bk * a.max_pages + up) >> 8);
-            a.p_out[(size_t)bh * lstride + (size_t)page * P + t] = p;
-        }
-        return (blk * a.Hkv + kvh) * P + t;
+        const int page = dense ? up : (__ldcg(a.ws.union_e + (size_t)bk * a.max_pages + up) >> 8);
+        a.p_out[(size_t)bh * lstride + (size_t)page * P + t] = p;
     };
     auto gather8 = [&](int nr, int row, float p) {
         // lanes 0..nr-1 hold (row, p) of up to eight support tokens
@@ -567,70 +602,32 @@ __global__ void __launch_bounds__(TAU_THREADS) tau_pv_kernel(const __grid_consta
 #pragma unroll
             for (int cc = 0; cc < CPL; ++cc) acc[cc] = fma((double)pp[i], (double)vv[i][cc], acc[cc]);
     };
-    if (onchip) {
-        // in-place ordered compaction of the support: p overwrites z, position kept
-        constexpr int PER = ZCAP / TAU_THREADS;
-        const int per = ceil_div(nc, TAU_THREADS);
-        const int c0 = threadIdx.x * per;
-        float pz[PER];
-        int pp_[PER];
-        unsigned bits = 0;
+    // candidate c belongs to warp c % 16 (lane (c / 16) % 32), so a small
+    // support spreads over all warps
+    for (int k0 = 0; k0 < nloop; k0 += TAU_THREADS) {
+        const int c = k0 + lane * TAU_WARPS + warp;
+        const float z = c < nloop ? cz_at(c) : -INFINITY;
+        const float p = pos_pow(z - tau, r, ri);
+        unsigned bal = __ballot_sync(FULL, p > 0.f);
+        while (bal) {
+            int src = 0, nr = 0;
 #pragma unroll
-        for (int k = 0; k < PER; ++k) {
-            pz[k] = 0.f;
-            pp_[k] = 0;
-            if (k < per && c0 + k < nc) {
-                pz[k] = pos_pow(cz[c0 + k] - tau, r, ri);
-                pp_[k] = cpos[c0 + k];
-                if (pz[k] > 0.f) bits |= 1u << k;
-            }
-        }
-        int ns;
-        int w = block_excl_scan(__popc(bits), sh, &ns);
-        __syncthreads();
-#pragma unroll
-        for (int k = 0; k < PER; ++k)
-            if (bits & (1u << k)) {
-                cz[w] = pz[k];
-                cpos[w] = pp_[k];
-                ++w;
-            }
-        __syncthreads();
-        const int mine = ns > warp ? ceil_div(ns - warp, TAU_WARPS) : 0;  // tokens warp, warp+16, ...
-        for (int base = 0; base < mine; base += 8) {
-            const int nr = min(8, mine - base);
+            for (int i = 0; i < 8; ++i)
+                if (bal) {
+                    const int l = __ffs(bal) - 1;
+                    bal &= bal - 1;
+                    if (lane == i) src = l;
+                    nr = i + 1;
+                }
+            const int cs = k0 + __shfl_sync(FULL, lane, src) * TAU_WARPS + warp;
+            const float pl = __shfl_sync(FULL, p, src);
             int row = 0;
-            float p = 0.f;
             if (lane < nr) {
-                const int i = warp + TAU_WARPS * (base + lane);
-                p = cz[i];
-                row = row_of(cpos[i], p);
+                const int pos = onchip ? cpos[cs] : cs;
+                row = onchip ? crow[cs] : row_of_pos(pos);
+                put_p(pos, pl);
             }
-            gather8(nr, row, p);
-        }
-    } else {
-        for (int c0 = warp * 32; c0 < nloop; c0 += TAU_WARPS * 32) {
-            const int c = c0 + lane;
-            const float z = c < nloop ? cz_at(c) : -INFINITY;
-            const float p = pos_pow(z - tau, r, ri);
-            unsigned bal = __ballot_sync(FULL, p > 0.f);
-            while (bal) {
-                // the next (up to) eight lanes with weight move to lanes 0..7
-                int src = 0, nr = 0;
-#pragma unroll
-                for (int i = 0; i < 8; ++i)
-                    if (bal) {
-                        const int l = __ffs(bal) - 1;
-                        bal &= bal - 1;
-                        if (lane == i) src = l;
-                        nr = i + 1;
-                    }
-                const int cc = c0 + __shfl_sync(FULL, lane, src);
-                const float pl = __shfl_sync(FULL, p, src);
-                int row = 0;
-                if (lane < nr) row = row_of(cc, pl);
-                gather8(nr, row, lane < nr ? pl : 0.f);
-            }
+            gather8(nr, row, lane < nr ? pl : 0.f);
         }
     }
     __syncthreads();  // every warp is done with the candidates
@@ -638,10 +635,10 @@ __global__ void __launch_bounds__(TAU_THREADS) tau_pv_kernel(const __grid_consta
     for (int cc = 0; cc < CPL; ++cc) accs[warp][lane * CPL + cc] = acc[cc];
     __syncthreads();
     for (int j = threadIdx.x; j < D; j += TAU_THREADS) {
-        double s = 0.0;
+        double sum = 0.0;
 #pragma unroll
-        for (int w = 0; w < TAU_WARPS; ++w) s += accs[w][j];
-        a.out[(size_t)bh * D + j] = (float)s;
+        for (int w = 0; w < TAU_WARPS; ++w) sum += accs[w][j];
+        a.out[(size_t)bh * D + j] = (float)sum;
     }
 }
 
@@ -1037,11 +1034,12 @@ template <int D, int G>
 cudaError_t sparse_t(const DecodeArgs &a, cudaStream_t st) {
     cudaError_t e;
     const int groups = a.B * a.Hkv;
-    const size_t ub = (size_t)ceil_div(a.max_pages, 4) * 4;
+    const size_t ub = (size_t)ceil_div(ceil_div(a.max_pages, UCL), 4) * 4;
     if ((e = set_smem(union_kernel, ub)) != cudaSuccess) return e;
-    if ((e = launch_pdl(union_kernel, dim3(groups), dim3(512), ub, st, a)) != cudaSuccess) return e;
+    if ((e = launch_pdl(union_kernel, dim3(groups * UCL), dim3(UTH), ub, st, a)) != cudaSuccess) return e;
     if ((e = launch_qk<D, G, false>(a, st)) != cudaSuccess) return e;
-    return launch_pdl(tau_pv_kernel<D, true>, dim3(a.B * a.Hq), dim3(TAU_THREADS), 0, st, a, 0);
+    if ((e = set_smem(tau_pv_kernel<D, true>, TAU_SMEM)) != cudaSuccess) return e;
+    return launch_pdl(tau_pv_kernel<D, true>, dim3(a.B * a.Hq), dim3(TAU_THREADS), TAU_SMEM, st, a, 0);
 }
 
 template <int D, int G>
@@ -1051,7 +1049,8 @@ cudaError_t dense_entmax_t(const DecodeArgs &a, cudaStream_t st) {
     const int n = a.B * a.Hq > groups ? a.B * a.Hq : groups;
     if ((e = launch_pdl(dense_init_kernel, dim3(ceil_div(n, 256)), dim3(256), 0, st, a)) != cudaSuccess) return e;
     if ((e = launch_qk<D, G, true>(a, st)) != cudaSuccess) return e;
-    if ((e = launch_pdl(tau_pv_kernel<D, false>, dim3(a.B * a.Hq), dim3(TAU_THREADS), 0, st, a, 1)) != cudaSuccess) return e;
+    if ((e = set_smem(tau_pv_kernel<D, false>, TAU_SMEM)) != cudaSuccess) return e;
+    if ((e = launch_pdl(tau_pv_kernel<D, false>, dim3(a.B * a.Hq), dim3(TAU_THREADS), TAU_SMEM, st, a, 1)) != cudaSuccess) return e;
     using RG = Ring<D, G, 4, 1>;
     auto k = pv_stream_kernel<D, G>;
     if ((e = set_smem(k, RG::BYTES)) != cudaSuccess) return e;
