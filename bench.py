@@ -44,9 +44,9 @@ PAPER_CONTEXT = {"speedup_vs_full_softmax_flashdecoding": 3.36, "speedup_vs_full
 # DRAM bytes per launch from ncu captures (dram__bytes_read.sum + dram__bytes_write.sum),
 # keyed by kernel and workload, valid only while the kernel source is unchanged.
 NCU_TRAFFIC = {
-    # captured at L=524,288 (100.73 MB read + 5.94 MB written per launch), scaled by 2 for the
+    # captured at L=524,288 (100.69 MB read + 3.61 MB written per launch), scaled by 2 for the
     # 1,048,576-token context: the scan is linear in the page count (profiles/step_kernels_*)
-    "score_pages/gauss_gqa_L1m": {"bytes": 2 * (100726016 + 5942016), "src": "761bf1cf5895"},
+    "score_pages/gauss_gqa_L1m": {"bytes": 2 * (100689152 + 3609088), "src": "edea3177cd8b"},
 }
 
 
@@ -342,23 +342,24 @@ def run_gpu(args, rank, world):
     assert nv.get_status(clear=True) & ~nv.STATUS_OVERFLOW == 0
 
     peak, peak_kind = measured_peaks()
-    # dominant kernel of the step
-    dom = max(("score_pages", "decode_sparse"), key=lambda s: stage_us[s])
-    if dom == "score_pages":
-        alg = nbytes["meta"] + nbytes["scores"] + wl.B * wl.Hq * wl.d * 2
-        src = "score.cu"
-    else:
-        alg = nbytes["gather_k"] + nbytes["gather_v"] + nbytes["qo"]
-        src = "decode.cu"
+    # dominant kernel of the step: score_pages is a single launch (the sparse
+    # decode stage is three kernels and is reported beside it)
+    dom = "score_pages"
+    alg = nbytes["meta"] + nbytes["scores"] + wl.B * wl.Hq * wl.d * 2
     achieved = alg / (stage_us[dom] * 1e-6) / 1e9
     tr = NCU_TRAFFIC.get(f"{dom}/{args.workload}")
-    traffic = tr["bytes"] if tr and tr.get("src") == _src_hash(src) else None  # null once the kernel changed
+    traffic = tr["bytes"] if tr and tr.get("src") == _src_hash("score.cu") else None  # null once the kernel changed
     roofline = {"bound": "hbm", "kernel": dom, "achieved": round(achieved, 1), "peak": peak, "unit": "GB/s",
                 "frac": round(achieved / peak, 4), "traffic": traffic, "algorithmic_bytes": alg,
                 "peak_kind": f"{peak_kind} copy bandwidth (burst)"}
+    galg = nbytes["gather_k"] + nbytes["gather_v"] + nbytes["qo"]
+    gach = galg / (stage_us["decode_sparse"] * 1e-6) / 1e9
+    roofline_gather = {"bound": "hbm", "kernel": "decode_sparse (union, q.K, tau with p.V)",
+                       "achieved": round(gach, 1), "peak": peak, "unit": "GB/s", "frac": round(gach / peak, 4),
+                       "algorithmic_bytes": galg}
     res = dict(wl=wl, step_ms=step_ms, eager_step_ms=eager_step_ms, e2e_eager_ms=e2e_eager_ms,
                stage_us=stage_us, dense=dense, nbytes=nbytes, clocks=clocks,
-               roofline=roofline, e2e_ms=e2e_step_ms, e2e_bytes=(q_host.numel() * 2 + k_new.numel() * 4,
+               roofline=roofline, roofline_gather=roofline_gather, e2e_ms=e2e_step_ms, e2e_bytes=(q_host.numel() * 2 + k_new.numel() * 4,
                                                                out_host.numel() * 4),
                launches=kernels_per_step(policy == "gauss", True) * args.steps, t_wall=t_wall,
                host=dict(inp=inp, dec=dec) if (rank == 0 and not args.no_cpu_baseline) else None)
@@ -493,7 +494,8 @@ def main():
             "us_per_step": round(res["step_ms"] * 1e3, 2), "higher_is_better": True, "scaling": "weak",
             "vs_baseline": None, "dtype": "bf16", "data": "synthetic", "config": config_of(wl),
             "frac_of_hbm_peak": round(value / world / res["roofline"]["peak"], 4),
-            "roofline": res["roofline"], "stages_us": res["stage_us"], "bytes_per_step": nb,
+            "roofline": res["roofline"], "roofline_gather": res["roofline_gather"],
+            "stages_us": res["stage_us"], "bytes_per_step": nb,
             "e2e": {"value": round(e2e_val, 2), "unit": "GB/s", "us_per_step": round(res["e2e_ms"] * 1e3, 2),
                     "h2d_bytes_per_step": res["e2e_bytes"][0], "d2h_bytes_per_step": res["e2e_bytes"][1],
                     "how": "H2D of q and the appended token's k/v from pinned memory, append, step, D2H of the "

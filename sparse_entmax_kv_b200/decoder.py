@@ -66,5 +66,5 @@ class EntmaxKVDecoder:
 
 def kernels_per_step(policy_gauss: bool, append: bool) -> int:
     """Kernel launches one ``step`` issues: build_meta (1, if appending),
-    score (1), select (1), decode_sparse (union, q.K, tau, p.V = 4)."""
-    return (1 if append else 0) + 1 + 1 + 4
+    score (1), select (1), decode_sparse (union, q.K, tau with p.V = 3)."""
+    return (1 if append else 0) + 1 + 1 + 3
