@@ -50,6 +50,21 @@ NCU_TRAFFIC = {
 }
 
 
+def max_over_ranks(vals, world, device):
+    """Each value's maximum over all ranks (the slowest rank's device time)."""
+    if world == 1:
+        return [float(v) for v in vals]
+    t = torch.tensor([float(v) for v in vals], dtype=torch.float64, device=device)
+    torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
+    return t.tolist()
+
+
+def whole_job_gbs(bytes_per_rank, world, step_ms):
+    """Whole-job throughput: every rank moves bytes_per_rank per step (weak
+    scaling, one independent problem per rank), timed by the slowest rank."""
+    return world * bytes_per_rank / (step_ms * 1e-3) / 1e9
+
+
 def _src_hash(fname):
     p = os.path.join(ROOT, "sparse_entmax_kv_b200", "csrc", fname)
     return hashlib.sha1(open(p, "rb").read()).hexdigest()[:12]
@@ -262,10 +277,7 @@ def run_gpu(args, rank, world):
     step_ms = float(np.mean([a.elapsed_time(b) for a, b in gev]))
     stage_ms = np.array([[ev[i][j].elapsed_time(ev[i][j + 1]) for j in range(nst)] for i in range(args.steps)])
     eager_step_ms = float(stage_ms.sum(axis=1).mean())
-    if world > 1:
-        t = torch.tensor([step_ms], device=dev)
-        torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
-        step_ms = float(t.item())
+    step_ms, = max_over_ranks([step_ms], world, dev)
     stage_us = dict(zip(["build_meta_append", "score_pages", "select", "decode_sparse"],
                         (stage_ms.mean(axis=0) * 1e3).round(2).tolist()))
 
@@ -335,10 +347,7 @@ def run_gpu(args, rank, world):
     torch.cuda.synchronize()
     e2e_step_ms = time_e2e(g2.replay)
     e2e_eager_ms = time_e2e(e2e_once)
-    if world > 1:
-        t = torch.tensor([e2e_step_ms, e2e_eager_ms], device=dev)
-        torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
-        e2e_step_ms, e2e_eager_ms = (float(x) for x in t.tolist())
+    e2e_step_ms, e2e_eager_ms = max_over_ranks([e2e_step_ms, e2e_eager_ms], world, dev)
     assert nv.get_status(clear=True) & ~nv.STATUS_OVERFLOW == 0
 
     peak, peak_kind = measured_peaks()
@@ -487,8 +496,8 @@ def main():
     res = run_gpu(args, rank, world)
     wl = res["wl"]
     nb = res["nbytes"]
-    value = world * nb["kv_touched"] / (res["step_ms"] * 1e-3) / 1e9
-    e2e_val = world * nb["kv_touched"] / (res["e2e_ms"] * 1e-3) / 1e9
+    value = whole_job_gbs(nb["kv_touched"], world, res["step_ms"])
+    e2e_val = whole_job_gbs(nb["kv_touched"], world, res["e2e_ms"])
     line = {"metric": METRIC, "value": round(value, 2), "unit": "GB/s", "n_gpus": world, "steps": args.steps,
             "warmup": args.warmup, "ms_per_step": round(res["step_ms"], 5),
             "us_per_step": round(res["step_ms"] * 1e3, 2), "higher_is_better": True, "scaling": "weak",
