@@ -3,8 +3,8 @@
 // One CTA per (sequence, query head).
 //
 // Top-k: radix select on the order-preserving 32-bit image of the fp32 bound
-// (four 8-bit digits, most significant first; warp-aggregated shared-memory
-// histograms), which pins the k-th largest key T and how many keys equal to T
+// (four 8-bit digits, most significant first; per-warp shared-memory
+// histograms summed after each pass), which pins the k-th largest key T and how many keys equal to T
 // are still needed; a single ordered pass then keeps keys > T plus the first
 // such keys == T in page order (ties to the lower page index) and writes them
 // in ascending page order.  No sort.
@@ -42,6 +42,7 @@ __device__ __forceinline__ unsigned key_of(float f) {
 // ordered compaction; longer sequences take several tiles per pass.
 __global__ void __launch_bounds__(SEL_THREADS) topk_kernel(SelectArgs a) {
     pdl_wait();
+    __shared__ int whist[SEL_THREADS / 32][256];  // one histogram per warp (contention stays inside a warp)
     __shared__ int hist[256];
     __shared__ int sh[72];
     __shared__ int pick[2];
@@ -56,7 +57,7 @@ __global__ void __launch_bounds__(SEL_THREADS) topk_kernel(SelectArgs a) {
         if (threadIdx.x == 0) a.cnt[bh] = n;
         return;
     }
-    const int lane = threadIdx.x & 31;
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
     const bool one_tile = n <= TILE;
     unsigned key[ITEMS];
     auto load_tile = [&](int t0) {
@@ -68,18 +69,21 @@ __global__ void __launch_bounds__(SEL_THREADS) topk_kernel(SelectArgs a) {
     unsigned prefix = 0, mask = 0;
     int remaining = k;
     for (int shift = 24; shift >= 0; shift -= 8) {
-        for (int i = threadIdx.x; i < 256; i += blockDim.x) hist[i] = 0;
+        for (int i = threadIdx.x; i < (SEL_THREADS / 32) * 256; i += blockDim.x) (&whist[0][0])[i] = 0;
         __syncthreads();
         for (int t0 = 0; t0 < n; t0 += TILE) {
             if (!one_tile) load_tile(t0);
             const int p0 = t0 + threadIdx.x * ITEMS;
 #pragma unroll
-            for (int i = 0; i < ITEMS; ++i) {
-                int bucket = 256 + lane;  // unique dummy for lanes with nothing to count
-                if (p0 + i < n && (key[i] & mask) == prefix) bucket = (key[i] >> shift) & 255;
-                const unsigned peers = __match_any_sync(FULL, bucket);
-                if (bucket < 256 && lane == __ffs(peers) - 1) atomicAdd(&hist[bucket], __popc(peers));
-            }
+            for (int i = 0; i < ITEMS; ++i)
+                if (p0 + i < n && (key[i] & mask) == prefix) atomicAdd(&whist[warp][(key[i] >> shift) & 255], 1);
+        }
+        __syncthreads();
+        if (threadIdx.x < 256) {
+            int c = 0;
+#pragma unroll 8
+            for (int w = 0; w < SEL_THREADS / 32; ++w) c += whist[w][threadIdx.x];
+            hist[threadIdx.x] = c;
         }
         __syncthreads();
         if (threadIdx.x < 32) {
