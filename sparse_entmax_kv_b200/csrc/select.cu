@@ -40,9 +40,11 @@ __device__ __forceinline__ unsigned key_of(float f) {
 // Top-k: the keys of one tile (TILE pages) stay in registers, ITEMS
 // consecutive pages per thread, through the four radix passes and the final
 // ordered compaction; longer sequences take several tiles per pass.
-__global__ void __launch_bounds__(SEL_THREADS) topk_kernel(SelectArgs a) {
+template <int NT>
+__global__ void __launch_bounds__(NT) topk_kernel(SelectArgs a) {
+    constexpr int TILE_NT = NT * ITEMS;
     pdl_wait();
-    __shared__ int whist[SEL_THREADS / 32][256];  // one histogram per warp (contention stays inside a warp)
+    __shared__ int whist[NT / 32][256];  // one histogram per warp (contention stays inside a warp)
     __shared__ int hist[256];
     __shared__ int sh[72];
     __shared__ int pick[2];
@@ -58,7 +60,7 @@ __global__ void __launch_bounds__(SEL_THREADS) topk_kernel(SelectArgs a) {
         return;
     }
     const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
-    const bool one_tile = n <= TILE;
+    const bool one_tile = n <= TILE_NT;
     unsigned key[ITEMS];
     auto load_tile = [&](int t0) {
         const int p0 = t0 + threadIdx.x * ITEMS;
@@ -69,9 +71,9 @@ __global__ void __launch_bounds__(SEL_THREADS) topk_kernel(SelectArgs a) {
     unsigned prefix = 0, mask = 0;
     int remaining = k;
     for (int shift = 24; shift >= 0; shift -= 8) {
-        for (int i = threadIdx.x; i < (SEL_THREADS / 32) * 256; i += blockDim.x) (&whist[0][0])[i] = 0;
+        for (int i = threadIdx.x; i < (NT / 32) * 256; i += blockDim.x) (&whist[0][0])[i] = 0;
         __syncthreads();
-        for (int t0 = 0; t0 < n; t0 += TILE) {
+        for (int t0 = 0; t0 < n; t0 += TILE_NT) {
             if (!one_tile) load_tile(t0);
             const int p0 = t0 + threadIdx.x * ITEMS;
 #pragma unroll
@@ -82,7 +84,7 @@ __global__ void __launch_bounds__(SEL_THREADS) topk_kernel(SelectArgs a) {
         if (threadIdx.x < 256) {
             int c = 0;
 #pragma unroll 8
-            for (int w = 0; w < SEL_THREADS / 32; ++w) c += whist[w][threadIdx.x];
+            for (int w = 0; w < NT / 32; ++w) c += whist[w][threadIdx.x];
             hist[threadIdx.x] = c;
         }
         __syncthreads();
@@ -125,7 +127,7 @@ __global__ void __launch_bounds__(SEL_THREADS) topk_kernel(SelectArgs a) {
     const unsigned T = prefix;
     // keys == T are taken in page order up to `remaining` of them
     int eq_base = 0, base = 0;
-    for (int t0 = 0; t0 < n; t0 += TILE) {
+    for (int t0 = 0; t0 < n; t0 += TILE_NT) {
         if (!one_tile) load_tile(t0);
         const int p0 = t0 + threadIdx.x * ITEMS;
         unsigned gt = 0, eq = 0;
@@ -631,7 +633,11 @@ cudaError_t launch_select(const SelectArgs &a, cudaStream_t st) {
     const int grid = a.B * a.Hq;
     cudaError_t e = cudaSuccess;
     if (a.policy == ENTMAXKV_TOPK) {
-        e = launch_pdl(topk_kernel, dim3(grid), dim3(SEL_THREADS), 0, st, a);
+        // short sequences: a quarter of the threads holds every page in registers
+        if (a.max_pages <= 256 * ITEMS)
+            e = launch_pdl(topk_kernel<256>, dim3(grid), dim3(256), 0, st, a);
+        else
+            e = launch_pdl(topk_kernel<SEL_THREADS>, dim3(grid), dim3(SEL_THREADS), 0, st, a);
     } else if (a.max_pages <= GCL * GTH * GIT) {
         switch (a.r_int) {
             case 1: e = launch_pdl(gauss_cluster_kernel<1>, dim3(grid * GCL), dim3(GTH), 0, st, a); break;
