@@ -458,6 +458,60 @@ def run_reference(args, rank, world):
     print(json.dumps(line), flush=True)
 
 
+def run_l_sweep(args):
+    """Selection scaling with context length: for each L and policy (top-k 64,
+    Gaussian with the bound, Gaussian with the capped estimate), the eager
+    device time of each call of one step, medians over args.steps steps with
+    the L2 flushed before each.  One JSON line per (L, policy)."""
+    from sparse_entmax_kv_b200 import native as nv
+    from sparse_entmax_kv_b200.decoder import EntmaxKVDecoder
+    from sparse_entmax_kv_b200.workloads import CONFIGS, make_inputs
+    base = CONFIGS[args.workload]
+    dev = torch.device("cuda", torch.cuda.current_device())
+    flush_w = torch.empty(256 << 20, dtype=torch.uint8, device=dev)
+    flush_r = torch.ones(32 << 20, dtype=torch.int64, device=dev)
+    st = torch.cuda.current_stream()
+    for L in (65536, 131072, 262144, 524288, 1048576):
+        wl = base.shrink(L=L)
+        inp = make_inputs(wl, 4000, device=dev)
+        for policy in ("topk", "gauss", "gauss_est"):
+            dec = EntmaxKVDecoder(inp["k_cache"], inp["v_cache"], inp["page_table"], inp["seq_lens"], wl.Hq,
+                                  alpha=wl.alpha, policy=policy, k=64, delta=wl.delta or 0.5)
+            dec.build_meta()
+            calls = [
+                lambda: nv.entmaxkv_score_pages(dec.shape, inp["q"], dec.meta, dec.seq_lens, dec.bbox, dec.mu,
+                                                dec.sigma),
+                lambda: nv.entmaxkv_select(dec.shape, dec.seq_lens, dec.bbox, dec.mu, dec.sigma, dec.policy, dec.k,
+                                           dec.alpha, dec.delta, dec.sel, dec.cnt, dec.tau_hat),
+                lambda: nv.entmaxkv_decode_sparse(dec.shape, inp["q"], dec.k_cache, dec.v_cache, dec.page_table,
+                                                  dec.seq_lens, dec.sel, dec.cnt, dec.alpha, dec.out, dec.tau, None,
+                                                  dec.ws)]
+            ts = []
+            for i in range(args.warmup + args.steps):
+                flush_w.fill_(1)
+                torch.amax(flush_r)
+                ev = [torch.cuda.Event(enable_timing=True) for _ in range(len(calls) + 1)]
+                ev[0].record(st)
+                for c, e in zip(calls, ev[1:]):
+                    c()
+                    e.record(st)
+                torch.cuda.synchronize()
+                if i >= args.warmup:
+                    ts.append([ev[j].elapsed_time(ev[j + 1]) * 1e3 for j in range(len(calls))])
+            assert nv.get_status(clear=True) & ~nv.STATUS_OVERFLOW == 0
+            med = np.median(np.array(ts), axis=0)
+            print(json.dumps({"sweep": "context_length", "workload": base.name, "L": L, "policy": policy,
+                              "k": 64 if policy == "topk" else None, "delta": None if policy == "topk" else wl.delta,
+                              "score_us": round(float(med[0]), 2), "select_us": round(float(med[1]), 2),
+                              "decode_sparse_us": round(float(med[2]), 2),
+                              "step_us_eager": round(float(med.sum()), 2),
+                              "pages_selected_mean": round(float(dec.cnt.float().mean()), 1),
+                              "pages": wl.max_pages}), flush=True)
+            del dec
+        del inp
+        torch.cuda.empty_cache()
+
+
 def config_of(wl):
     return {"workload": wl.name, "B": wl.B, "Hq": wl.Hq, "Hkv": wl.Hkv, "d": wl.d, "L": wl.L,
             "page_size": wl.P, "alpha": wl.alpha, "policy": wl.policy, "k": wl.k, "delta": wl.delta,
@@ -476,6 +530,8 @@ def main():
     ap.add_argument("--dense-steps", type=int, default=5)
     ap.add_argument("--skip-dense", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--l-sweep", action="store_true",
+                    help="instead of the benchmark line: selection scaling with context length (one line per L, policy)")
     args = ap.parse_args()
     args.warmup = max(args.warmup, 3)
 
@@ -487,6 +543,9 @@ def main():
         return
 
     torch.cuda.set_device(local)
+    if args.l_sweep:
+        run_l_sweep(args)
+        return
     if world > 1:
         import datetime
         torch.distributed.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),

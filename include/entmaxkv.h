@@ -89,7 +89,7 @@ enum {
 /* Size of the fixed on-device scratch used by entmaxkv_decode_sparse_static. */
 #define ENTMAXKV_STATIC_SCRATCH_BYTES ((size_t)16 << 20)
 
-enum { ENTMAXKV_TOPK = 0, ENTMAXKV_GAUSS = 1 };
+enum { ENTMAXKV_TOPK = 0, ENTMAXKV_GAUSS = 1, ENTMAXKV_GAUSS_EST = 2 };
 
 /* `call` argument of entmaxkv_workspace_size */
 enum {
@@ -202,8 +202,14 @@ ENTMAXKV_API int entmaxkv_score_pages(const entmaxkv_shape *shape, const void *q
  *                  and the pages kept are those with (alpha-1) bbox_p >
  *                  tau_hat - delta (the bound is the estimated max score).
  *                  tau_hat (nullable, fp32 [B][Hq]) receives the solution.
+ *  ENTMAXKV_GAUSS_EST: as ENTMAXKV_GAUSS, but the estimated max score of a
+ *                  page comes from its Gaussian model, capped by the bound:
+ *                  keep p if (alpha-1) min(bbox_p, mu_p + z(n_p) sigma_p) >
+ *                  tau_hat - delta, z(n) = sqrt(2 ln n) (z(1) = 0).  Keeps a
+ *                  subset of ENTMAXKV_GAUSS's pages; unlike it, it can drop a
+ *                  page holding a support token.
  * sel is int32 [B][Hq][max_pages], cnt int32 [B][Hq].  Needs alpha > 1 for
- * the Gaussian policy.  workspace may be NULL when entmaxkv_workspace_size
+ * the Gaussian policies.  workspace may be NULL when entmaxkv_workspace_size
  * reports 0.
  */
 ENTMAXKV_API int entmaxkv_select(const entmaxkv_shape *shape, const int32_t *seq_lens,

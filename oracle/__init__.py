@@ -35,6 +35,10 @@ def lib():
         L.orc_select_topk.restype = i
         L.orc_select_gauss.argtypes = [i, P, dbl, dbl, dbl, P]
         L.orc_select_gauss.restype = i
+        L.orc_select_gauss_est.argtypes = [i, P, P, P, P, dbl, dbl, dbl, P]
+        L.orc_select_gauss_est.restype = i
+        L.orc_zmax_of.argtypes = [i]
+        L.orc_zmax_of.restype = dbl
         for fn in ("orc_sparsemax_tau", "orc_entmax15_tau"):
             getattr(L, fn).argtypes = [P, i]
             getattr(L, fn).restype = dbl
@@ -117,6 +121,20 @@ def select_gauss(bbox, alpha, tau_hat_v, delta):
     return sel[:n]
 
 
+def select_gauss_est(bbox, mu, sigma, n_tok, alpha, tau_hat_v, delta):
+    """Gaussian rule with the capped Gaussian estimate of each page's max."""
+    bbox, mu, sigma = (_c(x, np.float32) for x in (bbox, mu, sigma))
+    n_tok = _c(n_tok, np.int32)
+    sel = np.zeros(max(1, len(bbox)), np.int32)
+    n = lib().orc_select_gauss_est(len(bbox), _p(bbox), _p(mu), _p(sigma), _p(n_tok), float(alpha),
+                                   float(tau_hat_v), float(delta), _p(sel))
+    return sel[:n]
+
+
+def zmax_of(n: int) -> float:
+    return lib().orc_zmax_of(int(n))
+
+
 def select(seq_lens, bbox, mu, sigma, P, policy, k, alpha, delta):
     """Batched selection: sel [B][Hq][max_pages], cnt [B][Hq], tau_hat [B][Hq]."""
     seq_lens = _c(seq_lens, np.int32)
@@ -127,7 +145,7 @@ def select(seq_lens, bbox, mu, sigma, P, policy, k, alpha, delta):
     sel = np.full((B, Hq, max_pages), -1, np.int32)
     cnt = np.zeros((B, Hq), np.int32)
     th = np.full((B, Hq), np.nan, np.float64)
-    pol = {"topk": 0, "gauss": 1}[policy]
+    pol = {"topk": 0, "gauss": 1, "gauss_est": 2}[policy]
     lib().orc_select(B, Hq, P, max_pages, _p(seq_lens), _p(bbox), _p(mu), _p(sigma),
                      pol, int(k), float(alpha), float(delta), _p(sel), _p(cnt), _p(th))
     return sel, cnt, th

@@ -30,6 +30,9 @@
  *     with X_p ~ N((alpha-1) mu_p, (alpha-1)^2 sigma_p^2), r = 1/(alpha-1);
  *   the "estimated max score" of a page is its bounding-box bound, compared on
  *     the z = (alpha-1) s scale: keep p if (alpha-1) u_p > tau_hat - Delta;
+ *   a variant estimates it from the page's Gaussian model, capped by the
+ *     bound: min(u_p, mu_p + z(n_p) sigma_p), z(n) = sqrt(2 ln n) (the usual
+ *     estimate of the largest of n standard normal draws; z(1) = 0);
  *   top-k ties go to the lower page index; selections are listed ascending.
  *
  * Arithmetic rules (so that results are defined to the bit where stated):
@@ -289,6 +292,32 @@ int orc_select_gauss(int n_pages, const float *bbox, double alpha,
     return c;
 }
 
+/*
+ * Section 2.B, Gaussian rule with the estimated maximum taken from the page's
+ * Gaussian model and capped by the bound (the bound is never below the true
+ * maximum, the model's estimate may be):
+ *   keep p if (alpha-1) min(u_p, mu_p + z(n_p) sigma_p) > tau_hat - Delta,
+ *   z(n) = sqrt(2 ln n) for n >= 2, z(1) = 0.
+ */
+double orc_zmax_of(int n)
+{
+    return n >= 2 ? sqrt(2.0 * log((double)n)) : 0.0;
+}
+
+int orc_select_gauss_est(int n_pages, const float *bbox, const float *mu,
+                         const float *sigma, const int32_t *n_tok, double alpha,
+                         double tau_hat, double delta, int32_t *sel)
+{
+    int c = 0;
+    double thr = tau_hat - delta;
+    for (int p = 0; p < n_pages; ++p) {
+        double est = (double)mu[p] + orc_zmax_of(n_tok[p]) * (double)sigma[p];
+        if ((double)bbox[p] < est) est = (double)bbox[p];
+        if ((alpha - 1.0) * est > thr) sel[c++] = p;
+    }
+    return c;
+}
+
 /* ------------------------------------------------------ entmax threshold */
 
 static int cmp_double_desc(const void *a, const void *b)
@@ -472,7 +501,8 @@ void orc_decode(int B, int Hq, int Hkv, int d, int P, int max_pages,
 
 /*
  * Scores and page selection for a whole batch (the middle of one decode step):
- * per (b, h) either top-k (policy 0) or the Gaussian rule (policy 1).
+ * per (b, h) either top-k (policy 0), the Gaussian rule with the bound as the
+ * estimated maximum (policy 1) or with the capped Gaussian estimate (policy 2).
  * sel is [B][Hq][max_pages], cnt and tau_hat are [B][Hq] (tau_hat NAN for top-k).
  */
 void orc_select(int B, int Hq, int P, int max_pages, const int32_t *seq_lens,
@@ -494,9 +524,13 @@ void orc_select(int B, int Hq, int P, int max_pages, const int32_t *seq_lens,
                 int32_t *nt = (int32_t *)malloc(sizeof(int32_t) * (size_t)(np ? np : 1));
                 for (int p = 0; p < np; ++p) nt[p] = tokens_in_page(seq_lens[b], P, p);
                 double th = orc_tau_hat(np, mu + bh * max_pages, sigma + bh * max_pages, nt, alpha);
-                free(nt);
                 tau_hat[bh] = th;
-                cnt[bh] = orc_select_gauss(np, bb, alpha, th, delta, sl);
+                if (policy == 1)
+                    cnt[bh] = orc_select_gauss(np, bb, alpha, th, delta, sl);
+                else
+                    cnt[bh] = orc_select_gauss_est(np, bb, mu + bh * max_pages, sigma + bh * max_pages, nt,
+                                                   alpha, th, delta, sl);
+                free(nt);
             }
         }
     }

@@ -257,7 +257,7 @@ int entmaxkv_select(const entmaxkv_shape *s, const int32_t *seq_lens, const floa
     SelectArgs a{};
     if (policy == ENTMAXKV_TOPK) {
         if (k < 1) return ENTMAXKV_ERR_POLICY;
-    } else if (policy == ENTMAXKV_GAUSS) {
+    } else if (policy == ENTMAXKV_GAUSS || policy == ENTMAXKV_GAUSS_EST) {
         if (!mu || !sigma) return ENTMAXKV_ERR_NULL;
         if (!std::isfinite(delta)) return ENTMAXKV_ERR_POLICY;
         if (!std::isfinite(alpha) || !(alpha > 1.f)) return ENTMAXKV_ERR_ALPHA;

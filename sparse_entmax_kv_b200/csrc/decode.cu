@@ -385,7 +385,7 @@ __global__ void __launch_bounds__(DEC_THREADS) qk_kernel(const __grid_constant__
 
 constexpr int TAU_THREADS = 512;
 constexpr int TAU_WARPS = TAU_THREADS / 32;
-constexpr int ZCAP = 4096;  // candidates held on chip per head
+constexpr int ZCAP = 8192;  // candidates held on chip per head
 constexpr int TAU_TB = 8;   // tile maxima in flight per lane
 constexpr size_t TAU_SMEM = (size_t)ZCAP * 16;
 
@@ -525,9 +525,19 @@ __global__ void __launch_bounds__(TAU_THREADS) tau_pv_kernel(const __grid_consta
                 const int c1 = min(nc, (warp + 1) * per);
                 for (int c = warp * per; c < c1; ++c) f += pos_pow(cz[c] - t, r, ri);
             } else {
-                for (int c = warp; c < n_tok; c += TAU_WARPS) {
-                    const float z = __ldcg(zr + c);
-                    if (z > thr) f += pos_pow(z - t, r, ri);
+                // too many candidates to hold: stream the z row through shared
+                // memory in coalesced chunks of ZCAP, each warp summing a slice
+                for (int c0 = 0; c0 < n_tok; c0 += ZCAP) {
+                    const int m = min(ZCAP, n_tok - c0);
+                    __syncthreads();  // the previous chunk has been read
+                    for (int i = threadIdx.x; i < m; i += TAU_THREADS) cz[i] = __ldcg(zr + c0 + i);
+                    __syncthreads();
+                    const int per = ceil_div(m, TAU_WARPS);
+                    const int c1 = min(m, (warp + 1) * per);
+                    for (int c = warp * per; c < c1; ++c) {
+                        const float z = cz[c];
+                        if (z > thr) f += pos_pow(z - t, r, ri);
+                    }
                 }
             }
             red[warp][lane] = f;

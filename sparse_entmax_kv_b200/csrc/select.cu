@@ -9,7 +9,9 @@
 // such keys == T in page order (ties to the lower page index) and writes them
 // in ascending page order.  No sort.
 //
-// Gaussian: tau_hat solves F(tau) = sum_p n_p E[(X_p - tau)_+^r] = 1 with
+// Gaussian (and its estimated-max variant, which keeps a page when
+// (alpha-1) min(bound, mu + sqrt(2 ln n) sigma) clears the cut):
+// tau_hat solves F(tau) = sum_p n_p E[(X_p - tau)_+^r] = 1 with
 // X_p ~ N(m_p, s_p^2), m_p = (alpha-1) mu_p, s_p = (alpha-1) sigma_p, using the
 // closed-form Gaussian partial moments.  F is decreasing, F >= 1 at
 // tau0 = max_p (m_p - n_p^(-1/r)) (Jensen) and F < 1 at max_p (m_p + 10 s_p)
@@ -217,6 +219,9 @@ __device__ __forceinline__ void gauss_contrib(float m, float s, float w, float t
     }
 }
 
+// Estimated maximum of n standard normal draws, sqrt(2 ln n) (0 for n = 1).
+__device__ __forceinline__ float zmax_of(int n) { return n >= 2 ? sqrtf(2.f * logf((float)n)) : 0.f; }
+
 // One Newton step on g = F^(1/R) from tau towards the root, kept below hi.
 // Returns false when tau has converged (F <= 1 within 2e-6, or a step below
 // 1e-7 max(1, |tau|)).
@@ -381,6 +386,8 @@ __global__ void __launch_bounds__(SEL_THREADS) gauss_kernel(SelectArgs a) {
     if (threadIdx.x == 0 && a.tau_hat) a.tau_hat[bh] = tau;
 
     const float thr = tau - a.delta;
+    const bool est = a.policy == ENTMAXKV_GAUSS_EST;
+    const float z_full = zmax_of(a.P), z_last = zmax_of(tokens_in_page(seq, a.P, n - 1));
     int *sel = a.sel + row;
     int base = 0;
     for (int t0 = 0; t0 < n; t0 += TILE) {
@@ -391,8 +398,15 @@ __global__ void __launch_bounds__(SEL_THREADS) gauss_kernel(SelectArgs a) {
         }
         unsigned bits = 0;
 #pragma unroll
-        for (int i = 0; i < ITEMS; ++i)
-            if (p0 + i < n && a1 * ub[i] > thr) bits |= 1u << i;
+        for (int i = 0; i < ITEMS; ++i) {
+            if (!(p0 + i < n)) continue;
+            float e = a1 * ub[i];
+            if (est) {
+                const int p = p0 + i;
+                e = fminf(e, a1 * __ldg(a.mu + row + p) + (p == n - 1 ? z_last : z_full) * a1 * __ldg(a.sigma + row + p));
+            }
+            if (e > thr) bits |= 1u << i;
+        }
         int tot;
         int w = base + block_excl_scan(__popc(bits), shi, &tot);
 #pragma unroll
@@ -603,12 +617,17 @@ __global__ void __cluster_dims__(GCL, 1, 1) __launch_bounds__(GTH) gauss_cluster
     }
     if (rank == 0 && threadIdx.x == 0 && a.tau_hat) a.tau_hat[bh] = tau;
 
-    // (4) pages with (alpha-1) bbox > tau_hat - Delta, ascending
+    // (4) pages with (alpha-1) x (estimated max) > tau_hat - Delta, ascending;
+    // the estimate is the bound, or min(bound, mu + z(n) sigma)
     const float thr = tau - a.delta;
+    const bool est = a.policy == ENTMAXKV_GAUSS_EST;
+    const float z_full = zmax_of(a.P), z_last = zmax_of(tokens_in_page(seq, a.P, n - 1));
     unsigned bits = 0;
 #pragma unroll
-    for (int i = 0; i < GIT; ++i)
-        if (p0 + i < hi_p && a1 * ub[i] > thr) bits |= 1u << i;
+    for (int i = 0; i < GIT; ++i) {
+        const float e = est ? fminf(a1 * ub[i], mm[i] + (p0 + i == n - 1 ? z_last : z_full) * ss[i]) : a1 * ub[i];
+        if (p0 + i < hi_p && e > thr) bits |= 1u << i;
+    }
     int ls;
     int o = block_excl_scan(__popc(bits), sh, &ls);
     if (threadIdx.x < GCL) cl_sti(cl_map(&rsel[rank], threadIdx.x), ls);

@@ -28,8 +28,8 @@ class EntmaxKVDecoder:
         self.k_cache, self.v_cache = k_cache, v_cache
         self.page_table, self.seq_lens = page_table, seq_lens
         self.alpha, self.k, self.delta = float(alpha), int(k), float(delta)
-        self.policy = {"topk": nv.TOPK, "gauss": nv.GAUSS}[policy]
-        gauss = self.policy == nv.GAUSS
+        self.policy = {"topk": nv.TOPK, "gauss": nv.GAUSS, "gauss_est": nv.GAUSS_EST}[policy]
+        gauss = self.policy in (nv.GAUSS, nv.GAUSS_EST)
         self.meta = nv.alloc_meta(self.shape, dev)
         f32 = dict(dtype=torch.float32, device=dev)
         self.bbox = torch.empty((B, Hq, max_pages), **f32)

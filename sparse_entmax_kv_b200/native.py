@@ -21,7 +21,7 @@ OK = 0
 ERR = {0: "OK", -1: "ERR_NULL", -2: "ERR_SHAPE", -3: "ERR_ALPHA", -4: "ERR_POLICY",
        -5: "ERR_WORKSPACE", -6: "ERR_CUDA", -7: "ERR_UNSUPPORTED", -8: "ERR_ALIGN", -9: "ERR_TOO_LARGE"}
 STATIC_SCRATCH_BYTES = 16 << 20
-TOPK, GAUSS = 0, 1
+TOPK, GAUSS, GAUSS_EST = 0, 1, 2
 CALL_SELECT, CALL_DECODE_SPARSE, CALL_DECODE_DENSE = 2, 3, 4
 STATUS_BAD_PAGE, STATUS_BAD_SELECTION, STATUS_TIMEOUT, STATUS_OVERFLOW = 1, 2, 4, 8
 

@@ -195,10 +195,10 @@ def _oracle_scores(host, wl):
 
 
 @pytest.mark.parametrize("name", list(SMALL))
-@pytest.mark.parametrize("policy", ["topk", "gauss"])
+@pytest.mark.parametrize("policy", ["topk", "gauss", "gauss_est"])
 def test_select_parity(name, policy):
     wl = SMALL[name]
-    if policy == "gauss" and abs(1.0 / (wl.alpha - 1) - round(1.0 / (wl.alpha - 1))) > 1e-9:
+    if policy != "topk" and abs(1.0 / (wl.alpha - 1) - round(1.0 / (wl.alpha - 1))) > 1e-9:
         pytest.skip("Gaussian policy needs integer 1/(alpha-1)")
     inp, host = gpu_inputs(wl, 2)
     bbox, mu, sig = _oracle_scores(host, wl)   # oracle scores as the shared input
@@ -210,7 +210,7 @@ def test_select_parity(name, policy):
     th = torch.zeros((B, Hq), device="cuda")
     k = wl.k if wl.k else 16
     delta = wl.delta if wl.delta else 0.5
-    pol = nv.TOPK if policy == "topk" else nv.GAUSS
+    pol = {"topk": nv.TOPK, "gauss": nv.GAUSS, "gauss_est": nv.GAUSS_EST}[policy]
     nv.entmaxkv_select(s, inp["seq_lens"], tb, tm, ts, pol, k, wl.alpha, delta, sel, cnt, th)
     osel, ocnt, oth = orc.select(host["seq_lens"], np.nan_to_num(bbox, nan=0.0), np.nan_to_num(mu, nan=0.0),
                                  np.nan_to_num(sig, nan=0.0), wl.P, policy, k, wl.alpha, delta)
@@ -224,8 +224,13 @@ def test_select_parity(name, policy):
                 np.testing.assert_array_equal(gs, os_)
             else:
                 assert th[b, h] == pytest.approx(oth[b, h], abs=1e-5 * max(1.0, abs(oth[b, h])))
-                check_selection(gs, os_, (wl.alpha - 1) * bbox[b, h].astype(np.float64),
-                                oth[b, h] - delta, f"b{b}h{h}")
+                est = bbox[b, h].astype(np.float64)
+                if policy == "gauss_est":
+                    npb = n_pages(host, wl, b)
+                    ntok = [min(wl.P, int(host["seq_lens"][b]) - p * wl.P) for p in range(npb)]
+                    z = np.array([orc.zmax_of(t) for t in ntok] + [0.0] * (mp - npb))
+                    est = np.minimum(est, mu[b, h].astype(np.float64) + z * sig[b, h].astype(np.float64))
+                check_selection(gs, os_, (wl.alpha - 1) * est, oth[b, h] - delta, f"b{b}h{h}")
 
 
 def _oracle_selection(host, wl, policy, k, delta):

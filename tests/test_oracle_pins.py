@@ -378,6 +378,65 @@ def test_gauss_select_keeps_support_pages_when_threshold_is_low(orc):
         assert supp_pages <= set(sel.tolist())
 
 
+def test_zmax_of_closed_forms(orc):
+    """z(n)^2 = 2 ln n: z(64)^2 = 12 ln 2, z(e^2) would be 2; one token: 0."""
+    assert orc.zmax_of(64) ** 2 == pytest.approx(12 * math.log(2), rel=1e-15)
+    assert orc.zmax_of(2) ** 2 == pytest.approx(2 * math.log(2), rel=1e-15)
+    assert orc.zmax_of(1) == 0.0
+
+
+def test_gauss_est_hand_example(orc):
+    """Three pages worked by hand: alpha 1.5, tau_hat 1, Delta 0.5 (cut 0.5 on z).
+    Estimate: p0 min(2, 1 + 0.5 sqrt(2 ln 64)) = 2 -> z 1.0, kept; p1 min(1, 0.5 +
+    0.1 sqrt(2 ln 64)) = 0.788 -> 0.394, dropped; p2 min(3, 0.2 + 0.3 sqrt(2 ln 10))
+    = 0.844 -> 0.422, dropped.  Bound alone: z = 1.0, 0.5 (not above the cut), 1.5."""
+    bbox = np.array([2.0, 1.0, 3.0], np.float32)
+    mu = np.array([1.0, 0.5, 0.2], np.float32)
+    sig = np.array([0.5, 0.1, 0.3], np.float32)
+    n = np.array([64, 64, 10], np.int32)
+    np.testing.assert_array_equal(orc.select_gauss_est(bbox, mu, sig, n, 1.5, 1.0, 0.5), [0])
+    np.testing.assert_array_equal(orc.select_gauss(bbox, 1.5, 1.0, 0.5), [0, 2])
+
+
+@pytest.mark.parametrize("seed", range(6))
+def test_gauss_est_keeps_a_subset_of_the_bound_rule(orc, seed):
+    """min(u, mu + z sigma) <= u, so the estimate keeps a subset of what the
+    bound keeps, and the same pages where mu + z sigma >= u."""
+    rng = np.random.default_rng(1300 + seed)
+    n = 500
+    bbox = rng.normal(2.0, 1.0, n).astype(np.float32)
+    mu = (bbox - np.abs(rng.normal(1.0, 0.5, n))).astype(np.float32)
+    sig = np.abs(rng.normal(0.3, 0.3, n)).astype(np.float32)
+    nt = rng.integers(1, 65, n).astype(np.int32)
+    tau_hat, delta, alpha = float(rng.normal(1.0, 0.3)), 0.25, 1.5
+    est = set(orc.select_gauss_est(bbox, mu, sig, nt, alpha, tau_hat, delta).tolist())
+    bnd = set(orc.select_gauss(bbox, alpha, tau_hat, delta).tolist())
+    assert est <= bnd
+    capped = {p for p in range(n) if mu[p] + orc.zmax_of(int(nt[p])) * float(sig[p]) >= float(bbox[p])}
+    assert {p for p in bnd if p in capped} <= est
+
+
+def test_gauss_est_equals_bound_rule_on_constant_pages(orc):
+    """Pages whose tokens are all the same key: sigma = 0 and mu equals the bound
+    (both are q.k/sqrt(d) summed in the same order), so both rules agree."""
+    rng = np.random.default_rng(77)
+    Hq, Hkv, d, P, npg = 2, 1, 16, 8, 30
+    base = _random_pages(rng, npg, Hkv, 1, d)
+    K = np.repeat(base, P, axis=2)
+    q = f32_to_bf16_bits(rng.normal(size=(1, Hq, d)).astype(np.float32))
+    pt = np.arange(npg, dtype=np.int32).reshape(1, npg)
+    seq = np.array([npg * P], np.int32)
+    meta = orc.build_meta(K, pt, seq, Hkv, d, P, npg)
+    bbox, mu, sig = orc.score_pages(q, meta, pt, seq, Hkv, P)
+    assert np.all(sig == 0.0)
+    np.testing.assert_array_equal(mu, bbox)
+    nt = np.full(npg, P, np.int32)
+    for h in range(Hq):
+        t = float(np.median(bbox[0, h])) * 0.5
+        np.testing.assert_array_equal(orc.select_gauss_est(bbox[0, h], mu[0, h], sig[0, h], nt, 1.5, t, 0.1),
+                                      orc.select_gauss(bbox[0, h], 1.5, t, 0.1))
+
+
 # ----------------------------------------------------------------- decode
 
 def _decode_setup(seed, alpha, Hq=2, Hkv=1, d=16, P=8, npg=12):
