@@ -512,6 +512,75 @@ def run_l_sweep(args):
         torch.cuda.empty_cache()
 
 
+def run_quality(args):
+    """Approximation quality of sparse decoding at one kept set, entmax vs
+    softmax (synthetic data): for each selection policy, per head, against
+    the full-cache result of the same attention,
+      entmax:  discarded mass delta = sum of full-cache p off the kept tokens,
+               support recall (full-cache support tokens that were kept),
+               relative output error, and its ratio to the 2 B delta bound
+               (B = the largest value-row norm);
+      softmax: discarded mass 1 - exp(lse_kept - lse_full) and the relative
+               output error, on the same kept pages.
+    One JSON line per policy (means and extremes over heads)."""
+    from sparse_entmax_kv_b200 import native as nv
+    from sparse_entmax_kv_b200.decoder import EntmaxKVDecoder
+    from sparse_entmax_kv_b200.workloads import CONFIGS, make_inputs
+    wl = CONFIGS[args.workload]
+    dev = torch.device("cuda", torch.cuda.current_device())
+    inp = make_inputs(wl, 4000, device=dev)
+    B, Hq, d, P, mp = wl.B, wl.Hq, wl.d, wl.P, wl.max_pages
+    shape = nv.Shape(B, Hq, wl.Hkv, d, P, mp, wl.num_blocks)
+    wsd = nv.alloc_workspace(shape, nv.CALL_DECODE_DENSE, dev)
+    o_full = torch.empty((B, Hq, d), device=dev)
+    p_full = torch.zeros((B, Hq, mp * P), device=dev)
+    nv.entmaxkv_decode_dense(shape, inp["q"], inp["k_cache"], inp["v_cache"], inp["page_table"], inp["seq_lens"],
+                             wl.alpha, o_full, None, p_full, wsd)
+    s_full = torch.empty((B, Hq, d), device=dev)
+    lse_full = torch.empty((B, Hq), device=dev)
+    nv.entmaxkv_decode_dense(shape, inp["q"], inp["k_cache"], inp["v_cache"], inp["page_table"], inp["seq_lens"],
+                             1.0, s_full, lse_full, None, wsd)
+    vnorm = inp["v_cache"].float().norm(dim=-1).amax().item()  # B of the 2 B delta bound
+    tok = torch.arange(mp * P, device=dev)
+    valid = tok[None, :] < inp["seq_lens"][:, None].long()  # [B][tokens]
+    for policy in ("topk", "gauss", "gauss_est"):
+        dec = EntmaxKVDecoder(inp["k_cache"], inp["v_cache"], inp["page_table"], inp["seq_lens"], Hq,
+                              alpha=wl.alpha, policy=policy, k=wl.k or 64, delta=wl.delta or 0.5)
+        dec.build_meta()
+        dec.step(inp["q"])
+        o_sm = torch.empty((B, Hq, d), device=dev)
+        lse_sm = torch.empty((B, Hq), device=dev)
+        nv.entmaxkv_decode_sparse(shape, inp["q"], inp["k_cache"], inp["v_cache"], inp["page_table"],
+                                  inp["seq_lens"], dec.sel, dec.cnt, 1.0, o_sm, lse_sm, None, dec.ws)
+        torch.cuda.synchronize()
+        assert nv.get_status(clear=True) & ~nv.STATUS_OVERFLOW == 0
+        # kept tokens per head: the pages of its selection
+        # (entries past cnt are not written by the selection: they go to a spare column)
+        keep_p = torch.zeros((B, Hq, mp + 1), dtype=torch.bool, device=dev)
+        cnt = dec.cnt.long()
+        used = torch.arange(mp, device=dev)[None, None, :] < cnt[..., None]
+        keep_p.scatter_(2, torch.where(used, dec.sel.long().clamp(0, mp - 1), mp), True)
+        keep_t = keep_p[..., :mp].repeat_interleave(P, dim=2) & valid[:, None, :]
+        delta = (p_full * (~keep_t)).sum(-1)
+        supp = p_full > 0
+        recall = (supp & keep_t).sum(-1).float() / supp.sum(-1).clamp(min=1).float()
+        rel_e = (dec.out - o_full).norm(dim=-1) / o_full.norm(dim=-1).clamp(min=1e-30)
+        bound = (dec.out - o_full).norm(dim=-1) / (2 * vnorm * delta).clamp(min=1e-30)
+        d_sm = 1 - torch.exp(lse_sm - lse_full)
+        rel_s = (o_sm - s_full).norm(dim=-1) / s_full.norm(dim=-1).clamp(min=1e-30)
+        f = lambda t: [float(f"{float(x):.4e}") for x in (t.mean(), t.min(), t.max())]
+        print(json.dumps({"study": "quality", "workload": wl.name, "policy": policy,
+                          "k": (wl.k or 64) if policy == "topk" else None,
+                          "delta_margin": None if policy == "topk" else (wl.delta or 0.5),
+                          "kept_pages_mean": round(float(dec.cnt.float().mean()), 1), "pages": mp,
+                          "stats": "[mean, min, max] over (sequence, head)",
+                          "entmax": {"alpha": wl.alpha, "discarded_mass": f(delta), "support_recall": f(recall),
+                                     "rel_err": f(rel_e),
+                                     "err_over_2B_delta": f(bound[delta > 0]) if bool((delta > 0).any()) else None},
+                          "softmax": {"discarded_mass": f(d_sm), "rel_err": f(rel_s)}}), flush=True)
+        del dec
+
+
 def config_of(wl):
     return {"workload": wl.name, "B": wl.B, "Hq": wl.Hq, "Hkv": wl.Hkv, "d": wl.d, "L": wl.L,
             "page_size": wl.P, "alpha": wl.alpha, "policy": wl.policy, "k": wl.k, "delta": wl.delta,
@@ -530,6 +599,8 @@ def main():
     ap.add_argument("--dense-steps", type=int, default=5)
     ap.add_argument("--skip-dense", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--quality", action="store_true",
+                    help="instead of the benchmark line: sparse vs full-cache error, entmax vs softmax at one kept set")
     ap.add_argument("--l-sweep", action="store_true",
                     help="instead of the benchmark line: selection scaling with context length (one line per L, policy)")
     args = ap.parse_args()
@@ -545,6 +616,9 @@ def main():
     torch.cuda.set_device(local)
     if args.l_sweep:
         run_l_sweep(args)
+        return
+    if args.quality:
+        run_quality(args)
         return
     if world > 1:
         import datetime

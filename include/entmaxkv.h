@@ -227,11 +227,14 @@ ENTMAXKV_API int entmaxkv_select(const entmaxkv_shape *shape, const int32_t *seq
  * If T contains the full-cache support, out equals the full-cache result.
  * Each page selected by any head of a GQA group is read once for the whole
  * group; value rows whose weight is zero for every head of the group are not
- * read.  alpha > 1.  tau_out (nullable) fp32 [B][Hq].  p_out (nullable, for
- * checking) fp32 [B][Hq][max_pages*P] in logical token order: for every
- * selected page, p of its valid tokens is written (0 off the support); other
- * entries are left untouched.  A head with no selected page gets out = 0 and
- * tau = NaN.
+ * read.  tau_out (nullable) fp32 [B][Hq].  p_out (nullable, for checking)
+ * fp32 [B][Hq][max_pages*P] in logical token order: for every selected page,
+ * p of its valid tokens is written (0 off the support); other entries are
+ * left untouched.  A head with no selected page gets out = 0 and tau = NaN.
+ * alpha == 1 gives softmax over the same tokens T (for comparing entmax and
+ * softmax at one kept set): out = sum_T softmax(s)_t v_t, every selected
+ * token carries weight, so K and V of the group's selected pages are read;
+ * tau_out receives log sum_T exp(s_t); p_out must be NULL.
  */
 ENTMAXKV_API int entmaxkv_decode_sparse(const entmaxkv_shape *shape, const void *q,
                            const void *k_cache, const void *v_cache,
@@ -274,7 +277,8 @@ ENTMAXKV_API int entmaxkv_decode_sparse_static(const entmaxkv_shape *shape, cons
  *  alpha > 1:  full-cache alpha-entmax (all of K and all of V are read):
  *              out = sum_t p_t v_t; tau_out (nullable) gets tau.
  *  alpha == 1: full-cache softmax, split over pages with a combine step:
- *              out = sum_t softmax(s)_t v_t; tau_out (nullable) gets max_t s_t.
+ *              out = sum_t softmax(s)_t v_t; tau_out (nullable) gets the
+ *              log-sum-exp log sum_t exp(s_t).
  * out fp32 [B][Hq][d].  p_out as in entmaxkv_decode_sparse (alpha > 1 only;
  * must be NULL for alpha == 1).
  */

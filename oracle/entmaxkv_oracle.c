@@ -425,7 +425,7 @@ double orc_entmax_tau(const double *z, int n, double alpha)
  *               p_t = [z_t - tau]_+^{1/(alpha-1)}
  *   alpha == 1: p_t = exp(s_t - max s) / sum exp(s - max s)   (softmax)
  *   o = sum_t p_t v_t                         (fp64)
- * Outputs: o [B][Hq][d], tau [B][Hq] (max s for softmax), and optionally
+ * Outputs: o [B][Hq][d], tau [B][Hq] (log sum exp(s) for softmax), and optionally
  * p_out [B][Hq][max_pages*P] in logical token order (only tokens of T written)
  * and z_out with the same layout (z for entmax, s for softmax).
  */
@@ -484,7 +484,7 @@ void orc_decode(int B, int Hq, int Hkv, int d, int P, int max_pages,
                 for (int i = 0; i < n; ++i) if (zs[i] > m) m = zs[i];
                 for (int i = 0; i < n; ++i) { pw[i] = exp(zs[i] - m); den += pw[i]; }
                 for (int i = 0; i < n; ++i) pw[i] /= den;
-                tau = m;
+                tau = m + log(den);  /* softmax: log-sum-exp of the scores */
             }
             for (int i = 0; i < n; ++i) {
                 if (pw[i] == 0.0) continue;

@@ -330,7 +330,8 @@ int entmaxkv_decode_sparse(const entmaxkv_shape *s, const void *q, const void *k
                            const int32_t *cnt, float alpha, float *out, float *tau_out, float *p_out,
                            void *workspace, size_t ws_bytes, void *stream) {
     if (!sel || !cnt) return ENTMAXKV_ERR_NULL;
-    if (!(alpha > 1.f)) return ENTMAXKV_ERR_ALPHA;
+    if (!(alpha >= 1.f)) return ENTMAXKV_ERR_ALPHA;
+    if (alpha == 1.f && p_out) return ENTMAXKV_ERR_NULL;
     if (s && s->max_pages > MAX_SEL_PAGES) return ENTMAXKV_ERR_SHAPE;
     DecodeArgs a;
     int rc = fill_decode(false, s, q, k_cache, v_cache, page_table, seq_lens, alpha, out, tau_out, p_out, workspace,
@@ -339,6 +340,7 @@ int entmaxkv_decode_sparse(const entmaxkv_shape *s, const void *q, const void *k
     a.sel = sel;
     a.cnt = cnt;
     if ((rc = make_kv_map(&a.kmap, k_cache, s))) return rc;
+    if (alpha == 1.f && (rc = make_kv_map(&a.vmap, v_cache, s))) return rc;
     return cuda_rc(launch_decode_sparse(a, static_cast<cudaStream_t>(stream)));
 }
 

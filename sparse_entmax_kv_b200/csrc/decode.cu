@@ -67,6 +67,7 @@ __global__ void __cluster_dims__(UCL, 1, 1) __launch_bounds__(UTH) union_kernel(
         cnts[threadIdx.x] = c;
         if (rank == 0) a.ws.zmax[bh] = ORD_NEG_INF;
     }
+    if (rank == 0 && threadIdx.x == 0) a.ws.counters[bk] = 0;  // the softmax path's last-CTA combine
     __syncthreads();
     if (threadIdx.x == 0) {
         offs[0] = 0;
@@ -687,7 +688,7 @@ __device__ __forceinline__ void combine_last(const DecodeArgs &a, int bk, int b,
                 num += sc * __ldcg(pp + 2 + j);
             }
             a.out[(size_t)bh * D + j] = den > 0.f ? num / den : 0.f;
-            if (j == 0 && a.tau_out) a.tau_out[bh] = M;
+            if (j == 0 && a.tau_out) a.tau_out[bh] = den > 0.f ? M + logf(den) : __int_as_float(0x7fc00000);
         }
     }
     if (threadIdx.x == 0) a.ws.counters[bk] = 0;
@@ -812,7 +813,7 @@ __global__ void __launch_bounds__(DEC_THREADS) pv_stream_kernel(const __grid_con
 
 // ----------------------------------------------------- softmax split-K
 
-template <int D, int G>
+template <int D, int G, bool SPARSE>
 __global__ void __launch_bounds__(DEC_THREADS) softmax_kernel(const __grid_constant__ DecodeArgs a) {
     pdl_wait();
     constexpr int NS = 3;
@@ -833,7 +834,8 @@ __global__ void __launch_bounds__(DEC_THREADS) softmax_kernel(const __grid_const
     const int P = a.P, PPS = TPS / P;
     const int seq = a.seq_lens[b];
     const int np = n_pages_of(seq, P);
-    const int nsteps = ceil_div(np, PPS);
+    const int U = SPARSE ? a.ws.union_cnt[bk] : np;  // pages to read: the group's union, or all
+    const int nsteps = ceil_div(U, PPS);
     const int S = gridDim.x;
     const int my_n = nsteps > (int)blockIdx.x ? ceil_div(nsteps - blockIdx.x, S) : 0;
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -861,7 +863,7 @@ __global__ void __launch_bounds__(DEC_THREADS) softmax_kernel(const __grid_const
     }
 
     if (warp == NWC) {
-        produce<D, 2>(a, &a.kmap, &a.vmap, true, b, kvh, bk, np, my_n, PPS, NS, RG::STAGE, HALF, R.stages, R.full,
+        produce<D, 2>(a, &a.kmap, &a.vmap, !SPARSE, b, kvh, bk, U, my_n, PPS, NS, RG::STAGE, HALF, R.stages, R.full,
                       R.empty, R.pinfo, R.stash);
     } else {
         unsigned qb[G >= 2 ? D / 16 : 1][2];
@@ -905,7 +907,9 @@ __global__ void __launch_bounds__(DEC_THREADS) softmax_kernel(const __grid_const
                     for (int v = 0; v < 4; ++v) {
                         const int hh = 2 * (lane & 3) + (v & 1);
                         const int t = r0 + (lane >> 2) + (v >= 2 ? 8 : 0);
-                        if (hh < G) sc[tok0 - r0 + t][hh] = (t < pi.nval) ? c4[v] * sscale : -INFINITY;
+                        // a head scores only the pages it selected (the mask is all ones when dense)
+                        if (hh < G)
+                            sc[tok0 - r0 + t][hh] = (t < pi.nval && ((pi.mask >> hh) & 1)) ? c4[v] * sscale : -INFINITY;
                     }
                 }
             } else {
@@ -913,7 +917,7 @@ __global__ void __launch_bounds__(DEC_THREADS) softmax_kernel(const __grid_const
                 const int pi_i = tk / P, r = tk % P;
                 const PageInfo pi = pis[pi_i];
                 float s = -INFINITY;
-                if (r < pi.nval) {
+                if (r < pi.nval && (pi.mask & 1)) {
                     const unsigned char *pbase = stage + (size_t)pi_i * P * D * 2;
                     float accd = 0.f;
 #pragma unroll
@@ -972,7 +976,8 @@ __global__ void __launch_bounds__(DEC_THREADS) softmax_kernel(const __grid_const
                 }
 #pragma unroll
                 for (int g = 0; g < G; ++g) {
-                    const float p = expf(sc[t][g] - m[g]);
+                    const float sv = sc[t][g];  // -inf: a padded token or a page this head did not select
+                    const float p = sv > -INFINITY ? expf(sv - m[g]) : 0.f;
                     l[g] += p;
 #pragma unroll
                     for (int c = 0; c < CPL; ++c) acc[g][c] = fmaf(p, vv[c], acc[g][c]);
@@ -1047,6 +1052,14 @@ cudaError_t sparse_t(const DecodeArgs &a, cudaStream_t st) {
     const size_t ub = (size_t)ceil_div(ceil_div(a.max_pages, UCL), 4) * 4;
     if ((e = set_smem(union_kernel, ub)) != cudaSuccess) return e;
     if ((e = launch_pdl(union_kernel, dim3(groups * UCL), dim3(UTH), ub, st, a)) != cudaSuccess) return e;
+    if (a.alpha == 1.f) {
+        // softmax over the selected pages: K and V of the union, split over pages
+        using RG = Ring<D, G, 3, 2>;
+        auto k = softmax_kernel<D, G, true>;
+        if ((e = set_smem(k, RG::BYTES)) != cudaSuccess) return e;
+        const int S = pick_splits(a.sms, 2, groups, ceil_div(a.max_pages, RG::TPS / a.P), MAX_SPLITS);
+        return launch_pdl(k, dim3(S, groups), dim3(DEC_THREADS), RG::BYTES, st, a);
+    }
     if ((e = launch_qk<D, G, false>(a, st)) != cudaSuccess) return e;
     if ((e = set_smem(tau_pv_kernel<D, true>, TAU_SMEM)) != cudaSuccess) return e;
     return launch_pdl(tau_pv_kernel<D, true>, dim3(a.B * a.Hq), dim3(TAU_THREADS), TAU_SMEM, st, a, 0);
@@ -1075,7 +1088,7 @@ cudaError_t dense_softmax_t(const DecodeArgs &a, cudaStream_t st) {
     const int n = a.B * a.Hq > groups ? a.B * a.Hq : groups;
     if ((e = launch_pdl(dense_init_kernel, dim3(ceil_div(n, 256)), dim3(256), 0, st, a)) != cudaSuccess) return e;
     using RG = Ring<D, G, 3, 2>;
-    auto k = softmax_kernel<D, G>;
+    auto k = softmax_kernel<D, G, false>;
     if ((e = set_smem(k, RG::BYTES)) != cudaSuccess) return e;
     const int S = pick_splits(a.sms, 2, groups, ceil_div(a.max_pages, RG::TPS / a.P), MAX_SPLITS);
     return launch_pdl(k, dim3(S, groups), dim3(DEC_THREADS), RG::BYTES, st, a);
@@ -1125,7 +1138,7 @@ size_t decode_ws_bytes(bool dense, int B, int Hq, int Hkv, int d, int P, int max
     const size_t o_zmax = take((size_t)B * Hq * 4);
     const size_t o_tau = take((size_t)B * Hq * 4);
     const size_t o_cnt = take((size_t)B * Hkv * 4);
-    const size_t o_part = take(dense ? (size_t)MAX_SPLITS * B * Hq * (d + 2) * 4 : 0);
+    const size_t o_part = take((size_t)MAX_SPLITS * B * Hq * (d + 2) * 4);  // split-K softmax partials
     const size_t o_z = take(tokens * 4);
     const size_t o_t = take(tokens / 16 * 4);
     if (carve && base) {

@@ -50,7 +50,9 @@ def test_sizes():
     assert nv.workspace_size(s, nv.CALL_SELECT) == 0
     ws = nv.workspace_size(s, nv.CALL_DECODE_SPARSE)
     assert ws >= 2 * 8 * 64 * 32 * 4            # z of every token of the page list
-    assert nv.workspace_size(s, nv.CALL_DECODE_DENSE) > ws
+    part = 64 * 2 * 8 * (128 + 2) * 4           # split-K softmax partials (both paths)
+    assert ws >= 2 * 8 * 64 * 32 * 4 + part
+    assert nv.workspace_size(s, nv.CALL_DECODE_DENSE) >= 2 * 8 * 64 * 32 * 4 + part
     assert nv.workspace_size(s, 99) == (1 << 64) - 1
     assert nv.meta_bytes(shp(d=96)) == 0
 
@@ -96,10 +98,11 @@ def test_null_alignment_and_argument_codes():
                              None, None, 0, None) == -2
     # decode
     need = nv.workspace_size(shp(), nv.CALL_DECODE_SPARSE)
-    dec = lambda a, ws, wsb, q=FAKE, sl=FAKE: L.entmaxkv_decode_sparse(
-        s, q, FAKE, FAKE, FAKE, FAKE, sl, FAKE, a, FAKE, None, None, ws, wsb, None)
-    assert dec(1.0, FAKE, need) == -3
+    dec = lambda a, ws, wsb, q=FAKE, sl=FAKE, p=None: L.entmaxkv_decode_sparse(
+        s, q, FAKE, FAKE, FAKE, FAKE, sl, FAKE, a, FAKE, None, p, ws, wsb, None)
     assert dec(0.5, FAKE, need) == -3
+    assert dec(float("nan"), FAKE, need) == -3
+    assert dec(1.0, FAKE, need, p=FAKE) == -1    # softmax over the kept pages: no p_out
     assert dec(1.5, FAKE, need, sl=None) == -1
     assert dec(1.5, FAKE, need - 1) == -5
     assert dec(1.5, None, need) == -5

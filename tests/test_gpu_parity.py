@@ -273,6 +273,31 @@ def test_decode_sparse_parity(name):
     assert torch.equal(out, out2)
 
 
+@pytest.mark.parametrize("name", list(SMALL))
+def test_decode_sparse_softmax_parity(name):
+    """alpha = 1 on the sparse call: softmax over the tokens of the selected
+    pages, and the log-sum-exp of their scores."""
+    wl = SMALL[name]
+    inp, host = gpu_inputs(wl, 8)
+    k = wl.k if wl.k else 32
+    osel, ocnt, _ = _oracle_selection(host, wl, "topk", k, 0.5)
+    s = shape_of(wl)
+    sel, cnt = torch.from_numpy(osel).cuda(), torch.from_numpy(ocnt).cuda()
+    out = torch.empty((wl.B, wl.Hq, wl.d), device="cuda")
+    lse = torch.empty((wl.B, wl.Hq), device="cuda")
+    ws = nv.alloc_workspace(s, nv.CALL_DECODE_SPARSE, "cuda")
+    nv.entmaxkv_decode_sparse(s, inp["q"], inp["k_cache"], inp["v_cache"], inp["page_table"], inp["seq_lens"],
+                              sel, cnt, 1.0, out, lse, None, ws)
+    o, olse, _, _ = orc.decode(host["q"], host["K"], host["V"], host["page_table"], host["seq_lens"], wl.Hkv,
+                               wl.P, 1.0, sel=osel, cnt=ocnt)
+    assert_outputs_close(out.cpu().numpy(), o, f"{name} softmax")
+    np.testing.assert_allclose(lse.cpu().numpy(), olse, atol=2e-5 * max(1.0, np.abs(olse).max()))
+    out2 = torch.empty_like(out)
+    nv.entmaxkv_decode_sparse(s, inp["q"], inp["k_cache"], inp["v_cache"], inp["page_table"], inp["seq_lens"],
+                              sel, cnt, 1.0, out2, None, None, ws)
+    assert torch.equal(out, out2)
+
+
 @pytest.mark.parametrize("name", ["tiny_ragged", "dense_small", "mha_small", "gqa2_d64", "gqa8_d128"])
 @pytest.mark.parametrize("alpha", [1.0, 1.5, 2.0, 1.25])
 def test_decode_dense_parity(name, alpha):
