@@ -186,6 +186,13 @@ __device__ __forceinline__ void ldsm_x4(unsigned addr, unsigned &r0, unsigned &r
                  : "r"(addr));
 }
 
+// The same with each 8x8 matrix transposed on the way into registers.
+__device__ __forceinline__ void ldsm_x4_t(unsigned addr, unsigned &r0, unsigned &r1, unsigned &r2, unsigned &r3) {
+    asm volatile("ldmatrix.sync.aligned.m8n8.x4.trans.shared.b16 {%0, %1, %2, %3}, [%4];"
+                 : "=r"(r0), "=r"(r1), "=r"(r2), "=r"(r3)
+                 : "r"(addr));
+}
+
 // D = A(16x16 bf16, row) * B(16x8 bf16, col) + C, fp32 accumulate.
 __device__ __forceinline__ void mma_bf16_16816(float (&c)[4], unsigned a0, unsigned a1, unsigned a2, unsigned a3,
                                                unsigned b0, unsigned b1) {
@@ -201,6 +208,12 @@ __device__ __forceinline__ void mma_bf16_16816(float (&c)[4], unsigned a0, unsig
 __device__ __forceinline__ float bf16lo(unsigned w) { return __uint_as_float(w << 16); }
 __device__ __forceinline__ float bf16hi(unsigned w) { return __uint_as_float(w & 0xffff0000u); }
 __device__ __forceinline__ float bf16f(uint16_t h) { return __uint_as_float(((unsigned)h) << 16); }
+// float -> bf16, round to nearest even.
+__device__ __forceinline__ uint16_t f2bf(float x) {
+    uint16_t r;
+    asm("cvt.rn.bf16.f32 %0, %1;" : "=h"(r) : "f"(x));
+    return r;
+}
 
 // Order-preserving map float -> int32 (for atomicMax) and back.
 __device__ __forceinline__ int f2ord(float f) {

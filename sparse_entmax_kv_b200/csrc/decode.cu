@@ -147,11 +147,14 @@ __global__ void dense_init_kernel(DecodeArgs a) {
 // group's page list), resolve the pages 32 steps at a time with all lanes,
 // then lane 0 waits for each stage to be free, publishes the step's pages and
 // issues the box loads (map m0, and m1 into the second half when NMAP == 2).
+// With ZG > 0 it also copies the z rows of the step's pages for the ZG heads
+// of the group into zst ([stage][head][token], TPS tokens a row).
 // Returns early (all lanes) if a wait ran out.
-template <int D, int NMAP>
+template <int D, int NMAP, int ZG = 0>
 __device__ void produce(const DecodeArgs &a, const CUtensorMap *m0, const CUtensorMap *m1, bool dense, int b,
                         int kvh, int bk, int U, int my_n, int PPS, int NS, int stage_bytes, int stage_half,
-                        unsigned char *stages, uint64_t *full, uint64_t *empty, PageInfo *pinfo, PageInfo *stash) {
+                        unsigned char *stages, uint64_t *full, uint64_t *empty, PageInfo *pinfo, PageInfo *stash,
+                        float *zst = nullptr, int TPS = 0) {
     const int lane = threadIdx.x & 31;
     const int seq = a.seq_lens[b];
     const int S = gridDim.x;
@@ -195,6 +198,7 @@ __device__ void produce(const DecodeArgs &a, const CUtensorMap *m0, const CUtens
                     const PageInfo r = stash[j * PPS + i];
                     pinfo[st * PPS_MAX + i] = r;
                     if (r.blk >= 0) bytes += (unsigned)(a.P * D * 2 * NMAP);
+                    if (ZG > 0 && r.page >= 0) bytes += (unsigned)(ZG * a.P * 4);
                 }
                 mbar_arrive_expect_tx(&full[st], bytes);
                 unsigned char *stage = stages + (size_t)st * stage_bytes;
@@ -209,6 +213,15 @@ __device__ void produce(const DecodeArgs &a, const CUtensorMap *m0, const CUtens
                         if (NMAP == 2) tma_load_2d(dst + stage_half + box * a.P * 128, m1, box * 64, y, &full[st]);
                     }
                 }
+                if (ZG > 0)
+                    for (int i = 0; i < PPS; ++i) {
+                        const PageInfo r = stash[j * PPS + i];
+                        if (r.page < 0) continue;
+#pragma unroll
+                        for (int g = 0; g < ZG; ++g)
+                            bulk_g2s(zst + (size_t)(st * ZG + g) * TPS + i * a.P,
+                                     a.ws.zbuf + tok_row(a, b, kvh * ZG + g) + (size_t)r.upos * a.P, a.P * 4, &full[st]);
+                    }
             }
         }
         ok = __shfl_sync(FULL, ok, 0);
@@ -696,15 +709,27 @@ __device__ __forceinline__ void combine_last(const DecodeArgs &a, int bk, int b,
 
 // ------------------------------------------------- p.V, full-cache stream
 
+// Every V tile of the cache passes through a TMA ring; the producer also
+// copies the tiles' z rows for the G heads, so p = [z - tau]_+^r is formed in
+// registers straight in the B-operand layout (lane: head lane / 4, tokens
+// 2 (lane % 4) + {0, 1, 8, 9}).  A warp takes whole 16-token steps and skips
+// the MMAs of a step whose p are all zero (most of them: entmax is sparse).
+constexpr int PVS_NS = 3;
+
+template <int D, int G>
+constexpr size_t pvs_smem() {
+    return ((Ring<D, G, PVS_NS, 1>::BYTES + 127) & ~(size_t)127) + (size_t)PVS_NS * G * Tile<G>::TPS * 4;
+}
+
 template <int D, int G>
 __global__ void __launch_bounds__(DEC_THREADS) pv_stream_kernel(const __grid_constant__ DecodeArgs a) {
     pdl_wait();
-    constexpr int NS = 4;
+    constexpr int NS = PVS_NS;
     using RG = Ring<D, G, NS, 1>;
     constexpr int TPS = RG::TPS;
-    constexpr int CPL = D / 32;
     extern __shared__ unsigned char smem_raw[];
     RingView<D, G, NS, 1> R(smem_raw);
+    float *zst = reinterpret_cast<float *>(smem_raw + ((RG::BYTES + 127) & ~(size_t)127));
     __shared__ float red[NWC][G][D];
 
     const int bk = blockIdx.y;
@@ -726,78 +751,60 @@ __global__ void __launch_bounds__(DEC_THREADS) pv_stream_kernel(const __grid_con
     }
     __syncthreads();
 
-    float acc[G][CPL];
-#pragma unroll
-    for (int g = 0; g < G; ++g)
-#pragma unroll
-        for (int c = 0; c < CPL; ++c) acc[g][c] = 0.f;
-
     if (warp == NWC) {
-        produce<D, 1>(a, &a.vmap, &a.vmap, true, b, kvh, bk, np, my_n, PPS, NS, RG::STAGE, 0, R.stages, R.full,
-                      R.empty, R.pinfo, R.stash);
+        produce<D, 1, G>(a, &a.vmap, &a.vmap, true, b, kvh, bk, np, my_n, PPS, NS, RG::STAGE, 0, R.stages, R.full,
+                         R.empty, R.pinfo, R.stash, zst, TPS);
     } else {
         const float r = 1.f / (a.alpha - 1.f);
         const int ri = a.r_int;
-        float tau[G];
+        const int n = lane >> 2, kp = 2 * (lane & 3);  // B operand: head n, tokens kp, kp+1, kp+8, kp+9
+        const float tau = n < G ? a.ws.tau[b * a.Hq + kvh * G + n] : __int_as_float(0x7fc00000);
+        float acc[D / 16][4];
 #pragma unroll
-        for (int g = 0; g < G; ++g) tau[g] = a.ws.tau[b * a.Hq + kvh * G + g];
+        for (int mt = 0; mt < D / 16; ++mt) acc[mt][0] = acc[mt][1] = acc[mt][2] = acc[mt][3] = 0.f;
         for (int it = 0; it < my_n; ++it) {
             const int st = it % NS, ph = (it / NS) & 1;
             if (!mbar_wait(&R.full[st], ph, a.status)) break;
             const unsigned char *stage = R.stages + (size_t)st * RG::STAGE;
             const PageInfo *pis = R.pinfo + st * PPS_MAX;
-            for (int bt = warp; bt < TPS / 32; bt += NWC) {
-                const int tk = bt * 32 + lane;
-                const int pi_i = tk / P, rr = tk % P;
+            for (int kt = warp; kt < TPS / 16; kt += NWC) {
+                const int tok0 = kt * 16, pi_i = tok0 / P, r0 = tok0 % P;
                 const PageInfo pi = pis[pi_i];
-                float p[G];
-                bool any = false;
+                if (pi.nval <= r0) continue;  // no page, or no valid token in this step
+                float p[4] = {0.f, 0.f, 0.f, 0.f};
+                if (n < G) {
+                    const float *zr = zst + (size_t)(st * G + n) * TPS + tok0 + kp;
+                    const float2 za = *reinterpret_cast<const float2 *>(zr);
+                    const float2 zb = *reinterpret_cast<const float2 *>(zr + 8);
+                    p[0] = pos_pow(za.x - tau, r, ri);
+                    p[1] = pos_pow(za.y - tau, r, ri);
+                    p[2] = pos_pow(zb.x - tau, r, ri);
+                    p[3] = pos_pow(zb.y - tau, r, ri);
+                    if (a.p_out) {
+                        float *po = a.p_out + tok_row(a, b, kvh * G + n) + (size_t)pi.page * P + r0 + kp;
 #pragma unroll
-                for (int g = 0; g < G; ++g) {
-                    p[g] = 0.f;
-                    if (pi.page >= 0 && rr < pi.nval) {
-                        const float z = __ldcg(a.ws.zbuf + tok_row(a, b, kvh * G + g) + (size_t)pi.page * P + rr);
-                        p[g] = pos_pow(z - tau[g], r, ri);
-                        if (a.p_out) a.p_out[tok_row(a, b, kvh * G + g) + (size_t)pi.page * P + rr] = p[g];
-                    }
-                    any |= p[g] > 0.f;
-                }
-                unsigned bal = __ballot_sync(FULL, any);
-                while (bal) {
-                    const int tt = __ffs(bal) - 1;
-                    bal &= bal - 1;
-                    const int tk2 = bt * 32 + tt;
-                    const int pj = tk2 / P, r2 = tk2 % P;
-                    const unsigned char *pbase = stage + (size_t)pj * P * D * 2;
-                    float vv[CPL];
-                    if (CPL == 4) {
-                        const uint2 w =
-                            *reinterpret_cast<const uint2 *>(tile_chunk(pbase, P, r2, lane >> 1) + (lane & 1) * 8);
-                        vv[0] = bf16lo(w.x);
-                        vv[1] = bf16hi(w.x);
-                        vv[2] = bf16lo(w.y);
-                        vv[3] = bf16hi(w.y);
-                    } else {
-                        const unsigned w =
-                            *reinterpret_cast<const unsigned *>(tile_chunk(pbase, P, r2, lane >> 2) + (lane & 3) * 4);
-                        vv[0] = bf16lo(w);
-                        vv[1] = bf16hi(w);
-                    }
-#pragma unroll
-                    for (int g = 0; g < G; ++g) {
-                        const float pg = __shfl_sync(FULL, p[g], tt);
-#pragma unroll
-                        for (int c = 0; c < CPL; ++c) acc[g][c] = fmaf(pg, vv[c], acc[g][c]);
+                        for (int v = 0; v < 4; ++v)
+                            if (r0 + kp + (v & 1) + 8 * (v >> 1) < pi.nval) po[(v & 1) + 8 * (v >> 1)] = p[v];
                     }
                 }
+                if (!__any_sync(FULL, p[0] > 0.f || p[1] > 0.f || p[2] > 0.f || p[3] > 0.f)) continue;
+                unsigned bh0, bh1, bl0, bl1;
+                split_pair(p[0], p[1], bh0, bl0);
+                split_pair(p[2], p[3], bh1, bl1);
+                pv_mma<D>(acc, stage + (size_t)pi_i * P * D * 2, P, r0, pi.nval, bh0, bh1, bl0, bl1);
             }
             __syncwarp();
             if (lane == 0) mbar_arrive(&R.empty[st]);
         }
+        // acc[mt][v]: coordinate 16 mt + lane/4 + 8 (v >> 1), head 2 (lane % 4) + (v & 1)
+        const int h0 = 2 * (lane & 3);
 #pragma unroll
-        for (int g = 0; g < G; ++g)
+        for (int mt = 0; mt < D / 16; ++mt)
 #pragma unroll
-            for (int c = 0; c < CPL; ++c) red[warp][g][lane * CPL + c] = acc[g][c];
+            for (int v = 0; v < 4; ++v) {
+                const int hh = h0 + (v & 1);
+                if (hh < G) red[warp][hh][16 * mt + (lane >> 2) + 8 * (v >> 1)] = acc[mt][v];
+            }
     }
     __syncthreads();
     const int BH = a.B * a.Hq;
@@ -813,21 +820,24 @@ __global__ void __launch_bounds__(DEC_THREADS) pv_stream_kernel(const __grid_con
 
 // ----------------------------------------------------- softmax split-K
 
+// K and V tiles of each step through one TMA ring.  A warp owns whole
+// 16-token steps: scores on the tensor cores (tokens as M, the group's heads
+// as N), its own running max and sum per head (the lane's two heads), p
+// through a small per-warp scratch into the B-operand layout, then P.V on the
+// tensor cores.  The warps' states are merged at the end of the CTA, and the
+// CTAs' in a fixed order by the last one of the group.
 template <int D, int G, bool SPARSE>
 __global__ void __launch_bounds__(DEC_THREADS) softmax_kernel(const __grid_constant__ DecodeArgs a) {
     pdl_wait();
     constexpr int NS = 3;
     using RG = Ring<D, G, NS, 2>;
     constexpr int TPS = RG::TPS;
-    constexpr int CPL = D / 32;
     constexpr int HALF = RG::STAGE / 2;
     extern __shared__ unsigned char smem_raw[];
     RingView<D, G, NS, 2> R(smem_raw);
-    __shared__ float st_s[2][TPS][G];  // scores of the stage, double-buffered
-    __shared__ float qs[G == 1 ? D : 1];
+    __shared__ __align__(16) uint16_t pw[NWC][2][8][16];  // per warp: p as [hi/lo][head][token]
     __shared__ float red[NWC][G][D];
-    __shared__ float redl[NWC][G];
-    __shared__ int s_abort;
+    __shared__ float redm[NWC][G], redl[NWC][G];
 
     const int bk = blockIdx.y;
     const int b = bk / a.Hkv, kvh = bk % a.Hkv;
@@ -847,28 +857,17 @@ __global__ void __launch_bounds__(DEC_THREADS) softmax_kernel(const __grid_const
             mbar_init(&R.empty[s], NWC);
         }
         mbar_fence_init();
-        s_abort = 0;
     }
-    if (G == 1)
-        for (int j = threadIdx.x; j < D; j += blockDim.x) qs[j] = bf16f(a.q[((size_t)b * a.Hq + kvh) * D + j]);
     __syncthreads();
-
-    float m[G], l[G], acc[G][CPL];
-#pragma unroll
-    for (int g = 0; g < G; ++g) {
-        m[g] = -INFINITY;
-        l[g] = 0.f;
-#pragma unroll
-        for (int c = 0; c < CPL; ++c) acc[g][c] = 0.f;
-    }
 
     if (warp == NWC) {
         produce<D, 2>(a, &a.kmap, &a.vmap, !SPARSE, b, kvh, bk, U, my_n, PPS, NS, RG::STAGE, HALF, R.stages, R.full,
                       R.empty, R.pinfo, R.stash);
     } else {
-        unsigned qb[G >= 2 ? D / 16 : 1][2];
-        if constexpr (G >= 2) {
-            const int n = lane >> 2, kp = 2 * (lane & 3);
+        // B fragments of q: head n = lane/4 (zero for n >= G), coordinate pair 2 (lane % 4)
+        unsigned qb[D / 16][2];
+        const int n = lane >> 2, kp = 2 * (lane & 3);
+        {
             const uint16_t *qh = a.q + ((size_t)b * a.Hq + kvh * G + (n < G ? n : 0)) * D;
 #pragma unroll
             for (int ks = 0; ks < D / 16; ++ks) {
@@ -876,144 +875,134 @@ __global__ void __launch_bounds__(DEC_THREADS) softmax_kernel(const __grid_const
                 qb[ks][1] = n < G ? *reinterpret_cast<const unsigned *>(qh + 16 * ks + kp + 8) : 0u;
             }
         }
+        const int h0 = kp;  // this lane's heads in the score and output fragments: h0, h0 + 1
+        float m0 = -INFINITY, m1 = -INFINITY, l0 = 0.f, l1 = 0.f;
+        float acc[D / 16][4];
+#pragma unroll
+        for (int mt = 0; mt < D / 16; ++mt) acc[mt][0] = acc[mt][1] = acc[mt][2] = acc[mt][3] = 0.f;
+        uint16_t(*pwh)[16] = pw[warp][0];
+        uint16_t(*pwl)[16] = pw[warp][1];
         for (int it = 0; it < my_n; ++it) {
             const int st = it % NS, ph = (it / NS) & 1;
-            // a warp whose wait ran out still takes part in the named barrier
-            // below; all consumer warps then leave together
-            const bool ready = mbar_wait(&R.full[st], ph, a.status);
-            if (!ready) s_abort = 1;
+            if (!mbar_wait(&R.full[st], ph, a.status)) break;
             const unsigned char *stage = R.stages + (size_t)st * RG::STAGE;
             const PageInfo *pis = R.pinfo + st * PPS_MAX;
-            float(*sc)[G] = st_s[it & 1];
-            // scores of the stage's tokens
-            if (!ready) {
-            } else if constexpr (G >= 2) {
-                for (int mt = warp; mt < TPS / 16; mt += NWC) {
-                    const int tok0 = mt * 16, pi_i = tok0 / P, r0 = tok0 % P;
-                    const PageInfo pi = pis[pi_i];
-                    float c4[4] = {0.f, 0.f, 0.f, 0.f};
-                    if (pi.nval > 0) {
-                        const unsigned char *pbase = stage + (size_t)pi_i * P * D * 2;
-                        const int mat = lane >> 3, rr = lane & 7;
-                        const int row = r0 + (mat & 1) * 8 + rr;
-#pragma unroll
-                        for (int ks = 0; ks < D / 16; ++ks) {
-                            unsigned a0, a1, a2, a3;
-                            ldsm_x4(smem_u32(tile_chunk(pbase, P, row, ks * 2 + (mat >> 1))), a0, a1, a2, a3);
-                            mma_bf16_16816(c4, a0, a1, a2, a3, qb[ks][0], qb[ks][1]);
-                        }
-                    }
-#pragma unroll
-                    for (int v = 0; v < 4; ++v) {
-                        const int hh = 2 * (lane & 3) + (v & 1);
-                        const int t = r0 + (lane >> 2) + (v >= 2 ? 8 : 0);
-                        // a head scores only the pages it selected (the mask is all ones when dense)
-                        if (hh < G)
-                            sc[tok0 - r0 + t][hh] = (t < pi.nval && ((pi.mask >> hh) & 1)) ? c4[v] * sscale : -INFINITY;
-                    }
-                }
-            } else {
-                const int tk = threadIdx.x;  // 128 consumer threads, TPS == 128
-                const int pi_i = tk / P, r = tk % P;
+            for (int kt = warp; kt < TPS / 16; kt += NWC) {
+                const int tok0 = kt * 16, pi_i = tok0 / P, r0 = tok0 % P;
                 const PageInfo pi = pis[pi_i];
-                float s = -INFINITY;
-                if (r < pi.nval && (pi.mask & 1)) {
-                    const unsigned char *pbase = stage + (size_t)pi_i * P * D * 2;
-                    float accd = 0.f;
+                if (pi.nval <= r0) continue;  // no page, or no valid token in this step
+                const unsigned char *kbase = stage + (size_t)pi_i * P * D * 2;
+                float c4[4] = {0.f, 0.f, 0.f, 0.f};
+                {
+                    const int mat = lane >> 3, rr = lane & 7;
+                    const int row = r0 + (mat & 1) * 8 + rr;
 #pragma unroll
-                    for (int c16 = 0; c16 < D / 8; ++c16) {
-                        const uint4 kv = *reinterpret_cast<const uint4 *>(tile_chunk(pbase, P, r, c16));
-                        const float4 q0 = *reinterpret_cast<const float4 *>(qs + 8 * c16);
-                        const float4 q1 = *reinterpret_cast<const float4 *>(qs + 8 * c16 + 4);
-                        accd = fmaf(q0.x, bf16lo(kv.x), accd);
-                        accd = fmaf(q0.y, bf16hi(kv.x), accd);
-                        accd = fmaf(q0.z, bf16lo(kv.y), accd);
-                        accd = fmaf(q0.w, bf16hi(kv.y), accd);
-                        accd = fmaf(q1.x, bf16lo(kv.z), accd);
-                        accd = fmaf(q1.y, bf16hi(kv.z), accd);
-                        accd = fmaf(q1.z, bf16lo(kv.w), accd);
-                        accd = fmaf(q1.w, bf16hi(kv.w), accd);
+                    for (int ks = 0; ks < D / 16; ++ks) {
+                        unsigned a0, a1, a2, a3;
+                        ldsm_x4(smem_u32(tile_chunk(kbase, P, row, ks * 2 + (mat >> 1))), a0, a1, a2, a3);
+                        mma_bf16_16816(c4, a0, a1, a2, a3, qb[ks][0], qb[ks][1]);
                     }
-                    s = accd * sscale;
                 }
-                sc[tk][0] = s;
-            }
-            asm volatile("bar.sync 1, %0;" ::"n"(NWC * 32) : "memory");
-            if (s_abort) break;
-            // tile max per head (every warp computes it identically)
-            float mn[G], scl[G];
+                // c4[v]: token r0 + lane/4 + 8 (v >> 1), head h0 + (v & 1); a head
+                // scores only the pages it selected (all of them when dense)
+                float sv[4];
 #pragma unroll
-            for (int g = 0; g < G; ++g) {
-                float x = -INFINITY;
-                for (int t = lane; t < TPS; t += 32) x = fmaxf(x, sc[t][g]);
-#pragma unroll
-                for (int o = 16; o; o >>= 1) x = fmaxf(x, __shfl_xor_sync(FULL, x, o));
-                mn[g] = fmaxf(m[g], x);
-                scl[g] = (mn[g] == -INFINITY) ? 1.f : expf(m[g] - mn[g]);
-                m[g] = mn[g];
-                l[g] *= scl[g];
-#pragma unroll
-                for (int c = 0; c < CPL; ++c) acc[g][c] *= scl[g];
-            }
-            for (int t = warp; t < TPS; t += NWC) {
-                const int pj = t / P, r2 = t % P;
-                const PageInfo pi = pis[pj];
-                if (r2 >= pi.nval) continue;
-                const unsigned char *vbase = stage + HALF + (size_t)pj * P * D * 2;
-                float vv[CPL];
-                if (CPL == 4) {
-                    const uint2 w =
-                        *reinterpret_cast<const uint2 *>(tile_chunk(vbase, P, r2, lane >> 1) + (lane & 1) * 8);
-                    vv[0] = bf16lo(w.x);
-                    vv[1] = bf16hi(w.x);
-                    vv[2] = bf16lo(w.y);
-                    vv[3] = bf16hi(w.y);
-                } else {
-                    const unsigned w =
-                        *reinterpret_cast<const unsigned *>(tile_chunk(vbase, P, r2, lane >> 2) + (lane & 3) * 4);
-                    vv[0] = bf16lo(w);
-                    vv[1] = bf16hi(w);
+                for (int v = 0; v < 4; ++v) {
+                    const int hh = h0 + (v & 1);
+                    const int t = r0 + (lane >> 2) + 8 * (v >> 1);
+                    sv[v] = (hh < G && t < pi.nval && ((pi.mask >> hh) & 1)) ? c4[v] * sscale : -INFINITY;
                 }
+                float x0 = fmaxf(sv[0], sv[2]), x1 = fmaxf(sv[1], sv[3]);
 #pragma unroll
-                for (int g = 0; g < G; ++g) {
-                    const float sv = sc[t][g];  // -inf: a padded token or a page this head did not select
-                    const float p = sv > -INFINITY ? expf(sv - m[g]) : 0.f;
-                    l[g] += p;
-#pragma unroll
-                    for (int c = 0; c < CPL; ++c) acc[g][c] = fmaf(p, vv[c], acc[g][c]);
+                for (int o = 4; o < 32; o <<= 1) {
+                    x0 = fmaxf(x0, __shfl_xor_sync(FULL, x0, o));
+                    x1 = fmaxf(x1, __shfl_xor_sync(FULL, x1, o));
                 }
+                const float n0 = fmaxf(m0, x0), n1 = fmaxf(m1, x1);
+                const float c0 = n0 == -INFINITY ? 1.f : expf(m0 - n0);
+                const float c1 = n1 == -INFINITY ? 1.f : expf(m1 - n1);
+                if (__any_sync(FULL, c0 != 1.f || c1 != 1.f)) {
+#pragma unroll
+                    for (int mt = 0; mt < D / 16; ++mt) {
+                        acc[mt][0] *= c0;
+                        acc[mt][2] *= c0;
+                        acc[mt][1] *= c1;
+                        acc[mt][3] *= c1;
+                    }
+                }
+                m0 = n0;
+                m1 = n1;
+                float p[4];
+#pragma unroll
+                for (int v = 0; v < 4; ++v) p[v] = sv[v] > -INFINITY ? expf(sv[v] - ((v & 1) ? n1 : n0)) : 0.f;
+                l0 = l0 * c0 + (p[0] + p[2]);
+                l1 = l1 * c1 + (p[1] + p[3]);
+                // p^T into the B-operand layout through the warp's scratch
+                __syncwarp();
+#pragma unroll
+                for (int v = 0; v < 4; ++v) {
+                    const int hh = h0 + (v & 1), t = (lane >> 2) + 8 * (v >> 1);
+                    const uint16_t hi = f2bf(p[v]);
+                    pwh[hh][t] = hi;
+                    pwl[hh][t] = f2bf(p[v] - bf16f(hi));
+                }
+                __syncwarp();
+                const unsigned bh0 = *reinterpret_cast<const unsigned *>(&pwh[n][kp]);
+                const unsigned bh1 = *reinterpret_cast<const unsigned *>(&pwh[n][kp + 8]);
+                const unsigned bl0 = *reinterpret_cast<const unsigned *>(&pwl[n][kp]);
+                const unsigned bl1 = *reinterpret_cast<const unsigned *>(&pwl[n][kp + 8]);
+                pv_mma<D>(acc, stage + HALF + (size_t)pi_i * P * D * 2, P, r0, pi.nval, bh0, bh1, bl0, bl1);
             }
             __syncwarp();
             if (lane == 0) mbar_arrive(&R.empty[st]);
         }
+        // sums over the lanes that hold the same heads; then the warp's state
 #pragma unroll
-        for (int g = 0; g < G; ++g) {
-#pragma unroll
-            for (int c = 0; c < CPL; ++c) red[warp][g][lane * CPL + c] = acc[g][c];
-            if (lane == 0) redl[warp][g] = l[g];
+        for (int o = 4; o < 32; o <<= 1) {
+            l0 += __shfl_xor_sync(FULL, l0, o);
+            l1 += __shfl_xor_sync(FULL, l1, o);
         }
+        if (lane < 4) {
+            if (h0 < G) {
+                redm[warp][h0] = m0;
+                redl[warp][h0] = l0;
+            }
+            if (h0 + 1 < G) {
+                redm[warp][h0 + 1] = m1;
+                redl[warp][h0 + 1] = l1;
+            }
+        }
+#pragma unroll
+        for (int mt = 0; mt < D / 16; ++mt)
+#pragma unroll
+            for (int v = 0; v < 4; ++v) {
+                const int hh = h0 + (v & 1);
+                if (hh < G) red[warp][hh][16 * mt + (lane >> 2) + 8 * (v >> 1)] = acc[mt][v];
+            }
     }
     __syncthreads();
-    // all consumer warps share m; sum l and acc over warps
+    // the CTA's partial per head: max, sum and numerator, the warps merged in order
     const int BH = a.B * a.Hq;
     for (int i = threadIdx.x; i < G * D; i += blockDim.x) {
         const int g = i / D, j = i % D;
         const size_t o = ((size_t)blockIdx.x * BH + b * a.Hq + kvh * G + g) * (D + 2);
-        float s = 0.f;
+        float M = -INFINITY;
 #pragma unroll
-        for (int w = 0; w < NWC; ++w) s += red[w][g][j];
-        a.ws.partial[o + 2 + j] = s;
-        if (j == 0) {
-            float ls = 0.f;
+        for (int w = 0; w < NWC; ++w) M = fmaxf(M, redm[w][g]);
+        float num = 0.f, den = 0.f;
 #pragma unroll
-            for (int w = 0; w < NWC; ++w) ls += redl[w][g];
-            a.ws.partial[o + 1] = ls;
+        for (int w = 0; w < NWC; ++w) {
+            const float mw = redm[w][g];
+            if (!(mw > -INFINITY)) continue;
+            const float sc = expf(mw - M);
+            num = fmaf(sc, red[w][g][j], num);
+            den = fmaf(sc, redl[w][g], den);
         }
-    }
-    // m lives in the consumer warps' registers; thread 0 (consumer warp 0) publishes it
-    if (threadIdx.x == 0) {
-#pragma unroll
-        for (int g = 0; g < G; ++g) a.ws.partial[((size_t)blockIdx.x * BH + b * a.Hq + kvh * G + g) * (D + 2)] = m[g];
+        a.ws.partial[o + 2 + j] = num;
+        if (j == 0) {
+            a.ws.partial[o] = M;
+            a.ws.partial[o + 1] = den;
+        }
     }
     combine_last<D, G>(a, bk, b, kvh, S, true);
 }
@@ -1074,11 +1063,11 @@ cudaError_t dense_entmax_t(const DecodeArgs &a, cudaStream_t st) {
     if ((e = launch_qk<D, G, true>(a, st)) != cudaSuccess) return e;
     if ((e = set_smem(tau_pv_kernel<D, false>, TAU_SMEM)) != cudaSuccess) return e;
     if ((e = launch_pdl(tau_pv_kernel<D, false>, dim3(a.B * a.Hq), dim3(TAU_THREADS), TAU_SMEM, st, a, 1)) != cudaSuccess) return e;
-    using RG = Ring<D, G, 4, 1>;
     auto k = pv_stream_kernel<D, G>;
-    if ((e = set_smem(k, RG::BYTES)) != cudaSuccess) return e;
-    const int S = pick_splits(a.sms, 3, groups, ceil_div(a.max_pages, RG::TPS / a.P), MAX_SPLITS);
-    return launch_pdl(k, dim3(S, groups), dim3(DEC_THREADS), RG::BYTES, st, a);
+    constexpr size_t smem = pvs_smem<D, G>();
+    if ((e = set_smem(k, smem)) != cudaSuccess) return e;
+    const int S = pick_splits(a.sms, 3, groups, ceil_div(a.max_pages, Tile<G>::TPS / a.P), MAX_SPLITS);
+    return launch_pdl(k, dim3(S, groups), dim3(DEC_THREADS), smem, st, a);
 }
 
 template <int D, int G>

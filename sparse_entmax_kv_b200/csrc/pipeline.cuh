@@ -63,4 +63,46 @@ __device__ __forceinline__ const unsigned char *tile_chunk(const unsigned char *
     return page_base + box * P * 128 + r * 128 + ((cc ^ (r & 7)) << 4);
 }
 
+// P.V on the tensor cores for one 16-token step of one warp.
+//   acc[mt] (m16n8 fragment): rows = value coordinates 16 mt .. 16 mt + 15,
+//   columns = the group's heads (lane holds heads 2 (lane % 4) and + 1).
+// A = V^T of rows r0 .. r0 + 15 of a swizzled page tile, read with transposing
+// ldmatrix; B = P^T of those tokens as bf16 hi and lo parts (p = hi + lo to
+// about 2^-17 relative), two MMAs per tile.  Value halves of tokens at or past
+// nval are zeroed (those rows of the tile may hold anything, and 0 * NaN is
+// NaN).
+template <int D>
+__device__ __forceinline__ void pv_mma(float (&acc)[D / 16][4], const unsigned char *vpage, int P, int r0, int nval,
+                                       unsigned bh0, unsigned bh1, unsigned bl0, unsigned bl1) {
+    const int lane = threadIdx.x & 31;
+    const int row = r0 + ((lane >> 4) << 3) + (lane & 7);
+    const int csel = (lane >> 3) & 1;
+    unsigned m01 = 0xffffffffu, m23 = 0xffffffffu;
+    if (r0 + 16 > nval) {
+        const int t = r0 + 2 * (lane & 3);
+        m01 = (t < nval ? 0x0000ffffu : 0u) | (t + 1 < nval ? 0xffff0000u : 0u);
+        m23 = (t + 8 < nval ? 0x0000ffffu : 0u) | (t + 9 < nval ? 0xffff0000u : 0u);
+    }
+#pragma unroll
+    for (int mt = 0; mt < D / 16; ++mt) {
+        unsigned a0, a1, a2, a3;
+        ldsm_x4_t(smem_u32(tile_chunk(vpage, P, row, 2 * mt + csel)), a0, a1, a2, a3);
+        a0 &= m01;
+        a1 &= m01;
+        a2 &= m23;
+        a3 &= m23;
+        mma_bf16_16816(acc[mt], a0, a1, a2, a3, bh0, bh1);
+        mma_bf16_16816(acc[mt], a0, a1, a2, a3, bl0, bl1);
+    }
+}
+
+// p0, p1 (two consecutive tokens of one head) as the hi and lo bf16 pairs of
+// a B fragment register (first token in the low half).
+__device__ __forceinline__ void split_pair(float p0, float p1, unsigned &hi, unsigned &lo) {
+    const uint16_t h0 = f2bf(p0), h1 = f2bf(p1);
+    const uint16_t l0 = f2bf(p0 - bf16f(h0)), l1 = f2bf(p1 - bf16f(h1));
+    hi = (unsigned)h0 | ((unsigned)h1 << 16);
+    lo = (unsigned)l0 | ((unsigned)l1 << 16);
+}
+
 }  // namespace ekv
