@@ -108,6 +108,13 @@ __device__ __forceinline__ void prefetch_tmap(const CUtensorMap *map) {
 }
 
 // Ampere-style 16-byte async copy (bypasses L1), grouped with commit/wait.
+// Ask for the 128-byte lines of one row of D bf16 values to be brought into L2.
+template <int D>
+__device__ __forceinline__ void prefetch_l2_row(const uint16_t *row) {
+#pragma unroll
+    for (int o = 0; o < D * 2; o += 128) asm volatile("prefetch.global.L2 [%0];" ::"l"(reinterpret_cast<const char *>(row) + o));
+}
+
 __device__ __forceinline__ void cp_async16(void *dst, const void *src) {
     asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(smem_u32(dst)), "l"(src) : "memory");
 }

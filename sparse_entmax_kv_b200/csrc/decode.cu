@@ -397,29 +397,41 @@ __global__ void __launch_bounds__(DEC_THREADS) qk_kernel(const __grid_constant__
 
 // -------------------------------------------------------- tau and p . V
 
-constexpr int TAU_THREADS = 512;
-constexpr int TAU_WARPS = TAU_THREADS / 32;
-constexpr int ZCAP = 8192;  // candidates held on chip per head
-constexpr int TAU_TB = 8;   // tile maxima in flight per lane
-constexpr size_t TAU_SMEM = (size_t)ZCAP * 16;
+constexpr int TAU_NT = 256;  // threads per head
+constexpr int TAU_NW = TAU_NT / 32;
+constexpr int TAU_TB = 16;   // tile maxima per thread and round
+constexpr int ZCAP_MAX = 8192;
+
+// Candidate buffers for zcap candidates: z, list position and value row
+// (zcap each), and up to zcap / 2 candidate 16-token tiles.
+inline size_t tau_smem(int zcap) { return (size_t)zcap * 14; }
+
+// The largest candidate capacity (a power of two in [1024, ZCAP_MAX]) that
+// still lets the grid's CTAs share each SM in one wave.
+inline int tau_zcap(int ctas, int sms) {
+    const int per_sm = ctas > sms && sms > 0 ? ceil_div(ctas, sms) : 1;
+    const size_t budget = (size_t)(220 << 10) / per_sm - (4 << 10);
+    int z = ZCAP_MAX;
+    while (z > 1024 && tau_smem(z) > budget) z >>= 1;
+    return z;
+}
 
 // Exact threshold and (GATHER) the weighted sum of the support's value rows.
 template <int D, bool GATHER>
-__global__ void __launch_bounds__(TAU_THREADS) tau_pv_kernel(const __grid_constant__ DecodeArgs a, int dense) {
+__global__ void __launch_bounds__(TAU_NT, D == 64 ? 4 : 3) tau_pv_kernel(const __grid_constant__ DecodeArgs a, int dense, int zcap) {
     pdl_wait();
     constexpr int CPL = D / 32;
-    // candidates in list order: z, value row and list position; once the
+    // candidates in list order: z, list position and value row; once the
     // gather has read them, the same bytes hold the per-warp output partials
     extern __shared__ __align__(16) unsigned char tsm[];
     float *cz = reinterpret_cast<float *>(tsm);
-    int *crow = reinterpret_cast<int *>(tsm + ZCAP * 4);
-    int *cpos = reinterpret_cast<int *>(tsm + ZCAP * 8);
-    int *ctile = reinterpret_cast<int *>(tsm + ZCAP * 12);  // candidate 16-token tiles
+    int *cpos = reinterpret_cast<int *>(tsm + (size_t)zcap * 4);
+    int *crow = reinterpret_cast<int *>(tsm + (size_t)zcap * 8);
+    int *ctile = reinterpret_cast<int *>(tsm + (size_t)zcap * 12);  // candidate 16-token tiles
+    const int tcap = zcap / 2;
     double(*accs)[D] = reinterpret_cast<double(*)[D]>(tsm);
-    static_assert(TAU_WARPS * D * 8 <= TAU_SMEM, "partials must fit the candidate buffer");
     __shared__ int wcnt[72];  // block scan scratch
-    __shared__ float red[TAU_WARPS][33];
-    __shared__ float br[2];
+    __shared__ float red[2][TAU_NW][2];  // double-buffered pass sums
     const int bh = blockIdx.x;
     const int b = bh / a.Hq, h = bh % a.Hq;
     const int G = a.Hq / a.Hkv, kvh = h / G;
@@ -434,7 +446,7 @@ __global__ void __launch_bounds__(TAU_THREADS) tau_pv_kernel(const __grid_consta
     const int ri = a.r_int;
     if (!(zmax > -INFINITY)) {  // no token at all
         if (GATHER)
-            for (int j = threadIdx.x; j < D; j += TAU_THREADS) a.out[(size_t)bh * D + j] = 0.f;
+            for (int j = threadIdx.x; j < D; j += TAU_NT) a.out[(size_t)bh * D + j] = 0.f;
         if (threadIdx.x == 0) {
             a.ws.tau[bh] = __int_as_float(0x7fc00000);
             if (a.tau_out) a.tau_out[bh] = __int_as_float(0x7fc00000);
@@ -443,7 +455,8 @@ __global__ void __launch_bounds__(TAU_THREADS) tau_pv_kernel(const __grid_consta
     }
     const float thr = zmax - 1.f;
     const float *zr = a.ws.zbuf + tok_row(a, b, h);
-    const float *tr = a.ws.tmax + tile_row(a, b, h);
+    const size_t trow = tile_row(a, b, h);
+    const float *tr = a.ws.tmax + trow;
     auto row_of_pos = [&](int pos) -> int {
         const int up = pos / P, t = pos - up * P;
         const int blk = dense ? __ldg(a.page_table + (size_t)b * a.max_pages + up)
@@ -452,131 +465,159 @@ __global__ void __launch_bounds__(TAU_THREADS) tau_pv_kernel(const __grid_consta
     };
 
     // Candidates (z > z_max - 1) in list order, in two ordered block-wide
-    // compactions: the 16-token tiles whose max clears the bar, then their
-    // tokens (z and, for the gather, the value row are loaded together).
+    // compactions: the 16-token tiles whose max clears the bar (TAU_TB tile
+    // maxima per thread, loaded together), then their tokens (one tile per
+    // thread: its 16 z and, for the gather, its page's value row, loaded
+    // together).
     const int n_tiles = n_tok / 16;
+    const bool tvec = (trow & 3) == 0;
     int ntc = 0;
-    for (int t0 = 0; t0 < n_tiles; t0 += TAU_THREADS * TAU_TB) {
+    for (int t0 = 0; t0 < n_tiles; t0 += TAU_NT * TAU_TB) {
         const int p0 = t0 + threadIdx.x * TAU_TB;
         float v[TAU_TB];
+        if (tvec && p0 + TAU_TB <= n_tiles) {
 #pragma unroll
-        for (int i = 0; i < TAU_TB; ++i) v[i] = p0 + i < n_tiles ? __ldcg(tr + p0 + i) : -INFINITY;
+            for (int i = 0; i < TAU_TB / 4; ++i) {
+                const float4 f = __ldcg(reinterpret_cast<const float4 *>(tr + p0) + i);
+                v[4 * i] = f.x;
+                v[4 * i + 1] = f.y;
+                v[4 * i + 2] = f.z;
+                v[4 * i + 3] = f.w;
+            }
+        } else {
+#pragma unroll
+            for (int i = 0; i < TAU_TB; ++i) v[i] = p0 + i < n_tiles ? __ldcg(tr + p0 + i) : -INFINITY;
+        }
         unsigned bits = 0;
 #pragma unroll
         for (int i = 0; i < TAU_TB; ++i)
             if (v[i] > thr) bits |= 1u << i;
         int tot;
         int w = ntc + block_excl_scan(__popc(bits), wcnt, &tot);
-        while (bits) {
-            const int k = __ffs(bits) - 1;
-            bits &= bits - 1;
-            if (w < ZCAP) ctile[w] = p0 + k;
-            ++w;
-        }
+#pragma unroll
+        for (int i = 0; i < TAU_TB; ++i)
+            if ((bits >> i) & 1u) {
+                if (w < tcap) ctile[w] = p0 + i;
+                ++w;
+            }
         ntc += tot;
     }
     __syncthreads();
     int nc = 0;
-    if (ntc <= ZCAP) {
-        // the tiles' tokens, ZCAP at a time, TPT consecutive ones per thread
-        constexpr int TPT = ZCAP / TAU_THREADS;
-        for (int e0 = 0; e0 < ntc * 16 && nc <= ZCAP; e0 += ZCAP) {
-            float zz[TPT];
-            int pp[TPT], rr[TPT];
+    if (ntc <= tcap) {
+        for (int r0 = 0; r0 < ntc && nc <= zcap; r0 += TAU_NT) {
+            const int i = r0 + threadIdx.x;
+            float zz[16];
+            int pos0 = 0, row0 = 0;
             unsigned bits = 0;
+            if (i < ntc) {
+                pos0 = ctile[i] * 16;
+                const float4 *zp = reinterpret_cast<const float4 *>(zr + pos0);
 #pragma unroll
-            for (int i = 0; i < TPT; ++i) {
-                const int e = e0 + threadIdx.x * TPT + i;
-                zz[i] = -INFINITY;
-                pp[i] = 0;
-                rr[i] = 0;
-                if (e < ntc * 16) {
-                    pp[i] = ctile[e >> 4] * 16 + (e & 15);
-                    zz[i] = __ldcg(zr + pp[i]);
-                    if (GATHER) rr[i] = row_of_pos(pp[i]);
-                    if (zz[i] > thr) bits |= 1u << i;
+                for (int q4 = 0; q4 < 4; ++q4) {
+                    const float4 f = __ldcg(zp + q4);
+                    zz[4 * q4] = f.x;
+                    zz[4 * q4 + 1] = f.y;
+                    zz[4 * q4 + 2] = f.z;
+                    zz[4 * q4 + 3] = f.w;
                 }
+                if (GATHER) row0 = row_of_pos(pos0);  // tiles never straddle pages
+#pragma unroll
+                for (int k = 0; k < 16; ++k)
+                    if (zz[k] > thr) bits |= 1u << k;
+                // the value rows of the candidates travel to L2 while tau is solved
+                if (GATHER)
+#pragma unroll
+                    for (int k = 0; k < 16; ++k)
+                        if ((bits >> k) & 1u) prefetch_l2_row<D>(a.v + (size_t)(row0 + k) * D);
             }
             int tot;
             int w = nc + block_excl_scan(__popc(bits), wcnt, &tot);
 #pragma unroll
-            for (int i = 0; i < TPT; ++i)
-                if (bits & (1u << i)) {
-                    if (w < ZCAP) {
-                        cz[w] = zz[i];
-                        cpos[w] = pp[i];
-                        if (GATHER) crow[w] = rr[i];
+            for (int k = 0; k < 16; ++k)
+                if ((bits >> k) & 1u) {
+                    if (w < zcap) {
+                        cz[w] = zz[k];
+                        cpos[w] = pos0 + k;
+                        if (GATHER) crow[w] = row0 + k;
                     }
                     ++w;
                 }
             nc += tot;
         }
     } else {
-        nc = ZCAP + 1;  // too many candidate tiles to list: the whole-row path below
+        nc = zcap + 1;  // too many candidate tiles to list: the whole-row path below
     }
     __syncthreads();
-    const bool onchip = nc <= ZCAP;
+    const bool onchip = nc <= zcap;
     if (!onchip && threadIdx.x == 0) atomicOr(a.status, ENTMAXKV_STATUS_OVERFLOW);
     const int nloop = onchip ? nc : n_tok;
     auto cz_at = [&](int i) -> float { return onchip ? cz[i] : __ldcg(zr + i); };
 
-    // Multisection on [z_max - 1, z_max - n^(1-alpha)]: 32 points per pass,
-    // lane l of every warp evaluates point l over the warp's slice of the
-    // candidates (slices and order are fixed, so the sums are reproducible),
-    // and the warps' partial sums are added in warp order.
+    // Newton's method on F(t) = sum_c [z_c - t]_+^r - 1, which is decreasing
+    // on [z_max - 1, z_max - n^(1-alpha)] and convex for r >= 1 (alpha <= 2),
+    // concave for r < 1: started from the end of that bracket where F has the
+    // sign that keeps the iterates on one side of the root, they move to it
+    // monotonically.  Each thread sums [x]_+^r and [x]_+^(r-1) over its
+    // strided share of the candidates, the warps' sums are added in warp
+    // order (reproducible), and every warp takes the same step.
     // (on chip nc is the exact candidate count; off chip only a lower bound on
     // it, so the bracket uses every token of the list)
-    float lo = thr;
-    float hi = zmax - powf((float)(onchip ? nc : n_tok), 1.f - a.alpha);
+    const float lo = thr;
+    const float hi = zmax - powf((float)(onchip ? nc : n_tok), 1.f - a.alpha);
+    float tau = lo;
     if (nc > 1 && hi > lo) {
         const float tol = 1e-7f * fmaxf(1.f, fabsf(zmax));
-        for (int pass = 0; pass < 12 && hi - lo > tol; ++pass) {
-            const float w = (hi - lo) / 33.f;
-            const float t = lo + w * (float)(lane + 1);
-            float f = 0.f;
+        const int rim1 = ri >= 2 ? ri - 1 : 0;
+        float t = r >= 1.f ? lo : hi;
+        for (int it = 0; it < 40; ++it) {
+            float s0 = 0.f, s1 = 0.f;  // sum x^r, sum x^(r-1) over x = z - t > 0
+            auto add = [&](float z) {
+                const float x = z - t;
+                if (x > 0.f) {
+                    const float y = ri == 1 ? 1.f : pos_pow(x, r - 1.f, rim1);
+                    s0 = fmaf(x, y, s0);
+                    s1 += y;
+                }
+            };
             if (onchip) {
-                const int per = ceil_div(nc, TAU_WARPS);
-                const int c1 = min(nc, (warp + 1) * per);
-                for (int c = warp * per; c < c1; ++c) f += pos_pow(cz[c] - t, r, ri);
+                for (int c = threadIdx.x; c < nc; c += TAU_NT) add(cz[c]);
             } else {
                 // too many candidates to hold: stream the z row through shared
-                // memory in coalesced chunks of ZCAP, each warp summing a slice
-                for (int c0 = 0; c0 < n_tok; c0 += ZCAP) {
-                    const int m = min(ZCAP, n_tok - c0);
+                // memory in coalesced chunks of zcap
+                for (int c0 = 0; c0 < n_tok; c0 += zcap) {
+                    const int m = min(zcap, n_tok - c0);
                     __syncthreads();  // the previous chunk has been read
-                    for (int i = threadIdx.x; i < m; i += TAU_THREADS) cz[i] = __ldcg(zr + c0 + i);
+                    for (int i = threadIdx.x; i < m; i += TAU_NT) cz[i] = __ldcg(zr + c0 + i);
                     __syncthreads();
-                    const int per = ceil_div(m, TAU_WARPS);
-                    const int c1 = min(m, (warp + 1) * per);
-                    for (int c = warp * per; c < c1; ++c) {
-                        const float z = cz[c];
-                        if (z > thr) f += pos_pow(z - t, r, ri);
-                    }
+                    for (int c = threadIdx.x; c < m; c += TAU_NT) add(cz[c]);
                 }
             }
-            red[warp][lane] = f;
-            __syncthreads();
-            if (warp == 0) {
-                float tot = 0.f;
-                for (int ww = 0; ww < TAU_WARPS; ++ww) tot += red[ww][lane];
-                // points increase with the lane and F decreases: the ones at or
-                // left of the root form a prefix
-                const int cntge = __popc(__ballot_sync(FULL, tot >= 1.f));
-                if (lane == 0) {
-                    br[0] = cntge > 0 ? lo + w * (float)cntge : lo;
-                    br[1] = cntge < 32 ? lo + w * (float)(cntge + 1) : hi;
-                }
+#pragma unroll
+            for (int o = 16; o; o >>= 1) {
+                s0 += __shfl_xor_sync(FULL, s0, o);
+                s1 += __shfl_xor_sync(FULL, s1, o);
             }
-            __syncthreads();
-            const float wold = hi - lo;
-            lo = br[0];
-            hi = br[1];
-            if (!(hi - lo < wold)) break;  // at the float resolution of the bracket
+            if (lane == 0) {
+                red[it & 1][warp][0] = s0;
+                red[it & 1][warp][1] = s1;
+            }
+            __syncthreads();  // (the other buffer takes the next pass: one barrier a pass)
+            float S0 = 0.f, S1 = 0.f;
+#pragma unroll
+            for (int ww = 0; ww < TAU_NW; ++ww) {
+                S0 += red[it & 1][ww][0];
+                S1 += red[it & 1][ww][1];
+            }
+            if (!(S1 > 0.f)) break;  // no weight right of t (t at the top already)
+            // t' = t - F(t) / F'(t), F' = -r S1
+            const float tn = fminf(hi, fmaxf(lo, t + (S0 - 1.f) / (r * S1)));
+            const bool done = !(fabsf(tn - t) > tol);
+            t = tn;
+            if (done) break;
         }
-    } else {
-        hi = lo;
+        tau = t;
     }
-    const float tau = 0.5f * (lo + hi);
     if (threadIdx.x == 0) {
         a.ws.tau[bh] = tau;
         if (a.tau_out) a.tau_out[bh] = tau;
@@ -597,39 +638,36 @@ __global__ void __launch_bounds__(TAU_THREADS) tau_pv_kernel(const __grid_consta
         a.p_out[(size_t)bh * lstride + (size_t)page * P + t] = p;
     };
     auto gather8 = [&](int nr, int row, float p) {
-        // lanes 0..nr-1 hold (row, p) of up to eight support tokens
-        float vv[8][CPL], pp[8];
+        // lanes 0..nr-1 hold (row, p) of up to eight support tokens; the
+        // rows' bf16 words are all loaded before the first product
+        unsigned vw[8][CPL / 2];
+        float pp[8];
 #pragma unroll
         for (int i = 0; i < 8; ++i) {
             const int rw = __shfl_sync(FULL, row, i);
             pp[i] = i < nr ? __shfl_sync(FULL, p, i) : 0.f;
-            if (i < nr) {
-                const uint16_t *vr = a.v + (size_t)rw * D + lane * CPL;
-                if (CPL == 4) {
-                    const uint2 w = __ldg(reinterpret_cast<const uint2 *>(vr));
-                    vv[i][0] = bf16lo(w.x);
-                    vv[i][1] = bf16hi(w.x);
-                    vv[i][2] = bf16lo(w.y);
-                    vv[i][3] = bf16hi(w.y);
-                } else {
-                    const unsigned w = __ldg(reinterpret_cast<const unsigned *>(vr));
-                    vv[i][0] = bf16lo(w);
-                    vv[i][1] = bf16hi(w);
-                }
+            const uint16_t *vr = a.v + (size_t)rw * D + lane * CPL;
+            if (CPL == 4) {
+                uint2 w = make_uint2(0u, 0u);
+                if (i < nr) w = __ldg(reinterpret_cast<const uint2 *>(vr));
+                vw[i][0] = w.x;
+                vw[i][CPL / 2 - 1] = w.y;
             } else {
-#pragma unroll
-                for (int cc = 0; cc < CPL; ++cc) vv[i][cc] = 0.f;
+                vw[i][0] = i < nr ? __ldg(reinterpret_cast<const unsigned *>(vr)) : 0u;
             }
         }
 #pragma unroll
         for (int i = 0; i < 8; ++i)
 #pragma unroll
-            for (int cc = 0; cc < CPL; ++cc) acc[cc] = fma((double)pp[i], (double)vv[i][cc], acc[cc]);
+            for (int cc = 0; cc < CPL; ++cc) {
+                const unsigned w = vw[i][cc >> 1];
+                acc[cc] = fma((double)pp[i], (double)((cc & 1) ? bf16hi(w) : bf16lo(w)), acc[cc]);
+            }
     };
-    // candidate c belongs to warp c % 16 (lane (c / 16) % 32), so a small
-    // support spreads over all warps
-    for (int k0 = 0; k0 < nloop; k0 += TAU_THREADS) {
-        const int c = k0 + lane * TAU_WARPS + warp;
+    // candidate c belongs to warp c % TAU_NW (lane (c / TAU_NW) % 32), so a
+    // small support spreads over all warps
+    for (int k0 = 0; k0 < nloop; k0 += TAU_NT) {
+        const int c = k0 + lane * TAU_NW + warp;
         const float z = c < nloop ? cz_at(c) : -INFINITY;
         const float p = pos_pow(z - tau, r, ri);
         unsigned bal = __ballot_sync(FULL, p > 0.f);
@@ -643,7 +681,7 @@ __global__ void __launch_bounds__(TAU_THREADS) tau_pv_kernel(const __grid_consta
                     if (lane == i) src = l;
                     nr = i + 1;
                 }
-            const int cs = k0 + __shfl_sync(FULL, lane, src) * TAU_WARPS + warp;
+            const int cs = k0 + __shfl_sync(FULL, lane, src) * TAU_NW + warp;
             const float pl = __shfl_sync(FULL, p, src);
             int row = 0;
             if (lane < nr) {
@@ -658,10 +696,10 @@ __global__ void __launch_bounds__(TAU_THREADS) tau_pv_kernel(const __grid_consta
 #pragma unroll
     for (int cc = 0; cc < CPL; ++cc) accs[warp][lane * CPL + cc] = acc[cc];
     __syncthreads();
-    for (int j = threadIdx.x; j < D; j += TAU_THREADS) {
+    for (int j = threadIdx.x; j < D; j += TAU_NT) {
         double sum = 0.0;
 #pragma unroll
-        for (int w = 0; w < TAU_WARPS; ++w) sum += accs[w][j];
+        for (int w = 0; w < TAU_NW; ++w) sum += accs[w][j];
         a.out[(size_t)bh * D + j] = (float)sum;
     }
 }
@@ -1050,8 +1088,9 @@ cudaError_t sparse_t(const DecodeArgs &a, cudaStream_t st) {
         return launch_pdl(k, dim3(S, groups), dim3(DEC_THREADS), RG::BYTES, st, a);
     }
     if ((e = launch_qk<D, G, false>(a, st)) != cudaSuccess) return e;
-    if ((e = set_smem(tau_pv_kernel<D, true>, TAU_SMEM)) != cudaSuccess) return e;
-    return launch_pdl(tau_pv_kernel<D, true>, dim3(a.B * a.Hq), dim3(TAU_THREADS), TAU_SMEM, st, a, 0);
+    const int zcap = tau_zcap(a.B * a.Hq, a.sms);
+    if ((e = set_smem(tau_pv_kernel<D, true>, tau_smem(ZCAP_MAX))) != cudaSuccess) return e;
+    return launch_pdl(tau_pv_kernel<D, true>, dim3(a.B * a.Hq), dim3(TAU_NT), tau_smem(zcap), st, a, 0, zcap);
 }
 
 template <int D, int G>
@@ -1061,8 +1100,11 @@ cudaError_t dense_entmax_t(const DecodeArgs &a, cudaStream_t st) {
     const int n = a.B * a.Hq > groups ? a.B * a.Hq : groups;
     if ((e = launch_pdl(dense_init_kernel, dim3(ceil_div(n, 256)), dim3(256), 0, st, a)) != cudaSuccess) return e;
     if ((e = launch_qk<D, G, true>(a, st)) != cudaSuccess) return e;
-    if ((e = set_smem(tau_pv_kernel<D, false>, TAU_SMEM)) != cudaSuccess) return e;
-    if ((e = launch_pdl(tau_pv_kernel<D, false>, dim3(a.B * a.Hq), dim3(TAU_THREADS), TAU_SMEM, st, a, 1)) != cudaSuccess) return e;
+    const int zcap = tau_zcap(a.B * a.Hq, a.sms);
+    if ((e = set_smem(tau_pv_kernel<D, false>, tau_smem(ZCAP_MAX))) != cudaSuccess) return e;
+    if ((e = launch_pdl(tau_pv_kernel<D, false>, dim3(a.B * a.Hq), dim3(TAU_NT), tau_smem(zcap), st, a, 1, zcap)) !=
+        cudaSuccess)
+        return e;
     auto k = pv_stream_kernel<D, G>;
     constexpr size_t smem = pvs_smem<D, G>();
     if ((e = set_smem(k, smem)) != cudaSuccess) return e;
