@@ -3,9 +3,9 @@
 // full-cache entmax and full-cache softmax as comparison points).
 //
 // Sparse path, three launches on one stream, no host round trip:
-//   union_kernel   per (sequence, kv head), a cluster of 8 CTAs: union of
-//                  the G query heads' selected pages, ascending, each with a
-//                  G-bit head mask; also resets the per-head maxima.
+//   union_kernel   per (sequence, kv head), one CTA: union of the G query
+//                  heads' selected pages, ascending, each with a G-bit head
+//                  mask; also resets the per-head maxima.
 //   qk_kernel      split over the union: TMA 2-D loads (128-byte swizzle) of
 //                  the K tiles through a 4-stage mbarrier ring fed by one
 //                  producer warp (which resolves union entries and page-table
@@ -17,10 +17,10 @@
 //   tau_pv_kernel  per (sequence, query head): every token that can carry
 //                  weight has z > max z - 1 (no weight exceeds 1), so those
 //                  candidates are compacted on chip in list order; the exact
-//                  root of sum (z - tau)_+^r = 1 is bracketed in
-//                  [z_max - 1, z_max - n^(1-alpha)] and narrowed by
-//                  multisection, and p v is summed over the support, reading
-//                  only those value rows.
+//                  root of sum (z - tau)_+^r = 1 lies in
+//                  [z_max - 1, z_max - n^(1-alpha)] and is reached by Newton's
+//                  method from the end where it is monotone, and p v is summed
+//                  over the support, reading only those value rows.
 // Full-cache entmax runs qk_kernel over every page, tau_pv_kernel for tau, and
 // pv_stream_kernel, which streams every V tile through the TMA ring.  Full-cache softmax runs softmax_kernel (K and V
 // tiles per stage, online max / sum per split); both dense paths combine
@@ -34,103 +34,97 @@ namespace {
 // ------------------------------------------------------------------ union
 
 // Union of the G heads' selections of a group, ascending, each entry with its
-// head mask.  A cluster of UCL CTAs per (sequence, kv head): CTA r owns pages
-// [r Q, (r+1) Q) (Q a multiple of 4), reads every head's list and marks the
-// pages in its range in a shared-memory bitmap (one byte of head bits per
-// page), compacts them in page order, and learns where its entries start
-// from the counts the lower-ranked CTAs push into its shared memory.
-constexpr int UCL = 8;
-constexpr int UTH = 256;
+// head mask.  One CTA per (sequence, kv head): the pages are taken UCH at a
+// time; every head's entries that fall in the chunk mark a shared-memory
+// bitmap (one byte of head bits per page), which is then compacted in page
+// order behind the entries of the earlier chunks.
+constexpr int UTH = 512;
+constexpr int UCH = 16384;  // pages per chunk (one byte each)
 
-__global__ void __cluster_dims__(UCL, 1, 1) __launch_bounds__(UTH) union_kernel(DecodeArgs a) {
+__global__ void __launch_bounds__(UTH) union_kernel(DecodeArgs a) {
     pdl_wait();
-    extern __shared__ unsigned words[];
+    __shared__ unsigned words[UCH / 4];
     __shared__ int sh[72];
     __shared__ int cnts[8], offs[9];
-    __shared__ int rcount[UCL];  // pushed by every CTA of the cluster
-    const unsigned rank = cl_rank();
-    const int bk = blockIdx.x / UCL;
+    const int bk = blockIdx.x;
     const int b = bk / a.Hkv, kvh = bk % a.Hkv;
     const int G = a.Hq / a.Hkv;
     const int np = n_pages_of(a.seq_lens[b], a.P);
-    const int Q = ceil_div(ceil_div(np, UCL), 4) * 4;
-    const int lo = min(np, (int)rank * Q), hi = min(np, (int)(rank + 1) * Q);
-    const int nw = ceil_div(hi - lo, 4);
-    for (int i = threadIdx.x; i < nw; i += UTH) words[i] = 0u;
     if (threadIdx.x < G) {
         const int bh = b * a.Hq + kvh * G + threadIdx.x;
         int c = a.cnt[bh];
         if (c < 0 || c > np) {
-            if (rank == 0) atomicOr(a.status, ENTMAXKV_STATUS_BAD_SELECTION);
+            atomicOr(a.status, ENTMAXKV_STATUS_BAD_SELECTION);
             c = c < 0 ? 0 : np;
         }
         cnts[threadIdx.x] = c;
-        if (rank == 0) a.ws.zmax[bh] = ORD_NEG_INF;
+        a.ws.zmax[bh] = ORD_NEG_INF;
     }
-    if (rank == 0 && threadIdx.x == 0) a.ws.counters[bk] = 0;  // the softmax path's last-CTA combine
+    if (threadIdx.x == 0) a.ws.counters[bk] = 0;  // the softmax path's last-CTA combine
     __syncthreads();
     if (threadIdx.x == 0) {
         offs[0] = 0;
         for (int g = 0; g < G; ++g) offs[g + 1] = offs[g] + cnts[g];
     }
     __syncthreads();
-    // every head's entries as one flat range, four loads in flight per thread
-    const int total = offs[G];
-    for (int k0 = threadIdx.x; k0 < total; k0 += 4 * UTH) {
-        int p[4], g[4];
+    const int total = offs[G];  // every head's entries as one flat range
+    int *ue = a.ws.union_e + (size_t)bk * a.max_pages;
+    int done = 0;
+    for (int lo = 0; lo < np; lo += UCH) {
+        const int hi = min(np, lo + UCH);
+        const int nw = ceil_div(hi - lo, 4);
+        for (int i = threadIdx.x; i < nw; i += UTH) words[i] = 0u;
+        __syncthreads();
+        // four loads in flight per thread
+        for (int k0 = threadIdx.x; k0 < total; k0 += 4 * UTH) {
+            int p[4], g[4];
 #pragma unroll
-        for (int u = 0; u < 4; ++u) {
-            const int k = k0 + u * UTH;
-            p[u] = -1;
-            g[u] = 0;
-            if (k < total) {
-                int gg = 0;
-                while (k >= offs[gg + 1]) ++gg;
-                g[u] = gg;
-                p[u] = __ldg(a.sel + (size_t)(b * a.Hq + kvh * G + gg) * a.max_pages + (k - offs[gg]));
+            for (int u = 0; u < 4; ++u) {
+                const int k = k0 + u * UTH;
+                p[u] = -1;
+                g[u] = 0;
+                if (k < total) {
+                    int gg = 0;
+                    while (k >= offs[gg + 1]) ++gg;
+                    g[u] = gg;
+                    p[u] = __ldg(a.sel + (size_t)(b * a.Hq + kvh * G + gg) * a.max_pages + (k - offs[gg]));
+                }
+            }
+#pragma unroll
+            for (int u = 0; u < 4; ++u) {
+                if (k0 + u * UTH >= total) continue;
+                if (p[u] >= lo && p[u] < hi)
+                    atomicOr(&words[(p[u] - lo) >> 2], 1u << ((p[u] & 3) * 8 + g[u]));
+                else if ((p[u] < 0 || p[u] >= np) && lo == 0)
+                    atomicOr(a.status, ENTMAXKV_STATUS_BAD_SELECTION);
             }
         }
+        __syncthreads();
+        // the chunk's entries in page order: thread t owns words [t*wpt, (t+1)*wpt)
+        const int wpt = ceil_div(nw, UTH);
+        const int w0 = threadIdx.x * wpt;
+        int mine = 0;
+        for (int i = 0; i < wpt; ++i)
+            if (w0 + i < nw) {
+                const unsigned w = words[w0 + i];
 #pragma unroll
-        for (int u = 0; u < 4; ++u) {
-            if (k0 + u * UTH >= total) continue;
-            if (p[u] >= lo && p[u] < hi)
-                atomicOr(&words[(p[u] - lo) >> 2], 1u << ((p[u] & 3) * 8 + g[u]));
-            else if ((p[u] < 0 || p[u] >= np) && rank == 0)
-                atomicOr(a.status, ENTMAXKV_STATUS_BAD_SELECTION);
-        }
-    }
-    __syncthreads();
-    // this CTA's entries in page order: thread t owns words [t*wpt, (t+1)*wpt)
-    const int wpt = ceil_div(nw, UTH);
-    const int w0 = threadIdx.x * wpt;
-    int mine = 0;
-    for (int i = 0; i < wpt; ++i)
-        if (w0 + i < nw) {
+                for (int j = 0; j < 4; ++j) mine += ((w >> (8 * j)) & 0xffu) ? 1 : 0;
+            }
+        int chunk_total;
+        int pos = done + block_excl_scan(mine, sh, &chunk_total);
+        for (int i = 0; i < wpt; ++i) {
+            if (w0 + i >= nw) break;
             const unsigned w = words[w0 + i];
 #pragma unroll
-            for (int j = 0; j < 4; ++j) mine += ((w >> (8 * j)) & 0xffu) ? 1 : 0;
+            for (int j = 0; j < 4; ++j) {
+                const unsigned m = (w >> (8 * j)) & 0xffu;
+                if (m) ue[pos++] = ((lo + 4 * (w0 + i) + j) << 8) | (int)m;
+            }
         }
-    int local;
-    int pos = block_excl_scan(mine, sh, &local);
-    if (threadIdx.x < UCL) cl_sti(cl_map(&rcount[rank], threadIdx.x), local);
-    cl_sync();
-    int before = 0, all = 0;
-#pragma unroll
-    for (int r = 0; r < UCL; ++r) {
-        before += r < (int)rank ? rcount[r] : 0;
-        all += rcount[r];
+        done += chunk_total;
+        __syncthreads();  // the bitmap is read before the next chunk clears it
     }
-    int *ue = a.ws.union_e + (size_t)bk * a.max_pages + before;
-    for (int i = 0; i < wpt; ++i) {
-        if (w0 + i >= nw) break;
-        const unsigned w = words[w0 + i];
-#pragma unroll
-        for (int j = 0; j < 4; ++j) {
-            const unsigned m = (w >> (8 * j)) & 0xffu;
-            if (m) ue[pos++] = ((lo + 4 * (w0 + i) + j) << 8) | (int)m;
-        }
-    }
-    if (rank == 0 && threadIdx.x == 0) a.ws.union_cnt[bk] = all;
+    if (threadIdx.x == 0) a.ws.union_cnt[bk] = done;
 }
 
 __global__ void dense_init_kernel(DecodeArgs a) {
@@ -1076,9 +1070,7 @@ template <int D, int G>
 cudaError_t sparse_t(const DecodeArgs &a, cudaStream_t st) {
     cudaError_t e;
     const int groups = a.B * a.Hkv;
-    const size_t ub = (size_t)ceil_div(ceil_div(a.max_pages, UCL), 4) * 4;
-    if ((e = set_smem(union_kernel, ub)) != cudaSuccess) return e;
-    if ((e = launch_pdl(union_kernel, dim3(groups * UCL), dim3(UTH), ub, st, a)) != cudaSuccess) return e;
+    if ((e = launch_pdl(union_kernel, dim3(groups), dim3(UTH), 0, st, a)) != cudaSuccess) return e;
     if (a.alpha == 1.f) {
         // softmax over the selected pages: K and V of the union, split over pages
         using RG = Ring<D, G, 3, 2>;
