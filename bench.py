@@ -1,9 +1,10 @@
 """Benchmark of one EntmaxKV sparse alpha-entmax decode step on B200.
 
-A step is the whole hot path for one batch: refresh the metadata of the page
-the newest token went to (entmaxkv_build_meta, one page per sequence), score
-every page (entmaxkv_score_pages), select (entmaxkv_select, top-k or Gaussian
-tau_hat - Delta) and decode over the selected pages (entmaxkv_decode_sparse).
+A step is the whole hot path for one batch: append each sequence's newest
+token (its key/value rows written to its slot and its page's metadata rebuilt,
+entmaxkv_append), score every page (entmaxkv_score_pages), select
+(entmaxkv_select, top-k or Gaussian tau_hat - Delta) and decode over the
+selected pages (entmaxkv_decode_sparse).
 Default workload: B=1, Hq=32, Hkv=8, d=128, 1,048,576-token context, 64-token
 pages, alpha=1.5, Gaussian selection with Delta=0.5 (the long-context setting of
 the EntmaxKV efficiency study), synthetic clustered keys with 64 needles per
@@ -168,7 +169,7 @@ def support_rows_of(wl, p_out):
 
 def run_gpu(args, rank, world):
     from sparse_entmax_kv_b200 import native as nv
-    from sparse_entmax_kv_b200.decoder import EntmaxKVDecoder, kernels_per_step
+    from sparse_entmax_kv_b200.decoder import EntmaxKVDecoder, kernels_per_step, last_token_rows
     from sparse_entmax_kv_b200.workloads import CONFIGS, make_inputs
 
     wl = CONFIGS[args.workload]
@@ -180,9 +181,12 @@ def run_gpu(args, rank, world):
     dec = EntmaxKVDecoder(inp["k_cache"], inp["v_cache"], inp["page_table"], inp["seq_lens"], wl.Hq,
                           alpha=wl.alpha, policy=policy, k=k, delta=delta)
     dec.build_meta()
-    # the newest token of sequence 0 sits in its last page; appends rewrite it
+    # each sequence's newest token (position seq_len-1) is appended again every
+    # step: its key/value rows are written to their slot and its page's
+    # metadata is rebuilt, leaving the cache as it was
     L0 = int(inp["seq_lens"][0])
-    append_page = (L0 - 1) // wl.P
+    k_new, v_new = last_token_rows(inp["k_cache"], inp["v_cache"], inp["page_table"], inp["seq_lens"])
+    new_kv = (k_new, v_new)
     flush_w = torch.empty(256 << 20, dtype=torch.uint8, device=dev)
     flush_r = torch.ones(32 << 20, dtype=torch.int64, device=dev)
 
@@ -196,7 +200,7 @@ def run_gpu(args, rank, world):
 
     # byte model from one untimed step with p written out
     p_out = torch.zeros((wl.B, wl.Hq, wl.max_pages * wl.P), device=dev)
-    dec.step(q, append_page, p_out=p_out)
+    dec.step(q, p_out=p_out, new_kv=new_kv)
     torch.cuda.synchronize()
     nbytes = step_bytes(wl, dec, support_rows_of(wl, p_out))
     del p_out
@@ -207,16 +211,16 @@ def run_gpu(args, rank, world):
 
     # One step (the four C-ABI calls) captured as a CUDA graph: the timed
     # region replays it, so host launch latency does not enter the device time.
-    dec.step(q, append_page)  # eager first call: per-device set-up happens outside capture
+    dec.step(q, new_kv=new_kv)  # eager first call: per-device set-up happens outside capture
     torch.cuda.synchronize()
     graph = torch.cuda.CUDAGraph()
     side = torch.cuda.Stream()
     side.wait_stream(torch.cuda.current_stream())
     with torch.cuda.stream(side):
-        dec.step(q, append_page)
+        dec.step(q, new_kv=new_kv)
     torch.cuda.current_stream().wait_stream(side)
     with torch.cuda.graph(graph):
-        dec.step(q, append_page)
+        dec.step(q, new_kv=new_kv)
     torch.cuda.synchronize()
     gev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(args.steps)]
 
@@ -255,7 +259,8 @@ def run_gpu(args, rank, world):
             l2_flush()
             e = ev[i]
             e[0].record(st)
-            nv.entmaxkv_build_meta(dec.shape, dec.k_cache, dec.page_table, dec.seq_lens, append_page, 1, dec.meta)
+            nv.entmaxkv_append(dec.shape, k_new, v_new, dec.page_table, dec.seq_lens, dec.k_cache, dec.v_cache,
+                               dec.meta)
             e[1].record(st)
             nv.entmaxkv_score_pages(dec.shape, q, dec.meta, dec.seq_lens, dec.bbox, dec.mu,
                                     dec.sigma)
@@ -278,7 +283,7 @@ def run_gpu(args, rank, world):
     stage_ms = np.array([[ev[i][j].elapsed_time(ev[i][j + 1]) for j in range(nst)] for i in range(args.steps)])
     eager_step_ms = float(stage_ms.sum(axis=1).mean())
     step_ms, = max_over_ranks([step_ms], world, dev)
-    stage_us = dict(zip(["build_meta_append", "score_pages", "select", "decode_sparse"],
+    stage_us = dict(zip(["append", "score_pages", "select", "decode_sparse"],
                         (stage_ms.mean(axis=0) * 1e3).round(2).tolist()))
 
     # comparison paths at the same context: full-cache entmax and softmax
@@ -301,25 +306,20 @@ def run_gpu(args, rank, world):
             dense[name] = statistics.median(ts) * 1e3
         del ws
 
-    # end to end through the C ABI with host buffers: q and the appended token's
-    # k/v come from pinned host memory each step, the output goes back to host
-    G = wl.G
-    tok = (L0 - 1) % wl.P
-    blk = int(inp["page_table"][0, append_page])
-    k_new = inp["k_cache"][blk, :, tok].clone().cpu().pin_memory()
-    v_new = inp["v_cache"][blk, :, tok].clone().cpu().pin_memory()
-    q_host = q.cpu().pin_memory()
+    # end to end through the C ABI with host buffers: q and the appended
+    # token's k/v rows come from one pinned host buffer each step (one
+    # host-to-device copy), the output goes back to host
+    n_q, n_kv = q.numel(), k_new.numel()
+    stage_host = torch.cat([q.reshape(-1), k_new.reshape(-1), v_new.reshape(-1)]).cpu().pin_memory()
+    stage_dev = torch.empty_like(stage_host, device=dev)
+    q_dev = stage_dev[:n_q].view_as(q)
+    k_dev = stage_dev[n_q:n_q + n_kv].view_as(k_new)
+    v_dev = stage_dev[n_q + n_kv:].view_as(v_new)
     out_host = torch.empty((wl.B, wl.Hq, wl.d), dtype=torch.float32).pin_memory()
-    k_dev = torch.empty_like(inp["k_cache"][blk, :, tok])
-    v_dev = torch.empty_like(k_dev)
-    q_dev = torch.empty_like(q)
+
     def e2e_once():
-        q_dev.copy_(q_host, non_blocking=True)
-        k_dev.copy_(k_new, non_blocking=True)
-        v_dev.copy_(v_new, non_blocking=True)
-        inp["k_cache"][blk, :, tok] = k_dev
-        inp["v_cache"][blk, :, tok] = v_dev
-        dec.step(q_dev, append_page)
+        stage_dev.copy_(stage_host, non_blocking=True)
+        dec.step(q_dev, new_kv=(k_dev, v_dev))
         out_host.copy_(dec.out, non_blocking=True)
 
     def time_e2e(fn):
@@ -368,7 +368,7 @@ def run_gpu(args, rank, world):
                        "algorithmic_bytes": galg}
     res = dict(wl=wl, step_ms=step_ms, eager_step_ms=eager_step_ms, e2e_eager_ms=e2e_eager_ms,
                stage_us=stage_us, dense=dense, nbytes=nbytes, clocks=clocks,
-               roofline=roofline, roofline_gather=roofline_gather, e2e_ms=e2e_step_ms, e2e_bytes=(q_host.numel() * 2 + k_new.numel() * 4,
+               roofline=roofline, roofline_gather=roofline_gather, e2e_ms=e2e_step_ms, e2e_bytes=(stage_host.numel() * 2,
                                                                out_host.numel() * 4),
                launches=kernels_per_step(policy == "gauss", True) * args.steps, t_wall=t_wall,
                host=dict(inp=inp, dec=dec) if (rank == 0 and not args.no_cpu_baseline) else None)
@@ -640,8 +640,9 @@ def main():
             "stages_us": res["stage_us"], "bytes_per_step": nb,
             "e2e": {"value": round(e2e_val, 2), "unit": "GB/s", "us_per_step": round(res["e2e_ms"] * 1e3, 2),
                     "h2d_bytes_per_step": res["e2e_bytes"][0], "d2h_bytes_per_step": res["e2e_bytes"][1],
-                    "how": "H2D of q and the appended token's k/v from pinned memory, append, step, D2H of the "
-                           "output, captured as one CUDA graph",
+                    "how": "one H2D copy of q and the appended token's k/v rows from one pinned buffer, the four "
+                           "C-ABI calls (append writes the rows and refreshes their pages' metadata), one D2H copy "
+                           "of the output, captured as one CUDA graph",
                     "eager_us_per_step": round(res["e2e_eager_ms"] * 1e3, 2)},
             "timing": "step = CUDA-graph replay of the four C-ABI calls; stages_us from the same calls issued "
                       "eagerly with events around each (eager step sum %.2f us)" % (res["eager_step_ms"] * 1e3),

@@ -8,6 +8,8 @@
  * every (sequence b, query head h), against a paged bf16 K/V cache:
  *
  *   entmaxkv_build_meta     per-page metadata (section 2.A)
+ *   entmaxkv_append         write each sequence's new key/value row and
+ *                           refresh the metadata of its page (section 2.A)
  *   entmaxkv_score_pages    query-aware page scores (section 2.A)
  *   entmaxkv_select         candidate pages: top-k or Gaussian tau_hat - Delta
  *                           (section 2.B)
@@ -171,6 +173,24 @@ ENTMAXKV_API int entmaxkv_build_meta(const entmaxkv_shape *shape, const void *k_
                         const int32_t *page_table, const int32_t *seq_lens,
                         int32_t first_page, int32_t n_pages, void *meta,
                         void *stream);
+
+/*
+ * Section 2.A, the append step of decoding: each sequence b with
+ * seq_lens[b] = L > 0 has just grown by one token, at position L-1.  For every
+ * kv head, write that token's key row k_new[b][kvh][0..d) and value row
+ * v_new[b][kvh][0..d) (bf16, device, [B][Hkv][d] contiguous) into slot
+ * (L-1) mod P of block page_table[b][(L-1)/P] of k_cache / v_cache, then
+ * rebuild the metadata record of logical page (L-1)/P exactly as
+ * entmaxkv_build_meta does (same bits).  Sequences with L <= 0 are skipped.  A
+ * page-table entry outside [0, num_blocks), or (L-1)/P >= max_pages, sets
+ * ENTMAXKV_STATUS_BAD_PAGE and skips that sequence.  One kernel launch on
+ * `stream`; no allocation.  k_cache, v_cache and meta must be 16-byte aligned
+ * (ENTMAXKV_ERR_ALIGN).
+ */
+ENTMAXKV_API int entmaxkv_append(const entmaxkv_shape *shape, const void *k_new,
+                    const void *v_new, const int32_t *page_table,
+                    const int32_t *seq_lens, void *k_cache, void *v_cache,
+                    void *meta, void *stream);
 
 /*
  * Section 2.A (query-aware page scoring): for every (b, h) and page p < N_b,

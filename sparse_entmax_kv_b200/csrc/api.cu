@@ -217,6 +217,35 @@ int entmaxkv_build_meta(const entmaxkv_shape *s, const void *k_cache, const int3
     return cuda_rc(launch_build_meta(a, static_cast<cudaStream_t>(stream)));
 }
 
+int entmaxkv_append(const entmaxkv_shape *s, const void *k_new, const void *v_new, const int32_t *page_table,
+                    const int32_t *seq_lens, void *k_cache, void *v_cache, void *meta, void *stream) {
+    int rc = check_shape(s);
+    if (rc) return rc;
+    if (!k_new || !v_new || !page_table || !seq_lens || !k_cache || !v_cache || !meta) return ENTMAXKV_ERR_NULL;
+    if (!aligned16(k_cache) || !aligned16(v_cache) || !aligned16(meta)) return ENTMAXKV_ERR_ALIGN;
+    DevInfo di;
+    if ((rc = device_info(&di))) return rc;
+    AppendArgs a{};
+    a.m.page_table = page_table;
+    a.m.seq_lens = seq_lens;
+    a.m.meta = static_cast<uint8_t *>(meta);
+    a.m.n_tiles = meta_tiles(s->max_pages);
+    a.m.n_tiles_total = (long long)s->B * s->Hkv * a.m.n_tiles;
+    a.m.B = s->B;
+    a.m.Hkv = s->Hkv;
+    a.m.d = s->d;
+    a.m.P = s->page_size;
+    a.m.max_pages = s->max_pages;
+    a.m.num_blocks = s->num_blocks;
+    a.m.status = di.status;
+    a.k_cache = static_cast<uint16_t *>(k_cache);
+    a.v_cache = static_cast<uint16_t *>(v_cache);
+    a.m.k = a.k_cache;
+    a.k_new = static_cast<const uint16_t *>(k_new);
+    a.v_new = static_cast<const uint16_t *>(v_new);
+    return cuda_rc(launch_append(a, static_cast<cudaStream_t>(stream)));
+}
+
 int entmaxkv_score_pages(const entmaxkv_shape *s, const void *q, const void *meta, const int32_t *seq_lens,
                          float *bbox, float *mu, float *sigma, void *stream) {
     int rc = check_shape(s);

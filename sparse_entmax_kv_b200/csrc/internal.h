@@ -34,6 +34,16 @@ struct MetaArgs {
 };
 cudaError_t launch_build_meta(const MetaArgs &a, cudaStream_t st);
 
+// One new token per sequence: its k/v rows go to slot seq_len-1 and the
+// metadata record of its page is rebuilt (the MetaArgs fields first_page and
+// n_pages are unused).
+struct AppendArgs {
+    MetaArgs m;
+    uint16_t *k_cache, *v_cache;
+    const uint16_t *k_new, *v_new;  // [B][Hkv][d]
+};
+cudaError_t launch_append(const AppendArgs &a, cudaStream_t st);
+
 struct ScoreArgs {
     const uint16_t *q;
     const uint8_t *meta;

@@ -1,6 +1,7 @@
 // meta.cu -- per-page key metadata (EntmaxKV summary, section 2.A: coordinate-
 // wise k_min / k_max for the bounding box, key mean and variance for the
-// Gaussian page model), rebuilt for a range of logical pages.
+// Gaussian page model), rebuilt for a range of logical pages, or written
+// together with each sequence's newest key/value row (append).
 //
 // One CTA per (page, sequence, kv head); thread j owns coordinate j and walks
 // the page's valid tokens in order.  Sums run in fp64 (every bf16 value and
@@ -13,28 +14,22 @@
 
 namespace ekv {
 
+// Thread j of a D-thread CTA: the record of coordinate j of logical page p of
+// (b, kvh), whose n valid keys are col[t * D], t < n.  When t_new >= 0 the
+// key of token t_new is k_new (it was just written by this thread, so it is
+// not read back through the read-only path).
 template <int D, int P>
-__global__ void __launch_bounds__(D) build_meta_kernel(MetaArgs a) {
-    pdl_wait();
-    const int b = blockIdx.y;
-    const int kvh = blockIdx.z;
-    const int p = a.first_page + blockIdx.x;
-    const int seq = a.seq_lens[b];
-    if (p >= n_pages_of(seq, P)) return;
-    const int blk = a.page_table[(size_t)b * a.max_pages + p];
-    if (blk < 0 || blk >= a.num_blocks) {
-        if (threadIdx.x == 0) atomicOr(a.status, ENTMAXKV_STATUS_BAD_PAGE);
-        return;
-    }
-    const int n = tokens_in_page(seq, P, p);
-    const long long rec = (long long)blk * a.Hkv + kvh;  // the page's keys: k_cache[blk][kvh]
-    const int j = threadIdx.x;
-    const uint16_t *col = a.k + (size_t)rec * P * D + j;
-
+__device__ __forceinline__ void page_record(const MetaArgs &a, const uint16_t *col, int n, int t_new, uint16_t k_new,
+                                            int b, int kvh, int p) {
     // every load of the page is issued before the first use
     uint16_t h[P];
 #pragma unroll
-    for (int t = 0; t < P; ++t) h[t] = t < n ? __ldg(col + (size_t)t * D) : (uint16_t)0;
+    for (int t = 0; t < P; ++t) h[t] = t < n && t != t_new ? __ldg(col + (size_t)t * D) : (uint16_t)0;
+    if (t_new >= 0) {
+#pragma unroll
+        for (int t = 0; t < P; ++t)
+            if (t == t_new) h[t] = k_new;
+    }
 
     uint16_t bmin = h[0], bmax = h[0];
     float vmin = bf16f(bmin), vmax = vmin;
@@ -55,6 +50,7 @@ __global__ void __launch_bounds__(D) build_meta_kernel(MetaArgs a) {
     double v = __dsub_rn(__ddiv_rn(s2, dn), __dmul_rn(m, m));
     if (v < 0.0) v = 0.0;
 
+    const int j = threadIdx.x;
     const int tile = p / META_TILE, sl = p % META_TILE;
     const long long T = ((long long)b * a.Hkv + kvh) * a.n_tiles + tile;
     const int c = j / 16, e = j % 16;
@@ -68,6 +64,50 @@ __global__ void __launch_bounds__(D) build_meta_kernel(MetaArgs a) {
     *reinterpret_cast<float *>(mm + 2048 + om) = (float)v;
 }
 
+template <int D, int P>
+__global__ void __launch_bounds__(D) build_meta_kernel(MetaArgs a) {
+    pdl_wait();
+    const int b = blockIdx.y;
+    const int kvh = blockIdx.z;
+    const int p = a.first_page + blockIdx.x;
+    const int seq = a.seq_lens[b];
+    if (p >= n_pages_of(seq, P)) return;
+    const int blk = a.page_table[(size_t)b * a.max_pages + p];
+    if (blk < 0 || blk >= a.num_blocks) {
+        if (threadIdx.x == 0) atomicOr(a.status, ENTMAXKV_STATUS_BAD_PAGE);
+        return;
+    }
+    const long long rec = (long long)blk * a.Hkv + kvh;  // the page's keys: k_cache[blk][kvh]
+    page_record<D, P>(a, a.k + (size_t)rec * P * D + threadIdx.x, tokens_in_page(seq, P, p), -1, 0, b, kvh, p);
+}
+
+// One CTA per (sequence, kv head): the new token's key and value rows land in
+// slot seq_len-1 of the paged cache, then the record of that page is rebuilt.
+template <int D, int P>
+__global__ void __launch_bounds__(D) append_kernel(AppendArgs a) {
+    pdl_wait();
+    const int b = blockIdx.x, kvh = blockIdx.y;
+    const int seq = a.m.seq_lens[b];
+    if (seq <= 0) return;
+    const int p = (seq - 1) / P, t = (seq - 1) % P;
+    if (p >= a.m.max_pages) {
+        if (threadIdx.x == 0) atomicOr(a.m.status, ENTMAXKV_STATUS_BAD_PAGE);
+        return;
+    }
+    const int blk = a.m.page_table[(size_t)b * a.m.max_pages + p];
+    if (blk < 0 || blk >= a.m.num_blocks) {
+        if (threadIdx.x == 0) atomicOr(a.m.status, ENTMAXKV_STATUS_BAD_PAGE);
+        return;
+    }
+    const int j = threadIdx.x;
+    const size_t src = ((size_t)b * a.m.Hkv + kvh) * D + j;
+    const size_t rec = ((size_t)blk * a.m.Hkv + kvh) * P * D;
+    const uint16_t kn = a.k_new[src];
+    a.k_cache[rec + (size_t)t * D + j] = kn;
+    a.v_cache[rec + (size_t)t * D + j] = a.v_new[src];
+    page_record<D, P>(a.m, a.k_cache + rec + j, t + 1, t, kn, b, kvh, p);
+}
+
 template <int D>
 cudaError_t launch_d(const MetaArgs &a, cudaStream_t st) {
     dim3 grid(a.n_pages, a.B, a.Hkv);
@@ -79,6 +119,21 @@ cudaError_t launch_d(const MetaArgs &a, cudaStream_t st) {
         default: return cudaErrorInvalidValue;
     }
     return e;
+}
+
+template <int D>
+cudaError_t launch_append_d(const AppendArgs &a, cudaStream_t st) {
+    dim3 grid(a.m.B, a.m.Hkv);
+    switch (a.m.P) {
+        case 16: return launch_pdl(append_kernel<D, 16>, dim3(grid), dim3(D), 0, st, a);
+        case 32: return launch_pdl(append_kernel<D, 32>, dim3(grid), dim3(D), 0, st, a);
+        case 64: return launch_pdl(append_kernel<D, 64>, dim3(grid), dim3(D), 0, st, a);
+    }
+    return cudaErrorInvalidValue;
+}
+
+cudaError_t launch_append(const AppendArgs &a, cudaStream_t st) {
+    return a.m.d == 64 ? launch_append_d<64>(a, st) : launch_append_d<128>(a, st);
 }
 
 cudaError_t launch_build_meta(const MetaArgs &a, cudaStream_t st) {

@@ -21,7 +21,8 @@
 // mbarrier, so HBM sees long contiguous reads and the SM issues no per-lane
 // copy instructions.  Each lane scores its page for all G query heads of the
 // group, so every byte crosses HBM once per group.  q sits in shared memory
-// as q+ and q- (fp64, [j][head]) and fp32 ([head][j]).
+// as (q-, q+) pairs (fp64, [j][head], one 16-byte load each) and fp32
+// ([head][j]).
 #include "common.cuh"
 #include "internal.h"
 
@@ -60,9 +61,8 @@ __global__ void __launch_bounds__(THREADS, G <= 4 ? 2 : 1) score_kernel(ScoreArg
     constexpr int NCH = D / CHK;
     constexpr int NST = RG::NST;
     extern __shared__ __align__(128) unsigned char smem[];
-    double *qp = reinterpret_cast<double *>(smem);  // [D][G] max(q, 0)
-    double *qn = qp + D * G;                         // [D][G] min(q, 0)
-    float *qh = reinterpret_cast<float *>(qn + D * G);  // [G][D] q
+    double2 *qq = reinterpret_cast<double2 *>(smem);        // [D][G] (min(q, 0), max(q, 0))
+    float *qh = reinterpret_cast<float *>(qq + D * G);       // [G][D] q
     uint64_t *bars = reinterpret_cast<uint64_t *>(smem + QBytes<D, G>::VALUE);
     unsigned char *ring = smem + ((QBytes<D, G>::VALUE + WARPS * NST * 8 + 127) & ~127);
 
@@ -73,8 +73,7 @@ __global__ void __launch_bounds__(THREADS, G <= 4 ? 2 : 1) score_kernel(ScoreArg
     for (int i = threadIdx.x; i < G * D; i += THREADS) {
         const int g = i / D, j = i % D;
         const float v = bf16f(a.q[((size_t)b * a.Hq + kvh * G + g) * D + j]);
-        qp[j * G + g] = v > 0.f ? (double)v : 0.0;
-        qn[j * G + g] = v < 0.f ? (double)v : 0.0;
+        qq[j * G + g] = make_double2(v < 0.f ? (double)v : 0.0, v > 0.f ? (double)v : 0.0);
         qh[g * D + j] = v;
     }
     if (threadIdx.x < WARPS * NST) mbar_init(&bars[threadIdx.x], 1);
@@ -151,8 +150,9 @@ __global__ void __launch_bounds__(THREADS, G <= 4 ? 2 : 1) score_kernel(ScoreArg
                 const int j = j0 + jj;
 #pragma unroll
                 for (int g = 0; g < G; ++g) {
-                    ab[g] = __fma_rn(qn[j * G + g], lo, ab[g]);
-                    ab[g] = __fma_rn(qp[j * G + g], hi, ab[g]);
+                    const double2 qg = qq[j * G + g];
+                    ab[g] = __fma_rn(qg.x, lo, ab[g]);
+                    ab[g] = __fma_rn(qg.y, hi, ab[g]);
                 }
             }
         }

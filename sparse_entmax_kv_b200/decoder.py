@@ -3,7 +3,9 @@
 ``EntmaxKVDecoder`` owns the device buffers the calls need (metadata, page
 scores, selections, workspace, output) and issues, on the current stream:
 
-  entmaxkv_build_meta    (the page each sequence's newest token landed in)
+  entmaxkv_append        (each sequence's new key/value row and its page's
+                          metadata) or entmaxkv_build_meta (a page the caller
+                          already wrote the token to)
   entmaxkv_score_pages
   entmaxkv_select        (top-k or Gaussian tau_hat - Delta)
   entmaxkv_decode_sparse
@@ -47,11 +49,16 @@ class EntmaxKVDecoder:
         nv.entmaxkv_build_meta(self.shape, self.k_cache, self.page_table, self.seq_lens,
                                first_page, n_pages, self.meta)
 
-    def step(self, q, append_page=None, p_out=None):
-        """One decode step for query q (bf16 [B, Hq, d]).  ``append_page``:
-        logical page whose metadata is refreshed first (the page the newest
-        token was written to), or None."""
-        if append_page is not None:
+    def step(self, q, append_page=None, p_out=None, new_kv=None):
+        """One decode step for query q (bf16 [B, Hq, d]).  ``new_kv``: the
+        (k_new, v_new) rows (bf16 [B, Hkv, d]) of the token each sequence just
+        gained, at position seq_lens-1, written into the cache together with
+        its page's metadata; or ``append_page``: a logical page whose metadata
+        is refreshed (the caller wrote the token already); or neither."""
+        if new_kv is not None:
+            nv.entmaxkv_append(self.shape, new_kv[0], new_kv[1], self.page_table, self.seq_lens,
+                               self.k_cache, self.v_cache, self.meta)
+        elif append_page is not None:
             nv.entmaxkv_build_meta(self.shape, self.k_cache, self.page_table, self.seq_lens,
                                    append_page, 1, self.meta)
         nv.entmaxkv_score_pages(self.shape, q, self.meta, self.seq_lens,
@@ -64,7 +71,18 @@ class EntmaxKVDecoder:
         return self.out
 
 
+def last_token_rows(k_cache, v_cache, page_table, seq_lens):
+    """(k, v) rows, bf16 [B, Hkv, d], of each sequence's token at position
+    seq_lens-1 as the cache holds them (appending them again leaves the cache
+    as it is).  Indexing only."""
+    P = k_cache.shape[2]
+    pos = (seq_lens.long() - 1).clamp(min=0)
+    blk = page_table.long().gather(1, (pos // P)[:, None])[:, 0]
+    tok = pos % P
+    return k_cache[blk, :, tok].contiguous(), v_cache[blk, :, tok].contiguous()
+
+
 def kernels_per_step(policy_gauss: bool, append: bool) -> int:
-    """Kernel launches one ``step`` issues: build_meta (1, if appending),
+    """Kernel launches one ``step`` issues: append or build_meta (1, if appending),
     score (1), select (1), decode_sparse (union, q.K, tau with p.V = 3)."""
     return (1 if append else 0) + 1 + 1 + 3

@@ -26,7 +26,7 @@ CALL_SELECT, CALL_DECODE_SPARSE, CALL_DECODE_DENSE = 2, 3, 4
 STATUS_BAD_PAGE, STATUS_BAD_SELECTION, STATUS_TIMEOUT, STATUS_OVERFLOW = 1, 2, 4, 8
 
 EXPORTED = ("entmaxkv_strerror", "entmaxkv_version", "entmaxkv_meta_bytes",
-            "entmaxkv_workspace_size", "entmaxkv_get_status", "entmaxkv_build_meta",
+            "entmaxkv_workspace_size", "entmaxkv_get_status", "entmaxkv_build_meta", "entmaxkv_append",
             "entmaxkv_score_pages", "entmaxkv_select", "entmaxkv_decode_sparse",
             "entmaxkv_decode_sparse_static", "entmaxkv_decode_dense")
 
@@ -74,6 +74,7 @@ def lib():
         L.entmaxkv_workspace_size.argtypes = [sp, C.c_int]
         L.entmaxkv_get_status.argtypes = [C.POINTER(i32), C.c_int, vp]
         L.entmaxkv_build_meta.argtypes = [sp, vp, vp, vp, i32, i32, vp, vp]
+        L.entmaxkv_append.argtypes = [sp, vp, vp, vp, vp, vp, vp, vp, vp]
         L.entmaxkv_score_pages.argtypes = [sp, vp, vp, vp, vp, vp, vp, vp]
         L.entmaxkv_select.argtypes = [sp, vp, vp, vp, vp, i32, i32, f32, f32, vp, vp, vp, vp, sz, vp]
         L.entmaxkv_decode_sparse.argtypes = [sp, vp, vp, vp, vp, vp, vp, vp, f32, vp, vp, vp, vp, sz, vp]
@@ -142,6 +143,14 @@ def entmaxkv_build_meta(shape, k_cache, page_table, seq_lens, first_page, n_page
         C.byref(shape), _ptr(k_cache, torch.bfloat16, "k_cache"), _ptr(page_table, torch.int32, "page_table"),
         _ptr(seq_lens, torch.int32, "seq_lens"), int(first_page), int(n_pages), _ptr(meta, None, "meta"),
         _stream(stream)))
+
+
+def entmaxkv_append(shape, k_new, v_new, page_table, seq_lens, k_cache, v_cache, meta, stream=None):
+    _check("entmaxkv_append", lib().entmaxkv_append(
+        C.byref(shape), _ptr(k_new, torch.bfloat16, "k_new"), _ptr(v_new, torch.bfloat16, "v_new"),
+        _ptr(page_table, torch.int32, "page_table"), _ptr(seq_lens, torch.int32, "seq_lens"),
+        _ptr(k_cache, torch.bfloat16, "k_cache"), _ptr(v_cache, torch.bfloat16, "v_cache"),
+        _ptr(meta, None, "meta"), _stream(stream)))
 
 
 def entmaxkv_score_pages(shape, q, meta, seq_lens, bbox, mu=None, sigma=None, stream=None):

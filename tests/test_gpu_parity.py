@@ -430,6 +430,70 @@ def test_append_rebuild_matches_full_build():
                                       y[bl * wl.Hkv:(bl + 1) * wl.Hkv].view(np.uint8))
 
 
+@pytest.mark.parametrize("name", list(SMALL))
+def test_append_writes_rows_and_rebuilds_page(name):
+    """entmaxkv_append: each sequence's new key/value rows land in slot
+    seq_len-1 (nothing else in the caches changes) and every metadata record
+    equals the oracle's build over the updated cache, to the bit."""
+    wl = SMALL[name]
+    inp, _ = gpu_inputs(wl, 11)
+    s = shape_of(wl)
+    meta = nv.alloc_meta(s, "cuda")
+    nv.entmaxkv_build_meta(s, inp["k_cache"], inp["page_table"], inp["seq_lens"], 0, -1, meta)
+    g = torch.Generator(device="cuda").manual_seed(5)
+    k_new = (torch.randn(wl.B, wl.Hkv, wl.d, device="cuda", generator=g) * 2).to(torch.bfloat16)
+    v_new = torch.randn(wl.B, wl.Hkv, wl.d, device="cuda", generator=g).to(torch.bfloat16)
+    k_new[:, :, ::7] = 0.0  # exact zeros and ties with the page's other keys
+    k_ref, v_ref = inp["k_cache"].clone(), inp["v_cache"].clone()
+    for b in range(wl.B):
+        L = int(inp["seq_lens"][b])
+        if L > 0:
+            blk = int(inp["page_table"][b, (L - 1) // wl.P])
+            k_ref[blk, :, (L - 1) % wl.P] = k_new[b]
+            v_ref[blk, :, (L - 1) % wl.P] = v_new[b]
+    nv.get_status(clear=True)
+    nv.entmaxkv_append(s, k_new, v_new, inp["page_table"], inp["seq_lens"], inp["k_cache"], inp["v_cache"], meta)
+    torch.cuda.synchronize()
+    assert nv.get_status(clear=True) == 0
+    assert torch.equal(inp["k_cache"].view(torch.int16), k_ref.view(torch.int16))
+    assert torch.equal(inp["v_cache"].view(torch.int16), v_ref.view(torch.int16))
+    host = dict(K=to_host_u16(k_ref), page_table=inp["page_table"].cpu().numpy(),
+                seq_lens=inp["seq_lens"].cpu().numpy())
+    got = unpack_meta(meta, wl, host["page_table"], host["seq_lens"])
+    want = orc.build_meta(host["K"], host["page_table"], host["seq_lens"], wl.Hkv, wl.d, wl.P, wl.num_blocks)
+    recs = referenced_records(host, wl)
+    for gi, oi, nm in zip(got, want, ("kmin", "kmax", "mean", "var")):
+        np.testing.assert_array_equal(gi[recs].view(np.uint32 if gi.dtype == np.float32 else np.uint16),
+                                      oi[recs].view(np.uint32 if oi.dtype == np.float32 else np.uint16),
+                                      err_msg=nm)
+
+
+def test_append_bad_page_sets_status_and_skips():
+    """A page-table entry outside [0, num_blocks) flags the status and that
+    sequence writes nothing; the other sequences append as usual."""
+    wl = SMALL["gqa2_d64"]
+    inp, _ = gpu_inputs(wl, 12)
+    s = shape_of(wl)
+    meta = nv.alloc_meta(s, "cuda")
+    pt = inp["page_table"].clone()
+    L = [int(x) for x in inp["seq_lens"]]
+    pt[0, (L[0] - 1) // wl.P] = wl.num_blocks  # out of range
+    k_new = torch.full((wl.B, wl.Hkv, wl.d), 2.0, device="cuda", dtype=torch.bfloat16)
+    v_new = torch.full((wl.B, wl.Hkv, wl.d), -3.0, device="cuda", dtype=torch.bfloat16)
+    k_ref, v_ref = inp["k_cache"].clone(), inp["v_cache"].clone()
+    for b in range(1, wl.B):
+        if L[b] > 0:
+            blk = int(pt[b, (L[b] - 1) // wl.P])
+            k_ref[blk, :, (L[b] - 1) % wl.P] = k_new[b]
+            v_ref[blk, :, (L[b] - 1) % wl.P] = v_new[b]
+    nv.get_status(clear=True)
+    nv.entmaxkv_append(s, k_new, v_new, pt, inp["seq_lens"], inp["k_cache"], inp["v_cache"], meta)
+    torch.cuda.synchronize()
+    assert nv.get_status(clear=True) & nv.STATUS_BAD_PAGE
+    assert torch.equal(inp["k_cache"].view(torch.int16), k_ref.view(torch.int16))
+    assert torch.equal(inp["v_cache"].view(torch.int16), v_ref.view(torch.int16))
+
+
 # ---------------------------------------------------- full-size workloads
 
 def _sub_problem(inp, wl, b, kvh):
