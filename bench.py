@@ -45,9 +45,9 @@ PAPER_CONTEXT = {"speedup_vs_full_softmax_flashdecoding": 3.36, "speedup_vs_full
 # DRAM bytes per launch from ncu captures (dram__bytes_read.sum + dram__bytes_write.sum),
 # keyed by kernel and workload, valid only while the kernel source is unchanged.
 NCU_TRAFFIC = {
-    # captured at L=524,288 (100.69 MB read + 3.61 MB written per launch), scaled by 2 for the
-    # 1,048,576-token context: the scan is linear in the page count (profiles/step_kernels_*)
-    "score_pages/gauss_gqa_L1m": {"bytes": 2 * (100689152 + 3609088), "src": "edea3177cd8b"},
+    # one full-size launch at L=1,048,576 (201.35 MB read + 5.69 MB written), ncu --set full
+    # (profiles/score_kernel_gauss_gqa_L1m_full.md)
+    "score_pages/gauss_gqa_L1m": {"bytes": 201354752 + 5691904, "src": "f35c72a117ea"},
 }
 
 

@@ -568,7 +568,11 @@ __global__ void __launch_bounds__(TAU_NT, D == 64 ? 4 : 3) tau_pv_kernel(const _
             float s0 = 0.f, s1 = 0.f;  // sum x^r, sum x^(r-1) over x = z - t > 0
             auto add = [&](float z) {
                 const float x = z - t;
-                if (x > 0.f) {
+                if (ri == 2) {  // alpha = 3/2: branch-free
+                    const float y = fmaxf(x, 0.f);
+                    s0 = fmaf(y, y, s0);
+                    s1 += y;
+                } else if (x > 0.f) {
                     const float y = ri == 1 ? 1.f : pos_pow(x, r - 1.f, rim1);
                     s0 = fmaf(x, y, s0);
                     s1 += y;

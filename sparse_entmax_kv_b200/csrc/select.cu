@@ -461,16 +461,31 @@ __global__ void __cluster_dims__(GCL, 1, 1) __launch_bounds__(GTH) gauss_cluster
         }
         return;
     }
-    const int Q = ceil_div(n, GCL);
+    const int Q = ceil_div(ceil_div(n, GCL), GIT) * GIT;  // whole GIT-page runs per thread
     const int lo_p = min(n, (int)rank * Q), hi_p = min(n, (int)(rank + 1) * Q);
     const int p0 = lo_p + threadIdx.x * GIT;
     float ub[GIT], mm[GIT], ss[GIT];
+    const bool al16 = ((reinterpret_cast<uintptr_t>(a.bbox) | reinterpret_cast<uintptr_t>(a.mu) |
+                        reinterpret_cast<uintptr_t>(a.sigma)) & 15) == 0;
+    if (al16 && (row & 3) == 0 && p0 + GIT <= hi_p) {
+        // a full run on a 16-byte boundary: 128-bit loads, all issued together
 #pragma unroll
-    for (int i = 0; i < GIT; ++i) {
-        const bool v = p0 + i < hi_p;
-        ub[i] = v ? __ldg(a.bbox + row + p0 + i) : 0.f;
-        mm[i] = v ? a1 * __ldg(a.mu + row + p0 + i) : -INFINITY;
-        ss[i] = v ? a1 * __ldg(a.sigma + row + p0 + i) : 0.f;
+        for (int i = 0; i < GIT; i += 4) {
+            const float4 u = __ldg(reinterpret_cast<const float4 *>(a.bbox + row + p0 + i));
+            const float4 m = __ldg(reinterpret_cast<const float4 *>(a.mu + row + p0 + i));
+            const float4 v = __ldg(reinterpret_cast<const float4 *>(a.sigma + row + p0 + i));
+            ub[i] = u.x; ub[i + 1] = u.y; ub[i + 2] = u.z; ub[i + 3] = u.w;
+            mm[i] = a1 * m.x; mm[i + 1] = a1 * m.y; mm[i + 2] = a1 * m.z; mm[i + 3] = a1 * m.w;
+            ss[i] = a1 * v.x; ss[i + 1] = a1 * v.y; ss[i + 2] = a1 * v.z; ss[i + 3] = a1 * v.w;
+        }
+    } else {
+#pragma unroll
+        for (int i = 0; i < GIT; ++i) {
+            const bool v = p0 + i < hi_p;
+            ub[i] = v ? __ldg(a.bbox + row + p0 + i) : 0.f;
+            mm[i] = v ? a1 * __ldg(a.mu + row + p0 + i) : -INFINITY;
+            ss[i] = v ? a1 * __ldg(a.sigma + row + p0 + i) : 0.f;
+        }
     }
     // (1) bracket: tau_hat >= max_p (m_p - n_p^(-1/R)) (Jensen); F < 1 at
     // max_p (m_p + 10 s_p)
