@@ -72,6 +72,14 @@ typedef struct entmaxkv_shape {
     int32_t page_size;  /* P, tokens per page */
     int32_t max_pages;  /* row length of page_table (pages per sequence at most) */
     int32_t num_blocks; /* physical blocks held by k_cache / v_cache */
+    /* kv-head range a call works on: kv heads [kv_begin, kv_begin + n) of
+     * every sequence, and their query heads, with n = kv_count, or
+     * Hkv - kv_begin when kv_count is 0 (a zero-filled struct means all
+     * heads).  Every buffer keeps its full-size layout; entries of heads
+     * outside the range are neither read nor written, so calls on disjoint
+     * ranges may run concurrently, and may share one workspace. */
+    int32_t kv_begin;
+    int32_t kv_count;
 } entmaxkv_shape;
 
 enum {
@@ -145,7 +153,7 @@ ENTMAXKV_API size_t entmaxkv_meta_bytes(const entmaxkv_shape *shape);
  * invalid shape or call.  The caller allocates it (any device memory, 256-byte
  * aligned) and passes it with its size; contents need not be initialised and
  * are scratch after the call.  Calls that may overlap on the GPU need separate
- * workspaces.
+ * workspaces, unless their kv-head ranges are disjoint.
  */
 ENTMAXKV_API size_t entmaxkv_workspace_size(const entmaxkv_shape *shape, int call);
 

@@ -119,7 +119,15 @@ int check_shape(const entmaxkv_shape *s) {
     if ((long long)s->max_pages * s->page_size >= (1ll << 31)) return ENTMAXKV_ERR_SHAPE;
     if ((long long)s->num_blocks * s->Hkv * s->page_size >= (1ll << 31)) return ENTMAXKV_ERR_SHAPE;
     if (s->B > 65535 || s->Hq > 65535 || (long long)s->B * s->Hq >= (1ll << 31)) return ENTMAXKV_ERR_SHAPE;
+    if (s->kv_begin < 0 || s->kv_begin >= s->Hkv || s->kv_count < 0 || s->kv_begin + s->kv_count > s->Hkv)
+        return ENTMAXKV_ERR_SHAPE;
     return ENTMAXKV_OK;
+}
+
+// The call's kv-head range [kv0, kv0 + nk) (check_shape has accepted s).
+void kv_range(const entmaxkv_shape *s, int *kv0, int *nk) {
+    *kv0 = s->kv_begin;
+    *nk = s->kv_count ? s->kv_count : s->Hkv - s->kv_begin;
 }
 
 // 1/(alpha-1) when it is an integer in 1..8, else 0.
@@ -213,6 +221,7 @@ int entmaxkv_build_meta(const entmaxkv_shape *s, const void *k_cache, const int3
     a.num_blocks = s->num_blocks;
     a.first_page = first_page;
     a.n_pages = n;
+    kv_range(s, &a.kv0, &a.nk);
     a.status = di.status;
     return cuda_rc(launch_build_meta(a, static_cast<cudaStream_t>(stream)));
 }
@@ -237,6 +246,7 @@ int entmaxkv_append(const entmaxkv_shape *s, const void *k_new, const void *v_ne
     a.m.P = s->page_size;
     a.m.max_pages = s->max_pages;
     a.m.num_blocks = s->num_blocks;
+    kv_range(s, &a.m.kv0, &a.m.nk);
     a.m.status = di.status;
     a.k_cache = static_cast<uint16_t *>(k_cache);
     a.v_cache = static_cast<uint16_t *>(v_cache);
@@ -270,6 +280,7 @@ int entmaxkv_score_pages(const entmaxkv_shape *s, const void *q, const void *met
     a.d = s->d;
     a.P = s->page_size;
     a.max_pages = s->max_pages;
+    kv_range(s, &a.kv0, &a.nk);
     a.status = di.status;
     return cuda_rc(launch_score_pages(a, static_cast<cudaStream_t>(stream)));
 }
@@ -312,6 +323,13 @@ int entmaxkv_select(const entmaxkv_shape *s, const int32_t *seq_lens, const floa
     a.k = k;
     a.alpha = alpha;
     a.delta = delta;
+    {
+        int kv0, nk;
+        kv_range(s, &kv0, &nk);
+        const int G = s->Hq / s->Hkv;
+        a.h0 = kv0 * G;
+        a.nh = nk * G;
+    }
     a.status = di.status;
     return cuda_rc(launch_select(a, static_cast<cudaStream_t>(stream)));
 }
@@ -350,6 +368,7 @@ static int fill_decode(bool dense, const entmaxkv_shape *s, const void *q, const
     a->alpha = alpha;
     a->r_int = alpha > 1.f ? integer_r(alpha) : 0;
     a->sms = di.sms;
+    kv_range(s, &a->kv0, &a->nk);
     a->status = di.status;
     return ENTMAXKV_OK;
 }

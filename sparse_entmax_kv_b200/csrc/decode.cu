@@ -46,8 +46,9 @@ __global__ void __launch_bounds__(UTH) union_kernel(DecodeArgs a) {
     __shared__ unsigned words[UCH / 4];
     __shared__ int sh[72];
     __shared__ int cnts[8], offs[9];
-    const int bk = blockIdx.x;
-    const int b = bk / a.Hkv, kvh = bk % a.Hkv;
+    int b, kvh;
+    group_of(blockIdx.x, a.kv0, a.nk, b, kvh);
+    const int bk = b * a.Hkv + kvh;
     const int G = a.Hq / a.Hkv;
     const int np = n_pages_of(a.seq_lens[b], a.P);
     if (threadIdx.x < G) {
@@ -130,8 +131,16 @@ __global__ void __launch_bounds__(UTH) union_kernel(DecodeArgs a) {
 __global__ void dense_init_kernel(DecodeArgs a) {
     pdl_wait();
     const int i = blockIdx.x * blockDim.x + threadIdx.x;
-    if (i < a.B * a.Hq) a.ws.zmax[i] = ORD_NEG_INF;
-    if (i < a.B * a.Hkv) a.ws.counters[i] = 0;
+    const int G = a.Hq / a.Hkv;
+    int b, x;
+    if (i < a.B * a.nk * G) {
+        head_of(i, a.kv0 * G, a.nk * G, b, x);
+        a.ws.zmax[b * a.Hq + x] = ORD_NEG_INF;
+    }
+    if (i < a.B * a.nk) {
+        group_of(i, a.kv0, a.nk, b, x);
+        a.ws.counters[b * a.Hkv + x] = 0;
+    }
 }
 
 // ------------------------------------------------------ page producer
@@ -236,8 +245,9 @@ __global__ void __launch_bounds__(DEC_THREADS) qk_kernel(const __grid_constant__
     RingView<D, G, NS, 1> R(smem_raw);
     __shared__ float qs[G == 1 ? D : 1];
 
-    const int bk = blockIdx.y;
-    const int b = bk / a.Hkv, kvh = bk % a.Hkv;
+    int b, kvh;
+    group_of(blockIdx.y, a.kv0, a.nk, b, kvh);
+    const int bk = b * a.Hkv + kvh;
     const int P = a.P, PPS = TPS / P;
     const int seq = a.seq_lens[b];
     const int np = n_pages_of(seq, P);
@@ -426,9 +436,10 @@ __global__ void __launch_bounds__(TAU_NT, D == 64 ? 4 : 3) tau_pv_kernel(const _
     double(*accs)[D] = reinterpret_cast<double(*)[D]>(tsm);
     __shared__ int wcnt[72];  // block scan scratch
     __shared__ float red[2][TAU_NW][2];  // double-buffered pass sums
-    const int bh = blockIdx.x;
-    const int b = bh / a.Hq, h = bh % a.Hq;
-    const int G = a.Hq / a.Hkv, kvh = h / G;
+    const int G = a.Hq / a.Hkv;
+    int b, h;
+    head_of(blockIdx.x, a.kv0 * G, a.nk * G, b, h);
+    const int bh = b * a.Hq + h, kvh = h / G;
     const int bk = b * a.Hkv + kvh;
     const int P = a.P;
     const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
@@ -768,8 +779,9 @@ __global__ void __launch_bounds__(DEC_THREADS) pv_stream_kernel(const __grid_con
     float *zst = reinterpret_cast<float *>(smem_raw + ((RG::BYTES + 127) & ~(size_t)127));
     __shared__ float red[NWC][G][D];
 
-    const int bk = blockIdx.y;
-    const int b = bk / a.Hkv, kvh = bk % a.Hkv;
+    int b, kvh;
+    group_of(blockIdx.y, a.kv0, a.nk, b, kvh);
+    const int bk = b * a.Hkv + kvh;
     const int P = a.P, PPS = TPS / P;
     const int seq = a.seq_lens[b];
     const int np = n_pages_of(seq, P);
@@ -875,8 +887,9 @@ __global__ void __launch_bounds__(DEC_THREADS) softmax_kernel(const __grid_const
     __shared__ float red[NWC][G][D];
     __shared__ float redm[NWC][G], redl[NWC][G];
 
-    const int bk = blockIdx.y;
-    const int b = bk / a.Hkv, kvh = bk % a.Hkv;
+    int b, kvh;
+    group_of(blockIdx.y, a.kv0, a.nk, b, kvh);
+    const int bk = b * a.Hkv + kvh;
     const int P = a.P, PPS = TPS / P;
     const int seq = a.seq_lens[b];
     const int np = n_pages_of(seq, P);
@@ -1065,7 +1078,7 @@ cudaError_t launch_qk(const DecodeArgs &a, cudaStream_t st) {
     auto k = qk_kernel<D, G, DENSE>;
     cudaError_t e = set_smem(k, RG::BYTES);
     if (e != cudaSuccess) return e;
-    const int groups = a.B * a.Hkv;
+    const int groups = a.B * a.nk;
     const int S = pick_splits(a.sms, 3, groups, ceil_div(a.max_pages, RG::TPS / a.P), 1 << 16);
     return launch_pdl(k, dim3(S, groups), dim3(DEC_THREADS), RG::BYTES, st, a);
 }
@@ -1073,7 +1086,7 @@ cudaError_t launch_qk(const DecodeArgs &a, cudaStream_t st) {
 template <int D, int G>
 cudaError_t sparse_t(const DecodeArgs &a, cudaStream_t st) {
     cudaError_t e;
-    const int groups = a.B * a.Hkv;
+    const int groups = a.B * a.nk;
     if ((e = launch_pdl(union_kernel, dim3(groups), dim3(UTH), 0, st, a)) != cudaSuccess) return e;
     if (a.alpha == 1.f) {
         // softmax over the selected pages: K and V of the union, split over pages
@@ -1084,21 +1097,23 @@ cudaError_t sparse_t(const DecodeArgs &a, cudaStream_t st) {
         return launch_pdl(k, dim3(S, groups), dim3(DEC_THREADS), RG::BYTES, st, a);
     }
     if ((e = launch_qk<D, G, false>(a, st)) != cudaSuccess) return e;
-    const int zcap = tau_zcap(a.B * a.Hq, a.sms);
+    const int nheads = a.B * a.nk * (a.Hq / a.Hkv);
+    const int zcap = tau_zcap(nheads, a.sms);
     if ((e = set_smem(tau_pv_kernel<D, true>, tau_smem(ZCAP_MAX))) != cudaSuccess) return e;
-    return launch_pdl(tau_pv_kernel<D, true>, dim3(a.B * a.Hq), dim3(TAU_NT), tau_smem(zcap), st, a, 0, zcap);
+    return launch_pdl(tau_pv_kernel<D, true>, dim3(nheads), dim3(TAU_NT), tau_smem(zcap), st, a, 0, zcap);
 }
 
 template <int D, int G>
 cudaError_t dense_entmax_t(const DecodeArgs &a, cudaStream_t st) {
     cudaError_t e;
-    const int groups = a.B * a.Hkv;
-    const int n = a.B * a.Hq > groups ? a.B * a.Hq : groups;
+    const int groups = a.B * a.nk;
+    const int n = a.B * a.nk * (a.Hq / a.Hkv);
     if ((e = launch_pdl(dense_init_kernel, dim3(ceil_div(n, 256)), dim3(256), 0, st, a)) != cudaSuccess) return e;
     if ((e = launch_qk<D, G, true>(a, st)) != cudaSuccess) return e;
-    const int zcap = tau_zcap(a.B * a.Hq, a.sms);
+    const int nheads = a.B * a.nk * (a.Hq / a.Hkv);
+    const int zcap = tau_zcap(nheads, a.sms);
     if ((e = set_smem(tau_pv_kernel<D, false>, tau_smem(ZCAP_MAX))) != cudaSuccess) return e;
-    if ((e = launch_pdl(tau_pv_kernel<D, false>, dim3(a.B * a.Hq), dim3(TAU_NT), tau_smem(zcap), st, a, 1, zcap)) !=
+    if ((e = launch_pdl(tau_pv_kernel<D, false>, dim3(nheads), dim3(TAU_NT), tau_smem(zcap), st, a, 1, zcap)) !=
         cudaSuccess)
         return e;
     auto k = pv_stream_kernel<D, G>;
@@ -1111,8 +1126,8 @@ cudaError_t dense_entmax_t(const DecodeArgs &a, cudaStream_t st) {
 template <int D, int G>
 cudaError_t dense_softmax_t(const DecodeArgs &a, cudaStream_t st) {
     cudaError_t e;
-    const int groups = a.B * a.Hkv;
-    const int n = a.B * a.Hq > groups ? a.B * a.Hq : groups;
+    const int groups = a.B * a.nk;
+    const int n = a.B * a.nk * (a.Hq / a.Hkv);
     if ((e = launch_pdl(dense_init_kernel, dim3(ceil_div(n, 256)), dim3(256), 0, st, a)) != cudaSuccess) return e;
     using RG = Ring<D, G, 3, 2>;
     auto k = softmax_kernel<D, G, false>;

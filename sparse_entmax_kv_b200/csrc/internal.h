@@ -17,6 +17,17 @@ struct DevInfo {
     int *status;  // device address of the status word
 };
 
+// Grid index -> (sequence, kv head) of a kv-head range [kv0, kv0 + nk), and
+// -> (sequence, query head) of a query-head range [h0, h0 + nh).
+__host__ __device__ inline void group_of(int idx, int kv0, int nk, int &b, int &kvh) {
+    b = idx / nk;
+    kvh = kv0 + idx % nk;
+}
+__host__ __device__ inline void head_of(int idx, int h0, int nh, int &b, int &h) {
+    b = idx / nh;
+    h = h0 + idx % nh;
+}
+
 // Pages per metadata tile and the tile count of one (sequence, kv head).
 constexpr int META_TILE = 32;
 inline int meta_tiles(int max_pages) { return (max_pages + META_TILE - 1) / META_TILE; }
@@ -30,6 +41,7 @@ struct MetaArgs {
     long long n_tiles_total;  // B * Hkv * n_tiles
     int B, Hkv, d, P, max_pages, num_blocks;
     int first_page, n_pages;  // n_pages >= 0 here (resolved by the caller)
+    int kv0, nk;              // kv-head range [kv0, kv0 + nk)
     int *status;
 };
 cudaError_t launch_build_meta(const MetaArgs &a, cudaStream_t st);
@@ -52,6 +64,7 @@ struct ScoreArgs {
     int n_tiles;
     long long n_tiles_total;
     int B, Hq, Hkv, d, P, max_pages;
+    int kv0, nk;  // kv-head range [kv0, kv0 + nk)
     int *status;
 };
 cudaError_t launch_score_pages(const ScoreArgs &a, cudaStream_t st);
@@ -65,6 +78,7 @@ struct SelectArgs {
     int policy, k;
     float alpha, delta;
     int r_int;  // 1/(alpha-1) for the Gaussian policy
+    int h0, nh;  // query-head range [h0, h0 + nh)
     int *status;
 };
 cudaError_t launch_select(const SelectArgs &a, cudaStream_t st);
@@ -94,6 +108,7 @@ struct DecodeArgs {
     float alpha;
     int r_int;  // 1/(alpha-1) if an integer 1..8, else 0
     int sms;
+    int kv0, nk;  // kv-head range [kv0, kv0 + nk); query heads [kv0 G, (kv0 + nk) G)
     int *status;
 };
 cudaError_t launch_decode_sparse(const DecodeArgs &a, cudaStream_t st);

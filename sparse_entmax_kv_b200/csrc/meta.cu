@@ -68,7 +68,7 @@ template <int D, int P>
 __global__ void __launch_bounds__(D) build_meta_kernel(MetaArgs a) {
     pdl_wait();
     const int b = blockIdx.y;
-    const int kvh = blockIdx.z;
+    const int kvh = a.kv0 + blockIdx.z;
     const int p = a.first_page + blockIdx.x;
     const int seq = a.seq_lens[b];
     if (p >= n_pages_of(seq, P)) return;
@@ -86,7 +86,7 @@ __global__ void __launch_bounds__(D) build_meta_kernel(MetaArgs a) {
 template <int D, int P>
 __global__ void __launch_bounds__(D) append_kernel(AppendArgs a) {
     pdl_wait();
-    const int b = blockIdx.x, kvh = blockIdx.y;
+    const int b = blockIdx.x, kvh = a.m.kv0 + blockIdx.y;
     const int seq = a.m.seq_lens[b];
     if (seq <= 0) return;
     const int p = (seq - 1) / P, t = (seq - 1) % P;
@@ -110,7 +110,7 @@ __global__ void __launch_bounds__(D) append_kernel(AppendArgs a) {
 
 template <int D>
 cudaError_t launch_d(const MetaArgs &a, cudaStream_t st) {
-    dim3 grid(a.n_pages, a.B, a.Hkv);
+    dim3 grid(a.n_pages, a.B, a.nk);
     cudaError_t e = cudaSuccess;
     switch (a.P) {
         case 16: e = launch_pdl(build_meta_kernel<D, 16>, dim3(grid), dim3(D), 0, st, a); break;
@@ -123,7 +123,7 @@ cudaError_t launch_d(const MetaArgs &a, cudaStream_t st) {
 
 template <int D>
 cudaError_t launch_append_d(const AppendArgs &a, cudaStream_t st) {
-    dim3 grid(a.m.B, a.m.Hkv);
+    dim3 grid(a.m.B, a.m.nk);
     switch (a.m.P) {
         case 16: return launch_pdl(append_kernel<D, 16>, dim3(grid), dim3(D), 0, st, a);
         case 32: return launch_pdl(append_kernel<D, 32>, dim3(grid), dim3(D), 0, st, a);

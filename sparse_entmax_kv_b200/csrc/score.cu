@@ -66,8 +66,8 @@ __global__ void __launch_bounds__(THREADS, G <= 4 ? 2 : 1) score_kernel(ScoreArg
     uint64_t *bars = reinterpret_cast<uint64_t *>(smem + QBytes<D, G>::VALUE);
     unsigned char *ring = smem + ((QBytes<D, G>::VALUE + WARPS * NST * 8 + 127) & ~127);
 
-    const int bk = blockIdx.y;
-    const int b = bk / a.Hkv, kvh = bk % a.Hkv;
+    int b, kvh;
+    group_of(blockIdx.y, a.kv0, a.nk, b, kvh);
     const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
 
     for (int i = threadIdx.x; i < G * D; i += THREADS) {
@@ -180,7 +180,7 @@ cudaError_t launch_t(const ScoreArgs &a, cudaStream_t st) {
     auto kern = score_kernel<D, G, GAUSS>;
     cudaError_t e = ensure_smem(reinterpret_cast<const void *>(kern), smem);
     if (e != cudaSuccess) return e;
-    dim3 grid(ceil_div(a.n_tiles, WARPS), a.B * a.Hkv);
+    dim3 grid(ceil_div(a.n_tiles, WARPS), a.B * a.nk);
     return launch_pdl(kern, dim3(grid), dim3(THREADS), smem, st, a);
 }
 

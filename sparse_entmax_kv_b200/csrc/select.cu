@@ -50,8 +50,9 @@ __global__ void __launch_bounds__(NT) topk_kernel(SelectArgs a) {
     __shared__ int hist[256];
     __shared__ int sh[72];
     __shared__ int pick[2];
-    const int bh = blockIdx.x;
-    const int b = bh / a.Hq;
+    int b, h;
+    head_of(blockIdx.x, a.h0, a.nh, b, h);
+    const int bh = b * a.Hq + h;
     const int n = n_pages_of(a.seq_lens[b], a.P);
     const float *sc = a.bbox + (size_t)bh * a.max_pages;
     int *sel = a.sel + (size_t)bh * a.max_pages;
@@ -250,8 +251,9 @@ __global__ void __launch_bounds__(SEL_THREADS) gauss_kernel(SelectArgs a) {
     __shared__ float shm[32], shm2[32];
     __shared__ int shi[72];
     __shared__ int ncand;
-    const int bh = blockIdx.x;
-    const int b = bh / a.Hq;
+    int b, h;
+    head_of(blockIdx.x, a.h0, a.nh, b, h);
+    const int bh = b * a.Hq + h;
     const int seq = a.seq_lens[b];
     const int n = n_pages_of(seq, a.P);
     const size_t row = (size_t)bh * a.max_pages;
@@ -447,8 +449,9 @@ __global__ void __cluster_dims__(GCL, 1, 1) __launch_bounds__(GTH) gauss_cluster
     __shared__ float wa[GTH / 32], wb[GTH / 32];
     __shared__ int sh[72];
     const unsigned rank = cl_rank();
-    const int bh = blockIdx.x / GCL;
-    const int b = bh / a.Hq;
+    int b, h;
+    head_of(blockIdx.x / GCL, a.h0, a.nh, b, h);
+    const int bh = b * a.Hq + h;
     const int seq = a.seq_lens[b];
     const int n = n_pages_of(seq, a.P);
     const size_t row = (size_t)bh * a.max_pages;
@@ -664,7 +667,7 @@ __global__ void __cluster_dims__(GCL, 1, 1) __launch_bounds__(GTH) gauss_cluster
 }  // namespace
 
 cudaError_t launch_select(const SelectArgs &a, cudaStream_t st) {
-    const int grid = a.B * a.Hq;
+    const int grid = a.B * a.nh;
     cudaError_t e = cudaSuccess;
     if (a.policy == ENTMAXKV_TOPK) {
         // short sequences: a quarter of the threads holds every page in registers

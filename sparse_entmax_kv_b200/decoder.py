@@ -22,7 +22,7 @@ from . import native as nv
 
 class EntmaxKVDecoder:
     def __init__(self, k_cache, v_cache, page_table, seq_lens, Hq, *, alpha=1.5, policy="topk",
-                 k=64, delta=0.5):
+                 k=64, delta=0.5, kv_splits=1):
         dev = k_cache.device
         nb, Hkv, P, d = k_cache.shape
         B, max_pages = page_table.shape
@@ -44,6 +44,16 @@ class EntmaxKVDecoder:
         self.out = torch.empty((B, Hq, d), **f32)
         self.ws = nv.alloc_workspace(self.shape, nv.CALL_DECODE_SPARSE, dev)
         self.launches_per_step = 0
+        # kv-head ranges, each stepped on its own stream (disjoint heads: the
+        # buffers and the workspace are shared); a range's scoring waits for
+        # the previous range's, so its selection and decode overlap the next
+        # range's metadata scan
+        n = max(1, min(int(kv_splits), Hkv))
+        cut = [(i * Hkv) // n for i in range(n + 1)]
+        self.ranges = [(cut[i], cut[i + 1] - cut[i]) for i in range(n) if cut[i + 1] > cut[i]]
+        self.shapes = [self.shape.kv_range(k0, nk) for k0, nk in self.ranges] if n > 1 else [self.shape]
+        self.streams = [torch.cuda.Stream(device=dev) for _ in self.shapes] if n > 1 else None
+        self.scored = [torch.cuda.Event() for _ in self.shapes] if n > 1 else None
 
     def build_meta(self, first_page=0, n_pages=-1):
         nv.entmaxkv_build_meta(self.shape, self.k_cache, self.page_table, self.seq_lens,
@@ -55,20 +65,37 @@ class EntmaxKVDecoder:
         gained, at position seq_lens-1, written into the cache together with
         its page's metadata; or ``append_page``: a logical page whose metadata
         is refreshed (the caller wrote the token already); or neither."""
+        if self.streams is None:
+            self._step_range(self.shape, q, append_page, p_out, new_kv, None, None)
+            return self.out
+        cur = torch.cuda.current_stream()
+        prev = None
+        for shape, st, ev in zip(self.shapes, self.streams, self.scored):
+            st.wait_stream(cur)
+            with torch.cuda.stream(st):
+                self._step_range(shape, q, append_page, p_out, new_kv, prev, ev)
+            prev = ev
+        for st in self.streams:
+            cur.wait_stream(st)
+        return self.out
+
+    def _step_range(self, shape, q, append_page, p_out, new_kv, after, scored):
         if new_kv is not None:
-            nv.entmaxkv_append(self.shape, new_kv[0], new_kv[1], self.page_table, self.seq_lens,
+            nv.entmaxkv_append(shape, new_kv[0], new_kv[1], self.page_table, self.seq_lens,
                                self.k_cache, self.v_cache, self.meta)
         elif append_page is not None:
-            nv.entmaxkv_build_meta(self.shape, self.k_cache, self.page_table, self.seq_lens,
+            nv.entmaxkv_build_meta(shape, self.k_cache, self.page_table, self.seq_lens,
                                    append_page, 1, self.meta)
-        nv.entmaxkv_score_pages(self.shape, q, self.meta, self.seq_lens,
-                                self.bbox, self.mu, self.sigma)
-        nv.entmaxkv_select(self.shape, self.seq_lens, self.bbox, self.mu, self.sigma, self.policy,
+        if after is not None:
+            torch.cuda.current_stream().wait_event(after)
+        nv.entmaxkv_score_pages(shape, q, self.meta, self.seq_lens, self.bbox, self.mu, self.sigma)
+        if scored is not None:  # the next range's scan follows this one
+            scored.record(torch.cuda.current_stream())
+        nv.entmaxkv_select(shape, self.seq_lens, self.bbox, self.mu, self.sigma, self.policy,
                            self.k, self.alpha, self.delta, self.sel, self.cnt, self.tau_hat)
-        nv.entmaxkv_decode_sparse(self.shape, q, self.k_cache, self.v_cache, self.page_table,
+        nv.entmaxkv_decode_sparse(shape, q, self.k_cache, self.v_cache, self.page_table,
                                   self.seq_lens, self.sel, self.cnt, self.alpha, self.out,
                                   self.tau, p_out, self.ws)
-        return self.out
 
 
 def last_token_rows(k_cache, v_cache, page_table, seq_lens):

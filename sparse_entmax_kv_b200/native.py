@@ -38,8 +38,17 @@ class EntmaxKVError(RuntimeError):
 
 
 class Shape(C.Structure):
+    """entmaxkv_shape; kv_begin / kv_count restrict a call to a kv-head range
+    (both 0: every head)."""
     _fields_ = [("B", C.c_int32), ("Hq", C.c_int32), ("Hkv", C.c_int32), ("d", C.c_int32),
-                ("page_size", C.c_int32), ("max_pages", C.c_int32), ("num_blocks", C.c_int32)]
+                ("page_size", C.c_int32), ("max_pages", C.c_int32), ("num_blocks", C.c_int32),
+                ("kv_begin", C.c_int32), ("kv_count", C.c_int32)]
+
+    def kv_range(self, kv_begin: int, kv_count: int) -> "Shape":
+        """A copy restricted to kv heads [kv_begin, kv_begin + kv_count)."""
+        t = Shape(*self.astuple())
+        t.kv_begin, t.kv_count = int(kv_begin), int(kv_count)
+        return t
 
     @classmethod
     def of(cls, q: torch.Tensor, k_cache: torch.Tensor, page_table: torch.Tensor) -> "Shape":

@@ -38,7 +38,7 @@ def test_strerror_and_version():
 
 
 def shp(**kw):
-    d = dict(B=2, Hq=8, Hkv=2, d=128, page_size=32, max_pages=64, num_blocks=128)
+    d = dict(B=2, Hq=8, Hkv=2, d=128, page_size=32, max_pages=64, num_blocks=128, kv_begin=0, kv_count=0)
     d.update(kw)
     return nv.Shape(*[d[f] for f, _ in nv.Shape._fields_])
 
@@ -59,7 +59,8 @@ def test_sizes():
 
 @pytest.mark.parametrize("bad", [dict(d=96), dict(page_size=8), dict(Hq=6, Hkv=4), dict(Hq=24, Hkv=2),
                                  dict(B=0), dict(max_pages=0), dict(num_blocks=0),
-                                 dict(max_pages=1 << 26, page_size=64)])
+                                 dict(max_pages=1 << 26, page_size=64), dict(kv_begin=2), dict(kv_begin=-1),
+                                 dict(kv_count=3), dict(kv_begin=1, kv_count=2), dict(kv_count=-1)])
 def test_bad_shapes_rejected_everywhere(bad):
     L = nv.lib()
     s = C.byref(shp(**bad))

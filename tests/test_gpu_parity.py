@@ -20,7 +20,7 @@ import torch
 
 import oracle as orc
 from sparse_entmax_kv_b200 import native as nv
-from sparse_entmax_kv_b200.decoder import EntmaxKVDecoder
+from sparse_entmax_kv_b200.decoder import EntmaxKVDecoder, last_token_rows
 from sparse_entmax_kv_b200.workloads import CONFIGS, Workload, make_inputs, to_host_u16
 
 pytestmark = pytest.mark.gpu
@@ -492,6 +492,46 @@ def test_append_bad_page_sets_status_and_skips():
     assert nv.get_status(clear=True) & nv.STATUS_BAD_PAGE
     assert torch.equal(inp["k_cache"].view(torch.int16), k_ref.view(torch.int16))
     assert torch.equal(inp["v_cache"].view(torch.int16), v_ref.view(torch.int16))
+
+
+@pytest.mark.parametrize("name", ["gauss_small", "topk_small", "mha_small"])
+@pytest.mark.parametrize("splits", [2, 4])
+def test_kv_head_ranges_match_one_call(name, splits):
+    """A step issued per kv-head range (entmaxkv_shape.kv_begin / kv_count, one
+    stream each, shared buffers) writes exactly what one whole-shape step
+    writes, and nothing for heads outside a range."""
+    wl = SMALL[name]
+    inp, _ = gpu_inputs(wl, 21)
+    new_kv = last_token_rows(inp["k_cache"], inp["v_cache"], inp["page_table"], inp["seq_lens"])
+    outs = []
+    for ks in (1, splits):
+        dec = EntmaxKVDecoder(inp["k_cache"], inp["v_cache"], inp["page_table"], inp["seq_lens"], wl.Hq,
+                              alpha=wl.alpha, policy=wl.policy, k=wl.k or 64, delta=wl.delta or 0.5, kv_splits=ks)
+        dec.build_meta()
+        dec.out.fill_(float("nan"))
+        dec.step(inp["q"], new_kv=new_kv)
+        torch.cuda.synchronize()
+        outs.append((dec.out.clone(), dec.sel.clone(), dec.cnt.clone(), dec.bbox.clone()))
+    (o1, s1, c1, b1), (o2, s2, c2, b2) = outs
+    assert torch.equal(o1.view(torch.int32), o2.view(torch.int32))
+    assert torch.equal(c1, c2)
+    for b in range(wl.B):
+        for h in range(wl.Hq):
+            n = int(c1[b, h])
+            assert torch.equal(s1[b, h, :n], s2[b, h, :n])
+    # a single range leaves the other heads' outputs alone
+    s = shape_of(wl).kv_range(0, 1)
+    out = torch.full((wl.B, wl.Hq, wl.max_pages), float("nan"), device="cuda")
+    dec = EntmaxKVDecoder(inp["k_cache"], inp["v_cache"], inp["page_table"], inp["seq_lens"], wl.Hq,
+                          alpha=wl.alpha, policy=wl.policy, k=wl.k or 64, delta=wl.delta or 0.5)
+    dec.build_meta()
+    nv.entmaxkv_score_pages(s, inp["q"], dec.meta, inp["seq_lens"], out)
+    torch.cuda.synchronize()
+    G = wl.Hq // wl.Hkv
+    assert torch.isnan(out[:, G:]).all()
+    for b in range(wl.B):
+        npb = -(-int(inp["seq_lens"][b]) // wl.P)
+        assert torch.equal(out[b, :G, :npb], b1[b, :G, :npb])
 
 
 # ---------------------------------------------------- full-size workloads
