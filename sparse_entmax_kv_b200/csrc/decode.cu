@@ -70,6 +70,8 @@ __global__ void __launch_bounds__(UTH) union_kernel(DecodeArgs a) {
     __syncthreads();
     const int total = offs[G];  // every head's entries as one flat range
     int *ue = a.ws.union_e + (size_t)bk * a.max_pages;
+    int *ub = a.ws.union_blk + (size_t)bk * a.max_pages;
+    const int *pt = a.page_table + (size_t)b * a.max_pages;
     int done = 0;
     for (int lo = 0; lo < np; lo += UCH) {
         const int hi = min(np, lo + UCH);
@@ -101,27 +103,39 @@ __global__ void __launch_bounds__(UTH) union_kernel(DecodeArgs a) {
             }
         }
         __syncthreads();
-        // the chunk's entries in page order: thread t owns words [t*wpt, (t+1)*wpt)
+        // the chunk's entries in page order: thread t owns words [t*wpt, (t+1)*wpt);
+        // the page-table entries of its selected pages are all loaded first
+        constexpr int WPT_MAX = UCH / 4 / UTH;
         const int wpt = ceil_div(nw, UTH);
         const int w0 = threadIdx.x * wpt;
+        unsigned wv[WPT_MAX];
+        int blk[WPT_MAX][4];
         int mine = 0;
-        for (int i = 0; i < wpt; ++i)
-            if (w0 + i < nw) {
-                const unsigned w = words[w0 + i];
 #pragma unroll
-                for (int j = 0; j < 4; ++j) mine += ((w >> (8 * j)) & 0xffu) ? 1 : 0;
-            }
-        int chunk_total;
-        int pos = done + block_excl_scan(mine, sh, &chunk_total);
-        for (int i = 0; i < wpt; ++i) {
-            if (w0 + i >= nw) break;
-            const unsigned w = words[w0 + i];
+        for (int i = 0; i < WPT_MAX; ++i) {
+            wv[i] = i < wpt && w0 + i < nw ? words[w0 + i] : 0u;
 #pragma unroll
             for (int j = 0; j < 4; ++j) {
-                const unsigned m = (w >> (8 * j)) & 0xffu;
-                if (m) ue[pos++] = ((lo + 4 * (w0 + i) + j) << 8) | (int)m;
+                const bool sel = (wv[i] >> (8 * j)) & 0xffu;
+                blk[i][j] = sel ? __ldg(pt + lo + 4 * (w0 + i) + j) : -1;
+                mine += sel ? 1 : 0;
             }
         }
+        int chunk_total;
+        int pos = done + block_excl_scan(mine, sh, &chunk_total);
+#pragma unroll
+        for (int i = 0; i < WPT_MAX; ++i)
+#pragma unroll
+            for (int j = 0; j < 4; ++j) {
+                const unsigned m = (wv[i] >> (8 * j)) & 0xffu;
+                if (m) {
+                    // the entry and its physical block (-1 if the page-table entry is bad)
+                    const bool ok = blk[i][j] >= 0 && blk[i][j] < a.num_blocks;
+                    if (!ok) atomicOr(a.status, ENTMAXKV_STATUS_BAD_PAGE);
+                    ue[pos] = ((lo + 4 * (w0 + i) + j) << 8) | (int)m;
+                    ub[pos++] = ok ? blk[i][j] : -1;
+                }
+            }
         done += chunk_total;
         __syncthreads();  // the bitmap is read before the next chunk clears it
     }
@@ -172,17 +186,19 @@ __device__ void produce(const DecodeArgs &a, const CUtensorMap *m0, const CUtens
             const int e = (blockIdx.x + it * S) * PPS + i;
             PageInfo r{-1, 0, 0, e, -1};
             if (e < U) {
+                // sparse: the union entry and the block the union kernel resolved
+                // for it, loaded together; dense: page e and its page-table entry
                 const int entry = dense ? ((e << 8) | 0xff) : __ldg(a.ws.union_e + (size_t)bk * a.max_pages + e);
+                const int blk = dense ? __ldg(a.page_table + (size_t)b * a.max_pages + e)
+                                      : __ldg(a.ws.union_blk + (size_t)bk * a.max_pages + e);
                 r.page = entry >> 8;
                 r.mask = entry & 0xff;
-                const int blk = __ldg(a.page_table + (size_t)b * a.max_pages + r.page);
                 if (blk >= 0 && blk < a.num_blocks) {
                     r.blk = blk;
                     r.nval = tokens_in_page(seq, a.P, r.page);
-                } else {
+                } else if (dense) {
                     atomicOr(a.status, ENTMAXKV_STATUS_BAD_PAGE);
                 }
-                if (!dense) a.ws.union_blk[(size_t)bk * a.max_pages + e] = r.blk;
             }
             stash[k] = r;
         }
@@ -559,11 +575,11 @@ __global__ void __launch_bounds__(TAU_NT, D == 64 ? 4 : 3) tau_pv_kernel(const _
     const int nloop = onchip ? nc : n_tok;
     auto cz_at = [&](int i) -> float { return onchip ? cz[i] : __ldcg(zr + i); };
 
-    // Newton's method on F(t) = sum_c [z_c - t]_+^r - 1, which is decreasing
-    // on [z_max - 1, z_max - n^(1-alpha)] and convex for r >= 1 (alpha <= 2),
-    // concave for r < 1: started from the end of that bracket where F has the
-    // sign that keeps the iterates on one side of the root, they move to it
-    // monotonically.  Each thread sums [x]_+^r and [x]_+^(r-1) over its
+    // Newton's method on the normalisation, on [z_max - 1, z_max - n^(1-alpha)]
+    // where F(t) = sum_c [z_c - t]_+^r - 1 decreases.  For r >= 1 (alpha <= 2)
+    // on g(t) = (sum_c [z_c - t]_+^r)^(1/r), a norm of (z - t)_+ and so convex,
+    // from the left end; for r < 1 on F, which is then concave, from the right
+    // end.  Either way the iterates move to the root monotonically.  Each thread sums [x]_+^r and [x]_+^(r-1) over its
     // strided share of the candidates, the warps' sums are added in warp
     // order (reproducible), and every warp takes the same step.
     // (on chip nc is the exact candidate count; off chip only a lower bound on
@@ -619,8 +635,15 @@ __global__ void __launch_bounds__(TAU_NT, D == 64 ? 4 : 3) tau_pv_kernel(const _
                 S1 += red[it & 1][ww][1];
             }
             if (!(S1 > 0.f)) break;  // no weight right of t (t at the top already)
-            // t' = t - F(t) / F'(t), F' = -r S1
-            const float tn = fminf(hi, fmaxf(lo, t + (S0 - 1.f) / (r * S1)));
+            // r >= 1: Newton on g = S0^(1/r) = 1 (convex, nearly linear: one step
+            // when the support's z are equal), t' = t + (S0 - S0^(1-1/r)) / S1;
+            // r < 1: Newton on F = S0 - 1 from the right, t' = t + (S0 - 1) / (r S1)
+            float step;
+            if (ri == 2) step = (S0 - sqrtf(S0)) / S1;
+            else if (ri == 1) step = (S0 - 1.f) / S1;
+            else if (r >= 1.f) step = (S0 - powf(S0, 1.f - 1.f / r)) / S1;
+            else step = (S0 - 1.f) / (r * S1);
+            const float tn = fminf(hi, fmaxf(lo, t + step));
             const bool done = !(fabsf(tn - t) > tol);
             t = tn;
             if (done) break;
