@@ -140,7 +140,7 @@ def step_bytes(wl, dec, support_rows):
     value rows with non-zero weight for some head of the group."""
     seq = dec.seq_lens.cpu().numpy()
     npb = -(-seq // wl.P)
-    rec_bytes = (12 if wl.policy == "gauss" else 4) * wl.d
+    rec_bytes = (12 if wl.policy in ("gauss", "gauss_est") else 4) * wl.d
     meta = int(npb.sum()) * wl.Hkv * rec_bytes
     sel, cnt = dec.sel.cpu().numpy(), dec.cnt.cpu().numpy()
     union = 0
@@ -400,7 +400,7 @@ def oracle_step_sample(wl, inp_host, seconds_target=10.0, max_reps=3):
         if time.perf_counter() > t_end:
             break
     npb = -(-h["seq_lens"] // wl.P)
-    meta_b = int(npb.sum()) * wl.Hkv * (12 if policy == "gauss" else 4) * wl.d
+    meta_b = int(npb.sum()) * wl.Hkv * (12 if policy in ("gauss", "gauss_est") else 4) * wl.d
     union = 0
     supp = 0
     for b in range(wl.B):
