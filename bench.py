@@ -47,7 +47,7 @@ PAPER_CONTEXT = {"speedup_vs_full_softmax_flashdecoding": 3.36, "speedup_vs_full
 NCU_TRAFFIC = {
     # one full-size launch at L=1,048,576 (201.35 MB read + 5.69 MB written), ncu --set full
     # (profiles/score_kernel_gauss_gqa_L1m_full.md)
-    "score_pages/gauss_gqa_L1m": {"bytes": 201354752 + 5691904, "src": "f35c72a117ea"},
+    "score_pages/gauss_gqa_L1m": {"bytes": 201360384 + 6459136, "src": "c014ace8a9b9"},
 }
 
 

@@ -301,6 +301,55 @@ ENTMAXKV_API int entmaxkv_decode_sparse_static(const entmaxkv_shape *shape, cons
                                   void *stream);
 
 /*
+ * Sequence-sharded sparse decode: one context split across S devices, each
+ * holding a consecutive range of its logical pages (the summary's section 2.C
+ * computation, done in pieces with three small exchanges).  Shard r holds
+ * global pages [page_begin, page_begin + max_pages) in its own paged cache,
+ * page table and seq_lens (its tokens only); sel/cnt are the GLOBAL selection
+ * (every shard runs entmaxkv_select on the all-gathered page scores, so all
+ * hold the same lists, rows of sel_max_pages global page ids).  Per step:
+ *   1. entmaxkv_decode_sparse_begin       this shard's pages of sel: union,
+ *      z of their tokens (kept in the workspace) and the shard's max z per
+ *      head, zmax_out fp32 [B][Hq] (-inf if the shard has none);
+ *   2. the caller all-reduces zmax with max;
+ *   3. entmaxkv_decode_sparse_candidates  the shard's tokens with
+ *      z > zmax_in - 1 (every token that can carry weight), in list order:
+ *      cand_z fp32 [B][Hq][cap], cand_n int32 [B][Hq] (the exact count; if it
+ *      exceeds cap only cap values are written and ENTMAXKV_STATUS_OVERFLOW is
+ *      set: call again with a larger cap);
+ *   4. the caller all-gathers cand_z / cand_n into [S][B][Hq][cap] / [S][B][Hq]
+ *      (shards in page order);
+ *   5. entmaxkv_entmax_threshold          the exact tau of each head from all
+ *      shards' candidates (the same Newton solve as entmaxkv_decode_sparse, on
+ *      the same list in the same order, so the same tau), tau_out fp32 [B][Hq];
+ *   6. entmaxkv_decode_sparse_finish      out[b][h] = sum over the shard's
+ *      support of p_t v_t (a partial sum: entmax weights are absolute, so the
+ *      shards' partials add up to the output);
+ *   7. the caller all-reduces out with sum.
+ * The workspace carries state from step 1 to step 6 (one workspace per shard
+ * and step in flight).  alpha must be > 1.  n_shards * cap * 4 bytes must fit
+ * in 200 KiB (ENTMAXKV_ERR_SHAPE).  kv-head ranges apply as in every call.
+ */
+ENTMAXKV_API int entmaxkv_decode_sparse_begin(const entmaxkv_shape *shape, const void *q,
+                    const void *k_cache, const void *v_cache, const int32_t *page_table,
+                    const int32_t *seq_lens, const int32_t *sel, const int32_t *cnt,
+                    int32_t sel_max_pages, int32_t page_begin, float alpha,
+                    float *zmax_out, void *workspace, size_t ws_bytes, void *stream);
+ENTMAXKV_API int entmaxkv_decode_sparse_candidates(const entmaxkv_shape *shape, const void *q,
+                    const void *k_cache, const void *v_cache, const int32_t *page_table,
+                    const int32_t *seq_lens, float alpha, const float *zmax_in, int32_t cap,
+                    float *cand_z, int32_t *cand_n, void *workspace, size_t ws_bytes,
+                    void *stream);
+ENTMAXKV_API int entmaxkv_entmax_threshold(const entmaxkv_shape *shape, int32_t n_shards,
+                    int32_t cap, const float *cand_z, const int32_t *cand_n,
+                    const float *zmax_in, float alpha, float *tau_out, void *stream);
+ENTMAXKV_API int entmaxkv_decode_sparse_finish(const entmaxkv_shape *shape, const void *q,
+                    const void *k_cache, const void *v_cache, const int32_t *page_table,
+                    const int32_t *seq_lens, float alpha, const float *zmax_in,
+                    const float *tau_in, float *out, float *p_out, void *workspace,
+                    size_t ws_bytes, void *stream);
+
+/*
  * Section 4 comparison paths, over every token of every sequence:
  *  alpha > 1:  full-cache alpha-entmax (all of K and all of V are read):
  *              out = sum_t p_t v_t; tau_out (nullable) gets tau.

@@ -369,6 +369,7 @@ static int fill_decode(bool dense, const entmaxkv_shape *s, const void *q, const
     a->r_int = alpha > 1.f ? integer_r(alpha) : 0;
     a->sms = di.sms;
     kv_range(s, &a->kv0, &a->nk);
+    a->sel_stride = s->max_pages;  // single-device call: sel rows are this shape's
     a->status = di.status;
     return ENTMAXKV_OK;
 }
@@ -390,6 +391,92 @@ int entmaxkv_decode_sparse(const entmaxkv_shape *s, const void *q, const void *k
     if ((rc = make_kv_map(&a.kmap, k_cache, s))) return rc;
     if (alpha == 1.f && (rc = make_kv_map(&a.vmap, v_cache, s))) return rc;
     return cuda_rc(launch_decode_sparse(a, static_cast<cudaStream_t>(stream)));
+}
+
+int entmaxkv_decode_sparse_begin(const entmaxkv_shape *s, const void *q, const void *k_cache, const void *v_cache,
+                                 const int32_t *page_table, const int32_t *seq_lens, const int32_t *sel,
+                                 const int32_t *cnt, int32_t sel_max_pages, int32_t page_begin, float alpha,
+                                 float *zmax_out, void *workspace, size_t ws_bytes, void *stream) {
+    if (!sel || !cnt || !zmax_out) return ENTMAXKV_ERR_NULL;
+    if (!(alpha > 1.f)) return ENTMAXKV_ERR_ALPHA;
+    // (the last shard's page range may reach past the global page count: its
+    // token count keeps those pages empty)
+    if (s && (s->max_pages > MAX_SEL_PAGES || page_begin < 0 || sel_max_pages < 1 || page_begin >= sel_max_pages))
+        return ENTMAXKV_ERR_SHAPE;
+    DecodeArgs a;
+    int rc = fill_decode(false, s, q, k_cache, v_cache, page_table, seq_lens, alpha, zmax_out, nullptr, nullptr,
+                         workspace, ws_bytes, &a);
+    if (rc) return rc;
+    a.out = nullptr;
+    a.sel = sel;
+    a.cnt = cnt;
+    a.sharded = 1;
+    a.page_begin = page_begin;
+    a.sel_stride = sel_max_pages;
+    a.zmax_out = zmax_out;
+    if ((rc = make_kv_map(&a.kmap, k_cache, s))) return rc;
+    return cuda_rc(launch_decode_sparse_begin(a, static_cast<cudaStream_t>(stream)));
+}
+
+int entmaxkv_decode_sparse_candidates(const entmaxkv_shape *s, const void *q, const void *k_cache,
+                                      const void *v_cache, const int32_t *page_table, const int32_t *seq_lens,
+                                      float alpha, const float *zmax_in, int32_t cap, float *cand_z,
+                                      int32_t *cand_n, void *workspace, size_t ws_bytes, void *stream) {
+    if (!zmax_in || !cand_z || !cand_n) return ENTMAXKV_ERR_NULL;
+    if (!(alpha > 1.f)) return ENTMAXKV_ERR_ALPHA;
+    if (cap < 1) return ENTMAXKV_ERR_SHAPE;
+    DecodeArgs a;
+    int rc = fill_decode(false, s, q, k_cache, v_cache, page_table, seq_lens, alpha, cand_z, nullptr, nullptr,
+                         workspace, ws_bytes, &a);
+    if (rc) return rc;
+    a.out = nullptr;
+    a.zmax_in = zmax_in;
+    a.cand_z = cand_z;
+    a.cand_n = cand_n;
+    a.cap = cap;
+    return cuda_rc(launch_decode_sparse_candidates(a, static_cast<cudaStream_t>(stream)));
+}
+
+int entmaxkv_entmax_threshold(const entmaxkv_shape *s, int32_t n_shards, int32_t cap, const float *cand_z,
+                              const int32_t *cand_n, const float *zmax_in, float alpha, float *tau_out,
+                              void *stream) {
+    int rc = check_shape(s);
+    if (rc) return rc;
+    if (!cand_z || !cand_n || !zmax_in || !tau_out) return ENTMAXKV_ERR_NULL;
+    if (!std::isfinite(alpha) || !(alpha > 1.f)) return ENTMAXKV_ERR_ALPHA;
+    if (n_shards < 1 || cap < 1 || (long long)n_shards * cap * 4 > (200ll << 10)) return ENTMAXKV_ERR_SHAPE;
+    DevInfo di;
+    if ((rc = device_info(&di))) return rc;
+    ThresholdArgs a{};
+    a.cand_z = cand_z;
+    a.cand_n = cand_n;
+    a.zmax = zmax_in;
+    a.tau = tau_out;
+    a.S = n_shards;
+    a.cap = cap;
+    a.B = s->B;
+    a.Hq = s->Hq;
+    a.Hkv = s->Hkv;
+    kv_range(s, &a.kv0, &a.nk);
+    a.alpha = alpha;
+    a.r_int = integer_r(alpha);
+    a.status = di.status;
+    return cuda_rc(launch_entmax_threshold(a, static_cast<cudaStream_t>(stream)));
+}
+
+int entmaxkv_decode_sparse_finish(const entmaxkv_shape *s, const void *q, const void *k_cache, const void *v_cache,
+                                  const int32_t *page_table, const int32_t *seq_lens, float alpha,
+                                  const float *zmax_in, const float *tau_in, float *out, float *p_out,
+                                  void *workspace, size_t ws_bytes, void *stream) {
+    if (!zmax_in || !tau_in) return ENTMAXKV_ERR_NULL;
+    if (!(alpha > 1.f)) return ENTMAXKV_ERR_ALPHA;
+    DecodeArgs a;
+    int rc = fill_decode(false, s, q, k_cache, v_cache, page_table, seq_lens, alpha, out, nullptr, p_out, workspace,
+                         ws_bytes, &a);
+    if (rc) return rc;
+    a.zmax_in = zmax_in;
+    a.tau_in = tau_in;
+    return cuda_rc(launch_decode_sparse_finish(a, static_cast<cudaStream_t>(stream)));
 }
 
 int entmaxkv_decode_dense(const entmaxkv_shape *s, const void *q, const void *k_cache, const void *v_cache,

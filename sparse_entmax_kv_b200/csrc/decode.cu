@@ -54,9 +54,10 @@ __global__ void __launch_bounds__(UTH) union_kernel(DecodeArgs a) {
     if (threadIdx.x < G) {
         const int bh = b * a.Hq + kvh * G + threadIdx.x;
         int c = a.cnt[bh];
-        if (c < 0 || c > np) {
+        const int cmax = a.sharded ? a.sel_stride : np;  // sharded: counts over all shards' pages
+        if (c < 0 || c > cmax) {
             atomicOr(a.status, ENTMAXKV_STATUS_BAD_SELECTION);
-            c = c < 0 ? 0 : np;
+            c = c < 0 ? 0 : cmax;
         }
         cnts[threadIdx.x] = c;
         a.ws.zmax[bh] = ORD_NEG_INF;
@@ -90,7 +91,8 @@ __global__ void __launch_bounds__(UTH) union_kernel(DecodeArgs a) {
                     int gg = 0;
                     while (k >= offs[gg + 1]) ++gg;
                     g[u] = gg;
-                    p[u] = __ldg(a.sel + (size_t)(b * a.Hq + kvh * G + gg) * a.max_pages + (k - offs[gg]));
+                    p[u] = __ldg(a.sel + (size_t)(b * a.Hq + kvh * G + gg) * a.sel_stride + (k - offs[gg])) -
+                           a.page_begin;  // this shard's page index
                 }
             }
 #pragma unroll
@@ -98,8 +100,9 @@ __global__ void __launch_bounds__(UTH) union_kernel(DecodeArgs a) {
                 if (k0 + u * UTH >= total) continue;
                 if (p[u] >= lo && p[u] < hi)
                     atomicOr(&words[(p[u] - lo) >> 2], 1u << ((p[u] & 3) * 8 + g[u]));
-                else if ((p[u] < 0 || p[u] >= np) && lo == 0)
-                    atomicOr(a.status, ENTMAXKV_STATUS_BAD_SELECTION);
+                else if (lo == 0 && (a.sharded ? (p[u] + a.page_begin < 0 || p[u] + a.page_begin >= a.sel_stride)
+                                               : (p[u] < 0 || p[u] >= np)))
+                    atomicOr(a.status, ENTMAXKV_STATUS_BAD_SELECTION);  // (sharded: other shards' pages are skipped)
             }
         }
         __syncthreads();
@@ -436,6 +439,69 @@ inline int tau_zcap(int ctas, int sms) {
     return z;
 }
 
+// The entmax threshold: the root t of sum_c [z_c - t]_+^r = 1 over the
+// candidates (every token with weight has z > z_max - 1), which lies in
+// [lo, hi] = [z_max - 1, z_max - n^(1-alpha)] where F(t) = sum - 1 decreases.
+// Newton's method, for r >= 1 (alpha <= 2) on g(t) = (sum_c [z_c - t]_+^r)^(1/r),
+// a norm of (z - t)_+ and so convex (one step when the support's z are equal),
+// from the left end; for r < 1 on F, which is then concave, from the right
+// end: either way the iterates move to the root monotonically.  for_each(add)
+// calls add(z) on this thread's share of the candidates; each thread's sums
+// are added in warp order (reproducible) and every warp takes the same step,
+// one barrier per pass (red is double-buffered).  All TAU_NT threads call it.
+template <class ForEach>
+__device__ float entmax_tau(ForEach for_each, float lo, float hi, float zmax, float r, int ri,
+                            float (*red)[TAU_NW][2]) {
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+    const float tol = 1e-7f * fmaxf(1.f, fabsf(zmax));
+    const int rim1 = ri >= 2 ? ri - 1 : 0;
+    float t = r >= 1.f ? lo : hi;
+    for (int it = 0; it < 40; ++it) {
+        float s0 = 0.f, s1 = 0.f;  // sum x^r, sum x^(r-1) over x = z - t > 0
+        auto add = [&](float z) {
+            const float x = z - t;
+            if (ri == 2) {  // alpha = 3/2: branch-free
+                const float y = fmaxf(x, 0.f);
+                s0 = fmaf(y, y, s0);
+                s1 += y;
+            } else if (x > 0.f) {
+                const float y = ri == 1 ? 1.f : pos_pow(x, r - 1.f, rim1);
+                s0 = fmaf(x, y, s0);
+                s1 += y;
+            }
+        };
+        for_each(add);
+#pragma unroll
+        for (int o = 16; o; o >>= 1) {
+            s0 += __shfl_xor_sync(FULL, s0, o);
+            s1 += __shfl_xor_sync(FULL, s1, o);
+        }
+        if (lane == 0) {
+            red[it & 1][warp][0] = s0;
+            red[it & 1][warp][1] = s1;
+        }
+        __syncthreads();
+        float S0 = 0.f, S1 = 0.f;
+#pragma unroll
+        for (int ww = 0; ww < TAU_NW; ++ww) {
+            S0 += red[it & 1][ww][0];
+            S1 += red[it & 1][ww][1];
+        }
+        if (!(S1 > 0.f)) break;  // no weight right of t (t at the top already)
+        // r >= 1: t' = t + (S0 - S0^(1-1/r)) / S1;  r < 1: t' = t + (S0 - 1) / (r S1)
+        float step;
+        if (ri == 2) step = (S0 - sqrtf(S0)) / S1;
+        else if (ri == 1) step = (S0 - 1.f) / S1;
+        else if (r >= 1.f) step = (S0 - powf(S0, 1.f - 1.f / r)) / S1;
+        else step = (S0 - 1.f) / (r * S1);
+        const float tn = fminf(hi, fmaxf(lo, t + step));
+        const bool done = !(fabsf(tn - t) > tol);
+        t = tn;
+        if (done) break;
+    }
+    return t;
+}
+
 // Exact threshold and (GATHER) the weighted sum of the support's value rows.
 template <int D, bool GATHER>
 __global__ void __launch_bounds__(TAU_NT, D == 64 ? 4 : 3) tau_pv_kernel(const __grid_constant__ DecodeArgs a, int dense, int zcap) {
@@ -462,19 +528,29 @@ __global__ void __launch_bounds__(TAU_NT, D == 64 ? 4 : 3) tau_pv_kernel(const _
     const int np = n_pages_of(a.seq_lens[b], P);
     const int U = dense ? np : a.ws.union_cnt[bk];
     const int n_tok = U * P;  // a multiple of 16
-    const float zmax = ord2f(a.ws.zmax[bh]);
+    // sequence-sharded phases: the global max z and tau come in; the
+    // candidates phase writes out this shard's candidate z values
+    const float zmax = a.zmax_in ? a.zmax_in[bh] : ord2f(a.ws.zmax[bh]);
+    const bool given_tau = a.tau_in != nullptr;
+    const bool export_cand = a.cand_z != nullptr;
     const float r = 1.f / (a.alpha - 1.f);
     const int ri = a.r_int;
-    if (!(zmax > -INFINITY)) {  // no token at all
+    if (!(zmax > -INFINITY) || (given_tau && !(a.tau_in[bh] == a.tau_in[bh]))) {  // no token at all
+        if (export_cand) {
+            if (threadIdx.x == 0) a.cand_n[bh] = 0;
+            return;
+        }
         if (GATHER)
             for (int j = threadIdx.x; j < D; j += TAU_NT) a.out[(size_t)bh * D + j] = 0.f;
-        if (threadIdx.x == 0) {
+        if (threadIdx.x == 0 && !given_tau) {
             a.ws.tau[bh] = __int_as_float(0x7fc00000);
             if (a.tau_out) a.tau_out[bh] = __int_as_float(0x7fc00000);
         }
         return;
     }
-    const float thr = zmax - 1.f;
+    // tokens that can carry weight: z > z_max - 1 (no weight exceeds 1), or,
+    // with tau known, z > tau
+    const float thr = given_tau ? a.tau_in[bh] : zmax - 1.f;
     const float *zr = a.ws.zbuf + tok_row(a, b, h);
     const size_t trow = tile_row(a, b, h);
     const float *tr = a.ws.tmax + trow;
@@ -571,86 +647,74 @@ __global__ void __launch_bounds__(TAU_NT, D == 64 ? 4 : 3) tau_pv_kernel(const _
     }
     __syncthreads();
     const bool onchip = nc <= zcap;
+    if (export_cand) {
+        // this shard's candidates, in list order, at most cap of them (the
+        // count is exact either way)
+        float *cz_out = a.cand_z + (size_t)bh * a.cap;
+        int total = 0;
+        if (onchip) {
+            for (int i = threadIdx.x; i < min(nc, a.cap); i += TAU_NT) cz_out[i] = cz[i];
+            total = nc;
+        } else {
+            for (int t0 = 0; t0 < n_tok; t0 += TAU_NT * 16) {
+                const int e0 = t0 + threadIdx.x * 16;
+                float zz[16];
+                unsigned bits = 0;
+#pragma unroll
+                for (int k = 0; k < 16; ++k) {
+                    zz[k] = e0 + k < n_tok ? __ldcg(zr + e0 + k) : -INFINITY;
+                    if (zz[k] > thr) bits |= 1u << k;
+                }
+                int tot;
+                int w = total + block_excl_scan(__popc(bits), wcnt, &tot);
+#pragma unroll
+                for (int k = 0; k < 16; ++k)
+                    if ((bits >> k) & 1u) {
+                        if (w < a.cap) cz_out[w] = zz[k];
+                        ++w;
+                    }
+                total += tot;
+            }
+        }
+        if (threadIdx.x == 0) {
+            a.cand_n[bh] = total;
+            if (total > a.cap) atomicOr(a.status, ENTMAXKV_STATUS_OVERFLOW);
+        }
+        return;
+    }
     if (!onchip && threadIdx.x == 0) atomicOr(a.status, ENTMAXKV_STATUS_OVERFLOW);
     const int nloop = onchip ? nc : n_tok;
     auto cz_at = [&](int i) -> float { return onchip ? cz[i] : __ldcg(zr + i); };
 
-    // Newton's method on the normalisation, on [z_max - 1, z_max - n^(1-alpha)]
-    // where F(t) = sum_c [z_c - t]_+^r - 1 decreases.  For r >= 1 (alpha <= 2)
-    // on g(t) = (sum_c [z_c - t]_+^r)^(1/r), a norm of (z - t)_+ and so convex,
-    // from the left end; for r < 1 on F, which is then concave, from the right
-    // end.  Either way the iterates move to the root monotonically.  Each thread sums [x]_+^r and [x]_+^(r-1) over its
-    // strided share of the candidates, the warps' sums are added in warp
-    // order (reproducible), and every warp takes the same step.
-    // (on chip nc is the exact candidate count; off chip only a lower bound on
-    // it, so the bracket uses every token of the list)
-    const float lo = thr;
-    const float hi = zmax - powf((float)(onchip ? nc : n_tok), 1.f - a.alpha);
-    float tau = lo;
-    if (nc > 1 && hi > lo) {
-        const float tol = 1e-7f * fmaxf(1.f, fabsf(zmax));
-        const int rim1 = ri >= 2 ? ri - 1 : 0;
-        float t = r >= 1.f ? lo : hi;
-        for (int it = 0; it < 40; ++it) {
-            float s0 = 0.f, s1 = 0.f;  // sum x^r, sum x^(r-1) over x = z - t > 0
-            auto add = [&](float z) {
-                const float x = z - t;
-                if (ri == 2) {  // alpha = 3/2: branch-free
-                    const float y = fmaxf(x, 0.f);
-                    s0 = fmaf(y, y, s0);
-                    s1 += y;
-                } else if (x > 0.f) {
-                    const float y = ri == 1 ? 1.f : pos_pow(x, r - 1.f, rim1);
-                    s0 = fmaf(x, y, s0);
-                    s1 += y;
-                }
-            };
+    // the exact threshold (on chip nc is the exact candidate count; off chip
+    // only a lower bound on it, so the bracket uses every token of the list);
+    // the finish phase of a sharded decode takes it as given
+    float tau = thr;
+    if (!given_tau) {
+        const float lo = thr;
+        const float hi = zmax - powf((float)(onchip ? nc : n_tok), 1.f - a.alpha);
+        if (nc > 1 && hi > lo) {
             if (onchip) {
-                for (int c = threadIdx.x; c < nc; c += TAU_NT) add(cz[c]);
+                tau = entmax_tau([&](auto add) { for (int c = threadIdx.x; c < nc; c += TAU_NT) add(cz[c]); },
+                                 lo, hi, zmax, r, ri, red);
             } else {
                 // too many candidates to hold: stream the z row through shared
                 // memory in coalesced chunks of zcap
-                for (int c0 = 0; c0 < n_tok; c0 += zcap) {
-                    const int m = min(zcap, n_tok - c0);
-                    __syncthreads();  // the previous chunk has been read
-                    for (int i = threadIdx.x; i < m; i += TAU_NT) cz[i] = __ldcg(zr + c0 + i);
-                    __syncthreads();
-                    for (int c = threadIdx.x; c < m; c += TAU_NT) add(cz[c]);
-                }
+                tau = entmax_tau(
+                    [&](auto add) {
+                        for (int c0 = 0; c0 < n_tok; c0 += zcap) {
+                            const int m = min(zcap, n_tok - c0);
+                            __syncthreads();  // the previous chunk has been read
+                            for (int i = threadIdx.x; i < m; i += TAU_NT) cz[i] = __ldcg(zr + c0 + i);
+                            __syncthreads();
+                            for (int c = threadIdx.x; c < m; c += TAU_NT) add(cz[c]);
+                        }
+                    },
+                    lo, hi, zmax, r, ri, red);
             }
-#pragma unroll
-            for (int o = 16; o; o >>= 1) {
-                s0 += __shfl_xor_sync(FULL, s0, o);
-                s1 += __shfl_xor_sync(FULL, s1, o);
-            }
-            if (lane == 0) {
-                red[it & 1][warp][0] = s0;
-                red[it & 1][warp][1] = s1;
-            }
-            __syncthreads();  // (the other buffer takes the next pass: one barrier a pass)
-            float S0 = 0.f, S1 = 0.f;
-#pragma unroll
-            for (int ww = 0; ww < TAU_NW; ++ww) {
-                S0 += red[it & 1][ww][0];
-                S1 += red[it & 1][ww][1];
-            }
-            if (!(S1 > 0.f)) break;  // no weight right of t (t at the top already)
-            // r >= 1: Newton on g = S0^(1/r) = 1 (convex, nearly linear: one step
-            // when the support's z are equal), t' = t + (S0 - S0^(1-1/r)) / S1;
-            // r < 1: Newton on F = S0 - 1 from the right, t' = t + (S0 - 1) / (r S1)
-            float step;
-            if (ri == 2) step = (S0 - sqrtf(S0)) / S1;
-            else if (ri == 1) step = (S0 - 1.f) / S1;
-            else if (r >= 1.f) step = (S0 - powf(S0, 1.f - 1.f / r)) / S1;
-            else step = (S0 - 1.f) / (r * S1);
-            const float tn = fminf(hi, fmaxf(lo, t + step));
-            const bool done = !(fabsf(tn - t) > tol);
-            t = tn;
-            if (done) break;
         }
-        tau = t;
     }
-    if (threadIdx.x == 0) {
+    if (threadIdx.x == 0 && !given_tau) {
         a.ws.tau[bh] = tau;
         if (a.tau_out) a.tau_out[bh] = tau;
     }
@@ -734,6 +798,66 @@ __global__ void __launch_bounds__(TAU_NT, D == 64 ? 4 : 3) tau_pv_kernel(const _
         for (int w = 0; w < TAU_NW; ++w) sum += accs[w][j];
         a.out[(size_t)bh * D + j] = (float)sum;
     }
+}
+
+// ------------------------------------------- sequence-sharded decode pieces
+
+// Per head: the shard's max z (after q.K) as a float, -inf when it has none.
+__global__ void zmax_export_kernel(DecodeArgs a) {
+    pdl_wait();
+    const int G = a.Hq / a.Hkv;
+    const int i = blockIdx.x * blockDim.x + threadIdx.x;
+    if (i >= a.B * a.nk * G) return;
+    int b, h;
+    head_of(i, a.kv0 * G, a.nk * G, b, h);
+    a.zmax_out[b * a.Hq + h] = ord2f(a.ws.zmax[b * a.Hq + h]);
+}
+
+// Per head: the exact threshold over the candidates of all S shards (each
+// shard's list in list order, the shards in order: the single-device list
+// order when shards hold consecutive page ranges).
+__global__ void __launch_bounds__(TAU_NT) threshold_kernel(const __grid_constant__ ThresholdArgs a) {
+    pdl_wait();
+    extern __shared__ float tz[];  // up to S * cap candidates
+    __shared__ float red[2][TAU_NW][2];
+    __shared__ int s_n, s_over;
+    const int G = a.Hq / a.Hkv;
+    int b, h;
+    head_of(blockIdx.x, a.kv0 * G, a.nk * G, b, h);
+    const int bh = b * a.Hq + h;
+    const size_t BH = (size_t)a.B * a.Hq;
+    const float zmax = a.zmax[bh];
+    if (!(zmax > -INFINITY)) {
+        if (threadIdx.x == 0) a.tau[bh] = __int_as_float(0x7fc00000);
+        return;
+    }
+    if (threadIdx.x == 0) {
+        int n = 0, over = 0;
+        for (int sh = 0; sh < a.S; ++sh) {
+            const int c = a.cand_n[sh * BH + bh];
+            over |= c > a.cap || c < 0;
+            n += min(max(c, 0), a.cap);
+        }
+        s_n = n;
+        s_over = over;
+    }
+    __syncthreads();
+    int n = 0;
+    for (int sh = 0; sh < a.S; ++sh) {
+        const int c = min(max(a.cand_n[sh * BH + bh], 0), a.cap);
+        const float *src = a.cand_z + (sh * BH + bh) * a.cap;
+        for (int i = threadIdx.x; i < c; i += TAU_NT) tz[n + i] = __ldcg(src + i);
+        n += c;
+    }
+    __syncthreads();
+    if (s_over && threadIdx.x == 0) atomicOr(a.status, ENTMAXKV_STATUS_OVERFLOW);
+    const float r = 1.f / (a.alpha - 1.f);
+    const float lo = zmax - 1.f, hi = zmax - powf((float)n, 1.f - a.alpha);
+    float tau = lo;
+    if (n > 1 && hi > lo)
+        tau = entmax_tau([&](auto add) { for (int c = threadIdx.x; c < n; c += TAU_NT) add(tz[c]); }, lo, hi, zmax,
+                         r, a.r_int, red);
+    if (threadIdx.x == 0) a.tau[bh] = tau;
 }
 
 // ------------------------------------------------- partial-sum combination
@@ -1127,6 +1251,34 @@ cudaError_t sparse_t(const DecodeArgs &a, cudaStream_t st) {
 }
 
 template <int D, int G>
+cudaError_t begin_t(const DecodeArgs &a, cudaStream_t st) {
+    cudaError_t e;
+    const int groups = a.B * a.nk;
+    if ((e = launch_pdl(union_kernel, dim3(groups), dim3(UTH), 0, st, a)) != cudaSuccess) return e;
+    if ((e = launch_qk<D, G, false>(a, st)) != cudaSuccess) return e;
+    const int n = a.B * a.nk * G;
+    return launch_pdl(zmax_export_kernel, dim3(ceil_div(n, 256)), dim3(256), 0, st, a);
+}
+
+template <int D, int G>
+cudaError_t candidates_t(const DecodeArgs &a, cudaStream_t st) {
+    cudaError_t e;
+    const int nheads = a.B * a.nk * G;
+    const int zcap = tau_zcap(nheads, a.sms);
+    if ((e = set_smem(tau_pv_kernel<D, false>, tau_smem(ZCAP_MAX))) != cudaSuccess) return e;
+    return launch_pdl(tau_pv_kernel<D, false>, dim3(nheads), dim3(TAU_NT), tau_smem(zcap), st, a, 0, zcap);
+}
+
+template <int D, int G>
+cudaError_t finish_t(const DecodeArgs &a, cudaStream_t st) {
+    cudaError_t e;
+    const int nheads = a.B * a.nk * G;
+    const int zcap = tau_zcap(nheads, a.sms);
+    if ((e = set_smem(tau_pv_kernel<D, true>, tau_smem(ZCAP_MAX))) != cudaSuccess) return e;
+    return launch_pdl(tau_pv_kernel<D, true>, dim3(nheads), dim3(TAU_NT), tau_smem(zcap), st, a, 0, zcap);
+}
+
+template <int D, int G>
 cudaError_t dense_entmax_t(const DecodeArgs &a, cudaStream_t st) {
     cudaError_t e;
     const int groups = a.B * a.nk;
@@ -1183,6 +1335,19 @@ cudaError_t dense_softmax_t(const DecodeArgs &a, cudaStream_t st) {
     } while (0)
 
 cudaError_t launch_decode_sparse(const DecodeArgs &a, cudaStream_t st) { EKV_DISPATCH(sparse_t, a, st); }
+cudaError_t launch_decode_sparse_begin(const DecodeArgs &a, cudaStream_t st) { EKV_DISPATCH(begin_t, a, st); }
+cudaError_t launch_decode_sparse_candidates(const DecodeArgs &a, cudaStream_t st) {
+    EKV_DISPATCH(candidates_t, a, st);
+}
+cudaError_t launch_decode_sparse_finish(const DecodeArgs &a, cudaStream_t st) { EKV_DISPATCH(finish_t, a, st); }
+
+cudaError_t launch_entmax_threshold(const ThresholdArgs &a, cudaStream_t st) {
+    const size_t smem = (size_t)a.S * a.cap * 4;
+    cudaError_t e = set_smem(threshold_kernel, smem);
+    if (e != cudaSuccess) return e;
+    const int nheads = a.B * a.nk * (a.Hq / a.Hkv);
+    return launch_pdl(threshold_kernel, dim3(nheads), dim3(TAU_NT), smem, st, a);
+}
 cudaError_t launch_decode_dense_entmax(const DecodeArgs &a, cudaStream_t st) { EKV_DISPATCH(dense_entmax_t, a, st); }
 cudaError_t launch_decode_dense_softmax(const DecodeArgs &a, cudaStream_t st) {
     EKV_DISPATCH(dense_softmax_t, a, st);

@@ -109,9 +109,34 @@ struct DecodeArgs {
     int r_int;  // 1/(alpha-1) if an integer 1..8, else 0
     int sms;
     int kv0, nk;  // kv-head range [kv0, kv0 + nk); query heads [kv0 G, (kv0 + nk) G)
+    // sequence-sharded phases: sel rows of sel_stride global page ids, this
+    // shard's page i being global page page_begin + i (entries of other shards
+    // are skipped); the global max z / tau per head come in, the shard's max z
+    // and candidate z values go out
+    int sharded, page_begin, sel_stride;
+    const float *zmax_in, *tau_in;
+    float *zmax_out;
+    float *cand_z;
+    int *cand_n;
+    int cap;
     int *status;
 };
 cudaError_t launch_decode_sparse(const DecodeArgs &a, cudaStream_t st);
+cudaError_t launch_decode_sparse_begin(const DecodeArgs &a, cudaStream_t st);
+cudaError_t launch_decode_sparse_candidates(const DecodeArgs &a, cudaStream_t st);
+cudaError_t launch_decode_sparse_finish(const DecodeArgs &a, cudaStream_t st);
+
+struct ThresholdArgs {
+    const float *cand_z;  // [S][B*Hq][cap]
+    const int *cand_n;    // [S][B*Hq]
+    const float *zmax;    // [B*Hq]
+    float *tau;           // [B*Hq]
+    int S, cap, B, Hq, Hkv, kv0, nk;
+    float alpha;
+    int r_int;
+    int *status;
+};
+cudaError_t launch_entmax_threshold(const ThresholdArgs &a, cudaStream_t st);
 cudaError_t launch_decode_dense_entmax(const DecodeArgs &a, cudaStream_t st);
 cudaError_t launch_decode_dense_softmax(const DecodeArgs &a, cudaStream_t st);
 

@@ -28,7 +28,8 @@ STATUS_BAD_PAGE, STATUS_BAD_SELECTION, STATUS_TIMEOUT, STATUS_OVERFLOW = 1, 2, 4
 EXPORTED = ("entmaxkv_strerror", "entmaxkv_version", "entmaxkv_meta_bytes",
             "entmaxkv_workspace_size", "entmaxkv_get_status", "entmaxkv_build_meta", "entmaxkv_append",
             "entmaxkv_score_pages", "entmaxkv_select", "entmaxkv_decode_sparse",
-            "entmaxkv_decode_sparse_static", "entmaxkv_decode_dense")
+            "entmaxkv_decode_sparse_static", "entmaxkv_decode_dense", "entmaxkv_decode_sparse_begin",
+            "entmaxkv_decode_sparse_candidates", "entmaxkv_entmax_threshold", "entmaxkv_decode_sparse_finish")
 
 
 class EntmaxKVError(RuntimeError):
@@ -89,6 +90,10 @@ def lib():
         L.entmaxkv_decode_sparse.argtypes = [sp, vp, vp, vp, vp, vp, vp, vp, f32, vp, vp, vp, vp, sz, vp]
         L.entmaxkv_decode_dense.argtypes = [sp, vp, vp, vp, vp, vp, f32, vp, vp, vp, vp, sz, vp]
         L.entmaxkv_decode_sparse_static.argtypes = [sp, vp, vp, vp, vp, vp, vp, vp, f32, vp, vp, vp, vp]
+        L.entmaxkv_decode_sparse_begin.argtypes = [sp, vp, vp, vp, vp, vp, vp, vp, i32, i32, f32, vp, vp, sz, vp]
+        L.entmaxkv_decode_sparse_candidates.argtypes = [sp, vp, vp, vp, vp, vp, f32, vp, i32, vp, vp, vp, sz, vp]
+        L.entmaxkv_entmax_threshold.argtypes = [sp, i32, i32, vp, vp, vp, f32, vp, vp]
+        L.entmaxkv_decode_sparse_finish.argtypes = [sp, vp, vp, vp, vp, vp, f32, vp, vp, vp, vp, vp, sz, vp]
         for fn in EXPORTED:
             if fn not in ("entmaxkv_strerror", "entmaxkv_version", "entmaxkv_meta_bytes",
                           "entmaxkv_workspace_size"):
@@ -190,6 +195,46 @@ def entmaxkv_decode_sparse(shape, q, k_cache, v_cache, page_table, seq_lens, sel
         float(alpha), _ptr(out, torch.float32, "out"), _ptr(tau_out, torch.float32, "tau_out"),
         _ptr(p_out, torch.float32, "p_out"), _ptr(workspace, None, "workspace"),
         0 if workspace is None else workspace.numel(), _stream(stream)))
+
+
+def _kv_args(q, k_cache, v_cache, page_table, seq_lens):
+    return (_ptr(q, torch.bfloat16, "q"), _ptr(k_cache, torch.bfloat16, "k_cache"),
+            _ptr(v_cache, torch.bfloat16, "v_cache"), _ptr(page_table, torch.int32, "page_table"),
+            _ptr(seq_lens, torch.int32, "seq_lens"))
+
+
+def entmaxkv_decode_sparse_begin(shape, q, k_cache, v_cache, page_table, seq_lens, sel, cnt, sel_max_pages,
+                                 page_begin, alpha, zmax_out, workspace, stream=None):
+    _check("entmaxkv_decode_sparse_begin", lib().entmaxkv_decode_sparse_begin(
+        C.byref(shape), *_kv_args(q, k_cache, v_cache, page_table, seq_lens),
+        _ptr(sel, torch.int32, "sel"), _ptr(cnt, torch.int32, "cnt"), int(sel_max_pages), int(page_begin),
+        float(alpha), _ptr(zmax_out, torch.float32, "zmax_out"), _ptr(workspace, None, "workspace"),
+        workspace.numel(), _stream(stream)))
+
+
+def entmaxkv_decode_sparse_candidates(shape, q, k_cache, v_cache, page_table, seq_lens, alpha, zmax_in, cap,
+                                      cand_z, cand_n, workspace, stream=None):
+    _check("entmaxkv_decode_sparse_candidates", lib().entmaxkv_decode_sparse_candidates(
+        C.byref(shape), *_kv_args(q, k_cache, v_cache, page_table, seq_lens), float(alpha),
+        _ptr(zmax_in, torch.float32, "zmax_in"), int(cap), _ptr(cand_z, torch.float32, "cand_z"),
+        _ptr(cand_n, torch.int32, "cand_n"), _ptr(workspace, None, "workspace"), workspace.numel(),
+        _stream(stream)))
+
+
+def entmaxkv_entmax_threshold(shape, n_shards, cap, cand_z, cand_n, zmax_in, alpha, tau_out, stream=None):
+    _check("entmaxkv_entmax_threshold", lib().entmaxkv_entmax_threshold(
+        C.byref(shape), int(n_shards), int(cap), _ptr(cand_z, torch.float32, "cand_z"),
+        _ptr(cand_n, torch.int32, "cand_n"), _ptr(zmax_in, torch.float32, "zmax_in"), float(alpha),
+        _ptr(tau_out, torch.float32, "tau_out"), _stream(stream)))
+
+
+def entmaxkv_decode_sparse_finish(shape, q, k_cache, v_cache, page_table, seq_lens, alpha, zmax_in, tau_in, out,
+                                  p_out, workspace, stream=None):
+    _check("entmaxkv_decode_sparse_finish", lib().entmaxkv_decode_sparse_finish(
+        C.byref(shape), *_kv_args(q, k_cache, v_cache, page_table, seq_lens), float(alpha),
+        _ptr(zmax_in, torch.float32, "zmax_in"), _ptr(tau_in, torch.float32, "tau_in"),
+        _ptr(out, torch.float32, "out"), _ptr(p_out, torch.float32, "p_out"), _ptr(workspace, None, "workspace"),
+        workspace.numel(), _stream(stream)))
 
 
 def entmaxkv_decode_dense(shape, q, k_cache, v_cache, page_table, seq_lens, alpha, out, tau_out=None,

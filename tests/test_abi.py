@@ -24,7 +24,7 @@ def _declared():
 def test_library_exports_every_declared_symbol():
     L = nv.lib()
     names = _declared()
-    assert len(names) == 12
+    assert len(names) == 16
     assert set(names) == set(nv.EXPORTED)
     for n in names:
         assert hasattr(L, n)
