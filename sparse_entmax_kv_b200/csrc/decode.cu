@@ -7,7 +7,7 @@
 //                  heads' selected pages, ascending, each with a G-bit head
 //                  mask; also resets the per-head maxima.
 //   qk_kernel      split over the union: TMA 2-D loads (128-byte swizzle) of
-//                  the K tiles through a 4-stage mbarrier ring fed by one
+//                  the K tiles through a 3-stage mbarrier ring fed by one
 //                  producer warp (which resolves union entries and page-table
 //                  rows 32 steps at a time); z = (alpha-1) q.k/sqrt(d) for all
 //                  G heads of the group from one copy of each tile (tensor-core
@@ -254,10 +254,16 @@ __device__ void produce(const DecodeArgs &a, const CUtensorMap *m0, const CUtens
 
 // ----------------------------------------------------------------- q . K^T
 
+// q.K ring: three stages per CTA and four CTAs per SM (measured: more CTAs
+// with a shallower ring gather random pages faster than three CTAs of four
+// stages, e.g. 42 vs 46.5 us for the 128k-token top-k decode).
+constexpr int QK_NS = 3;
+constexpr int QK_PER_SM = 4;
+
 template <int D, int G, bool DENSE>
 __global__ void __launch_bounds__(DEC_THREADS) qk_kernel(const __grid_constant__ DecodeArgs a) {
     pdl_wait();
-    constexpr int NS = 4;
+    constexpr int NS = QK_NS;
     using RG = Ring<D, G, NS, 1>;
     constexpr int TPS = RG::TPS;
     extern __shared__ unsigned char smem_raw[];
@@ -1221,12 +1227,12 @@ cudaError_t set_smem(K kern, size_t bytes) {
 
 template <int D, int G, bool DENSE>
 cudaError_t launch_qk(const DecodeArgs &a, cudaStream_t st) {
-    using RG = Ring<D, G, 4, 1>;
+    using RG = Ring<D, G, QK_NS, 1>;
     auto k = qk_kernel<D, G, DENSE>;
     cudaError_t e = set_smem(k, RG::BYTES);
     if (e != cudaSuccess) return e;
     const int groups = a.B * a.nk;
-    const int S = pick_splits(a.sms, 3, groups, ceil_div(a.max_pages, RG::TPS / a.P), 1 << 16);
+    const int S = pick_splits(a.sms, QK_PER_SM, groups, ceil_div(a.max_pages, RG::TPS / a.P), 1 << 16);
     return launch_pdl(k, dim3(S, groups), dim3(DEC_THREADS), RG::BYTES, st, a);
 }
 
