@@ -259,6 +259,10 @@ ENTMAXKV_API int entmaxkv_select(const entmaxkv_shape *shape, const int32_t *seq
  * fp32 [B][Hq][max_pages*P] in logical token order: for every selected page,
  * p of its valid tokens is written (0 off the support); other entries are
  * left untouched.  A head with no selected page gets out = 0 and tau = NaN.
+ * out may be pinned host memory (allocated with cudaHostAlloc, which unified
+ * addressing maps into the device's address space): the kernels then write
+ * the result straight to the host, so no separate device-to-host copy is
+ * needed after the call.
  * alpha == 1 gives softmax over the same tokens T (for comparing entmax and
  * softmax at one kept set): out = sum_T softmax(s)_t v_t, every selected
  * token carries weight, so K and V of the group's selected pages are read;

@@ -59,27 +59,31 @@ class EntmaxKVDecoder:
         nv.entmaxkv_build_meta(self.shape, self.k_cache, self.page_table, self.seq_lens,
                                first_page, n_pages, self.meta)
 
-    def step(self, q, append_page=None, p_out=None, new_kv=None):
+    def step(self, q, append_page=None, p_out=None, new_kv=None, out=None):
         """One decode step for query q (bf16 [B, Hq, d]).  ``new_kv``: the
         (k_new, v_new) rows (bf16 [B, Hkv, d]) of the token each sequence just
         gained, at position seq_lens-1, written into the cache together with
         its page's metadata; or ``append_page``: a logical page whose metadata
-        is refreshed (the caller wrote the token already); or neither."""
+        is refreshed (the caller wrote the token already); or neither.
+        ``out``: where the output goes (fp32 [B, Hq, d]; device memory or
+        pinned host memory, which the decode writes directly); default the
+        decoder's own buffer."""
+        dst = self.out if out is None else out
         if self.streams is None:
-            self._step_range(self.shape, q, append_page, p_out, new_kv, None, None)
-            return self.out
+            self._step_range(self.shape, q, append_page, p_out, new_kv, None, None, dst)
+            return dst
         cur = torch.cuda.current_stream()
         prev = None
         for shape, st, ev in zip(self.shapes, self.streams, self.scored):
             st.wait_stream(cur)
             with torch.cuda.stream(st):
-                self._step_range(shape, q, append_page, p_out, new_kv, prev, ev)
+                self._step_range(shape, q, append_page, p_out, new_kv, prev, ev, dst)
             prev = ev
         for st in self.streams:
             cur.wait_stream(st)
-        return self.out
+        return dst
 
-    def _step_range(self, shape, q, append_page, p_out, new_kv, after, scored):
+    def _step_range(self, shape, q, append_page, p_out, new_kv, after, scored, out):
         if new_kv is not None:
             nv.entmaxkv_append(shape, new_kv[0], new_kv[1], self.page_table, self.seq_lens,
                                self.k_cache, self.v_cache, self.meta)
@@ -94,7 +98,7 @@ class EntmaxKVDecoder:
         nv.entmaxkv_select(shape, self.seq_lens, self.bbox, self.mu, self.sigma, self.policy,
                            self.k, self.alpha, self.delta, self.sel, self.cnt, self.tau_hat)
         nv.entmaxkv_decode_sparse(shape, q, self.k_cache, self.v_cache, self.page_table,
-                                  self.seq_lens, self.sel, self.cnt, self.alpha, self.out,
+                                  self.seq_lens, self.sel, self.cnt, self.alpha, out,
                                   self.tau, p_out, self.ws)
 
 

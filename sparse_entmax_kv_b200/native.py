@@ -107,12 +107,15 @@ def _check(fn, rc):
         raise EntmaxKVError(fn, rc, lib().entmaxkv_strerror(rc).decode())
 
 
-def _ptr(t, dtype=None, name="tensor"):
+def _ptr(t, dtype=None, name="tensor", pinned_ok=False):
+    """Device pointer of t.  pinned_ok: a pinned host tensor is accepted too
+    (with unified addressing its address is valid in kernels, which then
+    read or write host memory directly over the bus)."""
     if t is None:
         return None
     if not isinstance(t, torch.Tensor):
         raise TypeError(f"{name}: expected a torch.Tensor")
-    if t.device.type != "cuda":
+    if t.device.type != "cuda" and not (pinned_ok and t.device.type == "cpu" and t.is_pinned()):
         raise ValueError(f"{name}: must be a CUDA tensor (no CPU path exists)")
     if dtype is not None and t.dtype != dtype:
         raise TypeError(f"{name}: expected {dtype}, got {t.dtype}")
@@ -192,7 +195,7 @@ def entmaxkv_decode_sparse(shape, q, k_cache, v_cache, page_table, seq_lens, sel
         C.byref(shape), _ptr(q, torch.bfloat16, "q"), _ptr(k_cache, torch.bfloat16, "k_cache"),
         _ptr(v_cache, torch.bfloat16, "v_cache"), _ptr(page_table, torch.int32, "page_table"),
         _ptr(seq_lens, torch.int32, "seq_lens"), _ptr(sel, torch.int32, "sel"), _ptr(cnt, torch.int32, "cnt"),
-        float(alpha), _ptr(out, torch.float32, "out"), _ptr(tau_out, torch.float32, "tau_out"),
+        float(alpha), _ptr(out, torch.float32, "out", pinned_ok=True), _ptr(tau_out, torch.float32, "tau_out"),
         _ptr(p_out, torch.float32, "p_out"), _ptr(workspace, None, "workspace"),
         0 if workspace is None else workspace.numel(), _stream(stream)))
 

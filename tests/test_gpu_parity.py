@@ -468,6 +468,21 @@ def test_append_writes_rows_and_rebuilds_page(name):
                                       err_msg=nm)
 
 
+def test_decode_output_to_pinned_host_memory():
+    """out may be pinned host memory: the kernels write the result there
+    directly, equal to the device-buffer result bit for bit."""
+    wl = SMALL["gauss_small"]
+    inp, _ = gpu_inputs(wl, 13)
+    dec = EntmaxKVDecoder(inp["k_cache"], inp["v_cache"], inp["page_table"], inp["seq_lens"], wl.Hq,
+                          alpha=wl.alpha, policy=wl.policy, delta=wl.delta)
+    dec.build_meta()
+    dev_out = dec.step(inp["q"]).clone()
+    host_out = torch.full((wl.B, wl.Hq, wl.d), float("nan")).pin_memory()
+    dec.step(inp["q"], out=host_out)
+    torch.cuda.synchronize()
+    assert torch.equal(host_out, dev_out.cpu())
+
+
 def test_append_bad_page_sets_status_and_skips():
     """A page-table entry outside [0, num_blocks) flags the status and that
     sequence writes nothing; the other sequences append as usual."""
