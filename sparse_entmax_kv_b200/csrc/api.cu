@@ -334,12 +334,15 @@ int entmaxkv_select(const entmaxkv_shape *s, const int32_t *seq_lens, const floa
     return cuda_rc(launch_select(a, static_cast<cudaStream_t>(stream)));
 }
 
+// Shared argument checks and set-up of the decode calls.  out may be NULL only
+// where the call writes no output (need_out false: the sharded begin and
+// candidates phases).
 static int fill_decode(bool dense, const entmaxkv_shape *s, const void *q, const void *k_cache, const void *v_cache,
                        const int32_t *page_table, const int32_t *seq_lens, float alpha, float *out, float *tau_out,
-                       float *p_out, void *workspace, size_t ws_bytes, DecodeArgs *a) {
+                       float *p_out, void *workspace, size_t ws_bytes, DecodeArgs *a, bool need_out = true) {
     int rc = check_shape(s);
     if (rc) return rc;
-    if (!q || !k_cache || !v_cache || !page_table || !seq_lens || !out) return ENTMAXKV_ERR_NULL;
+    if (!q || !k_cache || !v_cache || !page_table || !seq_lens || (need_out && !out)) return ENTMAXKV_ERR_NULL;
     if (!aligned16(q) || !aligned16(k_cache) || !aligned16(v_cache)) return ENTMAXKV_ERR_ALIGN;
     if (!std::isfinite(alpha)) return ENTMAXKV_ERR_ALPHA;
     const size_t need =
@@ -404,10 +407,9 @@ int entmaxkv_decode_sparse_begin(const entmaxkv_shape *s, const void *q, const v
     if (s && (s->max_pages > MAX_SEL_PAGES || page_begin < 0 || sel_max_pages < 1 || page_begin >= sel_max_pages))
         return ENTMAXKV_ERR_SHAPE;
     DecodeArgs a;
-    int rc = fill_decode(false, s, q, k_cache, v_cache, page_table, seq_lens, alpha, zmax_out, nullptr, nullptr,
-                         workspace, ws_bytes, &a);
+    int rc = fill_decode(false, s, q, k_cache, v_cache, page_table, seq_lens, alpha, nullptr, nullptr, nullptr,
+                         workspace, ws_bytes, &a, false);
     if (rc) return rc;
-    a.out = nullptr;
     a.sel = sel;
     a.cnt = cnt;
     a.sharded = 1;
@@ -426,10 +428,9 @@ int entmaxkv_decode_sparse_candidates(const entmaxkv_shape *s, const void *q, co
     if (!(alpha > 1.f)) return ENTMAXKV_ERR_ALPHA;
     if (cap < 1) return ENTMAXKV_ERR_SHAPE;
     DecodeArgs a;
-    int rc = fill_decode(false, s, q, k_cache, v_cache, page_table, seq_lens, alpha, cand_z, nullptr, nullptr,
-                         workspace, ws_bytes, &a);
+    int rc = fill_decode(false, s, q, k_cache, v_cache, page_table, seq_lens, alpha, nullptr, nullptr, nullptr,
+                         workspace, ws_bytes, &a, false);
     if (rc) return rc;
-    a.out = nullptr;
     a.zmax_in = zmax_in;
     a.cand_z = cand_z;
     a.cand_n = cand_n;

@@ -724,85 +724,85 @@ __global__ void __launch_bounds__(TAU_NT, D == 64 ? 4 : 3) tau_pv_kernel(const _
         a.ws.tau[bh] = tau;
         if (a.tau_out) a.tau_out[bh] = tau;
     }
-    if (!GATHER) return;
-
-    // p v over the support: every warp takes a strided share of the
-    // candidates, moves the lanes with weight to the front eight at a time and
-    // sums p v of their value rows in fp64 (exact products).
-    double acc[CPL];
-#pragma unroll
-    for (int c = 0; c < CPL; ++c) acc[c] = 0.0;
-    const size_t lstride = (size_t)a.max_pages * P;
-    auto put_p = [&](int pos, float p) {
-        if (!a.p_out) return;
-        const int up = pos / P, t = pos - up * P;
-        const int page = dense ? up : (__ldcg(a.ws.union_e + (size_t)bk * a.max_pages + up) >> 8);
-        a.p_out[(size_t)bh * lstride + (size_t)page * P + t] = p;
-    };
-    auto gather8 = [&](int nr, int row, float p) {
-        // lanes 0..nr-1 hold (row, p) of up to eight support tokens; the
-        // rows' bf16 words are all loaded before the first product
-        unsigned vw[8][CPL / 2];
-        float pp[8];
-#pragma unroll
-        for (int i = 0; i < 8; ++i) {
-            const int rw = __shfl_sync(FULL, row, i);
-            pp[i] = i < nr ? __shfl_sync(FULL, p, i) : 0.f;
-            const uint16_t *vr = a.v + (size_t)rw * D + lane * CPL;
-            if (CPL == 4) {
-                uint2 w = make_uint2(0u, 0u);
-                if (i < nr) w = __ldg(reinterpret_cast<const uint2 *>(vr));
-                vw[i][0] = w.x;
-                vw[i][CPL / 2 - 1] = w.y;
-            } else {
-                vw[i][0] = i < nr ? __ldg(reinterpret_cast<const unsigned *>(vr)) : 0u;
-            }
-        }
-#pragma unroll
-        for (int i = 0; i < 8; ++i)
-#pragma unroll
-            for (int cc = 0; cc < CPL; ++cc) {
-                const unsigned w = vw[i][cc >> 1];
-                acc[cc] = fma((double)pp[i], (double)((cc & 1) ? bf16hi(w) : bf16lo(w)), acc[cc]);
-            }
-    };
-    // candidate c belongs to warp c % TAU_NW (lane (c / TAU_NW) % 32), so a
-    // small support spreads over all warps
-    for (int k0 = 0; k0 < nloop; k0 += TAU_NT) {
-        const int c = k0 + lane * TAU_NW + warp;
-        const float z = c < nloop ? cz_at(c) : -INFINITY;
-        const float p = pos_pow(z - tau, r, ri);
-        unsigned bal = __ballot_sync(FULL, p > 0.f);
-        while (bal) {
-            int src = 0, nr = 0;
-#pragma unroll
-            for (int i = 0; i < 8; ++i)
-                if (bal) {
-                    const int l = __ffs(bal) - 1;
-                    bal &= bal - 1;
-                    if (lane == i) src = l;
-                    nr = i + 1;
+    if constexpr (GATHER) {
+        // p v over the support: every warp takes a strided share of the
+        // candidates, moves the lanes with weight to the front eight at a time and
+        // sums p v of their value rows in fp64 (exact products).
+        double acc[CPL];
+    #pragma unroll
+        for (int c = 0; c < CPL; ++c) acc[c] = 0.0;
+        const size_t lstride = (size_t)a.max_pages * P;
+        auto put_p = [&](int pos, float p) {
+            if (!a.p_out) return;
+            const int up = pos / P, t = pos - up * P;
+            const int page = dense ? up : (__ldcg(a.ws.union_e + (size_t)bk * a.max_pages + up) >> 8);
+            a.p_out[(size_t)bh * lstride + (size_t)page * P + t] = p;
+        };
+        auto gather8 = [&](int nr, int row, float p) {
+            // lanes 0..nr-1 hold (row, p) of up to eight support tokens; the
+            // rows' bf16 words are all loaded before the first product
+            unsigned vw[8][CPL / 2];
+            float pp[8];
+    #pragma unroll
+            for (int i = 0; i < 8; ++i) {
+                const int rw = __shfl_sync(FULL, row, i);
+                pp[i] = i < nr ? __shfl_sync(FULL, p, i) : 0.f;
+                const uint16_t *vr = a.v + (size_t)rw * D + lane * CPL;
+                if (CPL == 4) {
+                    uint2 w = make_uint2(0u, 0u);
+                    if (i < nr) w = __ldg(reinterpret_cast<const uint2 *>(vr));
+                    vw[i][0] = w.x;
+                    vw[i][CPL / 2 - 1] = w.y;
+                } else {
+                    vw[i][0] = i < nr ? __ldg(reinterpret_cast<const unsigned *>(vr)) : 0u;
                 }
-            const int cs = k0 + __shfl_sync(FULL, lane, src) * TAU_NW + warp;
-            const float pl = __shfl_sync(FULL, p, src);
-            int row = 0;
-            if (lane < nr) {
-                const int pos = onchip ? cpos[cs] : cs;
-                row = onchip ? crow[cs] : row_of_pos(pos);
-                put_p(pos, pl);
             }
-            gather8(nr, row, lane < nr ? pl : 0.f);
+    #pragma unroll
+            for (int i = 0; i < 8; ++i)
+    #pragma unroll
+                for (int cc = 0; cc < CPL; ++cc) {
+                    const unsigned w = vw[i][cc >> 1];
+                    acc[cc] = fma((double)pp[i], (double)((cc & 1) ? bf16hi(w) : bf16lo(w)), acc[cc]);
+                }
+        };
+        // candidate c belongs to warp c % TAU_NW (lane (c / TAU_NW) % 32), so a
+        // small support spreads over all warps
+        for (int k0 = 0; k0 < nloop; k0 += TAU_NT) {
+            const int c = k0 + lane * TAU_NW + warp;
+            const float z = c < nloop ? cz_at(c) : -INFINITY;
+            const float p = pos_pow(z - tau, r, ri);
+            unsigned bal = __ballot_sync(FULL, p > 0.f);
+            while (bal) {
+                int src = 0, nr = 0;
+    #pragma unroll
+                for (int i = 0; i < 8; ++i)
+                    if (bal) {
+                        const int l = __ffs(bal) - 1;
+                        bal &= bal - 1;
+                        if (lane == i) src = l;
+                        nr = i + 1;
+                    }
+                const int cs = k0 + __shfl_sync(FULL, lane, src) * TAU_NW + warp;
+                const float pl = __shfl_sync(FULL, p, src);
+                int row = 0;
+                if (lane < nr) {
+                    const int pos = onchip ? cpos[cs] : cs;
+                    row = onchip ? crow[cs] : row_of_pos(pos);
+                    put_p(pos, pl);
+                }
+                gather8(nr, row, lane < nr ? pl : 0.f);
+            }
         }
-    }
-    __syncthreads();  // every warp is done with the candidates
-#pragma unroll
-    for (int cc = 0; cc < CPL; ++cc) accs[warp][lane * CPL + cc] = acc[cc];
-    __syncthreads();
-    for (int j = threadIdx.x; j < D; j += TAU_NT) {
-        double sum = 0.0;
-#pragma unroll
-        for (int w = 0; w < TAU_NW; ++w) sum += accs[w][j];
-        a.out[(size_t)bh * D + j] = (float)sum;
+        __syncthreads();  // every warp is done with the candidates
+    #pragma unroll
+        for (int cc = 0; cc < CPL; ++cc) accs[warp][lane * CPL + cc] = acc[cc];
+        __syncthreads();
+        for (int j = threadIdx.x; j < D; j += TAU_NT) {
+            double sum = 0.0;
+    #pragma unroll
+            for (int w = 0; w < TAU_NW; ++w) sum += accs[w][j];
+            a.out[(size_t)bh * D + j] = (float)sum;
+        }
     }
 }
 
@@ -826,7 +826,7 @@ __global__ void __launch_bounds__(TAU_NT) threshold_kernel(const __grid_constant
     pdl_wait();
     extern __shared__ float tz[];  // up to S * cap candidates
     __shared__ float red[2][TAU_NW][2];
-    __shared__ int s_n, s_over;
+    __shared__ int s_over;
     const int G = a.Hq / a.Hkv;
     int b, h;
     head_of(blockIdx.x, a.kv0 * G, a.nk * G, b, h);
@@ -838,13 +838,11 @@ __global__ void __launch_bounds__(TAU_NT) threshold_kernel(const __grid_constant
         return;
     }
     if (threadIdx.x == 0) {
-        int n = 0, over = 0;
+        int over = 0;
         for (int sh = 0; sh < a.S; ++sh) {
             const int c = a.cand_n[sh * BH + bh];
             over |= c > a.cap || c < 0;
-            n += min(max(c, 0), a.cap);
         }
-        s_n = n;
         s_over = over;
     }
     __syncthreads();
