@@ -435,7 +435,7 @@ __global__ void __launch_bounds__(SEL_THREADS) gauss_kernel(SelectArgs a) {
 constexpr int GCL = 4;
 constexpr int GTH = 256;
 constexpr int GIT = 16;
-constexpr int GCAPR = 256;  // candidates per CTA that rank 0 holds
+constexpr int GCAPR = 768;  // candidates per CTA that rank 0 holds
 
 template <int R>
 __global__ void __cluster_dims__(GCL, 1, 1) __launch_bounds__(GTH) gauss_cluster_kernel(SelectArgs a) {
