@@ -311,17 +311,18 @@ def run_gpu(args, rank, world):
     # host-to-device copy), the output goes back to host
     n_q, n_kv = q.numel(), k_new.numel()
     stage_host = torch.cat([q.reshape(-1), k_new.reshape(-1), v_new.reshape(-1)]).cpu().pin_memory()
-    stage_dev = torch.empty_like(stage_host, device=dev)
-    q_dev = stage_dev[:n_q].view_as(q)
-    k_dev = stage_dev[n_q:n_q + n_kv].view_as(k_new)
-    v_dev = stage_dev[n_q + n_kv:].view_as(v_new)
+    q_dev = torch.empty_like(q)  # where append stages the queries for the later calls
     out_host = torch.empty((wl.B, wl.Hq, wl.d), dtype=torch.float32).pin_memory()
 
+    q_host = stage_host[:n_q].view_as(q)
+    k_host = stage_host[n_q:n_q + n_kv].view_as(k_new)
+    v_host = stage_host[n_q + n_kv:].view_as(v_new)
+
     def e2e_once():
-        # the decode writes the output straight into pinned host memory (the
-        # device-to-host transfer of the result happens inside the step)
-        stage_dev.copy_(stage_host, non_blocking=True)
-        dec.step(q_dev, new_kv=(k_dev, v_dev), out=out_host)
+        # the append kernel reads q and the new rows from pinned host memory
+        # (the host-to-device transfer of the inputs happens inside the step)
+        # and the decode writes the output straight into pinned host memory
+        dec.step(q_dev, new_kv=(k_host, v_host), out=out_host, q_in=q_host)
 
     def time_e2e(fn):
         ts = []
@@ -644,9 +645,10 @@ def main():
             "stages_us": res["stage_us"], "bytes_per_step": nb,
             "e2e": {"value": round(e2e_val, 2), "unit": "GB/s", "us_per_step": round(res["e2e_ms"] * 1e3, 2),
                     "h2d_bytes_per_step": res["e2e_bytes"][0], "d2h_bytes_per_step": res["e2e_bytes"][1],
-                    "how": "one H2D copy of q and the appended token's k/v rows from one pinned buffer, the four "
-                           "C-ABI calls (append writes the rows and refreshes their pages' metadata; the decode "
-                           "writes the output straight into pinned host memory), captured as one CUDA graph",
+                    "how": "the four C-ABI calls, captured as one CUDA graph: append reads q and the appended "
+                           "token's k/v rows from pinned host memory over the bus (copying q to the device, writing "
+                           "the rows and refreshing their pages' metadata); the decode writes the output straight "
+                           "into pinned host memory",
                     "eager_us_per_step": round(res["e2e_eager_ms"] * 1e3, 2)},
             "timing": "step = CUDA-graph replay of the four C-ABI calls; stages_us from the same calls issued "
                       "eagerly with events around each (eager step sum %.2f us)" % (res["eager_step_ms"] * 1e3),

@@ -191,14 +191,20 @@ ENTMAXKV_API int entmaxkv_build_meta(const entmaxkv_shape *shape, const void *k_
  * rebuild the metadata record of logical page (L-1)/P exactly as
  * entmaxkv_build_meta does (same bits).  Sequences with L <= 0 are skipped.  A
  * page-table entry outside [0, num_blocks), or (L-1)/P >= max_pages, sets
- * ENTMAXKV_STATUS_BAD_PAGE and skips that sequence.  One kernel launch on
- * `stream`; no allocation.  k_cache, v_cache and meta must be 16-byte aligned
+ * ENTMAXKV_STATUS_BAD_PAGE and skips that sequence.  If q_in and q_out are
+ * both given (bf16 [B][Hq][d]), the step's queries of the kv heads in range
+ * are copied from q_in to q_out as well (one of them NULL without the other:
+ * ENTMAXKV_ERR_NULL).  k_new, v_new and q_in may be pinned host memory
+ * (cudaHostAlloc; unified addressing maps it into the device's address
+ * space): the kernel then reads the step's inputs over the bus itself, so no
+ * separate host-to-device copy is needed.  One kernel launch on `stream`; no
+ * allocation.  k_cache, v_cache and meta must be 16-byte aligned
  * (ENTMAXKV_ERR_ALIGN).
  */
 ENTMAXKV_API int entmaxkv_append(const entmaxkv_shape *shape, const void *k_new,
                     const void *v_new, const int32_t *page_table,
                     const int32_t *seq_lens, void *k_cache, void *v_cache,
-                    void *meta, void *stream);
+                    void *meta, const void *q_in, void *q_out, void *stream);
 
 /*
  * Section 2.A (query-aware page scoring): for every (b, h) and page p < N_b,

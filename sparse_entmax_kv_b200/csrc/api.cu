@@ -227,10 +227,12 @@ int entmaxkv_build_meta(const entmaxkv_shape *s, const void *k_cache, const int3
 }
 
 int entmaxkv_append(const entmaxkv_shape *s, const void *k_new, const void *v_new, const int32_t *page_table,
-                    const int32_t *seq_lens, void *k_cache, void *v_cache, void *meta, void *stream) {
+                    const int32_t *seq_lens, void *k_cache, void *v_cache, void *meta, const void *q_in,
+                    void *q_out, void *stream) {
     int rc = check_shape(s);
     if (rc) return rc;
     if (!k_new || !v_new || !page_table || !seq_lens || !k_cache || !v_cache || !meta) return ENTMAXKV_ERR_NULL;
+    if ((q_in == nullptr) != (q_out == nullptr)) return ENTMAXKV_ERR_NULL;
     if (!aligned16(k_cache) || !aligned16(v_cache) || !aligned16(meta)) return ENTMAXKV_ERR_ALIGN;
     DevInfo di;
     if ((rc = device_info(&di))) return rc;
@@ -253,6 +255,9 @@ int entmaxkv_append(const entmaxkv_shape *s, const void *k_new, const void *v_ne
     a.m.k = a.k_cache;
     a.k_new = static_cast<const uint16_t *>(k_new);
     a.v_new = static_cast<const uint16_t *>(v_new);
+    a.q_in = static_cast<const uint16_t *>(q_in);
+    a.q_out = static_cast<uint16_t *>(q_out);
+    a.Hq = s->Hq;
     return cuda_rc(launch_append(a, static_cast<cudaStream_t>(stream)));
 }
 

@@ -53,6 +53,9 @@ struct AppendArgs {
     MetaArgs m;
     uint16_t *k_cache, *v_cache;
     const uint16_t *k_new, *v_new;  // [B][Hkv][d]
+    const uint16_t *q_in;           // [B][Hq][d] or null: copied to q_out
+    uint16_t *q_out;
+    int Hq;
 };
 cudaError_t launch_append(const AppendArgs &a, cudaStream_t st);
 

@@ -82,11 +82,20 @@ __global__ void __launch_bounds__(D) build_meta_kernel(MetaArgs a) {
 }
 
 // One CTA per (sequence, kv head): the new token's key and value rows land in
-// slot seq_len-1 of the paged cache, then the record of that page is rebuilt.
+// slot seq_len-1 of the paged cache, then the record of that page is rebuilt;
+// optionally the group's query rows are copied too (the inputs may be read
+// straight from pinned host memory).
 template <int D, int P>
 __global__ void __launch_bounds__(D) append_kernel(AppendArgs a) {
     pdl_wait();
     const int b = blockIdx.x, kvh = a.m.kv0 + blockIdx.y;
+    if (a.q_in) {  // the step's queries of this group, staged for the later calls
+        const int G = a.Hq / a.m.Hkv;
+        for (int g = 0; g < G; ++g) {
+            const size_t o = ((size_t)b * a.Hq + kvh * G + g) * D + threadIdx.x;
+            a.q_out[o] = a.q_in[o];
+        }
+    }
     const int seq = a.m.seq_lens[b];
     if (seq <= 0) return;
     const int p = (seq - 1) / P, t = (seq - 1) % P;

@@ -59,7 +59,7 @@ class EntmaxKVDecoder:
         nv.entmaxkv_build_meta(self.shape, self.k_cache, self.page_table, self.seq_lens,
                                first_page, n_pages, self.meta)
 
-    def step(self, q, append_page=None, p_out=None, new_kv=None, out=None):
+    def step(self, q, append_page=None, p_out=None, new_kv=None, out=None, q_in=None):
         """One decode step for query q (bf16 [B, Hq, d]).  ``new_kv``: the
         (k_new, v_new) rows (bf16 [B, Hkv, d]) of the token each sequence just
         gained, at position seq_lens-1, written into the cache together with
@@ -67,26 +67,28 @@ class EntmaxKVDecoder:
         is refreshed (the caller wrote the token already); or neither.
         ``out``: where the output goes (fp32 [B, Hq, d]; device memory or
         pinned host memory, which the decode writes directly); default the
-        decoder's own buffer."""
+        decoder's own buffer.  ``q_in``: with ``new_kv``, the queries as they
+        arrive (bf16 [B, Hq, d], possibly pinned host memory, like the new
+        rows), copied into q by the append kernel."""
         dst = self.out if out is None else out
         if self.streams is None:
-            self._step_range(self.shape, q, append_page, p_out, new_kv, None, None, dst)
+            self._step_range(self.shape, q, append_page, p_out, new_kv, None, None, dst, q_in)
             return dst
         cur = torch.cuda.current_stream()
         prev = None
         for shape, st, ev in zip(self.shapes, self.streams, self.scored):
             st.wait_stream(cur)
             with torch.cuda.stream(st):
-                self._step_range(shape, q, append_page, p_out, new_kv, prev, ev, dst)
+                self._step_range(shape, q, append_page, p_out, new_kv, prev, ev, dst, q_in)
             prev = ev
         for st in self.streams:
             cur.wait_stream(st)
         return dst
 
-    def _step_range(self, shape, q, append_page, p_out, new_kv, after, scored, out):
+    def _step_range(self, shape, q, append_page, p_out, new_kv, after, scored, out, q_in=None):
         if new_kv is not None:
             nv.entmaxkv_append(shape, new_kv[0], new_kv[1], self.page_table, self.seq_lens,
-                               self.k_cache, self.v_cache, self.meta)
+                               self.k_cache, self.v_cache, self.meta, q_in, None if q_in is None else q)
         elif append_page is not None:
             nv.entmaxkv_build_meta(shape, self.k_cache, self.page_table, self.seq_lens,
                                    append_page, 1, self.meta)

@@ -84,7 +84,7 @@ def lib():
         L.entmaxkv_workspace_size.argtypes = [sp, C.c_int]
         L.entmaxkv_get_status.argtypes = [C.POINTER(i32), C.c_int, vp]
         L.entmaxkv_build_meta.argtypes = [sp, vp, vp, vp, i32, i32, vp, vp]
-        L.entmaxkv_append.argtypes = [sp, vp, vp, vp, vp, vp, vp, vp, vp]
+        L.entmaxkv_append.argtypes = [sp, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp]
         L.entmaxkv_score_pages.argtypes = [sp, vp, vp, vp, vp, vp, vp, vp]
         L.entmaxkv_select.argtypes = [sp, vp, vp, vp, vp, i32, i32, f32, f32, vp, vp, vp, vp, sz, vp]
         L.entmaxkv_decode_sparse.argtypes = [sp, vp, vp, vp, vp, vp, vp, vp, f32, vp, vp, vp, vp, sz, vp]
@@ -162,12 +162,16 @@ def entmaxkv_build_meta(shape, k_cache, page_table, seq_lens, first_page, n_page
         _stream(stream)))
 
 
-def entmaxkv_append(shape, k_new, v_new, page_table, seq_lens, k_cache, v_cache, meta, stream=None):
+def entmaxkv_append(shape, k_new, v_new, page_table, seq_lens, k_cache, v_cache, meta, q_in=None, q_out=None,
+                    stream=None):
+    """k_new, v_new and q_in may be pinned host tensors (read by the kernel over the bus)."""
     _check("entmaxkv_append", lib().entmaxkv_append(
-        C.byref(shape), _ptr(k_new, torch.bfloat16, "k_new"), _ptr(v_new, torch.bfloat16, "v_new"),
+        C.byref(shape), _ptr(k_new, torch.bfloat16, "k_new", pinned_ok=True),
+        _ptr(v_new, torch.bfloat16, "v_new", pinned_ok=True),
         _ptr(page_table, torch.int32, "page_table"), _ptr(seq_lens, torch.int32, "seq_lens"),
         _ptr(k_cache, torch.bfloat16, "k_cache"), _ptr(v_cache, torch.bfloat16, "v_cache"),
-        _ptr(meta, None, "meta"), _stream(stream)))
+        _ptr(meta, None, "meta"), _ptr(q_in, torch.bfloat16, "q_in", pinned_ok=True),
+        _ptr(q_out, torch.bfloat16, "q_out"), _stream(stream)))
 
 
 def entmaxkv_score_pages(shape, q, meta, seq_lens, bbox, mu=None, sigma=None, stream=None):

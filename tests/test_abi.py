@@ -66,7 +66,7 @@ def test_bad_shapes_rejected_everywhere(bad):
     s = C.byref(shp(**bad))
     E = -2
     assert L.entmaxkv_build_meta(s, FAKE, FAKE, FAKE, 0, -1, FAKE, None) == E
-    assert L.entmaxkv_append(s, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, None) == E
+    assert L.entmaxkv_append(s, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, None, None, None) == E
     assert L.entmaxkv_score_pages(s, FAKE, FAKE, FAKE, FAKE, None, None, None) == E
     assert L.entmaxkv_select(s, FAKE, FAKE, None, None, 0, 4, 1.5, 0.0, FAKE, FAKE, None, None, 0, None) == E
     assert L.entmaxkv_decode_sparse(s, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, 1.5, FAKE, None, None,
@@ -87,10 +87,13 @@ def test_null_alignment_and_argument_codes():
     for i in range(7):
         args = [FAKE] * 7
         args[i] = None
-        assert L.entmaxkv_append(s, *args, None) == -1
-    assert L.entmaxkv_append(s, FAKE, FAKE, FAKE, FAKE, FAKE_ODD, FAKE, FAKE, None) == -8
-    assert L.entmaxkv_append(s, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE_ODD, FAKE, None) == -8
-    assert L.entmaxkv_append(s, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE_ODD, None) == -8
+        assert L.entmaxkv_append(s, *args, None, None, None) == -1
+    assert L.entmaxkv_append(s, FAKE, FAKE, FAKE, FAKE, FAKE_ODD, FAKE, FAKE, None, None, None) == -8
+    assert L.entmaxkv_append(s, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE_ODD, FAKE, None, None, None) == -8
+    assert L.entmaxkv_append(s, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE_ODD, None, None, None) == -8
+    # q_in and q_out come together
+    assert L.entmaxkv_append(s, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, None, None) == -1
+    assert L.entmaxkv_append(s, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, None, FAKE, None) == -1
     assert L.entmaxkv_score_pages(s, FAKE, FAKE, FAKE, FAKE, FAKE, None, None) == -1  # mu w/o sigma
     assert L.entmaxkv_score_pages(s, FAKE, FAKE, None, FAKE, None, None, None) == -1  # no seq_lens
     assert L.entmaxkv_score_pages(s, FAKE_ODD, FAKE, FAKE, FAKE, None, None, None) == -8

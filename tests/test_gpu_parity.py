@@ -483,6 +483,37 @@ def test_decode_output_to_pinned_host_memory():
     assert torch.equal(host_out, dev_out.cpu())
 
 
+def test_append_reads_pinned_host_inputs_and_stages_q():
+    """k_new, v_new and q_in in pinned host memory: the kernel reads them over
+    the bus; the cache, the records and the staged q equal the device-input
+    call's bit for bit."""
+    wl = SMALL["topk_small"]
+    s = shape_of(wl)
+    outs = []
+    for pinned in (False, True):
+        inp, _ = gpu_inputs(wl, 14)
+        meta = nv.alloc_meta(s, "cuda")
+        nv.entmaxkv_build_meta(s, inp["k_cache"], inp["page_table"], inp["seq_lens"], 0, -1, meta)
+        g = torch.Generator().manual_seed(3)
+        k_new = torch.randn(wl.B, wl.Hkv, wl.d, generator=g).to(torch.bfloat16)
+        v_new = torch.randn(wl.B, wl.Hkv, wl.d, generator=g).to(torch.bfloat16)
+        q_in = torch.randn(wl.B, wl.Hq, wl.d, generator=g).to(torch.bfloat16)
+        if pinned:
+            k_new, v_new, q_in = k_new.pin_memory(), v_new.pin_memory(), q_in.pin_memory()
+        else:
+            k_new, v_new, q_in = k_new.cuda(), v_new.cuda(), q_in.cuda()
+        q_out = torch.zeros(wl.B, wl.Hq, wl.d, dtype=torch.bfloat16, device="cuda")
+        nv.get_status(clear=True)
+        nv.entmaxkv_append(s, k_new, v_new, inp["page_table"], inp["seq_lens"], inp["k_cache"], inp["v_cache"], meta,
+                           q_in, q_out)
+        torch.cuda.synchronize()
+        assert nv.get_status(clear=True) == 0
+        assert torch.equal(q_out.cpu().view(torch.int16), q_in.cpu().view(torch.int16))
+        outs.append((inp["k_cache"].view(torch.int16), inp["v_cache"].view(torch.int16), meta))
+    for x, y in zip(*outs):
+        assert torch.equal(x, y)
+
+
 def test_append_bad_page_sets_status_and_skips():
     """A page-table entry outside [0, num_blocks) flags the status and that
     sequence writes nothing; the other sequences append as usual."""
