@@ -144,6 +144,43 @@ def test_sequence_sharded_matches_one_device(name, S):
         assert torch.equal(outs[r], outs[0])
 
 
+@pytest.mark.gpu
+def test_sequence_sharded_full_size_1m_tokens():
+    """The 1M-token Gaussian workload split across two shards (host threads
+    on one device): the same selection and tau as one device, the output
+    within fp32 summation order."""
+    from sparse_entmax_kv_b200 import native as nv
+    from sparse_entmax_kv_b200.decoder import EntmaxKVDecoder
+    from sparse_entmax_kv_b200.sharded import NativeShard, split_context
+    wl = CONFIGS["gauss_gqa_L1m"]
+    inp = make_inputs(wl, 32, device="cuda")
+    dec = EntmaxKVDecoder(inp["k_cache"], inp["v_cache"], inp["page_table"], inp["seq_lens"], wl.Hq,
+                          alpha=wl.alpha, policy=wl.policy, delta=wl.delta)
+    dec.build_meta()
+    nv.get_status(clear=True)
+    dec.step(inp["q"])
+    torch.cuda.synchronize()
+    ref_out, ref_tau, ref_cnt = dec.out.clone(), dec.tau.clone(), dec.cnt.clone()
+    del dec
+    S = 2
+    shards = []
+    for r in range(S):
+        pt, sl, p0 = split_context(inp["page_table"], inp["seq_lens"], wl.P, S, r)
+        sh = NativeShard(inp["k_cache"], inp["v_cache"], pt, sl, inp["seq_lens"], wl.Hq, p0, wl.max_pages,
+                         alpha=wl.alpha, policy=wl.policy, delta=wl.delta, cap=8192)
+        sh.build_meta()
+        shards.append(sh)
+    shared = {"slots": [None] * S, "barrier": threading.Barrier(S, timeout=60)}
+    _BARRIERS[:] = [shared["barrier"]]
+    outs = _run_threads([lambda r=r: sharded_step(shards[r], ThreadComm(shared, r), inp["q"]) for r in range(S)])
+    torch.cuda.synchronize()
+    assert nv.get_status(clear=True) & ~nv.STATUS_OVERFLOW == 0
+    for r in range(S):
+        assert torch.equal(shards[r].cnt, ref_cnt)
+        assert torch.equal(shards[r].tau.view(torch.int32), ref_tau.view(torch.int32))
+        torch.testing.assert_close(outs[r], ref_out, rtol=1e-5, atol=1e-6)
+
+
 # ------------------------------------------------------------------- CPU
 
 class OracleShard:
