@@ -53,11 +53,14 @@ __device__ __forceinline__ void mbar_arrive(uint64_t *bar) {
     asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(smem_u32(bar)) : "memory");
 }
 
-__device__ __forceinline__ bool mbar_test(uint64_t *bar, unsigned parity) {
+// One potentially blocking probe: the thread is suspended until the phase
+// completes or a hardware time limit passes (so a waiting warp does not take
+// issue slots from the warps that compute).
+__device__ __forceinline__ bool mbar_try(uint64_t *bar, unsigned parity) {
     unsigned ok;
     asm volatile(
         "{\n\t.reg .pred p;\n\t"
-        "mbarrier.test_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+        "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
         "selp.u32 %0, 1, 0, p;\n\t}"
         : "=r"(ok)
         : "r"(smem_u32(bar)), "r"(parity)
@@ -68,14 +71,11 @@ __device__ __forceinline__ bool mbar_test(uint64_t *bar, unsigned parity) {
 // Bounded wait for the phase with the given parity.  Returns false (and sets
 // the TIMEOUT status bit) if it did not complete within WAIT_LIMIT_NS.
 __device__ __forceinline__ bool mbar_wait(uint64_t *bar, unsigned parity, int *status) {
-    if (mbar_test(bar, parity)) return true;
-    unsigned long long t0 = globaltimer();
+    if (mbar_try(bar, parity)) return true;
+    const unsigned long long t0 = globaltimer();
     for (unsigned it = 0; it < (1u << 30); ++it) {
-        if (mbar_test(bar, parity)) return true;
-        if ((it & 63u) == 63u) {
-            __nanosleep(64);
-            if (globaltimer() - t0 > WAIT_LIMIT_NS) break;
-        }
+        if (mbar_try(bar, parity)) return true;
+        if (globaltimer() - t0 > WAIT_LIMIT_NS) break;
     }
     if (status) atomicOr(status, ENTMAXKV_STATUS_TIMEOUT);
     return false;
