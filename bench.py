@@ -47,7 +47,7 @@ PAPER_CONTEXT = {"speedup_vs_full_softmax_flashdecoding": 3.36, "speedup_vs_full
 NCU_TRAFFIC = {
     # one full-size launch at L=1,048,576 (201.35 MB read + 5.69 MB written), ncu --set full
     # (profiles/score_kernel_gauss_gqa_L1m_full.md)
-    "score_pages/gauss_gqa_L1m": {"bytes": 201360384 + 6459136, "src": "c014ace8a9b9"},
+    "score_pages/gauss_gqa_L1m": {"bytes": 201355520 + 7096576, "src": "9c6482263062"},
 }
 
 
@@ -67,8 +67,11 @@ def whole_job_gbs(bytes_per_rank, world, step_ms):
 
 
 def _src_hash(fname):
-    p = os.path.join(ROOT, "sparse_entmax_kv_b200", "csrc", fname)
-    return hashlib.sha1(open(p, "rb").read()).hexdigest()[:12]
+    """Hash of a kernel source together with the shared device helpers it includes."""
+    h = hashlib.sha1()
+    for f in (fname, "common.cuh"):
+        h.update(open(os.path.join(ROOT, "sparse_entmax_kv_b200", "csrc", f), "rb").read())
+    return h.hexdigest()[:12]
 
 
 def measured_peaks():

@@ -229,7 +229,8 @@ __device__ __forceinline__ float zmax_of(int n) { return n >= 2 ? sqrtf(2.f * lo
 template <int R>
 __device__ __forceinline__ bool newton_step(float F, float Fp, float hi, float &tau) {
     if (!(F > 1.f + 2e-6f) || !(Fp < 0.f)) return false;
-    const float step = (float)R * (F - powf(F, 1.f - 1.f / (float)R)) / (-Fp);
+    const float Fr = R == 1 ? 1.f : (R == 2 ? sqrtf(F) : powf(F, 1.f - 1.f / (float)R));  // F^(1-1/R)
+    const float step = (float)R * (F - Fr) / (-Fp);
     float nt = tau + step;
     if (!(nt < hi)) nt = 0.5f * (tau + hi);  // stay inside the bracket
     const bool done = !(nt - tau > 1e-7f * fmaxf(1.f, fabsf(tau)));
