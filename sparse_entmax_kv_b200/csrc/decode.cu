@@ -2,25 +2,31 @@
 // summary: section 2.C sparse attention over the selected pages; section 4
 // full-cache entmax and full-cache softmax as comparison points).
 //
-// Sparse path, three launches on one stream, no host round trip:
+// Sparse path, two or three launches on one stream, no host round trip:
 //   union_kernel   per (sequence, kv head), one CTA: union of the G query
 //                  heads' selected pages, ascending, each with a G-bit head
-//                  mask; also resets the per-head maxima.
+//                  mask and its physical block.  Skipped when the q.K grid
+//                  has at most two CTAs per group (many groups): each q.K CTA
+//                  then builds its group's union itself, in its still unused
+//                  ring memory (one page bitmap per head), and writes the
+//                  entries of its own steps.
 //   qk_kernel      split over the union: TMA 2-D loads (128-byte swizzle) of
 //                  the K tiles through a 3-stage mbarrier ring fed by one
-//                  producer warp (which resolves union entries and page-table
-//                  rows 32 steps at a time); z = (alpha-1) q.k/sqrt(d) for all
-//                  G heads of the group from one copy of each tile (tensor-core
+//                  producer warp; z = (alpha-1) q.k/sqrt(d) for all G heads
+//                  of the group from one copy of each tile (tensor-core
 //                  m16n8k16, tokens as M and the heads as N, when G >= 2; CUDA
-//                  cores when G == 1), stored in list order, and the per-head
-//                  max of z.
-//   tau_pv_kernel  per (sequence, query head): every token that can carry
-//                  weight has z > max z - 1 (no weight exceeds 1), so those
-//                  candidates are compacted on chip in list order; the exact
-//                  root of sum (z - tau)_+^r = 1 lies in
-//                  [z_max - 1, z_max - n^(1-alpha)] and is reached by Newton's
-//                  method from the end where it is monotone, and p v is summed
-//                  over the support, reading only those value rows.
+//                  cores when G == 1), stored in list order with the max of
+//                  every 16-token tile.
+//   tau_pv_kernel  per (sequence, query head): max z is the max of the tile
+//                  maxima; every token that can carry weight has
+//                  z > max z - 1 (no weight exceeds 1), so those candidates
+//                  are compacted on chip in list order; the exact root of
+//                  sum (z - tau)_+^r = 1 lies in [z_max - 1, z_max - n^(1-alpha)]
+//                  and is reached by Newton's method from the end where it is
+//                  monotone, and p v is summed over the support, reading only
+//                  those value rows.
+// Sparse softmax (alpha = 1) builds the union with union_kernel and runs
+// softmax_kernel over its pages.
 // Full-cache entmax runs qk_kernel over every page, tau_pv_kernel for tau, and
 // pv_stream_kernel, which streams every V tile through the TMA ring.  Full-cache softmax runs softmax_kernel (K and V
 // tiles per stage, online max / sum per split); both dense paths combine
@@ -60,7 +66,7 @@ __global__ void __launch_bounds__(UTH) union_kernel(DecodeArgs a) {
             c = c < 0 ? 0 : cmax;
         }
         cnts[threadIdx.x] = c;
-        a.ws.zmax[bh] = ORD_NEG_INF;
+        a.ws.zmax[bh] = ORD_NEG_INF;  // the q.K kernel's running max
     }
     if (threadIdx.x == 0) a.ws.counters[bk] = 0;  // the softmax path's last-CTA combine
     __syncthreads();
@@ -189,11 +195,12 @@ __device__ void produce(const DecodeArgs &a, const CUtensorMap *m0, const CUtens
             const int e = (blockIdx.x + it * S) * PPS + i;
             PageInfo r{-1, 0, 0, e, -1};
             if (e < U) {
-                // sparse: the union entry and the block the union kernel resolved
-                // for it, loaded together; dense: page e and its page-table entry
-                const int entry = dense ? ((e << 8) | 0xff) : __ldg(a.ws.union_e + (size_t)bk * a.max_pages + e);
+                // sparse: the union entry and its resolved block, loaded
+                // together (through L2: the q.K kernel writes them itself);
+                // dense: page e and its page-table entry
+                const int entry = dense ? ((e << 8) | 0xff) : __ldcg(a.ws.union_e + (size_t)bk * a.max_pages + e);
                 const int blk = dense ? __ldg(a.page_table + (size_t)b * a.max_pages + e)
-                                      : __ldg(a.ws.union_blk + (size_t)bk * a.max_pages + e);
+                                      : __ldcg(a.ws.union_blk + (size_t)bk * a.max_pages + e);
                 r.page = entry >> 8;
                 r.mask = entry & 0xff;
                 if (blk >= 0 && blk < a.num_blocks) {
@@ -252,6 +259,122 @@ __device__ void produce(const DecodeArgs &a, const CUtensorMap *m0, const CUtens
     }
 }
 
+// ------------------------------------------------------ union in the q.K CTA
+
+// The union of the G heads' selections of group (b, kvh), built by every CTA
+// of the group's q.K grid in shared memory it does not use yet (its ring,
+// which holds G page bitmaps of np bits): each head's entries set bits of its
+// bitmap; the union's pages are then counted in page order (a block scan
+// over the bitmap words), which gives every entry its list position e.  The
+// CTA writes the entries of its own steps (e / PPS = blockIdx.x mod gridDim.x)
+// to the workspace, each with its G-bit head mask and physical block (the
+// page-table loads issued eight at a time), for its producer and for the tau
+// kernel; CTA 0 also writes the count.  Every CTA reads the same lists, so all
+// agree on U and on the positions.  Used when the grid has at most a few CTAs
+// per group (many groups), where the rebuild is not repeated much; all threads
+// call it; it returns U.
+__device__ int union_in_cta(const DecodeArgs &a, int b, int kvh, int bk, int np, int PPS, unsigned *bm, int *s_cnt,
+                            int *s_off, int *sh) {
+    const int G = a.Hq / a.Hkv;
+    const int nt = blockDim.x, S = gridDim.x;
+    const int *selg = a.sel + (size_t)(b * a.Hq + kvh * G) * a.sel_stride;  // head g's list at g * sel_stride
+    const int *pt = a.page_table + (size_t)b * a.max_pages;
+    int *ue = a.ws.union_e + (size_t)bk * a.max_pages;
+    int *ub = a.ws.union_blk + (size_t)bk * a.max_pages;
+    const bool report = blockIdx.x == 0;  // argument errors are flagged by one CTA
+    const int W = ceil_div(np, 32);
+    for (int i = threadIdx.x; i < G * W; i += nt) bm[i] = 0u;
+    if (threadIdx.x < G) {
+        int c = a.cnt[b * a.Hq + kvh * G + threadIdx.x];
+        const int cmax = a.sharded ? a.sel_stride : np;  // sharded: counts over all shards' pages
+        if (c < 0 || c > cmax) {
+            if (report) atomicOr(a.status, ENTMAXKV_STATUS_BAD_SELECTION);
+            c = c < 0 ? 0 : cmax;
+        }
+        s_cnt[threadIdx.x] = c;
+    }
+    __syncthreads();
+    if (threadIdx.x == 0) {
+        s_off[0] = 0;
+        for (int g = 0; g < G; ++g) s_off[g + 1] = s_off[g] + s_cnt[g];
+    }
+    __syncthreads();
+    const int total = s_off[G];  // every head's entries as one flat range
+    // four list entries in flight per thread
+    for (int k0 = threadIdx.x; k0 < total; k0 += 4 * nt) {
+        int p[4], g[4];
+#pragma unroll
+        for (int u = 0; u < 4; ++u) {
+            const int k = k0 + u * nt;
+            p[u] = 0;
+            g[u] = 0;
+            if (k < total) {
+                int gg = 0;
+                while (k >= s_off[gg + 1]) ++gg;
+                g[u] = gg;
+                p[u] = __ldg(selg + (size_t)gg * a.sel_stride + (k - s_off[gg])) - a.page_begin;
+            }
+        }
+#pragma unroll
+        for (int u = 0; u < 4; ++u) {
+            if (k0 + u * nt >= total) continue;
+            if (p[u] >= 0 && p[u] < np)
+                atomicOr(&bm[g[u] * W + (p[u] >> 5)], 1u << (p[u] & 31));
+            else if (report && (a.sharded ? (p[u] + a.page_begin < 0 || p[u] + a.page_begin >= a.sel_stride)
+                                          : true))
+                atomicOr(a.status, ENTMAXKV_STATUS_BAD_SELECTION);  // (sharded: other shards' pages are skipped)
+        }
+    }
+    __syncthreads();
+    // thread t counts the union pages of words [t*wpt, (t+1)*wpt)
+    const int wpt = ceil_div(W, nt);
+    const int w0 = threadIdx.x * wpt;
+    int mine = 0;
+    for (int i = 0; i < wpt && w0 + i < W; ++i) {
+        unsigned u = 0u;
+        for (int g = 0; g < G; ++g) u |= bm[g * W + w0 + i];
+        mine += __popc(u);
+    }
+    int U;
+    int pos = block_excl_scan(mine, sh, &U);
+    int q_page[8], q_e[8], q_mask[8];
+    int nq = 0;
+    auto resolve = [&]() {
+        int blk[8];
+#pragma unroll
+        for (int j = 0; j < 8; ++j) blk[j] = j < nq ? __ldg(pt + q_page[j]) : -1;
+#pragma unroll
+        for (int j = 0; j < 8; ++j)
+            if (j < nq) {
+                const bool ok = blk[j] >= 0 && blk[j] < a.num_blocks;
+                if (!ok) atomicOr(a.status, ENTMAXKV_STATUS_BAD_PAGE);
+                ue[q_e[j]] = (q_page[j] << 8) | q_mask[j];
+                ub[q_e[j]] = ok ? blk[j] : -1;
+            }
+        nq = 0;
+    };
+    for (int i = 0; i < wpt && w0 + i < W; ++i) {
+        const int w = w0 + i;
+        unsigned u = 0u;
+        for (int g = 0; g < G; ++g) u |= bm[g * W + w];
+        while (u) {
+            const int bit = __ffs(u) - 1;
+            u &= u - 1;
+            const int e = pos++;
+            if ((e / PPS) % S != (int)blockIdx.x) continue;  // another CTA's step
+            int mask = 0;
+            for (int g = 0; g < G; ++g) mask |= (int)((bm[g * W + w] >> bit) & 1u) << g;
+            q_page[nq] = 32 * w + bit;
+            q_e[nq] = e;
+            q_mask[nq] = mask;
+            if (++nq == 8) resolve();
+        }
+    }
+    resolve();
+    if (report && threadIdx.x == 0) a.ws.union_cnt[bk] = U;
+    return U;
+}
+
 // ----------------------------------------------------------------- q . K^T
 
 // q.K ring: three stages per CTA and four CTAs per SM (measured: more CTAs
@@ -269,6 +392,7 @@ __global__ void __launch_bounds__(DEC_THREADS) qk_kernel(const __grid_constant__
     extern __shared__ unsigned char smem_raw[];
     RingView<D, G, NS, 1> R(smem_raw);
     __shared__ float qs[G == 1 ? D : 1];
+    __shared__ int s_cnt[8], s_off[9], s_sh[72];
 
     int b, kvh;
     group_of(blockIdx.y, a.kv0, a.nk, b, kvh);
@@ -276,7 +400,19 @@ __global__ void __launch_bounds__(DEC_THREADS) qk_kernel(const __grid_constant__
     const int P = a.P, PPS = TPS / P;
     const int seq = a.seq_lens[b];
     const int np = n_pages_of(seq, P);
-    const int U = DENSE ? np : a.ws.union_cnt[bk];
+    int U = np;
+    if constexpr (!DENSE) {
+        if (a.union_in_qk) {
+            // the union of the group's selections, in the ring's memory
+            U = union_in_cta(a, b, kvh, bk, np, PPS, reinterpret_cast<unsigned *>(R.stages), s_cnt, s_off, s_sh);
+            // the ring's bytes were written through the generic proxy; the TMA
+            // copies that refill them come through the async proxy
+            asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+            __syncthreads();
+        } else {
+            U = a.ws.union_cnt[bk];  // from union_kernel
+        }
+    }
     const int nsteps = ceil_div(U, PPS);
     const int S = gridDim.x;
     const int my_n = nsteps > (int)blockIdx.x ? ceil_div(nsteps - blockIdx.x, S) : 0;
@@ -316,8 +452,6 @@ __global__ void __launch_bounds__(DEC_THREADS) qk_kernel(const __grid_constant__
             }
         }
         const int h0 = 2 * (lane & 3);  // this lane's two heads: h0, h0+1
-        const int bh0 = b * a.Hq + kvh * G + (h0 < G ? h0 : 0);
-        const int bh1 = b * a.Hq + kvh * G + (h0 + 1 < G ? h0 + 1 : 0);
         float run0 = -INFINITY, run1 = -INFINITY;  // this lane's max of z for heads h0, h0+1
         for (int it = 0; it < my_n; ++it) {
             const int st = it % NS, ph = (it / NS) & 1;
@@ -370,13 +504,15 @@ __global__ void __launch_bounds__(DEC_THREADS) qk_kernel(const __grid_constant__
             __syncwarp();
             if (lane == 0) mbar_arrive(&R.empty[st]);
         }
-        if (lane < 4) {
+        // the running max of z per head (reset by the kernel before this one;
+        // with the union built here the tau kernel takes it from the tile maxima)
+        if (lane < 4 && !a.union_in_qk) {
+            const int bh0 = b * a.Hq + kvh * G + h0;
             if (h0 < G && run0 > -INFINITY) atomicMax(&a.ws.zmax[bh0], f2ord(run0));
-            if (h0 + 1 < G && run1 > -INFINITY) atomicMax(&a.ws.zmax[bh1], f2ord(run1));
+            if (h0 + 1 < G && run1 > -INFINITY) atomicMax(&a.ws.zmax[bh0 + 1], f2ord(run1));
         }
     } else {
         // G == 1: thread per token, q broadcast from shared memory
-        const int bh = b * a.Hq + kvh;
         float run = -INFINITY;
         const int ti = threadIdx.x;  // token within the stage
         for (int it = 0; it < my_n; ++it) {
@@ -418,9 +554,11 @@ __global__ void __launch_bounds__(DEC_THREADS) qk_kernel(const __grid_constant__
             __syncwarp();
             if (lane == 0) mbar_arrive(&R.empty[st]);
         }
+        if (!a.union_in_qk) {
 #pragma unroll
-        for (int o = 16; o; o >>= 1) run = fmaxf(run, __shfl_xor_sync(FULL, run, o));
-        if (lane == 0 && run > -INFINITY) atomicMax(&a.ws.zmax[bh], f2ord(run));
+            for (int o = 16; o; o >>= 1) run = fmaxf(run, __shfl_xor_sync(FULL, run, o));
+            if (lane == 0 && run > -INFINITY) atomicMax(&a.ws.zmax[b * a.Hq + kvh], f2ord(run));
+        }
     }
 }
 
@@ -531,12 +669,62 @@ __global__ void __launch_bounds__(TAU_NT, D == 64 ? 4 : 3) tau_pv_kernel(const _
     const int bk = b * a.Hkv + kvh;
     const int P = a.P;
     const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+    // max z of the head: the q.K kernel's running max, or, when the q.K CTAs
+    // built the union themselves (nothing reset the running max), the max of
+    // the tile maxima; in the sequence-sharded phases the global max z comes
+    // in (and the candidates phase writes out this shard's candidate z values)
+    const bool zmax_from_tiles = !a.zmax_in && a.union_in_qk;
+    const int zord = a.zmax_in || zmax_from_tiles ? 0 : a.ws.zmax[bh];
     const int np = n_pages_of(a.seq_lens[b], P);
     const int U = dense ? np : a.ws.union_cnt[bk];
     const int n_tok = U * P;  // a multiple of 16
-    // sequence-sharded phases: the global max z and tau come in; the
-    // candidates phase writes out this shard's candidate z values
-    const float zmax = a.zmax_in ? a.zmax_in[bh] : ord2f(a.ws.zmax[bh]);
+    const size_t trow = tile_row(a, b, h);
+    const float *tr = a.ws.tmax + trow;
+    const int n_tiles = n_tok / 16;
+    const bool tvec = (trow & 3) == 0;
+    // this thread's TAU_TB tile maxima of the round starting at tile t0
+    auto load_tiles = [&](int t0, float(&v)[TAU_TB]) {
+        const int p0 = t0 + threadIdx.x * TAU_TB;
+        if (tvec && p0 + TAU_TB <= n_tiles) {
+#pragma unroll
+            for (int i = 0; i < TAU_TB / 4; ++i) {
+                const float4 f = __ldcg(reinterpret_cast<const float4 *>(tr + p0) + i);
+                v[4 * i] = f.x;
+                v[4 * i + 1] = f.y;
+                v[4 * i + 2] = f.z;
+                v[4 * i + 3] = f.w;
+            }
+        } else {
+#pragma unroll
+            for (int i = 0; i < TAU_TB; ++i) v[i] = p0 + i < n_tiles ? __ldcg(tr + p0 + i) : -INFINITY;
+        }
+    };
+    float v0[TAU_TB];  // the first round's tile maxima, kept for the candidate pass
+    load_tiles(0, v0);
+    float zmax;
+    if (a.zmax_in) {
+        zmax = a.zmax_in[bh];
+    } else if (!zmax_from_tiles) {
+        zmax = ord2f(zord);
+    } else {
+        __shared__ float s_wmax[TAU_NW];
+        float m = -INFINITY;
+#pragma unroll
+        for (int i = 0; i < TAU_TB; ++i) m = fmaxf(m, v0[i]);
+        for (int t0 = TAU_NT * TAU_TB; t0 < n_tiles; t0 += TAU_NT * TAU_TB) {
+            float v[TAU_TB];
+            load_tiles(t0, v);
+#pragma unroll
+            for (int i = 0; i < TAU_TB; ++i) m = fmaxf(m, v[i]);
+        }
+#pragma unroll
+        for (int o = 16; o; o >>= 1) m = fmaxf(m, __shfl_xor_sync(FULL, m, o));
+        if (lane == 0) s_wmax[warp] = m;
+        __syncthreads();
+        zmax = s_wmax[0];
+#pragma unroll
+        for (int w = 1; w < TAU_NW; ++w) zmax = fmaxf(zmax, s_wmax[w]);
+    }
     const bool given_tau = a.tau_in != nullptr;
     const bool export_cand = a.cand_z != nullptr;
     const float r = 1.f / (a.alpha - 1.f);
@@ -558,8 +746,6 @@ __global__ void __launch_bounds__(TAU_NT, D == 64 ? 4 : 3) tau_pv_kernel(const _
     // with tau known, z > tau
     const float thr = given_tau ? a.tau_in[bh] : zmax - 1.f;
     const float *zr = a.ws.zbuf + tok_row(a, b, h);
-    const size_t trow = tile_row(a, b, h);
-    const float *tr = a.ws.tmax + trow;
     auto row_of_pos = [&](int pos) -> int {
         const int up = pos / P, t = pos - up * P;
         const int blk = dense ? __ldg(a.page_table + (size_t)b * a.max_pages + up)
@@ -572,24 +758,15 @@ __global__ void __launch_bounds__(TAU_NT, D == 64 ? 4 : 3) tau_pv_kernel(const _
     // maxima per thread, loaded together), then their tokens (one tile per
     // thread: its 16 z and, for the gather, its page's value row, loaded
     // together).
-    const int n_tiles = n_tok / 16;
-    const bool tvec = (trow & 3) == 0;
     int ntc = 0;
     for (int t0 = 0; t0 < n_tiles; t0 += TAU_NT * TAU_TB) {
         const int p0 = t0 + threadIdx.x * TAU_TB;
         float v[TAU_TB];
-        if (tvec && p0 + TAU_TB <= n_tiles) {
+        if (t0 == 0) {
 #pragma unroll
-            for (int i = 0; i < TAU_TB / 4; ++i) {
-                const float4 f = __ldcg(reinterpret_cast<const float4 *>(tr + p0) + i);
-                v[4 * i] = f.x;
-                v[4 * i + 1] = f.y;
-                v[4 * i + 2] = f.z;
-                v[4 * i + 3] = f.w;
-            }
+            for (int i = 0; i < TAU_TB; ++i) v[i] = v0[i];
         } else {
-#pragma unroll
-            for (int i = 0; i < TAU_TB; ++i) v[i] = p0 + i < n_tiles ? __ldcg(tr + p0 + i) : -INFINITY;
+            load_tiles(t0, v);
         }
         unsigned bits = 0;
 #pragma unroll
@@ -808,15 +985,32 @@ __global__ void __launch_bounds__(TAU_NT, D == 64 ? 4 : 3) tau_pv_kernel(const _
 
 // ------------------------------------------- sequence-sharded decode pieces
 
-// Per head: the shard's max z (after q.K) as a float, -inf when it has none.
-__global__ void zmax_export_kernel(DecodeArgs a) {
+// Per head: the shard's max z (after q.K): the q.K kernel's running max, or,
+// when the q.K CTAs built the union themselves, the max of the 16-token tile
+// maxima; -inf when it has none.  One CTA per head.
+constexpr int ZX_NT = 128;
+__global__ void __launch_bounds__(ZX_NT) zmax_export_kernel(DecodeArgs a) {
     pdl_wait();
+    __shared__ float s_wmax[ZX_NT / 32];
     const int G = a.Hq / a.Hkv;
-    const int i = blockIdx.x * blockDim.x + threadIdx.x;
-    if (i >= a.B * a.nk * G) return;
     int b, h;
-    head_of(i, a.kv0 * G, a.nk * G, b, h);
-    a.zmax_out[b * a.Hq + h] = ord2f(a.ws.zmax[b * a.Hq + h]);
+    head_of(blockIdx.x, a.kv0 * G, a.nk * G, b, h);
+    if (!a.union_in_qk) {
+        if (threadIdx.x == 0) a.zmax_out[b * a.Hq + h] = ord2f(a.ws.zmax[b * a.Hq + h]);
+        return;
+    }
+    const int n_tiles = a.ws.union_cnt[b * a.Hkv + h / G] * a.P / 16;
+    const float *tr = a.ws.tmax + tile_row(a, b, h);
+    float m = -INFINITY;
+    for (int i = threadIdx.x; i < n_tiles; i += ZX_NT) m = fmaxf(m, __ldcg(tr + i));
+#pragma unroll
+    for (int o = 16; o; o >>= 1) m = fmaxf(m, __shfl_xor_sync(FULL, m, o));
+    if ((threadIdx.x & 31) == 0) s_wmax[threadIdx.x >> 5] = m;
+    __syncthreads();
+    if (threadIdx.x == 0) {
+        for (int w = 1; w < ZX_NT / 32; ++w) m = fmaxf(m, s_wmax[w]);
+        a.zmax_out[b * a.Hq + h] = fmaxf(m, s_wmax[0]);
+    }
 }
 
 // Per head: the exact threshold over the candidates of all S shards (each
@@ -1234,34 +1428,56 @@ cudaError_t launch_qk(const DecodeArgs &a, cudaStream_t st) {
     return launch_pdl(k, dim3(S, groups), dim3(DEC_THREADS), RG::BYTES, st, a);
 }
 
+// The union of each group's selections for the sparse q.K pass.  With at
+// most UNION_IN_QK_SPLITS q.K CTAs per group (many groups) each CTA builds its
+// group's union itself (union_in_cta) when the G page bitmaps fit in its ring;
+// otherwise union_kernel builds it first, once per group, rather than every
+// CTA of a wide split repeating it.  Returns the arguments for q.K and the
+// kernels after it, with the choice recorded.
+constexpr int UNION_IN_QK_SPLITS = 2;
+
+template <int D, int G>
+cudaError_t launch_union(const DecodeArgs &a, cudaStream_t st, DecodeArgs &out) {
+    using RG = Ring<D, G, QK_NS, 1>;
+    out = a;
+    const int groups = a.B * a.nk;
+    const int S = pick_splits(a.sms, QK_PER_SM, groups, ceil_div(a.max_pages, RG::TPS / a.P), 1 << 16);
+    const bool fits = (size_t)G * ceil_div(a.max_pages, 32) * 4 <= (size_t)QK_NS * RG::STAGE;
+    out.union_in_qk = S <= UNION_IN_QK_SPLITS && fits;
+    if (out.union_in_qk) return cudaSuccess;
+    return launch_pdl(union_kernel, dim3(groups), dim3(UTH), 0, st, out);
+}
+
 template <int D, int G>
 cudaError_t sparse_t(const DecodeArgs &a, cudaStream_t st) {
     cudaError_t e;
     const int groups = a.B * a.nk;
-    if ((e = launch_pdl(union_kernel, dim3(groups), dim3(UTH), 0, st, a)) != cudaSuccess) return e;
     if (a.alpha == 1.f) {
-        // softmax over the selected pages: K and V of the union, split over pages
+        // softmax over the selected pages: the union, then K and V of its
+        // pages, split over pages
+        if ((e = launch_pdl(union_kernel, dim3(groups), dim3(UTH), 0, st, a)) != cudaSuccess) return e;
         using RG = Ring<D, G, 3, 2>;
         auto k = softmax_kernel<D, G, true>;
         if ((e = set_smem(k, RG::BYTES)) != cudaSuccess) return e;
         const int S = pick_splits(a.sms, 2, groups, ceil_div(a.max_pages, RG::TPS / a.P), MAX_SPLITS);
         return launch_pdl(k, dim3(S, groups), dim3(DEC_THREADS), RG::BYTES, st, a);
     }
-    if ((e = launch_qk<D, G, false>(a, st)) != cudaSuccess) return e;
+    DecodeArgs u;
+    if ((e = launch_union<D, G>(a, st, u)) != cudaSuccess) return e;
+    if ((e = launch_qk<D, G, false>(u, st)) != cudaSuccess) return e;
     const int nheads = a.B * a.nk * (a.Hq / a.Hkv);
     const int zcap = tau_zcap(nheads, a.sms);
     if ((e = set_smem(tau_pv_kernel<D, true>, tau_smem(ZCAP_MAX))) != cudaSuccess) return e;
-    return launch_pdl(tau_pv_kernel<D, true>, dim3(nheads), dim3(TAU_NT), tau_smem(zcap), st, a, 0, zcap);
+    return launch_pdl(tau_pv_kernel<D, true>, dim3(nheads), dim3(TAU_NT), tau_smem(zcap), st, u, 0, zcap);
 }
 
 template <int D, int G>
 cudaError_t begin_t(const DecodeArgs &a, cudaStream_t st) {
     cudaError_t e;
-    const int groups = a.B * a.nk;
-    if ((e = launch_pdl(union_kernel, dim3(groups), dim3(UTH), 0, st, a)) != cudaSuccess) return e;
-    if ((e = launch_qk<D, G, false>(a, st)) != cudaSuccess) return e;
-    const int n = a.B * a.nk * G;
-    return launch_pdl(zmax_export_kernel, dim3(ceil_div(n, 256)), dim3(256), 0, st, a);
+    DecodeArgs u;
+    if ((e = launch_union<D, G>(a, st, u)) != cudaSuccess) return e;
+    if ((e = launch_qk<D, G, false>(u, st)) != cudaSuccess) return e;
+    return launch_pdl(zmax_export_kernel, dim3(a.B * a.nk * G), dim3(ZX_NT), 0, st, u);
 }
 
 template <int D, int G>

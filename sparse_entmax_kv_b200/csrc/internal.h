@@ -91,7 +91,7 @@ struct DecodeWs {
     int *union_e;    // [B*Hkv][max_pages]   (page << 8) | head mask (sparse)
     int *union_blk;  // [B*Hkv][max_pages]   physical block of each union entry (sparse)
     int *union_cnt;  // [B*Hkv]
-    int *zmax;       // [B*Hq] order-mapped max z
+    int *zmax;       // [B*Hq] order-mapped max z (when union_kernel or the dense init resets it)
     float *tau;      // [B*Hq]
     int *counters;   // [B*Hkv] last-CTA combine counters
     float *partial;  // [MAX_SPLITS][B*Hq][d+2]  (dense paths)
@@ -117,6 +117,7 @@ struct DecodeArgs {
     // are skipped); the global max z / tau per head come in, the shard's max z
     // and candidate z values go out
     int sharded, page_begin, sel_stride;
+    int union_in_qk;  // sparse q.K: each CTA builds the group's union itself (set by the launcher)
     const float *zmax_in, *tau_in;
     float *zmax_out;
     float *cand_z;

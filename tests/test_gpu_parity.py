@@ -45,6 +45,12 @@ SMALL = {
                          k=20, keys="offset", needles=3, ragged=True),
     "gqa8_d128": Workload("gqa8_d128", B=1, Hq=8, Hkv=1, d=128, L=2000, P=64, alpha=2.0, policy="gauss",
                           delta=0.25, keys="cluster", needles=2, ragged=True),
+    # 320 (sequence, kv head) groups: the q.K grid has one CTA per group, and
+    # each q.K CTA builds its group's union of selected pages itself
+    "groups320_gqa": Workload("groups320_gqa", B=40, Hq=16, Hkv=8, d=128, L=1500, P=32, alpha=1.5,
+                              policy="topk", k=12, keys="offset", needles=3, ragged=True),
+    "groups320_mha": Workload("groups320_mha", B=80, Hq=4, Hkv=4, d=64, L=700, P=16, alpha=1.5,
+                              policy="gauss", delta=0.5, keys="cluster", needles=2, ragged=True),
 }
 
 
@@ -375,6 +381,17 @@ def test_decode_sparse_long_sequence_small_pages():
     assert wl.max_pages > 32768
     inp, host = gpu_inputs(wl, 12)
     _sparse_vs_oracle(wl, inp, host, "topk", wl.k, "long_p16")
+
+
+def test_decode_sparse_union_over_several_chunks():
+    """A group of eight query heads (d = 64) over 61,443 pages: the union of
+    the heads' selections is built 16,384 pages at a time, so the list
+    positions run on across four chunks."""
+    wl = Workload("union_chunks", B=1, Hq=8, Hkv=1, d=64, L=61443 * 16 - 8, P=16, alpha=1.5, policy="topk",
+                  k=48, keys="offset", needles=6, needle_scale=4.0)
+    assert wl.max_pages > 2 * 24576
+    inp, host = gpu_inputs(wl, 14)
+    _sparse_vs_oracle(wl, inp, host, "topk", wl.k, "union_chunks")
 
 
 def test_decode_sparse_all_tokens_candidates():

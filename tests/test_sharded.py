@@ -38,6 +38,9 @@ SMALL = {
                                                    ragged=True, needles=8),
     "mha_small": CONFIGS["sweep_mha_L64k"].shrink(name="mha_small", B=3, Hq=4, Hkv=4, L=2048,
                                                   ragged=True, needles=4),
+    # 320 groups: each q.K CTA builds its group's union of selected pages
+    "groups320": Workload("groups320", B=40, Hq=16, Hkv=8, d=128, L=1500, P=32, alpha=1.5, policy="topk",
+                          k=12, keys="offset", needles=3, ragged=True),
 }
 
 
