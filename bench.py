@@ -45,9 +45,9 @@ PAPER_CONTEXT = {"speedup_vs_full_softmax_flashdecoding": 3.36, "speedup_vs_full
 # DRAM bytes per launch from ncu captures (dram__bytes_read.sum + dram__bytes_write.sum),
 # keyed by kernel and workload, valid only while the kernel source is unchanged.
 NCU_TRAFFIC = {
-    # one full-size launch at L=1,048,576 (201.35 MB read + 5.69 MB written), ncu --set full
+    # one full-size launch at L=1,048,576 (201.38 MB read + 6.32 MB written), ncu --set full
     # (profiles/score_kernel_gauss_gqa_L1m_full.md)
-    "score_pages/gauss_gqa_L1m": {"bytes": 201355520 + 7096576, "src": "9c6482263062"},
+    "score_pages/gauss_gqa_L1m": {"bytes": 201378048 + 6317312, "src": "7a36380605cc"},
 }
 
 
@@ -378,7 +378,7 @@ def run_gpu(args, rank, world):
                stage_us=stage_us, dense=dense, nbytes=nbytes, clocks=clocks,
                roofline=roofline, roofline_gather=roofline_gather, e2e_ms=e2e_step_ms, e2e_bytes=(stage_host.numel() * 2,
                                                                out_host.numel() * 4),
-               launches=kernels_per_step(policy == "gauss", True) * args.steps, t_wall=t_wall,
+               launches=kernels_per_step(dec.shape, wl.alpha, True) * args.steps, t_wall=t_wall,
                host=dict(inp=inp, dec=dec) if (rank == 0 and not args.no_cpu_baseline) else None)
     return res
 

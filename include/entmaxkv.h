@@ -282,6 +282,16 @@ ENTMAXKV_API int entmaxkv_decode_sparse(const entmaxkv_shape *shape, const void 
                            void *workspace, size_t ws_bytes, void *stream);
 
 /*
+ * The number of kernels one entmaxkv_decode_sparse call with this shape and
+ * alpha launches on the current device (2 or 3: the union of each GQA group's
+ * selections is built by its own kernel, or inside the q.K kernel when that
+ * kernel has at most two CTAs per group), for callers that count launches or
+ * size CUDA graphs.  Negative ENTMAXKV_ERR_* on a bad shape or alpha < 1.
+ * Launches nothing.
+ */
+ENTMAXKV_API int entmaxkv_decode_sparse_kernels(const entmaxkv_shape *shape, float alpha);
+
+/*
  * Allocation-free form of entmaxkv_decode_sparse (the EntmaxKV summary has no
  * counterpart; this is a library convenience).  Same arguments, results and
  * errors, minus the workspace: the scratch lives in a fixed array of

@@ -401,6 +401,26 @@ int entmaxkv_decode_sparse(const entmaxkv_shape *s, const void *q, const void *k
     return cuda_rc(launch_decode_sparse(a, static_cast<cudaStream_t>(stream)));
 }
 
+int entmaxkv_decode_sparse_kernels(const entmaxkv_shape *s, float alpha) {
+    int rc = check_shape(s);
+    if (rc) return rc;
+    if (!(alpha >= 1.f)) return ENTMAXKV_ERR_ALPHA;
+    DevInfo di;
+    if ((rc = device_info(&di))) return rc;
+    DecodeArgs a;
+    std::memset(&a, 0, sizeof(a));
+    a.B = s->B;
+    a.Hq = s->Hq;
+    a.Hkv = s->Hkv;
+    a.d = s->d;
+    a.P = s->page_size;
+    a.max_pages = s->max_pages;
+    a.alpha = alpha;
+    a.sms = di.sms;
+    kv_range(s, &a.kv0, &a.nk);
+    return decode_sparse_kernels(a);
+}
+
 int entmaxkv_decode_sparse_begin(const entmaxkv_shape *s, const void *q, const void *k_cache, const void *v_cache,
                                  const int32_t *page_table, const int32_t *seq_lens, const int32_t *sel,
                                  const int32_t *cnt, int32_t sel_max_pages, int32_t page_begin, float alpha,

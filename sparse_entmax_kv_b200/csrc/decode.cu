@@ -1437,15 +1437,27 @@ cudaError_t launch_qk(const DecodeArgs &a, cudaStream_t st) {
 constexpr int UNION_IN_QK_SPLITS = 2;
 
 template <int D, int G>
-cudaError_t launch_union(const DecodeArgs &a, cudaStream_t st, DecodeArgs &out) {
+bool union_in_qk_for(const DecodeArgs &a) {
     using RG = Ring<D, G, QK_NS, 1>;
-    out = a;
-    const int groups = a.B * a.nk;
-    const int S = pick_splits(a.sms, QK_PER_SM, groups, ceil_div(a.max_pages, RG::TPS / a.P), 1 << 16);
+    const int S = pick_splits(a.sms, QK_PER_SM, a.B * a.nk, ceil_div(a.max_pages, RG::TPS / a.P), 1 << 16);
     const bool fits = (size_t)G * ceil_div(a.max_pages, 32) * 4 <= (size_t)QK_NS * RG::STAGE;
-    out.union_in_qk = S <= UNION_IN_QK_SPLITS && fits;
+    return S <= UNION_IN_QK_SPLITS && fits;
+}
+
+template <int D, int G>
+cudaError_t launch_union(const DecodeArgs &a, cudaStream_t st, DecodeArgs &out) {
+    out = a;
+    out.union_in_qk = union_in_qk_for<D, G>(a);
     if (out.union_in_qk) return cudaSuccess;
-    return launch_pdl(union_kernel, dim3(groups), dim3(UTH), 0, st, out);
+    return launch_pdl(union_kernel, dim3(a.B * a.nk), dim3(UTH), 0, st, out);
+}
+
+// Kernels one sparse decode launches: softmax (union, softmax_kernel), or
+// entmax ([union,] q.K, tau with p.V).
+template <int D, int G>
+int sparse_kernels_t(const DecodeArgs &a) {
+    if (a.alpha == 1.f) return 2;
+    return union_in_qk_for<D, G>(a) ? 2 : 3;
 }
 
 template <int D, int G>
@@ -1555,6 +1567,26 @@ cudaError_t dense_softmax_t(const DecodeArgs &a, cudaStream_t st) {
     } while (0)
 
 cudaError_t launch_decode_sparse(const DecodeArgs &a, cudaStream_t st) { EKV_DISPATCH(sparse_t, a, st); }
+
+int decode_sparse_kernels(const DecodeArgs &a) {
+    const int G = a.Hq / a.Hkv;
+    if (a.d == 64) {
+        switch (G) {
+            case 1: return sparse_kernels_t<64, 1>(a);
+            case 2: return sparse_kernels_t<64, 2>(a);
+            case 4: return sparse_kernels_t<64, 4>(a);
+            case 8: return sparse_kernels_t<64, 8>(a);
+        }
+    } else {
+        switch (G) {
+            case 1: return sparse_kernels_t<128, 1>(a);
+            case 2: return sparse_kernels_t<128, 2>(a);
+            case 4: return sparse_kernels_t<128, 4>(a);
+            case 8: return sparse_kernels_t<128, 8>(a);
+        }
+    }
+    return -1;
+}
 cudaError_t launch_decode_sparse_begin(const DecodeArgs &a, cudaStream_t st) { EKV_DISPATCH(begin_t, a, st); }
 cudaError_t launch_decode_sparse_candidates(const DecodeArgs &a, cudaStream_t st) {
     EKV_DISPATCH(candidates_t, a, st);

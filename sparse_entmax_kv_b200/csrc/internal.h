@@ -126,6 +126,7 @@ struct DecodeArgs {
     int *status;
 };
 cudaError_t launch_decode_sparse(const DecodeArgs &a, cudaStream_t st);
+int decode_sparse_kernels(const DecodeArgs &a);  // launches of one launch_decode_sparse
 cudaError_t launch_decode_sparse_begin(const DecodeArgs &a, cudaStream_t st);
 cudaError_t launch_decode_sparse_candidates(const DecodeArgs &a, cudaStream_t st);
 cudaError_t launch_decode_sparse_finish(const DecodeArgs &a, cudaStream_t st);

@@ -54,8 +54,11 @@ constexpr size_t smem_bytes() {
            (size_t)WARPS * Ring<GAUSS>::NST * Ring<GAUSS>::STAGE;
 }
 
+// Two CTAs per SM for the Gaussian policy (its 6 KB stages fill shared
+// memory); three for top-k (2 KB stages), whose bounds-only stream does the
+// same fp64 work per chunk on a third of the bytes and gains from more warps.
 template <int D, int G, bool GAUSS>
-__global__ void __launch_bounds__(THREADS, G <= 4 ? 2 : 1) score_kernel(ScoreArgs a) {
+__global__ void __launch_bounds__(THREADS, G <= 4 ? (GAUSS ? 2 : 3) : 1) score_kernel(ScoreArgs a) {
     pdl_wait();
     using RG = Ring<GAUSS>;
     constexpr int NCH = D / CHK;

@@ -115,7 +115,7 @@ def last_token_rows(k_cache, v_cache, page_table, seq_lens):
     return k_cache[blk, :, tok].contiguous(), v_cache[blk, :, tok].contiguous()
 
 
-def kernels_per_step(policy_gauss: bool, append: bool) -> int:
-    """Kernel launches one ``step`` issues: append or build_meta (1, if appending),
-    score (1), select (1), decode_sparse (union, q.K, tau with p.V = 3)."""
-    return (1 if append else 0) + 1 + 1 + 3
+def kernels_per_step(shape, alpha: float, append: bool) -> int:
+    """Kernel launches one ``step`` issues: append (1, if appending), score (1),
+    select (1) and decode_sparse (2 or 3, as the library reports for the shape)."""
+    return (1 if append else 0) + 1 + 1 + nv.entmaxkv_decode_sparse_kernels(shape, alpha)

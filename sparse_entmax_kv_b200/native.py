@@ -29,7 +29,8 @@ EXPORTED = ("entmaxkv_strerror", "entmaxkv_version", "entmaxkv_meta_bytes",
             "entmaxkv_workspace_size", "entmaxkv_get_status", "entmaxkv_build_meta", "entmaxkv_append",
             "entmaxkv_score_pages", "entmaxkv_select", "entmaxkv_decode_sparse",
             "entmaxkv_decode_sparse_static", "entmaxkv_decode_dense", "entmaxkv_decode_sparse_begin",
-            "entmaxkv_decode_sparse_candidates", "entmaxkv_entmax_threshold", "entmaxkv_decode_sparse_finish")
+            "entmaxkv_decode_sparse_candidates", "entmaxkv_entmax_threshold", "entmaxkv_decode_sparse_finish",
+            "entmaxkv_decode_sparse_kernels")
 
 
 class EntmaxKVError(RuntimeError):
@@ -202,6 +203,13 @@ def entmaxkv_decode_sparse(shape, q, k_cache, v_cache, page_table, seq_lens, sel
         float(alpha), _ptr(out, torch.float32, "out", pinned_ok=True), _ptr(tau_out, torch.float32, "tau_out"),
         _ptr(p_out, torch.float32, "p_out"), _ptr(workspace, None, "workspace"),
         0 if workspace is None else workspace.numel(), _stream(stream)))
+
+
+def entmaxkv_decode_sparse_kernels(shape, alpha):
+    """Kernel launches of one entmaxkv_decode_sparse call for this shape."""
+    n = lib().entmaxkv_decode_sparse_kernels(C.byref(shape), float(alpha))
+    _check("entmaxkv_decode_sparse_kernels", min(n, 0))
+    return n
 
 
 def _kv_args(q, k_cache, v_cache, page_table, seq_lens):

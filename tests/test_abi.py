@@ -24,7 +24,7 @@ def _declared():
 def test_library_exports_every_declared_symbol():
     L = nv.lib()
     names = _declared()
-    assert len(names) == 16
+    assert len(names) == 17
     assert set(names) == set(nv.EXPORTED)
     for n in names:
         assert hasattr(L, n)
@@ -41,6 +41,12 @@ def shp(**kw):
     d = dict(B=2, Hq=8, Hkv=2, d=128, page_size=32, max_pages=64, num_blocks=128, kv_begin=0, kv_count=0)
     d.update(kw)
     return nv.Shape(*[d[f] for f, _ in nv.Shape._fields_])
+
+
+def test_decode_sparse_kernels_checks_its_arguments():
+    L = nv.lib()
+    assert L.entmaxkv_decode_sparse_kernels(C.byref(shp(Hq=6, Hkv=4)), C.c_float(1.5)) == -2  # ERR_SHAPE
+    assert L.entmaxkv_decode_sparse_kernels(C.byref(shp()), C.c_float(0.5)) == -3              # ERR_ALPHA
 
 
 def test_sizes():

@@ -394,6 +394,17 @@ def test_decode_sparse_union_over_several_chunks():
     _sparse_vs_oracle(wl, inp, host, "topk", wl.k, "union_chunks")
 
 
+def test_decode_sparse_kernel_count():
+    """The library's own count of a sparse decode's launches: a separate union
+    kernel when the q.K grid splits each group widely, none when every group
+    has one q.K CTA (the q.K CTAs build the union), two for softmax."""
+    wide = shape_of(CONFIGS["gauss_gqa_L1m"])                      # 8 groups
+    narrow = shape_of(SMALL["groups320_gqa"])                      # 320 groups
+    assert nv.entmaxkv_decode_sparse_kernels(wide, 1.5) == 3
+    assert nv.entmaxkv_decode_sparse_kernels(narrow, 1.5) == 2
+    assert nv.entmaxkv_decode_sparse_kernels(wide, 1.0) == 2
+
+
 def test_decode_sparse_all_tokens_candidates():
     """Equal keys put every selected token within 1 of the max z, more
     candidates than a head holds on chip: the exact path that rescans the z
