@@ -95,6 +95,7 @@ def lib():
         L.entmaxkv_decode_sparse_candidates.argtypes = [sp, vp, vp, vp, vp, vp, f32, vp, i32, vp, vp, vp, sz, vp]
         L.entmaxkv_entmax_threshold.argtypes = [sp, i32, i32, vp, vp, vp, f32, vp, vp]
         L.entmaxkv_decode_sparse_finish.argtypes = [sp, vp, vp, vp, vp, vp, f32, vp, vp, vp, vp, vp, sz, vp]
+        L.entmaxkv_decode_sparse_kernels.argtypes = [sp, f32]
         for fn in EXPORTED:
             if fn not in ("entmaxkv_strerror", "entmaxkv_version", "entmaxkv_meta_bytes",
                           "entmaxkv_workspace_size"):

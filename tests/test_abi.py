@@ -47,6 +47,8 @@ def test_decode_sparse_kernels_checks_its_arguments():
     L = nv.lib()
     assert L.entmaxkv_decode_sparse_kernels(C.byref(shp(Hq=6, Hkv=4)), C.c_float(1.5)) == -2  # ERR_SHAPE
     assert L.entmaxkv_decode_sparse_kernels(C.byref(shp()), C.c_float(0.5)) == -3              # ERR_ALPHA
+    with pytest.raises(nv.EntmaxKVError, match="ERR_ALPHA"):  # through the binding
+        nv.entmaxkv_decode_sparse_kernels(shp(), 0.5)
 
 
 def test_sizes():
