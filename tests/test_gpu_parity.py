@@ -51,6 +51,10 @@ SMALL = {
                               policy="topk", k=12, keys="offset", needles=3, ragged=True),
     "groups320_mha": Workload("groups320_mha", B=80, Hq=4, Hkv=4, d=64, L=700, P=16, alpha=1.5,
                               policy="gauss", delta=0.5, keys="cluster", needles=2, ragged=True),
+    # 200 groups: two q.K CTAs per group, each building the union and writing
+    # the entries of every other step
+    "groups200_gqa": Workload("groups200_gqa", B=25, Hq=32, Hkv=8, d=64, L=1200, P=16, alpha=2.0,
+                              policy="topk", k=16, keys="offset", needles=3, ragged=True),
 }
 
 
@@ -400,8 +404,10 @@ def test_decode_sparse_kernel_count():
     has one q.K CTA (the q.K CTAs build the union), two for softmax."""
     wide = shape_of(CONFIGS["gauss_gqa_L1m"])                      # 8 groups
     narrow = shape_of(SMALL["groups320_gqa"])                      # 320 groups
+    two = shape_of(SMALL["groups200_gqa"])                          # 200 groups
     assert nv.entmaxkv_decode_sparse_kernels(wide, 1.5) == 3
     assert nv.entmaxkv_decode_sparse_kernels(narrow, 1.5) == 2
+    assert nv.entmaxkv_decode_sparse_kernels(two, 1.5) == 2
     assert nv.entmaxkv_decode_sparse_kernels(wide, 1.0) == 2
 
 
