@@ -29,6 +29,7 @@ import os
 import statistics
 import subprocess
 import sys
+import tempfile
 import time
 
 import numpy as np
@@ -85,9 +86,9 @@ def measured_peaks():
 class ClockSampler:
     """nvidia-smi clock / throttle sampling while the timed region runs."""
 
-    def __init__(self, index):
+    def __init__(self, index, directory=None):
         self.proc = None
-        self.path = os.path.join(ROOT, "gpurun_out", f"clocks_rank{index}.csv")
+        self.path = os.path.join(directory or tempfile.gettempdir(), f"entmaxkv_clocks_rank{index}.csv")
         self.index = index
 
     def __enter__(self):
@@ -230,7 +231,7 @@ def run_gpu(args, rank, world):
     # The timed region lasts milliseconds, far below nvidia-smi's sampling
     # period, so clocks are sampled over a loaded window that brackets it:
     # warm-up steps for >= 1 s before, untimed steps for >= 0.5 s after.
-    with ClockSampler(dev.index) as clk:
+    with ClockSampler(dev.index, args.clocks_dir) as clk:
         t0 = time.perf_counter()
         i = 0
         while i < args.warmup or time.perf_counter() - t0 < 1.0:
@@ -607,6 +608,8 @@ def main():
     ap.add_argument("--dense-steps", type=int, default=5)
     ap.add_argument("--skip-dense", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--clocks-dir", default=None,
+                    help="where the nvidia-smi clock samples of the timed region are kept (default: temp dir)")
     ap.add_argument("--quality", action="store_true",
                     help="instead of the benchmark line: sparse vs full-cache error, entmax vs softmax at one kept set")
     ap.add_argument("--l-sweep", action="store_true",
