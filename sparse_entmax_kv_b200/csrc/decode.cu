@@ -266,13 +266,13 @@ __device__ void produce(const DecodeArgs &a, const CUtensorMap *m0, const CUtens
 // which holds G page bitmaps of np bits): each head's entries set bits of its
 // bitmap; the union's pages are then counted in page order (a block scan
 // over the bitmap words), which gives every entry its list position e.  The
-// CTA writes the entries of its own steps (e / PPS = blockIdx.x mod gridDim.x)
-// to the workspace, each with its G-bit head mask and physical block (the
-// page-table loads issued eight at a time), for its producer and for the tau
-// kernel; CTA 0 also writes the count.  Every CTA reads the same lists, so all
-// agree on U and on the positions.  Used when the grid has at most a few CTAs
-// per group (many groups), where the rebuild is not repeated much; all threads
-// call it; it returns U.
+// CTA writes the entries of its own steps (step e / PPS, owned by CTA
+// step mod gridDim.x) to the workspace, each with its G-bit head mask and
+// physical block (the page-table loads issued eight at a time), for its
+// producer and for the tau kernel; CTA 0 also writes the count.  Every CTA
+// reads the same lists, so all agree on U and on the positions.  Used when the
+// grid has at most two CTAs per group (many groups), where the rebuild is
+// repeated little; all threads call it; it returns U.
 __device__ int union_in_cta(const DecodeArgs &a, int b, int kvh, int bk, int np, int PPS, unsigned *bm, int *s_cnt,
                             int *s_off, int *sh) {
     const int G = a.Hq / a.Hkv;
