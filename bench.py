@@ -44,10 +44,10 @@ PAPER_CONTEXT = {"speedup_vs_full_softmax_flashdecoding": 3.36, "speedup_vs_full
                  "source": "EntmaxKV summary, section 4 (Efficiency)"}
 
 # DRAM bytes per launch from ncu captures (dram__bytes_read.sum + dram__bytes_write.sum),
-# keyed by kernel and workload, valid only while the kernel source is unchanged.
+# keyed by kernel and workload, valid only while the kernel source is unchanged
+# (the source hash below); the line reports null traffic once it has changed.
 NCU_TRAFFIC = {
     # one full-size launch at L=1,048,576 (201.38 MB read + 6.32 MB written), ncu --set full
-    # (profiles/score_kernel_gauss_gqa_L1m_full.md)
     "score_pages/gauss_gqa_L1m": {"bytes": 201378048 + 6317312, "src": "7a36380605cc"},
 }
 
@@ -363,12 +363,16 @@ def run_gpu(args, rank, world):
     # dominant kernel of the step: score_pages is a single launch (the sparse
     # decode stage is three kernels and is reported beside it)
     dom = "score_pages"
-    alg = nbytes["meta"] + nbytes["scores"] + wl.B * wl.Hq * wl.d * 2
+    # algorithmic bytes of the scan: the metadata records and the queries; the
+    # page scores it writes are reported beside them as actual bytes
+    alg = nbytes["meta"] + wl.B * wl.Hq * wl.d * 2
+    actual = alg + nbytes["scores"]
     achieved = alg / (stage_us[dom] * 1e-6) / 1e9
     tr = NCU_TRAFFIC.get(f"{dom}/{args.workload}")
     traffic = tr["bytes"] if tr and tr.get("src") == _src_hash("score.cu") else None  # null once the kernel changed
     roofline = {"bound": "hbm", "kernel": dom, "achieved": round(achieved, 1), "peak": peak, "unit": "GB/s",
                 "frac": round(achieved / peak, 4), "traffic": traffic, "algorithmic_bytes": alg,
+                "actual_bytes": actual,
                 "peak_kind": f"{peak_kind} copy bandwidth (burst)"}
     galg = nbytes["gather_k"] + nbytes["gather_v"] + nbytes["qo"]
     gach = galg / (stage_us["decode_sparse"] * 1e-6) / 1e9

@@ -31,15 +31,21 @@
  *   return means nothing was enqueued.  ENTMAXKV_ERR_CUDA reports a failed
  *   launch (cudaGetLastError).
  * - Errors the host cannot see (a page-table entry outside [0, num_blocks), a
- *   selected page index outside the sequence, a wait that ran out) are
- *   recorded in a per-device status word (ENTMAXKV_STATUS_* bits, OR-ed) read
- *   with entmaxkv_get_status.  Kernels never trap; the offending page is
- *   skipped.
+ *   selected page index outside the sequence, a sequence length above
+ *   max_pages * P, a non-finite query, a wait that ran out) are recorded in a
+ *   per-device status word (ENTMAXKV_STATUS_* bits, OR-ed) read with
+ *   entmaxkv_get_status.  Kernels never trap; the offending page is skipped,
+ *   an over-long sequence is clamped to max_pages * P tokens.
+ * - Non-finite queries: a query row (b, h) holding a NaN or +-Inf gets NaN
+ *   scores from entmaxkv_score_pages (bbox, mu and sigma of every page), and
+ *   out[b][h][*] = NaN, tau_out[b][h] = NaN from every decode call; the call
+ *   sets ENTMAXKV_STATUS_NONFINITE.  Other heads are computed as usual.
  * - Layouts (row-major, all contiguous):
  *     k_cache, v_cache  bf16  [num_blocks][Hkv][P][d]   16-byte aligned
  *     q                 bf16  [B][Hq][d]                 16-byte aligned
  *     page_table        int32 [B][max_pages]  logical page -> physical block
- *     seq_lens          int32 [B]             tokens per sequence (<= max_pages*P)
+ *     seq_lens          int32 [B]             tokens per sequence (<= max_pages*P;
+ *                                             longer: ENTMAXKV_STATUS_BAD_LENGTH)
  *   Query head h reads kv head h / G, G = Hq / Hkv.  Sequence b has
  *   N_b = ceil(seq_lens[b] / P) pages; page p holds min(P, seq_lens[b] - p*P)
  *   valid tokens.  Scores are s = q.k / sqrt(d); entmax uses z = (alpha-1) s
@@ -113,8 +119,13 @@ enum {
     ENTMAXKV_STATUS_BAD_PAGE = 1,      /* page_table entry outside [0, num_blocks) */
     ENTMAXKV_STATUS_BAD_SELECTION = 2, /* sel entry outside [0, N_b) or cnt > N_b */
     ENTMAXKV_STATUS_TIMEOUT = 4,       /* an on-device wait hit its limit */
-    ENTMAXKV_STATUS_OVERFLOW = 8       /* a candidate list overflowed on-chip storage
+    ENTMAXKV_STATUS_OVERFLOW = 8,      /* a candidate list overflowed on-chip storage
                                           (handled by a slower exact path) */
+    ENTMAXKV_STATUS_BAD_LENGTH = 16,   /* seq_lens[b] > max_pages * P: the sequence was
+                                          treated as max_pages * P tokens long
+                                          (entmaxkv_append skips it instead) */
+    ENTMAXKV_STATUS_NONFINITE = 32     /* a query row held a NaN or an infinity: that
+                                          head's scores and output are NaN */
 };
 
 /* Text for an ENTMAXKV_* return code. Static storage; never NULL. */
@@ -165,6 +176,18 @@ ENTMAXKV_API size_t entmaxkv_workspace_size(const entmaxkv_shape *shape, int cal
 ENTMAXKV_API int entmaxkv_get_status(int32_t *status_out, int clear, void *stream);
 
 /*
+ * Diagnostic with no counterpart in the EntmaxKV summary: launch one kernel
+ * whose single thread waits on an mbarrier that nothing ever arrives at,
+ * through the same bounded wait that every pipelined kernel of the library
+ * uses, with the limit limit_ns (1 .. 2e9 nanoseconds of the GPU's global
+ * timer, else ENTMAXKV_ERR_SHAPE).  When the limit passes the kernel sets
+ * ENTMAXKV_STATUS_TIMEOUT and returns, so the stream and the context stay
+ * usable: a caller can check that an on-device wait that runs out is
+ * reported instead of hanging.  No copy is in flight during the wait.
+ */
+ENTMAXKV_API int entmaxkv_selftest_wait(uint64_t limit_ns, void *stream);
+
+/*
  * Section 2.A (bounding box and Gaussian statistics, "maintained on append"):
  * for each sequence b, each logical page p in [first_page, first_page+n_pages)
  * with p < N_b (n_pages = -1: to the end), and each kv head, recompute the
@@ -190,8 +213,9 @@ ENTMAXKV_API int entmaxkv_build_meta(const entmaxkv_shape *shape, const void *k_
  * (L-1) mod P of block page_table[b][(L-1)/P] of k_cache / v_cache, then
  * rebuild the metadata record of logical page (L-1)/P exactly as
  * entmaxkv_build_meta does (same bits).  Sequences with L <= 0 are skipped.  A
- * page-table entry outside [0, num_blocks), or (L-1)/P >= max_pages, sets
- * ENTMAXKV_STATUS_BAD_PAGE and skips that sequence.  If q_in and q_out are
+ * page-table entry outside [0, num_blocks) sets ENTMAXKV_STATUS_BAD_PAGE, and
+ * L > max_pages * P sets ENTMAXKV_STATUS_BAD_LENGTH; either skips that
+ * sequence.  If q_in and q_out are
  * both given (bf16 [B][Hq][d]), the step's queries of the kv heads in range
  * are copied from q_in to q_out as well (one of them NULL without the other:
  * ENTMAXKV_ERR_NULL).  k_new, v_new and q_in may be pinned host memory
@@ -211,9 +235,13 @@ ENTMAXKV_API int entmaxkv_append(const entmaxkv_shape *shape, const void *k_new,
  *   bbox[b][h][p]  = fp32( (sum_j max(q_j kmin_j, q_j kmax_j)) / sqrt(d) )
  *   mu[b][h][p]    = fp32( (sum_j q_j mean_j) / sqrt(d) )
  *   sigma[b][h][p] = fp32( sqrt( (sum_j q_j^2 var_j) / d ) )
- * bbox bounds every token score s of the page from above.  Each sum runs in
- * fp64 over j in index order (products are exact), so results are defined to
- * the bit.  Outputs are fp32 [B][Hq][max_pages]; entries for p >= N_b are not
+ * bbox bounds every token score s of the page from above.  Its sum runs in
+ * fp64 over j in index order (every product is exact there) and is rounded
+ * once, so the bound is defined to the bit.  mu and sigma feed only the
+ * approximate threshold tau_hat of the Gaussian policies; their sums are
+ * fp32, accurate to the forward error bound of a d-term fp32 dot product
+ * (|error| <= 2 d 2^-24 sum_j |term_j|, plus the final rounding), not to the
+ * bit.  Outputs are fp32 [B][Hq][max_pages]; entries for p >= N_b are not
  * written.  mu and sigma may both be NULL (bound only, reads 4d bytes per
  * page and kv head instead of 12d); if one is non-NULL both must be.  The
  * metadata is addressed by logical page, so no page table is needed; pages
@@ -243,7 +271,9 @@ ENTMAXKV_API int entmaxkv_score_pages(const entmaxkv_shape *shape, const void *q
  *                  subset of ENTMAXKV_GAUSS's pages; unlike it, it can drop a
  *                  page holding a support token.
  * sel is int32 [B][Hq][max_pages], cnt int32 [B][Hq].  Needs alpha > 1 for
- * the Gaussian policies.  workspace may be NULL when entmaxkv_workspace_size
+ * the Gaussian policies.  Non-finite scores (a non-finite query): top-k ranks
+ * NaN above every number (ties to the lower page index); the Gaussian
+ * policies keep no page when tau_hat is NaN.  workspace may be NULL when entmaxkv_workspace_size
  * reports 0.
  */
 ENTMAXKV_API int entmaxkv_select(const entmaxkv_shape *shape, const int32_t *seq_lens,

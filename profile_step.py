@@ -1,7 +1,7 @@
 """Run a few decode steps of a workload for profiling (ncu) with no timing logic.
 
-  python -m sparse_entmax_kv_b200.profile_step --workload gauss_gqa_L1m --steps 2 [--dense]
-  python -m sparse_entmax_kv_b200.profile_step --workload gauss_gqa_L1m --steps 3 --score-only
+  python profile_step.py --workload gauss_gqa_L1m --steps 2 [--dense]
+  python profile_step.py --workload gauss_gqa_L1m --steps 3 --score-only
 
 Launch order per step: append (each sequence's newest token again), score_pages, select,
 decode_sparse (union, q.K, tau, p.V); with --dense, one full-cache entmax and
@@ -11,12 +11,16 @@ the metadata build and each step is one score_pages call, so a profiler that
 saves and restores device memory between passes handles only the metadata.
 """
 import argparse
+import os
+import sys
 
 import torch
 
-from . import native as nv
-from .decoder import EntmaxKVDecoder, last_token_rows
-from .workloads import CONFIGS, make_inputs
+sys.path.insert(0, os.path.dirname(os.path.abspath(__file__)))
+
+from sparse_entmax_kv_b200 import native as nv  # noqa: E402
+from sparse_entmax_kv_b200.decoder import EntmaxKVDecoder, last_token_rows  # noqa: E402
+from sparse_entmax_kv_b200.workloads import CONFIGS, make_inputs  # noqa: E402
 
 
 def main():

@@ -140,6 +140,17 @@ int integer_r(float alpha) {
 
 int cuda_rc(cudaError_t e) { return e == cudaSuccess ? ENTMAXKV_OK : ENTMAXKV_ERR_CUDA; }
 
+// Thread 0 waits on an mbarrier of its own that nothing arrives at (no copy
+// is in flight), through the bounded wait every pipelined kernel uses, with
+// the given limit; it sets ENTMAXKV_STATUS_TIMEOUT when the limit passes.
+__global__ void wait_selftest_kernel(unsigned long long limit_ns, int *status) {
+    __shared__ uint64_t bar;
+    if (threadIdx.x != 0) return;
+    mbar_init(&bar, 1);
+    mbar_fence_init();
+    mbar_wait_for(&bar, 0, status, limit_ns);
+}
+
 }  // namespace
 
 extern "C" {
@@ -193,6 +204,15 @@ int entmaxkv_get_status(int32_t *status_out, int clear, void *stream) {
     if (clear && cudaMemsetAsync(di.status, 0, sizeof(int), st) != cudaSuccess) return ENTMAXKV_ERR_CUDA;
     *status_out = v;
     return ENTMAXKV_OK;
+}
+
+int entmaxkv_selftest_wait(uint64_t limit_ns, void *stream) {
+    if (limit_ns == 0 || limit_ns > WAIT_LIMIT_NS) return ENTMAXKV_ERR_SHAPE;
+    DevInfo di;
+    int rc = device_info(&di);
+    if (rc) return rc;
+    wait_selftest_kernel<<<1, 32, 0, static_cast<cudaStream_t>(stream)>>>(limit_ns, di.status);
+    return cuda_rc(cudaGetLastError());
 }
 
 int entmaxkv_build_meta(const entmaxkv_shape *s, const void *k_cache, const int32_t *page_table,

@@ -69,16 +69,23 @@ __device__ __forceinline__ bool mbar_try(uint64_t *bar, unsigned parity) {
 }
 
 // Bounded wait for the phase with the given parity.  Returns false (and sets
-// the TIMEOUT status bit) if it did not complete within WAIT_LIMIT_NS.
-__device__ __forceinline__ bool mbar_wait(uint64_t *bar, unsigned parity, int *status) {
+// the TIMEOUT status bit) if it did not complete within limit_ns nanoseconds
+// of %globaltimer (or 2^30 probes, whichever comes first).
+__device__ __forceinline__ bool mbar_wait_for(uint64_t *bar, unsigned parity, int *status,
+                                              unsigned long long limit_ns) {
     if (mbar_try(bar, parity)) return true;
     const unsigned long long t0 = globaltimer();
     for (unsigned it = 0; it < (1u << 30); ++it) {
         if (mbar_try(bar, parity)) return true;
-        if (globaltimer() - t0 > WAIT_LIMIT_NS) break;
+        if (globaltimer() - t0 > limit_ns) break;
     }
     if (status) atomicOr(status, ENTMAXKV_STATUS_TIMEOUT);
     return false;
+}
+
+// The kernels' waits: bounded by WAIT_LIMIT_NS.
+__device__ __forceinline__ bool mbar_wait(uint64_t *bar, unsigned parity, int *status) {
+    return mbar_wait_for(bar, parity, status, WAIT_LIMIT_NS);
 }
 
 // -------------------------------------------------------- bulk / TMA copies
@@ -233,6 +240,30 @@ constexpr int ORD_NEG_INF = (int)(0xff800000u ^ 0x7fffffffu);  // f2ord(-inf)
 __host__ __device__ __forceinline__ int ceil_div(int a, int b) { return (a + b - 1) / b; }
 
 __device__ __forceinline__ int n_pages_of(int seq_len, int P) { return seq_len > 0 ? (seq_len + P - 1) / P : 0; }
+
+// Tokens of sequence b as every kernel uses them: seq_lens[b] clamped to
+// [0, max_pages * P].  A longer length is a caller error the host cannot see
+// (the lengths live on the device); thread 0 of each CTA that meets one sets
+// ENTMAXKV_STATUS_BAD_LENGTH, and the sequence is treated as max_pages * P
+// tokens long, so no kernel indexes past a row of max_pages pages.
+__device__ __forceinline__ int seq_len_of(const int *seq_lens, int b, int P, int max_pages, int *status) {
+    const int s = seq_lens[b];
+    const int cap = max_pages * P;
+    if (s > cap) {
+        if (threadIdx.x == 0 && status) atomicOr(status, ENTMAXKV_STATUS_BAD_LENGTH);
+        return cap;
+    }
+    return s < 0 ? 0 : s;
+}
+
+// True when every bf16 value of the d-element query row is finite (a bf16 is
+// NaN or +-Inf exactly when its eight exponent bits are all ones).
+__device__ __forceinline__ bool q_row_finite(const uint16_t *q, int d) {
+    bool ok = true;
+    for (int j = 0; j < d; ++j) ok &= (q[j] & 0x7f80u) != 0x7f80u;
+    return ok;
+}
+
 __device__ __forceinline__ int tokens_in_page(int seq_len, int P, int p) {
     int n = seq_len - p * P;
     return n > P ? P : (n < 0 ? 0 : n);

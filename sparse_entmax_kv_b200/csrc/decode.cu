@@ -56,7 +56,7 @@ __global__ void __launch_bounds__(UTH) union_kernel(DecodeArgs a) {
     group_of(blockIdx.x, a.kv0, a.nk, b, kvh);
     const int bk = b * a.Hkv + kvh;
     const int G = a.Hq / a.Hkv;
-    const int np = n_pages_of(a.seq_lens[b], a.P);
+    const int np = n_pages_of(seq_len_of(a.seq_lens, b, a.P, a.max_pages, a.status), a.P);
     if (threadIdx.x < G) {
         const int bh = b * a.Hq + kvh * G + threadIdx.x;
         int c = a.cnt[bh];
@@ -182,7 +182,7 @@ __device__ void produce(const DecodeArgs &a, const CUtensorMap *m0, const CUtens
                         unsigned char *stages, uint64_t *full, uint64_t *empty, PageInfo *pinfo, PageInfo *stash,
                         float *zst = nullptr, int TPS = 0) {
     const int lane = threadIdx.x & 31;
-    const int seq = a.seq_lens[b];
+    const int seq = seq_len_of(a.seq_lens, b, a.P, a.max_pages, nullptr);  // (flagged by the caller kernel)
     const int S = gridDim.x;
     if (lane == 0) {
         prefetch_tmap(m0);
@@ -398,7 +398,7 @@ __global__ void __launch_bounds__(DEC_THREADS) qk_kernel(const __grid_constant__
     group_of(blockIdx.y, a.kv0, a.nk, b, kvh);
     const int bk = b * a.Hkv + kvh;
     const int P = a.P, PPS = TPS / P;
-    const int seq = a.seq_lens[b];
+    const int seq = seq_len_of(a.seq_lens, b, P, a.max_pages, a.status);
     const int np = n_pages_of(seq, P);
     int U = np;
     if constexpr (!DENSE) {
@@ -669,13 +669,30 @@ __global__ void __launch_bounds__(TAU_NT, D == 64 ? 4 : 3) tau_pv_kernel(const _
     const int bk = b * a.Hkv + kvh;
     const int P = a.P;
     const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+    const bool given_tau = a.tau_in != nullptr;
+    const bool export_cand = a.cand_z != nullptr;
+    // a query with a NaN or an infinity: NaN output and threshold, no candidates
+    if (!__syncthreads_and(threadIdx.x >= D || (a.q[(size_t)bh * D + threadIdx.x] & 0x7f80u) != 0x7f80u)) {
+        if (threadIdx.x == 0) atomicOr(a.status, ENTMAXKV_STATUS_NONFINITE);
+        if (export_cand) {
+            if (threadIdx.x == 0) a.cand_n[bh] = 0;
+            return;
+        }
+        if (GATHER)
+            for (int j = threadIdx.x; j < D; j += TAU_NT) a.out[(size_t)bh * D + j] = __int_as_float(0x7fc00000);
+        if (threadIdx.x == 0 && !given_tau) {
+            a.ws.tau[bh] = __int_as_float(0x7fc00000);
+            if (a.tau_out) a.tau_out[bh] = __int_as_float(0x7fc00000);
+        }
+        return;
+    }
     // max z of the head: the q.K kernel's running max, or, when the q.K CTAs
     // built the union themselves (nothing reset the running max), the max of
     // the tile maxima; in the sequence-sharded phases the global max z comes
     // in (and the candidates phase writes out this shard's candidate z values)
     const bool zmax_from_tiles = !a.zmax_in && a.union_in_qk;
     const int zord = a.zmax_in || zmax_from_tiles ? 0 : a.ws.zmax[bh];
-    const int np = n_pages_of(a.seq_lens[b], P);
+    const int np = n_pages_of(seq_len_of(a.seq_lens, b, P, a.max_pages, a.status), P);
     const int U = dense ? np : a.ws.union_cnt[bk];
     const int n_tok = U * P;  // a multiple of 16
     const size_t trow = tile_row(a, b, h);
@@ -725,8 +742,6 @@ __global__ void __launch_bounds__(TAU_NT, D == 64 ? 4 : 3) tau_pv_kernel(const _
 #pragma unroll
         for (int w = 1; w < TAU_NW; ++w) zmax = fmaxf(zmax, s_wmax[w]);
     }
-    const bool given_tau = a.tau_in != nullptr;
-    const bool export_cand = a.cand_z != nullptr;
     const float r = 1.f / (a.alpha - 1.f);
     const int ri = a.r_int;
     if (!(zmax > -INFINITY) || (given_tau && !(a.tau_in[bh] == a.tau_in[bh]))) {  // no token at all
@@ -1066,16 +1081,30 @@ __global__ void __launch_bounds__(TAU_NT) threshold_kernel(const __grid_constant
 template <int D, int G>
 __device__ __forceinline__ void combine_last(const DecodeArgs &a, int bk, int b, int kvh, int S, bool softmax) {
     __shared__ int s_last;
+    __shared__ unsigned s_qbad;  // bit g: head g's query is not finite (its output is NaN)
     __threadfence();
     __syncthreads();
     if (threadIdx.x == 0) s_last = atomicAdd(&a.ws.counters[bk], 1) == S - 1;
     __syncthreads();
     if (!s_last) return;
     __threadfence();
+    if (threadIdx.x == 0) {
+        unsigned m = 0u;
+        for (int g = 0; g < G; ++g)
+            if (!q_row_finite(a.q + ((size_t)b * a.Hq + kvh * G + g) * D, D)) m |= 1u << g;
+        s_qbad = m;
+        if (m) atomicOr(a.status, ENTMAXKV_STATUS_NONFINITE);
+    }
+    __syncthreads();
     const int BH = a.B * a.Hq;
     for (int i = threadIdx.x; i < G * D; i += blockDim.x) {
         const int g = i / D, j = i % D;
         const int bh = b * a.Hq + kvh * G + g;
+        if ((s_qbad >> g) & 1u) {
+            a.out[(size_t)bh * D + j] = __int_as_float(0x7fc00000);
+            if (j == 0 && softmax && a.tau_out) a.tau_out[bh] = __int_as_float(0x7fc00000);
+            continue;
+        }
         if (!softmax) {
             float s = 0.f;
             for (int sl = 0; sl < S; ++sl) s += __ldcg(&a.ws.partial[((size_t)sl * BH + bh) * (D + 2) + 2 + j]);
@@ -1128,7 +1157,7 @@ __global__ void __launch_bounds__(DEC_THREADS) pv_stream_kernel(const __grid_con
     group_of(blockIdx.y, a.kv0, a.nk, b, kvh);
     const int bk = b * a.Hkv + kvh;
     const int P = a.P, PPS = TPS / P;
-    const int seq = a.seq_lens[b];
+    const int seq = seq_len_of(a.seq_lens, b, P, a.max_pages, a.status);
     const int np = n_pages_of(seq, P);
     const int nsteps = ceil_div(np, PPS);
     const int S = gridDim.x;
@@ -1236,7 +1265,7 @@ __global__ void __launch_bounds__(DEC_THREADS) softmax_kernel(const __grid_const
     group_of(blockIdx.y, a.kv0, a.nk, b, kvh);
     const int bk = b * a.Hkv + kvh;
     const int P = a.P, PPS = TPS / P;
-    const int seq = a.seq_lens[b];
+    const int seq = seq_len_of(a.seq_lens, b, P, a.max_pages, a.status);
     const int np = n_pages_of(seq, P);
     const int U = SPARSE ? a.ws.union_cnt[bk] : np;  // pages to read: the group's union, or all
     const int nsteps = ceil_div(U, PPS);

@@ -70,7 +70,7 @@ __global__ void __launch_bounds__(D) build_meta_kernel(MetaArgs a) {
     const int b = blockIdx.y;
     const int kvh = a.kv0 + blockIdx.z;
     const int p = a.first_page + blockIdx.x;
-    const int seq = a.seq_lens[b];
+    const int seq = seq_len_of(a.seq_lens, b, P, a.max_pages, a.status);
     if (p >= n_pages_of(seq, P)) return;
     const int blk = a.page_table[(size_t)b * a.max_pages + p];
     if (blk < 0 || blk >= a.num_blocks) {
@@ -100,7 +100,7 @@ __global__ void __launch_bounds__(D) append_kernel(AppendArgs a) {
     if (seq <= 0) return;
     const int p = (seq - 1) / P, t = (seq - 1) % P;
     if (p >= a.m.max_pages) {
-        if (threadIdx.x == 0) atomicOr(a.m.status, ENTMAXKV_STATUS_BAD_PAGE);
+        if (threadIdx.x == 0) atomicOr(a.m.status, ENTMAXKV_STATUS_BAD_LENGTH);
         return;
     }
     const int blk = a.m.page_table[(size_t)b * a.m.max_pages + p];

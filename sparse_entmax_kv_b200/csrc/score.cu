@@ -73,17 +73,23 @@ __global__ void __launch_bounds__(THREADS, G <= 4 ? (GAUSS ? 2 : 3) : 1) score_k
     group_of(blockIdx.y, a.kv0, a.nk, b, kvh);
     const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
 
+    __shared__ unsigned q_bad;  // bit g: head g's query has a NaN or an infinity
+    if (threadIdx.x == 0) q_bad = 0u;
+    __syncthreads();
     for (int i = threadIdx.x; i < G * D; i += THREADS) {
         const int g = i / D, j = i % D;
         const float v = bf16f(a.q[((size_t)b * a.Hq + kvh * G + g) * D + j]);
+        if (!isfinite(v)) atomicOr(&q_bad, 1u << g);
         qq[j * G + g] = make_double2(v < 0.f ? (double)v : 0.0, v > 0.f ? (double)v : 0.0);
         qh[g * D + j] = v;
     }
     if (threadIdx.x < WARPS * NST) mbar_init(&bars[threadIdx.x], 1);
     mbar_fence_init();
     __syncthreads();
+    const unsigned bad = q_bad;
+    if (bad && threadIdx.x == 0 && blockIdx.x == 0) atomicOr(a.status, ENTMAXKV_STATUS_NONFINITE);
 
-    const int np = n_pages_of(a.seq_lens[b], a.P);
+    const int np = n_pages_of(seq_len_of(a.seq_lens, b, a.P, a.max_pages, a.status), a.P);
     const int tile = blockIdx.x * WARPS + warp;
     const int page0 = tile * TP;
     if (page0 >= np) return;  // whole warp past the end
@@ -166,13 +172,15 @@ __global__ void __launch_bounds__(THREADS, G <= 4 ? (GAUSS ? 2 : 3) : 1) score_k
     if (!ok || page >= np) return;
     const double inv_sqrt_d = __ddiv_rn(1.0, __dsqrt_rn((double)D));
     const float inv_sqrt_df = D == 64 ? 0.125f : 0.08838834764831845f;
+    const float qnan = __int_as_float(0x7fc00000);
 #pragma unroll
     for (int g = 0; g < G; ++g) {
         const size_t o = ((size_t)b * a.Hq + kvh * G + g) * a.max_pages + page;
-        a.bbox[o] = (float)__dmul_rn(ab[g], inv_sqrt_d);
+        const bool hb = (bad >> g) & 1u;
+        a.bbox[o] = hb ? qnan : (float)__dmul_rn(ab[g], inv_sqrt_d);
         if (GAUSS) {
-            a.mu[o] = (am[g].x + am[g].y) * inv_sqrt_df;
-            a.sigma[o] = sqrtf((av[g].x + av[g].y) * (1.f / (float)D));
+            a.mu[o] = hb ? qnan : (am[g].x + am[g].y) * inv_sqrt_df;
+            a.sigma[o] = hb ? qnan : sqrtf((av[g].x + av[g].y) * (1.f / (float)D));
         }
     }
 }

@@ -53,7 +53,7 @@ __global__ void __launch_bounds__(NT) topk_kernel(SelectArgs a) {
     int b, h;
     head_of(blockIdx.x, a.h0, a.nh, b, h);
     const int bh = b * a.Hq + h;
-    const int n = n_pages_of(a.seq_lens[b], a.P);
+    const int n = n_pages_of(seq_len_of(a.seq_lens, b, a.P, a.max_pages, a.status), a.P);
     const float *sc = a.bbox + (size_t)bh * a.max_pages;
     int *sel = a.sel + (size_t)bh * a.max_pages;
     const int k = min(a.k, n);
@@ -255,7 +255,7 @@ __global__ void __launch_bounds__(SEL_THREADS) gauss_kernel(SelectArgs a) {
     int b, h;
     head_of(blockIdx.x, a.h0, a.nh, b, h);
     const int bh = b * a.Hq + h;
-    const int seq = a.seq_lens[b];
+    const int seq = seq_len_of(a.seq_lens, b, a.P, a.max_pages, a.status);
     const int n = n_pages_of(seq, a.P);
     const size_t row = (size_t)bh * a.max_pages;
     const float a1 = a.alpha - 1.f;
@@ -453,7 +453,7 @@ __global__ void __cluster_dims__(GCL, 1, 1) __launch_bounds__(GTH) gauss_cluster
     int b, h;
     head_of(blockIdx.x / GCL, a.h0, a.nh, b, h);
     const int bh = b * a.Hq + h;
-    const int seq = a.seq_lens[b];
+    const int seq = seq_len_of(a.seq_lens, b, a.P, a.max_pages, a.status);
     const int n = n_pages_of(seq, a.P);
     const size_t row = (size_t)bh * a.max_pages;
     const float a1 = a.alpha - 1.f;

@@ -24,13 +24,14 @@ STATIC_SCRATCH_BYTES = 16 << 20
 TOPK, GAUSS, GAUSS_EST = 0, 1, 2
 CALL_SELECT, CALL_DECODE_SPARSE, CALL_DECODE_DENSE = 2, 3, 4
 STATUS_BAD_PAGE, STATUS_BAD_SELECTION, STATUS_TIMEOUT, STATUS_OVERFLOW = 1, 2, 4, 8
+STATUS_BAD_LENGTH, STATUS_NONFINITE = 16, 32
 
 EXPORTED = ("entmaxkv_strerror", "entmaxkv_version", "entmaxkv_meta_bytes",
             "entmaxkv_workspace_size", "entmaxkv_get_status", "entmaxkv_build_meta", "entmaxkv_append",
             "entmaxkv_score_pages", "entmaxkv_select", "entmaxkv_decode_sparse",
             "entmaxkv_decode_sparse_static", "entmaxkv_decode_dense", "entmaxkv_decode_sparse_begin",
             "entmaxkv_decode_sparse_candidates", "entmaxkv_entmax_threshold", "entmaxkv_decode_sparse_finish",
-            "entmaxkv_decode_sparse_kernels")
+            "entmaxkv_decode_sparse_kernels", "entmaxkv_selftest_wait")
 
 
 class EntmaxKVError(RuntimeError):
@@ -96,6 +97,7 @@ def lib():
         L.entmaxkv_entmax_threshold.argtypes = [sp, i32, i32, vp, vp, vp, f32, vp, vp]
         L.entmaxkv_decode_sparse_finish.argtypes = [sp, vp, vp, vp, vp, vp, f32, vp, vp, vp, vp, vp, sz, vp]
         L.entmaxkv_decode_sparse_kernels.argtypes = [sp, f32]
+        L.entmaxkv_selftest_wait.argtypes = [C.c_uint64, vp]
         for fn in EXPORTED:
             if fn not in ("entmaxkv_strerror", "entmaxkv_version", "entmaxkv_meta_bytes",
                           "entmaxkv_workspace_size"):
@@ -149,6 +151,12 @@ def alloc_workspace(shape: Shape, call: int, device) -> torch.Tensor:
     if n == (1 << 64) - 1:
         raise EntmaxKVError("entmaxkv_workspace_size", -2, "invalid shape or call")
     return torch.empty(max(n, 1), dtype=torch.uint8, device=device)
+
+
+def entmaxkv_selftest_wait(limit_ns: int, stream=None):
+    """One bounded on-device wait that nothing ends: the kernel returns after
+    limit_ns nanoseconds and sets STATUS_TIMEOUT."""
+    _check("entmaxkv_selftest_wait", lib().entmaxkv_selftest_wait(int(limit_ns), _stream(stream)))
 
 
 def get_status(clear=True, stream=None) -> int:

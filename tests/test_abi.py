@@ -24,10 +24,25 @@ def _declared():
 def test_library_exports_every_declared_symbol():
     L = nv.lib()
     names = _declared()
-    assert len(names) == 17
+    assert len(names) == 18
     assert set(names) == set(nv.EXPORTED)
     for n in names:
         assert hasattr(L, n)
+
+
+def test_status_bits_match_the_header():
+    txt = open(HDR).read()
+    bits = dict((m.group(1), int(m.group(2))) for m in re.finditer(r"ENTMAXKV_STATUS_(\w+)\s*=\s*(\d+)", txt))
+    assert bits == {"BAD_PAGE": nv.STATUS_BAD_PAGE, "BAD_SELECTION": nv.STATUS_BAD_SELECTION,
+                    "TIMEOUT": nv.STATUS_TIMEOUT, "OVERFLOW": nv.STATUS_OVERFLOW,
+                    "BAD_LENGTH": nv.STATUS_BAD_LENGTH, "NONFINITE": nv.STATUS_NONFINITE}
+    assert len(set(bits.values())) == len(bits) and all(v & (v - 1) == 0 for v in bits.values())
+
+
+def test_selftest_wait_rejects_limits_out_of_range():
+    L = nv.lib()
+    assert L.entmaxkv_selftest_wait(0, None) == -2
+    assert L.entmaxkv_selftest_wait(2_000_000_001, None) == -2
 
 
 def test_strerror_and_version():

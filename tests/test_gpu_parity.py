@@ -21,7 +21,7 @@ import torch
 import oracle as orc
 from sparse_entmax_kv_b200 import native as nv
 from sparse_entmax_kv_b200.decoder import EntmaxKVDecoder, last_token_rows
-from sparse_entmax_kv_b200.workloads import CONFIGS, Workload, make_inputs, to_host_u16
+from sparse_entmax_kv_b200.workloads import CONFIGS, Workload, make_inputs, sweep_points, to_host_u16
 
 pytestmark = pytest.mark.gpu
 
@@ -617,17 +617,8 @@ def test_kv_head_ranges_match_one_call(name, splits):
 # ---------------------------------------------------- full-size workloads
 
 def _sub_problem(inp, wl, b, kvh):
-    """(sequence b, kv head kvh) as a self-contained host problem (identity page table)."""
-    L = int(inp["seq_lens"][b])
-    npb = -(-L // wl.P)
-    blocks = inp["page_table"][b, :npb].long()
-    G = wl.G
-    K = inp["k_cache"][blocks, kvh:kvh + 1].contiguous()
-    V = inp["v_cache"][blocks, kvh:kvh + 1].contiguous()
-    q = inp["q"][b:b + 1, kvh * G:(kvh + 1) * G].contiguous()
-    return dict(q=to_host_u16(q), K=to_host_u16(K), V=to_host_u16(V),
-                page_table=np.arange(npb, dtype=np.int32)[None], seq_lens=np.array([L], np.int32), npb=npb,
-                blocks=blocks.cpu().numpy())
+    from tests.helpers import sub_problem
+    return sub_problem(inp, wl, b, kvh)
 
 
 FULL = ["tiny_h1_L4k", "dense_gqa_L32k", "topk_gqa_L128k", "gauss_gqa_L1m", "sweep_mha_L64k"]
@@ -671,6 +662,12 @@ def test_full_size_step_sampled(name):
         gsel = dec.sel[b, hs].cpu().numpy()
         gcnt = dec.cnt[b, hs].cpu().numpy()
         gout = dec.out[b, hs].cpu().numpy()
+        gtau = dec.tau[b, hs].cpu().numpy()
+        # the decode of the GPU's own selection, by the oracle: the output check
+        # holds for every head, also where a page inside the cutoff band made
+        # the two selections differ
+        og, otg, _, _ = orc.decode(sp["q"], sp["K"], sp["V"], sp["page_table"], sp["seq_lens"], 1, wl.P,
+                                   wl.alpha, sel=gsel[None, :, :sp["npb"]], cnt=gcnt[None])
         for g in range(G):
             gs, os_ = gsel[g, :gcnt[g]], osel[0, g, :ocnt[0, g]]
             if policy == "topk":
@@ -679,9 +676,11 @@ def test_full_size_step_sampled(name):
                 gth = float(dec.tau_hat[b, kvh * G + g])
                 assert gth == pytest.approx(oth[0, g], abs=1e-5 * max(1.0, abs(oth[0, g])))
                 check_selection(gs, os_, (wl.alpha - 1) * ob[0, g].astype(np.float64), oth[0, g] - delta)
+            assert_outputs_close(gout[g], og[0, g], f"{name} b{b} h{kvh * G + g} (GPU selection)")
+            assert float(gtau[g]) == pytest.approx(otg[0, g], abs=2e-5 * max(1, abs(otg[0, g])))
             if np.array_equal(gs, os_):
                 assert_outputs_close(gout[g], o[0, g], f"{name} b{b} h{kvh * G + g}")
-                assert float(dec.tau[b, kvh * G + g]) == pytest.approx(otau[0, g], abs=2e-5 * max(1, abs(otau[0, g])))
+                assert float(gtau[g]) == pytest.approx(otau[0, g], abs=2e-5 * max(1, abs(otau[0, g])))
 
 
 @pytest.mark.parametrize("name,alpha", [("dense_gqa_L32k", 1.5), ("dense_gqa_L32k", 1.0),
@@ -705,14 +704,22 @@ def test_full_size_dense_sampled(name, alpha):
                                    atol=2e-5 * max(1.0, np.abs(otau).max()))
 
 
-@pytest.mark.parametrize("pt", [dict(alpha=1.25, P=16, policy="topk", k=128, delta=0.0, needles=256),
-                                dict(alpha=2.0, P=64, policy="gauss", k=0, delta=1.0, needles=1),
-                                dict(alpha=1.5, P=32, policy="gauss", k=0, delta=0.25, needles=16)])
+def _sweep_id(pt):
+    pol = f"topk{pt['k']}" if pt["policy"] == "topk" else f"gauss{pt['delta']}"
+    return f"a{pt['alpha']}-P{pt['P']}-{pol}-n{pt['needles']}"
+
+
+@pytest.mark.parametrize("pt", sweep_points(), ids=_sweep_id)
 def test_sweep_points_reduced_batch(pt):
-    wl = CONFIGS["sweep_mha_L64k"].shrink(B=2, Hq=4, Hkv=4, **pt)
+    """Every point of the MHA sweep (alpha x page size x policy x needles, 108
+    in all) at its full 65,536-token context with two sequences of two heads:
+    the whole step as the benchmark launches it, against the oracle."""
+    wl = CONFIGS["sweep_mha_L64k"].shrink(B=2, Hq=2, Hkv=2, **pt)
     inp = make_inputs(wl, 13, device="cuda")
+    k = wl.k or 32
+    delta = wl.delta or 0.5
     dec = EntmaxKVDecoder(inp["k_cache"], inp["v_cache"], inp["page_table"], inp["seq_lens"], wl.Hq,
-                          alpha=wl.alpha, policy=wl.policy, k=wl.k or 32, delta=wl.delta or 0.5)
+                          alpha=wl.alpha, policy=wl.policy, k=k, delta=delta)
     dec.build_meta()
     dec.step(inp["q"])
     torch.cuda.synchronize()
@@ -720,17 +727,63 @@ def test_sweep_points_reduced_batch(pt):
                 page_table=inp["page_table"].cpu().numpy(), seq_lens=inp["seq_lens"].cpu().numpy())
     ob, omu, osg = _oracle_scores(host, wl)
     assert np.array_equal(dec.bbox.cpu().numpy().view(np.uint32), ob.view(np.uint32))
-    osel, ocnt, oth = orc.select(host["seq_lens"], ob, omu, osg, wl.P, wl.policy, wl.k or 32, wl.alpha,
-                                 wl.delta or 0.5)
+    osel, ocnt, oth = orc.select(host["seq_lens"], ob, omu, osg, wl.P, wl.policy, k, wl.alpha, delta)
+    gsel, gcnt, gout = dec.sel.cpu().numpy(), dec.cnt.cpu().numpy(), dec.out.cpu().numpy()
+    gtau = dec.tau.cpu().numpy()
+    # the oracle's decode of the GPU's own selection: checked for every head
+    og, otg, _, _ = orc.decode(host["q"], host["K"], host["V"], host["page_table"], host["seq_lens"], wl.Hkv,
+                               wl.P, wl.alpha, sel=gsel, cnt=gcnt)
     o, _, _, _ = orc.decode(host["q"], host["K"], host["V"], host["page_table"], host["seq_lens"], wl.Hkv, wl.P,
                             wl.alpha, sel=osel, cnt=ocnt)
-    gsel, gcnt, gout = dec.sel.cpu().numpy(), dec.cnt.cpu().numpy(), dec.out.cpu().numpy()
+    th = dec.tau_hat.cpu().numpy()
     for b in range(wl.B):
         for h in range(wl.Hq):
             gs, os_ = gsel[b, h, :gcnt[b, h]], osel[b, h, :ocnt[b, h]]
+            assert np.all(np.diff(gs) > 0)
             if wl.policy == "gauss":
-                check_selection(gs, os_, (wl.alpha - 1) * ob[b, h].astype(np.float64), oth[b, h] - wl.delta)
+                assert th[b, h] == pytest.approx(oth[b, h], abs=1e-5 * max(1.0, abs(oth[b, h])))
+                check_selection(gs, os_, (wl.alpha - 1) * ob[b, h].astype(np.float64), oth[b, h] - delta)
             else:
                 np.testing.assert_array_equal(gs, os_)
+            assert_outputs_close(gout[b, h], og[b, h], f"b{b}h{h} (GPU selection)")
+            assert float(gtau[b, h]) == pytest.approx(otg[b, h], abs=2e-5 * max(1, abs(otg[b, h])))
             if np.array_equal(gs, os_):
                 assert_outputs_close(gout[b, h], o[b, h], f"b{b}h{h}")
+
+
+@pytest.mark.parametrize("alpha", [1.25, 1.5, 2.0])
+@pytest.mark.parametrize("policy", ["gauss", "gauss_est"])
+def test_select_gauss_beyond_cluster_capacity(alpha, policy):
+    """Sequences of more than 16,384 pages take the single-CTA Gaussian
+    selection kernel (the four-CTA cluster form holds at most 16,384 pages):
+    tau_hat and the kept pages against the oracle's, on 25,000 and 24,990
+    pages of 16 tokens (d = 64, one kv head of four query heads)."""
+    wl = Workload("gauss_long", B=2, Hq=4, Hkv=1, d=64, L=25000 * 16, P=16, alpha=alpha, policy="gauss",
+                  delta=0.5, keys="cluster", needles=8, ragged=True)
+    assert wl.max_pages > 16384
+    inp, host = gpu_inputs(wl, 23)
+    bbox, mu, sig = _oracle_scores(host, wl)
+    s = shape_of(wl)
+    B, Hq, mp = wl.B, wl.Hq, wl.max_pages
+    tb, tm, ts = (torch.from_numpy(np.nan_to_num(x, nan=0.0)).cuda() for x in (bbox, mu, sig))
+    sel = torch.full((B, Hq, mp), -1, dtype=torch.int32, device="cuda")
+    cnt = torch.zeros((B, Hq), dtype=torch.int32, device="cuda")
+    th = torch.zeros((B, Hq), device="cuda")
+    pol = {"gauss": nv.GAUSS, "gauss_est": nv.GAUSS_EST}[policy]
+    nv.entmaxkv_select(s, inp["seq_lens"], tb, tm, ts, pol, 1, alpha, wl.delta, sel, cnt, th)
+    osel, ocnt, oth = orc.select(host["seq_lens"], np.nan_to_num(bbox, nan=0.0), np.nan_to_num(mu, nan=0.0),
+                                 np.nan_to_num(sig, nan=0.0), wl.P, policy, 1, alpha, wl.delta)
+    sel, cnt, th = sel.cpu().numpy(), cnt.cpu().numpy(), th.cpu().numpy()
+    for b in range(B):
+        npb = n_pages(host, wl, b)
+        assert npb > 16384
+        for h in range(Hq):
+            gs, os_ = sel[b, h, :cnt[b, h]], osel[b, h, :ocnt[b, h]]
+            assert np.all(np.diff(gs) > 0) and (gs.size == 0 or (gs[0] >= 0 and gs[-1] < npb))
+            assert th[b, h] == pytest.approx(oth[b, h], abs=1e-5 * max(1.0, abs(oth[b, h])))
+            est = bbox[b, h].astype(np.float64)
+            if policy == "gauss_est":
+                ntok = [min(wl.P, int(host["seq_lens"][b]) - p * wl.P) for p in range(npb)]
+                z = np.array([orc.zmax_of(t) for t in ntok] + [0.0] * (mp - npb))
+                est = np.minimum(est, mu[b, h].astype(np.float64) + z * sig[b, h].astype(np.float64))
+            check_selection(gs, os_, (alpha - 1) * est, oth[b, h] - wl.delta, f"b{b}h{h}")

@@ -145,6 +145,65 @@ def test_sequence_sharded_matches_one_device(name, S):
         assert torch.equal(shards[r].tau.view(torch.int32), ref_tau.view(torch.int32))
         torch.testing.assert_close(outs[r], ref_out, rtol=1e-5, atol=1e-6)
         assert torch.equal(outs[r], outs[0])
+    # and against the oracle: its decode of the global selection, every head
+    host = dict(q=to_host_u16(inp["q"]), K=to_host_u16(inp["k_cache"]), V=to_host_u16(inp["v_cache"]),
+                page_table=inp["page_table"].cpu().numpy(), seq_lens=inp["seq_lens"].cpu().numpy())
+    sel, cnt = ref_sel.cpu().numpy(), ref_cnt.cpu().numpy()
+    o, otau, _, _ = orc.decode(host["q"], host["K"], host["V"], host["page_table"], host["seq_lens"], wl.Hkv,
+                               wl.P, wl.alpha, sel=sel, cnt=cnt)
+    _assert_oracle_close(outs[0].cpu().numpy(), o, shards[0].tau.cpu().numpy(), otau, f"{name} S={S}")
+
+
+def _assert_oracle_close(out, o, tau, otau, what):
+    """Output within max abs 2e-3 and relative L2 1e-3 of the oracle's, tau
+    within 2e-5 max(1, |tau|); heads with no selected token (NaN tau, zero
+    output) must be so on both sides."""
+    out, o = np.asarray(out, np.float64), np.asarray(o, np.float64)
+    err = np.abs(out - o).max()
+    rel = np.linalg.norm(out - o) / max(np.linalg.norm(o), 1e-30)
+    assert err <= 2e-3 and rel <= 1e-3, f"{what}: max abs {err:.3e}, rel L2 {rel:.3e}"
+    none = np.isnan(tau)
+    assert np.array_equal(none, np.isnan(otau)) or np.all(~np.isfinite(otau[none]))
+    ok = ~none
+    assert np.all(np.abs(tau[ok] - otau[ok]) <= 2e-5 * np.maximum(1.0, np.abs(otau[ok]))), f"{what}: tau"
+
+
+@pytest.mark.gpu
+def test_sequence_sharded_candidate_cap_overflow():
+    """The candidates phase with a cap smaller than a head's candidate list:
+    the count stays exact, the first cap candidates are written in list
+    order, and STATUS_OVERFLOW is set."""
+    from sparse_entmax_kv_b200 import native as nv
+    from sparse_entmax_kv_b200.sharded import NativeShard, split_context
+    wl = Workload("capped", B=1, Hq=2, Hkv=1, d=64, L=64 * 40, P=64, alpha=2.0, policy="topk", k=40,
+                  keys="offset", needles=0)
+    inp = make_inputs(wl, 33, device="cuda")
+    inp["k_cache"][:] = inp["k_cache"][0, 0, 0]  # equal keys: every selected token is a candidate
+    pt, sl, p0 = split_context(inp["page_table"], inp["seq_lens"], wl.P, 1, 0)
+    cap = 100
+    sh = NativeShard(inp["k_cache"], inp["v_cache"], pt, sl, inp["seq_lens"], wl.Hq, p0, wl.max_pages,
+                     alpha=wl.alpha, policy="topk", k=wl.k, cap=cap)
+    sh.build_meta()
+    nv.get_status(clear=True)
+    sh.select(*sh.score(inp["q"]))
+    zmax = sh.begin(inp["q"]).clone()
+    cz, cn = sh.candidates(inp["q"], zmax)
+    torch.cuda.synchronize()
+    assert nv.get_status(clear=True) & nv.STATUS_OVERFLOW
+    host = dict(q=to_host_u16(inp["q"]), K=to_host_u16(inp["k_cache"]), V=to_host_u16(inp["v_cache"]),
+                page_table=inp["page_table"].cpu().numpy(), seq_lens=inp["seq_lens"].cpu().numpy())
+    sel, cnt = sh.sel.cpu().numpy(), sh.cnt.cpu().numpy()
+    _, _, _, zz = orc.decode(host["q"], host["K"], host["V"], host["page_table"], host["seq_lens"], wl.Hkv, wl.P,
+                             wl.alpha, sel=sel, cnt=cnt, want_z=True)
+    cn, cz = cn.cpu().numpy(), cz.cpu().numpy()
+    for h in range(wl.Hq):
+        z = zz[0, h]
+        zl = np.concatenate([z[p * wl.P:(p + 1) * wl.P] for p in sel[0, h, :cnt[0, h]]])  # list order
+        zm = float(zmax[0, h])
+        assert abs(zm - zl.max()) <= 1e-5 * max(1.0, abs(zl.max()))
+        want = zl[zl > zm - 1.0]
+        assert int(cn[0, h]) == want.size == cnt[0, h] * wl.P > cap
+        np.testing.assert_allclose(cz[0, h, :cap], want[:cap], rtol=0, atol=1e-5)
 
 
 @pytest.mark.gpu
@@ -182,6 +241,19 @@ def test_sequence_sharded_full_size_1m_tokens():
         assert torch.equal(shards[r].cnt, ref_cnt)
         assert torch.equal(shards[r].tau.view(torch.int32), ref_tau.view(torch.int32))
         torch.testing.assert_close(outs[r], ref_out, rtol=1e-5, atol=1e-6)
+    # sampled (sequence, kv head) groups against the oracle's decode of the
+    # selection every rank holds
+    from tests.helpers import sub_problem
+    G = wl.G
+    sel = shards[0].sel.cpu().numpy()
+    cnt = shards[0].cnt.cpu().numpy()
+    for kvh in (0, wl.Hkv - 1):
+        sp = sub_problem(inp, wl, 0, kvh)
+        hs = slice(kvh * G, (kvh + 1) * G)
+        o, otau, _, _ = orc.decode(sp["q"], sp["K"], sp["V"], sp["page_table"], sp["seq_lens"], 1, wl.P, wl.alpha,
+                                   sel=sel[0:1, hs, :sp["npb"]], cnt=cnt[0:1, hs])
+        _assert_oracle_close(outs[0][0, hs].cpu().numpy(), o[0], shards[0].tau[0, hs].cpu().numpy(), otau[0],
+                             f"1M kvh{kvh}")
 
 
 # ------------------------------------------------------------------- CPU
