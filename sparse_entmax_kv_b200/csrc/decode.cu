@@ -48,6 +48,15 @@ constexpr int UTH = 512;
 constexpr int UCH = 16384;  // pages per chunk (one byte each)
 
 __global__ void __launch_bounds__(UTH) union_kernel(DecodeArgs a) {
+    {
+        // the group's page-table row, on its way to L2 while the previous
+        // kernel finishes (a hint only: nothing is read before the dependency
+        // wait), so the lookups below find it there
+        const int b0 = blockIdx.x / a.nk;
+        const char *row = reinterpret_cast<const char *>(a.page_table + (size_t)b0 * a.max_pages);
+        for (int l = threadIdx.x; l * 32 < a.max_pages; l += UTH)
+            asm volatile("prefetch.global.L2 [%0];" ::"l"(row + (size_t)l * 128));
+    }
     pdl_wait();
     __shared__ unsigned words[UCH / 4];
     __shared__ int sh[72];
@@ -270,13 +279,16 @@ __device__ void produce(const DecodeArgs &a, const CUtensorMap *m0, const CUtens
 // step mod gridDim.x) to the workspace, each with its G-bit head mask and
 // physical block (the page-table loads issued eight at a time), for its
 // producer and for the tau kernel; CTA 0 also writes the count.  Every CTA
-// reads the same lists, so all agree on U and on the positions.  Used when the
-// grid has at most two CTAs per group (many groups), where the rebuild is
-// repeated little; all threads call it; it returns U.
+// reads the same lists, so all agree on U and on the positions.  A warp marks
+// 32 consecutive list entries at a time: lanes whose entries fall in the same
+// bitmap word (a run of neighbouring pages of one head's ascending list) OR
+// their bits together first, and the first lane of each run sets them with one
+// shared-memory atomic.  All threads call it; it returns U.
 __device__ int union_in_cta(const DecodeArgs &a, int b, int kvh, int bk, int np, int PPS, unsigned *bm, int *s_cnt,
                             int *s_off, int *sh) {
     const int G = a.Hq / a.Hkv;
     const int nt = blockDim.x, S = gridDim.x;
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5, nwarps = nt >> 5;
     const int *selg = a.sel + (size_t)(b * a.Hq + kvh * G) * a.sel_stride;  // head g's list at g * sel_stride
     const int *pt = a.page_table + (size_t)b * a.max_pages;
     int *ue = a.ws.union_e + (size_t)bk * a.max_pages;
@@ -300,29 +312,39 @@ __device__ int union_in_cta(const DecodeArgs &a, int b, int kvh, int bk, int np,
     }
     __syncthreads();
     const int total = s_off[G];  // every head's entries as one flat range
-    // four list entries in flight per thread
-    for (int k0 = threadIdx.x; k0 < total; k0 += 4 * nt) {
-        int p[4], g[4];
+    // each warp takes 32 consecutive entries per round, two rounds' loads in flight
+    for (int k0 = warp * 32; k0 < total; k0 += 2 * nwarps * 32) {
+        int wd[2];
+        unsigned bit[2];
 #pragma unroll
-        for (int u = 0; u < 4; ++u) {
-            const int k = k0 + u * nt;
-            p[u] = 0;
-            g[u] = 0;
+        for (int u = 0; u < 2; ++u) {
+            const int k = k0 + u * nwarps * 32 + lane;
+            wd[u] = -1 - lane;  // unique: merges with no other lane
+            bit[u] = 0u;
             if (k < total) {
                 int gg = 0;
                 while (k >= s_off[gg + 1]) ++gg;
-                g[u] = gg;
-                p[u] = __ldg(selg + (size_t)gg * a.sel_stride + (k - s_off[gg])) - a.page_begin;
+                const int p = __ldg(selg + (size_t)gg * a.sel_stride + (k - s_off[gg])) - a.page_begin;
+                if (p >= 0 && p < np) {
+                    wd[u] = gg * W + (p >> 5);
+                    bit[u] = 1u << (p & 31);
+                } else if (report && (!a.sharded || p + a.page_begin < 0 || p + a.page_begin >= a.sel_stride)) {
+                    atomicOr(a.status, ENTMAXKV_STATUS_BAD_SELECTION);  // (sharded: other shards' pages are skipped)
+                }
             }
         }
 #pragma unroll
-        for (int u = 0; u < 4; ++u) {
-            if (k0 + u * nt >= total) continue;
-            if (p[u] >= 0 && p[u] < np)
-                atomicOr(&bm[g[u] * W + (p[u] >> 5)], 1u << (p[u] & 31));
-            else if (report && (a.sharded ? (p[u] + a.page_begin < 0 || p[u] + a.page_begin >= a.sel_stride)
-                                          : true))
-                atomicOr(a.status, ENTMAXKV_STATUS_BAD_SELECTION);  // (sharded: other shards' pages are skipped)
+        for (int u = 0; u < 2; ++u) {
+            // OR over the lane's run of equal words (suffix scan within runs)
+            unsigned acc = bit[u];
+#pragma unroll
+            for (int o = 1; o < 32; o <<= 1) {
+                const unsigned y = __shfl_down_sync(FULL, acc, o);
+                const int wy = __shfl_down_sync(FULL, wd[u], o);
+                if (lane + o < 32 && wy == wd[u]) acc |= y;
+            }
+            const int wprev = __shfl_up_sync(FULL, wd[u], 1);
+            if (acc && (lane == 0 || wprev != wd[u])) atomicOr(&bm[wd[u]], acc);
         }
     }
     __syncthreads();

@@ -199,6 +199,37 @@ def test_meta_and_scores_bit_exact(name):
         assert torch.equal(bb2[b, :, :npb], out[0][b, :, :npb])
 
 
+@pytest.mark.parametrize("policy", ["topk", "gauss"])
+def test_scores_bit_exact_with_several_tiles_per_warp(policy):
+    """128 (sequence, kv head) groups of 32 metadata tiles: more tiles than
+    resident warps, so every scoring warp streams two tiles back to back
+    (ragged lengths leave some tiles partial or empty)."""
+    wl = Workload("tiles2", B=16, Hq=32, Hkv=8, d=64, L=16384, P=16, alpha=1.5, policy=policy, k=16, delta=0.5,
+                  keys="offset", needles=2, ragged=True)
+    inp, host = gpu_inputs(wl, 29)
+    inp["seq_lens"][3] = 16 * 100 + 5  # a short sequence: most of its tiles are empty
+    host["seq_lens"] = inp["seq_lens"].cpu().numpy()
+    s = shape_of(wl)
+    meta = nv.alloc_meta(s, "cuda")
+    nv.entmaxkv_build_meta(s, inp["k_cache"], inp["page_table"], inp["seq_lens"], 0, -1, meta)
+    o = orc.build_meta(host["K"], host["page_table"], host["seq_lens"], wl.Hkv, wl.d, wl.P, wl.num_blocks)
+    B, Hq, mp = wl.B, wl.Hq, wl.max_pages
+    out = [torch.full((B, Hq, mp), float("nan"), device="cuda") for _ in range(3)]
+    gauss = policy == "gauss"
+    nv.entmaxkv_score_pages(s, inp["q"], meta, inp["seq_lens"], out[0], out[1] if gauss else None,
+                            out[2] if gauss else None)
+    ob = orc.score_pages(host["q"], o, host["page_table"], host["seq_lens"], wl.Hkv, wl.P)
+    gb, gm, gs = (t.cpu().numpy() for t in out)
+    for b in range(B):
+        npb = n_pages(host, wl, b)
+        np.testing.assert_array_equal(gb[b, :, :npb].view(np.uint32), ob[0][b, :, :npb].view(np.uint32))
+        assert np.isnan(gb[b, :, npb:]).all()  # nothing written past the sequence
+        if gauss:
+            recs = (host["page_table"][b, :npb][None, :] * wl.Hkv + (np.arange(Hq) // wl.G)[:, None])
+            check_mu_sigma(gm[b, :, :npb], gs[b, :, :npb], ob[1][b, :, :npb], ob[2][b, :, :npb], host["q"][b],
+                           o[2], o[3], recs, f"b{b}")
+
+
 def _oracle_scores(host, wl):
     meta = orc.build_meta(host["K"], host["page_table"], host["seq_lens"], wl.Hkv, wl.d, wl.P, wl.num_blocks)
     return orc.score_pages(host["q"], meta, host["page_table"], host["seq_lens"], wl.Hkv, wl.P)
