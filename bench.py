@@ -181,7 +181,7 @@ def run_gpu(args, rank, world):
     k = wl.k or 64
     delta = wl.delta or 0.5
     dev = torch.device("cuda", torch.cuda.current_device())
-    inp = make_inputs(wl, 1000 * 4 + rank, device=dev)
+    inp = make_inputs(wl, 1000 * 4 + rank, device=dev, sequential_pages=args.page_table == "sequential")
     dec = EntmaxKVDecoder(inp["k_cache"], inp["v_cache"], inp["page_table"], inp["seq_lens"], wl.Hq,
                           alpha=wl.alpha, policy=policy, k=k, delta=delta)
     dec.build_meta()
@@ -594,10 +594,75 @@ def run_quality(args):
         del dec
 
 
+def run_crossover(args):
+    """Where the sparse step starts to beat reading the whole cache: the
+    single-head tiny shape (B=1, Hq=Hkv=1, d=64, 16-token pages, alpha 1.5,
+    top-k 32 pages, 8 needles) at growing context lengths.  Per L: the sparse
+    step (append, score, select, decode) as one CUDA-graph replay, and the
+    full-cache entmax and softmax decodes, eager; device time per call from
+    CUDA events, mean over args.steps after args.warmup, L2 flushed before
+    each.  One JSON line per L."""
+    from sparse_entmax_kv_b200 import native as nv
+    from sparse_entmax_kv_b200.decoder import EntmaxKVDecoder, last_token_rows
+    from sparse_entmax_kv_b200.workloads import CONFIGS, make_inputs
+    base = CONFIGS["tiny_h1_L4k"]
+    dev = torch.device("cuda", torch.cuda.current_device())
+    flush_w = torch.empty(256 << 20, dtype=torch.uint8, device=dev)
+    flush_r = torch.ones(32 << 20, dtype=torch.int64, device=dev)
+    st = torch.cuda.current_stream()
+
+    def timed(fn):
+        ts = []
+        for i in range(args.warmup + args.steps):
+            flush_w.fill_(1)
+            torch.amax(flush_r)
+            a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            a.record(st)
+            fn()
+            b.record(st)
+            torch.cuda.synchronize()
+            if i >= args.warmup:
+                ts.append(a.elapsed_time(b) * 1e3)
+        return float(np.mean(ts))
+
+    for L in (4096, 8192, 16384, 32768, 65536, 131072):
+        wl = base.shrink(L=L)
+        inp = make_inputs(wl, 4000, device=dev)
+        dec = EntmaxKVDecoder(inp["k_cache"], inp["v_cache"], inp["page_table"], inp["seq_lens"], wl.Hq,
+                              alpha=wl.alpha, policy="topk", k=wl.k)
+        dec.build_meta()
+        nkv = last_token_rows(inp["k_cache"], inp["v_cache"], inp["page_table"], inp["seq_lens"])
+        dec.step(inp["q"], new_kv=nkv)
+        torch.cuda.synchronize()
+        g = torch.cuda.CUDAGraph()
+        side = torch.cuda.Stream()
+        side.wait_stream(torch.cuda.current_stream())
+        with torch.cuda.stream(side):
+            dec.step(inp["q"], new_kv=nkv)
+        torch.cuda.current_stream().wait_stream(side)
+        with torch.cuda.graph(g):
+            dec.step(inp["q"], new_kv=nkv)
+        torch.cuda.synchronize()
+        sparse = timed(g.replay)
+        out = torch.empty((wl.B, wl.Hq, wl.d), device=dev)
+        ws = nv.alloc_workspace(dec.shape, nv.CALL_DECODE_DENSE, dev)
+        dense = {}
+        for alpha, name in ((wl.alpha, "dense_entmax_us"), (1.0, "dense_softmax_us")):
+            dense[name] = round(timed(lambda: nv.entmaxkv_decode_dense(
+                dec.shape, inp["q"], dec.k_cache, dec.v_cache, dec.page_table, dec.seq_lens, alpha, out, None, None,
+                ws)), 2)
+        assert nv.get_status(clear=True) & ~nv.STATUS_OVERFLOW == 0
+        print(json.dumps({"sweep": "crossover", "workload": base.name, "L": L, "sparse_step_us": round(sparse, 2),
+                          **dense, "kv_bytes_full_cache": 2 * L * wl.d * 2,
+                          "sparse_over_dense_softmax": round(sparse / dense["dense_softmax_us"], 3)}), flush=True)
+        del dec, g, inp, ws
+        torch.cuda.empty_cache()
+
+
 def config_of(wl):
     return {"workload": wl.name, "B": wl.B, "Hq": wl.Hq, "Hkv": wl.Hkv, "d": wl.d, "L": wl.L,
             "page_size": wl.P, "alpha": wl.alpha, "policy": wl.policy, "k": wl.k, "delta": wl.delta,
-            "keys": wl.keys, "needles_per_head": wl.needles,
+            "keys": wl.keys, "needles_per_head": wl.needles, "page_table": "seeded permutation of the blocks",
             "l2": "flushed before every step (256 MiB write, then 256 MiB read of a clean buffer), "
                   "outside the per-step events"}
 
@@ -618,6 +683,10 @@ def main():
                     help="instead of the benchmark line: sparse vs full-cache error, entmax vs softmax at one kept set")
     ap.add_argument("--l-sweep", action="store_true",
                     help="instead of the benchmark line: selection scaling with context length (one line per L, policy)")
+    ap.add_argument("--crossover", action="store_true",
+                    help="instead of the benchmark line: sparse step vs full-cache decodes at growing L, tiny shape")
+    ap.add_argument("--page-table", default="random", choices=["random", "sequential"],
+                    help="physical placement of the logical pages: a seeded permutation (default) or in order")
     args = ap.parse_args()
     args.warmup = max(args.warmup, 3)
 
@@ -635,6 +704,9 @@ def main():
     if args.quality:
         run_quality(args)
         return
+    if args.crossover:
+        run_crossover(args)
+        return
     if world > 1:
         import datetime
         torch.distributed.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
@@ -646,10 +718,13 @@ def main():
     nb = res["nbytes"]
     value = whole_job_gbs(nb["kv_touched"], world, res["step_ms"])
     e2e_val = whole_job_gbs(nb["kv_touched"], world, res["e2e_ms"])
+    cfg = config_of(wl)
+    if args.page_table == "sequential":
+        cfg["page_table"] = "identity: logical pages in block order"
     line = {"metric": METRIC, "value": round(value, 2), "unit": "GB/s", "n_gpus": world, "steps": args.steps,
             "warmup": args.warmup, "ms_per_step": round(res["step_ms"], 5),
             "us_per_step": round(res["step_ms"] * 1e3, 2), "higher_is_better": True, "scaling": "weak",
-            "vs_baseline": None, "dtype": "bf16", "data": "synthetic", "config": config_of(wl),
+            "vs_baseline": None, "dtype": "bf16", "data": "synthetic", "config": cfg,
             "frac_of_hbm_peak": round(value / world / res["roofline"]["peak"], 4),
             "roofline": res["roofline"], "roofline_gather": res["roofline_gather"],
             "stages_us": res["stage_us"], "bytes_per_step": nb,

@@ -693,8 +693,19 @@ __global__ void __launch_bounds__(TAU_NT, D == 64 ? 4 : 3) tau_pv_kernel(const _
     const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
     const bool given_tau = a.tau_in != nullptr;
     const bool export_cand = a.cand_z != nullptr;
+    // the loads that depend on nothing are issued together: the query row (its
+    // finite check), the running max of z and the union size
+    const uint16_t qbits = threadIdx.x < D ? a.q[(size_t)bh * D + threadIdx.x] : (uint16_t)0;
+    // max z of the head: the q.K kernel's running max, or, when the q.K CTAs
+    // built the union themselves (nothing reset the running max), the max of
+    // the tile maxima; in the sequence-sharded phases the global max z comes
+    // in (and the candidates phase writes out this shard's candidate z values)
+    const bool zmax_from_tiles = !a.zmax_in && a.union_in_qk;
+    const int zord = a.zmax_in || zmax_from_tiles ? 0 : a.ws.zmax[bh];
+    const int np = n_pages_of(seq_len_of(a.seq_lens, b, P, a.max_pages, a.status), P);
+    const int U = dense ? np : a.ws.union_cnt[bk];
     // a query with a NaN or an infinity: NaN output and threshold, no candidates
-    if (!__syncthreads_and(threadIdx.x >= D || (a.q[(size_t)bh * D + threadIdx.x] & 0x7f80u) != 0x7f80u)) {
+    if (!__syncthreads_and(threadIdx.x >= D || (qbits & 0x7f80u) != 0x7f80u)) {
         if (threadIdx.x == 0) atomicOr(a.status, ENTMAXKV_STATUS_NONFINITE);
         if (export_cand) {
             if (threadIdx.x == 0) a.cand_n[bh] = 0;
@@ -708,14 +719,6 @@ __global__ void __launch_bounds__(TAU_NT, D == 64 ? 4 : 3) tau_pv_kernel(const _
         }
         return;
     }
-    // max z of the head: the q.K kernel's running max, or, when the q.K CTAs
-    // built the union themselves (nothing reset the running max), the max of
-    // the tile maxima; in the sequence-sharded phases the global max z comes
-    // in (and the candidates phase writes out this shard's candidate z values)
-    const bool zmax_from_tiles = !a.zmax_in && a.union_in_qk;
-    const int zord = a.zmax_in || zmax_from_tiles ? 0 : a.ws.zmax[bh];
-    const int np = n_pages_of(seq_len_of(a.seq_lens, b, P, a.max_pages, a.status), P);
-    const int U = dense ? np : a.ws.union_cnt[bk];
     const int n_tok = U * P;  // a multiple of 16
     const size_t trow = tile_row(a, b, h);
     const float *tr = a.ws.tmax + trow;

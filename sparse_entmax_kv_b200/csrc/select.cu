@@ -305,36 +305,40 @@ __global__ void __launch_bounds__(SEL_THREADS) gauss_kernel(SelectArgs a) {
 #pragma unroll
     for (int o = 16; o; o >>= 1) mloc = fmaxf(mloc, __shfl_xor_sync(FULL, mloc, o));
     if (lane == 0) shm[warp] = mloc;
-    if (threadIdx.x == 0) ncand = 0;
     __syncthreads();
     float tau0 = -INFINITY;
     for (int w = 0; w < SEL_THREADS / 32; ++w) tau0 = fmaxf(tau0, shm[w]);
 
     // Pages with m + 10 s below tau0 add less than n_p s^R J_R(10) to F at any
     // tau >= tau0 (a relative 1e-23 of one page's worth): they are dropped.
+    // The kept pages take their slots from a block scan in thread order (then
+    // item order), so the list, and every sum over it, is the same each call.
     float hloc = -INFINITY;  // max over pages of m + 10 s: F < 1 there
+    int nkept = 0;
     for (int t0 = 0; t0 < n; t0 += TILE) {
         if (!one_tile) load_ms(t0);
+        unsigned keep = 0;
 #pragma unroll
         for (int i = 0; i < ITEMS; ++i) {
             const int p = t0 + threadIdx.x + SEL_THREADS * i;
             if (p < n) hloc = fmaxf(hloc, mm[i] + 10.f * ss[i]);
-            const bool keep = p < n && mm[i] + 10.f * ss[i] >= tau0;
-            const unsigned bal = __ballot_sync(FULL, keep);
-            if (!bal) continue;
-            int base = 0;
-            if (lane == __ffs(bal) - 1) base = atomicAdd(&ncand, __popc(bal));
-            base = __shfl_sync(FULL, base, __ffs(bal) - 1);
-            if (keep) {
-                const int slot = base + __popc(bal & ((1u << lane) - 1u));
+            if (p < n && mm[i] + 10.f * ss[i] >= tau0) keep |= 1u << i;
+        }
+        int tot;
+        int slot = nkept + block_excl_scan(__popc(keep), shi, &tot);
+#pragma unroll
+        for (int i = 0; i < ITEMS; ++i)
+            if ((keep >> i) & 1u) {
                 if (slot < GCAP) {
                     cm[slot] = mm[i];
                     cs[slot] = ss[i];
-                    cn[slot] = (float)tokens_in_page(seq, a.P, p);
+                    cn[slot] = (float)tokens_in_page(seq, a.P, t0 + threadIdx.x + SEL_THREADS * i);
                 }
+                ++slot;
             }
-        }
+        nkept += tot;
     }
+    if (threadIdx.x == 0) ncand = nkept;
 #pragma unroll
     for (int o = 16; o; o >>= 1) hloc = fmaxf(hloc, __shfl_xor_sync(FULL, hloc, o));
     if (lane == 0) shm2[warp] = hloc;

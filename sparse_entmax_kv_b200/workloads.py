@@ -107,8 +107,11 @@ def _bf16(x: torch.Tensor) -> torch.Tensor:
     return x.to(torch.bfloat16)
 
 
-def make_inputs(wl: Workload, seed: int, device="cpu"):
-    """Draw one workload instance.
+def make_inputs(wl: Workload, seed: int, device="cpu", sequential_pages: bool = False):
+    """Draw one workload instance.  sequential_pages: logical page p of
+    sequence b sits in block b * max_pages + p (an identity page table)
+    instead of a seeded permutation of the blocks; every other draw is the
+    same.
 
     Returns a dict of tensors on ``device``:
       q          bf16  [B, Hq, d]
@@ -132,6 +135,8 @@ def make_inputs(wl: Workload, seed: int, device="cpu"):
         return torch.randint(0, hi, shape, generator=g, device=dev)
 
     perm = torch.randperm(nb, generator=g, device=dev).to(torch.int32)
+    if sequential_pages:
+        perm = torch.arange(nb, device=dev, dtype=torch.int32)
     page_table = perm.view(B, Np).contiguous()
 
     if wl.ragged:
