@@ -19,7 +19,7 @@ ARCH = ["-gencode", "arch=compute_100a,code=sm_100a"]
 FLAGS = ["-O3", "-std=c++17", "-lineinfo", "-Xcompiler", "-fPIC", "-Xcompiler", "-fvisibility=hidden",
          "--expt-relaxed-constexpr", "-I" + os.path.join(ROOT, "include")]
 SOURCES = ["api.cu", "meta.cu", "score.cu", "select.cu", "decode.cu"]
-HEADERS = ["common.cuh", "internal.h", "pipeline.cuh"]
+HEADERS = ["common.cuh", "internal.h", "pipeline.cuh", "record.cuh"]
 
 
 def _newer(target, deps):
