@@ -37,10 +37,16 @@ constexpr int THREADS = WARPS * 32;
 constexpr int BOUND_CHUNK = 128 * CHK;  // kmin + kmax block of one chunk: 2048 B
 constexpr int MOM_CHUNK = 256 * CHK;    // mean + var block of one chunk:  4096 B
 
+// A ring stage holds CPS chunks: the Gaussian policy's one chunk of bounds
+// and moments (2 KB + 4 KB), or top-k's two consecutive chunks of bounds
+// (one 4 KB copy: the bound-only stream measured faster with 4 KB copies in
+// two stages than with 2 KB copies in four, 24 vs 31 us of loads alone for
+// the 128k-token batch of 8).
 template <bool GAUSS>
 struct Ring {
-    static constexpr int STAGE = GAUSS ? BOUND_CHUNK + MOM_CHUNK : BOUND_CHUNK;
-    static constexpr int NST = GAUSS ? 2 : 4;
+    static constexpr int CPS = GAUSS ? 1 : 2;
+    static constexpr int STAGE = GAUSS ? BOUND_CHUNK + MOM_CHUNK : CPS * BOUND_CHUNK;
+    static constexpr int NST = 2;
 };
 
 template <int D, int G>
@@ -55,13 +61,14 @@ constexpr size_t smem_bytes() {
 }
 
 // Two CTAs per SM for the Gaussian policy (its 6 KB stages fill shared
-// memory); three for top-k (2 KB stages), whose bounds-only stream does the
+// memory); three for top-k (4 KB stages), whose bounds-only stream does the
 // same fp64 work per chunk on a third of the bytes and gains from more warps.
 template <int D, int G, bool GAUSS>
 __global__ void __launch_bounds__(THREADS, G <= 4 ? (GAUSS ? 2 : 3) : 1) score_kernel(ScoreArgs a) {
     pdl_wait();
     using RG = Ring<GAUSS>;
-    constexpr int NCH = D / CHK;
+    constexpr int CPS = RG::CPS;
+    constexpr int NCH = D / CHK / CPS;  // ring stages per tile
     constexpr int NST = RG::NST;
     extern __shared__ __align__(128) unsigned char smem[];
     double2 *qq = reinterpret_cast<double2 *>(smem);        // [D][G] (min(q, 0), max(q, 0))
@@ -105,7 +112,7 @@ __global__ void __launch_bounds__(THREADS, G <= 4 ? (GAUSS ? 2 : 3) : 1) score_k
             unsigned char *st = wring + (c % NST) * RG::STAGE;
             uint64_t *bar = &wbar[c % NST];
             mbar_arrive_expect_tx(bar, RG::STAGE);
-            bulk_g2s(st, gb + c * BOUND_CHUNK, BOUND_CHUNK, bar);
+            bulk_g2s(st, gb + c * CPS * BOUND_CHUNK, CPS * BOUND_CHUNK, bar);
             if (GAUSS) bulk_g2s(st + BOUND_CHUNK, gm + c * MOM_CHUNK, MOM_CHUNK, bar);
         }
     };
@@ -123,10 +130,13 @@ __global__ void __launch_bounds__(THREADS, G <= 4 ? (GAUSS ? 2 : 3) : 1) score_k
     const int s = lane;
     const int xb = (s >> 2) & 1, xm = (s >> 1) & 3;  // the layout's swizzles
     bool ok = true;
-    for (int c = 0; c < NCH; ++c) {
-        if (c + NST - 1 < NCH) issue(c + NST - 1);
-        ok &= mbar_wait(&wbar[c % NST], (c / NST) & 1, a.status);
-        const unsigned char *st = wring + (c % NST) * RG::STAGE;
+    for (int ci = 0; ci < NCH; ++ci) {
+        if (ci + NST - 1 < NCH) issue(ci + NST - 1);
+        ok &= mbar_wait(&wbar[ci % NST], (ci / NST) & 1, a.status);
+#pragma unroll
+        for (int k = 0; k < CPS; ++k) {
+        const unsigned char *st = wring + (ci % NST) * RG::STAGE + k * BOUND_CHUNK;  // chunk c's bounds
+        const int c = ci * CPS + k;
 #pragma unroll
         for (int hf = 0; hf < 2; ++hf) {  // two halves of 8 coordinates
             const uint4 kn = *reinterpret_cast<const uint4 *>(st + s * 32 + 16 * (hf ^ xb));
@@ -164,6 +174,7 @@ __global__ void __launch_bounds__(THREADS, G <= 4 ? (GAUSS ? 2 : 3) : 1) score_k
                     ab[g] = __fma_rn(qg.y, hi, ab[g]);
                 }
             }
+        }
         }
         __syncwarp();  // every lane is done with this stage before it is refilled
     }
