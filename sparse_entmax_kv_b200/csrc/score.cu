@@ -6,9 +6,10 @@
 //   sigma = sqrt((sum_j q_j^2 var_j) / d)                   Gaussian std
 //
 // The bound is one fp64 chain over j in index order, so it is reproducible to
-// the bit.  max(q a, q b) with a <= b equals q- a + q+ b, q+ = max(q, 0) and
-// q- = min(q, 0): one of the two products is an exact zero, so two fused
-// multiply-adds per coordinate add exactly the oracle's term with no select.
+// the bit.  max(q a, q b) with a <= b is q b for q >= 0 and q a for q < 0: the
+// chain takes one fused multiply-add per coordinate and head, of q (fp64) and
+// the bound its sign picks.  A bf16 value widened to fp64 has an all-zero low
+// word, so the pick is a select of the two high words.
 // mu and sigma feed only the approximate tau_hat; they are fp32 sums kept as
 // two interleaved chains (even and odd j) so that packed f32x2 FMAs do two
 // coordinates per instruction.
@@ -21,8 +22,10 @@
 // mbarrier, so HBM sees long contiguous reads and the SM issues no per-lane
 // copy instructions.  Each lane scores its page for all G query heads of the
 // group, so every byte crosses HBM once per group.  q sits in shared memory
-// as (q-, q+) pairs (fp64, [j][head], one 16-byte load each) and fp32
-// ([head][j]).
+// as fp64 ([j][head]: one 16-byte load serves two heads) and fp32 ([head][j]).
+// (An earlier form kept (min(q,0), max(q,0)) pairs, one 16-byte load and two
+// FMAs per coordinate and head; its shared-memory loads filled 79% of the LSU
+// data pipe in the bound-only scan, which then stalled on the MIO queue.)
 #include "common.cuh"
 #include "internal.h"
 
@@ -51,7 +54,7 @@ struct Ring {
 
 template <int D, int G>
 struct QBytes {
-    static constexpr int VALUE = D * G * 8 * 2 + D * G * 4;
+    static constexpr int VALUE = D * G * 8 + D * G * 4;
 };
 
 template <int D, int G, bool GAUSS>
@@ -71,8 +74,8 @@ __global__ void __launch_bounds__(THREADS, G <= 4 ? (GAUSS ? 2 : 3) : 1) score_k
     constexpr int NCH = D / CHK / CPS;  // ring stages per tile
     constexpr int NST = RG::NST;
     extern __shared__ __align__(128) unsigned char smem[];
-    double2 *qq = reinterpret_cast<double2 *>(smem);        // [D][G] (min(q, 0), max(q, 0))
-    float *qh = reinterpret_cast<float *>(qq + D * G);       // [G][D] q
+    double *qd = reinterpret_cast<double *>(smem);          // [D][G] q
+    float *qh = reinterpret_cast<float *>(qd + D * G);       // [G][D] q
     uint64_t *bars = reinterpret_cast<uint64_t *>(smem + QBytes<D, G>::VALUE);
     unsigned char *ring = smem + ((QBytes<D, G>::VALUE + WARPS * NST * 8 + 127) & ~127);
 
@@ -87,7 +90,7 @@ __global__ void __launch_bounds__(THREADS, G <= 4 ? (GAUSS ? 2 : 3) : 1) score_k
         const int g = i / D, j = i % D;
         const float v = bf16f(a.q[((size_t)b * a.Hq + kvh * G + g) * D + j]);
         if (!isfinite(v)) atomicOr(&q_bad, 1u << g);
-        qq[j * G + g] = make_double2(v < 0.f ? (double)v : 0.0, v > 0.f ? (double)v : 0.0);
+        qd[j * G + g] = (double)v;
         qh[g * D + j] = v;
     }
     if (threadIdx.x < WARPS * NST) mbar_init(&bars[threadIdx.x], 1);
@@ -164,14 +167,25 @@ __global__ void __launch_bounds__(THREADS, G <= 4 ? (GAUSS ? 2 : 3) : 1) score_k
 #pragma unroll
             for (int jj = 0; jj < 8; ++jj) {
                 const unsigned w_n = wn[jj >> 1], w_x = wx[jj >> 1];
-                const double lo = (double)((jj & 1) ? bf16hi(w_n) : bf16lo(w_n));
-                const double hi = (double)((jj & 1) ? bf16hi(w_x) : bf16lo(w_x));
+                // high words of kmin_j and kmax_j widened to fp64 (low words zero)
+                const int lo_h = __double2hiint((double)((jj & 1) ? bf16hi(w_n) : bf16lo(w_n)));
+                const int hi_h = __double2hiint((double)((jj & 1) ? bf16hi(w_x) : bf16lo(w_x)));
                 const int j = j0 + jj;
+                double q[G];
+                if constexpr (G == 1) {
+                    q[0] = qd[j];
+                } else {
+#pragma unroll
+                    for (int g = 0; g < G; g += 2) {
+                        const double2 q2 = *reinterpret_cast<const double2 *>(qd + j * G + g);
+                        q[g] = q2.x;
+                        q[g + 1] = q2.y;
+                    }
+                }
 #pragma unroll
                 for (int g = 0; g < G; ++g) {
-                    const double2 qg = qq[j * G + g];
-                    ab[g] = __fma_rn(qg.x, lo, ab[g]);
-                    ab[g] = __fma_rn(qg.y, hi, ab[g]);
+                    const double k = __hiloint2double(__double2hiint(q[g]) < 0 ? lo_h : hi_h, 0);
+                    ab[g] = __fma_rn(q[g], k, ab[g]);
                 }
             }
         }
