@@ -173,7 +173,7 @@ def support_rows_of(wl, p_out):
 
 def run_gpu(args, rank, world):
     from sparse_entmax_kv_b200 import native as nv
-    from sparse_entmax_kv_b200.decoder import EntmaxKVDecoder, kernels_per_step, last_token_rows
+    from sparse_entmax_kv_b200.decoder import EntmaxKVDecoder, last_token_rows
     from sparse_entmax_kv_b200.workloads import CONFIGS, make_inputs
 
     wl = CONFIGS[args.workload]
@@ -183,7 +183,7 @@ def run_gpu(args, rank, world):
     dev = torch.device("cuda", torch.cuda.current_device())
     inp = make_inputs(wl, 1000 * 4 + rank, device=dev, sequential_pages=args.page_table == "sequential")
     dec = EntmaxKVDecoder(inp["k_cache"], inp["v_cache"], inp["page_table"], inp["seq_lens"], wl.Hq,
-                          alpha=wl.alpha, policy=policy, k=k, delta=delta)
+                          alpha=wl.alpha, policy=policy, k=k, delta=delta, fused=not args.unfused)
     dec.build_meta()
     # each sequence's newest token (position seq_len-1) is appended again every
     # step: its key/value rows are written to their slot and its page's
@@ -276,6 +276,19 @@ def run_gpu(args, rank, world):
                                       dec.sel, dec.cnt, dec.alpha, dec.out, dec.tau, None, dec.ws)
             e[4].record(st)
         torch.cuda.synchronize()
+        # the fused call of the product step (scores, selection with the
+        # union, q.K, tau with p.V), eagerly, after the same flush
+        fev = []
+        if dec.fused:
+            for i in range(args.steps):
+                l2_flush()
+                fev.append((torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)))
+                fev[-1][0].record(st)
+                nv.entmaxkv_decode_step(dec.shape, q, dec.meta, dec.k_cache, dec.v_cache, dec.page_table,
+                                        dec.seq_lens, dec.policy, dec.k, dec.alpha, dec.delta, dec.bbox, dec.mu,
+                                        dec.sigma, dec.sel, dec.cnt, dec.out, dec.tau_hat, dec.tau, None, dec.ws)
+                fev[-1][1].record(st)
+            torch.cuda.synchronize()
         t1 = time.perf_counter()
         while time.perf_counter() - t1 < 0.5:
             for _ in range(16):
@@ -307,6 +320,8 @@ def run_gpu(args, rank, world):
     step_ms, = max_over_ranks([step_ms], world, dev)
     stage_us = dict(zip(["append", "score_pages", "select", "decode_sparse"],
                         (stage_ms.mean(axis=0) * 1e3).round(2).tolist()))
+    if fev:
+        stage_us["decode_step"] = round(float(np.mean([a.elapsed_time(b) for a, b in fev])) * 1e3, 2)
     scan_b2b_us, = max_over_ranks([scan_b2b_us if scan_b2b_us is not None else -1.0], world, dev)
     scan_b2b_us = None if scan_b2b_us < 0 else scan_b2b_us
 
@@ -412,7 +427,7 @@ def run_gpu(args, rank, world):
                stage_us=stage_us, dense=dense, nbytes=nbytes, clocks=clocks,
                roofline=roofline, roofline_gather=roofline_gather, e2e_ms=e2e_step_ms, e2e_bytes=(stage_host.numel() * 2,
                                                                out_host.numel() * 4),
-               launches=kernels_per_step(dec.shape, wl.alpha, True) * args.steps, t_wall=t_wall,
+               launches=dec.kernels_per_step(True) * args.steps, fused=dec.fused, t_wall=t_wall,
                host=dict(inp=inp, dec=dec) if (rank == 0 and not args.no_cpu_baseline) else None)
     return res
 
@@ -714,6 +729,9 @@ def main():
                     help="instead of the benchmark line: selection scaling with context length (one line per L, policy)")
     ap.add_argument("--crossover", action="store_true",
                     help="instead of the benchmark line: sparse step vs full-cache decodes at growing L, tiny shape")
+    ap.add_argument("--unfused", action="store_true",
+                    help="step with the three separate calls (score, select, decode_sparse) instead of the fused "
+                         "entmaxkv_decode_step")
     ap.add_argument("--page-table", default="random", choices=["random", "sequential"],
                     help="physical placement of the logical pages: a seeded permutation (default) or in order")
     args = ap.parse_args()
@@ -748,6 +766,8 @@ def main():
     value = whole_job_gbs(nb["kv_touched"], world, res["step_ms"])
     e2e_val = whole_job_gbs(nb["kv_touched"], world, res["e2e_ms"])
     cfg = config_of(wl)
+    cfg["step"] = ("append + decode_step (scores, selection with the union, q.K, tau with p.V)" if res["fused"] else
+                   "append + score_pages + select + decode_sparse")
     if args.page_table == "sequential":
         cfg["page_table"] = "identity: logical pages in block order"
     line = {"metric": METRIC, "value": round(value, 2), "unit": "GB/s", "n_gpus": world, "steps": args.steps,
@@ -759,13 +779,17 @@ def main():
             "stages_us": res["stage_us"], "bytes_per_step": nb,
             "e2e": {"value": round(e2e_val, 2), "unit": "GB/s", "us_per_step": round(res["e2e_ms"] * 1e3, 2),
                     "h2d_bytes_per_step": res["e2e_bytes"][0], "d2h_bytes_per_step": res["e2e_bytes"][1],
-                    "how": "the four C-ABI calls, captured as one CUDA graph: append reads q and the appended "
+                    "how": "the step's C-ABI calls, captured as one CUDA graph: append reads q and the appended "
                            "token's k/v rows from pinned host memory over the bus (copying q to the device, writing "
                            "the rows and refreshing their pages' metadata); the decode writes the output straight "
                            "into pinned host memory",
                     "eager_us_per_step": round(res["e2e_eager_ms"] * 1e3, 2)},
-            "timing": "step = CUDA-graph replay of the four C-ABI calls; stages_us from the same calls issued "
-                      "eagerly with events around each (eager step sum %.2f us)" % (res["eager_step_ms"] * 1e3),
+            "timing": "step = CUDA-graph replay of %s; stages_us: entmaxkv_append, entmaxkv_score_pages, "
+                      "entmaxkv_select and entmaxkv_decode_sparse issued eagerly with events around each (sum %.2f "
+                      "us)%s" % ("entmaxkv_append + entmaxkv_decode_step" if res["fused"] else
+                                 "entmaxkv_append + entmaxkv_score_pages + entmaxkv_select + entmaxkv_decode_sparse",
+                                 res["eager_step_ms"] * 1e3,
+                                 ", decode_step the fused call alone" if res["fused"] else ""),
             "gpu_launches": res["launches"], "clocks": res["clocks"], "paper_context": PAPER_CONTEXT}
     if res["dense"]:
         de, ds = res["dense"]["dense_entmax"], res["dense"]["dense_softmax"]

@@ -111,7 +111,8 @@ enum { ENTMAXKV_TOPK = 0, ENTMAXKV_GAUSS = 1, ENTMAXKV_GAUSS_EST = 2 };
 enum {
     ENTMAXKV_CALL_SELECT = 2,
     ENTMAXKV_CALL_DECODE_SPARSE = 3,
-    ENTMAXKV_CALL_DECODE_DENSE = 4
+    ENTMAXKV_CALL_DECODE_DENSE = 4,
+    ENTMAXKV_CALL_DECODE_STEP = 5
 };
 
 /* bits of the device status word */
@@ -320,6 +321,46 @@ ENTMAXKV_API int entmaxkv_decode_sparse(const entmaxkv_shape *shape, const void 
  * Launches nothing.
  */
 ENTMAXKV_API int entmaxkv_decode_sparse_kernels(const entmaxkv_shape *shape, float alpha);
+
+/*
+ * One sparse decode step in one call: sections 2.A, 2.B and 2.C of the
+ * summary in sequence -- page scores (as entmaxkv_score_pages), selection (as
+ * entmaxkv_select) and sparse entmax attention over the selected pages (as
+ * entmaxkv_decode_sparse) -- with the same arguments, outputs and errors as
+ * those three calls made one after the other, and bit-identical results.
+ * What differs is the work between them: the selection kernel also prepares
+ * each GQA group's union of selected pages -- it marks its kept pages in a
+ * per-group page map in the workspace, which one small kernel per group then
+ * compacts (one read of the map, no pass over the selection lists); with one
+ * query head per group the selection list is the union and is written as
+ * such, with its physical blocks.  The step is five kernels (scoring,
+ * selection, union, q.K, tau with p.V), four with one query head per group;
+ * entmaxkv_decode_step_kernels gives the count.  Rows of more than 16384
+ * pages fall back to the separate union pass of entmaxkv_decode_sparse.
+ * - alpha must be > 1 (entmax; ENTMAXKV_ERR_ALPHA otherwise).  mu and sigma
+ *   are required by the Gaussian policies; with top-k they may both be NULL
+ *   (the bound alone is scored).
+ * - workspace: entmaxkv_workspace_size(shape, ENTMAXKV_CALL_DECODE_STEP)
+ *   bytes, 256-byte aligned; its contents need no initialisation (the scoring
+ *   kernel clears the page map every call).
+ * - bbox/mu/sigma, sel/cnt/tau_hat, out/tau_out/p_out: as in the three calls.
+ */
+ENTMAXKV_API int entmaxkv_decode_step(const entmaxkv_shape *shape, const void *q, const void *meta,
+                         const void *k_cache, const void *v_cache,
+                         const int32_t *page_table, const int32_t *seq_lens,
+                         int32_t policy, int32_t k, float alpha, float delta,
+                         float *bbox, float *mu, float *sigma,
+                         int32_t *sel, int32_t *cnt, float *tau_hat,
+                         float *out, float *tau_out, float *p_out,
+                         void *workspace, size_t ws_bytes, void *stream);
+
+/*
+ * The number of kernels one entmaxkv_decode_step call with this shape, policy
+ * and alpha launches (5, 4 with one query head per group, more for rows of
+ * more than 16384 pages).  Negative
+ * ENTMAXKV_ERR_* on a bad shape, policy or alpha.  Launches nothing.
+ */
+ENTMAXKV_API int entmaxkv_decode_step_kernels(const entmaxkv_shape *shape, int32_t policy, float alpha);
 
 /*
  * Allocation-free form of entmaxkv_decode_sparse (the EntmaxKV summary has no

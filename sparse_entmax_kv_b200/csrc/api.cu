@@ -187,6 +187,9 @@ size_t entmaxkv_workspace_size(const entmaxkv_shape *s, int call) {
         case ENTMAXKV_CALL_DECODE_DENSE:
             return decode_ws_bytes(call == ENTMAXKV_CALL_DECODE_DENSE, s->B, s->Hq, s->Hkv, s->d, s->page_size,
                                    s->max_pages, nullptr, nullptr);
+        case ENTMAXKV_CALL_DECODE_STEP:
+            return decode_ws_bytes(false, s->B, s->Hq, s->Hkv, s->d, s->page_size, s->max_pages, nullptr, nullptr,
+                                   true);
         default: return (size_t)-1;
     }
 }
@@ -419,6 +422,120 @@ int entmaxkv_decode_sparse(const entmaxkv_shape *s, const void *q, const void *k
     if ((rc = make_kv_map(&a.kmap, k_cache, s))) return rc;
     if (alpha == 1.f && (rc = make_kv_map(&a.vmap, v_cache, s))) return rc;
     return cuda_rc(launch_decode_sparse(a, static_cast<cudaStream_t>(stream)));
+}
+
+int entmaxkv_decode_step(const entmaxkv_shape *s, const void *q, const void *meta, const void *k_cache,
+                         const void *v_cache, const int32_t *page_table, const int32_t *seq_lens, int32_t policy,
+                         int32_t k, float alpha, float delta, float *bbox, float *mu, float *sigma, int32_t *sel,
+                         int32_t *cnt, float *tau_hat, float *out, float *tau_out, float *p_out, void *workspace,
+                         size_t ws_bytes, void *stream) {
+    int rc = check_shape(s);
+    if (rc) return rc;
+    if (s->max_pages > MAX_SEL_PAGES) return ENTMAXKV_ERR_SHAPE;
+    if (!meta || !bbox || !sel || !cnt) return ENTMAXKV_ERR_NULL;
+    if ((mu == nullptr) != (sigma == nullptr)) return ENTMAXKV_ERR_NULL;
+    if (!std::isfinite(alpha) || !(alpha > 1.f)) return ENTMAXKV_ERR_ALPHA;
+    SelectArgs la{};
+    if (policy == ENTMAXKV_TOPK) {
+        if (k < 1) return ENTMAXKV_ERR_POLICY;
+    } else if (policy == ENTMAXKV_GAUSS || policy == ENTMAXKV_GAUSS_EST) {
+        if (!mu) return ENTMAXKV_ERR_NULL;
+        if (!std::isfinite(delta)) return ENTMAXKV_ERR_POLICY;
+        la.r_int = integer_r(alpha);
+        if (la.r_int == 0) return ENTMAXKV_ERR_UNSUPPORTED;
+    } else {
+        return ENTMAXKV_ERR_POLICY;
+    }
+    if (!aligned16(meta)) return ENTMAXKV_ERR_ALIGN;
+    const size_t need =
+        decode_ws_bytes(false, s->B, s->Hq, s->Hkv, s->d, s->page_size, s->max_pages, nullptr, nullptr, true);
+    if (!workspace || ws_bytes < need) return ENTMAXKV_ERR_WORKSPACE;
+    DecodeArgs da;
+    if ((rc = fill_decode(false, s, q, k_cache, v_cache, page_table, seq_lens, alpha, out, tau_out, p_out,
+                          workspace, ws_bytes, &da)))
+        return rc;
+    decode_ws_bytes(false, s->B, s->Hq, s->Hkv, s->d, s->page_size, s->max_pages, &da.ws, workspace, true);
+    da.sel = sel;
+    da.cnt = cnt;
+    if ((rc = make_kv_map(&da.kmap, k_cache, s))) return rc;
+
+    const int G = s->Hq / s->Hkv;
+    la.seq_lens = seq_lens;
+    la.bbox = bbox;
+    la.mu = mu;
+    la.sigma = sigma;
+    la.sel = sel;
+    la.cnt = cnt;
+    la.tau_hat = tau_hat;
+    la.B = s->B;
+    la.Hq = s->Hq;
+    la.P = s->page_size;
+    la.max_pages = s->max_pages;
+    la.policy = policy;
+    la.k = k;
+    la.alpha = alpha;
+    la.delta = delta;
+    la.h0 = da.kv0 * G;
+    la.nh = da.nk * G;
+    la.status = da.status;
+    la.Hkv = s->Hkv;
+    la.num_blocks = s->num_blocks;
+    const bool fused = select_marks_union(la);
+    if (fused) {
+        la.umap = da.ws.umap;
+        la.uwords = da.ws.uwords;
+        la.union_e = da.ws.union_e;
+        la.union_blk = da.ws.union_blk;
+        la.union_cnt = da.ws.union_cnt;
+        la.zmax = da.ws.zmax;
+        la.page_table = page_table;
+    }
+
+    ScoreArgs sa{};
+    sa.q = static_cast<const uint16_t *>(q);
+    sa.meta = static_cast<const uint8_t *>(meta);
+    sa.seq_lens = seq_lens;
+    sa.bbox = bbox;
+    sa.mu = mu;
+    sa.sigma = sigma;
+    sa.n_tiles = meta_tiles(s->max_pages);
+    sa.n_tiles_total = (long long)s->B * s->Hkv * sa.n_tiles;
+    sa.B = s->B;
+    sa.Hq = s->Hq;
+    sa.Hkv = s->Hkv;
+    sa.d = s->d;
+    sa.P = s->page_size;
+    sa.max_pages = s->max_pages;
+    sa.kv0 = da.kv0;
+    sa.nk = da.nk;
+    sa.status = da.status;
+    if (fused && G > 1) {
+        // the union marks: from umap to the end of the workspace
+        sa.zero = reinterpret_cast<uint4 *>(da.ws.umap);
+        sa.zero16 = (long long)((static_cast<char *>(workspace) + need) - reinterpret_cast<char *>(da.ws.umap)) / 16;
+    }
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    cudaError_t e = launch_score_pages(sa, st);
+    if (e == cudaSuccess) e = launch_select(la, st);
+    if (e == cudaSuccess) e = fused ? launch_decode_step_tail(da, st) : launch_decode_sparse(da, st);
+    return cuda_rc(e);
+}
+
+int entmaxkv_decode_step_kernels(const entmaxkv_shape *s, int32_t policy, float alpha) {
+    int rc = check_shape(s);
+    if (rc) return rc;
+    if (!std::isfinite(alpha) || !(alpha > 1.f)) return ENTMAXKV_ERR_ALPHA;
+    if (policy != ENTMAXKV_TOPK && policy != ENTMAXKV_GAUSS && policy != ENTMAXKV_GAUSS_EST)
+        return ENTMAXKV_ERR_POLICY;
+    if ((rc = entmaxkv_decode_sparse_kernels(s, alpha)) < 0) return rc;
+    SelectArgs la{};
+    la.policy = policy;
+    la.max_pages = s->max_pages;
+    if (!select_marks_union(la)) return 2 + rc;  // score, select, then the separate decode
+    DecodeArgs da{};
+    da.Hq = s->Hq;
+    da.Hkv = s->Hkv;
+    return 2 + decode_step_tail_kernels(da);
 }
 
 int entmaxkv_decode_sparse_kernels(const entmaxkv_shape *s, float alpha) {

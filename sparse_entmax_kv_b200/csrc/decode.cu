@@ -160,6 +160,110 @@ __global__ void __launch_bounds__(UTH) union_kernel(DecodeArgs a) {
     if (threadIdx.x == 0) a.ws.union_cnt[bk] = done;
 }
 
+// Union of a group's selections from the marks the selection kernel left
+// (decode step, G > 1): byte p of the group's row of ws.umap holds the head
+// bits of page p.  One CTA per (sequence, kv head); the page-table row is
+// sent to L2 before the dependency wait.  Per pass of UM_WPT words (4 UM_WPT
+// pages) a thread, all loads of a pass issued together:
+//   1. its words go to shared memory and a block scan of their marked-page
+//      counts gives each thread its first position;
+//   2. the entries are dealt round-robin to the threads, each finding its
+//      entry's page by a binary search over those positions, and the
+//      page-table entries of four entries per thread are loaded together
+//      before they are written.
+// It also resets the q.K pass's running max of the group's heads.
+constexpr int UMT = 512;
+constexpr int UM_WPT = 8;
+
+// Bit j set where byte j of w is non-zero.
+__device__ __forceinline__ unsigned nz_bytes(unsigned w) {
+    return (w & 0xffu ? 1u : 0u) | (w & 0xff00u ? 2u : 0u) | (w & 0xff0000u ? 4u : 0u) | (w & 0xff000000u ? 8u : 0u);
+}
+
+__global__ void __launch_bounds__(UMT) union_map_kernel(DecodeArgs a) {
+    {
+        const int b0 = blockIdx.x / a.nk;
+        const char *prow = reinterpret_cast<const char *>(a.page_table + (size_t)b0 * a.max_pages);
+        for (int l = threadIdx.x; l * 32 < a.max_pages; l += UMT)
+            asm volatile("prefetch.global.L2 [%0];" ::"l"(prow + (size_t)l * 128));
+    }
+    pdl_wait();
+    __shared__ unsigned words[UMT * UM_WPT];
+    __shared__ int pre[UMT];
+    __shared__ int sh[72];
+    int b, kvh;
+    group_of(blockIdx.x, a.kv0, a.nk, b, kvh);
+    const int bk = b * a.Hkv + kvh;
+    const int G = a.Hq / a.Hkv;
+    if (threadIdx.x < G) a.ws.zmax[b * a.Hq + kvh * G + threadIdx.x] = ORD_NEG_INF;
+    const int np = n_pages_of(seq_len_of(a.seq_lens, b, a.P, a.max_pages, a.status), a.P);
+    const int nw = ceil_div(np, 4);
+    const unsigned *row = a.ws.umap + (size_t)bk * a.ws.uwords;
+    const int *pt = a.page_table + (size_t)b * a.max_pages;
+    int *ue = a.ws.union_e + (size_t)bk * a.max_pages;
+    int *ub = a.ws.union_blk + (size_t)bk * a.max_pages;
+    int done = 0;
+    for (int base = 0; base < nw; base += UMT * UM_WPT) {
+        const int w0 = base + threadIdx.x * UM_WPT;  // a multiple of 4: 16-byte loads (rows are 16-byte aligned)
+        int mine = 0;
+#pragma unroll
+        for (int i = 0; i < UM_WPT; i += 4) {
+            uint4 v = make_uint4(0u, 0u, 0u, 0u);
+            if (w0 + i < nw) v = __ldcg(reinterpret_cast<const uint4 *>(row + w0 + i));
+            unsigned *dst = words + threadIdx.x * UM_WPT + i;
+            dst[0] = v.x;
+            dst[1] = v.y;
+            dst[2] = v.z;
+            dst[3] = v.w;
+            mine += __popc(nz_bytes(v.x)) + __popc(nz_bytes(v.y)) + __popc(nz_bytes(v.z)) + __popc(nz_bytes(v.w));
+        }
+        int tot;
+        pre[threadIdx.x] = block_excl_scan(mine, sh, &tot);
+        __syncthreads();
+        for (int e0 = 0; e0 < tot; e0 += 4 * UMT) {
+            int page[4], mask[4], blk[4];
+#pragma unroll
+            for (int u = 0; u < 4; ++u) {
+                const int e = e0 + u * UMT + (int)threadIdx.x;
+                page[u] = -1;
+                if (e >= tot) continue;
+                int lo = 0, hi = UMT - 1;  // the last thread whose first position is <= e
+                while (lo < hi) {
+                    const int mid = (lo + hi + 1) >> 1;
+                    if (pre[mid] <= e) lo = mid;
+                    else hi = mid - 1;
+                }
+                int r = e - pre[lo];  // that thread holds more than r marked pages
+                const unsigned *wsrc = words + lo * UM_WPT;
+                int i = 0;
+                unsigned m = nz_bytes(wsrc[0]);
+                while (r >= __popc(m)) {
+                    r -= __popc(m);
+                    m = nz_bytes(wsrc[++i]);
+                }
+                while (r-- > 0) m &= m - 1u;
+                const int j = __ffs(m) - 1;
+                page[u] = 4 * (base + lo * UM_WPT + i) + j;
+                mask[u] = (int)((wsrc[i] >> (8 * j)) & 0xffu);
+            }
+#pragma unroll
+            for (int u = 0; u < 4; ++u) blk[u] = page[u] >= 0 ? __ldg(pt + page[u]) : -1;
+#pragma unroll
+            for (int u = 0; u < 4; ++u)
+                if (page[u] >= 0) {
+                    const bool ok = blk[u] >= 0 && blk[u] < a.num_blocks;
+                    if (!ok) atomicOr(a.status, ENTMAXKV_STATUS_BAD_PAGE);
+                    const int pos = done + e0 + u * UMT + (int)threadIdx.x;
+                    ue[pos] = (page[u] << 8) | mask[u];
+                    ub[pos] = ok ? blk[u] : -1;
+                }
+        }
+        done += tot;
+        __syncthreads();  // the words are read before the next pass overwrites them
+    }
+    if (threadIdx.x == 0) a.ws.union_cnt[bk] = done;
+}
+
 __global__ void dense_init_kernel(DecodeArgs a) {
     pdl_wait();
     const int i = blockIdx.x * blockDim.x + threadIdx.x;
@@ -611,18 +715,25 @@ inline int tau_zcap(int ctas, int sms) {
 // Newton's method, for r >= 1 (alpha <= 2) on g(t) = (sum_c [z_c - t]_+^r)^(1/r),
 // a norm of (z - t)_+ and so convex (one step when the support's z are equal),
 // from the left end; for r < 1 on F, which is then concave, from the right
-// end: either way the iterates move to the root monotonically.  for_each(add)
-// calls add(z) on this thread's share of the candidates; each thread's sums
-// are added in warp order (reproducible) and every warp takes the same step,
-// one barrier per pass (red is double-buffered).  All TAU_NT threads call it.
+// end: either way the iterates move to the root monotonically.
+// for_each(add, first, stride) calls add(z) on candidates first, first +
+// stride, ...  With n candidates, n <= TAU_WARP_MAX, warp 0 runs every pass
+// by itself (lane-strided sums, a shuffle butterfly) and hands t to the other
+// warps with one barrier at the end.  Otherwise each thread takes a
+// TAU_NT-strided share and the warps' sums are added in warp order
+// (reproducible), one barrier per pass (red is double-buffered).  All TAU_NT
+// threads call it and return the same t.
+constexpr int TAU_WARP_MAX = 256;
 template <class ForEach>
-__device__ float entmax_tau(ForEach for_each, float lo, float hi, float zmax, float r, int ri,
+__device__ float entmax_tau(ForEach for_each, int n, float lo, float hi, float zmax, float r, int ri,
                             float (*red)[TAU_NW][2]) {
     const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+    const bool per_warp = n <= TAU_WARP_MAX;
+    const int first = per_warp ? lane : (int)threadIdx.x, stride = per_warp ? 32 : TAU_NT;
     const float tol = 1e-7f * fmaxf(1.f, fabsf(zmax));
     const int rim1 = ri >= 2 ? ri - 1 : 0;
     float t = r >= 1.f ? lo : hi;
-    for (int it = 0; it < 40; ++it) {
+    for (int it = 0; it < 40 && (!per_warp || warp == 0); ++it) {
         float s0 = 0.f, s1 = 0.f;  // sum x^r, sum x^(r-1) over x = z - t > 0
         auto add = [&](float z) {
             const float x = z - t;
@@ -636,22 +747,26 @@ __device__ float entmax_tau(ForEach for_each, float lo, float hi, float zmax, fl
                 s1 += y;
             }
         };
-        for_each(add);
+        for_each(add, first, stride);
 #pragma unroll
         for (int o = 16; o; o >>= 1) {
             s0 += __shfl_xor_sync(FULL, s0, o);
             s1 += __shfl_xor_sync(FULL, s1, o);
         }
-        if (lane == 0) {
-            red[it & 1][warp][0] = s0;
-            red[it & 1][warp][1] = s1;
-        }
-        __syncthreads();
-        float S0 = 0.f, S1 = 0.f;
+        float S0 = s0, S1 = s1;
+        if (!per_warp) {
+            if (lane == 0) {
+                red[it & 1][warp][0] = s0;
+                red[it & 1][warp][1] = s1;
+            }
+            __syncthreads();
+            S0 = 0.f;
+            S1 = 0.f;
 #pragma unroll
-        for (int ww = 0; ww < TAU_NW; ++ww) {
-            S0 += red[it & 1][ww][0];
-            S1 += red[it & 1][ww][1];
+            for (int ww = 0; ww < TAU_NW; ++ww) {
+                S0 += red[it & 1][ww][0];
+                S1 += red[it & 1][ww][1];
+            }
         }
         if (!(S1 > 0.f)) break;  // no weight right of t (t at the top already)
         // r >= 1: t' = t + (S0 - S0^(1-1/r)) / S1;  r < 1: t' = t + (S0 - 1) / (r S1)
@@ -664,6 +779,12 @@ __device__ float entmax_tau(ForEach for_each, float lo, float hi, float zmax, fl
         const bool done = !(fabsf(tn - t) > tol);
         t = tn;
         if (done) break;
+    }
+    if (per_warp) {
+        __syncthreads();  // every warp is past the caller's earlier use of red
+        if (threadIdx.x == 0) red[0][0][0] = t;
+        __syncthreads();
+        t = red[0][0][0];
     }
     return t;
 }
@@ -918,22 +1039,23 @@ __global__ void __launch_bounds__(TAU_NT, D == 64 ? 4 : 3) tau_pv_kernel(const _
         const float hi = zmax - powf((float)(onchip ? nc : n_tok), 1.f - a.alpha);
         if (nc > 1 && hi > lo) {
             if (onchip) {
-                tau = entmax_tau([&](auto add) { for (int c = threadIdx.x; c < nc; c += TAU_NT) add(cz[c]); },
+                tau = entmax_tau([&](auto add, int f, int st) { for (int c = f; c < nc; c += st) add(cz[c]); }, nc,
                                  lo, hi, zmax, r, ri, red);
             } else {
                 // too many candidates to hold: stream the z row through shared
                 // memory in coalesced chunks of zcap
+                // (n_tok > zcap >= 1024 here: the block-wide form)
                 tau = entmax_tau(
-                    [&](auto add) {
+                    [&](auto add, int f, int st) {
                         for (int c0 = 0; c0 < n_tok; c0 += zcap) {
                             const int m = min(zcap, n_tok - c0);
                             __syncthreads();  // the previous chunk has been read
                             for (int i = threadIdx.x; i < m; i += TAU_NT) cz[i] = __ldcg(zr + c0 + i);
                             __syncthreads();
-                            for (int c = threadIdx.x; c < m; c += TAU_NT) add(cz[c]);
+                            for (int c = f; c < m; c += st) add(cz[c]);
                         }
                     },
-                    lo, hi, zmax, r, ri, red);
+                    n_tok, lo, hi, zmax, r, ri, red);
             }
         }
     }
@@ -1093,8 +1215,8 @@ __global__ void __launch_bounds__(TAU_NT) threshold_kernel(const __grid_constant
     const float lo = zmax - 1.f, hi = zmax - powf((float)n, 1.f - a.alpha);
     float tau = lo;
     if (n > 1 && hi > lo)
-        tau = entmax_tau([&](auto add) { for (int c = threadIdx.x; c < n; c += TAU_NT) add(tz[c]); }, lo, hi, zmax,
-                         r, a.r_int, red);
+        tau = entmax_tau([&](auto add, int f, int st) { for (int c = f; c < n; c += st) add(tz[c]); }, n, lo, hi,
+                         zmax, r, a.r_int, red);
     if (threadIdx.x == 0) a.tau[bh] = tau;
 }
 
@@ -1537,6 +1659,22 @@ cudaError_t sparse_t(const DecodeArgs &a, cudaStream_t st) {
     return launch_pdl(tau_pv_kernel<D, true>, dim3(nheads), dim3(TAU_NT), tau_smem(zcap), st, u, 0, zcap);
 }
 
+// The decode of a step whose selection kernel marked each group's union in
+// ws.umap (G > 1: union_map_kernel compacts it) or wrote it (G = 1), then
+// q.K and tau with p.V.
+template <int D, int G>
+cudaError_t step_tail_t(const DecodeArgs &a, cudaStream_t st) {
+    cudaError_t e;
+    DecodeArgs u = a;
+    u.union_in_qk = 0;
+    if (G > 1 && (e = launch_pdl(union_map_kernel, dim3(a.B * a.nk), dim3(UMT), 0, st, u)) != cudaSuccess) return e;
+    if ((e = launch_qk<D, G, false>(u, st)) != cudaSuccess) return e;
+    const int nheads = a.B * a.nk * G;
+    const int zcap = tau_zcap(nheads, a.sms);
+    if ((e = set_smem(tau_pv_kernel<D, true>, tau_smem(ZCAP_MAX))) != cudaSuccess) return e;
+    return launch_pdl(tau_pv_kernel<D, true>, dim3(nheads), dim3(TAU_NT), tau_smem(zcap), st, u, 0, zcap);
+}
+
 template <int D, int G>
 cudaError_t begin_t(const DecodeArgs &a, cudaStream_t st) {
     cudaError_t e;
@@ -1641,6 +1779,8 @@ int decode_sparse_kernels(const DecodeArgs &a) {
     }
     return -1;
 }
+cudaError_t launch_decode_step_tail(const DecodeArgs &a, cudaStream_t st) { EKV_DISPATCH(step_tail_t, a, st); }
+int decode_step_tail_kernels(const DecodeArgs &a) { return a.Hq / a.Hkv > 1 ? 3 : 2; }
 cudaError_t launch_decode_sparse_begin(const DecodeArgs &a, cudaStream_t st) { EKV_DISPATCH(begin_t, a, st); }
 cudaError_t launch_decode_sparse_candidates(const DecodeArgs &a, cudaStream_t st) {
     EKV_DISPATCH(candidates_t, a, st);
@@ -1660,7 +1800,7 @@ cudaError_t launch_decode_dense_softmax(const DecodeArgs &a, cudaStream_t st) {
 }
 
 size_t decode_ws_bytes(bool dense, int B, int Hq, int Hkv, int d, int P, int max_pages, DecodeWs *carve,
-                       void *base) {
+                       void *base, bool step) {
     size_t off = 0;
     auto take = [&](size_t bytes) {
         size_t o = off;
@@ -1668,6 +1808,7 @@ size_t decode_ws_bytes(bool dense, int B, int Hq, int Hkv, int d, int P, int max
         return o;
     };
     const size_t tokens = (size_t)B * Hq * max_pages * P;
+    const int uwords = (ceil_div(max_pages, 4) + 3) & ~3;
     const size_t o_union = take(dense ? 0 : (size_t)B * Hkv * max_pages * 4);
     const size_t o_ublk = take(dense ? 0 : (size_t)B * Hkv * max_pages * 4);
     const size_t o_ucnt = take((size_t)B * Hkv * 4);
@@ -1677,6 +1818,8 @@ size_t decode_ws_bytes(bool dense, int B, int Hq, int Hkv, int d, int P, int max
     const size_t o_part = take((size_t)MAX_SPLITS * B * Hq * (d + 2) * 4);  // split-K softmax partials
     const size_t o_z = take(tokens * 4);
     const size_t o_t = take(tokens / 16 * 4);
+    // decode step: the union marks, last (cleared from there to the end)
+    const size_t o_umap = take(step ? (size_t)B * Hkv * uwords * 4 : 0);
     if (carve && base) {
         char *p = static_cast<char *>(base);
         carve->union_e = reinterpret_cast<int *>(p + o_union);
@@ -1688,6 +1831,8 @@ size_t decode_ws_bytes(bool dense, int B, int Hq, int Hkv, int d, int P, int max
         carve->partial = reinterpret_cast<float *>(p + o_part);
         carve->zbuf = reinterpret_cast<float *>(p + o_z);
         carve->tmax = reinterpret_cast<float *>(p + o_t);
+        carve->umap = step ? reinterpret_cast<unsigned *>(p + o_umap) : nullptr;
+        carve->uwords = uwords;
     }
     return off;
 }

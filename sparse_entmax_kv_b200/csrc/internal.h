@@ -69,6 +69,10 @@ struct ScoreArgs {
     int B, Hq, Hkv, d, P, max_pages;
     int kv0, nk;  // kv-head range [kv0, kv0 + nk)
     int *status;
+    // decode step: zero16 16-byte words at zero are cleared (the union marks
+    // and group counters that the selection of the same step then fills)
+    uint4 *zero;
+    long long zero16;
 };
 cudaError_t launch_score_pages(const ScoreArgs &a, cudaStream_t st);
 
@@ -83,8 +87,21 @@ struct SelectArgs {
     int r_int;  // 1/(alpha-1) for the Gaussian policy
     int h0, nh;  // query-head range [h0, h0 + nh)
     int *status;
+    // decode step (umap non-null): the union of each group's selections for
+    // the q.K pass.  G > 1: each CTA ORs the head bit of every page it keeps
+    // into that page's byte of the group's row of umap (zero on entry, uwords
+    // words a row), which the decode's union_map_kernel compacts.  G = 1: the
+    // selection list is written as the union (union_e / union_blk / union_cnt,
+    // the decode workspace's layout, with page_table looked up) and zmax is
+    // reset.
+    unsigned *umap;
+    int uwords;
+    int *union_e, *union_blk, *union_cnt, *zmax;
+    const int *page_table;
+    int Hkv, num_blocks;
 };
 cudaError_t launch_select(const SelectArgs &a, cudaStream_t st);
+bool select_marks_union(const SelectArgs &a);  // whether launch_select can prepare the union for this shape
 
 // Workspace carve-up shared by the decode paths.
 struct DecodeWs {
@@ -97,6 +114,8 @@ struct DecodeWs {
     float *partial;  // [MAX_SPLITS][B*Hq][d+2]  (dense paths)
     float *zbuf;     // [B*Hq][max_pages*P]  z of every token of the page list, in list order
     float *tmax;     // [B*Hq][max_pages*P/16]  max z of each 16-token tile of zbuf
+    unsigned *umap;  // [B*Hkv][uwords]  decode step: head bits per page, a byte each (4 pages a word)
+    int uwords;      // words per umap row: ceil(max_pages / 4) rounded up to a multiple of 4
 };
 
 struct DecodeArgs {
@@ -130,6 +149,10 @@ int decode_sparse_kernels(const DecodeArgs &a);  // launches of one launch_decod
 cudaError_t launch_decode_sparse_begin(const DecodeArgs &a, cudaStream_t st);
 cudaError_t launch_decode_sparse_candidates(const DecodeArgs &a, cudaStream_t st);
 cudaError_t launch_decode_sparse_finish(const DecodeArgs &a, cudaStream_t st);
+// The decode of a step whose selection marked the union (G > 1: union_map_kernel
+// compacts the marks) or wrote it (G = 1): then q.K and tau with p.V
+cudaError_t launch_decode_step_tail(const DecodeArgs &a, cudaStream_t st);
+int decode_step_tail_kernels(const DecodeArgs &a);
 
 struct ThresholdArgs {
     const float *cand_z;  // [S][B*Hq][cap]
@@ -145,7 +168,9 @@ cudaError_t launch_entmax_threshold(const ThresholdArgs &a, cudaStream_t st);
 cudaError_t launch_decode_dense_entmax(const DecodeArgs &a, cudaStream_t st);
 cudaError_t launch_decode_dense_softmax(const DecodeArgs &a, cudaStream_t st);
 
+// Workspace of a decode call; step adds the union marks of
+// entmaxkv_decode_step (last, so that one clear from there to the end covers them).
 size_t decode_ws_bytes(bool dense, int B, int Hq, int Hkv, int d, int P, int max_pages, DecodeWs *carve,
-                      void *base);
+                      void *base, bool step = false);
 
 }  // namespace ekv

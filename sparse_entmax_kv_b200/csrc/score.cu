@@ -69,6 +69,12 @@ constexpr size_t smem_bytes() {
 template <int D, int G, bool GAUSS>
 __global__ void __launch_bounds__(THREADS, G <= 4 ? (GAUSS ? 2 : 3) : 1) score_kernel(ScoreArgs a) {
     pdl_wait();
+    if (a.zero) {  // decode step: clear the selection's union marks and counters
+        const long long stride = (long long)gridDim.x * gridDim.y * THREADS;
+        for (long long i = ((long long)blockIdx.y * gridDim.x + blockIdx.x) * THREADS + threadIdx.x; i < a.zero16;
+             i += stride)
+            a.zero[i] = make_uint4(0u, 0u, 0u, 0u);
+    }
     using RG = Ring<GAUSS>;
     constexpr int CPS = RG::CPS;
     constexpr int NCH = D / CHK / CPS;  // ring stages per tile

@@ -39,6 +39,47 @@ __device__ __forceinline__ unsigned key_of(float f) {
 
 
 
+// ------------------------------------------ the group union (decode step)
+//
+// With a.umap set (the decode step), the selection also prepares the union
+// of the G heads' selections of each (sequence, kv head) group for the q.K
+// pass.  With G = 1 the selection list is the union: each entry is written
+// beside the selection with its page-table entry (union_e / union_blk /
+// union_cnt, as the decode workspace holds them), and the q.K pass's running
+// max is reset.  With G > 1 every CTA ORs head g's bit into byte p of its
+// group's row of umap for each page p it keeps (the row is zero on entry);
+// a separate kernel of the decode then compacts the rows.
+
+// Page-table entries of the kept pages among p0 .. p0+15 (bit i: page p0+i),
+// all loads issued together; -1 elsewhere.
+__device__ __forceinline__ void blocks16(const int *pt, int p0, unsigned bits, int (&blk)[16]) {
+#pragma unroll
+    for (int i = 0; i < 16; ++i) blk[i] = (bits >> i) & 1u ? __ldg(pt + p0 + i) : -1;
+}
+
+// G = 1: union entry `pos` is the kept page p with physical block blk.
+__device__ __forceinline__ void union_entry(const SelectArgs &a, int *ue, int *ub, int pos, int p, int blk) {
+    const bool ok = blk >= 0 && blk < a.num_blocks;
+    if (!ok) atomicOr(a.status, ENTMAXKV_STATUS_BAD_PAGE);
+    ue[pos] = (p << 8) | 1;
+    ub[pos] = ok ? blk : -1;
+}
+
+// G > 1: marks the kept pages among p0 .. p0+15 (p0 a multiple of 16) for
+// head g: one OR per 4-page word holding a kept page.
+__device__ __forceinline__ void mark16(unsigned *row, int p0, unsigned bits, int g) {
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+        const unsigned nib = (bits >> (4 * j)) & 0xfu;
+        if (nib) {
+            unsigned w = 0u;
+#pragma unroll
+            for (int i = 0; i < 4; ++i) w |= ((nib >> i) & 1u) << (8 * i + g);
+            atomicOr(row + (p0 >> 2) + j, w);
+        }
+    }
+}
+
 // Top-k: the keys of one tile (TILE pages) stay in registers, ITEMS
 // consecutive pages per thread, through the four radix passes and the final
 // ordered compaction; longer sequences take several tiles per pass.
@@ -57,9 +98,36 @@ __global__ void __launch_bounds__(NT) topk_kernel(SelectArgs a) {
     const float *sc = a.bbox + (size_t)bh * a.max_pages;
     int *sel = a.sel + (size_t)bh * a.max_pages;
     const int k = min(a.k, n);
+    // decode step: the group's union (see above)
+    const int G = a.Hq / a.Hkv;
+    const bool uni = a.umap != nullptr;
+    const int bk = b * a.Hkv + h / G;
+    const int *pt = a.page_table + (size_t)b * a.max_pages;  // (read only when uni)
     if (k >= n) {
+        unsigned *urow = a.umap + (size_t)bk * a.uwords;
+        int *ue = a.union_e + (size_t)bk * a.max_pages, *ub = a.union_blk + (size_t)bk * a.max_pages;
         for (int p = threadIdx.x; p < n; p += blockDim.x) sel[p] = p;
         if (threadIdx.x == 0) a.cnt[bh] = n;
+        if (uni) {
+            for (int p0 = threadIdx.x * 16; p0 < n; p0 += NT * 16) {
+                const unsigned bits = n - p0 >= 16 ? 0xffffu : (1u << (n - p0)) - 1u;
+                if (G > 1) {
+                    mark16(a.umap + (size_t)bk * a.uwords, p0, bits, h % G);
+                } else {
+                    int blk[16];
+                    blocks16(pt, p0, bits, blk);
+#pragma unroll
+                    for (int i = 0; i < 16; ++i)
+                        if ((bits >> i) & 1u)
+                            union_entry(a, a.union_e + (size_t)bk * a.max_pages,
+                                        a.union_blk + (size_t)bk * a.max_pages, p0 + i, p0 + i, blk[i]);
+                }
+            }
+            if (G == 1 && threadIdx.x == 0) {
+                a.union_cnt[bk] = n;
+                a.zmax[bh] = ORD_NEG_INF;
+            }
+        }
         return;
     }
     const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
@@ -130,6 +198,8 @@ __global__ void __launch_bounds__(NT) topk_kernel(SelectArgs a) {
     const unsigned T = prefix;
     // keys == T are taken in page order up to `remaining` of them
     int eq_base = 0, base = 0;
+    unsigned u_take = 0u;  // decode step (one tile): this thread's kept pages
+    int u_pos = 0;         // and the list position of the first
     for (int t0 = 0; t0 < n; t0 += TILE_NT) {
         if (!one_tile) load_tile(t0);
         const int p0 = t0 + threadIdx.x * ITEMS;
@@ -150,8 +220,15 @@ __global__ void __launch_bounds__(NT) topk_kernel(SelectArgs a) {
                 if (eq_off < remaining) take |= 1u << i;
                 ++eq_off;
             }
+        if (uni && G > 1) mark16(a.umap + (size_t)bk * a.uwords, p0, take, h % G);  // complete behind the scan
+        if (uni && G == 1)  // page-table entries to L2 during the scan (no registers held)
+#pragma unroll
+            for (int i = 0; i < ITEMS; ++i)
+                if ((take >> i) & 1u) asm volatile("prefetch.global.L2 [%0];" ::"l"(pt + p0 + i));
         int tot;
         int w = base + block_excl_scan(__popc(take), sh, &tot);
+        u_take = take;
+        u_pos = w;
 #pragma unroll
         for (int i = 0; i < ITEMS; ++i)
             if (take & (1u << i)) sel[w++] = p0 + i;
@@ -159,6 +236,22 @@ __global__ void __launch_bounds__(NT) topk_kernel(SelectArgs a) {
         eq_base += eq_tot;
     }
     if (threadIdx.x == 0) a.cnt[bh] = base;
+    if (uni && G == 1) {
+        // one tile (the decode step's limit): this thread's kept pages and
+        // their first list position are u_take and u_pos; the keys are dead
+        // now, which leaves registers for the page-table entries
+        const int p0 = threadIdx.x * ITEMS;
+        int blk[ITEMS];
+        blocks16(pt, p0, u_take, blk);
+        int *ue = a.union_e + (size_t)bk * a.max_pages, *ub = a.union_blk + (size_t)bk * a.max_pages;
+#pragma unroll
+        for (int i = 0; i < ITEMS; ++i)
+            if ((u_take >> i) & 1u) union_entry(a, ue, ub, u_pos++, p0 + i, blk[i]);
+        if (threadIdx.x == 0) {
+            a.union_cnt[bk] = base;
+            a.zmax[bh] = ORD_NEG_INF;
+        }
+    }
 }
 
 // Gaussian partial moments of a standard normal: J_R(c) = E[(Z-c)_+^R] and
@@ -462,10 +555,18 @@ __global__ void __cluster_dims__(GCL, 1, 1) __launch_bounds__(GTH) gauss_cluster
     const size_t row = (size_t)bh * a.max_pages;
     const float a1 = a.alpha - 1.f;
     const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+    // decode step: the group's union (see above)
+    const int G = a.Hq / a.Hkv;
+    const bool uni = a.umap != nullptr;
+    const int bk = b * a.Hkv + h / G;
     if (n == 0) {  // the same in every CTA of the cluster: no barrier is skipped by half of it
         if (rank == 0 && threadIdx.x == 0) {
             a.cnt[bh] = 0;
             if (a.tau_hat) a.tau_hat[bh] = __int_as_float(0x7fc00000);
+        }
+        if (uni && G == 1 && rank == 0 && threadIdx.x == 0) {
+            a.union_cnt[bk] = 0;
+            a.zmax[bh] = ORD_NEG_INF;
         }
         return;
     }
@@ -567,8 +668,10 @@ __global__ void __cluster_dims__(GCL, 1, 1) __launch_bounds__(GTH) gauss_cluster
     float tau = tau0;
     if (!spill) {
         if (rank == 0) {
-            // rank 0 alone: candidate c of CTA r is item (r, c); thread t
-            // takes items t, t + GTH, ... of the concatenated lists
+            // rank 0 alone: candidate c of CTA r is item (r, c) of the
+            // concatenated lists; thread t takes items t, t + GTH, ...  (One
+            // warp running the steps alone, with no barrier, measured slower:
+            // each lane's Gaussian moments are a long dependent chain.)
             const int n0 = rcnt[0], n1 = n0 + rcnt[1], n2 = n1 + rcnt[2], n3 = n2 + rcnt[3];
             for (int it = 0; it < 48; ++it) {
                 float F = 0.f, Fp = 0.f;
@@ -651,6 +754,9 @@ __global__ void __cluster_dims__(GCL, 1, 1) __launch_bounds__(GTH) gauss_cluster
         const float e = est ? fminf(a1 * ub[i], mm[i] + (p0 + i == n - 1 ? z_last : z_full) * ss[i]) : a1 * ub[i];
         if (p0 + i < hi_p && e > thr) bits |= 1u << i;
     }
+    int blk[GIT];
+    if (uni && G == 1) blocks16(a.page_table + (size_t)b * a.max_pages, p0, bits, blk);  // in flight during the scan
+    if (uni && G > 1) mark16(a.umap + (size_t)bk * a.uwords, p0, bits, h % G);  // the marks complete behind the scan
     int ls;
     int o = block_excl_scan(__popc(bits), sh, &ls);
     if (threadIdx.x < GCL) cl_sti(cl_map(&rsel[rank], threadIdx.x), ls);
@@ -665,11 +771,26 @@ __global__ void __cluster_dims__(GCL, 1, 1) __launch_bounds__(GTH) gauss_cluster
     o += off;
 #pragma unroll
     for (int i = 0; i < GIT; ++i)
-        if (bits & (1u << i)) sel[o++] = p0 + i;
+        if (bits & (1u << i)) {
+            if (uni && G == 1)
+                union_entry(a, a.union_e + (size_t)bk * a.max_pages, a.union_blk + (size_t)bk * a.max_pages, o,
+                            p0 + i, blk[i]);
+            sel[o++] = p0 + i;
+        }
     if (rank == 0 && threadIdx.x == 0) a.cnt[bh] = total;
+    if (uni && G == 1 && rank == 0 && threadIdx.x == 0) {
+        a.union_cnt[bk] = total;
+        a.zmax[bh] = ORD_NEG_INF;
+    }
 }
 
 }  // namespace
+
+bool select_marks_union(const SelectArgs &a) {
+    // one top-k tile, or the cluster form of the Gaussian selection: both
+    // hold up to 16384 pages
+    return a.max_pages <= SEL_THREADS * ITEMS && a.max_pages <= GCL * GTH * GIT;
+}
 
 cudaError_t launch_select(const SelectArgs &a, cudaStream_t st) {
     const int grid = a.B * a.nh;

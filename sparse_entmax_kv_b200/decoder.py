@@ -6,12 +6,13 @@ scores, selections, workspace, output) and issues, on the current stream:
   entmaxkv_append        (each sequence's new key/value row and its page's
                           metadata) or entmaxkv_build_meta (a page the caller
                           already wrote the token to)
-  entmaxkv_score_pages
-  entmaxkv_select        (top-k or Gaussian tau_hat - Delta)
-  entmaxkv_decode_sparse
+  entmaxkv_decode_step   (scores, selection -- top-k or Gaussian tau_hat -
+                          Delta -- and the sparse decode in one call)
 
-It does no arithmetic itself; see include/entmaxkv.h for what each call
-computes.
+or, with ``fused=False`` (and always for alpha = 1 or several kv-head
+ranges), the three calls it stands for: entmaxkv_score_pages,
+entmaxkv_select and entmaxkv_decode_sparse, with identical results.  It does
+no arithmetic itself; see include/entmaxkv.h for what each call computes.
 """
 from __future__ import annotations
 
@@ -22,7 +23,7 @@ from . import native as nv
 
 class EntmaxKVDecoder:
     def __init__(self, k_cache, v_cache, page_table, seq_lens, Hq, *, alpha=1.5, policy="topk",
-                 k=64, delta=0.5, kv_splits=1):
+                 k=64, delta=0.5, kv_splits=1, fused=True):
         dev = k_cache.device
         nb, Hkv, P, d = k_cache.shape
         B, max_pages = page_table.shape
@@ -42,7 +43,6 @@ class EntmaxKVDecoder:
         self.tau_hat = torch.empty((B, Hq), **f32)
         self.tau = torch.empty((B, Hq), **f32)
         self.out = torch.empty((B, Hq, d), **f32)
-        self.ws = nv.alloc_workspace(self.shape, nv.CALL_DECODE_SPARSE, dev)
         self.launches_per_step = 0
         # kv-head ranges, each stepped on its own stream (disjoint heads: the
         # buffers and the workspace are shared); a range's scoring waits for
@@ -54,6 +54,12 @@ class EntmaxKVDecoder:
         self.shapes = [self.shape.kv_range(k0, nk) for k0, nk in self.ranges] if n > 1 else [self.shape]
         self.streams = [torch.cuda.Stream(device=dev) for _ in self.shapes] if n > 1 else None
         self.scored = [torch.cuda.Event() for _ in self.shapes] if n > 1 else None
+        self.fused = bool(fused) and self.alpha > 1.0 and n == 1
+        self.ws = nv.alloc_workspace(self.shape, nv.CALL_DECODE_STEP if self.fused else nv.CALL_DECODE_SPARSE, dev)
+
+    def kernels_per_step(self, append: bool) -> int:
+        """Kernel launches of one ``step`` of this decoder."""
+        return kernels_per_step(self.shape, self.alpha, append, self.policy if self.fused else None)
 
     def build_meta(self, first_page=0, n_pages=-1):
         nv.entmaxkv_build_meta(self.shape, self.k_cache, self.page_table, self.seq_lens,
@@ -92,6 +98,12 @@ class EntmaxKVDecoder:
         elif append_page is not None:
             nv.entmaxkv_build_meta(shape, self.k_cache, self.page_table, self.seq_lens,
                                    append_page, 1, self.meta)
+        if self.fused:
+            nv.entmaxkv_decode_step(shape, q, self.meta, self.k_cache, self.v_cache, self.page_table,
+                                    self.seq_lens, self.policy, self.k, self.alpha, self.delta, self.bbox,
+                                    self.mu, self.sigma, self.sel, self.cnt, out, self.tau_hat, self.tau, p_out,
+                                    self.ws)
+            return
         if after is not None:
             torch.cuda.current_stream().wait_event(after)
         nv.entmaxkv_score_pages(shape, q, self.meta, self.seq_lens, self.bbox, self.mu, self.sigma)
@@ -115,7 +127,11 @@ def last_token_rows(k_cache, v_cache, page_table, seq_lens):
     return k_cache[blk, :, tok].contiguous(), v_cache[blk, :, tok].contiguous()
 
 
-def kernels_per_step(shape, alpha: float, append: bool) -> int:
-    """Kernel launches one ``step`` issues: append (1, if appending), score (1),
-    select (1) and decode_sparse (2 or 3, as the library reports for the shape)."""
+def kernels_per_step(shape, alpha: float, append: bool, policy=None) -> int:
+    """Kernel launches one ``step`` issues: append (1, if appending), then for
+    the fused step (policy given) what entmaxkv_decode_step reports, else
+    score (1), select (1) and decode_sparse (2 or 3, as the library reports
+    for the shape)."""
+    if policy is not None:
+        return (1 if append else 0) + nv.entmaxkv_decode_step_kernels(shape, policy, alpha)
     return (1 if append else 0) + 1 + 1 + nv.entmaxkv_decode_sparse_kernels(shape, alpha)

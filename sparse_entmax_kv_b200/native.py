@@ -22,7 +22,7 @@ ERR = {0: "OK", -1: "ERR_NULL", -2: "ERR_SHAPE", -3: "ERR_ALPHA", -4: "ERR_POLIC
        -5: "ERR_WORKSPACE", -6: "ERR_CUDA", -7: "ERR_UNSUPPORTED", -8: "ERR_ALIGN", -9: "ERR_TOO_LARGE"}
 STATIC_SCRATCH_BYTES = 16 << 20
 TOPK, GAUSS, GAUSS_EST = 0, 1, 2
-CALL_SELECT, CALL_DECODE_SPARSE, CALL_DECODE_DENSE = 2, 3, 4
+CALL_SELECT, CALL_DECODE_SPARSE, CALL_DECODE_DENSE, CALL_DECODE_STEP = 2, 3, 4, 5
 STATUS_BAD_PAGE, STATUS_BAD_SELECTION, STATUS_TIMEOUT, STATUS_OVERFLOW = 1, 2, 4, 8
 STATUS_BAD_LENGTH, STATUS_NONFINITE = 16, 32
 
@@ -31,7 +31,8 @@ EXPORTED = ("entmaxkv_strerror", "entmaxkv_version", "entmaxkv_meta_bytes",
             "entmaxkv_score_pages", "entmaxkv_select", "entmaxkv_decode_sparse",
             "entmaxkv_decode_sparse_static", "entmaxkv_decode_dense", "entmaxkv_decode_sparse_begin",
             "entmaxkv_decode_sparse_candidates", "entmaxkv_entmax_threshold", "entmaxkv_decode_sparse_finish",
-            "entmaxkv_decode_sparse_kernels", "entmaxkv_selftest_wait")
+            "entmaxkv_decode_sparse_kernels", "entmaxkv_selftest_wait", "entmaxkv_decode_step",
+            "entmaxkv_decode_step_kernels")
 
 
 class EntmaxKVError(RuntimeError):
@@ -98,6 +99,9 @@ def lib():
         L.entmaxkv_decode_sparse_finish.argtypes = [sp, vp, vp, vp, vp, vp, f32, vp, vp, vp, vp, vp, sz, vp]
         L.entmaxkv_decode_sparse_kernels.argtypes = [sp, f32]
         L.entmaxkv_selftest_wait.argtypes = [C.c_uint64, vp]
+        L.entmaxkv_decode_step.argtypes = [sp, vp, vp, vp, vp, vp, vp, i32, i32, f32, f32, vp, vp, vp, vp, vp, vp,
+                                           vp, vp, vp, vp, sz, vp]
+        L.entmaxkv_decode_step_kernels.argtypes = [sp, i32, f32]
         for fn in EXPORTED:
             if fn not in ("entmaxkv_strerror", "entmaxkv_version", "entmaxkv_meta_bytes",
                           "entmaxkv_workspace_size"):
@@ -218,6 +222,28 @@ def entmaxkv_decode_sparse_kernels(shape, alpha):
     """Kernel launches of one entmaxkv_decode_sparse call for this shape."""
     n = lib().entmaxkv_decode_sparse_kernels(C.byref(shape), float(alpha))
     _check("entmaxkv_decode_sparse_kernels", min(n, 0))
+    return n
+
+
+def entmaxkv_decode_step(shape, q, meta, k_cache, v_cache, page_table, seq_lens, policy, k, alpha, delta, bbox,
+                         mu, sigma, sel, cnt, out, tau_hat=None, tau_out=None, p_out=None, workspace=None,
+                         stream=None):
+    """Scores, selection and sparse decode in one call (workspace of CALL_DECODE_STEP)."""
+    _check("entmaxkv_decode_step", lib().entmaxkv_decode_step(
+        C.byref(shape), _ptr(q, torch.bfloat16, "q"), _ptr(meta, None, "meta"),
+        _ptr(k_cache, torch.bfloat16, "k_cache"), _ptr(v_cache, torch.bfloat16, "v_cache"),
+        _ptr(page_table, torch.int32, "page_table"), _ptr(seq_lens, torch.int32, "seq_lens"), int(policy),
+        int(k), float(alpha), float(delta), _ptr(bbox, torch.float32, "bbox"), _ptr(mu, torch.float32, "mu"),
+        _ptr(sigma, torch.float32, "sigma"), _ptr(sel, torch.int32, "sel"), _ptr(cnt, torch.int32, "cnt"),
+        _ptr(tau_hat, torch.float32, "tau_hat"), _ptr(out, torch.float32, "out", pinned_ok=True),
+        _ptr(tau_out, torch.float32, "tau_out"), _ptr(p_out, torch.float32, "p_out"),
+        _ptr(workspace, None, "workspace"), 0 if workspace is None else workspace.numel(), _stream(stream)))
+
+
+def entmaxkv_decode_step_kernels(shape, policy, alpha):
+    """Kernel launches of one entmaxkv_decode_step call."""
+    n = lib().entmaxkv_decode_step_kernels(C.byref(shape), int(policy), float(alpha))
+    _check("entmaxkv_decode_step_kernels", min(n, 0))
     return n
 
 

@@ -24,7 +24,7 @@ def _declared():
 def test_library_exports_every_declared_symbol():
     L = nv.lib()
     names = _declared()
-    assert len(names) == 18
+    assert len(names) == 20
     assert set(names) == set(nv.EXPORTED)
     for n in names:
         assert hasattr(L, n)
@@ -156,6 +156,36 @@ def test_binding_refuses_cpu_tensors():
     q = torch.zeros(1, 1, 64, dtype=torch.bfloat16)
     with pytest.raises(ValueError, match="CUDA"):
         nv._ptr(q, torch.bfloat16, "q")
+
+
+def test_decode_step_checks_its_arguments():
+    """The fused step's host-side checks, each returning before any GPU work."""
+    L = nv.lib()
+    s = C.byref(shp())
+    need = nv.workspace_size(shp(), nv.CALL_DECODE_STEP)
+    assert need > nv.workspace_size(shp(), nv.CALL_DECODE_SPARSE)   # plus the union marks and counters
+
+    def step(pol=0, k=4, a=1.5, dl=0.5, mu=None, sg=None, meta=FAKE, ws=FAKE, wsb=need, sh=s, sel=FAKE):
+        return L.entmaxkv_decode_step(sh, FAKE, meta, FAKE, FAKE, FAKE, FAKE, pol, k, a, dl, FAKE, mu, sg, sel,
+                                      FAKE, None, FAKE, None, None, ws, wsb, None)
+    assert step(a=1.0) == -3                       # entmax only
+    assert step(a=float("nan")) == -3
+    assert step(pol=7) == -4
+    assert step(k=0) == -4
+    assert step(pol=1, mu=FAKE, sg=FAKE, dl=float("inf")) == -4
+    assert step(pol=1) == -1                       # Gaussian without mu / sigma
+    assert step(mu=FAKE) == -1                     # mu without sigma
+    assert step(pol=1, a=1.3, mu=FAKE, sg=FAKE) == -7
+    assert step(sel=None) == -1
+    assert step(meta=FAKE_ODD) == -8
+    assert step(wsb=need - 1) == -5
+    assert step(ws=None) == -5
+    assert step(ws=C.c_void_p(0x10010)) == -8      # 256-byte alignment
+    assert step(sh=C.byref(shp(d=96))) == -2
+    assert step(sh=C.byref(shp(max_pages=200000))) == -2
+    assert L.entmaxkv_decode_step_kernels(s, 7, C.c_float(1.5)) == -4
+    assert L.entmaxkv_decode_step_kernels(s, 0, C.c_float(1.0)) == -3
+    assert L.entmaxkv_decode_step_kernels(C.byref(shp(Hq=6, Hkv=4)), 0, C.c_float(1.5)) == -2
 
 
 def test_static_decode_rejects_problems_beyond_its_scratch():

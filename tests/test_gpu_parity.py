@@ -645,6 +645,102 @@ def test_kv_head_ranges_match_one_call(name, splits):
         assert torch.equal(out[b, :G, :npb], b1[b, :G, :npb])
 
 
+# ------------------------------------------------------ the fused step
+
+def _step_outputs(wl, inp, policy, fused, queries, lens=None):
+    """Runs EntmaxKVDecoder.step once per query in `queries` (the last one
+    counts) and returns every output of the last step."""
+    seq_lens = inp["seq_lens"] if lens is None else lens
+    dec = EntmaxKVDecoder(inp["k_cache"], inp["v_cache"], inp["page_table"], seq_lens, wl.Hq, alpha=wl.alpha,
+                          policy=policy, k=wl.k or 16, delta=wl.delta or 0.5, fused=fused)
+    assert dec.fused == fused
+    dec.build_meta()
+    p = torch.full((wl.B, wl.Hq, wl.max_pages * wl.P), float("nan"), device="cuda")
+    for q in queries:
+        for t in (dec.out, dec.tau, dec.tau_hat, dec.bbox, p):  # (p is written on the selected pages only)
+            t.fill_(float("nan"))
+        dec.step(q, p_out=p)
+    torch.cuda.synchronize()
+    return dict(out=dec.out.clone(), tau=dec.tau.clone(), tau_hat=dec.tau_hat.clone(), bbox=dec.bbox.clone(),
+                mu=None if dec.mu is None else dec.mu.clone(), sigma=None if dec.sigma is None else dec.sigma.clone(),
+                sel=dec.sel.clone(), cnt=dec.cnt.clone(), p=p, launches=dec.kernels_per_step(False))
+
+
+def _assert_same_step(a, b, wl, lens, policy):
+    def same(x, y, what):
+        assert torch.equal(x.view(torch.int32), y.view(torch.int32)), what
+    same(a["out"], b["out"], "out")
+    same(a["tau"], b["tau"], "tau")
+    same(a["p"], b["p"], "p")
+    assert torch.equal(a["cnt"], b["cnt"])
+    for bb in range(wl.B):
+        npb = -(-int(lens[bb]) // wl.P)
+        same(a["bbox"][bb, :, :npb], b["bbox"][bb, :, :npb], "bbox")
+        if a["mu"] is not None:
+            same(a["mu"][bb, :, :npb], b["mu"][bb, :, :npb], "mu")
+            same(a["sigma"][bb, :, :npb], b["sigma"][bb, :, :npb], "sigma")
+        for h in range(wl.Hq):
+            n = int(a["cnt"][bb, h])
+            assert torch.equal(a["sel"][bb, h, :n], b["sel"][bb, h, :n])
+            if policy != "topk":
+                same(a["tau_hat"][bb, h], b["tau_hat"][bb, h], "tau_hat")
+
+
+@pytest.mark.parametrize("name", list(SMALL))
+@pytest.mark.parametrize("policy", ["topk", "gauss", "gauss_est"])
+def test_decode_step_matches_separate_calls(name, policy):
+    """entmaxkv_decode_step, whose selection kernel prepares each group's
+    union of pages (marks in the workspace that a small kernel compacts; with
+    one query head per group, the list itself), writes to the bit what
+    score_pages, select and decode_sparse write, in five launches (four with
+    G = 1).  The fused decoder first steps another query, so the marks of one
+    call must not leak into the next."""
+    wl = SMALL[name]
+    inp, _ = gpu_inputs(wl, 31)
+    q2 = (-inp["q"]).contiguous()
+    sep = _step_outputs(wl, inp, policy, False, [inp["q"]])
+    fus = _step_outputs(wl, inp, policy, True, [q2, inp["q"]])
+    _assert_same_step(sep, fus, wl, inp["seq_lens"].cpu().numpy(), policy)
+    assert fus["launches"] == (5 if wl.Hq > wl.Hkv else 4)
+
+
+@pytest.mark.parametrize("policy", ["topk", "gauss"])
+def test_decode_step_with_an_empty_sequence(policy):
+    """A sequence of no tokens in the batch: its group's union is empty, its
+    heads get out = 0 and tau = NaN, and the other sequences match the
+    separate calls."""
+    wl = SMALL["gauss_small"] if policy == "gauss" else SMALL["topk_small"]
+    inp, _ = gpu_inputs(wl, 32)
+    lens = inp["seq_lens"].clone()
+    lens[1] = 0
+    sep = _step_outputs(wl, inp, policy, False, [inp["q"]], lens)
+    fus = _step_outputs(wl, inp, policy, True, [inp["q"], inp["q"]], lens)
+    _assert_same_step(sep, fus, wl, lens.cpu().numpy(), policy)
+    assert (fus["out"][1] == 0).all() and torch.isnan(fus["tau"][1]).all()
+
+
+@pytest.mark.parametrize("policy", ["topk", "gauss", "gauss_est"])
+def test_decode_step_beyond_16384_pages(policy):
+    """Rows of more than 16384 pages (several top-k tiles; the single-CTA
+    Gaussian solver): the selection does not build the union, the step falls
+    back to the separate union pass and still matches the separate calls."""
+    wl = Workload("long_rows", B=1, Hq=4, Hkv=2, d=64, L=20000 * 16 + 5, P=16, alpha=1.5, policy="gauss",
+                  k=24, delta=0.5, keys="cluster", needles=8)
+    assert wl.max_pages > 16384
+    inp, _ = gpu_inputs(wl, 33)
+    sep = _step_outputs(wl, inp, policy, False, [inp["q"]])
+    fus = _step_outputs(wl, inp, policy, True, [inp["q"]])
+    _assert_same_step(sep, fus, wl, inp["seq_lens"].cpu().numpy(), policy)
+    assert fus["launches"] == 2 + nv.entmaxkv_decode_sparse_kernels(shape_of(wl), wl.alpha)
+
+
+def test_decode_step_kernel_count():
+    for name, n in (("gauss_gqa_L1m", 5), ("topk_gqa_L128k", 5), ("sweep_mha_L64k", 4)):
+        s = shape_of(CONFIGS[name])
+        for pol in (nv.TOPK, nv.GAUSS, nv.GAUSS_EST):
+            assert nv.entmaxkv_decode_step_kernels(s, pol, 1.5) == n
+
+
 # ---------------------------------------------------- full-size workloads
 
 def _sub_problem(inp, wl, b, kvh):
