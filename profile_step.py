@@ -3,8 +3,9 @@
   python profile_step.py --workload gauss_gqa_L1m --steps 2 [--dense]
   python profile_step.py --workload gauss_gqa_L1m --steps 3 --score-only
 
-Launch order per step: append (each sequence's newest token again), score_pages, select,
-decode_sparse (union, q.K, tau, p.V); with --dense, one full-cache entmax and
+Launch order per step: append (each sequence's newest token again), then the fused
+decode step (score, select, union from the selection's marks, q.K, tau with p.V); with
+--dense, one full-cache entmax and
 one full-cache softmax decode follow the steps.  The full metadata build runs
 once before the steps.  With --score-only the K/V caches are released after
 the metadata build and each step is one score_pages call, so a profiler that

@@ -503,11 +503,14 @@ __device__ int union_in_cta(const DecodeArgs &a, int b, int kvh, int bk, int np,
 
 // ----------------------------------------------------------------- q . K^T
 
-// q.K ring: three stages per CTA and four CTAs per SM (measured: more CTAs
-// with a shallower ring gather random pages faster than three CTAs of four
-// stages, e.g. 42 vs 46.5 us for the 128k-token top-k decode).
-constexpr int QK_NS = 3;
-constexpr int QK_PER_SM = 4;
+// q.K ring: two stages per CTA and five CTAs per SM.  Measured on the gathered
+// pass (device timeline, 1M-token Gaussian / 128k-token top-k steps): 5 x 2
+// stages 20.6 / 20.9 us, 4 x 3 22.0 / 21.3, 6 x 2 23.9 / 25.2; earlier, 4 x 3
+// beat 3 x 4 (42 vs 46.5 us for the whole 128k-token decode).  More CTAs with
+// a shallower ring gather random pages faster, up to the point where the
+// launch's CTAs no longer hide each other's ramp.
+constexpr int QK_NS = 2;
+constexpr int QK_PER_SM = 5;
 
 template <int D, int G, bool DENSE>
 __global__ void __launch_bounds__(DEC_THREADS) qk_kernel(const __grid_constant__ DecodeArgs a) {

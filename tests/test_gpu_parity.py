@@ -45,14 +45,19 @@ SMALL = {
                          k=20, keys="offset", needles=3, ragged=True),
     "gqa8_d128": Workload("gqa8_d128", B=1, Hq=8, Hkv=1, d=128, L=2000, P=64, alpha=2.0, policy="gauss",
                           delta=0.25, keys="cluster", needles=2, ragged=True),
-    # 320 (sequence, kv head) groups: the q.K grid has one CTA per group, and
-    # each q.K CTA builds its group's union of selected pages itself
+    # 400 (sequence, kv head) groups: the q.K grid (five CTAs per SM, 148
+    # SMs) has one CTA per group, and each q.K CTA builds its group's union
+    # of selected pages itself
+    "groups400_gqa": Workload("groups400_gqa", B=50, Hq=16, Hkv=8, d=128, L=1500, P=32, alpha=1.5,
+                              policy="topk", k=12, keys="offset", needles=3, ragged=True),
+    # 320 groups: two q.K CTAs per group, each building the union and writing
+    # the entries of every other step
     "groups320_gqa": Workload("groups320_gqa", B=40, Hq=16, Hkv=8, d=128, L=1500, P=32, alpha=1.5,
                               policy="topk", k=12, keys="offset", needles=3, ragged=True),
     "groups320_mha": Workload("groups320_mha", B=80, Hq=4, Hkv=4, d=64, L=700, P=16, alpha=1.5,
                               policy="gauss", delta=0.5, keys="cluster", needles=2, ragged=True),
-    # 200 groups: two q.K CTAs per group, each building the union and writing
-    # the entries of every other step
+    # 200 groups: three q.K CTAs per group, the union built once per group by
+    # its own kernel
     "groups200_gqa": Workload("groups200_gqa", B=25, Hq=32, Hkv=8, d=64, L=1200, P=16, alpha=2.0,
                               policy="topk", k=16, keys="offset", needles=3, ragged=True),
 }
@@ -431,14 +436,17 @@ def test_decode_sparse_union_over_several_chunks():
 
 def test_decode_sparse_kernel_count():
     """The library's own count of a sparse decode's launches: a separate union
-    kernel when the q.K grid splits each group widely, none when every group
-    has one q.K CTA (the q.K CTAs build the union), two for softmax."""
+    kernel when the q.K grid splits each group over more than two CTAs, none
+    when every group has one or two (those q.K CTAs build the union), two for
+    softmax."""
     wide = shape_of(CONFIGS["gauss_gqa_L1m"])                      # 8 groups
-    narrow = shape_of(SMALL["groups320_gqa"])                      # 320 groups
-    two = shape_of(SMALL["groups200_gqa"])                          # 200 groups
+    narrow = shape_of(SMALL["groups400_gqa"])                      # 400 groups: one CTA each
+    two = shape_of(SMALL["groups320_gqa"])                          # 320 groups: two CTAs each
+    three = shape_of(SMALL["groups200_gqa"])                        # 200 groups: three CTAs each
     assert nv.entmaxkv_decode_sparse_kernels(wide, 1.5) == 3
     assert nv.entmaxkv_decode_sparse_kernels(narrow, 1.5) == 2
     assert nv.entmaxkv_decode_sparse_kernels(two, 1.5) == 2
+    assert nv.entmaxkv_decode_sparse_kernels(three, 1.5) == 3
     assert nv.entmaxkv_decode_sparse_kernels(wide, 1.0) == 2
 
 
