@@ -309,11 +309,14 @@ __device__ void produce(const DecodeArgs &a, const CUtensorMap *m0, const CUtens
             PageInfo r{-1, 0, 0, e, -1};
             if (e < U) {
                 // sparse: the union entry and its resolved block, loaded
-                // together (through L2: the q.K kernel writes them itself);
-                // dense: page e and its page-table entry
-                const int entry = dense ? ((e << 8) | 0xff) : __ldcg(a.ws.union_e + (size_t)bk * a.max_pages + e);
+                // together (through L2 when the q.K CTAs wrote them
+                // themselves; else through L1, where the kernel's start sent
+                // the first batch); dense: page e and its page-table entry
+                const int *pe = a.ws.union_e + (size_t)bk * a.max_pages + e;
+                const int *pb = a.ws.union_blk + (size_t)bk * a.max_pages + e;
+                const int entry = dense ? ((e << 8) | 0xff) : (a.union_in_qk ? __ldcg(pe) : *pe);
                 const int blk = dense ? __ldg(a.page_table + (size_t)b * a.max_pages + e)
-                                      : __ldcg(a.ws.union_blk + (size_t)bk * a.max_pages + e);
+                                      : (a.union_in_qk ? __ldcg(pb) : *pb);
                 r.page = entry >> 8;
                 r.mask = entry & 0xff;
                 if (blk >= 0 && blk < a.num_blocks) {
@@ -518,6 +521,19 @@ __global__ void __launch_bounds__(DEC_THREADS) qk_kernel(const __grid_constant__
     constexpr int NS = QK_NS;
     using RG = Ring<D, G, NS, 1>;
     constexpr int TPS = RG::TPS;
+    if (!DENSE && !a.union_in_qk && (threadIdx.x >> 5) == NWC) {
+        // the producer's first 32 steps of union entries head for L1 together
+        // with the union size below (their addresses do not depend on it), so
+        // the first copies issue one round trip sooner
+        const int pps = TPS / a.P, bk0 = (a.kv0 + (int)blockIdx.y % a.nk) + ((int)blockIdx.y / a.nk) * a.Hkv;
+        for (int k = threadIdx.x & 31; k < 32 * pps; k += 32) {
+            const int e = ((int)blockIdx.x + (k / pps) * (int)gridDim.x) * pps + k % pps;
+            if (e < a.max_pages) {
+                asm volatile("prefetch.global.L1 [%0];" ::"l"(a.ws.union_e + (size_t)bk0 * a.max_pages + e));
+                asm volatile("prefetch.global.L1 [%0];" ::"l"(a.ws.union_blk + (size_t)bk0 * a.max_pages + e));
+            }
+        }
+    }
     extern __shared__ unsigned char smem_raw[];
     RingView<D, G, NS, 1> R(smem_raw);
     __shared__ float qs[G == 1 ? D : 1];

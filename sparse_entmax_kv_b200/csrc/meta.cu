@@ -39,11 +39,17 @@ __global__ void __launch_bounds__(D) append_kernel(AppendArgs a) {
     pdl_wait();
     const int b = blockIdx.x, kvh = a.m.kv0 + blockIdx.y;
     if (a.q_in) {  // the step's queries of this group, staged for the later calls
-        const int G = a.Hq / a.m.Hkv;
-        for (int g = 0; g < G; ++g) {
-            const size_t o = ((size_t)b * a.Hq + kvh * G + g) * D + threadIdx.x;
-            a.q_out[o] = a.q_in[o];
-        }
+        // (all rows loaded before the first store: one round trip over the
+        // bus when they sit in pinned host memory, not one per row)
+        const int G = a.Hq / a.m.Hkv;  // 1..8
+        const size_t o = ((size_t)b * a.Hq + kvh * G) * D + threadIdx.x;
+        uint16_t qv[8];
+#pragma unroll
+        for (int g = 0; g < 8; ++g)
+            if (g < G) qv[g] = a.q_in[o + (size_t)g * D];
+#pragma unroll
+        for (int g = 0; g < 8; ++g)
+            if (g < G) a.q_out[o + (size_t)g * D] = qv[g];
     }
     const int seq = a.m.seq_lens[b];
     if (seq <= 0) return;
@@ -60,9 +66,9 @@ __global__ void __launch_bounds__(D) append_kernel(AppendArgs a) {
     const int j = threadIdx.x;
     const size_t src = ((size_t)b * a.m.Hkv + kvh) * D + j;
     const size_t rec = ((size_t)blk * a.m.Hkv + kvh) * P * D;
-    const uint16_t kn = a.k_new[src];
+    const uint16_t kn = a.k_new[src], vn = a.v_new[src];  // both loads before the first store
     a.k_cache[rec + (size_t)t * D + j] = kn;
-    a.v_cache[rec + (size_t)t * D + j] = a.v_new[src];
+    a.v_cache[rec + (size_t)t * D + j] = vn;
     page_record<D, P>(a.m, a.k_cache + rec + j, t + 1, t, kn, b, kvh, p);
 }
 
