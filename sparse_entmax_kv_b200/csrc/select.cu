@@ -50,11 +50,12 @@ __device__ __forceinline__ unsigned key_of(float f) {
 // group's row of umap for each page p it keeps (the row is zero on entry);
 // a separate kernel of the decode then compacts the rows.
 
-// Page-table entries of the kept pages among p0 .. p0+15 (bit i: page p0+i),
-// all loads issued together; -1 elsewhere.
-__device__ __forceinline__ void blocks16(const int *pt, int p0, unsigned bits, int (&blk)[16]) {
+// Page-table entries of the kept pages among p0 .. p0+N-1 (bit i: page
+// p0+i), all loads issued together; -1 elsewhere.
+template <int N>
+__device__ __forceinline__ void blocks_run(const int *pt, int p0, unsigned bits, int (&blk)[N]) {
 #pragma unroll
-    for (int i = 0; i < 16; ++i) blk[i] = (bits >> i) & 1u ? __ldg(pt + p0 + i) : -1;
+    for (int i = 0; i < N; ++i) blk[i] = (bits >> i) & 1u ? __ldg(pt + p0 + i) : -1;
 }
 
 // G = 1: union entry `pos` is the kept page p with physical block blk.
@@ -65,11 +66,12 @@ __device__ __forceinline__ void union_entry(const SelectArgs &a, int *ue, int *u
     ub[pos] = ok ? blk : -1;
 }
 
-// G > 1: marks the kept pages among p0 .. p0+15 (p0 a multiple of 16) for
-// head g: one OR per 4-page word holding a kept page.
-__device__ __forceinline__ void mark16(unsigned *row, int p0, unsigned bits, int g) {
+// G > 1: marks the kept pages among p0 .. p0+N-1 (p0 and N multiples of 4)
+// for head g: one OR per 4-page word holding a kept page.
+template <int N>
+__device__ __forceinline__ void mark_run(unsigned *row, int p0, unsigned bits, int g) {
 #pragma unroll
-    for (int j = 0; j < 4; ++j) {
+    for (int j = 0; j < N / 4; ++j) {
         const unsigned nib = (bits >> (4 * j)) & 0xfu;
         if (nib) {
             unsigned w = 0u;
@@ -112,10 +114,10 @@ __global__ void __launch_bounds__(NT) topk_kernel(SelectArgs a) {
             for (int p0 = threadIdx.x * 16; p0 < n; p0 += NT * 16) {
                 const unsigned bits = n - p0 >= 16 ? 0xffffu : (1u << (n - p0)) - 1u;
                 if (G > 1) {
-                    mark16(a.umap + (size_t)bk * a.uwords, p0, bits, h % G);
+                    mark_run<ITEMS>(a.umap + (size_t)bk * a.uwords, p0, bits, h % G);
                 } else {
                     int blk[16];
-                    blocks16(pt, p0, bits, blk);
+                    blocks_run<ITEMS>(pt, p0, bits, blk);
 #pragma unroll
                     for (int i = 0; i < 16; ++i)
                         if ((bits >> i) & 1u)
@@ -220,7 +222,7 @@ __global__ void __launch_bounds__(NT) topk_kernel(SelectArgs a) {
                 if (eq_off < remaining) take |= 1u << i;
                 ++eq_off;
             }
-        if (uni && G > 1) mark16(a.umap + (size_t)bk * a.uwords, p0, take, h % G);  // complete behind the scan
+        if (uni && G > 1) mark_run<ITEMS>(a.umap + (size_t)bk * a.uwords, p0, take, h % G);  // complete behind the scan
         if (uni && G == 1)  // page-table entries to L2 during the scan (no registers held)
 #pragma unroll
             for (int i = 0; i < ITEMS; ++i)
@@ -242,7 +244,7 @@ __global__ void __launch_bounds__(NT) topk_kernel(SelectArgs a) {
         // now, which leaves registers for the page-table entries
         const int p0 = threadIdx.x * ITEMS;
         int blk[ITEMS];
-        blocks16(pt, p0, u_take, blk);
+        blocks_run<ITEMS>(pt, p0, u_take, blk);
         int *ue = a.union_e + (size_t)bk * a.max_pages, *ub = a.union_blk + (size_t)bk * a.max_pages;
 #pragma unroll
         for (int i = 0; i < ITEMS; ++i)
@@ -531,8 +533,11 @@ __global__ void __launch_bounds__(SEL_THREADS) gauss_kernel(SelectArgs a) {
 // over the cluster (one barrier per step); the iterates are the same in every
 // CTA.
 constexpr int GCL = 4;
-constexpr int GTH = 256;
-constexpr int GIT = 16;
+// 512 threads of 8 pages: 12.9 us at 1M tokens against 14.0 for 256 x 16
+// (the per-page loops are unrolled, and a launch fetches its code cold:
+// instruction fetch was the kernel's top stall); 1024 x 4 spills.
+constexpr int GTH = 512;
+constexpr int GIT = 8;
 constexpr int GCAPR = 768;  // candidates per CTA that rank 0 holds
 
 template <int R>
@@ -755,8 +760,8 @@ __global__ void __cluster_dims__(GCL, 1, 1) __launch_bounds__(GTH) gauss_cluster
         if (p0 + i < hi_p && e > thr) bits |= 1u << i;
     }
     int blk[GIT];
-    if (uni && G == 1) blocks16(a.page_table + (size_t)b * a.max_pages, p0, bits, blk);  // in flight during the scan
-    if (uni && G > 1) mark16(a.umap + (size_t)bk * a.uwords, p0, bits, h % G);  // the marks complete behind the scan
+    if (uni && G == 1) blocks_run<GIT>(a.page_table + (size_t)b * a.max_pages, p0, bits, blk);  // in flight during the scan
+    if (uni && G > 1) mark_run<GIT>(a.umap + (size_t)bk * a.uwords, p0, bits, h % G);  // the marks complete behind the scan
     int ls;
     int o = block_excl_scan(__popc(bits), sh, &ls);
     if (threadIdx.x < GCL) cl_sti(cl_map(&rsel[rank], threadIdx.x), ls);
