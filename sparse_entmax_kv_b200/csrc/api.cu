@@ -358,6 +358,7 @@ int entmaxkv_select(const entmaxkv_shape *s, const int32_t *seq_lens, const floa
         a.h0 = kv0 * G;
         a.nh = nk * G;
     }
+    a.sms = di.sms;
     a.status = di.status;
     return cuda_rc(launch_select(a, static_cast<cudaStream_t>(stream)));
 }
@@ -477,6 +478,7 @@ int entmaxkv_decode_step(const entmaxkv_shape *s, const void *q, const void *met
     la.delta = delta;
     la.h0 = da.kv0 * G;
     la.nh = da.nk * G;
+    la.sms = da.sms;
     la.status = da.status;
     la.Hkv = s->Hkv;
     la.num_blocks = s->num_blocks;

@@ -86,6 +86,7 @@ struct SelectArgs {
     float alpha, delta;
     int r_int;  // 1/(alpha-1) for the Gaussian policy
     int h0, nh;  // query-head range [h0, h0 + nh)
+    int sms;     // SMs of the device (grid shape choice)
     int *status;
     // decode step (umap non-null): the union of each group's selections for
     // the q.K pass.  G > 1: each CTA ORs the head bit of every page it keeps

@@ -82,12 +82,12 @@ __device__ __forceinline__ void mark_run(unsigned *row, int p0, unsigned bits, i
     }
 }
 
-// Top-k: the keys of one tile (TILE pages) stay in registers, ITEMS
+// Top-k: the keys of one tile (NT * IT pages) stay in registers, IT
 // consecutive pages per thread, through the four radix passes and the final
 // ordered compaction; longer sequences take several tiles per pass.
-template <int NT>
+template <int NT, int IT>
 __global__ void __launch_bounds__(NT) topk_kernel(SelectArgs a) {
-    constexpr int TILE_NT = NT * ITEMS;
+    constexpr int TILE_NT = NT * IT;
     pdl_wait();
     __shared__ int whist[NT / 32][256];  // one histogram per warp (contention stays inside a warp)
     __shared__ int hist[256];
@@ -111,15 +111,15 @@ __global__ void __launch_bounds__(NT) topk_kernel(SelectArgs a) {
         for (int p = threadIdx.x; p < n; p += blockDim.x) sel[p] = p;
         if (threadIdx.x == 0) a.cnt[bh] = n;
         if (uni) {
-            for (int p0 = threadIdx.x * 16; p0 < n; p0 += NT * 16) {
-                const unsigned bits = n - p0 >= 16 ? 0xffffu : (1u << (n - p0)) - 1u;
+            for (int p0 = threadIdx.x * IT; p0 < n; p0 += NT * IT) {
+                const unsigned bits = n - p0 >= IT ? (1u << IT) - 1u : (1u << (n - p0)) - 1u;
                 if (G > 1) {
-                    mark_run<ITEMS>(a.umap + (size_t)bk * a.uwords, p0, bits, h % G);
+                    mark_run<IT>(a.umap + (size_t)bk * a.uwords, p0, bits, h % G);
                 } else {
-                    int blk[16];
-                    blocks_run<ITEMS>(pt, p0, bits, blk);
+                    int blk[IT];
+                    blocks_run<IT>(pt, p0, bits, blk);
 #pragma unroll
-                    for (int i = 0; i < 16; ++i)
+                    for (int i = 0; i < IT; ++i)
                         if ((bits >> i) & 1u)
                             union_entry(a, a.union_e + (size_t)bk * a.max_pages,
                                         a.union_blk + (size_t)bk * a.max_pages, p0 + i, p0 + i, blk[i]);
@@ -134,11 +134,11 @@ __global__ void __launch_bounds__(NT) topk_kernel(SelectArgs a) {
     }
     const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
     const bool one_tile = n <= TILE_NT;
-    unsigned key[ITEMS];
+    unsigned key[IT];
     auto load_tile = [&](int t0) {
-        const int p0 = t0 + threadIdx.x * ITEMS;
+        const int p0 = t0 + threadIdx.x * IT;
 #pragma unroll
-        for (int i = 0; i < ITEMS; ++i) key[i] = (p0 + i < n) ? key_of(__ldg(sc + p0 + i)) : 0u;
+        for (int i = 0; i < IT; ++i) key[i] = (p0 + i < n) ? key_of(__ldg(sc + p0 + i)) : 0u;
     };
     if (one_tile) load_tile(0);
     unsigned prefix = 0, mask = 0;
@@ -148,9 +148,9 @@ __global__ void __launch_bounds__(NT) topk_kernel(SelectArgs a) {
         __syncthreads();
         for (int t0 = 0; t0 < n; t0 += TILE_NT) {
             if (!one_tile) load_tile(t0);
-            const int p0 = t0 + threadIdx.x * ITEMS;
+            const int p0 = t0 + threadIdx.x * IT;
 #pragma unroll
-            for (int i = 0; i < ITEMS; ++i)
+            for (int i = 0; i < IT; ++i)
                 if (p0 + i < n && (key[i] & mask) == prefix) atomicAdd(&whist[warp][(key[i] >> shift) & 255], 1);
         }
         __syncthreads();
@@ -204,10 +204,10 @@ __global__ void __launch_bounds__(NT) topk_kernel(SelectArgs a) {
     int u_pos = 0;         // and the list position of the first
     for (int t0 = 0; t0 < n; t0 += TILE_NT) {
         if (!one_tile) load_tile(t0);
-        const int p0 = t0 + threadIdx.x * ITEMS;
+        const int p0 = t0 + threadIdx.x * IT;
         unsigned gt = 0, eq = 0;
 #pragma unroll
-        for (int i = 0; i < ITEMS; ++i) {
+        for (int i = 0; i < IT; ++i) {
             if (p0 + i < n) {
                 if (key[i] > T) gt |= 1u << i;
                 if (key[i] == T) eq |= 1u << i;
@@ -217,22 +217,22 @@ __global__ void __launch_bounds__(NT) topk_kernel(SelectArgs a) {
         int eq_off = eq_base + block_excl_scan(__popc(eq), sh, &eq_tot);
         unsigned take = gt;
 #pragma unroll
-        for (int i = 0; i < ITEMS; ++i)
+        for (int i = 0; i < IT; ++i)
             if (eq & (1u << i)) {
                 if (eq_off < remaining) take |= 1u << i;
                 ++eq_off;
             }
-        if (uni && G > 1) mark_run<ITEMS>(a.umap + (size_t)bk * a.uwords, p0, take, h % G);  // complete behind the scan
+        if (uni && G > 1) mark_run<IT>(a.umap + (size_t)bk * a.uwords, p0, take, h % G);  // complete behind the scan
         if (uni && G == 1)  // page-table entries to L2 during the scan (no registers held)
 #pragma unroll
-            for (int i = 0; i < ITEMS; ++i)
+            for (int i = 0; i < IT; ++i)
                 if ((take >> i) & 1u) asm volatile("prefetch.global.L2 [%0];" ::"l"(pt + p0 + i));
         int tot;
         int w = base + block_excl_scan(__popc(take), sh, &tot);
         u_take = take;
         u_pos = w;
 #pragma unroll
-        for (int i = 0; i < ITEMS; ++i)
+        for (int i = 0; i < IT; ++i)
             if (take & (1u << i)) sel[w++] = p0 + i;
         base += tot;
         eq_base += eq_tot;
@@ -242,12 +242,12 @@ __global__ void __launch_bounds__(NT) topk_kernel(SelectArgs a) {
         // one tile (the decode step's limit): this thread's kept pages and
         // their first list position are u_take and u_pos; the keys are dead
         // now, which leaves registers for the page-table entries
-        const int p0 = threadIdx.x * ITEMS;
-        int blk[ITEMS];
-        blocks_run<ITEMS>(pt, p0, u_take, blk);
+        const int p0 = threadIdx.x * IT;
+        int blk[IT];
+        blocks_run<IT>(pt, p0, u_take, blk);
         int *ue = a.union_e + (size_t)bk * a.max_pages, *ub = a.union_blk + (size_t)bk * a.max_pages;
 #pragma unroll
-        for (int i = 0; i < ITEMS; ++i)
+        for (int i = 0; i < IT; ++i)
             if ((u_take >> i) & 1u) union_entry(a, ue, ub, u_pos++, p0 + i, blk[i]);
         if (threadIdx.x == 0) {
             a.union_cnt[bk] = base;
@@ -802,10 +802,17 @@ cudaError_t launch_select(const SelectArgs &a, cudaStream_t st) {
     cudaError_t e = cudaSuccess;
     if (a.policy == ENTMAXKV_TOPK) {
         // short sequences: a quarter of the threads holds every page in registers
-        if (a.max_pages <= 256 * ITEMS)
-            e = launch_pdl(topk_kernel<256>, dim3(grid), dim3(256), 0, st, a);
+        // rows of up to 4096 pages: 512 threads of 8 keys (less unrolled code,
+        // fetched cold each launch: 9.9 vs 11.0 us for the 128k-token batch of
+        // 8) while the heads fit one wave of two CTAs per SM, else 256 of 16
+        // (four per SM: the 512-head batch took 19.6 us in two waves against
+        // 15.1 in one)
+        if (a.max_pages <= 4096 && grid <= 2 * a.sms)
+            e = launch_pdl(topk_kernel<512, 8>, dim3(grid), dim3(512), 0, st, a);
+        else if (a.max_pages <= 4096)
+            e = launch_pdl(topk_kernel<256, ITEMS>, dim3(grid), dim3(256), 0, st, a);
         else
-            e = launch_pdl(topk_kernel<SEL_THREADS>, dim3(grid), dim3(SEL_THREADS), 0, st, a);
+            e = launch_pdl(topk_kernel<SEL_THREADS, ITEMS>, dim3(grid), dim3(SEL_THREADS), 0, st, a);
     } else if (a.max_pages <= GCL * GTH * GIT) {
         switch (a.r_int) {
             case 1: e = launch_pdl(gauss_cluster_kernel<1>, dim3(grid * GCL), dim3(GTH), 0, st, a); break;
