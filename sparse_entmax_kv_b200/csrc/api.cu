@@ -164,7 +164,7 @@ const char *entmaxkv_strerror(int code) {
         case ENTMAXKV_ERR_POLICY: return "unknown selection policy, k < 1, or delta not finite";
         case ENTMAXKV_ERR_WORKSPACE: return "workspace missing or too small";
         case ENTMAXKV_ERR_CUDA: return "CUDA runtime or driver error";
-        case ENTMAXKV_ERR_UNSUPPORTED: return "valid arguments that this build does not support";
+        case ENTMAXKV_ERR_UNSUPPORTED: return "valid arguments that the library does not support";
         case ENTMAXKV_ERR_ALIGN: return "pointer not 16-byte aligned";
         case ENTMAXKV_ERR_TOO_LARGE:
             return "problem needs more scratch than the fixed array of entmaxkv_decode_sparse_static";
