@@ -11,8 +11,8 @@
 //                  ring memory (one page bitmap per head), and writes the
 //                  entries of its own steps.
 //   qk_kernel      split over the union: TMA 2-D loads (128-byte swizzle) of
-//                  the K tiles through a 3-stage mbarrier ring fed by one
-//                  producer warp; z = (alpha-1) q.k/sqrt(d) for all G heads
+//                  the K tiles through a 2-stage mbarrier ring fed by one
+//                  producer warp, five CTAs per SM; z = (alpha-1) q.k/sqrt(d) for all G heads
 //                  of the group from one copy of each tile (tensor-core
 //                  m16n8k16, tokens as M and the heads as N, when G >= 2; CUDA
 //                  cores when G == 1), stored in list order with the max of
@@ -25,6 +25,9 @@
 //                  and is reached by Newton's method from the end where it is
 //                  monotone, and p v is summed over the support, reading only
 //                  those value rows.
+// In the fused decode step (entmaxkv_decode_step) the selection kernel has
+// marked each group's pages, and union_map_kernel compacts the marks in place
+// of union_kernel (with G = 1 the selection wrote the union itself).
 // Sparse softmax (alpha = 1) builds the union with union_kernel and runs
 // softmax_kernel over its pages.
 // Full-cache entmax runs qk_kernel over every page, tau_pv_kernel for tau, and

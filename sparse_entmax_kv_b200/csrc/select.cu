@@ -1,6 +1,8 @@
 // select.cu -- candidate page selection (EntmaxKV summary, section 2.B).
 //
-// One CTA per (sequence, query head).
+// One CTA per (sequence, query head), or for the Gaussian policies on rows of
+// up to 16384 pages a cluster of four.  In the fused decode step the kernels
+// also prepare each GQA group's union of selected pages (below).
 //
 // Top-k: radix select on the order-preserving 32-bit image of the fp32 bound
 // (four 8-bit digits, most significant first; per-warp shared-memory
