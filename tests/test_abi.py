@@ -168,6 +168,14 @@ def test_decode_step_checks_its_arguments():
     def step(pol=0, k=4, a=1.5, dl=0.5, mu=None, sg=None, meta=FAKE, ws=FAKE, wsb=need, sh=s, sel=FAKE):
         return L.entmaxkv_decode_step(sh, FAKE, meta, FAKE, FAKE, FAKE, FAKE, pol, k, a, dl, FAKE, mu, sg, sel,
                                       FAKE, None, FAKE, None, None, ws, wsb, None)
+    # the decode step's extra region: one byte of head bits per page and kv head (rows of
+    # ceil(max_pages / 4) words rounded up to a multiple of 4), 256-byte aligned, last
+    uwords = (-(-64 // 4) + 3) // 4 * 4
+    assert need - nv.workspace_size(shp(), nv.CALL_DECODE_SPARSE) == -(-(2 * 2 * uwords * 4) // 256) * 256
+    odd = shp(max_pages=70)
+    uw = (-(-70 // 4) + 3) // 4 * 4
+    assert (nv.workspace_size(odd, nv.CALL_DECODE_STEP) - nv.workspace_size(odd, nv.CALL_DECODE_SPARSE)
+            == -(-(2 * 2 * uw * 4) // 256) * 256)
     assert step(a=1.0) == -3                       # entmax only
     assert step(a=float("nan")) == -3
     assert step(pol=7) == -4
