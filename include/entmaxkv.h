@@ -342,7 +342,9 @@ ENTMAXKV_API int entmaxkv_decode_sparse_kernels(const entmaxkv_shape *shape, flo
  *   (the bound alone is scored).
  * - workspace: entmaxkv_workspace_size(shape, ENTMAXKV_CALL_DECODE_STEP)
  *   bytes, 256-byte aligned; its contents need no initialisation (the scoring
- *   kernel clears the page map every call).
+ *   kernel clears the page-map rows of the call's groups every call).  As
+ *   with every call, calls on disjoint kv-head ranges may share it and run
+ *   concurrently.
  * - bbox/mu/sigma, sel/cnt/tau_hat, out/tau_out/p_out: as in the three calls.
  */
 ENTMAXKV_API int entmaxkv_decode_step(const entmaxkv_shape *shape, const void *q, const void *meta,

@@ -511,10 +511,9 @@ int entmaxkv_decode_step(const entmaxkv_shape *s, const void *q, const void *met
     sa.kv0 = da.kv0;
     sa.nk = da.nk;
     sa.status = da.status;
-    if (fused && G > 1) {
-        // the union marks: from umap to the end of the workspace
-        sa.zero = reinterpret_cast<uint4 *>(da.ws.umap);
-        sa.zero16 = (long long)((static_cast<char *>(workspace) + need) - reinterpret_cast<char *>(da.ws.umap)) / 16;
+    if (fused && G > 1) {  // the union marks of the call's groups
+        sa.umap = da.ws.umap;
+        sa.uwords = da.ws.uwords;
     }
     cudaStream_t st = static_cast<cudaStream_t>(stream);
     cudaError_t e = launch_score_pages(sa, st);

@@ -1840,7 +1840,7 @@ size_t decode_ws_bytes(bool dense, int B, int Hq, int Hkv, int d, int P, int max
     const size_t o_part = take((size_t)MAX_SPLITS * B * Hq * (d + 2) * 4);  // split-K softmax partials
     const size_t o_z = take(tokens * 4);
     const size_t o_t = take(tokens / 16 * 4);
-    // decode step: the union marks, last (cleared from there to the end)
+    // decode step: the union marks, one row per group
     const size_t o_umap = take(step ? (size_t)B * Hkv * uwords * 4 : 0);
     if (carve && base) {
         char *p = static_cast<char *>(base);

@@ -69,10 +69,10 @@ struct ScoreArgs {
     int B, Hq, Hkv, d, P, max_pages;
     int kv0, nk;  // kv-head range [kv0, kv0 + nk)
     int *status;
-    // decode step: zero16 16-byte words at zero are cleared (the union marks
-    // and group counters that the selection of the same step then fills)
-    uint4 *zero;
-    long long zero16;
+    // decode step: the rows of umap (uwords words each, a multiple of 4) of
+    // the call's groups are cleared for the selection of the same step
+    unsigned *umap;
+    int uwords;
 };
 cudaError_t launch_score_pages(const ScoreArgs &a, cudaStream_t st);
 
@@ -170,7 +170,7 @@ cudaError_t launch_decode_dense_entmax(const DecodeArgs &a, cudaStream_t st);
 cudaError_t launch_decode_dense_softmax(const DecodeArgs &a, cudaStream_t st);
 
 // Workspace of a decode call; step adds the union marks of
-// entmaxkv_decode_step (last, so that one clear from there to the end covers them).
+// entmaxkv_decode_step (one row per group, each call clearing its groups' rows).
 size_t decode_ws_bytes(bool dense, int B, int Hq, int Hkv, int d, int P, int max_pages, DecodeWs *carve,
                       void *base, bool step = false);
 

@@ -69,11 +69,15 @@ constexpr size_t smem_bytes() {
 template <int D, int G, bool GAUSS>
 __global__ void __launch_bounds__(THREADS, G <= 4 ? (GAUSS ? 2 : 3) : 1) score_kernel(ScoreArgs a) {
     pdl_wait();
-    if (a.zero) {  // decode step: clear the selection's union marks and counters
-        const long long stride = (long long)gridDim.x * gridDim.y * THREADS;
-        for (long long i = ((long long)blockIdx.y * gridDim.x + blockIdx.x) * THREADS + threadIdx.x; i < a.zero16;
-             i += stride)
-            a.zero[i] = make_uint4(0u, 0u, 0u, 0u);
+    if (a.umap) {
+        // decode step: clear this group's row of the selection's union marks
+        // (the CTAs of the group share it; rows of other kv heads are left to
+        // their own calls)
+        int b0, k0;
+        group_of(blockIdx.y, a.kv0, a.nk, b0, k0);
+        uint4 *row = reinterpret_cast<uint4 *>(a.umap + (size_t)(b0 * a.Hkv + k0) * a.uwords);
+        for (int i = blockIdx.x * THREADS + threadIdx.x; i < a.uwords / 4; i += gridDim.x * THREADS)
+            row[i] = make_uint4(0u, 0u, 0u, 0u);
     }
     using RG = Ring<GAUSS>;
     constexpr int CPS = RG::CPS;

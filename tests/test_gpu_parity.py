@@ -742,6 +742,41 @@ def test_decode_step_beyond_16384_pages(policy):
     assert fus["launches"] == 2 + nv.entmaxkv_decode_sparse_kernels(shape_of(wl), wl.alpha)
 
 
+@pytest.mark.parametrize("policy", ["topk", "gauss"])
+def test_decode_step_on_a_kv_range_clears_only_its_rows(policy):
+    """A decode step on a kv-head range clears only its own groups' rows of the
+    union marks in the workspace (calls on disjoint ranges may share one and
+    overlap in time), and writes for its heads what the whole-shape step
+    writes."""
+    wl = SMALL["gauss_small"]  # B=2, Hq=8, Hkv=2
+    inp, _ = gpu_inputs(wl, 41)
+    s = shape_of(wl)
+    whole = _step_outputs(wl, inp, policy, True, [inp["q"]])
+    dec = EntmaxKVDecoder(inp["k_cache"], inp["v_cache"], inp["page_table"], inp["seq_lens"], wl.Hq,
+                          alpha=wl.alpha, policy=policy, k=wl.k or 16, delta=wl.delta or 0.5)
+    dec.build_meta()
+    # the marks are the step workspace's last region: one row of ceil(max_pages/4)
+    # words (rounded up to a multiple of 4) per (sequence, kv head)
+    off = nv.workspace_size(s, nv.CALL_DECODE_SPARSE)
+    uwords = (-(-wl.max_pages // 4) + 3) // 4 * 4
+    rows = dec.ws[off:off + wl.B * wl.Hkv * uwords * 4].view(torch.int32).view(wl.B, wl.Hkv, uwords)
+    rows.fill_(0x5A5A5A5A)
+    r = s.kv_range(1, 1)
+    G = wl.Hq // wl.Hkv
+    nv.entmaxkv_decode_step(r, inp["q"], dec.meta, inp["k_cache"], inp["v_cache"], inp["page_table"],
+                            inp["seq_lens"], dec.policy, dec.k, dec.alpha, dec.delta, dec.bbox, dec.mu, dec.sigma,
+                            dec.sel, dec.cnt, dec.out, dec.tau_hat, dec.tau, None, dec.ws)
+    torch.cuda.synchronize()
+    assert nv.get_status(clear=True) & ~nv.STATUS_OVERFLOW == 0
+    if G > 1:
+        assert (rows[:, 0] == 0x5A5A5A5A).all()          # kv head 0: not this call's
+        assert not (rows[:, 1] == 0x5A5A5A5A).any()      # kv head 1: cleared, then marked
+    hs = slice(G, 2 * G)
+    assert torch.equal(dec.out[:, hs].view(torch.int32), whole["out"][:, hs].view(torch.int32))
+    assert torch.equal(dec.tau[:, hs].view(torch.int32), whole["tau"][:, hs].view(torch.int32))
+    assert torch.equal(dec.cnt[:, hs], whole["cnt"][:, hs])
+
+
 def test_decode_step_kernel_count():
     for name, n in (("gauss_gqa_L1m", 5), ("topk_gqa_L128k", 5), ("sweep_mha_L64k", 4)):
         s = shape_of(CONFIGS[name])
