@@ -47,8 +47,9 @@ PAPER_CONTEXT = {"speedup_vs_full_softmax_flashdecoding": 3.36, "speedup_vs_full
 # keyed by kernel and workload, valid only while the kernel source is unchanged
 # (the source hash below); the line reports null traffic once it has changed.
 NCU_TRAFFIC = {
-    # one full-size launch at L=1,048,576 (201.36 MB read + 6.29 MB written), ncu --set full
-    "score_pages/gauss_gqa_L1m": {"bytes": 201362944 + 6286592, "src": "0aade4c8ae34"},
+    # one full-size launch at L=1,048,576 (201.36 MB read + 5.46 MB written), ncu --metrics
+    # dram__bytes_read.sum,dram__bytes_write.sum on the score-only profile run
+    "score_pages/gauss_gqa_L1m": {"bytes": 201361920 + 5464064, "src": "61c13daf6d60"},
 }
 
 
